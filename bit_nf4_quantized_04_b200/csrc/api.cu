@@ -1,0 +1,803 @@
+// C ABI of libqnf4 (declared in include/qnf4.h): argument checks, workspace
+// layout, tensor-map creation and kernel launches. All device code of the library
+// is compiled in this one translation unit.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "../../include/qnf4.h"
+#include "chanq.cuh"
+#include "common.cuh"
+#include "gemm.cuh"
+#include "quant.cuh"
+#include "tables.h"
+
+namespace qnf4 {
+namespace {
+
+thread_local std::string g_last = "";
+unsigned long long g_wait_ns = 1000000000ull;
+
+qnf4_status fail(qnf4_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last = buf;
+  return s;
+}
+qnf4_status ok() { return QNF4_OK; }
+
+bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+std::atomic<unsigned long long> g_launches{0};
+thread_local cudaEvent_t g_ev_start = nullptr, g_ev_stop = nullptr;
+
+// Check the last launch(es) and count `n` kernels of this library as launched.
+qnf4_status launched(const char* what, int n = 1) {
+  g_launches.fetch_add(static_cast<unsigned long long>(n), std::memory_order_relaxed);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(QNF4_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  return QNF4_OK;
+}
+
+int num_sms() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  static std::mutex mu;
+  static std::vector<int> cache;
+  std::lock_guard<std::mutex> lk(mu);
+  if (static_cast<int>(cache.size()) <= dev) cache.resize(dev + 1, 0);
+  if (cache[dev] == 0) {
+    int v = 0;
+    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    cache[dev] = v > 0 ? v : 148;
+  }
+  return cache[dev];
+}
+
+QuantTab make_tab() {
+  const Nf4Tables& t = nf4_tables();
+  QuantTab q;
+  std::memcpy(q.thr, t.thr, sizeof(q.thr));
+  std::memcpy(q.levels, t.levels, sizeof(q.levels));
+  q.nbins = t.nbins;
+  std::memcpy(q.bin_code, t.bin_code, sizeof(q.bin_code));
+  return q;
+}
+
+constexpr int kQuantMaxGrid = 1024;
+
+int quant_grid(int64_t nblocks) {
+  const int64_t per_cta = 32;  // 64-element blocks per CTA-step (256 threads, 8 per block)
+  int64_t g = (nblocks + per_cta * 4 - 1) / (per_cta * 4);
+  g = std::max<int64_t>(1, std::min<int64_t>(g, std::min(kQuantMaxGrid, num_sms() * 8)));
+  return static_cast<int>(g);
+}
+
+qnf4_status check_weight(const qnf4_weight* w) {
+  if (!w) return fail(QNF4_ERR_ARG, "weight is NULL");
+  if (w->block1 != 64 || w->block2 != 256)
+    return fail(QNF4_ERR_ARG, "block1 must be 64 and block2 256 (got %d, %d)", w->block1, w->block2);
+  if (w->N <= 0 || w->K <= 0) return fail(QNF4_ERR_SHAPE, "N and K must be positive");
+  if (w->K % 64) return fail(QNF4_ERR_SHAPE, "K must be a multiple of 64 (got %lld)", (long long)w->K);
+  if (!w->packed || !w->code2 || !w->scale2 || !w->mean) return fail(QNF4_ERR_ARG, "weight has a NULL buffer");
+  if (!al16(w->packed) || !al16(w->code2) || !al16(w->scale2) || !al16(w->mean))
+    return fail(QNF4_ERR_ALIGN, "weight buffers must be 16-byte aligned");
+  return ok();
+}
+
+
+// ---------------------------------------------------------------------------
+// tcgen05 GEMM planning: tile sizes, split-K and the workspace carve-up
+// ---------------------------------------------------------------------------
+using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                              const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                              const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                              CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeFn encode_fn() {
+  static EncodeFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeFn>(p);
+  });
+  return fn;
+}
+
+// 2-D tensor map over a row-major [outer, inner] matrix with row stride ld elements.
+bool make_map(CUtensorMap* m, const void* ptr, bool u8, uint64_t inner, uint64_t outer,
+              uint64_t ld, uint32_t box_in, uint32_t box_out, bool sw128) {
+  std::memset(m, 0, sizeof(*m));
+  EncodeFn fn = encode_fn();
+  if (!fn) return false;
+  const uint64_t es = u8 ? 1 : 2;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {ld * es};
+  cuuint32_t box[2] = {box_in, box_out};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(m, u8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                        const_cast<void*>(ptr), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        sw128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+struct GemmPlan {
+  int asrc = 0, tn = 16, has_ext = 0;
+  int64_t rows = 0, cols = 0;
+  int nsteps = 0, row_tiles = 0, col_tiles = 0, splits = 1, steps_per_split = 0, s1 = 1, s2 = 0;
+  size_t smem = 0;
+  size_t part_floats() const {
+    return splits > 1 ? static_cast<size_t>(row_tiles) * col_tiles * splits * tn * 128 : 0;
+  }
+  int64_t tiles() const { return static_cast<int64_t>(row_tiles) * col_tiles; }
+};
+
+constexpr size_t kSmemLimit = 227 * 1024;
+
+int tn_for_tokens(int64_t M) {
+  if (M <= 16) return 16;
+  if (M <= 32) return 32;
+  if (M <= 64) return 64;
+  if (M <= 128) return 128;
+  return 256;
+}
+
+GemmPlan plan_gemm(int asrc, int64_t rows, int64_t cols, int64_t contraction, int tn,
+                   int has_ext, int nsm) {
+  GemmPlan p;
+  p.asrc = asrc;
+  p.tn = tn;
+  p.has_ext = has_ext;
+  p.rows = rows;
+  p.cols = cols;
+  p.nsteps = static_cast<int>((contraction + kStep - 1) / kStep);
+  p.row_tiles = static_cast<int>((rows + kRowsTile - 1) / kRowsTile);
+  p.col_tiles = static_cast<int>((cols + tn - 1) / tn);
+  // Split the contraction only when the output tiles leave SMs idle. The cost model
+  // is waves x steps per CTA (one CTA per SM), ties to fewer splits.
+  const int64_t tiles = p.tiles();
+  int best = 1;
+  if (tiles < nsm && p.nsteps > 1) {
+    const int max_splits = std::max(1, p.nsteps / 2);
+    int64_t best_cost = INT64_MAX;
+    for (int sp = 1; sp <= max_splits; ++sp) {
+      const int spc = (p.nsteps + sp - 1) / sp;
+      const int real = (p.nsteps + spc - 1) / spc;
+      if (real != sp) continue;
+      const int64_t waves = (tiles * sp + nsm - 1) / nsm;
+      const int64_t cost = waves * spc * 16 + sp;  // small charge per split for the reduction
+      if (cost < best_cost) {
+        best_cost = cost;
+        best = sp;
+      }
+    }
+  }
+  p.steps_per_split = (p.nsteps + best - 1) / best;
+  p.splits = (p.nsteps + p.steps_per_split - 1) / p.steps_per_split;
+  // ring depths from the shared-memory budget
+  p.s2 = src_deq(asrc) ? (tn <= 64 ? 4 : 2) : 0;
+  const SmemPlan one = smem_plan(asrc, tn, 1, p.s2, has_ext);
+  const size_t fixed = one.total - one.slot1;
+  // 1 KB of slack to align the dynamic buffer to 1024 and 1 KB for static shared data
+  const size_t budget = kSmemLimit - 2048;
+  p.s1 = static_cast<int>(std::min<size_t>(kMaxS1, (budget - fixed) / one.slot1));
+  p.smem = smem_plan(asrc, tn, p.s1, p.s2, has_ext).total + 1024;
+  return p;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// Workspace of one linear-layer call (forward or backward).
+struct LinPlan {
+  int r16 = 16;
+  int64_t ldm = 0, ldn = 0;
+  GemmPlan u, v, main, da, db;
+  size_t off_up = 0, off_ut = 0, off_vp = 0, off_vt = 0, off_bt = 0, off_part = 0, off_cnt = 0;
+  size_t total = 0;
+};
+
+LinPlan plan_linear(int main_src, int64_t N, int64_t K, int64_t M, int r, bool bwd, int nsm) {
+  LinPlan L;
+  L.r16 = ((r + 15) / 16) * 16;
+  L.ldm = ((M + 7) / 8) * 8;
+  L.ldn = ((N + 7) / 8) * 8;
+  const int tnm = tn_for_tokens(M);
+  size_t part = 0;
+  int64_t cnt = 1;
+  L.u = plan_gemm(A_DENSE_K, M, L.r16, K, L.r16, 0, nsm);
+  part = std::max(part, L.u.part_floats());
+  cnt = std::max(cnt, L.u.tiles());
+  if (!bwd) {
+    L.main = plan_gemm(main_src, N, M, K, tnm, 1, nsm);
+  } else {
+    L.v = plan_gemm(A_DENSE_K, M, L.r16, N, L.r16, 0, nsm);
+    L.main = plan_gemm(main_src, K, M, N, tnm, 1, nsm);
+    L.da = plan_gemm(A_DENSE_MN, K, L.r16, M, L.r16, 0, nsm);
+    L.db = plan_gemm(A_DENSE_MN, N, L.r16, M, L.r16, 0, nsm);
+    for (const GemmPlan* g : {&L.v, &L.da, &L.db}) {
+      part = std::max(part, g->part_floats());
+      cnt = std::max(cnt, g->tiles());
+    }
+  }
+  part = std::max(part, L.main.part_floats());
+  cnt = std::max(cnt, L.main.tiles());
+  size_t o = 0;
+  L.off_up = o;
+  o = align256(o + static_cast<size_t>(M) * 64 * 2);
+  if (bwd) {
+    L.off_ut = o;
+    o = align256(o + static_cast<size_t>(L.r16) * L.ldm * 2);
+    L.off_vp = o;
+    o = align256(o + static_cast<size_t>(M) * 64 * 2);
+    L.off_vt = o;
+    o = align256(o + static_cast<size_t>(L.r16) * L.ldm * 2);
+    L.off_bt = o;
+    o = align256(o + static_cast<size_t>(L.r16) * L.ldn * 2);
+  }
+  L.off_part = o;
+  o = align256(o + part * sizeof(float));
+  L.off_cnt = o;
+  o = align256(o + static_cast<size_t>(cnt) * sizeof(unsigned int));
+  L.total = o;
+  return L;
+}
+
+bool g_smem_set[5][64] = {};
+
+template <int ASRC>
+qnf4_status launch_gemm(const GemmPlan& p, const CUtensorMap& a, const CUtensorMap& b,
+                        const CUtensorMap& bx, GemmArgs g, cudaStream_t s) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !g_smem_set[ASRC][dev]) {
+    const cudaError_t e = cudaFuncSetAttribute(k_gemm<ASRC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               static_cast<int>(kSmemLimit - 1024));
+    if (e != cudaSuccess) return fail(QNF4_ERR_CUDA, "smem attribute: %s", cudaGetErrorString(e));
+    g_smem_set[ASRC][dev] = true;
+  }
+  g.rows = p.rows;
+  g.cols = p.cols;
+  g.nsteps = p.nsteps;
+  g.steps_per_split = p.steps_per_split;
+  g.splits = p.splits;
+  g.tn = p.tn;
+  g.s1 = p.s1;
+  g.s2 = p.s2;
+  g.has_ext = p.has_ext;
+  g.wait_ns = g_wait_ns;
+  const dim3 grid(p.row_tiles, p.col_tiles, p.splits);
+  k_gemm<ASRC><<<grid, kGemmThreads, p.smem, s>>>(a, b, bx, g);
+  return launched("gemm");
+}
+
+qnf4_status launch_any(const GemmPlan& p, const CUtensorMap& a, const CUtensorMap& b,
+                       const CUtensorMap& bx, const GemmArgs& g, cudaStream_t s) {
+  switch (p.asrc) {
+    case A_NF4_K: return launch_gemm<A_NF4_K>(p, a, b, bx, g, s);
+    case A_NF4_MN: return launch_gemm<A_NF4_MN>(p, a, b, bx, g, s);
+    case A_DENSE_K: return launch_gemm<A_DENSE_K>(p, a, b, bx, g, s);
+    case A_DENSE_MN: return launch_gemm<A_DENSE_MN>(p, a, b, bx, g, s);
+    default: return launch_gemm<A_CHANQ_K>(p, a, b, bx, g, s);
+  }
+}
+
+GemmArgs base_args() {
+  GemmArgs g;
+  std::memset(&g, 0, sizeof(g));
+  const Nf4Tables& t = nf4_tables();
+  std::memcpy(g.levels, t.levels, sizeof(g.levels));
+  return g;
+}
+
+// The frozen base of one linear layer, in one of its three storage forms.
+struct BaseSrc {
+  int kind = A_NF4_K;        // A_NF4_K (NF4), A_DENSE_K (bf16), A_CHANQ_K (per-channel)
+  const qnf4_weight* w = nullptr;
+  const void* Wd = nullptr;  // dense bf16 [N, K]
+  const uint8_t* cq_packed = nullptr;
+  const int64_t* cq_row_off = nullptr;
+  const uint8_t* cq_bits = nullptr;
+  const float* cq_map = nullptr;
+  const int64_t* cq_map_off = nullptr;
+  const float* cq_absmax = nullptr;
+  int64_t N = 0, K = 0;
+};
+
+qnf4_status map_fail() { return fail(QNF4_ERR_CUDA, "cuTensorMapEncodeTiled unavailable or refused the layout"); }
+
+// u = x A^T (contraction K), written as bf16(scale u) into up [M, 64] and, when ut is
+// given, transposed into ut [r16, ldm].
+qnf4_status run_u(const LinPlan& L, const void* x, const void* A, int64_t M, int64_t K, int r,
+                  float scale, uint16_t* up, uint16_t* ut, float* part, unsigned* cnt, cudaStream_t s) {
+  CUtensorMap ma, mb, none;
+  std::memset(&none, 0, sizeof(none));
+  if (!make_map(&ma, x, false, K, M, K, 64, 128, true)) return map_fail();
+  if (!make_map(&mb, A, false, K, r, K, 64, L.r16, true)) return map_fail();
+  GemmArgs g = base_args();
+  g.epi = EPI_UV;
+  g.out = up;
+  g.out2 = ut;
+  g.o2_ld = L.ldm;
+  g.scale = scale;
+  g.part = part;
+  g.counters = cnt;
+  return launch_any(L.u, ma, mb, none, g, s);
+}
+
+qnf4_status linear_fwd(const BaseSrc& src, const void* x, int64_t M, const void* A, const void* B,
+                       int r, float scale, void* h, void* ws, size_t ws_bytes, cudaStream_t s) {
+  const int64_t N = src.N, K = src.K;
+  const LinPlan L = plan_linear(src.kind, N, K, M, r, false, num_sms());
+  if (!ws || ws_bytes < L.total) return fail(QNF4_ERR_WORKSPACE, "workspace too small (%zu < %zu)", ws_bytes, L.total);
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  uint16_t* up = reinterpret_cast<uint16_t*>(w8 + L.off_up);
+  float* part = reinterpret_cast<float*>(w8 + L.off_part);
+  unsigned* cnt = reinterpret_cast<unsigned*>(w8 + L.off_cnt);
+  if (cudaMemsetAsync(cnt, 0, L.total - L.off_cnt, s) != cudaSuccess) return launched("memset", 0);
+  qnf4_status st = run_u(L, x, A, M, K, r, scale, up, nullptr, part, cnt, s);
+  if (st != QNF4_OK) return st;
+  CUtensorMap ma, mb, mbx;
+  std::memset(&ma, 0, sizeof(ma));
+  const int tn = L.main.tn;
+  if (src.kind == A_NF4_K) {
+    if (!make_map(&ma, src.w->packed, true, K / 2, N, K / 2, 32, 128, false)) return map_fail();
+  } else if (src.kind == A_DENSE_K) {
+    if (!make_map(&ma, src.Wd, false, K, N, K, 64, 128, true)) return map_fail();
+  }
+  if (!make_map(&mb, x, false, K, M, K, 64, tn, true)) return map_fail();
+  if (!make_map(&mbx, up, false, 64, M, 64, 64, tn, true)) return map_fail();
+  GemmArgs g = base_args();
+  g.ext_k16 = L.r16 / 16;
+  g.ext_r = r;
+  g.ext_a = static_cast<const uint16_t*>(B);
+  g.ext_ld = r;
+  g.wN = N;
+  g.nbk = K / 64;
+  if (src.kind == A_NF4_K) {
+    g.code2 = src.w->code2;
+    g.scale2 = src.w->scale2;
+    g.mean = src.w->mean;
+  } else if (src.kind == A_CHANQ_K) {
+    g.cq_packed = src.cq_packed;
+    g.cq_row_off = src.cq_row_off;
+    g.cq_bits = src.cq_bits;
+    g.cq_map = src.cq_map;
+    g.cq_map_off = src.cq_map_off;
+    g.cq_absmax = src.cq_absmax;
+  }
+  g.epi = EPI_BF16;
+  g.out = h;
+  g.o_rs = 1;
+  g.o_cs = N;
+  g.part = part;
+  g.counters = cnt;
+  if (g_ev_start) cudaEventRecord(g_ev_start, s);
+  st = launch_any(L.main, ma, mb, mbx, g, s);
+  if (g_ev_stop) cudaEventRecord(g_ev_stop, s);
+  return st;
+}
+
+qnf4_status linear_bwd(const BaseSrc& src, const void* x, const void* dY, int64_t M, const void* A,
+                       const void* B, int r, float scale, void* dX, float* dA, float* dB, void* ws,
+                       size_t ws_bytes, cudaStream_t s) {
+  const int64_t N = src.N, K = src.K;
+  const int main_src = src.kind == A_NF4_K ? A_NF4_MN : A_DENSE_MN;
+  const LinPlan L = plan_linear(main_src, N, K, M, r, true, num_sms());
+  if (!ws || ws_bytes < L.total) return fail(QNF4_ERR_WORKSPACE, "workspace too small (%zu < %zu)", ws_bytes, L.total);
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  uint16_t* ut = reinterpret_cast<uint16_t*>(w8 + L.off_ut);
+  uint16_t* vp = reinterpret_cast<uint16_t*>(w8 + L.off_vp);
+  uint16_t* vt = reinterpret_cast<uint16_t*>(w8 + L.off_vt);
+  uint16_t* bt = reinterpret_cast<uint16_t*>(w8 + L.off_bt);
+  float* part = reinterpret_cast<float*>(w8 + L.off_part);
+  unsigned* cnt = reinterpret_cast<unsigned*>(w8 + L.off_cnt);
+  if (cudaMemsetAsync(cnt, 0, L.total - L.off_cnt, s) != cudaSuccess) return launched("memset", 0);
+  // B^T for v = dY B
+  {
+    const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((N * r + 255) / 256, num_sms() * 4)));
+    k_transpose_b<<<grid, 256, 0, s>>>(static_cast<const uint16_t*>(B), N, r, bt, L.ldn);
+    qnf4_status st = launched("transpose_b");
+    if (st != QNF4_OK) return st;
+  }
+  // (scale u)^T for dB
+  qnf4_status st = run_u(L, x, A, M, K, r, scale, nullptr, ut, part, cnt, s);
+  if (st != QNF4_OK) return st;
+  CUtensorMap none;
+  std::memset(&none, 0, sizeof(none));
+  // v = dY B  ->  vp = bf16(scale v) [M, 64], vt = its transpose [r16, ldm]
+  {
+    CUtensorMap ma, mb;
+    if (!make_map(&ma, dY, false, N, M, N, 64, 128, true)) return map_fail();
+    if (!make_map(&mb, bt, false, N, r, L.ldn, 64, L.r16, true)) return map_fail();
+    GemmArgs g = base_args();
+    g.epi = EPI_UV;
+    g.out = vp;
+    g.out2 = vt;
+    g.o2_ld = L.ldm;
+    g.scale = scale;
+    g.part = part;
+    g.counters = cnt;
+    st = launch_any(L.v, ma, mb, none, g, s);
+    if (st != QNF4_OK) return st;
+  }
+  // dX = dY W_hat + (scale v) A
+  {
+    CUtensorMap ma, mb, mbx;
+    const int tn = L.main.tn;
+    if (main_src == A_NF4_MN) {
+      if (!make_map(&ma, src.w->packed, true, K / 2, N, K / 2, 64, 64, false)) return map_fail();
+    } else {
+      if (!make_map(&ma, src.Wd, false, K, N, K, 64, 64, true)) return map_fail();
+    }
+    if (!make_map(&mb, dY, false, N, M, N, 64, tn, true)) return map_fail();
+    if (!make_map(&mbx, vp, false, 64, M, 64, 64, tn, true)) return map_fail();
+    GemmArgs g = base_args();
+    g.ext_k16 = L.r16 / 16;
+    g.ext_r = r;
+    g.ext_a = static_cast<const uint16_t*>(A);
+    g.ext_ld = K;
+    g.wN = N;
+    g.nbk = K / 64;
+    if (main_src == A_NF4_MN) {
+      g.code2 = src.w->code2;
+      g.scale2 = src.w->scale2;
+      g.mean = src.w->mean;
+    }
+    g.epi = EPI_BF16;
+    g.out = dX;
+    g.o_rs = 1;
+    g.o_cs = K;
+    g.part = part;
+    g.counters = cnt;
+    if (g_ev_start) cudaEventRecord(g_ev_start, s);
+    st = launch_any(L.main, ma, mb, mbx, g, s);
+    if (g_ev_stop) cudaEventRecord(g_ev_stop, s);
+    if (st != QNF4_OK) return st;
+  }
+  // dA = (scale v)^T x  -> [r, K]
+  {
+    CUtensorMap ma, mb;
+    if (!make_map(&ma, x, false, K, M, K, 64, 64, true)) return map_fail();
+    if (!make_map(&mb, vt, false, M, L.r16, L.ldm, 64, L.r16, true)) return map_fail();
+    GemmArgs g = base_args();
+    g.epi = EPI_F32;
+    g.out = dA;
+    g.o_rs = 1;
+    g.o_cs = K;
+    g.out_cols = r;
+    g.scale = 1.f;
+    g.part = part;
+    g.counters = cnt;
+    st = launch_any(L.da, ma, mb, none, g, s);
+    if (st != QNF4_OK) return st;
+  }
+  // dB = dY^T (scale u)  -> [N, r]
+  {
+    CUtensorMap ma, mb;
+    if (!make_map(&ma, dY, false, N, M, N, 64, 64, true)) return map_fail();
+    if (!make_map(&mb, ut, false, M, L.r16, L.ldm, 64, L.r16, true)) return map_fail();
+    GemmArgs g = base_args();
+    g.epi = EPI_F32;
+    g.out = dB;
+    g.o_rs = r;
+    g.o_cs = 1;
+    g.out_cols = r;
+    g.scale = 1.f;
+    g.part = part;
+    g.counters = cnt;
+    st = launch_any(L.db, ma, mb, none, g, s);
+    if (st != QNF4_OK) return st;
+  }
+  return QNF4_OK;
+}
+
+qnf4_status check_linear_args(int64_t N, int64_t K, int64_t M, int r, bool bwd,
+                              std::initializer_list<const void*> ptrs) {
+  if (N <= 0 || K <= 0) return fail(QNF4_ERR_SHAPE, "N and K must be positive");
+  if (K % 64) return fail(QNF4_ERR_SHAPE, "K must be a multiple of 64 (got %lld)", (long long)K);
+  if (bwd && N % 8) return fail(QNF4_ERR_SHAPE, "the backward needs N to be a multiple of 8 (got %lld)", (long long)N);
+  if (M < 0) return fail(QNF4_ERR_SHAPE, "M must be >= 0");
+  if (M > (int64_t)INT32_MAX) return fail(QNF4_ERR_SHAPE, "M too large");
+  if (r < 1 || r > 64) return fail(QNF4_ERR_ARG, "r must be in [1, 64] (got %d)", r);
+  for (const void* p : ptrs) {
+    if (!p) return fail(QNF4_ERR_ARG, "NULL buffer");
+    if (!al16(p)) return fail(QNF4_ERR_ALIGN, "buffers must be 16-byte aligned");
+  }
+  return QNF4_OK;
+}
+
+}  // namespace
+}  // namespace qnf4
+
+using namespace qnf4;
+
+extern "C" {
+
+qnf4_status qnf4_nf4_codebook(float levels[16], float thresholds[15]) {
+  const Nf4Tables& t = nf4_tables();
+  if (levels) std::memcpy(levels, t.levels, 16 * sizeof(float));
+  if (thresholds) std::memcpy(thresholds, t.thr, 15 * sizeof(float));
+  return QNF4_OK;
+}
+
+const char* qnf4_last_error(void) { return g_last.c_str(); }
+
+unsigned long long qnf4_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+qnf4_status qnf4_set_timing_events(void* start, void* stop) {
+  if ((start == nullptr) != (stop == nullptr)) return fail(QNF4_ERR_ARG, "give both events or neither");
+  g_ev_start = static_cast<cudaEvent_t>(start);
+  g_ev_stop = static_cast<cudaEvent_t>(stop);
+  return QNF4_OK;
+}
+
+qnf4_status qnf4_set_wait_timeout_ns(uint64_t ns) {
+  if (ns == 0) return fail(QNF4_ERR_ARG, "timeout must be positive");
+  g_wait_ns = ns;
+  return QNF4_OK;
+}
+
+qnf4_status qnf4_check(void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return fail(QNF4_ERR_CUDA, "stream: %s", cudaGetErrorString(e));
+  unsigned int flag = 0;
+  e = cudaMemcpyFromSymbol(&flag, g_qnf4_err, sizeof(flag));
+  if (e != cudaSuccess) return fail(QNF4_ERR_CUDA, "error flag: %s", cudaGetErrorString(e));
+  if (flag) {
+    const unsigned int zero = 0;
+    cudaMemcpyToSymbol(g_qnf4_err, &zero, sizeof(zero));
+    return fail(QNF4_ERR_TIMEOUT, "a kernel wait gave up (site %u)", flag);
+  }
+  return QNF4_OK;
+}
+
+size_t qnf4_workspace_size(int32_t op, int64_t N, int64_t K, int64_t M, int32_t r) {
+  switch (op) {
+    case QNF4_OP_QUANTIZE: return kQuantMaxGrid * sizeof(double);
+    case QNF4_OP_DOUBLE_QUANT: return kDqPartials * sizeof(double);
+    case QNF4_OP_FWD: return plan_linear(A_NF4_K, N, K, M, r, false, num_sms()).total;
+    case QNF4_OP_BWD: return plan_linear(A_NF4_MN, N, K, M, r, true, num_sms()).total;
+    case QNF4_OP_CHANQ_FWD: return plan_linear(A_CHANQ_K, N, K, M, r, false, num_sms()).total;
+    default: return 0;
+  }
+}
+
+qnf4_status qnf4_nf4_quantize(const void* W, int64_t N, int64_t K, int32_t block1, uint8_t* packed,
+                              float* absmax, double* sse, void* ws, size_t ws_bytes, void* stream) {
+  if (block1 != 64) return fail(QNF4_ERR_ARG, "block1 must be 64");
+  if (N < 0 || K <= 0) return fail(QNF4_ERR_SHAPE, "bad shape");
+  if (K % 64) return fail(QNF4_ERR_SHAPE, "K must be a multiple of 64");
+  if (!W || !packed || !absmax) return fail(QNF4_ERR_ARG, "NULL buffer");
+  if (!al16(W) || !al16(packed) || !al16(absmax) || (sse && !al16(sse)))
+    return fail(QNF4_ERR_ALIGN, "buffers must be 16-byte aligned");
+  if (sse && (!ws || ws_bytes < qnf4_workspace_size(QNF4_OP_QUANTIZE, N, K, 0, 0)))
+    return fail(QNF4_ERR_WORKSPACE, "workspace too small");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t nblocks = N * K / 64;
+  if (nblocks == 0) {
+    if (sse) cudaMemsetAsync(sse, 0, sizeof(double), s);
+    return launched("quantize(empty)", 0);
+  }
+  const int grid = quant_grid(nblocks);
+  const QuantTab tab = make_tab();
+  if (sse) {
+    k_nf4_quant<true, true><<<grid, 256, 0, s>>>(static_cast<const uint16_t*>(W), nblocks,
+                                                 reinterpret_cast<uint32_t*>(packed), absmax,
+                                                 static_cast<double*>(ws), tab);
+    k_sum_partials<<<1, 256, 0, s>>>(static_cast<const double*>(ws), grid, sse);
+    return launched("nf4_quantize", 2);
+  } else {
+    k_nf4_quant<true, false><<<grid, 256, 0, s>>>(static_cast<const uint16_t*>(W), nblocks,
+                                                  reinterpret_cast<uint32_t*>(packed), absmax,
+                                                  nullptr, tab);
+  }
+  return launched("nf4_quantize");
+}
+
+qnf4_status qnf4_nf4_recon_error(const void* W, int64_t N, int64_t K, int32_t block1, double* sse,
+                                 void* ws, size_t ws_bytes, void* stream) {
+  if (block1 != 64) return fail(QNF4_ERR_ARG, "block1 must be 64");
+  if (N < 0 || K <= 0) return fail(QNF4_ERR_SHAPE, "bad shape");
+  if (K % 64) return fail(QNF4_ERR_SHAPE, "K must be a multiple of 64");
+  if (!W || !sse) return fail(QNF4_ERR_ARG, "NULL buffer");
+  if (!al16(W) || !al16(sse)) return fail(QNF4_ERR_ALIGN, "buffers must be 16-byte aligned");
+  if (!ws || ws_bytes < qnf4_workspace_size(QNF4_OP_QUANTIZE, N, K, 0, 0))
+    return fail(QNF4_ERR_WORKSPACE, "workspace too small");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t nblocks = N * K / 64;
+  if (nblocks == 0) {
+    cudaMemsetAsync(sse, 0, sizeof(double), s);
+    return launched("recon_error(empty)", 0);
+  }
+  const int grid = quant_grid(nblocks);
+  k_nf4_quant<false, true><<<grid, 256, 0, s>>>(static_cast<const uint16_t*>(W), nblocks, nullptr,
+                                                nullptr, static_cast<double*>(ws), make_tab());
+  k_sum_partials<<<1, 256, 0, s>>>(static_cast<const double*>(ws), grid, sse);
+  return launched("nf4_recon_error", 2);
+}
+
+qnf4_status qnf4_double_quant(const float* absmax, int64_t nb1, int32_t block2, uint8_t* code2,
+                              float* scale2, float* mean, void* ws, size_t ws_bytes, void* stream) {
+  if (block2 != 256) return fail(QNF4_ERR_ARG, "block2 must be 256");
+  if (nb1 <= 0) return fail(QNF4_ERR_SHAPE, "nb1 must be positive");
+  if (!absmax || !code2 || !scale2 || !mean) return fail(QNF4_ERR_ARG, "NULL buffer");
+  if (!al16(absmax) || !al16(code2) || !al16(scale2) || !al16(mean))
+    return fail(QNF4_ERR_ALIGN, "buffers must be 16-byte aligned");
+  if (!ws || ws_bytes < qnf4_workspace_size(QNF4_OP_DOUBLE_QUANT, 0, 0, 0, 0))
+    return fail(QNF4_ERR_WORKSPACE, "workspace too small");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  double* part = static_cast<double*>(ws);
+  k_dq_partial<<<kDqPartials, 256, 0, s>>>(absmax, nb1, part);
+  const int64_t nb2 = (nb1 + 255) / 256;
+  int grid = static_cast<int>(std::min<int64_t>((nb2 + 7) / 8, num_sms() * 4));
+  grid = std::max(grid, 1);
+  k_dq_encode<<<grid, 256, 0, s>>>(absmax, nb1, part, kDqPartials, code2, scale2, mean);
+  return launched("double_quant", 2);
+}
+
+qnf4_status qnf4_dequant(const qnf4_weight* w, void* out, int32_t out_dtype, void* stream) {
+  qnf4_status st = check_weight(w);
+  if (st != QNF4_OK) return st;
+  if (!out) return fail(QNF4_ERR_ARG, "NULL output");
+  if (!al16(out)) return fail(QNF4_ERR_ALIGN, "output must be 16-byte aligned");
+  if (out_dtype != QNF4_OUT_F32 && out_dtype != QNF4_OUT_BF16)
+    return fail(QNF4_ERR_ARG, "out_dtype must be QNF4_OUT_F32 or QNF4_OUT_BF16");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t n8 = w->N * w->K / 8;
+  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((n8 + 255) / 256, num_sms() * 8)));
+  const QuantTab tab = make_tab();
+  const uint32_t* p = reinterpret_cast<const uint32_t*>(w->packed);
+  if (out_dtype == QNF4_OUT_BF16)
+    k_dequant<true><<<grid, 256, 0, s>>>(p, w->code2, w->scale2, w->mean, n8, out, tab);
+  else
+    k_dequant<false><<<grid, 256, 0, s>>>(p, w->code2, w->scale2, w->mean, n8, out, tab);
+  return launched("dequant");
+}
+
+qnf4_status qnf4_rank_topk(const double* sse, const int64_t* n_params, int32_t n_layers, int32_t k,
+                           int32_t* out) {
+  if (!sse || !n_params || (!out && k > 0)) return fail(QNF4_ERR_ARG, "NULL host buffer");
+  if (n_layers < 0 || k < 0 || k > n_layers) return fail(QNF4_ERR_ARG, "need 0 <= k <= n_layers");
+  std::vector<int32_t> idx(n_layers);
+  for (int32_t i = 0; i < n_layers; ++i) {
+    if (n_params[i] <= 0) return fail(QNF4_ERR_ARG, "n_params must be positive");
+    idx[i] = i;
+  }
+  // epsilon_i = sse_i / n_i, descending; ties to the lower index (stable)
+  std::stable_sort(idx.begin(), idx.end(), [&](int32_t a, int32_t b) {
+    return sse[a] / static_cast<double>(n_params[a]) > sse[b] / static_cast<double>(n_params[b]);
+  });
+  for (int32_t i = 0; i < k; ++i) out[i] = idx[i];
+  return QNF4_OK;
+}
+
+qnf4_status qnf4_chanq_quantize(const void* W, int64_t N, int64_t K, const uint8_t* bits,
+                                const float* thr, const int64_t* thr_off, uint8_t* packed,
+                                const int64_t* row_off, float* absmax, void* stream) {
+  if (N < 0 || K <= 0) return fail(QNF4_ERR_SHAPE, "bad shape");
+  if (K % 64) return fail(QNF4_ERR_SHAPE, "K must be a multiple of 64");
+  if (!W || !bits || !thr || !thr_off || !packed || !row_off || !absmax)
+    return fail(QNF4_ERR_ARG, "NULL buffer");
+  if (!al16(W) || !al16(bits) || !al16(thr) || !al16(thr_off) || !al16(packed) || !al16(row_off) ||
+      !al16(absmax))
+    return fail(QNF4_ERR_ALIGN, "buffers must be 16-byte aligned");
+  if (N == 0) return QNF4_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((N + 7) / 8, num_sms() * 8)));
+  k_chanq_quant<<<grid, 256, 0, s>>>(static_cast<const uint16_t*>(W), N, K, bits, thr, thr_off,
+                                     packed, row_off, absmax);
+  return launched("chanq_quantize");
+}
+
+qnf4_status qnf4_qlora_linear_fwd(const qnf4_weight* w, const void* x, int64_t M, const void* A,
+                                  const void* B, int32_t r, float scale, void* h, void* ws,
+                                  size_t ws_bytes, void* stream) {
+  qnf4_status st = check_weight(w);
+  if (st != QNF4_OK) return st;
+  st = check_linear_args(w->N, w->K, M, r, false, {x, A, B, h});
+  if (st != QNF4_OK) return st;
+  if (M == 0) return QNF4_OK;
+  BaseSrc src;
+  src.kind = A_NF4_K;
+  src.w = w;
+  src.N = w->N;
+  src.K = w->K;
+  return linear_fwd(src, x, M, A, B, r, scale, h, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+qnf4_status qnf4_qlora_linear_bwd(const qnf4_weight* w, const void* x, const void* dY, int64_t M,
+                                  const void* A, const void* B, int32_t r, float scale, void* dX,
+                                  float* dA, float* dB, void* ws, size_t ws_bytes, void* stream) {
+  qnf4_status st = check_weight(w);
+  if (st != QNF4_OK) return st;
+  st = check_linear_args(w->N, w->K, M, r, true, {x, dY, A, B, dX, dA, dB});
+  if (st != QNF4_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (M == 0) {
+    cudaMemsetAsync(dA, 0, sizeof(float) * r * w->K, s);
+    cudaMemsetAsync(dB, 0, sizeof(float) * r * w->N, s);
+    return launched("bwd(M=0)", 0);
+  }
+  BaseSrc src;
+  src.kind = A_NF4_K;
+  src.w = w;
+  src.N = w->N;
+  src.K = w->K;
+  return linear_bwd(src, x, dY, M, A, B, r, scale, dX, dA, dB, ws, ws_bytes, s);
+}
+
+qnf4_status qnf4_dense_linear_fwd(const void* W, int64_t N, int64_t K, const void* x, int64_t M,
+                                  const void* A, const void* B, int32_t r, float scale, void* h,
+                                  void* ws, size_t ws_bytes, void* stream) {
+  qnf4_status st = check_linear_args(N, K, M, r, false, {W, x, A, B, h});
+  if (st != QNF4_OK) return st;
+  if (M == 0) return QNF4_OK;
+  BaseSrc src;
+  src.kind = A_DENSE_K;
+  src.Wd = W;
+  src.N = N;
+  src.K = K;
+  return linear_fwd(src, x, M, A, B, r, scale, h, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+qnf4_status qnf4_dense_linear_bwd(const void* W, int64_t N, int64_t K, const void* x, const void* dY,
+                                  int64_t M, const void* A, const void* B, int32_t r, float scale,
+                                  void* dX, float* dA, float* dB, void* ws, size_t ws_bytes,
+                                  void* stream) {
+  qnf4_status st = check_linear_args(N, K, M, r, true, {W, x, dY, A, B, dX, dA, dB});
+  if (st != QNF4_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (M == 0) {
+    cudaMemsetAsync(dA, 0, sizeof(float) * r * K, s);
+    cudaMemsetAsync(dB, 0, sizeof(float) * r * N, s);
+    return launched("bwd(M=0)", 0);
+  }
+  BaseSrc src;
+  src.kind = A_DENSE_K;
+  src.Wd = W;
+  src.N = N;
+  src.K = K;
+  return linear_bwd(src, x, dY, M, A, B, r, scale, dX, dA, dB, ws, ws_bytes, s);
+}
+
+qnf4_status qnf4_chanq_linear_fwd(const uint8_t* packed, const int64_t* row_off, const uint8_t* bits,
+                                  const float* map, const int64_t* map_off, const float* absmax,
+                                  int64_t N, int64_t K, const void* x, int64_t M, const void* A,
+                                  const void* B, int32_t r, float scale, void* h, void* ws,
+                                  size_t ws_bytes, void* stream) {
+  qnf4_status st = check_linear_args(N, K, M, r, false, {packed, row_off, bits, map, map_off, absmax, x, A, B, h});
+  if (st != QNF4_OK) return st;
+  if (M == 0) return QNF4_OK;
+  BaseSrc src;
+  src.kind = A_CHANQ_K;
+  src.cq_packed = packed;
+  src.cq_row_off = row_off;
+  src.cq_bits = bits;
+  src.cq_map = map;
+  src.cq_map_off = map_off;
+  src.cq_absmax = absmax;
+  src.N = N;
+  src.K = K;
+  return linear_fwd(src, x, M, A, B, r, scale, h, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,600 @@
+// One tcgen05 (5th-generation tensor core) GEMM skeleton for every contraction of
+// the QLoRA linear layer, with the A operand produced in one of five ways.
+//
+//   D[rows, cols] = sum_c Aop[row, c] * Bop[col, c]   (+ one extra "LoRA" chunk)
+//
+// The M side of the MMA ("rows", 128 per CTA) is the A operand; the N side ("cols",
+// tn per CTA, 16..256) is the B operand, always bf16 and K-major, loaded by TMA with
+// the 128-byte swizzle. The contraction runs in steps of 64.
+//
+// A operand sources:
+//   A_NF4_K    packed NF4 weight, rows = output features, contraction = input features
+//              (forward h = x W^T). TMA brings the packed bytes; converter warps
+//              dequantize each 64-element block with its two-level constant and
+//              write bf16 into a K-major SW128 tile.
+//   A_NF4_MN   packed NF4 weight read transposed: rows = input features, contraction
+//              = output features (backward dX = dY W). Same converter, MN-major tile.
+//   A_DENSE_K  bf16 matrix by TMA, K-major (dense layers, x for u = x A^T, dY for v).
+//   A_DENSE_MN bf16 matrix by TMA, MN-major (dense dX, x^T for dA, dY^T for dB).
+//   A_CHANQ_K  per-output-channel 1/2/4-bit codes with per-row mapping tables.
+//
+// The extra chunk adds sum_j Aext[row, j] * Bext[col, j] over j < r into the same
+// TMEM accumulator: the rank-r adapter term of "QLoRA: Efficient Finetuning of
+// Quantized LLMs" (Heng's Blog, opening formula h = dequant(W0) x + (alpha/r) B A x).
+//
+// Roles (192 threads): warp 0 issues TMA, warp 1 allocates TMEM and one lane issues
+// tcgen05.mma, warps 2-5 ("converters") dequantize and then run the epilogue
+// (tcgen05.ld from TMEM, optional split-K reduction in the last-arriving CTA).
+// Every wait is bounded; on timeout the kernel records an error, stops, drains its
+// own copies and MMAs, frees TMEM and returns.
+#pragma once
+#include "common.cuh"
+
+namespace qnf4 {
+
+enum : int { A_NF4_K = 0, A_NF4_MN = 1, A_DENSE_K = 2, A_DENSE_MN = 3, A_CHANQ_K = 4 };
+enum : int { EPI_BF16 = 0, EPI_F32 = 1, EPI_UV = 2 };
+
+constexpr int kRowsTile = 128;
+constexpr int kStep = 64;
+constexpr int kGemmThreads = 192;
+constexpr uint32_t kATile = 128u * 128u;  // 128 rows x 64 bf16 (or 2 x 64 x 64 MN-major)
+constexpr uint32_t kPTile = 4096u;         // packed NF4 bytes of one step
+constexpr int kMaxS1 = 16;
+constexpr int kMaxS2 = 4;
+constexpr uint32_t kCqStride = 17;  // floats per row of the chanq table (padding vs conflicts)
+
+__host__ __device__ constexpr bool src_deq(int a) {
+  return a == A_NF4_K || a == A_NF4_MN || a == A_CHANQ_K;
+}
+__host__ __device__ constexpr bool src_mn(int a) { return a == A_NF4_MN || a == A_DENSE_MN; }
+__host__ __device__ constexpr bool src_dense(int a) { return a == A_DENSE_K || a == A_DENSE_MN; }
+__host__ __device__ constexpr bool src_packed_tma(int a) { return a == A_NF4_K || a == A_NF4_MN; }
+
+struct GemmArgs {
+  int64_t rows, cols;     // extents of D
+  int nsteps;             // contraction steps of 64 in total
+  int steps_per_split;    // steps per blockIdx.z slice
+  int splits;             // gridDim.z
+  int tn;                 // N tile: multiple of 16, 16..256
+  int s1, s2;             // depth of the load ring and of the dequantized-A ring
+  int has_ext;            // add the adapter chunk (in split 0)
+  int ext_k16;            // K=16 sub-steps of the adapter chunk (ceil(r/16))
+  int ext_r;              // adapter rank r
+  const uint16_t* ext_a;  // B [rows, r] (K-major chunk) or A [r, K] (MN-major chunk)
+  int64_t ext_ld;         // row stride of ext_a in elements
+  // two-level NF4 constants
+  const uint8_t* code2;
+  const float* scale2;
+  const float* mean;
+  int64_t nbk;            // 64-blocks per weight row (K / 64)
+  int64_t wN;             // weight rows (output features)
+  float levels[16];
+  // per-channel quantizer
+  const uint8_t* cq_packed;
+  const int64_t* cq_row_off;
+  const uint8_t* cq_bits;
+  const float* cq_map;
+  const int64_t* cq_map_off;
+  const float* cq_absmax;
+  // epilogue
+  int epi;
+  void* out;
+  int64_t o_rs, o_cs;     // element strides of out for row / col
+  int64_t out_cols;       // columns written (EPI_F32)
+  void* out2;             // EPI_UV: transposed copy, [col][row] with stride o2_ld
+  int64_t o2_ld;
+  float scale;
+  float* part;            // split-K partial tiles
+  unsigned int* counters; // split-K arrival counters (zero on entry, left zero)
+  unsigned long long wait_ns;
+};
+
+struct SmemPlan {
+  uint32_t off_a1, off_b1, off_p1, slot1, slot2, ring2, ext, cq, total;
+};
+
+__host__ __device__ inline SmemPlan smem_plan(int asrc, int tn, int s1, int s2, int has_ext) {
+  SmemPlan p{};
+  uint32_t o = 0;
+  p.off_a1 = o;
+  if (src_dense(asrc)) o += kATile;
+  p.off_b1 = o;
+  o += static_cast<uint32_t>(tn) * 128u;
+  p.off_p1 = o;
+  if (src_packed_tma(asrc)) o += kPTile;
+  p.slot1 = (o + 1023u) & ~1023u;
+  p.slot2 = src_deq(asrc) ? kATile : 0u;
+  p.ring2 = static_cast<uint32_t>(s1) * p.slot1;
+  p.ext = p.ring2 + static_cast<uint32_t>(s2) * p.slot2;
+  p.cq = p.ext + (has_ext ? kATile : 0u);
+  p.total = p.cq + (asrc == A_CHANQ_K ? 128u * kCqStride * 4u : 0u);
+  return p;
+}
+
+// ---------------------------------------------------------------------------
+// device helpers
+// ---------------------------------------------------------------------------
+QNF4_DEV bool wait_or_abort(uint64_t* bar, uint32_t parity, unsigned long long wait_ns,
+                            volatile int* abort_flag, unsigned int site) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer() - t0 > wait_ns) {
+      set_err(site);
+      *abort_flag = 1;
+      return false;
+    }
+  }
+}
+
+QNF4_DEV void named_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// Write one 128-byte row slot (64 bf16 given as 32 packed words) of a SW128 tile:
+// 16-byte chunk c of row t lands at chunk position c ^ (t & 7).
+QNF4_DEV void store_row_sw128(uint8_t* tile, int t, const uint32_t (&w)[32]) {
+  uint8_t* row = tile + t * 128;
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    uint4 v = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+    *reinterpret_cast<uint4*>(row + ((c ^ (t & 7)) << 4)) = v;
+  }
+}
+
+// Dequantize one NF4 block: 32 packed bytes (element 2j in the high nibble of byte j)
+// times the block constant, rounded to bf16.
+QNF4_DEV void nf4_block_to_bf16(const uint8_t* src, float ch, const float* s_lv,
+                                uint32_t (&o)[32]) {
+  const uint4 a = *reinterpret_cast<const uint4*>(src);
+  const uint4 b = *reinterpret_cast<const uint4*>(src + 16);
+  const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t byte = (w[i] >> (8 * j)) & 0xFFu;
+      const float f0 = s_lv[byte >> 4] * ch;
+      const float f1 = s_lv[byte & 0xFu] * ch;
+      o[4 * i + j] = pack_bf16x2(f0, f1);
+    }
+  }
+}
+
+// One 64-element group of a per-channel row with B-bit codes (MSB first).
+template <int B>
+QNF4_DEV void chanq_group_to_bf16(const uint8_t* src, float g, const float* tab,
+                                  uint32_t (&o)[32]) {
+  constexpr int NW = 2 * B;  // 32-bit words holding 64 codes
+  uint32_t w[NW];
+#pragma unroll
+  for (int i = 0; i < NW / 2; ++i) {
+    const uint2 v = __ldg(reinterpret_cast<const uint2*>(src) + i);
+    w[2 * i] = v.x;
+    w[2 * i + 1] = v.y;
+  }
+  constexpr uint32_t mask = (1u << B) - 1u;
+#pragma unroll
+  for (int e = 0; e < 64; e += 2) {
+    uint32_t c[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int bit = (e + h) * B;           // position in the MSB-first stream
+      const int byte = bit >> 3;
+      const int sh = 8 - B - (bit & 7);      // shift inside that byte
+      const uint32_t by = (w[byte >> 2] >> (8 * (byte & 3))) & 0xFFu;
+      c[h] = (by >> sh) & mask;
+    }
+    o[e >> 1] = pack_bf16x2(tab[c[0]] * g, tab[c[1]] * g);
+  }
+}
+
+QNF4_DEV uint16_t f2bf(float f) {
+  return static_cast<uint16_t>(pack_bf16x2(f, 0.f) & 0xFFFFu);
+}
+
+QNF4_DEV void epi_store(const GemmArgs& g, int64_t row, int64_t col0, const float* v, int n) {
+  if (row >= g.rows) return;
+  if (g.epi == EPI_BF16) {
+    uint16_t* o = static_cast<uint16_t*>(g.out);
+    for (int j = 0; j < n; ++j) {
+      const int64_t col = col0 + j;
+      if (col < g.cols) o[row * g.o_rs + col * g.o_cs] = f2bf(v[j]);
+    }
+  } else if (g.epi == EPI_F32) {
+    float* o = static_cast<float*>(g.out);
+    for (int j = 0; j < n; ++j) {
+      const int64_t col = col0 + j;
+      if (col < g.out_cols) o[row * g.o_rs + col * g.o_cs] = v[j] * g.scale;
+    }
+  } else {  // EPI_UV: rows are tokens, cols the adapter rank (padded)
+    uint16_t* p = static_cast<uint16_t*>(g.out);
+    uint16_t* pt = static_cast<uint16_t*>(g.out2);
+    for (int j = 0; j < n; ++j) {
+      const int64_t col = col0 + j;
+      const uint16_t b = f2bf(v[j] * g.scale);
+      if (p) p[row * 64 + col] = b;
+      if (pt) pt[col * g.o2_ld + row] = b;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// the kernel
+// ---------------------------------------------------------------------------
+template <int ASRC>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+           const __grid_constant__ CUtensorMap tmBx, const GemmArgs g) {
+  constexpr bool DEQ = src_deq(ASRC);
+  constexpr bool MN = src_mn(ASRC);
+  extern __shared__ uint8_t dsmem[];
+  __shared__ __align__(8) uint64_t full1[kMaxS1], empty1[kMaxS1], full2[kMaxS2], empty2[kMaxS2];
+  __shared__ __align__(8) uint64_t acc_bar, ext_bar, fin_bar;
+  __shared__ uint32_t s_tmem;
+  __shared__ volatile int s_abort;
+  __shared__ int s_last;
+  __shared__ float s_lv[16];
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const SmemPlan sp = smem_plan(ASRC, g.tn, g.s1, g.s2, g.has_ext);
+  const int S1 = g.s1, S2 = g.s2;
+  const int z = blockIdx.z;
+  const int step0 = z * g.steps_per_split;
+  const int nst = max(0, min(g.nsteps - step0, g.steps_per_split));
+  const bool ext = g.has_ext && z == 0;
+  const int nload = nst + (ext ? 1 : 0);
+  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * kRowsTile;
+  const int64_t col0 = static_cast<int64_t>(blockIdx.y) * g.tn;
+  uint32_t ncols = 32;
+  while (ncols < static_cast<uint32_t>(g.tn)) ncols <<= 1;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < S1; ++i) {
+      mbar_init(&full1[i], 1);
+      mbar_init(&empty1[i], 1);
+    }
+    for (int i = 0; i < S2; ++i) {
+      mbar_init(&full2[i], 128);
+      mbar_init(&empty2[i], 1);
+    }
+    mbar_init(&acc_bar, 1);
+    mbar_init(&ext_bar, 128);
+    mbar_init(&fin_bar, 1);
+    s_abort = 0;
+    s_last = 0;
+    fence_mbar_init();
+  }
+  if (threadIdx.x < 16) s_lv[threadIdx.x] = g.levels[threadIdx.x];
+  if (warp == 1) {
+    tmem_alloc(&s_tmem, ncols);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  if (warp == 0 && lane == 0) {
+    if (src_dense(ASRC) || src_packed_tma(ASRC)) tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+    if (ext) tma_prefetch_desc(&tmBx);
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int issued = 0;
+      for (int i = 0; i < nload; ++i) {
+        const int s = i % S1;
+        if (!wait_or_abort(&empty1[s], ((i / S1) & 1) ^ 1, g.wait_ns, &s_abort, 11)) break;
+        uint8_t* slot = base + s * sp.slot1;
+        if (i < nst) {
+          const int32_t kc = (step0 + i) * kStep;
+          uint32_t bytes = static_cast<uint32_t>(g.tn) * 128u;
+          if (src_dense(ASRC)) bytes += kATile;
+          if (src_packed_tma(ASRC)) bytes += kPTile;
+          mbar_expect_tx(&full1[s], bytes);
+          if (ASRC == A_DENSE_K) tma_load_2d(slot + sp.off_a1, &tmA, &full1[s], kc, (int32_t)row0);
+          if (ASRC == A_DENSE_MN) {
+            tma_load_2d(slot + sp.off_a1, &tmA, &full1[s], (int32_t)row0, kc);
+            tma_load_2d(slot + sp.off_a1 + 8192, &tmA, &full1[s], (int32_t)row0 + 64, kc);
+          }
+          if (ASRC == A_NF4_K) tma_load_2d(slot + sp.off_p1, &tmA, &full1[s], kc / 2, (int32_t)row0);
+          if (ASRC == A_NF4_MN) tma_load_2d(slot + sp.off_p1, &tmA, &full1[s], (int32_t)(row0 / 2), kc);
+          tma_load_2d(slot + sp.off_b1, &tmB, &full1[s], kc, (int32_t)col0);
+        } else {
+          mbar_expect_tx(&full1[s], static_cast<uint32_t>(g.tn) * 128u);
+          tma_load_2d(slot + sp.off_b1, &tmBx, &full1[s], 0, (int32_t)col0);
+        }
+        issued = i + 1;
+      }
+      // Drain: the last copy issued into each slot must land before the CTA exits.
+      // One deadline covers the whole drain.
+      const int nslots = min(issued, S1);
+      const uint64_t t0 = globaltimer();
+      bool late = false;
+      for (int s = 0; s < nslots && !late; ++s) {
+        const int j = s + S1 * ((issued - 1 - s) / S1);
+        while (!mbar_try_wait(&full1[s], (j / S1) & 1)) {
+          if (globaltimer() - t0 > g.wait_ns) {
+            set_err(12);
+            late = true;
+            break;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16(128, static_cast<uint32_t>(g.tn), MN ? 1u : 0u, 0u);
+      bool ok = true;
+      for (int i = 0; i < nst && ok; ++i) {
+        const int s = i % S1;
+        if (!wait_or_abort(&full1[s], (i / S1) & 1, g.wait_ns, &s_abort, 21)) { ok = false; break; }
+        uint8_t* slot = base + s * sp.slot1;
+        uint8_t* a = slot + sp.off_a1;
+        int s2 = 0;
+        if (DEQ) {
+          s2 = i % S2;
+          if (!wait_or_abort(&full2[s2], (i / S2) & 1, g.wait_ns, &s_abort, 22)) { ok = false; break; }
+          a = base + sp.ring2 + s2 * sp.slot2;
+        }
+        tc_fence_after();
+        const uint32_t aa = smem_u32(a), bb = smem_u32(slot + sp.off_b1);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t ad = MN ? smem_desc(aa + kk * 2048, 8192, 1024, kLayoutSW128)
+                                 : smem_desc(aa + kk * 32, 16, 1024, kLayoutSW128);
+          const uint64_t bd = smem_desc(bb + kk * 32, 16, 1024, kLayoutSW128);
+          mma_ss(tmem, ad, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(&empty1[s]);
+        if (DEQ) mma_commit(&empty2[s2]);
+      }
+      if (ok && ext) {
+        const int i = nst;
+        const int s = i % S1;
+        if (wait_or_abort(&full1[s], (i / S1) & 1, g.wait_ns, &s_abort, 23) &&
+            wait_or_abort(&ext_bar, 0, g.wait_ns, &s_abort, 24)) {
+          tc_fence_after();
+          const uint32_t aa = smem_u32(base + sp.ext);
+          const uint32_t bb = smem_u32(base + s * sp.slot1 + sp.off_b1);
+          for (int kk = 0; kk < g.ext_k16; ++kk) {
+            const uint64_t ad = MN ? smem_desc(aa + kk * 2048, 8192, 1024, kLayoutSW128)
+                                   : smem_desc(aa + kk * 32, 16, 1024, kLayoutSW128);
+            const uint64_t bd = smem_desc(bb + kk * 32, 16, 1024, kLayoutSW128);
+            mma_ss(tmem, ad, bd, idesc, (nst > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(&empty1[s]);
+        }
+      }
+      mma_commit(&acc_bar);
+      // Drain: every MMA of this CTA completes before TMEM and smem are released.
+      mma_commit(&fin_bar);
+      const uint64_t t0 = globaltimer();
+      while (!mbar_try_wait(&fin_bar, 0)) {
+        if (globaltimer() - t0 > g.wait_ns) {
+          set_err(25);
+          break;
+        }
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ converters
+    const int t = threadIdx.x - 64;  // row slot 0..127
+    if (ext) {
+      uint32_t w[32];
+      if (!MN) {
+        // row slot t = D row (row0 + t): adapter B[row, 0..r), zero padded to 64
+        const int64_t row = row0 + t;
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const int j0 = 2 * c;
+          uint32_t lo = 0, hi = 0;
+          if (row < g.rows) {
+            if (j0 < g.ext_r) lo = g.ext_a[row * g.ext_ld + j0];
+            if (j0 + 1 < g.ext_r) hi = g.ext_a[row * g.ext_ld + j0 + 1];
+          }
+          w[c] = lo | (hi << 16);
+        }
+      } else {
+        // MN-major: row slot t = (atom kb, contraction j); A[j, row0 + 64 kb .. +64)
+        const int kb = t >> 6, j = t & 63;
+        const int64_t k0 = row0 + kb * 64;
+        if (j < g.ext_r && k0 < g.rows) {
+          const uint4* src = reinterpret_cast<const uint4*>(g.ext_a + j * g.ext_ld + k0);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const uint4 v = src[c];
+            w[4 * c] = v.x; w[4 * c + 1] = v.y; w[4 * c + 2] = v.z; w[4 * c + 3] = v.w;
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) w[c] = 0u;
+        }
+      }
+      store_row_sw128(base + sp.ext, t, w);
+      fence_proxy_async();
+      mbar_arrive(&ext_bar);
+    }
+
+    if constexpr (ASRC == A_NF4_K || ASRC == A_NF4_MN) {
+      const float mu = *g.mean;
+      // constants of the block this slot dequantizes at step i
+      auto blk = [&](int i, int64_t& b) -> bool {
+        if (ASRC == A_NF4_K) {
+          const int64_t n = row0 + t;
+          b = n * g.nbk + (step0 + i);
+          return n < g.wN;
+        } else {
+          const int kb = t >> 6, nr = t & 63;
+          const int64_t n = static_cast<int64_t>(step0 + i) * kStep + nr;
+          const int64_t kblk = row0 / 64 + kb;
+          b = n * g.nbk + kblk;
+          return n < g.wN && kblk < g.nbk;
+        }
+      };
+      constexpr int PF = 4;  // constants are fetched PF steps ahead
+      uint32_t pc[PF];
+      float ps[PF];
+      bool pv[PF];
+#pragma unroll
+      for (int j = 0; j < PF; ++j) {
+        int64_t b = 0;
+        pv[j] = j < nst && blk(j, b);
+        pc[j] = pv[j] ? g.code2[b] : 0u;
+        ps[j] = pv[j] ? __ldg(g.scale2 + (b >> 8)) : 0.f;
+      }
+      for (int i = 0; i < nst; ++i) {
+        const int s = i % S1, s2 = i % S2;
+        const bool valid = pv[0];
+        const float ch = valid ? fmaf(e4m3_to_f32(static_cast<uint8_t>(pc[0])), ps[0], mu) : 0.f;
+#pragma unroll
+        for (int j = 0; j < PF - 1; ++j) {
+          pc[j] = pc[j + 1];
+          ps[j] = ps[j + 1];
+          pv[j] = pv[j + 1];
+        }
+        {
+          int64_t b = 0;
+          const int ii = i + PF;
+          pv[PF - 1] = ii < nst && blk(ii, b);
+          pc[PF - 1] = pv[PF - 1] ? g.code2[b] : 0u;
+          ps[PF - 1] = pv[PF - 1] ? __ldg(g.scale2 + (b >> 8)) : 0.f;
+        }
+        if (!wait_or_abort(&full1[s], (i / S1) & 1, g.wait_ns, &s_abort, 31)) break;
+        if (!wait_or_abort(&empty2[s2], ((i / S2) & 1) ^ 1, g.wait_ns, &s_abort, 32)) break;
+        const uint8_t* pk = base + s * sp.slot1 + sp.off_p1;
+        const uint8_t* src = (ASRC == A_NF4_K) ? pk + t * 32 : pk + (t & 63) * 64 + (t >> 6) * 32;
+        uint32_t o[32];
+        nf4_block_to_bf16(src, ch, s_lv, o);
+        store_row_sw128(base + sp.ring2 + s2 * sp.slot2, t, o);
+        fence_proxy_async();
+        mbar_arrive(&full2[s2]);
+      }
+    } else if constexpr (ASRC == A_CHANQ_K) {
+      const int64_t n = row0 + t;
+      const bool valid = n < g.wN;
+      int bits = 1;
+      const uint8_t* prow = nullptr;
+      float* tab = reinterpret_cast<float*>(base + sp.cq) + t * kCqStride;
+      if (valid) {
+        bits = g.cq_bits[n];
+        prow = g.cq_packed + g.cq_row_off[n];
+        const int64_t mo = g.cq_map_off[n];
+        for (int c = 0; c < (1 << bits); ++c) tab[c] = g.cq_map[mo + c];
+      }
+      for (int i = 0; i < nst; ++i) {
+        const int s = i % S1, s2 = i % S2;
+        const int gi = step0 + i;
+        if (!wait_or_abort(&full1[s], (i / S1) & 1, g.wait_ns, &s_abort, 33)) break;
+        if (!wait_or_abort(&empty2[s2], ((i / S2) & 1) ^ 1, g.wait_ns, &s_abort, 34)) break;
+        uint32_t o[32];
+        if (valid) {
+          const float gm = __ldg(g.cq_absmax + n * g.nbk + gi);
+          const uint8_t* src = prow + static_cast<int64_t>(gi) * 8 * bits;
+          if (bits == 4) chanq_group_to_bf16<4>(src, gm, tab, o);
+          else if (bits == 2) chanq_group_to_bf16<2>(src, gm, tab, o);
+          else chanq_group_to_bf16<1>(src, gm, tab, o);
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) o[c] = 0u;
+        }
+        store_row_sw128(base + sp.ring2 + s2 * sp.slot2, t, o);
+        fence_proxy_async();
+        mbar_arrive(&full2[s2]);
+      }
+    }
+
+    // ------------------------------------------------------------ epilogue
+    // The decision to write is taken once, so all 128 threads take the same path
+    // through the named barriers below.
+    wait_or_abort(&acc_bar, 0, g.wait_ns, &s_abort, 41);
+    named_sync(1, 128);
+    if (t == 0) s_last = s_abort ? 0 : 2;
+    named_sync(1, 128);
+    const bool have = s_last == 2;
+    named_sync(1, 128);
+    tc_fence_after();
+    const int q = warp & 3;
+    const int rl = q * 32 + lane;
+    const int64_t row = row0 + rl;
+    const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16);
+    if (have) {
+      if (g.splits == 1) {
+        for (int c0 = 0; c0 < g.tn; c0 += 16) {
+          uint32_t r[16];
+          tmem_ld16(taddr + c0, r);
+          tmem_wait_ld();
+          float v[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r[j]);
+          epi_store(g, row, col0 + c0, v, 16);
+        }
+      } else {
+        const int64_t tile = static_cast<int64_t>(blockIdx.y) * gridDim.x + blockIdx.x;
+        const int64_t tsz = static_cast<int64_t>(g.tn) * 128;
+        float* mine = g.part + (tile * g.splits + z) * tsz;
+        for (int c0 = 0; c0 < g.tn; c0 += 16) {
+          uint32_t r[16];
+          tmem_ld16(taddr + c0, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) __stcg(mine + (c0 + j) * 128 + rl, __uint_as_float(r[j]));
+        }
+        __threadfence();
+        named_sync(1, 128);
+        if (t == 0) {
+          const unsigned int old = atomicAdd(g.counters + tile, 1u);
+          s_last = (old == static_cast<unsigned int>(g.splits - 1)) ? 1 : 0;
+        }
+        named_sync(1, 128);
+        if (s_last) {
+          __threadfence();
+          const float* all = g.part + tile * g.splits * tsz;
+          for (int c0 = 0; c0 < g.tn; c0 += 16) {
+            float v[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v[j] = 0.f;
+            for (int zz = 0; zz < g.splits; ++zz) {
+#pragma unroll
+              for (int j = 0; j < 16; ++j) v[j] += __ldcg(all + zz * tsz + (c0 + j) * 128 + rl);
+            }
+            epi_store(g, row, col0 + c0, v, 16);
+          }
+          if (t == 0) g.counters[tile] = 0u;
+        }
+      }
+    }
+    tc_fence_before();
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, ncols);
+  }
+}
+
+// Transpose the adapter B [N, r] (bf16) into BT [r, ldn] so it can serve as a
+// K-major TMA operand of v = dY B.
+__global__ void __launch_bounds__(256) k_transpose_b(const uint16_t* __restrict__ B, int64_t N,
+                                                     int r, uint16_t* __restrict__ BT,
+                                                     int64_t ldn) {
+  const int64_t total = N * r;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t j = i / N, n = i - j * N;
+    BT[j * ldn + n] = B[n * r + j];
+  }
+}
+
+}  // namespace qnf4

@@ -1,0 +1,230 @@
+/*
+ * qnf4.h -- C ABI of libqnf4.so: a B200 (sm_100a) library for the QLoRA-style
+ * NF4-quantized linear layer.
+ *
+ * Sources (page title, section):
+ *   [QLoRA]  "QLoRA: Efficient Finetuning of Quantized LLMs" (Heng's Blog):
+ *            opening formula h = dequant(W0^NF4) x + (alpha/r) B A x;
+ *            贡献一 4-bit NormalFloat (NF4); 贡献二 Double Quantization.
+ *   [AQLoRA] "AQLoRA: a zero-search scheme for fast quantized LoRA fine-tuning",
+ *            §3.1 profiling pass (blockwise NF4 reconstruction error).
+ *   [LowRA]  "LowRA" article (cloud.tencent.com.cn), §4.1 per-output-channel
+ *            quantization, group normalisation, thresholds and mappings (Fig. 3).
+ *
+ * Conventions shared by every entry point:
+ *   - All buffers are allocated and owned by the caller. The library never
+ *     allocates or frees device memory and never synchronises the stream, except
+ *     qnf4_check(), which synchronises to read the device error flag.
+ *   - Pointers are device pointers unless the comment says "host".
+ *   - Every device pointer must be 16-byte aligned (QNF4_ERR_ALIGN otherwise).
+ *   - Matrices are row-major. W0 is [N, K] (N output features, K input features),
+ *     x is [M, K] (M tokens), A is [r, K], B is [N, r], h is [M, N].
+ *   - bf16 buffers are passed as void*; fp32 as float*.
+ *   - K must be a multiple of 64 (QNF4_ERR_SHAPE otherwise). block1 must be 64 and
+ *     block2 256 (the sizes the QLoRA page fixes); other values give QNF4_ERR_ARG.
+ *   - Arguments are validated on the host before any launch; a bad argument returns
+ *     without touching the GPU. A launch failure returns QNF4_ERR_CUDA. A kernel
+ *     whose bounded wait gives up sets a device flag that qnf4_check() reports as
+ *     QNF4_ERR_TIMEOUT. qnf4_last_error() gives a message for the calling thread.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL is the legacy default
+ *     stream) and is asynchronous to the host.
+ *   - Workspace: entry points with (ws, ws_bytes) need at least
+ *     qnf4_workspace_size(op, ...) bytes of device scratch (QNF4_ERR_WORKSPACE
+ *     otherwise). The contents need not be initialised. Calls that share a
+ *     workspace must be ordered on one stream.
+ */
+#ifndef QNF4_H
+#define QNF4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define QNF4_API __attribute__((visibility("default")))
+#else
+#define QNF4_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  QNF4_OK = 0,
+  QNF4_ERR_ARG = 1,
+  QNF4_ERR_SHAPE = 2,
+  QNF4_ERR_ALIGN = 3,
+  QNF4_ERR_CUDA = 4,
+  QNF4_ERR_TIMEOUT = 5,
+  QNF4_ERR_WORKSPACE = 6
+} qnf4_status;
+
+/* Output dtype selector for qnf4_dequant. */
+enum { QNF4_OUT_F32 = 0, QNF4_OUT_BF16 = 1 };
+
+/* Operation selector for qnf4_workspace_size. */
+enum {
+  QNF4_OP_QUANTIZE = 0,     /* qnf4_nf4_quantize (with sse) and qnf4_nf4_recon_error */
+  QNF4_OP_DOUBLE_QUANT = 1, /* qnf4_double_quant                                    */
+  QNF4_OP_FWD = 2,          /* qnf4_qlora_linear_fwd, qnf4_dense_linear_fwd          */
+  QNF4_OP_BWD = 3,          /* qnf4_qlora_linear_bwd, qnf4_dense_linear_bwd          */
+  QNF4_OP_CHANQ_FWD = 4     /* qnf4_chanq_linear_fwd                                 */
+};
+
+/* A double-quantized NF4 weight [QLoRA 贡献一/贡献二]. All pointers are device
+ * pointers owned by the caller.
+ *   packed : uint8 [N*K/2]. Row-major flattened codes; element 2j in the high nibble
+ *            of byte j, element 2j+1 in the low nibble.
+ *   code2  : uint8 [nb1], nb1 = N*K/64. OCP FP8 E4M3 code of each first-level
+ *            constant minus the tensor mean, divided by its 256-block scale.
+ *   scale2 : fp32 [nb2], nb2 = ceil(nb1/256). absmax of (c - mean) over the block / 448.
+ *   mean   : fp32 [1]. The tensor mean of the first-level constants.
+ * The first-level constant of block b is restored as fma(e4m3(code2[b]),
+ * scale2[b/256], mean); weight i of block b as levels[code_i] * that constant. */
+typedef struct {
+  int64_t N, K;
+  int32_t block1; /* 64  */
+  int32_t block2; /* 256 */
+  const uint8_t* packed;
+  const uint8_t* code2;
+  const float* scale2;
+  const float* mean;
+} qnf4_weight;
+
+/* [QLoRA 贡献一] The 16 NF4 levels (sorted, exact 0 at index 7, -1 and +1 at the
+ * ends) and the 15 fp32 decision thresholds: threshold k is the smallest fp32
+ * strictly above the exact midpoint of levels k and k+1, so that
+ * code = #{k : x >= threshold[k]} is the nearest level with ties to the lower one.
+ * Levels come from 9 (positive) and 8 (negative) evenly spaced probabilities
+ * between 1 - (1/32 + 1/30)/2 and 1/2, through the inverse normal CDF, the shared
+ * zero kept once, normalised by the largest magnitude and rounded once to fp32.
+ * Host pointers; either may be NULL. Never fails once the library is loaded. */
+QNF4_API qnf4_status qnf4_nf4_codebook(float levels[16], float thresholds[15]);
+
+/* [QLoRA 贡献一] Blockwise NF4 quantization of a bf16 weight W [N, K].
+ * For each 64-element block b of the row-major flattened W:
+ *   absmax[b] = max |w| (fp32, exact); x = fp32(w / absmax[b]) (IEEE division);
+ *   code = #{k : x >= threshold[k]}; an all-zero block gets absmax 0 and code 7.
+ * Outputs: packed uint8 [N*K/2] (nibble order as in qnf4_weight), absmax fp32
+ * [N*K/64]. If sse is not NULL it receives (device, 1 double) the sum over all
+ * elements of (w - fp32(levels[code] * absmax))^2, the single-level round-trip
+ * error [AQLoRA §3.1]; then ws must hold qnf4_workspace_size(QNF4_OP_QUANTIZE,...). */
+QNF4_API qnf4_status qnf4_nf4_quantize(const void* W_bf16, int64_t N, int64_t K, int32_t block1,
+                              uint8_t* packed, float* absmax, double* sse,
+                              void* ws, size_t ws_bytes, void* stream);
+
+/* [QLoRA 贡献二] Double quantization of the first-level constants absmax [nb1].
+ *   mean = fp32(float64 sum of absmax / nb1), one per tensor, written to mean[0];
+ *   for each 256-block j: scale2[j] = fp32(max_b |absmax[b] - mean| / 448);
+ *   code2[b] = E4M3 round-to-nearest-even, saturating, of fp32((absmax[b]-mean)/scale2[j]).
+ *   A block whose mean-subtracted constants are all zero stores scale2 0, code2 0.
+ * Outputs are device buffers: code2 uint8 [nb1], scale2 fp32 [ceil(nb1/256)],
+ * mean fp32 [1]. */
+QNF4_API qnf4_status qnf4_double_quant(const float* absmax, int64_t nb1, int32_t block2,
+                              uint8_t* code2, float* scale2, float* mean,
+                              void* ws, size_t ws_bytes, void* stream);
+
+/* [QLoRA opening formula, 贡献二] Two-level dequantization of a whole weight to
+ * out [N, K] as fp32 (out_dtype QNF4_OUT_F32) or bf16 round-to-nearest-even
+ * (QNF4_OUT_BF16). Meant for tests and export: the linear layer never writes the
+ * dequantized weight to memory. */
+QNF4_API qnf4_status qnf4_dequant(const qnf4_weight* w, void* out, int32_t out_dtype, void* stream);
+
+/* [QLoRA opening formula] h = x * bf16(W_hat)^T + scale * (x A^T) B^T, with W_hat
+ * the two-level dequantized NF4 weight, fp32 accumulation, h written as bf16 [M, N].
+ * x [M, K], A [r, K], B [N, r] are bf16. scale is alpha/r (or any adapter scale,
+ * e.g. rank-stabilised). 1 <= r <= 64. M >= 0 (M = 0 is a no-op). */
+QNF4_API qnf4_status qnf4_qlora_linear_fwd(const qnf4_weight* w, const void* x, int64_t M,
+                                  const void* A, const void* B, int32_t r, float scale,
+                                  void* h, void* ws, size_t ws_bytes, void* stream);
+
+/* [QLoRA opening formula: gradients reach only A and B through the frozen base]
+ * Given dY [M, N] bf16:
+ *   v  = dY B                          (fp32, internal)
+ *   dX = dY bf16(W_hat) + scale v A    bf16 [M, K]
+ *   dA = scale v^T x                   fp32 [r, K]   (written, not accumulated)
+ *   dB = scale dY^T (x A^T)            fp32 [N, r]   (written, not accumulated)
+ * There is no gradient for the frozen base. */
+QNF4_API qnf4_status qnf4_qlora_linear_bwd(const qnf4_weight* w, const void* x, const void* dY,
+                                  int64_t M, const void* A, const void* B, int32_t r,
+                                  float scale, void* dX, float* dA, float* dB,
+                                  void* ws, size_t ws_bytes, void* stream);
+
+/* [AQLoRA §3.1] Per-layer NF4 reconstruction error of a bf16 weight [N, K]:
+ * sse (device, 1 double) = sum over 64-blocks b of ||b - absmax-NF4^-1(absmax-NF4(b))||^2,
+ * single-level (no double quantization), fp32 dequant values, float64 accumulation.
+ * The caller divides by N*K for epsilon and ranks layers (qnf4_rank_topk). */
+QNF4_API qnf4_status qnf4_nf4_recon_error(const void* W_bf16, int64_t N, int64_t K, int32_t block1,
+                                 double* sse, void* ws, size_t ws_bytes, void* stream);
+
+/* [AQLoRA abstract, §3.1] Host helper: indices of the k layers with the largest
+ * epsilon = sse[i] / n_params[i], in descending order, ties to the lower index.
+ * Host pointers; out holds k entries. */
+QNF4_API qnf4_status qnf4_rank_topk(const double* sse, const int64_t* n_params, int32_t n_layers,
+                           int32_t k, int32_t* out);
+
+/* [AQLoRA abstract: protected layers stay 16-bit and skip dequantization] Dense
+ * bf16 variants of the linear layer for those layers: W_bf16 [N, K] replaces the
+ * NF4 weight; everything else is as in qnf4_qlora_linear_fwd / _bwd. */
+QNF4_API qnf4_status qnf4_dense_linear_fwd(const void* W_bf16, int64_t N, int64_t K, const void* x,
+                                  int64_t M, const void* A, const void* B, int32_t r,
+                                  float scale, void* h, void* ws, size_t ws_bytes,
+                                  void* stream);
+QNF4_API qnf4_status qnf4_dense_linear_bwd(const void* W_bf16, int64_t N, int64_t K, const void* x,
+                                  const void* dY, int64_t M, const void* A, const void* B,
+                                  int32_t r, float scale, void* dX, float* dA, float* dB,
+                                  void* ws, size_t ws_bytes, void* stream);
+
+/* [LowRA §4.1, Fig. 3] Per-output-channel threshold quantization of W [N, K] bf16.
+ * Row i uses bits[i] in {1, 2, 4} and its 2^b - 1 sorted fp32 bin edges
+ * thr[thr_off[i] .. thr_off[i+1]). Per 64-element group: absmax[g] = max |w|;
+ * x = fp32(w / absmax[g]) (0 for an all-zero group); code = #{k : x > edge_k}.
+ * Row i's codes are written MSB-first, b bits each, at packed + row_off[i]
+ * (row_off [N+1] int64 byte offsets, row_off[i+1] - row_off[i] = K*b/8).
+ * bits, thr, thr_off, row_off are device pointers; absmax is fp32 [N*K/64]. */
+QNF4_API qnf4_status qnf4_chanq_quantize(const void* W_bf16, int64_t N, int64_t K, const uint8_t* bits,
+                                const float* thr, const int64_t* thr_off, uint8_t* packed,
+                                const int64_t* row_off, float* absmax, void* stream);
+
+/* [LowRA §3 (per-channel dequant kernel used in fine-tuning), §4.1] Forward of the
+ * linear layer over a per-channel quantized base:
+ *   w_hat[i, j] = fp32(map[map_off[i] + code_ij] * absmax[group]), rounded to bf16,
+ *   h = x w_hat^T + scale (x A^T) B^T, fp32 accumulation, h bf16 [M, N].
+ * map fp32 with 2^bits[i] entries per row at map_off[i] (map_off [N+1] int64). */
+QNF4_API qnf4_status qnf4_chanq_linear_fwd(const uint8_t* packed, const int64_t* row_off,
+                                  const uint8_t* bits, const float* map, const int64_t* map_off,
+                                  const float* absmax, int64_t N, int64_t K, const void* x,
+                                  int64_t M, const void* A, const void* B, int32_t r, float scale,
+                                  void* h, void* ws, size_t ws_bytes, void* stream);
+
+/* Bytes of device workspace an operation needs for these sizes (0 if none). */
+QNF4_API size_t qnf4_workspace_size(int32_t op, int64_t N, int64_t K, int64_t M, int32_t r);
+
+/* Synchronise `stream`, then report and clear the device error flag: QNF4_OK, or
+ * QNF4_ERR_TIMEOUT if a bounded wait inside a kernel gave up since the last check,
+ * or QNF4_ERR_CUDA if the stream holds a CUDA error. */
+QNF4_API qnf4_status qnf4_check(void* stream);
+
+/* Upper bound, in nanoseconds, on any single wait inside a kernel before it gives
+ * up with QNF4_ERR_TIMEOUT (default 1e9). Applies to kernels launched afterwards. */
+QNF4_API qnf4_status qnf4_set_wait_timeout_ns(uint64_t ns);
+
+/* Number of kernels this library has launched in this process (all threads, all
+ * devices). Memsets are not counted. For benchmarks that report their launches. */
+QNF4_API unsigned long long qnf4_launch_count(void);
+
+/* Profiling hook. While set (non-NULL), every linear forward / backward call made
+ * from the calling thread records the cudaEvent_t `start` on its stream right before
+ * launching its dequant-GEMM kernel (the forward h GEMM, or the backward dX GEMM)
+ * and `stop` right after it, so the caller can time that kernel alone. Both or
+ * neither (NULL, NULL turns it off). The events are owned by the caller. */
+QNF4_API qnf4_status qnf4_set_timing_events(void* start, void* stop);
+
+/* Message describing the last error returned on the calling thread. */
+QNF4_API const char* qnf4_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QNF4_H */

@@ -1,0 +1,163 @@
+"""GPU parity of the fused tcgen05 linear layer against the float64 oracle.
+
+h = x bf16(W_hat)^T + s (x A^T) B^T and its backward (dX, dA, dB) through the frozen
+NF4 base, the dense-base variant for protected layers and the per-channel quantized
+forward. The GPU receives the oracle's quantized weight, so these tests isolate the
+GEMM path. Tolerance (bf16 inputs, fp32 accumulation): max|err| <= 2e-2 max|ref| and
+relative Frobenius error <= 5e-3, element by element over every output (or over
+sampled token rows of the largest prefill shapes, where the oracle's float64 GEMM
+would take minutes).
+"""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import chanq as ochq
+from oracle import linear as olin
+
+from helpers import (assert_close, chanq_oracle, dev, f32, f64, oracle_base_bf16,
+                     oracle_quant, weight_from_oracle)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def q():
+    import bit_nf4_quantized_04_b200 as q
+    return q
+
+
+def _inputs(N, K, M, r, seed, wstd=0.02):
+    W = synth.llama_weight((N, K), seed, std=wstd)
+    x = synth.normal_bf16((M, K), 1.0, seed + 1)
+    A = synth.normal_bf16((r, K), 0.01, seed + 2)
+    B = synth.normal_bf16((N, r), 0.01, seed + 3)
+    dY = synth.normal_bf16((M, N), 1.0, seed + 4)
+    return W, x, A, B, dY
+
+
+def _run_nf4(q, N, K, M, r, seed, bwd=True, rows=None):
+    W, x, A, B, dY = _inputs(N, K, M, r, seed)
+    s = 2.0 / r * 8  # an alpha/r-like scale
+    oq = oracle_quant(W)
+    Wb = oracle_base_bf16(oq, N, K)
+    w = weight_from_oracle(q, oq, N, K)
+    xc, Ac, Bc, dYc = x.cuda(), A.cuda(), B.cuda(), dY.cuda()
+    h = q.qlora_linear_fwd(w, xc, Ac, Bc, s)
+    sel = np.arange(M) if rows is None else rows
+    xs = f64(x)
+    href = olin.forward(xs[sel], Wb, f64(A), f64(B), s)
+    assert_close(f64(h.cpu())[sel], href, f"h N={N} K={K} M={M} r={r}")
+    if not bwd:
+        return
+    dX, dA, dB = q.qlora_linear_bwd(w, xc, dYc, Ac, Bc, s)
+    torch.cuda.synchronize()
+    dYs = f64(dY)
+    v = dYs @ f64(B)
+    dXref = dYs[sel] @ Wb + s * (v[sel] @ f64(A))
+    assert_close(f64(dX.cpu())[sel], dXref, f"dX N={N} K={K} M={M} r={r}")
+    dAref = s * (v.T @ xs)
+    dBref = s * (dYs.T @ (xs @ f64(A).T))
+    assert_close(dA.cpu().double().numpy(), dAref, "dA")
+    assert_close(dB.cpu().double().numpy(), dBref, "dB")
+
+
+def test_tiny_layer_fwd_bwd(q):
+    t = synth.tiny_inputs()
+    W, x, A, B, dY, r, alpha = t["W"], t["x"], t["A"], t["B"], t["dY"], t["r"], t["alpha"]
+    N, K = W.shape
+    s = alpha / r
+    oq = oracle_quant(W)
+    Wb = oracle_base_bf16(oq, N, K)
+    w = weight_from_oracle(q, oq, N, K)
+    h = q.qlora_linear_fwd(w, x.cuda(), A.cuda(), B.cuda(), s)
+    assert_close(f64(h.cpu()), olin.forward(f64(x), Wb, f64(A), f64(B), s), "h")
+    dX, dA, dB = q.qlora_linear_bwd(w, x.cuda(), dY.cuda(), A.cuda(), B.cuda(), s)
+    rdX, rdA, rdB = olin.backward(f64(x), f64(dY), Wb, f64(A), f64(B), s)
+    assert_close(f64(dX.cpu()), rdX, "dX")
+    assert_close(dA.cpu().double().numpy(), rdA, "dA")
+    assert_close(dB.cpu().double().numpy(), rdB, "dB")
+
+
+@pytest.mark.parametrize("N,K,M,r", [
+    (200, 192, 3, 5),      # ragged N, three contraction steps, odd rank
+    (384, 640, 17, 16),
+    (136, 128, 130, 33),   # M spans two token tiles, r spans three K=16 sub-steps
+    (256, 256, 1, 64),     # single token, largest rank
+    (128, 1024, 300, 24),
+    (264, 320, 64, 8),
+])
+def test_ragged_shapes(q, N, K, M, r):
+    _run_nf4(q, N, K, M, r, seed=N * 7 + K + M + r)
+
+
+@pytest.mark.parametrize("M", [1, 4, 16])
+def test_llama7b_decode_shapes(q, M):
+    # q_proj and down_proj (K = 11008: 172 blocks per row, unaligned constant rows)
+    _run_nf4(q, 4096, 4096, M, 16, seed=1000, bwd=False)
+    _run_nf4(q, 4096, 11008, M, 16, seed=1006, bwd=False)
+
+
+def test_llama7b_prefill_q_proj_sampled(q):
+    rows = np.array([0, 1, 255, 256, 1000, 2047, 3071, 4095])
+    _run_nf4(q, 4096, 4096, 4096, 16, seed=1000, bwd=True, rows=rows)
+
+
+def test_zero_adapter_is_base_only(q):
+    N, K, M, r = 256, 512, 40, 8
+    W, x, A, B, _ = _inputs(N, K, M, r, 31)
+    w = q.quantize_weight(W.cuda())
+    h0 = q.qlora_linear_fwd(w, x.cuda(), A.cuda(), torch.zeros_like(B).cuda(), 2.0)
+    h1 = q.qlora_linear_fwd(w, x.cuda(), torch.zeros_like(A).cuda(), B.cuda(), 2.0)
+    assert torch.equal(h0, h1)
+
+
+def test_dense_base_fwd_bwd(q):
+    N, K, M, r = 384, 512, 100, 16
+    W, x, A, B, dY = _inputs(N, K, M, r, 41)
+    s = 2.0
+    Wd = f64(W)
+    h = q.dense_linear_fwd(W.cuda(), x.cuda(), A.cuda(), B.cuda(), s)
+    assert_close(f64(h.cpu()), olin.forward(f64(x), Wd, f64(A), f64(B), s), "dense h")
+    dX, dA, dB = q.dense_linear_bwd(W.cuda(), x.cuda(), dY.cuda(), A.cuda(), B.cuda(), s)
+    rdX, rdA, rdB = olin.backward(f64(x), f64(dY), Wd, f64(A), f64(B), s)
+    assert_close(f64(dX.cpu()), rdX, "dense dX")
+    assert_close(dA.cpu().double().numpy(), rdA, "dense dA")
+    assert_close(dB.cpu().double().numpy(), rdB, "dense dB")
+
+
+def _chanq_case(N, K, seed):
+    W = synth.llama_weight((N, K), seed)
+    bits = synth.chan_bits(N)
+    maps, map_off, thr, thr_off = synth.chan_tables(bits, seed=seed + 5)
+    roff = torch.from_numpy(ochq.row_offsets(bits.numpy(), K))
+    return W, bits, maps, map_off, thr, thr_off, roff
+
+
+@pytest.mark.parametrize("N,K", [(40, 128), (200, 448), (1100, 4096)])
+def test_chanq_quantize_bit_exact(q, N, K):
+    W, bits, maps, map_off, thr, thr_off, roff = _chanq_case(N, K, 500 + N)
+    packed, roff_o, g, _ = chanq_oracle(W, bits, thr, thr_off)
+    assert np.array_equal(roff.numpy(), roff_o)
+    gp, gg = q.chanq_quantize(W.cuda(), bits.cuda(), thr.cuda(), thr_off.cuda(), roff.cuda())
+    torch.cuda.synchronize()
+    assert np.array_equal(gg.cpu().numpy().view(np.uint32), g.view(np.uint32))
+    assert np.array_equal(gp.cpu().numpy()[: packed.size], packed)
+
+
+@pytest.mark.parametrize("N,K,M,r", [(40, 128, 5, 8), (200, 448, 70, 16), (1100, 4096, 260, 16)])
+def test_chanq_linear_fwd(q, N, K, M, r):
+    W, bits, maps, map_off, thr, thr_off, roff = _chanq_case(N, K, 600 + N)
+    packed, roff_o, g, _ = chanq_oracle(W, bits, thr, thr_off)
+    x = synth.normal_bf16((M, K), 1.0, 71)
+    A = synth.normal_bf16((r, K), 0.01, 72)
+    B = synth.normal_bf16((N, r), 0.01, 73)
+    s = 2.0
+    wh = ochq.dequant(packed, roff_o, bits.numpy(), maps.numpy(), map_off.numpy(), g, N, K)
+    href = olin.forward(f64(x), olin.base_bf16(wh), f64(A), f64(B), s)
+    pk = np.zeros(max(packed.size, 16), np.uint8)
+    pk[: packed.size] = packed
+    h = q.chanq_linear_fwd(dev(pk), roff.cuda(), bits.cuda(), maps.cuda(), map_off.cuda(),
+                           dev(g), N, K, x.cuda(), A.cuda(), B.cuda(), s)
+    assert_close(f64(h.cpu()), href, "chanq h")

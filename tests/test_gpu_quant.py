@@ -1,0 +1,119 @@
+"""GPU parity of the bandwidth kernels against the CPU oracle, element by element:
+NF4 codes and packed bytes, block constants, double-quantization codes/scales/mean
+(bit-exact), two-level dequantization (fp32 within 1e-6 relative, bf16 exact) and
+the AQLoRA reconstruction error (1e-5 relative), on the tiny layer, ragged shapes and
+full Llama-2-7B matrix shapes.
+"""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import nf4 as onf4
+from oracle import numerics as onum
+
+from helpers import dev, f32, oracle_quant, weight_from_oracle
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def q():
+    import bit_nf4_quantized_04_b200 as q
+    return q
+
+
+def _check_quant(q, W):
+    N, K = W.shape
+    oq = oracle_quant(W)
+    packed, absmax = q.nf4_quantize(W.cuda())
+    torch.cuda.synchronize()
+    assert np.array_equal(absmax.cpu().numpy().view(np.uint32), oq["absmax"].view(np.uint32))
+    got = packed.cpu().numpy()
+    if not np.array_equal(got, oq["packed"]):
+        bad = np.nonzero(got != oq["packed"])[0]
+        raise AssertionError(f"{bad.size} packed bytes differ, first at {bad[:5]}")
+    return oq
+
+
+def _crafted(N, K, seed):
+    g = torch.Generator().manual_seed(seed)
+    w = torch.randn(N, K, generator=g) * 0.02
+    flat = w.view(-1)
+    if flat.numel() >= 64:
+        flat[0:64] = 0.0                      # all-zero block
+    if flat.numel() >= 128:
+        flat[64:128] = 0.03125                # identical values
+    if flat.numel() >= 192:
+        flat[128:160] = -1e-30                # tiny constants: one block through the
+        flat[130] = 1e-30                     # reciprocal shortcut, one through the
+        flat[160:192] = 3e-33                 # exact-division path (absmax < 2^-100)
+    if flat.numel() >= 256:
+        q = torch.tensor(onf4.codebook())     # values on the grid and at midpoints
+        mid = (q[1:] + q[:-1]) / 2
+        blk = torch.cat([q, mid, q[:16] * 0.5, mid[:15] * 0.25, torch.tensor([1.0, -1.0])])[:64]
+        flat[192:256] = blk * 0.5
+    return w.to(torch.bfloat16)
+
+
+def test_quantize_tiny_layer(q):
+    _check_quant(q, synth.tiny_inputs()["W"])
+
+
+@pytest.mark.parametrize("N,K", [(1, 64), (3, 128), (5, 192), (7, 640), (33, 320), (300, 448)])
+def test_quantize_ragged_and_crafted(q, N, K):
+    _check_quant(q, _crafted(N, K, N * 1000 + K))
+
+
+@pytest.mark.parametrize("idx", [0, 4, 6])
+def test_quantize_llama7b_shapes(q, idx):
+    s = synth.LLAMA7B_SET[idx]
+    W = synth.llama_weight((s.N, s.K), synth.SEED_W + idx)
+    _check_quant(q, W)
+
+
+def _check_dq(q, absmax):
+    c2, s2, mu = onf4.double_quant(absmax)
+    g2, gs2, gmu = q.double_quant(dev(absmax))
+    torch.cuda.synchronize()
+    assert np.float32(gmu.item()) == mu
+    assert np.array_equal(gs2.cpu().numpy().view(np.uint32), s2.view(np.uint32))
+    diff = int(np.sum(g2.cpu().numpy() != c2))
+    assert diff == 0, f"{diff} of {c2.size} double-quantization codes differ"
+
+
+def test_double_quant_tiny_and_ragged(q):
+    _check_dq(q, oracle_quant(synth.tiny_inputs()["W"])["absmax"])
+    for N, K in [(3, 128), (7, 640), (300, 448)]:
+        _check_dq(q, oracle_quant(_crafted(N, K, 7 + N))["absmax"])
+    _check_dq(q, np.full(700, 0.25, np.float32))  # zero-spread blocks
+
+
+def test_double_quant_llama7b_gate(q):
+    W = synth.llama_weight((11008, 4096), synth.SEED_W + 4)
+    _, absmax = q.nf4_quantize(W.cuda())
+    _check_dq(q, absmax.cpu().numpy())
+
+
+@pytest.mark.parametrize("N,K", [(256, 512), (7, 640), (4096, 4096)])
+def test_dequant_two_level(q, N, K):
+    W = synth.llama_weight((N, K), 77 + N) if N > 8 else _crafted(N, K, 5)
+    oq = oracle_quant(W)
+    w = weight_from_oracle(q, oq, N, K)
+    ref = onf4.dequant(oq["packed"], oq["code2"], oq["scale2"], oq["mean"], N * K).reshape(N, K)
+    got = q.dequant(w, torch.float32).cpu().numpy()
+    rel = np.abs(got.astype(np.float64) - ref) / np.maximum(np.abs(ref).astype(np.float64), 1e-30)
+    assert float(rel.max()) <= 1e-6
+    gb = q.dequant(w, torch.bfloat16).view(torch.int16).cpu().numpy().view(np.uint16)
+    assert np.array_equal(gb, onum.f32_to_bf16_bits(ref))
+
+
+@pytest.mark.parametrize("N,K", [(256, 512), (33, 320), (4096, 11008)])
+def test_recon_error(q, N, K):
+    W = synth.llama_weight((N, K), 99 + N, std=0.013)
+    ref = onf4.recon_sse(f32(W))
+    got = q.nf4_recon_error(W.cuda()).item()
+    assert abs(got - ref) <= 1e-5 * ref
+    # the same figure from the quantize pass with its SSE output on
+    _, _, s = q.nf4_quantize(W.cuda(), sse=True)
+    assert abs(s.item() - ref) <= 1e-5 * ref
