@@ -1,0 +1,552 @@
+#!/usr/bin/env python
+"""Throughput of the QLoRA NF4 linear-layer hot path on B200.
+
+One step = one pass of the whole hot path over the Llama-2-7B layer set
+(q, k, v, o 4096x4096; gate, up 11008x4096; down 4096x11008; synthetic N(0, 0.02)
+weights with 0.1% Student-t(3) outliers):
+  * NF4 blockwise quantization of every bf16 weight, with the single-level
+    reconstruction error (AQLoRA layer-ranking statistic) from the same pass,
+    then double quantization of the block constants;
+  * the fused forward h = x W^T + s (x A^T) B^T and backward (dX, dA, dB) of every
+    layer at 4096 tokens (batch 4 x 1024), r = 16, alpha = 32;
+  * the per-output-channel 1/2/4-bit quantizer and its forward on an 11008x4096
+    weight at 2048 tokens.
+value = fwd + bwd + per-channel-forward FLOPs of the step / step time (TFLOP/s),
+with every other piece of the step inside the timed region.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU (torchrun): each rank runs its own copy of the step (independent layer
+sets, no collective on the data path: weak scaling); the time is the max over ranks.
+--impl reference times the CPU oracle (the plain NumPy restatement of the pages) on
+a bounded sample of the same step on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+M_TOK = 4096          # 4 x 1024 tokens
+RANK = 16
+ALPHA = 32.0
+CQ_N, CQ_K, CQ_M = 11008, 4096, 2048
+WORKLOAD = ("llama2-7b layer set (q,k,v,o 4096x4096; gate,up 11008x4096; down 4096x11008), "
+            "4096 tokens, LoRA r=16 alpha=32: NF4 quantize + recon error + double quant, "
+            "fused fwd+bwd; plus per-channel 1/2/4-bit quantize + fwd (11008x4096, 2048 tokens)")
+
+
+# ----------------------------------------------------------------------------- helpers
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return (float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d["bf16_tflops_sustained"]),
+                "measured")
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+class Clocks:
+    """nvidia-smi sampler of SM clock and throttle reasons while work runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: int):
+        self.proc = None
+        self.rows = []
+        try:
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", uuid, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out = ""
+        for line in out.strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9:
+                self.rows.append(parts)
+
+    def summary(self):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in self.rows if num(r[1]) is not None]
+        mx = [num(r[2]) for r in self.rows if num(r[2]) is not None]
+        load = [s for s in sm if s > 500] or sm
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in self.rows for i in range(4)
+                          if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(load) if load else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(self.rows)}
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        n = [d.get("num_threads", 1) for d in info if d.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+# ------------------------------------------------------------------------ flop / byte models
+def layer_shapes():
+    import synth
+    return [(s.N, s.K) for s in synth.LLAMA7B_SET]
+
+
+def fwd_flops(N, K, M, r):
+    return 2.0 * M * N * K + 2.0 * M * r * (N + K)
+
+
+def bwd_flops(N, K, M, r):
+    return 2.0 * M * N * K + 4.0 * M * r * (N + K)
+
+
+def step_flops():
+    f = sum(fwd_flops(N, K, M_TOK, RANK) + bwd_flops(N, K, M_TOK, RANK) for N, K in layer_shapes())
+    return f + fwd_flops(CQ_N, CQ_K, CQ_M, RANK)
+
+
+# ------------------------------------------------------------------------------ CPU oracle
+def oracle_sample(rows: int = 4096, m: int = 128):
+    """Time the oracle, as it stands, on a bounded sample of the step: NF4 quantize +
+    double quant + recon error of the first `rows` rows of the q_proj matrix (4096
+    columns), and its fwd + bwd for m of the 4096 tokens.
+    Returns (TFLOP/s, seconds, description, flops)."""
+    import synth
+    from oracle import linear as olin
+    from oracle import nf4 as onf4
+    N, K, r = rows, 4096, RANK
+    W = synth.llama_weight((4096, K), synth.SEED_W)[:N].float().numpy()
+    x = synth.normal_bf16((m, K), 1.0, synth.SEED_X).double().numpy()
+    A = synth.normal_bf16((r, K), 0.01, synth.SEED_A).double().numpy()
+    B = synth.normal_bf16((N, r), 0.01, synth.SEED_B).double().numpy()
+    dY = synth.normal_bf16((m, N), 1.0, synth.SEED_DY).double().numpy()
+    s = ALPHA / r
+    t0 = time.perf_counter()
+    codes, c = onf4.quantize(W)
+    code2, s2, mu = onf4.double_quant(c)
+    onf4.recon_sse(W)
+    wb = olin.base_bf16(onf4.dequant(onf4.pack(codes), code2, s2, mu, N * K).reshape(N, K))
+    olin.forward(x, wb, A, B, s)
+    olin.backward(x, dY, wb, A, B, s)
+    dt = time.perf_counter() - t0
+    flops = fwd_flops(N, K, m, r) + bwd_flops(N, K, m, r)
+    desc = (f"q_proj rows 0..{N} of 4096 (x4096 cols): NF4 quantize + double quant + recon "
+            f"error + dequant, then fwd+bwd on {m} of 4096 tokens (r={r}); "
+            "TFLOP/s = sample fwd+bwd FLOPs / time")
+    return flops / dt / 1e12, dt, desc, flops
+
+
+# ------------------------------------------------------------------------------ GPU arm
+class Workload:
+    """Device-resident inputs, outputs and workspace of one step."""
+
+    def __init__(self, q, dev, seed_offset=0):
+        import synth
+        self.q = q
+        self.dev = dev
+        self.s = ALPHA / RANK
+        self.layers = []
+        wsz = 0
+        for i, (N, K) in enumerate(layer_shapes()):
+            L = {}
+            L["N"], L["K"] = N, K
+            L["W"] = synth.llama_weight((N, K), synth.SEED_W + i + seed_offset, device=dev)
+            L["x"] = synth.normal_bf16((M_TOK, K), 1.0, synth.SEED_X + i, device=dev)
+            L["dY"] = synth.normal_bf16((M_TOK, N), 1.0, synth.SEED_DY + i, device=dev)
+            L["A"] = synth.normal_bf16((RANK, K), 0.01, synth.SEED_A + i, device=dev)
+            L["B"] = synth.normal_bf16((N, RANK), 0.01, synth.SEED_B + i, device=dev)
+            n = N * K
+            L["packed"] = torch.empty(n // 2, dtype=torch.uint8, device=dev)
+            L["absmax"] = torch.empty(n // 64, dtype=torch.float32, device=dev)
+            L["sse"] = torch.empty(2, dtype=torch.float64, device=dev)
+            nb2 = (n // 64 + 255) // 256
+            L["code2"] = torch.empty(n // 64, dtype=torch.uint8, device=dev)
+            L["scale2"] = torch.empty(nb2, dtype=torch.float32, device=dev)
+            L["mean"] = torch.empty(4, dtype=torch.float32, device=dev)
+            L["w"] = q.Nf4Weight(N, K, L["packed"], L["code2"], L["scale2"], L["mean"][:1])
+            L["h"] = torch.empty(M_TOK, N, dtype=torch.bfloat16, device=dev)
+            L["dX"] = torch.empty(M_TOK, K, dtype=torch.bfloat16, device=dev)
+            L["dA"] = torch.empty(RANK, K, dtype=torch.float32, device=dev)
+            L["dB"] = torch.empty(N, RANK, dtype=torch.float32, device=dev)
+            for op, m in ((q._lib.OP_QUANTIZE, 0), (q._lib.OP_DOUBLE_QUANT, 0),
+                          (q._lib.OP_FWD, M_TOK), (q._lib.OP_BWD, M_TOK)):
+                wsz = max(wsz, q.workspace_size(op, N, K, m, RANK))
+            self.layers.append(L)
+        # per-channel mixed precision layer
+        bits = synth.chan_bits(CQ_N)
+        maps, map_off, thr, thr_off = synth.chan_tables(bits)
+        rowbytes = CQ_K * bits.to(torch.int64) // 8
+        roff = torch.zeros(CQ_N + 1, dtype=torch.int64)
+        roff[1:] = torch.cumsum(rowbytes, 0)
+        self.cq = dict(
+            W=synth.llama_weight((CQ_N, CQ_K), synth.SEED_W + 100 + seed_offset, device=dev),
+            bits=bits.to(dev), maps=maps.to(dev), map_off=map_off.to(dev), thr=thr.to(dev),
+            thr_off=thr_off.to(dev), roff=roff.to(dev),
+            packed=torch.empty(int(roff[-1]) + 16, dtype=torch.uint8, device=dev),
+            absmax=torch.empty(CQ_N * CQ_K // 64, dtype=torch.float32, device=dev),
+            x=synth.normal_bf16((CQ_M, CQ_K), 1.0, synth.SEED_X + 50, device=dev),
+            A=synth.normal_bf16((RANK, CQ_K), 0.01, synth.SEED_A + 50, device=dev),
+            B=synth.normal_bf16((CQ_N, RANK), 0.01, synth.SEED_B + 50, device=dev),
+            h=torch.empty(CQ_M, CQ_N, dtype=torch.bfloat16, device=dev))
+        wsz = max(wsz, q.workspace_size(q._lib.OP_CHANQ_FWD, CQ_N, CQ_K, CQ_M, RANK))
+        self.ws = torch.empty(wsz, dtype=torch.uint8, device=dev)
+
+    # the pieces of one step
+    def quantize(self):
+        q = self.q
+        for L in self.layers:
+            q.nf4_quantize(L["W"], sse=True, packed=L["packed"], absmax=L["absmax"],
+                           sse_out=L["sse"], ws=self.ws)
+            q.double_quant(L["absmax"], code2=L["code2"], scale2=L["scale2"], mean=L["mean"],
+                           ws=self.ws)
+
+    def fwd(self, ev=None):
+        for i, L in enumerate(self.layers):
+            if ev is not None:
+                self.q.lib.qnf4_set_timing_events(ev[i][0].cuda_event, ev[i][1].cuda_event)
+            self.q.qlora_linear_fwd(L["w"], L["x"], L["A"], L["B"], self.s, h=L["h"], ws=self.ws)
+        if ev is not None:
+            self.q.lib.qnf4_set_timing_events(None, None)
+
+    def bwd(self, ev=None):
+        for i, L in enumerate(self.layers):
+            if ev is not None:
+                self.q.lib.qnf4_set_timing_events(ev[i][0].cuda_event, ev[i][1].cuda_event)
+            self.q.qlora_linear_bwd(L["w"], L["x"], L["dY"], L["A"], L["B"], self.s, dX=L["dX"],
+                                    dA=L["dA"], dB=L["dB"], ws=self.ws)
+        if ev is not None:
+            self.q.lib.qnf4_set_timing_events(None, None)
+
+    def chanq(self):
+        c = self.cq
+        self.q.chanq_quantize(c["W"], c["bits"], c["thr"], c["thr_off"], c["roff"],
+                              packed=c["packed"], absmax=c["absmax"])
+        self.q.chanq_linear_fwd(c["packed"], c["roff"], c["bits"], c["maps"], c["map_off"],
+                                c["absmax"], CQ_N, CQ_K, c["x"], c["A"], c["B"], self.s, h=c["h"],
+                                ws=self.ws)
+
+    def step(self, evf=None, evb=None):
+        self.quantize()
+        self.fwd(evf)
+        self.bwd(evb)
+        self.chanq()
+
+    def inputs(self):
+        """Every tensor the step reads from outside (for the end-to-end copies)."""
+        out = []
+        for L in self.layers:
+            out += [L["W"], L["x"], L["dY"], L["A"], L["B"]]
+        c = self.cq
+        out += [c["W"], c["x"], c["A"], c["B"], c["bits"], c["maps"], c["map_off"], c["thr"],
+                c["thr_off"], c["roff"]]
+        return out
+
+    def results(self):
+        """The step's training result read back by the host: adapter gradients and the
+        per-layer reconstruction errors."""
+        out = []
+        for L in self.layers:
+            out += [L["dA"], L["dB"], L["sse"][:1]]
+        return out
+
+
+def nbytes(ts):
+    return sum(t.numel() * t.element_size() for t in ts)
+
+
+def time_loop(fn, iters, stream):
+    s = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    s.record(stream)
+    for _ in range(iters):
+        fn()
+    e.record(stream)
+    e.synchronize()
+    return s.elapsed_time(e) / 1e3 / iters
+
+
+def breakdown(wl, q, hbm, tc_sus):
+    """Per-row throughput, each timed alone (short loops, L2-exceeding inputs)."""
+    st = torch.cuda.current_stream()
+    out = {}
+    nparam = sum(N * K for N, K in layer_shapes())
+    t = time_loop(wl.quantize, 10, st)
+    gbs = nparam * (2 + 0.5 + 1 / 64 + 4 / 16384) / t / 1e9
+    out["quant_dq_sse"] = {"GBps": round(gbs, 1), "frac_hbm": round(gbs / hbm, 3),
+                           "bytes_per_param": 2.5159}
+    t = time_loop(lambda: [q.nf4_recon_error(L["W"], sse=L["sse"], ws=wl.ws) for L in wl.layers],
+                  10, st)
+    gbs = nparam * 2 / t / 1e9
+    out["recon_error"] = {"GBps": round(gbs, 1), "frac_hbm": round(gbs / hbm, 3)}
+    ff = sum(fwd_flops(N, K, M_TOK, RANK) for N, K in layer_shapes())
+    bf = sum(bwd_flops(N, K, M_TOK, RANK) for N, K in layer_shapes())
+    t = time_loop(wl.fwd, 5, st)
+    out["fwd_prefill"] = {"TFLOPs": round(ff / t / 1e12, 1), "frac_tc": round(ff / t / 1e12 / tc_sus, 3)}
+    t = time_loop(wl.bwd, 5, st)
+    out["bwd_prefill"] = {"TFLOPs": round(bf / t / 1e12, 1), "frac_tc": round(bf / t / 1e12 / tc_sus, 3)}
+    c = wl.cq
+    t = time_loop(lambda: q.chanq_quantize(c["W"], c["bits"], c["thr"], c["thr_off"], c["roff"],
+                                           packed=c["packed"], absmax=c["absmax"]), 10, st)
+    nb = CQ_N * CQ_K * (2 + 4 / 64) + float(c["roff"][-1].item())
+    out["chanq_quantize"] = {"GBps": round(nb / t / 1e9, 1), "frac_hbm": round(nb / t / 1e9 / hbm, 3)}
+    cf = fwd_flops(CQ_N, CQ_K, CQ_M, RANK)
+    t = time_loop(lambda: q.chanq_linear_fwd(c["packed"], c["roff"], c["bits"], c["maps"],
+                                             c["map_off"], c["absmax"], CQ_N, CQ_K, c["x"], c["A"],
+                                             c["B"], wl.s, h=c["h"], ws=wl.ws), 5, st)
+    out["chanq_fwd"] = {"TFLOPs": round(cf / t / 1e12, 1), "frac_tc": round(cf / t / 1e12 / tc_sus, 3)}
+    # decode (memory-bound): rotate over weight copies whose total exceeds L2 twice over
+    l2 = torch.cuda.get_device_properties(wl.dev).L2_cache_size
+    wbytes = sum(L["w"].nbytes() for L in wl.layers)
+    copies = max(2, int(2 * l2 // wbytes) + 1)
+    pool = [[q.Nf4Weight(L["N"], L["K"], L["packed"].clone(), L["code2"].clone(),
+                         L["scale2"].clone(), L["mean"].clone()[:1]) for L in wl.layers]
+            for _ in range(copies)]
+    dec = {}
+    for m in (1, 4, 16):
+        xs = [L["x"][:m].contiguous() for L in wl.layers]
+        hs = [torch.empty(m, L["N"], dtype=torch.bfloat16, device=wl.dev) for L in wl.layers]
+        ctr = [0]
+
+        def run():
+            ws_ = pool[ctr[0] % copies]
+            ctr[0] += 1
+            for i, L in enumerate(wl.layers):
+                q.qlora_linear_fwd(ws_[i], xs[i], L["A"], L["B"], wl.s, h=hs[i], ws=wl.ws)
+        run()
+        t = time_loop(run, 3 * copies, st)
+        byt = sum(N * K * (0.5 + 1 / 64 + 4 / 16384) + m * K * 2 + RANK * (N + K) * 2 + m * N * 2
+                  for N, K in layer_shapes())
+        dec[f"M{m}"] = {"GBps": round(byt / t / 1e9, 1), "frac_hbm": round(byt / t / 1e9 / hbm, 3),
+                        "us": round(t * 1e6, 1)}
+    out["decode_fwd"] = dec
+    out["decode_fwd"]["pool_copies"] = copies
+    return out
+
+
+def traffic_for(kernel: str):
+    """DRAM bytes per unit of work from the committed ncu summary, if it was taken on
+    the current source of the GEMM kernel; else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        d = json.load(open(p))
+        src = open(os.path.join(ROOT, "bit_nf4_quantized_04_b200", "csrc", "gemm.cuh"), "rb").read()
+        if d.get("gemm_sha1") != hashlib.sha1(src).hexdigest():
+            return None
+        return d["kernels"].get(kernel)
+    except Exception:
+        return None
+
+
+def run_ours(args):
+    ws_, rank, local = dist_env()
+    if ws_ > 1:
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    import bit_nf4_quantized_04_b200 as q
+    hbm, tc_burst, tc_sus, peak_kind = peaks()
+    wl = Workload(q, dev, seed_offset=0)
+    stream = torch.cuda.current_stream()
+    K, W = args.steps, args.warmup
+    evf = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(K * 7)]
+    evb = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(K * 7)]
+    for _ in range(W):
+        wl.step()
+    q.check()
+    clocks = Clocks(local)
+    if ws_ > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_stop = torch.cuda.Event(enable_timing=True)
+    n0 = q.lib.qnf4_launch_count()
+    t_start.record(stream)
+    for k in range(K):
+        wl.step(evf[7 * k:7 * k + 7], evb[7 * k:7 * k + 7])
+    t_stop.record(stream)
+    torch.cuda.synchronize()
+    n1 = q.lib.qnf4_launch_count()
+    if ws_ > 1:
+        torch.distributed.barrier()
+    elapsed = t_start.elapsed_time(t_stop) / 1e3
+    q.check()
+    if ws_ > 1:
+        tt = torch.tensor([elapsed], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+        elapsed = float(tt.item())
+    # dominant kernel: the fwd h GEMM or the bwd dX GEMM, whichever took longer
+    tf = sum(a.elapsed_time(b) for a, b in evf) / 1e3
+    tb = sum(a.elapsed_time(b) for a, b in evb) / 1e3
+    shapes = layer_shapes()
+    fl_f = sum(2.0 * M_TOK * N * K + 2.0 * M_TOK * RANK * N for N, K in shapes) * K
+    fl_b = sum(2.0 * M_TOK * N * K + 2.0 * M_TOK * RANK * K for N, K in shapes) * K
+    if tf >= tb:
+        kname, kt, kfl = "k_gemm<A_NF4_K> (fwd h = x W^T + LoRA)", tf, fl_f
+    else:
+        kname, kt, kfl = "k_gemm<A_NF4_MN> (bwd dX = dY W + LoRA)", tb, fl_b
+    achieved = kfl / kt / 1e12
+    tr = traffic_for("k_gemm<A_NF4_K>" if tf >= tb else "k_gemm<A_NF4_MN>")
+    flops = step_flops()
+    value = flops * K * ws_ / elapsed / 1e12
+    extra = {}
+    if not args.no_breakdown:
+        extra = breakdown(wl, q, hbm, tc_sus)
+    clocks.stop()
+    # end to end through the public API: pinned host inputs in, gradients out, per step
+    ins = wl.inputs()
+    host_in = [t.cpu().pin_memory() for t in ins]
+    res = wl.results()
+    host_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in res]
+    h2d, d2h = nbytes(ins), nbytes(res)
+    ke = max(1, min(K, 5))
+
+    def e2e_step():
+        for d, h in zip(ins, host_in):
+            d.copy_(h, non_blocking=True)
+        wl.step()
+        for h, d in zip(host_out, res):
+            h.copy_(d, non_blocking=True)
+    e2e_step()
+    torch.cuda.synchronize()
+    if ws_ > 1:
+        torch.distributed.barrier()
+    te = time_loop(e2e_step, ke, stream)
+    if ws_ > 1:
+        tt = torch.tensor([te], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+        te = float(tt.item())
+    e2e_value = flops * ws_ / te / 1e12
+    cpu = None
+    if rank == 0 and ws_ == 1 and not args.no_cpu:
+        v, dt, desc, _ = oracle_sample()
+        cpu = {"value": round(v, 6), "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": desc, "seconds": round(dt, 2)}
+    if rank == 0:
+        l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+        touched = sum(nbytes([L["W"], L["x"], L["dY"], L["h"], L["dX"], L["packed"]]) for L in wl.layers)
+        line = {
+            "metric": "QLoRA NF4 linear fwd+bwd TFLOP/s & GB/s (% roofline); NF4 quant+DQ GB/s",
+            "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": ws_, "steps": K, "warmup": W,
+            "ms_per_step": round(elapsed / K * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "tokens": M_TOK, "r": RANK, "alpha": ALPHA,
+                       "layers": 7, "params": sum(N * K for N, K in shapes),
+                       "flops_per_step": flops, "parallelism": f"independent replicas x{ws_}",
+                       "l2": f"inputs larger than L2: {touched / 1e9:.2f} GB touched per step "
+                             f"vs {l2 / 1e6:.0f} MB L2"},
+            "roofline": {"bound": "tensor", "kernel": kname, "achieved": round(achieved, 1),
+                         "peak": tc_sus, "unit": "TFLOP/s", "frac": round(achieved / tc_sus, 3),
+                         "peak_kind": f"{peak_kind} bf16 sustained",
+                         "traffic": tr * (kfl / K / sum(2.0 * M_TOK * N * K for N, K in shapes))
+                         if tr else None},
+            "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": int(n1 - n0),
+            "clocks": clocks.summary(),
+            "cpu_baseline": cpu,
+            "breakdown": extra,
+        }
+        print(json.dumps(line), flush=True)
+    if ws_ > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+def run_reference(args):
+    ws_, rank, _ = dist_env()
+    if rank != 0:
+        return
+    K, W = args.steps, args.warmup
+    # each step: a ~1 s sample of the step (512 weight rows, 128 tokens)
+    for _ in range(W):
+        oracle_sample(rows=512)
+    times = []
+    desc = ""
+    flops = 0.0
+    for _ in range(K):
+        _, dt, desc, flops = oracle_sample(rows=512)
+        times.append(dt)
+    tot = sum(times)
+    value = flops * K / tot / 1e12
+    line = {
+        "impl": "reference",
+        "metric": "QLoRA NF4 linear fwd+bwd TFLOP/s & GB/s (% roofline); NF4 quant+DQ GB/s",
+        "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": ws_, "steps": K, "warmup": W,
+        "ms_per_step": round(tot / K * 1e3, 1), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "tokens": M_TOK, "r": RANK, "alpha": ALPHA,
+                   "sample": desc},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": blas_threads(),
+                         "kind": "oracle", "sample": desc},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-breakdown", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()
