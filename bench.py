@@ -397,6 +397,12 @@ def run_ours(args):
            for _ in range(K * 7)]
     evb = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(K * 7)]
+    # torch creates the CUDA event behind an Event on its first record: do that now, so
+    # the library's hook receives live handles
+    for a, b in evf + evb:
+        a.record(stream)
+        b.record(stream)
+    torch.cuda.synchronize()
     for _ in range(W):
         wl.step()
     q.check()
@@ -499,6 +505,39 @@ def run_ours(args):
         torch.distributed.destroy_process_group()
 
 
+def run_case(args):
+    """One operation on one gate-shaped layer (11008x4096 NF4 weight), warmup + steps
+    launches and nothing else: the small, L2-exceeding case for ncu captures."""
+    import synth
+    import bit_nf4_quantized_04_b200 as q
+    dev = torch.device("cuda", 0)
+    N, K = 11008, 4096
+    m = {"fwd": M_TOK, "bwd": M_TOK, "decode": 16}.get(args.case, M_TOK)
+    W = synth.llama_weight((N, K), synth.SEED_W + 4, device=dev)
+    x = synth.normal_bf16((m, K), 1.0, synth.SEED_X, device=dev)
+    dY = synth.normal_bf16((m, N), 1.0, synth.SEED_DY, device=dev)
+    A = synth.normal_bf16((RANK, K), 0.01, synth.SEED_A, device=dev)
+    B = synth.normal_bf16((N, RANK), 0.01, synth.SEED_B, device=dev)
+    w = q.quantize_weight(W)
+    s = ALPHA / RANK
+    wsz = max(q.workspace_size(q._lib.OP_FWD, N, K, m, RANK),
+              q.workspace_size(q._lib.OP_BWD, N, K, m, RANK),
+              q.workspace_size(q._lib.OP_QUANTIZE, N, K))
+    ws = torch.empty(wsz, dtype=torch.uint8, device=dev)
+    h = torch.empty(m, N, dtype=torch.bfloat16, device=dev)
+    if args.case in ("fwd", "decode"):
+        fn = lambda: q.qlora_linear_fwd(w, x, A, B, s, h=h, ws=ws)  # noqa: E731
+    elif args.case == "bwd":
+        fn = lambda: q.qlora_linear_bwd(w, x, dY, A, B, s, ws=ws)  # noqa: E731
+    else:  # quant
+        fn = lambda: q.nf4_quantize(W, sse=True, ws=ws)  # noqa: E731
+    for _ in range(args.warmup + args.steps):
+        fn()
+    torch.cuda.synchronize()
+    q.check()
+    print(json.dumps({"case": args.case, "N": N, "K": K, "M": m, "launches": args.warmup + args.steps}))
+
+
 def run_reference(args):
     ws_, rank, _ = dist_env()
     if rank != 0:
@@ -539,7 +578,12 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-breakdown", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--case", choices=["fwd", "bwd", "decode", "quant"], default=None,
+                    help="run one operation on one gate-shaped layer (for ncu captures)")
     args = ap.parse_args()
+    if args.case:
+        run_case(args)
+        return
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
     if args.impl == "reference":
