@@ -71,8 +71,8 @@ QuantTab make_tab() {
   QuantTab q;
   std::memcpy(q.thr, t.thr, sizeof(q.thr));
   std::memcpy(q.levels, t.levels, sizeof(q.levels));
-  q.nbins = t.nbins;
-  std::memcpy(q.bin_code, t.bin_code, sizeof(q.bin_code));
+  q.bin_h = t.bin_h;
+  std::memcpy(q.bin_tc, t.bin_tc, sizeof(q.bin_tc));
   return q;
 }
 
@@ -143,6 +143,7 @@ struct GemmPlan {
   int asrc = 0, tn = 16, has_ext = 0;
   int64_t rows = 0, cols = 0;
   int nsteps = 0, row_tiles = 0, col_tiles = 0, splits = 1, steps_per_split = 0, s1 = 1, s2 = 0;
+  int ctas_per_sm = 1;
   size_t smem = 0;
   size_t part_floats() const {
     return splits > 1 ? static_cast<size_t>(row_tiles) * col_tiles * splits * tn * 128 : 0;
@@ -171,35 +172,28 @@ GemmPlan plan_gemm(int asrc, int64_t rows, int64_t cols, int64_t contraction, in
   p.nsteps = static_cast<int>((contraction + kStep - 1) / kStep);
   p.row_tiles = static_cast<int>((rows + kRowsTile - 1) / kRowsTile);
   p.col_tiles = static_cast<int>((cols + tn - 1) / tn);
-  // Split the contraction only when the output tiles leave SMs idle. The cost model
-  // is waves x steps per CTA (one CTA per SM), ties to fewer splits.
+  // Thin N tiles (decode, rank-r GEMMs) are latency bound: give them two CTAs per SM
+  // and a shallower dequant ring; wide tiles take the whole shared memory.
+  const bool thin = tn <= 32;
+  p.ctas_per_sm = thin ? 2 : 1;
+  p.s2 = src_deq(asrc) ? (thin ? 2 : (tn <= 64 ? 4 : 2)) : 0;
+  const SmemPlan one = smem_plan(asrc, tn, 1, p.s2, has_ext);
+  const size_t fixed = one.total - one.slot1;
+  // 1 KB to align the dynamic buffer, 1 KB for static shared data, per CTA
+  const size_t budget = (thin ? (kSmemLimit / 2 - 2048) : kSmemLimit) - 2048;
+  p.s1 = static_cast<int>(std::min<size_t>(kMaxS1, (budget - fixed) / one.slot1));
+  p.smem = smem_plan(asrc, tn, p.s1, p.s2, has_ext).total + 1024;
+  // Split the contraction when the output tiles leave CTA slots idle: as many splits
+  // as fit in one wave, at least two steps each.
   const int64_t tiles = p.tiles();
+  const int64_t slots = static_cast<int64_t>(nsm) * p.ctas_per_sm;
   int best = 1;
-  if (tiles < nsm && p.nsteps > 1) {
+  if (tiles < slots && p.nsteps > 1) {
     const int max_splits = std::max(1, p.nsteps / 2);
-    int64_t best_cost = INT64_MAX;
-    for (int sp = 1; sp <= max_splits; ++sp) {
-      const int spc = (p.nsteps + sp - 1) / sp;
-      const int real = (p.nsteps + spc - 1) / spc;
-      if (real != sp) continue;
-      const int64_t waves = (tiles * sp + nsm - 1) / nsm;
-      const int64_t cost = waves * spc * 16 + sp;  // small charge per split for the reduction
-      if (cost < best_cost) {
-        best_cost = cost;
-        best = sp;
-      }
-    }
+    best = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(max_splits, slots / tiles)));
   }
   p.steps_per_split = (p.nsteps + best - 1) / best;
   p.splits = (p.nsteps + p.steps_per_split - 1) / p.steps_per_split;
-  // ring depths from the shared-memory budget
-  p.s2 = src_deq(asrc) ? (tn <= 64 ? 4 : 2) : 0;
-  const SmemPlan one = smem_plan(asrc, tn, 1, p.s2, has_ext);
-  const size_t fixed = one.total - one.slot1;
-  // 1 KB of slack to align the dynamic buffer to 1024 and 1 KB for static shared data
-  const size_t budget = kSmemLimit - 2048;
-  p.s1 = static_cast<int>(std::min<size_t>(kMaxS1, (budget - fixed) / one.slot1));
-  p.smem = smem_plan(asrc, tn, p.s1, p.s2, has_ext).total + 1024;
   return p;
 }
 
@@ -211,6 +205,7 @@ struct LinPlan {
   int64_t ldm = 0, ldn = 0;
   GemmPlan u, v, main, da, db;
   size_t off_up = 0, off_ut = 0, off_vp = 0, off_vt = 0, off_bt = 0, off_part = 0, off_cnt = 0;
+  size_t off_upart = 0, off_ucnt = 0;  // the u kernel's own split-K area (it may overlap the next)
   size_t total = 0;
 };
 
@@ -223,8 +218,6 @@ LinPlan plan_linear(int main_src, int64_t N, int64_t K, int64_t M, int r, bool b
   size_t part = 0;
   int64_t cnt = 1;
   L.u = plan_gemm(A_DENSE_K, M, L.r16, K, L.r16, 0, nsm);
-  part = std::max(part, L.u.part_floats());
-  cnt = std::max(cnt, L.u.tiles());
   if (!bwd) {
     L.main = plan_gemm(main_src, N, M, K, tnm, 1, nsm);
   } else {
@@ -252,8 +245,13 @@ LinPlan plan_linear(int main_src, int64_t N, int64_t K, int64_t M, int r, bool b
     L.off_bt = o;
     o = align256(o + static_cast<size_t>(L.r16) * L.ldn * 2);
   }
+  L.off_upart = o;
+  o = align256(o + L.u.part_floats() * sizeof(float));
   L.off_part = o;
   o = align256(o + part * sizeof(float));
+  // counters last, so one memset clears both areas
+  L.off_ucnt = o;
+  o = align256(o + static_cast<size_t>(L.u.tiles()) * sizeof(unsigned int));
   L.off_cnt = o;
   o = align256(o + static_cast<size_t>(cnt) * sizeof(unsigned int));
   L.total = o;
@@ -283,8 +281,23 @@ qnf4_status launch_gemm(const GemmPlan& p, const CUtensorMap& a, const CUtensorM
   g.s2 = p.s2;
   g.has_ext = p.has_ext;
   g.wait_ns = g_wait_ns;
-  const dim3 grid(p.row_tiles, p.col_tiles, p.splits);
-  k_gemm<ASRC><<<grid, kGemmThreads, p.smem, s>>>(a, b, bx, g);
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(p.row_tiles, p.col_tiles, p.splits);
+  cfg.blockDim = dim3(kGemmThreads, 1, 1);
+  cfg.dynamicSmemBytes = p.smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, k_gemm<ASRC>, a, b, bx, g);
+  if (e != cudaSuccess) {
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    cudaGetLastError();
+    return fail(QNF4_ERR_CUDA, "gemm launch: %s", cudaGetErrorString(e));
+  }
   return launched("gemm");
 }
 
@@ -351,8 +364,11 @@ qnf4_status linear_fwd(const BaseSrc& src, const void* x, int64_t M, const void*
   uint16_t* up = reinterpret_cast<uint16_t*>(w8 + L.off_up);
   float* part = reinterpret_cast<float*>(w8 + L.off_part);
   unsigned* cnt = reinterpret_cast<unsigned*>(w8 + L.off_cnt);
-  if (cudaMemsetAsync(cnt, 0, L.total - L.off_cnt, s) != cudaSuccess) return launched("memset", 0);
-  qnf4_status st = run_u(L, x, A, M, K, r, scale, up, nullptr, part, cnt, s);
+  if (cudaMemsetAsync(w8 + L.off_ucnt, 0, L.total - L.off_ucnt, s) != cudaSuccess)
+    return launched("memset", 0);
+  qnf4_status st = run_u(L, x, A, M, K, r, scale, up, nullptr,
+                         reinterpret_cast<float*>(w8 + L.off_upart),
+                         reinterpret_cast<unsigned*>(w8 + L.off_ucnt), s);
   if (st != QNF4_OK) return st;
   CUtensorMap ma, mb, mbx;
   std::memset(&ma, 0, sizeof(ma));
@@ -389,6 +405,7 @@ qnf4_status linear_fwd(const BaseSrc& src, const void* x, int64_t M, const void*
   g.o_cs = N;
   g.part = part;
   g.counters = cnt;
+  g.lazy_dep = 1;  // only the adapter chunk reads what the u kernel writes
   if (g_ev_start) cudaEventRecord(g_ev_start, s);
   st = launch_any(L.main, ma, mb, mbx, g, s);
   if (g_ev_stop) cudaEventRecord(g_ev_stop, s);
@@ -409,7 +426,8 @@ qnf4_status linear_bwd(const BaseSrc& src, const void* x, const void* dY, int64_
   uint16_t* bt = reinterpret_cast<uint16_t*>(w8 + L.off_bt);
   float* part = reinterpret_cast<float*>(w8 + L.off_part);
   unsigned* cnt = reinterpret_cast<unsigned*>(w8 + L.off_cnt);
-  if (cudaMemsetAsync(cnt, 0, L.total - L.off_cnt, s) != cudaSuccess) return launched("memset", 0);
+  if (cudaMemsetAsync(w8 + L.off_ucnt, 0, L.total - L.off_ucnt, s) != cudaSuccess)
+    return launched("memset", 0);
   // B^T for v = dY B
   {
     const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((N * r + 255) / 256, num_sms() * 4)));
@@ -418,7 +436,9 @@ qnf4_status linear_bwd(const BaseSrc& src, const void* x, const void* dY, int64_
     if (st != QNF4_OK) return st;
   }
   // (scale u)^T for dB
-  qnf4_status st = run_u(L, x, A, M, K, r, scale, nullptr, ut, part, cnt, s);
+  qnf4_status st = run_u(L, x, A, M, K, r, scale, nullptr, ut,
+                         reinterpret_cast<float*>(w8 + L.off_upart),
+                         reinterpret_cast<unsigned*>(w8 + L.off_ucnt), s);
   if (st != QNF4_OK) return st;
   CUtensorMap none;
   std::memset(&none, 0, sizeof(none));

@@ -113,29 +113,32 @@ void build(Nf4Tables& t) {
   }
   t.thr[15] = std::numeric_limits<float>::infinity();
 
-  // Bin shortcut: uniform bins over [-1, 1]; each bin may hold at most one
-  // threshold and every threshold must sit well away from a bin edge, so that a
-  // value's bin and one compare against thr[bin_code] decide its code.
-  t.nbins = 0;
+  // Bin shortcut (see tables.h): the smallest H whose bins each hold at most one
+  // threshold, every threshold at least 2^-16 from a bin edge.
+  t.bin_h = 0;
   const double min_gap = 1.0 / 65536.0;
-  for (int nb = 32; nb <= kMaxBins; nb += 4) {
+  for (int h = 16; h <= kMaxHalfBins; ++h) {
     bool ok = true;
     for (int k = 0; k < 15 && ok; ++k) {
-      const double u = (static_cast<double>(t.thr[k]) + 1.0) * nb * 0.5;  // bin units
-      const double frac = u - std::floor(u);
-      if (frac * 2.0 / nb < min_gap || (1.0 - frac) * 2.0 / nb < min_gap) ok = false;
+      const double u = static_cast<double>(t.thr[k]) * h + h;  // bin units; edges at j + 0.5
+      const double off = u - 0.5 - std::floor(u - 0.5);        // distance above the edge below
+      if (off / h < min_gap || (1.0 - off) / h < min_gap) ok = false;
       if (k < 14) {
-        const double u2 = (static_cast<double>(t.thr[k + 1]) + 1.0) * nb * 0.5;
-        if (std::floor(u2) == std::floor(u)) ok = false;
+        const double u2 = static_cast<double>(t.thr[k + 1]) * h + h;
+        if (std::floor(u2 + 0.5) == std::floor(u + 0.5)) ok = false;  // same bin
       }
     }
     if (!ok) continue;
-    t.nbins = nb;
-    for (int b = 0; b <= nb; ++b) {
-      const double edge = -1.0 + 2.0 * b / nb;
+    t.bin_h = h;
+    for (int b = 0; b <= 2 * h; ++b) {
+      const double lo = (b - 0.5) / h - 1.0;
       int c = 0;
-      for (int k = 0; k < 15; ++k) c += static_cast<double>(t.thr[k]) <= edge ? 1 : 0;
-      t.bin_code[b] = static_cast<uint8_t>(c);
+      for (int k = 0; k < 15; ++k) c += static_cast<double>(t.thr[k]) <= lo ? 1 : 0;
+      const float tk = c < 15 ? t.thr[c] : 2.0f;
+      uint32_t bits;
+      std::memcpy(&bits, &tk, 4);
+      bits = (bits & ~15u) | static_cast<uint32_t>(c);
+      std::memcpy(&t.bin_tc[b], &bits, 4);
     }
     break;
   }

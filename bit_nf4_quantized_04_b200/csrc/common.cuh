@@ -24,6 +24,10 @@ QNF4_DEV uint64_t globaltimer() {
   return t;
 }
 
+// Programmatic dependent launch (PDL) controls.
+QNF4_DEV void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+QNF4_DEV void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 QNF4_DEV uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

@@ -88,6 +88,9 @@ struct GemmArgs {
   float* part;            // split-K partial tiles
   unsigned int* counters; // split-K arrival counters (zero on entry, left zero)
   unsigned long long wait_ns;
+  int lazy_dep;           // programmatic dependent launch: 0 = every thread waits for the
+                          // previous grid after the prologue; 1 = only the adapter chunk's
+                          // copy waits (its operand is the one the previous grid writes)
 };
 
 struct SmemPlan {
@@ -285,6 +288,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s_tmem;
+  // Programmatic dependent launch: the prologue above overlapped the previous grid.
+  // Every kernel of the library waits for its predecessor before it lets its own
+  // dependents start, so a dependent may read anything older than its predecessor.
+  if (!g.lazy_dep) griddep_wait();
+  griddep_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -309,6 +317,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (ASRC == A_NF4_MN) tma_load_2d(slot + sp.off_p1, &tmA, &full1[s], (int32_t)(row0 / 2), kc);
           tma_load_2d(slot + sp.off_b1, &tmB, &full1[s], kc, (int32_t)col0);
         } else {
+          if (g.lazy_dep) griddep_wait();
           mbar_expect_tx(&full1[s], static_cast<uint32_t>(g.tn) * 128u);
           tma_load_2d(slot + sp.off_b1, &tmBx, &full1[s], 0, (int32_t)col0);
         }

@@ -14,8 +14,8 @@ namespace qnf4 {
 struct QuantTab {
   float thr[16];
   float levels[16];
-  int nbins;
-  uint8_t bin_code[kMaxBins + 1];
+  int bin_h;
+  float bin_tc[2 * kMaxHalfBins + 1];
 };
 
 QNF4_DEV uint4 ld_stream_u4(const void* p) {
@@ -26,24 +26,10 @@ QNF4_DEV uint4 ld_stream_u4(const void* p) {
   return v;
 }
 
-// Code of one bf16 value w in a block with absolute maximum c (c > 0), and
-// reciprocal r = RN(1/c). The normalised value is x = RN(w / c) (IEEE division).
-// Fast path: q0 = RN(w * r) is within 3 ulp of x; its uniform bin over [-1, 1]
-// names the one threshold that can fall inside the bin, and one compare against it
-// decides the code. When q0 lies within 2^-20 of that threshold (or the bin table
-// is unavailable, or c is tiny), x is computed exactly and all 15 thresholds are
-// counted.
-QNF4_DEV int nf4_code(float w, float c, float r, float half_nb, int nb, bool exact_only,
-                      const float* s_thr, const uint8_t* s_bin) {
-  if (!exact_only) {
-    const float q0 = w * r;
-    int bi = static_cast<int>(fmaf(q0, half_nb, half_nb));
-    bi = max(0, min(bi, nb));
-    const int cl = s_bin[bi];
-    const float t = s_thr[cl];
-    const float d = q0 - t;
-    if (fabsf(d) > 0x1p-20f) return cl + (d >= 0.f ? 1 : 0);
-  }
+// Exact code of w in a block with absolute maximum c > 0: x = RN(w / c) by IEEE
+// division, code = #{k : x >= thr[k]}. Kept out of line: it runs only for values
+// within 2^-19 of a decision threshold (or for blocks with a tiny absmax).
+__device__ __noinline__ int nf4_code_exact(float w, float c, const float* s_thr) {
   const float x = __fdiv_rn(w, c);
   int code = 0;
 #pragma unroll
@@ -55,6 +41,11 @@ QNF4_DEV int nf4_code(float w, float c, float r, float half_nb, int nb, bool exa
 // elements (one 16-byte load) and writes 4 packed bytes. Optional outputs:
 // WRITE -> packed codes and fp32 absmax; SSE -> per-CTA float64 partial sums of the
 // single-level squared round-trip error (fp32 within a block).
+//
+// Code search (see Nf4Tables): q0 = RN(w * RN(1/c)) is within 3 ulp of the exact
+// quotient x. Its bin k = round(H q0 + H), read off a magic-number float add, gives
+// one table entry t_k | c_k; the code is c_k + (q0 >= t_k) unless |q0 - t_k| <= 2^-19,
+// in which case the exact quotient and all thresholds decide.
 template <bool WRITE, bool SSE>
 __global__ void __launch_bounds__(256) k_nf4_quant(const uint16_t* __restrict__ W,
                                                    int64_t nblocks, uint32_t* __restrict__ packed,
@@ -62,17 +53,18 @@ __global__ void __launch_bounds__(256) k_nf4_quant(const uint16_t* __restrict__ 
                                                    double* __restrict__ sse_part, QuantTab tab) {
   __shared__ float s_thr[16];
   __shared__ float s_lv[16];
-  __shared__ uint8_t s_bin[kMaxBins + 1];
+  __shared__ float s_tc[2 * kMaxHalfBins + 1];
   __shared__ double s_red[8];
   for (int i = threadIdx.x; i < 16; i += blockDim.x) {
     s_thr[i] = tab.thr[i];
     s_lv[i] = tab.levels[i];
   }
-  for (int i = threadIdx.x; i <= kMaxBins; i += blockDim.x) s_bin[i] = tab.bin_code[i];
+  for (int i = threadIdx.x; i <= 2 * kMaxHalfBins; i += blockDim.x) s_tc[i] = tab.bin_tc[i];
   __syncthreads();
 
-  const int nb = tab.nbins;
-  const float half_nb = 0.5f * static_cast<float>(nb);
+  const int H = tab.bin_h;
+  const float hf = static_cast<float>(H);
+  const float magic = hf + 12582912.0f;  // 1.5 * 2^23: the low bits of the sum hold round(H q0 + H)
   const int lane8 = threadIdx.x & 7;
   const int grp = (threadIdx.x >> 3) & 3;  // group within the warp
   // Loop bounds are per warp (4 consecutive blocks per warp-step) so that every
@@ -109,28 +101,43 @@ __global__ void __launch_bounds__(256) k_nf4_quant(const uint16_t* __restrict__ 
       m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
       m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
       const float c = m;
-      uint32_t word = 0;
-      float sse = 0.f;
+      int code[8];
       if (c == 0.f) {
-        word = 0x77777777u;  // code 7 = the exact-zero level
+#pragma unroll
+        for (int j = 0; j < 8; ++j) code[j] = 7;  // the exact-zero level
       } else {
         const float r = __frcp_rn(c);
-        const bool exact_only = (nb == 0) || !(c >= 0x1p-100f);
+        uint32_t amb = (H == 0 || !(c >= 0x1p-100f)) ? 0xFFu : 0u;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          const int code = nf4_code(w[j], c, r, half_nb, nb, exact_only, s_thr, s_bin);
-          word |= static_cast<uint32_t>(code) << ((j & 1) ? 8 * (j >> 1) : 8 * (j >> 1) + 4);
-          if (SSE) {
-            const float e = w[j] - s_lv[code] * c;
-            sse = fmaf(e, e, sse);
-          }
+          const float q0 = w[j] * r;
+          const int k = __float_as_int(fmaf(q0, hf, magic)) - 0x4B400000;
+          const float tk = s_tc[min(max(k, 0), 2 * kMaxHalfBins)];
+          const float d = q0 - tk;
+          code[j] = (__float_as_int(tk) & 15) + (d >= 0.f ? 1 : 0);
+          amb |= (fabsf(d) <= 0x1p-19f ? 1u : 0u) << j;
+        }
+        if (amb) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            if ((amb >> j) & 1u) code[j] = nf4_code_exact(w[j], c, s_thr);
         }
       }
       if (WRITE && valid) {
+        uint32_t word = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          word |= static_cast<uint32_t>((code[2 * j] << 4) | code[2 * j + 1]) << (8 * j);
         packed[b * 8 + lane8] = word;
         if (lane8 == 0) absmax[b] = c;
       }
       if (SSE) {
+        float sse = 0.f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float e = w[j] - s_lv[code[j]] * c;
+          sse = fmaf(e, e, sse);
+        }
         sse += __shfl_xor_sync(0xffffffffu, sse, 1);
         sse += __shfl_xor_sync(0xffffffffu, sse, 2);
         sse += __shfl_xor_sync(0xffffffffu, sse, 4);

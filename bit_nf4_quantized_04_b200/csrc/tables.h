@@ -4,17 +4,25 @@
 
 namespace qnf4 {
 
-constexpr int kMaxBins = 256;
+constexpr int kMaxHalfBins = 128;
 
+// Bin shortcut for the code search. With H = bin_h, a normalised value x in [-1, 1]
+// falls in bin k = round(H x + H) (0 <= k <= 2H), which covers
+// [(k - 0.5)/H - 1, (k + 0.5)/H - 1). H is chosen so that every bin holds at most one
+// decision threshold and every threshold lies at least 2^-16 from a bin edge; then
+// code(x) = c_k + (x >= t_k), where c_k counts the thresholds below the bin and t_k is
+// the next threshold (2.0 past the last). bin_tc[k] stores t_k with c_k written into
+// its 4 lowest mantissa bits (a shift of at most 15 ulp, well inside the kernels'
+// 2^-19 ambiguity window, inside which they fall back to the exact count).
 struct Nf4Tables {
   float levels[16];      // sorted NF4 levels, exact 0 at index 7, -1 / +1 at the ends
   float thr[16];         // 15 decision thresholds, thr[15] = +inf sentinel
-  int nbins;             // uniform bins over [-1, 1] used to shortcut the code search
-  uint8_t bin_code[kMaxBins + 1];  // #{k : thr[k] <= lower edge of bin b}
+  int bin_h;             // H above; 0 if no valid H was found (exact count only)
+  float bin_tc[2 * kMaxHalfBins + 1];
 };
 
-// Builds the tables on first use (thread-safe). Aborts never; a failure to find a
-// valid bin count leaves nbins = 0 and the kernels use the plain threshold count.
+// Builds the tables on first use (thread-safe). Never aborts; a failure to find a
+// valid bin count leaves bin_h = 0 and the kernels use the plain threshold count.
 const Nf4Tables& nf4_tables();
 
 }  // namespace qnf4

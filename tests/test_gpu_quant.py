@@ -56,6 +56,40 @@ def _crafted(N, K, seed):
     return w.to(torch.bfloat16)
 
 
+def _near_threshold_blocks(nblocks, seed):
+    """bf16 blocks whose normalised values w / absmax fall within 2^-19 of an NF4
+    decision threshold (found by search over the bf16 grid), so the kernels' exact
+    fallback runs, mixed with values at the thresholds' bf16 neighbours."""
+    T = onf4.thresholds().astype(np.float64)
+    rng = np.random.default_rng(seed)
+    mant = np.arange(128, dtype=np.uint32)
+    bf = lambda e: ((np.uint32(127 + e) << 23) | (mant << 16)).view(np.float32)  # noqa: E731
+    cands = []
+    for c in bf(-5)[::3]:                      # absmax values in [1/32, 1/16)
+        ws = np.concatenate([bf(e) for e in range(-13, -4)])
+        ws = ws[ws <= c]
+        ws = np.concatenate([ws, -ws])
+        x = (ws / np.float32(c)).astype(np.float32).astype(np.float64)
+        d = np.min(np.abs(x[:, None] - T[None, :]), axis=1)
+        for w in ws[d <= 2.0 ** -19]:
+            cands.append((np.float32(c), np.float32(w)))
+    assert len(cands) > 0
+    out = np.zeros((nblocks, 64), np.float32)
+    for i in range(nblocks):
+        c, w0 = cands[rng.integers(len(cands))]
+        blk = [c] + [cands[rng.integers(len(cands))][1] for _ in range(63)]
+        # keep absmax = c: drop values whose magnitude exceeds it
+        blk = [v if abs(v) <= c else np.float32(0) for v in blk]
+        out[i] = rng.permutation(np.array(blk, np.float32))
+    return torch.from_numpy(out.reshape(-1, 128 if nblocks % 2 == 0 else 64)).to(torch.bfloat16)
+
+
+def test_quantize_near_thresholds(q):
+    W = _near_threshold_blocks(64, 11)
+    assert np.array_equal(f32(W), f32(W).astype(np.float32))
+    _check_quant(q, W)
+
+
 def test_quantize_tiny_layer(q):
     _check_quant(q, synth.tiny_inputs()["W"])
 
