@@ -356,13 +356,25 @@ def breakdown(wl, q, hbm, tc_sus):
             for i, L in enumerate(wl.layers):
                 q.qlora_linear_fwd(ws_[i], xs[i], L["A"], L["B"], wl.s, h=hs[i], ws=wl.ws)
         run()
-        t = time_loop(run, 3 * copies, st)
+        torch.cuda.synchronize()
+        # one decode pass is a few microseconds of GPU work per layer, far below the
+        # host's per-call cost: capture the 7-layer passes over every weight copy in
+        # one CUDA graph and time its replays
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for _ in range(copies):
+                run()
+        graph.replay()
+        torch.cuda.synchronize()
+        t = time_loop(graph.replay, 3, torch.cuda.current_stream()) / copies
         byt = sum(N * K * (0.5 + 1 / 64 + 4 / 16384) + m * K * 2 + RANK * (N + K) * 2 + m * N * 2
                   for N, K in layer_shapes())
         dec[f"M{m}"] = {"GBps": round(byt / t / 1e9, 1), "frac_hbm": round(byt / t / 1e9 / hbm, 3),
                         "us": round(t * 1e6, 1)}
     out["decode_fwd"] = dec
     out["decode_fwd"]["pool_copies"] = copies
+    out["decode_fwd"]["launch"] = "CUDA graph of all copies x 7 layers, PDL edges"
+    q.check()
     return out
 
 

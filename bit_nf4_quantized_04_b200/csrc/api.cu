@@ -144,6 +144,7 @@ struct GemmPlan {
   int64_t rows = 0, cols = 0;
   int nsteps = 0, row_tiles = 0, col_tiles = 0, splits = 1, steps_per_split = 0, s1 = 1, s2 = 0;
   int ctas_per_sm = 1;
+  int nset = 1;  // converter warp sets (4 warps each)
   size_t smem = 0;
   size_t part_floats() const {
     return splits > 1 ? static_cast<size_t>(row_tiles) * col_tiles * splits * tn * 128 : 0;
@@ -176,7 +177,10 @@ GemmPlan plan_gemm(int asrc, int64_t rows, int64_t cols, int64_t contraction, in
   // and a shallower dequant ring; wide tiles take the whole shared memory.
   const bool thin = tn <= 32;
   p.ctas_per_sm = thin ? 2 : 1;
-  p.s2 = src_deq(asrc) ? (thin ? 2 : (tn <= 64 ? 4 : 2)) : 0;
+  p.s2 = src_deq(asrc) ? ((thin && !src_tmem_a(asrc)) ? 2 : 4) : 0;
+  // Wide tiles need two converter sets to keep the tensor core fed; thin tiles run
+  // two CTAs per SM, which leaves registers for one set each.
+  p.nset = (src_deq(asrc) && !thin) ? 2 : 1;
   const SmemPlan one = smem_plan(asrc, tn, 1, p.s2, has_ext);
   const size_t fixed = one.total - one.slot1;
   // 1 KB to align the dynamic buffer, 1 KB for static shared data, per CTA
@@ -258,18 +262,19 @@ LinPlan plan_linear(int main_src, int64_t N, int64_t K, int64_t M, int r, bool b
   return L;
 }
 
-bool g_smem_set[5][64] = {};
+bool g_smem_set[5][2][64] = {};
 
-template <int ASRC>
+template <int ASRC, int NSET>
 qnf4_status launch_gemm(const GemmPlan& p, const CUtensorMap& a, const CUtensorMap& b,
                         const CUtensorMap& bx, GemmArgs g, cudaStream_t s) {
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev < 64 && !g_smem_set[ASRC][dev]) {
-    const cudaError_t e = cudaFuncSetAttribute(k_gemm<ASRC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (dev < 64 && !g_smem_set[ASRC][NSET - 1][dev]) {
+    const cudaError_t e = cudaFuncSetAttribute(k_gemm<ASRC, NSET>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                static_cast<int>(kSmemLimit - 1024));
     if (e != cudaSuccess) return fail(QNF4_ERR_CUDA, "smem attribute: %s", cudaGetErrorString(e));
-    g_smem_set[ASRC][dev] = true;
+    g_smem_set[ASRC][NSET - 1][dev] = true;
   }
   g.rows = p.rows;
   g.cols = p.cols;
@@ -284,7 +289,7 @@ qnf4_status launch_gemm(const GemmPlan& p, const CUtensorMap& a, const CUtensorM
   cudaLaunchConfig_t cfg;
   std::memset(&cfg, 0, sizeof(cfg));
   cfg.gridDim = dim3(p.row_tiles, p.col_tiles, p.splits);
-  cfg.blockDim = dim3(kGemmThreads, 1, 1);
+  cfg.blockDim = dim3(gemm_threads(NSET), 1, 1);
   cfg.dynamicSmemBytes = p.smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -292,7 +297,7 @@ qnf4_status launch_gemm(const GemmPlan& p, const CUtensorMap& a, const CUtensorM
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, k_gemm<ASRC>, a, b, bx, g);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, k_gemm<ASRC, NSET>, a, b, bx, g);
   if (e != cudaSuccess) {
     g_launches.fetch_add(1, std::memory_order_relaxed);
     cudaGetLastError();
@@ -303,12 +308,16 @@ qnf4_status launch_gemm(const GemmPlan& p, const CUtensorMap& a, const CUtensorM
 
 qnf4_status launch_any(const GemmPlan& p, const CUtensorMap& a, const CUtensorMap& b,
                        const CUtensorMap& bx, const GemmArgs& g, cudaStream_t s) {
+  const bool two = p.nset == 2;
   switch (p.asrc) {
-    case A_NF4_K: return launch_gemm<A_NF4_K>(p, a, b, bx, g, s);
-    case A_NF4_MN: return launch_gemm<A_NF4_MN>(p, a, b, bx, g, s);
-    case A_DENSE_K: return launch_gemm<A_DENSE_K>(p, a, b, bx, g, s);
-    case A_DENSE_MN: return launch_gemm<A_DENSE_MN>(p, a, b, bx, g, s);
-    default: return launch_gemm<A_CHANQ_K>(p, a, b, bx, g, s);
+    case A_NF4_K:
+      return two ? launch_gemm<A_NF4_K, 2>(p, a, b, bx, g, s) : launch_gemm<A_NF4_K, 1>(p, a, b, bx, g, s);
+    case A_NF4_MN:
+      return two ? launch_gemm<A_NF4_MN, 2>(p, a, b, bx, g, s) : launch_gemm<A_NF4_MN, 1>(p, a, b, bx, g, s);
+    case A_DENSE_K: return launch_gemm<A_DENSE_K, 1>(p, a, b, bx, g, s);
+    case A_DENSE_MN: return launch_gemm<A_DENSE_MN, 1>(p, a, b, bx, g, s);
+    default:
+      return two ? launch_gemm<A_CHANQ_K, 2>(p, a, b, bx, g, s) : launch_gemm<A_CHANQ_K, 1>(p, a, b, bx, g, s);
   }
 }
 

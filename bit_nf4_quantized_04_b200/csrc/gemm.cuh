@@ -22,11 +22,14 @@
 // TMEM accumulator: the rank-r adapter term of "QLoRA: Efficient Finetuning of
 // Quantized LLMs" (Heng's Blog, opening formula h = dequant(W0) x + (alpha/r) B A x).
 //
-// Roles (192 threads): warp 0 issues TMA, warp 1 allocates TMEM and one lane issues
-// tcgen05.mma, warps 2-5 ("converters") dequantize and then run the epilogue
-// (tcgen05.ld from TMEM, optional split-K reduction in the last-arriving CTA).
-// Every wait is bounded; on timeout the kernel records an error, stops, drains its
-// own copies and MMAs, frees TMEM and returns.
+// Roles (64 + 128 NSET threads): warp 0 issues TMA, warp 1 allocates TMEM and one
+// lane issues tcgen05.mma, and NSET sets of four "converter" warps dequantize (set h
+// takes the steps i with i % NSET == h, one 64-element NF4 block per thread and
+// step) and then run the epilogue (tcgen05.ld from TMEM, optional split-K reduction
+// in the last-arriving CTA). For A_NF4_K the dequantized operand goes straight into
+// tensor memory with tcgen05.st and the MMA reads A from there; the other sources
+// stage A in shared memory. Every wait is bounded; on timeout the kernel records an
+// error, stops, drains its own copies and MMAs, frees TMEM and returns.
 #pragma once
 #include "common.cuh"
 
@@ -37,7 +40,6 @@ enum : int { EPI_BF16 = 0, EPI_F32 = 1, EPI_UV = 2 };
 
 constexpr int kRowsTile = 128;
 constexpr int kStep = 64;
-constexpr int kGemmThreads = 192;
 constexpr uint32_t kATile = 128u * 128u;  // 128 rows x 64 bf16 (or 2 x 64 x 64 MN-major)
 constexpr uint32_t kPTile = 4096u;         // packed NF4 bytes of one step
 constexpr int kMaxS1 = 16;
@@ -50,6 +52,23 @@ __host__ __device__ constexpr bool src_deq(int a) {
 __host__ __device__ constexpr bool src_mn(int a) { return a == A_NF4_MN || a == A_DENSE_MN; }
 __host__ __device__ constexpr bool src_dense(int a) { return a == A_DENSE_K || a == A_DENSE_MN; }
 __host__ __device__ constexpr bool src_packed_tma(int a) { return a == A_NF4_K || a == A_NF4_MN; }
+// A operand staged in tensor memory (written by tcgen05.st) instead of shared memory
+__host__ __device__ constexpr bool src_tmem_a(int a) { return a == A_NF4_K; }
+__host__ __device__ constexpr int gemm_threads(int nset) { return 64 + 128 * nset; }
+
+// TMEM columns: the fp32 accumulator (a power of two >= tn, at least 32), then
+// (for A in tensor memory) s2 stages of 32 columns, one 128 x 64 bf16 A tile each.
+__host__ __device__ inline uint32_t acc_cols(int tn) {
+  uint32_t c = 32;
+  while (c < static_cast<uint32_t>(tn)) c <<= 1;
+  return c;
+}
+__host__ __device__ inline uint32_t tmem_cols(int asrc, int tn, int s2) {
+  uint32_t need = acc_cols(tn) + (src_tmem_a(asrc) ? 32u * static_cast<uint32_t>(s2) : 0u);
+  uint32_t c = 32;
+  while (c < need) c <<= 1;
+  return c;
+}
 
 struct GemmArgs {
   int64_t rows, cols;     // extents of D
@@ -107,7 +126,7 @@ __host__ __device__ inline SmemPlan smem_plan(int asrc, int tn, int s1, int s2, 
   p.off_p1 = o;
   if (src_packed_tma(asrc)) o += kPTile;
   p.slot1 = (o + 1023u) & ~1023u;
-  p.slot2 = src_deq(asrc) ? kATile : 0u;
+  p.slot2 = (src_deq(asrc) && !src_tmem_a(asrc)) ? kATile : 0u;
   p.ring2 = static_cast<uint32_t>(s1) * p.slot1;
   p.ext = p.ring2 + static_cast<uint32_t>(s2) * p.slot2;
   p.cq = p.ext + (has_ext ? kATile : 0u);
@@ -148,23 +167,68 @@ QNF4_DEV void store_row_sw128(uint8_t* tile, int t, const uint32_t (&w)[32]) {
   }
 }
 
-// Dequantize one NF4 block: 32 packed bytes (element 2j in the high nibble of byte j)
-// times the block constant, rounded to bf16.
-QNF4_DEV void nf4_block_to_bf16(const uint8_t* src, float ch, const float* s_lv,
+// Register-resident NF4 lookup. For one block with constant c, the 16 possible
+// dequantized values P[k] = bf16(fp32(levels[k] * c)) are computed once and split
+// into byte planes: l[j] / h[j] hold the low / high bytes of P[4j .. 4j+3]. A
+// byte-permute with a 3-bit selector then reads one plane entry per output byte,
+// a second permute picks the 0-7 or 8-15 half by the code's top bit, and a third
+// interleaves low and high bytes into bf16 pairs. The result equals rounding each
+// fp32 product q[code] * c to bf16, the dequantization the QLoRA page describes.
+struct Nf4Planes {
+  uint32_t l[4], h[4];
+};
+
+QNF4_DEV void nf4_planes(const float (&lv)[16], float c, Nf4Planes& P) {
+  uint32_t p[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) p[i] = pack_bf16x2(lv[2 * i] * c, lv[2 * i + 1] * c);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    P.l[j] = __byte_perm(p[2 * j], p[2 * j + 1], 0x6420);
+    P.h[j] = __byte_perm(p[2 * j], p[2 * j + 1], 0x7531);
+  }
+}
+
+// 8 codes (one packed word: element 2j in the high nibble of byte j) -> 4 bf16 pairs
+// (element 2j in the low half of o[j]).
+QNF4_DEV void nf4_lookup8(uint32_t w, const Nf4Planes& P, uint32_t* o) {
+  const uint32_t sa = w & 0x77777777u;
+  const uint32_t sb = sa >> 16;
+  const uint32_t ta = ((w >> 1) & 0x4444u) | 0x3210u;
+  const uint32_t tb = ((w >> 17) & 0x4444u) | 0x3210u;
+  const uint32_t la = __byte_perm(__byte_perm(P.l[0], P.l[1], sa), __byte_perm(P.l[2], P.l[3], sa), ta);
+  const uint32_t ha = __byte_perm(__byte_perm(P.h[0], P.h[1], sa), __byte_perm(P.h[2], P.h[3], sa), ta);
+  const uint32_t lb = __byte_perm(__byte_perm(P.l[0], P.l[1], sb), __byte_perm(P.l[2], P.l[3], sb), tb);
+  const uint32_t hb = __byte_perm(__byte_perm(P.h[0], P.h[1], sb), __byte_perm(P.h[2], P.h[3], sb), tb);
+  o[0] = __byte_perm(la, ha, 0x4051);
+  o[1] = __byte_perm(la, ha, 0x6273);
+  o[2] = __byte_perm(lb, hb, 0x4051);
+  o[3] = __byte_perm(lb, hb, 0x6273);
+}
+
+// Dequantize one NF4 block: 32 packed bytes at src (shared memory) times constant c.
+QNF4_DEV void nf4_block_to_bf16(const uint8_t* src, float c, const float (&lv)[16],
                                 uint32_t (&o)[32]) {
   const uint4 a = *reinterpret_cast<const uint4*>(src);
   const uint4 b = *reinterpret_cast<const uint4*>(src + 16);
+  Nf4Planes P;
+  nf4_planes(lv, c, P);
   const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const uint32_t byte = (w[i] >> (8 * j)) & 0xFFu;
-      const float f0 = s_lv[byte >> 4] * ch;
-      const float f1 = s_lv[byte & 0xFu] * ch;
-      o[4 * i + j] = pack_bf16x2(f0, f1);
-    }
-  }
+  for (int i = 0; i < 8; ++i) nf4_lookup8(w[i], P, &o[4 * i]);
+}
+
+QNF4_DEV void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+      "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
 }
 
 // One 64-element group of a per-channel row with B-bit codes (MSB first).
@@ -228,12 +292,14 @@ QNF4_DEV void epi_store(const GemmArgs& g, int64_t row, int64_t col0, const floa
 // ---------------------------------------------------------------------------
 // the kernel
 // ---------------------------------------------------------------------------
-template <int ASRC>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+template <int ASRC, int NSET>
+__global__ void __launch_bounds__(gemm_threads(NSET), 1)
     k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
            const __grid_constant__ CUtensorMap tmBx, const GemmArgs g) {
   constexpr bool DEQ = src_deq(ASRC);
   constexpr bool MN = src_mn(ASRC);
+  constexpr bool TMA_A = src_tmem_a(ASRC);
+  constexpr int NCONV = 128 * NSET;  // converter / epilogue threads
   extern __shared__ uint8_t dsmem[];
   __shared__ __align__(8) uint64_t full1[kMaxS1], empty1[kMaxS1], full2[kMaxS2], empty2[kMaxS2];
   __shared__ __align__(8) uint64_t acc_bar, ext_bar, fin_bar;
@@ -255,8 +321,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int nload = nst + (ext ? 1 : 0);
   const int64_t row0 = static_cast<int64_t>(blockIdx.x) * kRowsTile;
   const int64_t col0 = static_cast<int64_t>(blockIdx.y) * g.tn;
-  uint32_t ncols = 32;
-  while (ncols < static_cast<uint32_t>(g.tn)) ncols <<= 1;
+  const uint32_t ncols = tmem_cols(ASRC, g.tn, S2);
+  const uint32_t a_col = acc_cols(g.tn);  // first TMEM column of the A stages
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < S1; ++i) {
@@ -359,10 +425,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const uint32_t aa = smem_u32(a), bb = smem_u32(slot + sp.off_b1);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t ad = MN ? smem_desc(aa + kk * 2048, 8192, 1024, kLayoutSW128)
-                                 : smem_desc(aa + kk * 32, 16, 1024, kLayoutSW128);
           const uint64_t bd = smem_desc(bb + kk * 32, 16, 1024, kLayoutSW128);
-          mma_ss(tmem, ad, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+          const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
+          if (TMA_A) {
+            mma_ts(tmem, tmem + a_col + 32u * s2 + 8u * kk, bd, idesc, acc);
+          } else {
+            const uint64_t ad = MN ? smem_desc(aa + kk * 2048, 8192, 1024, kLayoutSW128)
+                                   : smem_desc(aa + kk * 32, 16, 1024, kLayoutSW128);
+            mma_ss(tmem, ad, bd, idesc, acc);
+          }
         }
         mma_commit(&empty1[s]);
         if (DEQ) mma_commit(&empty2[s2]);
@@ -398,8 +469,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ converters
-    const int t = threadIdx.x - 64;  // row slot 0..127
-    if (ext) {
+    const int ct = threadIdx.x - 64;  // 0 .. NCONV-1
+    const int set = ct >> 7;          // converter set: steps i with i % NSET == set
+    const int t = ct & 127;           // row slot 0..127
+    const int q = warp & 3;           // TMEM lane quarter this warp may access
+    if (ext && set == 0) {
       uint32_t w[32];
       if (!MN) {
         // row slot t = D row (row0 + t): adapter B[row, 0..r), zero padded to 64
@@ -436,33 +510,39 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
 
     if constexpr (ASRC == A_NF4_K || ASRC == A_NF4_MN) {
+      float lv[16];
+#pragma unroll
+      for (int k = 0; k < 16; ++k) lv[k] = s_lv[k];
       const float mu = *g.mean;
+      // In tensor memory the row slot must be the lane this warp may access.
+      const int slot = TMA_A ? (q * 32 + lane) : t;
       // constants of the block this slot dequantizes at step i
       auto blk = [&](int i, int64_t& b) -> bool {
         if (ASRC == A_NF4_K) {
-          const int64_t n = row0 + t;
+          const int64_t n = row0 + slot;
           b = n * g.nbk + (step0 + i);
           return n < g.wN;
         } else {
-          const int kb = t >> 6, nr = t & 63;
+          const int kb = slot >> 6, nr = slot & 63;
           const int64_t n = static_cast<int64_t>(step0 + i) * kStep + nr;
           const int64_t kblk = row0 / 64 + kb;
           b = n * g.nbk + kblk;
           return n < g.wN && kblk < g.nbk;
         }
       };
-      constexpr int PF = 4;  // constants are fetched PF steps ahead
+      constexpr int PF = 2;  // this set's constants are fetched PF of its steps ahead
       uint32_t pc[PF];
       float ps[PF];
       bool pv[PF];
 #pragma unroll
       for (int j = 0; j < PF; ++j) {
         int64_t b = 0;
-        pv[j] = j < nst && blk(j, b);
+        const int ii = set + NSET * j;
+        pv[j] = ii < nst && blk(ii, b);
         pc[j] = pv[j] ? g.code2[b] : 0u;
         ps[j] = pv[j] ? __ldg(g.scale2 + (b >> 8)) : 0.f;
       }
-      for (int i = 0; i < nst; ++i) {
+      for (int i = set; i < nst; i += NSET) {
         const int s = i % S1, s2 = i % S2;
         const bool valid = pv[0];
         const float ch = valid ? fmaf(e4m3_to_f32(static_cast<uint8_t>(pc[0])), ps[0], mu) : 0.f;
@@ -474,7 +554,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         {
           int64_t b = 0;
-          const int ii = i + PF;
+          const int ii = i + NSET * PF;
           pv[PF - 1] = ii < nst && blk(ii, b);
           pc[PF - 1] = pv[PF - 1] ? g.code2[b] : 0u;
           ps[PF - 1] = pv[PF - 1] ? __ldg(g.scale2 + (b >> 8)) : 0.f;
@@ -482,11 +562,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (!wait_or_abort(&full1[s], (i / S1) & 1, g.wait_ns, &s_abort, 31)) break;
         if (!wait_or_abort(&empty2[s2], ((i / S2) & 1) ^ 1, g.wait_ns, &s_abort, 32)) break;
         const uint8_t* pk = base + s * sp.slot1 + sp.off_p1;
-        const uint8_t* src = (ASRC == A_NF4_K) ? pk + t * 32 : pk + (t & 63) * 64 + (t >> 6) * 32;
+        const uint8_t* src =
+            (ASRC == A_NF4_K) ? pk + slot * 32 : pk + (slot & 63) * 64 + (slot >> 6) * 32;
         uint32_t o[32];
-        nf4_block_to_bf16(src, ch, s_lv, o);
-        store_row_sw128(base + sp.ring2 + s2 * sp.slot2, t, o);
-        fence_proxy_async();
+        nf4_block_to_bf16(src, ch, lv, o);
+        if (TMA_A) {
+          tc_fence_after();
+          tmem_st32(tmem + (static_cast<uint32_t>(q * 32) << 16) + a_col + 32u * s2, o);
+          tmem_wait_st();
+          tc_fence_before();
+        } else {
+          store_row_sw128(base + sp.ring2 + s2 * sp.slot2, slot, o);
+          fence_proxy_async();
+        }
         mbar_arrive(&full2[s2]);
       }
     } else if constexpr (ASRC == A_CHANQ_K) {
@@ -495,13 +583,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int bits = 1;
       const uint8_t* prow = nullptr;
       float* tab = reinterpret_cast<float*>(base + sp.cq) + t * kCqStride;
+      if (valid && set == 0) {
+        const int64_t mo = g.cq_map_off[n];
+        for (int c = 0; c < (1 << g.cq_bits[n]); ++c) tab[c] = g.cq_map[mo + c];
+      }
       if (valid) {
         bits = g.cq_bits[n];
         prow = g.cq_packed + g.cq_row_off[n];
-        const int64_t mo = g.cq_map_off[n];
-        for (int c = 0; c < (1 << bits); ++c) tab[c] = g.cq_map[mo + c];
       }
-      for (int i = 0; i < nst; ++i) {
+      if (NSET > 1) named_sync(2, NCONV);  // the tables are shared by both sets
+      for (int i = set; i < nst; i += NSET) {
         const int s = i % S1, s2 = i % S2;
         const int gi = step0 + i;
         if (!wait_or_abort(&full1[s], (i / S1) & 1, g.wait_ns, &s_abort, 33)) break;
@@ -524,22 +615,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
 
     // ------------------------------------------------------------ epilogue
-    // The decision to write is taken once, so all 128 threads take the same path
-    // through the named barriers below.
+    // The decision to write is taken once, so all converter threads take the same
+    // path through the named barriers below.
     wait_or_abort(&acc_bar, 0, g.wait_ns, &s_abort, 41);
-    named_sync(1, 128);
-    if (t == 0) s_last = s_abort ? 0 : 2;
-    named_sync(1, 128);
+    named_sync(1, NCONV);
+    if (ct == 0) s_last = s_abort ? 0 : 2;
+    named_sync(1, NCONV);
     const bool have = s_last == 2;
-    named_sync(1, 128);
+    named_sync(1, NCONV);
     tc_fence_after();
-    const int q = warp & 3;
     const int rl = q * 32 + lane;
     const int64_t row = row0 + rl;
     const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16);
+    // the sets split the tile's columns in 16-column chunks
+    const int nchunk = g.tn / 16;
     if (have) {
       if (g.splits == 1) {
-        for (int c0 = 0; c0 < g.tn; c0 += 16) {
+        for (int ck = set; ck < nchunk; ck += NSET) {
+          const int c0 = ck * 16;
           uint32_t r[16];
           tmem_ld16(taddr + c0, r);
           tmem_wait_ld();
@@ -552,7 +645,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int64_t tile = static_cast<int64_t>(blockIdx.y) * gridDim.x + blockIdx.x;
         const int64_t tsz = static_cast<int64_t>(g.tn) * 128;
         float* mine = g.part + (tile * g.splits + z) * tsz;
-        for (int c0 = 0; c0 < g.tn; c0 += 16) {
+        for (int ck = set; ck < nchunk; ck += NSET) {
+          const int c0 = ck * 16;
           uint32_t r[16];
           tmem_ld16(taddr + c0, r);
           tmem_wait_ld();
@@ -560,16 +654,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           for (int j = 0; j < 16; ++j) __stcg(mine + (c0 + j) * 128 + rl, __uint_as_float(r[j]));
         }
         __threadfence();
-        named_sync(1, 128);
-        if (t == 0) {
+        named_sync(1, NCONV);
+        if (ct == 0) {
           const unsigned int old = atomicAdd(g.counters + tile, 1u);
           s_last = (old == static_cast<unsigned int>(g.splits - 1)) ? 1 : 0;
         }
-        named_sync(1, 128);
+        named_sync(1, NCONV);
         if (s_last) {
           __threadfence();
           const float* all = g.part + tile * g.splits * tsz;
-          for (int c0 = 0; c0 < g.tn; c0 += 16) {
+          for (int ck = set; ck < nchunk; ck += NSET) {
+            const int c0 = ck * 16;
             float v[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) v[j] = 0.f;
@@ -579,7 +674,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
             epi_store(g, row, col0 + c0, v, 16);
           }
-          if (t == 0) g.counters[tile] = 0u;
+          if (ct == 0) g.counters[tile] = 0u;
         }
       }
     }
