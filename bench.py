@@ -543,11 +543,12 @@ def run_case(args):
         fn = lambda: q.qlora_linear_bwd(w, x, dY, A, B, s, ws=ws)  # noqa: E731
     else:  # quant
         fn = lambda: q.nf4_quantize(W, sse=True, ws=ws)  # noqa: E731
-    for _ in range(args.warmup + args.steps):
+    for _ in range(args.warmup):
         fn()
-    torch.cuda.synchronize()
+    t = time_loop(fn, args.steps, torch.cuda.current_stream())
     q.check()
-    print(json.dumps({"case": args.case, "N": N, "K": K, "M": m, "launches": args.warmup + args.steps}))
+    print(json.dumps({"case": args.case, "N": N, "K": K, "M": m, "calls": args.warmup + args.steps,
+                      "us_per_call": round(t * 1e6, 2)}))
 
 
 def run_reference(args):

@@ -79,10 +79,25 @@ QuantTab make_tab() {
 constexpr int kQuantMaxGrid = 1024;
 
 int quant_grid(int64_t nblocks) {
-  const int64_t per_cta = 32;  // 64-element blocks per CTA-step (256 threads, 8 per block)
-  int64_t g = (nblocks + per_cta * 4 - 1) / (per_cta * 4);
-  g = std::max<int64_t>(1, std::min<int64_t>(g, std::min(kQuantMaxGrid, num_sms() * 8)));
-  return static_cast<int>(g);
+  // persistent: two streaming CTAs per SM, never more CTAs than chunks
+  const int64_t chunks = (nblocks + kQChunkBlocks - 1) / kQChunkBlocks;
+  return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(chunks, num_sms() * 2)));
+}
+
+bool g_quant_smem_set[64] = {};
+
+qnf4_status quant_smem_attr() {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !g_quant_smem_set[dev]) {
+    for (auto fn : {k_nf4_quant<true, true>, k_nf4_quant<true, false>, k_nf4_quant<false, true>}) {
+      const cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 static_cast<int>(kQSmem));
+      if (e != cudaSuccess) return fail(QNF4_ERR_CUDA, "smem attribute: %s", cudaGetErrorString(e));
+    }
+    g_quant_smem_set[dev] = true;
+  }
+  return QNF4_OK;
 }
 
 qnf4_status check_weight(const qnf4_weight* w) {
@@ -154,11 +169,28 @@ struct GemmPlan {
 
 constexpr size_t kSmemLimit = 227 * 1024;
 
+// Tiling defaults (converter warp sets per CTA, CTAs per SM for thin N tiles).
+#ifndef QNF4_NSET_WIDE_TMEM
+#define QNF4_NSET_WIDE_TMEM 2
+#endif
+#ifndef QNF4_NSET_WIDE_SMEM
+#define QNF4_NSET_WIDE_SMEM 2
+#endif
+#ifndef QNF4_NSET_THIN
+#define QNF4_NSET_THIN 1
+#endif
+#ifndef QNF4_CTAS_THIN
+#define QNF4_CTAS_THIN 2
+#endif
+
+#ifndef QNF4_TN_MAX
+#define QNF4_TN_MAX 256
+#endif
 int tn_for_tokens(int64_t M) {
   if (M <= 16) return 16;
   if (M <= 32) return 32;
   if (M <= 64) return 64;
-  if (M <= 128) return 128;
+  if (M <= 128 || QNF4_TN_MAX == 128) return 128;
   return 256;
 }
 
@@ -176,16 +208,29 @@ GemmPlan plan_gemm(int asrc, int64_t rows, int64_t cols, int64_t contraction, in
   // Thin N tiles (decode, rank-r GEMMs) are latency bound: give them two CTAs per SM
   // and a shallower dequant ring; wide tiles take the whole shared memory.
   const bool thin = tn <= 32;
-  p.ctas_per_sm = thin ? 2 : 1;
-  p.s2 = src_deq(asrc) ? ((thin && !src_tmem_a(asrc)) ? 2 : 4) : 0;
-  // Wide tiles need two converter sets to keep the tensor core fed; thin tiles run
-  // two CTAs per SM, which leaves registers for one set each.
-  p.nset = (src_deq(asrc) && !thin) ? 2 : 1;
-  const SmemPlan one = smem_plan(asrc, tn, 1, p.s2, has_ext);
-  const size_t fixed = one.total - one.slot1;
+  p.ctas_per_sm = thin ? QNF4_CTAS_THIN : 1;
+  // Wide tiles need several converter sets to keep the tensor core fed; thin tiles
+  // run more CTAs per SM instead.
+  p.nset = src_deq(asrc) ? (thin ? QNF4_NSET_THIN : (src_tmem_a(asrc) ? QNF4_NSET_WIDE_TMEM
+                                                                       : QNF4_NSET_WIDE_SMEM))
+                         : 1;
+  if (asrc == A_CHANQ_K) p.nset = thin ? 1 : 2;
+  if (src_tmem_a(asrc)) {
+    p.s2 = 2 * p.nset;  // TMEM A stages: two per converter set
+    if (p.s2 < 4) p.s2 = 4;
+  } else {
+    p.s2 = src_deq(asrc) ? ((thin ? 2 : 4)) : 0;
+  }
   // 1 KB to align the dynamic buffer, 1 KB for static shared data, per CTA
-  const size_t budget = (thin ? (kSmemLimit / 2 - 2048) : kSmemLimit) - 2048;
-  p.s1 = static_cast<int>(std::min<size_t>(kMaxS1, (budget - fixed) / one.slot1));
+  const size_t budget = (p.ctas_per_sm == 2 ? (kSmemLimit / 2 - 2048) : kSmemLimit) - 2048;
+  for (int pass = 0; pass < 2; ++pass) {
+    const SmemPlan one = smem_plan(asrc, tn, 1, p.s2, has_ext);
+    const size_t fixed = one.total - one.slot1;
+    p.s1 = static_cast<int>(std::min<size_t>(kMaxS1, (budget - fixed) / one.slot1));
+    // the dequantized-A ring may not be deeper than the load ring (its stages are
+    // released through the load ring's barriers)
+    if (p.s2 > p.s1) p.s2 = p.s1;
+  }
   p.smem = smem_plan(asrc, tn, p.s1, p.s2, has_ext).total + 1024;
   // Split the contraction when the output tiles leave CTA slots idle: as many splits
   // as fit in one wave, at least two steps each.
@@ -262,20 +307,23 @@ LinPlan plan_linear(int main_src, int64_t N, int64_t K, int64_t M, int r, bool b
   return L;
 }
 
-bool g_smem_set[5][2][64] = {};
+bool g_smem_set[5][4][3][64] = {};
 
-template <int ASRC, int NSET>
+template <int ASRC, int NSET, int MINB>
 qnf4_status launch_gemm(const GemmPlan& p, const CUtensorMap& a, const CUtensorMap& b,
                         const CUtensorMap& bx, GemmArgs g, cudaStream_t s) {
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev < 64 && !g_smem_set[ASRC][NSET - 1][dev]) {
-    const cudaError_t e = cudaFuncSetAttribute(k_gemm<ASRC, NSET>,
+  if (dev < 64 && !g_smem_set[ASRC][NSET][MINB][dev]) {
+    const cudaError_t e = cudaFuncSetAttribute(k_gemm<ASRC, NSET, MINB>,
                                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                static_cast<int>(kSmemLimit - 1024));
     if (e != cudaSuccess) return fail(QNF4_ERR_CUDA, "smem attribute: %s", cudaGetErrorString(e));
-    g_smem_set[ASRC][NSET - 1][dev] = true;
+    g_smem_set[ASRC][NSET][MINB][dev] = true;
   }
+  if (p.s1 < 1 || p.s1 > kMaxS1 || p.s2 < 0 || p.s2 > kMaxS2 || p.s2 > p.s1 || p.tn < 16 || p.tn > 256 ||
+      p.tn % 16 || tmem_cols(ASRC, p.tn, p.s2) > (p.ctas_per_sm == 2 ? 256u : 512u))
+    return fail(QNF4_ERR_ARG, "internal tiling out of range (s1 %d, s2 %d, tn %d)", p.s1, p.s2, p.tn);
   g.rows = p.rows;
   g.cols = p.cols;
   g.nsteps = p.nsteps;
@@ -297,7 +345,7 @@ qnf4_status launch_gemm(const GemmPlan& p, const CUtensorMap& a, const CUtensorM
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, k_gemm<ASRC, NSET>, a, b, bx, g);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, k_gemm<ASRC, NSET, MINB>, a, b, bx, g);
   if (e != cudaSuccess) {
     g_launches.fetch_add(1, std::memory_order_relaxed);
     cudaGetLastError();
@@ -306,18 +354,33 @@ qnf4_status launch_gemm(const GemmPlan& p, const CUtensorMap& a, const CUtensorM
   return launched("gemm");
 }
 
+// The instantiated (source, converter sets, CTAs per SM) combinations.
+template <int ASRC>
+qnf4_status launch_deq(const GemmPlan& p, const CUtensorMap& a, const CUtensorMap& b,
+                       const CUtensorMap& bx, const GemmArgs& g, cudaStream_t s) {
+  const int key = p.nset * 10 + p.ctas_per_sm;
+  switch (key) {
+    case 11: return launch_gemm<ASRC, 1, 1>(p, a, b, bx, g, s);
+    case 12: return launch_gemm<ASRC, 1, 2>(p, a, b, bx, g, s);
+    case 21: return launch_gemm<ASRC, 2, 1>(p, a, b, bx, g, s);
+    case 22: return launch_gemm<ASRC, 2, 2>(p, a, b, bx, g, s);
+    case 31: return launch_gemm<ASRC, 3, 1>(p, a, b, bx, g, s);
+    default: return fail(QNF4_ERR_ARG, "no kernel for %d converter sets x %d CTAs/SM", p.nset, p.ctas_per_sm);
+  }
+}
+
 qnf4_status launch_any(const GemmPlan& p, const CUtensorMap& a, const CUtensorMap& b,
                        const CUtensorMap& bx, const GemmArgs& g, cudaStream_t s) {
-  const bool two = p.nset == 2;
   switch (p.asrc) {
-    case A_NF4_K:
-      return two ? launch_gemm<A_NF4_K, 2>(p, a, b, bx, g, s) : launch_gemm<A_NF4_K, 1>(p, a, b, bx, g, s);
-    case A_NF4_MN:
-      return two ? launch_gemm<A_NF4_MN, 2>(p, a, b, bx, g, s) : launch_gemm<A_NF4_MN, 1>(p, a, b, bx, g, s);
-    case A_DENSE_K: return launch_gemm<A_DENSE_K, 1>(p, a, b, bx, g, s);
-    case A_DENSE_MN: return launch_gemm<A_DENSE_MN, 1>(p, a, b, bx, g, s);
-    default:
-      return two ? launch_gemm<A_CHANQ_K, 2>(p, a, b, bx, g, s) : launch_gemm<A_CHANQ_K, 1>(p, a, b, bx, g, s);
+    case A_NF4_K: return launch_deq<A_NF4_K>(p, a, b, bx, g, s);
+    case A_NF4_MN: return launch_deq<A_NF4_MN>(p, a, b, bx, g, s);
+    case A_DENSE_K:
+      return p.ctas_per_sm == 2 ? launch_gemm<A_DENSE_K, 1, 2>(p, a, b, bx, g, s)
+                                : launch_gemm<A_DENSE_K, 1, 1>(p, a, b, bx, g, s);
+    case A_DENSE_MN:
+      return p.ctas_per_sm == 2 ? launch_gemm<A_DENSE_MN, 1, 2>(p, a, b, bx, g, s)
+                                : launch_gemm<A_DENSE_MN, 1, 1>(p, a, b, bx, g, s);
+    default: return launch_deq<A_CHANQ_K>(p, a, b, bx, g, s);
   }
 }
 
@@ -571,6 +634,19 @@ const char* qnf4_last_error(void) { return g_last.c_str(); }
 
 unsigned long long qnf4_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
+#ifdef QNF4_WAIT_STATS
+// Tracing builds only (not declared in the public header): copy and clear the
+// per-site wait-cycle counters of the GEMM kernel.
+extern "C" QNF4_API int qnf4_debug_wait_stats(unsigned long long out[64]) {
+  cudaDeviceSynchronize();
+  if (cudaMemcpyFromSymbol(out, g_wait_cycles, 64 * sizeof(unsigned long long)) != cudaSuccess)
+    return 1;
+  static const unsigned long long zero[64] = {};
+  cudaMemcpyToSymbol(g_wait_cycles, zero, sizeof(zero));
+  return 0;
+}
+#endif
+
 qnf4_status qnf4_set_timing_events(void* start, void* stop) {
   if ((start == nullptr) != (stop == nullptr)) return fail(QNF4_ERR_ARG, "give both events or neither");
   g_ev_start = static_cast<cudaEvent_t>(start);
@@ -626,19 +702,20 @@ qnf4_status qnf4_nf4_quantize(const void* W, int64_t N, int64_t K, int32_t block
     if (sse) cudaMemsetAsync(sse, 0, sizeof(double), s);
     return launched("quantize(empty)", 0);
   }
+  qnf4_status st = quant_smem_attr();
+  if (st != QNF4_OK) return st;
   const int grid = quant_grid(nblocks);
   const QuantTab tab = make_tab();
   if (sse) {
-    k_nf4_quant<true, true><<<grid, 256, 0, s>>>(static_cast<const uint16_t*>(W), nblocks,
-                                                 reinterpret_cast<uint32_t*>(packed), absmax,
-                                                 static_cast<double*>(ws), tab);
+    k_nf4_quant<true, true><<<grid, kQThreads, kQSmem, s>>>(
+        static_cast<const uint16_t*>(W), nblocks, reinterpret_cast<uint32_t*>(packed), absmax,
+        static_cast<double*>(ws), tab, g_wait_ns);
     k_sum_partials<<<1, 256, 0, s>>>(static_cast<const double*>(ws), grid, sse);
     return launched("nf4_quantize", 2);
-  } else {
-    k_nf4_quant<true, false><<<grid, 256, 0, s>>>(static_cast<const uint16_t*>(W), nblocks,
-                                                  reinterpret_cast<uint32_t*>(packed), absmax,
-                                                  nullptr, tab);
   }
+  k_nf4_quant<true, false><<<grid, kQThreads, kQSmem, s>>>(
+      static_cast<const uint16_t*>(W), nblocks, reinterpret_cast<uint32_t*>(packed), absmax,
+      nullptr, tab, g_wait_ns);
   return launched("nf4_quantize");
 }
 
@@ -657,9 +734,12 @@ qnf4_status qnf4_nf4_recon_error(const void* W, int64_t N, int64_t K, int32_t bl
     cudaMemsetAsync(sse, 0, sizeof(double), s);
     return launched("recon_error(empty)", 0);
   }
+  qnf4_status st = quant_smem_attr();
+  if (st != QNF4_OK) return st;
   const int grid = quant_grid(nblocks);
-  k_nf4_quant<false, true><<<grid, 256, 0, s>>>(static_cast<const uint16_t*>(W), nblocks, nullptr,
-                                                nullptr, static_cast<double*>(ws), make_tab());
+  k_nf4_quant<false, true><<<grid, kQThreads, kQSmem, s>>>(static_cast<const uint16_t*>(W), nblocks,
+                                                          nullptr, nullptr, static_cast<double*>(ws),
+                                                          make_tab(), g_wait_ns);
   k_sum_partials<<<1, 256, 0, s>>>(static_cast<const double*>(ws), grid, sse);
   return launched("nf4_recon_error", 2);
 }

@@ -43,7 +43,7 @@ constexpr int kStep = 64;
 constexpr uint32_t kATile = 128u * 128u;  // 128 rows x 64 bf16 (or 2 x 64 x 64 MN-major)
 constexpr uint32_t kPTile = 4096u;         // packed NF4 bytes of one step
 constexpr int kMaxS1 = 16;
-constexpr int kMaxS2 = 4;
+constexpr int kMaxS2 = 8;
 constexpr uint32_t kCqStride = 17;  // floats per row of the chanq table (padding vs conflicts)
 
 __host__ __device__ constexpr bool src_deq(int a) {
@@ -53,7 +53,10 @@ __host__ __device__ constexpr bool src_mn(int a) { return a == A_NF4_MN || a == 
 __host__ __device__ constexpr bool src_dense(int a) { return a == A_DENSE_K || a == A_DENSE_MN; }
 __host__ __device__ constexpr bool src_packed_tma(int a) { return a == A_NF4_K || a == A_NF4_MN; }
 // A operand staged in tensor memory (written by tcgen05.st) instead of shared memory
-__host__ __device__ constexpr bool src_tmem_a(int a) { return a == A_NF4_K; }
+#ifndef QNF4_NF4K_TMEM_A
+#define QNF4_NF4K_TMEM_A 1
+#endif
+__host__ __device__ constexpr bool src_tmem_a(int a) { return QNF4_NF4K_TMEM_A && a == A_NF4_K; }
 __host__ __device__ constexpr int gemm_threads(int nset) { return 64 + 128 * nset; }
 
 // TMEM columns: the fp32 accumulator (a power of two >= tn, at least 32), then
@@ -137,9 +140,23 @@ __host__ __device__ inline SmemPlan smem_plan(int asrc, int tn, int s1, int s2, 
 // ---------------------------------------------------------------------------
 // device helpers
 // ---------------------------------------------------------------------------
+#ifdef QNF4_WAIT_STATS
+// Tracing build only: clock cycles spent blocked at each wait site (index = site,
+// 0..63), summed over all threads that wait there. Read with qnf4_debug_wait_stats.
+__device__ unsigned long long g_wait_cycles[64];
+#endif
+
 QNF4_DEV bool wait_or_abort(uint64_t* bar, uint32_t parity, unsigned long long wait_ns,
                             volatile int* abort_flag, unsigned int site) {
   if (mbar_try_wait(bar, parity)) return true;
+#ifdef QNF4_WAIT_STATS
+  const long long c0 = clock64();
+  struct Acc {
+    long long c0;
+    unsigned int site;
+    QNF4_DEV ~Acc() { atomicAdd(&g_wait_cycles[site & 63], static_cast<unsigned long long>(clock64() - c0)); }
+  } acc{c0, site};
+#endif
   const uint64_t t0 = globaltimer();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -292,8 +309,8 @@ QNF4_DEV void epi_store(const GemmArgs& g, int64_t row, int64_t col0, const floa
 // ---------------------------------------------------------------------------
 // the kernel
 // ---------------------------------------------------------------------------
-template <int ASRC, int NSET>
-__global__ void __launch_bounds__(gemm_threads(NSET), 1)
+template <int ASRC, int NSET, int MINB>
+__global__ void __launch_bounds__(gemm_threads(NSET), MINB)
     k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
            const __grid_constant__ CUtensorMap tmBx, const GemmArgs g) {
   constexpr bool DEQ = src_deq(ASRC);
@@ -301,7 +318,7 @@ __global__ void __launch_bounds__(gemm_threads(NSET), 1)
   constexpr bool TMA_A = src_tmem_a(ASRC);
   constexpr int NCONV = 128 * NSET;  // converter / epilogue threads
   extern __shared__ uint8_t dsmem[];
-  __shared__ __align__(8) uint64_t full1[kMaxS1], empty1[kMaxS1], full2[kMaxS2], empty2[kMaxS2];
+  __shared__ __align__(8) uint64_t full1[kMaxS1], empty1[kMaxS1], full2[kMaxS2];
   __shared__ __align__(8) uint64_t acc_bar, ext_bar, fin_bar;
   __shared__ uint32_t s_tmem;
   __shared__ volatile int s_abort;
@@ -322,6 +339,9 @@ __global__ void __launch_bounds__(gemm_threads(NSET), 1)
   const int64_t row0 = static_cast<int64_t>(blockIdx.x) * kRowsTile;
   const int64_t col0 = static_cast<int64_t>(blockIdx.y) * g.tn;
   const uint32_t ncols = tmem_cols(ASRC, g.tn, S2);
+#ifdef QNF4_WAIT_STATS
+  const long long g_t_start = clock64();
+#endif
   const uint32_t a_col = acc_cols(g.tn);  // first TMEM column of the A stages
 
   if (threadIdx.x == 0) {
@@ -329,10 +349,7 @@ __global__ void __launch_bounds__(gemm_threads(NSET), 1)
       mbar_init(&full1[i], 1);
       mbar_init(&empty1[i], 1);
     }
-    for (int i = 0; i < S2; ++i) {
-      mbar_init(&full2[i], 128);
-      mbar_init(&empty2[i], 1);
-    }
+    for (int i = 0; i < S2; ++i) mbar_init(&full2[i], 128);
     mbar_init(&acc_bar, 1);
     mbar_init(&ext_bar, 128);
     mbar_init(&fin_bar, 1);
@@ -364,30 +381,39 @@ __global__ void __launch_bounds__(gemm_threads(NSET), 1)
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       int issued = 0;
+      int s = 0;
+      uint32_t ph = 0;
+      int32_t kc = step0 * kStep;
+      uint32_t bytes = static_cast<uint32_t>(g.tn) * 128u;
+      if (src_dense(ASRC)) bytes += kATile;
+      if (src_packed_tma(ASRC)) bytes += kPTile;
       for (int i = 0; i < nload; ++i) {
-        const int s = i % S1;
-        if (!wait_or_abort(&empty1[s], ((i / S1) & 1) ^ 1, g.wait_ns, &s_abort, 11)) break;
+        if (!mbar_try_wait(&empty1[s], ph ^ 1) &&
+            !wait_or_abort(&empty1[s], ph ^ 1, g.wait_ns, &s_abort, 11))
+          break;
         uint8_t* slot = base + s * sp.slot1;
+        uint64_t* fb = &full1[s];
         if (i < nst) {
-          const int32_t kc = (step0 + i) * kStep;
-          uint32_t bytes = static_cast<uint32_t>(g.tn) * 128u;
-          if (src_dense(ASRC)) bytes += kATile;
-          if (src_packed_tma(ASRC)) bytes += kPTile;
-          mbar_expect_tx(&full1[s], bytes);
-          if (ASRC == A_DENSE_K) tma_load_2d(slot + sp.off_a1, &tmA, &full1[s], kc, (int32_t)row0);
+          mbar_expect_tx(fb, bytes);
+          if (ASRC == A_DENSE_K) tma_load_2d(slot + sp.off_a1, &tmA, fb, kc, (int32_t)row0);
           if (ASRC == A_DENSE_MN) {
-            tma_load_2d(slot + sp.off_a1, &tmA, &full1[s], (int32_t)row0, kc);
-            tma_load_2d(slot + sp.off_a1 + 8192, &tmA, &full1[s], (int32_t)row0 + 64, kc);
+            tma_load_2d(slot + sp.off_a1, &tmA, fb, (int32_t)row0, kc);
+            tma_load_2d(slot + sp.off_a1 + 8192, &tmA, fb, (int32_t)row0 + 64, kc);
           }
-          if (ASRC == A_NF4_K) tma_load_2d(slot + sp.off_p1, &tmA, &full1[s], kc / 2, (int32_t)row0);
-          if (ASRC == A_NF4_MN) tma_load_2d(slot + sp.off_p1, &tmA, &full1[s], (int32_t)(row0 / 2), kc);
-          tma_load_2d(slot + sp.off_b1, &tmB, &full1[s], kc, (int32_t)col0);
+          if (ASRC == A_NF4_K) tma_load_2d(slot + sp.off_p1, &tmA, fb, kc / 2, (int32_t)row0);
+          if (ASRC == A_NF4_MN) tma_load_2d(slot + sp.off_p1, &tmA, fb, (int32_t)(row0 / 2), kc);
+          tma_load_2d(slot + sp.off_b1, &tmB, fb, kc, (int32_t)col0);
         } else {
           if (g.lazy_dep) griddep_wait();
-          mbar_expect_tx(&full1[s], static_cast<uint32_t>(g.tn) * 128u);
-          tma_load_2d(slot + sp.off_b1, &tmBx, &full1[s], 0, (int32_t)col0);
+          mbar_expect_tx(fb, static_cast<uint32_t>(g.tn) * 128u);
+          tma_load_2d(slot + sp.off_b1, &tmBx, fb, 0, (int32_t)col0);
         }
         issued = i + 1;
+        kc += kStep;
+        if (++s == S1) {
+          s = 0;
+          ph ^= 1;
+        }
       }
       // Drain: the last copy issued into each slot must land before the CTA exits.
       // One deadline covers the whole drain.
@@ -407,36 +433,48 @@ __global__ void __launch_bounds__(gemm_threads(NSET), 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    // One thread keeps the tensor core fed: the descriptors are built once and only
+    // offset per stage, stage indices and phases advance incrementally, and a step
+    // costs one barrier test, four MMAs and one commit (the stage's release).
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16(128, static_cast<uint32_t>(g.tn), MN ? 1u : 0u, 0u);
+      const uint64_t bdesc0 = smem_desc(smem_u32(base + sp.off_b1), 16, 1024, kLayoutSW128);
+      const uint32_t a_base = DEQ ? smem_u32(base + sp.ring2) : smem_u32(base + sp.off_a1);
+      const uint64_t adesc0 = MN ? smem_desc(a_base, 8192, 1024, kLayoutSW128)
+                                 : smem_desc(a_base, 16, 1024, kLayoutSW128);
+      const uint32_t b_stride = sp.slot1 >> 4;                 // descriptor units per ring-1 slot
+      const uint32_t a_stride = (DEQ ? sp.slot2 : sp.slot1) >> 4;
+      constexpr uint32_t a_kstep = MN ? (2048u >> 4) : (32u >> 4);  // one K=16 sub-step
+      const uint32_t tmem_a0 = tmem + a_col;
       bool ok = true;
-      for (int i = 0; i < nst && ok; ++i) {
-        const int s = i % S1;
-        if (!wait_or_abort(&full1[s], (i / S1) & 1, g.wait_ns, &s_abort, 21)) { ok = false; break; }
-        uint8_t* slot = base + s * sp.slot1;
-        uint8_t* a = slot + sp.off_a1;
-        int s2 = 0;
-        if (DEQ) {
-          s2 = i % S2;
-          if (!wait_or_abort(&full2[s2], (i / S2) & 1, g.wait_ns, &s_abort, 22)) { ok = false; break; }
-          a = base + sp.ring2 + s2 * sp.slot2;
+      int s = 0, s2 = 0;
+      uint32_t ph = 0, ph2 = 0;
+      for (int i = 0; i < nst; ++i) {
+        uint64_t* bar = DEQ ? &full2[s2] : &full1[s];
+        const uint32_t pp = DEQ ? ph2 : ph;
+        if (!mbar_try_wait(bar, pp) && !wait_or_abort(bar, pp, g.wait_ns, &s_abort, DEQ ? 22 : 21)) {
+          ok = false;
+          break;
         }
         tc_fence_after();
-        const uint32_t aa = smem_u32(a), bb = smem_u32(slot + sp.off_b1);
+        const uint64_t bd = bdesc0 + static_cast<uint64_t>(static_cast<uint32_t>(s) * b_stride);
+        const uint64_t ad = adesc0 + static_cast<uint64_t>(static_cast<uint32_t>(DEQ ? s2 : s) * a_stride);
+        const uint32_t ta = tmem_a0 + 32u * static_cast<uint32_t>(s2);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t bd = smem_desc(bb + kk * 32, 16, 1024, kLayoutSW128);
           const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
-          if (TMA_A) {
-            mma_ts(tmem, tmem + a_col + 32u * s2 + 8u * kk, bd, idesc, acc);
-          } else {
-            const uint64_t ad = MN ? smem_desc(aa + kk * 2048, 8192, 1024, kLayoutSW128)
-                                   : smem_desc(aa + kk * 32, 16, 1024, kLayoutSW128);
-            mma_ss(tmem, ad, bd, idesc, acc);
-          }
+          if (TMA_A) mma_ts(tmem, ta + 8u * kk, bd + 2u * kk, idesc, acc);
+          else mma_ss(tmem, ad + a_kstep * kk, bd + 2u * kk, idesc, acc);
         }
-        mma_commit(&empty1[s]);
-        if (DEQ) mma_commit(&empty2[s2]);
+        mma_commit(&empty1[s]);  // frees ring-1 slot s and, S2 steps later, A stage s2
+        if (++s == S1) {
+          s = 0;
+          ph ^= 1;
+        }
+        if (DEQ && ++s2 == S2) {
+          s2 = 0;
+          ph2 ^= 1;
+        }
       }
       if (ok && ext) {
         const int i = nst;
@@ -560,7 +598,12 @@ __global__ void __launch_bounds__(gemm_threads(NSET), 1)
           ps[PF - 1] = pv[PF - 1] ? __ldg(g.scale2 + (b >> 8)) : 0.f;
         }
         if (!wait_or_abort(&full1[s], (i / S1) & 1, g.wait_ns, &s_abort, 31)) break;
-        if (!wait_or_abort(&empty2[s2], ((i / S2) & 1) ^ 1, g.wait_ns, &s_abort, 32)) break;
+        // A stage s2 was last read by step i - S2; its commit released ring-1 slot
+        // (i - S2) % S1. Waiting for that phase means the stage is free again.
+        if (i >= S2) {
+          const int j = i - S2;
+          if (!wait_or_abort(&empty1[j % S1], (j / S1) & 1, g.wait_ns, &s_abort, 32)) break;
+        }
         const uint8_t* pk = base + s * sp.slot1 + sp.off_p1;
         const uint8_t* src =
             (ASRC == A_NF4_K) ? pk + slot * 32 : pk + (slot & 63) * 64 + (slot >> 6) * 32;
@@ -596,7 +639,10 @@ __global__ void __launch_bounds__(gemm_threads(NSET), 1)
         const int s = i % S1, s2 = i % S2;
         const int gi = step0 + i;
         if (!wait_or_abort(&full1[s], (i / S1) & 1, g.wait_ns, &s_abort, 33)) break;
-        if (!wait_or_abort(&empty2[s2], ((i / S2) & 1) ^ 1, g.wait_ns, &s_abort, 34)) break;
+        if (i >= S2) {
+          const int j = i - S2;
+          if (!wait_or_abort(&empty1[j % S1], (j / S1) & 1, g.wait_ns, &s_abort, 34)) break;
+        }
         uint32_t o[32];
         if (valid) {
           const float gm = __ldg(g.cq_absmax + n * g.nbk + gi);
@@ -681,6 +727,13 @@ __global__ void __launch_bounds__(gemm_threads(NSET), 1)
     tc_fence_before();
   }
 
+#ifdef QNF4_WAIT_STATS
+  if (lane == 0) {
+    // per-warp active time: 60 = producer, 61 = MMA, 62 = converters (sum of warps)
+    const unsigned int slot = warp == 0 ? 60 : (warp == 1 ? 61 : 62);
+    atomicAdd(&g_wait_cycles[slot], static_cast<unsigned long long>(clock64() - g_t_start));
+  }
+#endif
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();

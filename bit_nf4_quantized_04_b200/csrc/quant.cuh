@@ -37,66 +37,113 @@ __device__ __noinline__ int nf4_code_exact(float w, float c, const float* s_thr)
   return code;
 }
 
-// One group of 8 threads per 64-element block; each thread owns 8 consecutive
-// elements (one 16-byte load) and writes 4 packed bytes. Optional outputs:
-// WRITE -> packed codes and fp32 absmax; SSE -> per-CTA float64 partial sums of the
-// single-level squared round-trip error (fp32 within a block).
+QNF4_DEV float rcp_approx(float x) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+
+QNF4_DEV float lds_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+  return v;
+}
+
+constexpr int kQChunkBlocks = 128;  // 64-element blocks per streamed chunk (16 KB of bf16)
+constexpr int kQStages = 4;         // chunks in flight per CTA
+constexpr int kQThreads = 256;
+constexpr uint32_t kQChunkBytes = kQChunkBlocks * 128u;
+constexpr size_t kQSmem = kQStages * kQChunkBytes + 128;
+
+// Blockwise NF4 quantization, streamed: each CTA walks its chunks (chunk c holds
+// blocks [128 c, 128 c + 128)) through a ring of shared-memory stages filled by
+// cp.async.bulk. Inside a chunk, a group of 8 threads takes one 64-element block
+// (each thread 8 consecutive elements, one 16-byte shared load) and writes 4
+// packed bytes. Optional outputs: WRITE -> packed codes and fp32 absmax; SSE ->
+// per-CTA float64 partial sums of the single-level squared round-trip error.
 //
-// Code search (see Nf4Tables): q0 = RN(w * RN(1/c)) is within 3 ulp of the exact
-// quotient x. Its bin k = round(H q0 + H), read off a magic-number float add, gives
-// one table entry t_k | c_k; the code is c_k + (q0 >= t_k) unless |q0 - t_k| <= 2^-19,
-// in which case the exact quotient and all thresholds decide.
+// Code search (see Nf4Tables), for a block with absmax c > 0: the bin
+// k = round(w H/c + H) comes from one fused multiply-add with a magic constant
+// (1.5 * 2^23, whose low mantissa bits then hold k); the table entry t_k carries
+// c_k + 1 in its low mantissa bits; d = fma(-c, t_k, w) = w - c t_k rounded once,
+// so its sign is exactly that of w/c - t_k, and code = c_k + 1 - [d < 0]. Within
+// 2^-18 c of t_k the block falls back to the exact IEEE quotient and the full count.
+// Non-finite weights are outside the method: the table index is masked, so they
+// cannot read outside it, but their codes are unspecified.
 template <bool WRITE, bool SSE>
-__global__ void __launch_bounds__(256) k_nf4_quant(const uint16_t* __restrict__ W,
-                                                   int64_t nblocks, uint32_t* __restrict__ packed,
-                                                   float* __restrict__ absmax,
-                                                   double* __restrict__ sse_part, QuantTab tab) {
+__global__ void __launch_bounds__(kQThreads, 2)
+    k_nf4_quant(const uint16_t* __restrict__ W, int64_t nblocks, uint32_t* __restrict__ packed,
+                float* __restrict__ absmax, double* __restrict__ sse_part, QuantTab tab,
+                unsigned long long wait_ns) {
+  extern __shared__ uint8_t qsm_raw[];
+  __shared__ __align__(8) uint64_t full[kQStages];
   __shared__ float s_thr[16];
   __shared__ float s_lv[16];
   __shared__ float s_tc[2 * kMaxHalfBins + 1];
-  __shared__ double s_red[8];
-  for (int i = threadIdx.x; i < 16; i += blockDim.x) {
+  __shared__ double s_red[kQThreads / 32];
+  uint8_t* qsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(qsm_raw) + 127) &
+                                            ~static_cast<uintptr_t>(127));
+  const int tid = threadIdx.x;
+  for (int i = tid; i < 16; i += kQThreads) {
     s_thr[i] = tab.thr[i];
     s_lv[i] = tab.levels[i];
   }
-  for (int i = threadIdx.x; i <= 2 * kMaxHalfBins; i += blockDim.x) s_tc[i] = tab.bin_tc[i];
+  for (int i = tid; i <= 2 * kMaxHalfBins; i += kQThreads) s_tc[i] = tab.bin_tc[i];
+  const int64_t nchunks = (nblocks + kQChunkBlocks - 1) / kQChunkBlocks;
+  const int64_t my = blockIdx.x < nchunks ? (nchunks - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  if (tid == 0) {
+    for (int i = 0; i < kQStages; ++i) mbar_init(&full[i], 1);
+    fence_mbar_init();
+  }
   __syncthreads();
+  auto issue = [&](int64_t j) {
+    const int64_t c = blockIdx.x + j * gridDim.x;
+    const int64_t nb = min(static_cast<int64_t>(kQChunkBlocks), nblocks - c * kQChunkBlocks);
+    const uint32_t bytes = static_cast<uint32_t>(nb) * 128u;
+    uint64_t* bar = &full[j % kQStages];
+    mbar_expect_tx(bar, bytes);
+    bulk_load(qsm + (j % kQStages) * kQChunkBytes, W + c * kQChunkBlocks * 64, bytes, bar);
+  };
+  int64_t issued = 0;
+  if (tid == 0) {
+    for (; issued < min(static_cast<int64_t>(kQStages), my); ++issued) issue(issued);
+  }
 
   const int H = tab.bin_h;
   const float hf = static_cast<float>(H);
-  const float magic = hf + 12582912.0f;  // 1.5 * 2^23: the low bits of the sum hold round(H q0 + H)
-  const int lane8 = threadIdx.x & 7;
-  const int grp = (threadIdx.x >> 3) & 3;  // group within the warp
-  // Loop bounds are per warp (4 consecutive blocks per warp-step) so that every
-  // lane reaches the shuffles; groups past the end work on zeros and store nothing.
-  const int64_t w0 = ((static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5) * 4;
-  const int64_t gstride = ((static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5) * 4;
+  const float magic = hf + 12582912.0f;
+  const uint32_t tc_base = smem_u32(s_tc);
+  const int lane8 = tid & 7;
+  const int grp = tid >> 3;  // 32 groups of 8 threads
   double acc = 0.0;
+  bool aborted = false;
 
-  constexpr int U = 4;
-  for (int64_t base = w0; base < nblocks; base += U * gstride) {
-    uint4 v[U];
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int64_t b = base + u * gstride + grp;
-      v[u] = make_uint4(0u, 0u, 0u, 0u);
-      if (b < nblocks) v[u] = ld_stream_u4(W + b * 64 + lane8 * 8);
+  for (int64_t j = 0; j < my; ++j) {
+    const int st = static_cast<int>(j % kQStages);
+    const bool ok = mbar_wait(&full[st], static_cast<uint32_t>((j / kQStages) & 1), wait_ns, 51);
+    if (!__syncthreads_and(ok)) {
+      aborted = true;
+      break;
     }
+    const int64_t c0 = (blockIdx.x + j * gridDim.x) * kQChunkBlocks;
+    const int nb = static_cast<int>(min(static_cast<int64_t>(kQChunkBlocks), nblocks - c0));
+    const uint8_t* chunk = qsm + st * kQChunkBytes;
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      if (base + u * gstride >= nblocks) break;  // uniform across the warp
-      const int64_t b = base + u * gstride + grp;
-      const bool valid = b < nblocks;
+    for (int u = 0; u < kQChunkBlocks / 32; ++u) {
+      const int bl = grp + 32 * u;  // block within the chunk
+      const bool valid = bl < nb;   // groups past a partial chunk's end work on zeros
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (valid) v = *reinterpret_cast<const uint4*>(chunk + bl * 128 + lane8 * 16);
       float w[8];
-      const uint32_t words[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+      const uint32_t words[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        w[2 * j] = bf16lo(words[j]);
-        w[2 * j + 1] = bf16hi(words[j]);
+      for (int e = 0; e < 4; ++e) {
+        w[2 * e] = bf16lo(words[e]);
+        w[2 * e + 1] = bf16hi(words[e]);
       }
       float m = 0.f;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(w[j]));
+      for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(w[e]));
       m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
       m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
       m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
@@ -104,55 +151,69 @@ __global__ void __launch_bounds__(256) k_nf4_quant(const uint16_t* __restrict__ 
       int code[8];
       if (c == 0.f) {
 #pragma unroll
-        for (int j = 0; j < 8; ++j) code[j] = 7;  // the exact-zero level
+        for (int e = 0; e < 8; ++e) code[e] = 7;  // the exact-zero level
       } else {
-        const float r = __frcp_rn(c);
-        uint32_t amb = (H == 0 || !(c >= 0x1p-100f)) ? 0xFFu : 0u;
+        const float hr = hf * rcp_approx(c);
+        const float cw = c * 0x1p-18f;
+        bool amb = (H == 0) || !(c >= 0x1p-100f);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const float q0 = w[j] * r;
-          const int k = __float_as_int(fmaf(q0, hf, magic)) - 0x4B400000;
-          const float tk = s_tc[min(max(k, 0), 2 * kMaxHalfBins)];
-          const float d = q0 - tk;
-          code[j] = (__float_as_int(tk) & 15) + (d >= 0.f ? 1 : 0);
-          amb |= (fabsf(d) <= 0x1p-19f ? 1u : 0u) << j;
+        for (int e = 0; e < 8; ++e) {
+          const uint32_t kb = __float_as_uint(fmaf(w[e], hr, magic));
+          const float tk = lds_f32(tc_base + ((kb & 0xFFu) << 2));
+          const float d = fmaf(-c, tk, w[e]);
+          code[e] = (__float_as_int(tk) & 31) + (__float_as_int(d) >> 31);
+          amb = amb || (fabsf(d) <= cw);
         }
         if (amb) {
 #pragma unroll
-          for (int j = 0; j < 8; ++j)
-            if ((amb >> j) & 1u) code[j] = nf4_code_exact(w[j], c, s_thr);
+          for (int e = 0; e < 8; ++e) code[e] = nf4_code_exact(w[e], c, s_thr);
         }
       }
+      const int64_t b = c0 + bl;
       if (WRITE && valid) {
         uint32_t word = 0;
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-          word |= static_cast<uint32_t>((code[2 * j] << 4) | code[2 * j + 1]) << (8 * j);
+        for (int e = 0; e < 4; ++e)
+          word |= static_cast<uint32_t>((code[2 * e] << 4) | code[2 * e + 1]) << (8 * e);
         packed[b * 8 + lane8] = word;
         if (lane8 == 0) absmax[b] = c;
       }
       if (SSE) {
         float sse = 0.f;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const float e = w[j] - s_lv[code[j]] * c;
-          sse = fmaf(e, e, sse);
+        for (int e = 0; e < 8; ++e) {
+          const float r = fmaf(-c, s_lv[code[e]], w[e]);
+          sse = fmaf(r, r, sse);
         }
         sse += __shfl_xor_sync(0xffffffffu, sse, 1);
         sse += __shfl_xor_sync(0xffffffffu, sse, 2);
         sse += __shfl_xor_sync(0xffffffffu, sse, 4);
-        if (lane8 == 0) acc += static_cast<double>(sse);
+        if (lane8 == 0 && valid) acc += static_cast<double>(sse);
+      }
+    }
+    __syncthreads();  // every thread is done with this stage
+    if (tid == 0 && issued < my) issue(issued++);
+  }
+  if (aborted && tid == 0) {
+    // Drain: copies issued but not yet consumed must land before the CTA exits.
+    const uint64_t t0 = globaltimer();
+    for (int64_t jj = max(static_cast<int64_t>(0), issued - kQStages); jj < issued; ++jj) {
+      while (!mbar_try_wait(&full[jj % kQStages], static_cast<uint32_t>((jj / kQStages) & 1))) {
+        if (globaltimer() - t0 > wait_ns) {
+          set_err(52);
+          break;
+        }
       }
     }
   }
   if (SSE) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = acc;
+    if ((tid & 31) == 0) s_red[tid >> 5] = acc;
     __syncthreads();
-    if (threadIdx.x == 0) {
+    if (tid == 0) {
       double t = 0.0;
-      for (int i = 0; i < static_cast<int>(blockDim.x >> 5); ++i) t += s_red[i];
+      for (int i = 0; i < kQThreads / 32; ++i) t += s_red[i];
       sse_part[blockIdx.x] = t;
     }
   }
