@@ -171,10 +171,13 @@ constexpr size_t kSmemLimit = 227 * 1024;
 
 // Tiling defaults (converter warp sets per CTA, CTAs per SM for thin N tiles).
 #ifndef QNF4_NSET_WIDE_TMEM
-#define QNF4_NSET_WIDE_TMEM 2
+#define QNF4_NSET_WIDE_TMEM 3
 #endif
 #ifndef QNF4_NSET_WIDE_SMEM
-#define QNF4_NSET_WIDE_SMEM 2
+#define QNF4_NSET_WIDE_SMEM 3
+#endif
+#ifndef QNF4_S2_THIN_TMEM
+#define QNF4_S2_THIN_TMEM 7
 #endif
 #ifndef QNF4_NSET_THIN
 #define QNF4_NSET_THIN 1
@@ -216,8 +219,12 @@ GemmPlan plan_gemm(int asrc, int64_t rows, int64_t cols, int64_t contraction, in
                          : 1;
   if (asrc == A_CHANQ_K) p.nset = thin ? 1 : 2;
   if (src_tmem_a(asrc)) {
-    p.s2 = 2 * p.nset;  // TMEM A stages: two per converter set
-    if (p.s2 < 4) p.s2 = 4;
+    // TMEM A stages. Each is reusable only after the MMA that read it has completed,
+    // so the ring depth bounds the steps in flight per MMA round trip: as deep as the
+    // accumulator leaves room for (256 columns per CTA at two CTAs per SM, 512 at one).
+    const int room = static_cast<int>(((p.ctas_per_sm == 2 ? 256u : 512u) - acc_cols(tn)) / 32u);
+    p.s2 = std::min(room, thin ? QNF4_S2_THIN_TMEM : 8);
+    if (p.s2 > kMaxS2) p.s2 = kMaxS2;
   } else {
     p.s2 = src_deq(asrc) ? ((thin ? 2 : 4)) : 0;
   }

@@ -306,6 +306,39 @@ QNF4_DEV void epi_store(const GemmArgs& g, int64_t row, int64_t col0, const floa
   }
 }
 
+// Where a converter set's step i sits in the two rings, advanced without division
+// (NSET < S2 <= S1, so an index wraps at most once per advance): s / ph = load-ring
+// slot and phase of step i, s2 = its A stage, sj / phj = load-ring slot and phase of
+// step i - S2, the last reader of that A stage (valid once i >= S2).
+struct ConvCursor {
+  int i, s, s2, sj;
+  uint32_t ph, phj;
+  QNF4_DEV explicit ConvCursor(int set) : i(set), s(set), s2(set), sj(0), ph(0), phj(0) {}
+  QNF4_DEV void next(int nset, int S1, int S2) {
+    i += nset;
+    s += nset;
+    if (s >= S1) {
+      s -= S1;
+      ph ^= 1u;
+    }
+    s2 += nset;
+    if (s2 >= S2) s2 -= S2;
+    const int j = i - S2;
+    if (j >= 0) {
+      if (j < nset) {  // first step with a predecessor: j < nset < S1
+        sj = j;
+        phj = 0;
+      } else {
+        sj += nset;
+        if (sj >= S1) {
+          sj -= S1;
+          phj ^= 1u;
+        }
+      }
+    }
+  }
+};
+
 // ---------------------------------------------------------------------------
 // the kernel
 // ---------------------------------------------------------------------------
@@ -554,56 +587,44 @@ __global__ void __launch_bounds__(gemm_threads(NSET), MINB)
       const float mu = *g.mean;
       // In tensor memory the row slot must be the lane this warp may access.
       const int slot = TMA_A ? (q * 32 + lane) : t;
-      // constants of the block this slot dequantizes at step i
-      auto blk = [&](int i, int64_t& b) -> bool {
-        if (ASRC == A_NF4_K) {
-          const int64_t n = row0 + slot;
-          b = n * g.nbk + (step0 + i);
-          return n < g.wN;
-        } else {
-          const int kb = slot >> 6, nr = slot & 63;
-          const int64_t n = static_cast<int64_t>(step0 + i) * kStep + nr;
-          const int64_t kblk = row0 / 64 + kb;
-          b = n * g.nbk + kblk;
-          return n < g.wN && kblk < g.nbk;
-        }
-      };
-      constexpr int PF = 2;  // this set's constants are fetched PF of its steps ahead
-      uint32_t pc[PF];
-      float ps[PF];
-      bool pv[PF];
-#pragma unroll
-      for (int j = 0; j < PF; ++j) {
-        int64_t b = 0;
-        const int ii = set + NSET * j;
-        pv[j] = ii < nst && blk(ii, b);
-        pc[j] = pv[j] ? g.code2[b] : 0u;
-        ps[j] = pv[j] ? __ldg(g.scale2 + (b >> 8)) : 0.f;
+      ConvCursor cur(set);
+      // block index of this slot at step i and its per-step increment
+      int64_t bidx;
+      int64_t bstep;
+      bool rowok;
+      if (ASRC == A_NF4_K) {
+        const int64_t n = row0 + slot;
+        rowok = n < g.wN;
+        bidx = n * g.nbk + step0 + set;
+        bstep = NSET;
+      } else {
+        const int kb = slot >> 6, nr = slot & 63;
+        const int64_t kblk = row0 / 64 + kb;
+        rowok = kblk < g.nbk;
+        bidx = (static_cast<int64_t>(step0 + set) * kStep + nr) * g.nbk + kblk;
+        bstep = static_cast<int64_t>(NSET) * kStep * g.nbk;
       }
-      for (int i = set; i < nst; i += NSET) {
-        const int s = i % S1, s2 = i % S2;
-        const bool valid = pv[0];
-        const float ch = valid ? fmaf(e4m3_to_f32(static_cast<uint8_t>(pc[0])), ps[0], mu) : 0.f;
-#pragma unroll
-        for (int j = 0; j < PF - 1; ++j) {
-          pc[j] = pc[j + 1];
-          ps[j] = ps[j + 1];
-          pv[j] = pv[j + 1];
+      const int64_t nb1 = g.wN * g.nbk;
+      // constants of this set's next step, fetched one of its steps ahead
+      int64_t bnext = bidx;
+      bool vnext = rowok && set < nst && bnext < nb1;
+      uint32_t cnext = vnext ? g.code2[bnext] : 0u;
+      float snext = vnext ? __ldg(g.scale2 + (bnext >> 8)) : 0.f;
+      for (; cur.i < nst; cur.next(NSET, S1, S2)) {
+        const int i = cur.i;
+        const int s = cur.s, s2 = cur.s2;
+        const bool valid = vnext;
+        const float ch = valid ? fmaf(e4m3_to_f32(static_cast<uint8_t>(cnext)), snext, mu) : 0.f;
+        bnext += bstep;
+        vnext = rowok && (i + NSET) < nst && bnext < nb1;
+        if (vnext) {
+          cnext = g.code2[bnext];
+          snext = __ldg(g.scale2 + (bnext >> 8));
         }
-        {
-          int64_t b = 0;
-          const int ii = i + NSET * PF;
-          pv[PF - 1] = ii < nst && blk(ii, b);
-          pc[PF - 1] = pv[PF - 1] ? g.code2[b] : 0u;
-          ps[PF - 1] = pv[PF - 1] ? __ldg(g.scale2 + (b >> 8)) : 0.f;
-        }
-        if (!wait_or_abort(&full1[s], (i / S1) & 1, g.wait_ns, &s_abort, 31)) break;
-        // A stage s2 was last read by step i - S2; its commit released ring-1 slot
-        // (i - S2) % S1. Waiting for that phase means the stage is free again.
-        if (i >= S2) {
-          const int j = i - S2;
-          if (!wait_or_abort(&empty1[j % S1], (j / S1) & 1, g.wait_ns, &s_abort, 32)) break;
-        }
+        if (!wait_or_abort(&full1[s], cur.ph, g.wait_ns, &s_abort, 31)) break;
+        // A stage s2 was last read by step i - S2; its commit released load-ring slot
+        // cur.sj in phase cur.phj. Waiting for that phase means the stage is free again.
+        if (i >= S2 && !wait_or_abort(&empty1[cur.sj], cur.phj, g.wait_ns, &s_abort, 32)) break;
         const uint8_t* pk = base + s * sp.slot1 + sp.off_p1;
         const uint8_t* src =
             (ASRC == A_NF4_K) ? pk + slot * 32 : pk + (slot & 63) * 64 + (slot >> 6) * 32;
@@ -635,14 +656,12 @@ __global__ void __launch_bounds__(gemm_threads(NSET), MINB)
         prow = g.cq_packed + g.cq_row_off[n];
       }
       if (NSET > 1) named_sync(2, NCONV);  // the tables are shared by both sets
-      for (int i = set; i < nst; i += NSET) {
-        const int s = i % S1, s2 = i % S2;
+      for (ConvCursor cur(set); cur.i < nst; cur.next(NSET, S1, S2)) {
+        const int i = cur.i;
+        const int s2 = cur.s2;
         const int gi = step0 + i;
-        if (!wait_or_abort(&full1[s], (i / S1) & 1, g.wait_ns, &s_abort, 33)) break;
-        if (i >= S2) {
-          const int j = i - S2;
-          if (!wait_or_abort(&empty1[j % S1], (j / S1) & 1, g.wait_ns, &s_abort, 34)) break;
-        }
+        if (!wait_or_abort(&full1[cur.s], cur.ph, g.wait_ns, &s_abort, 33)) break;
+        if (i >= S2 && !wait_or_abort(&empty1[cur.sj], cur.phj, g.wait_ns, &s_abort, 34)) break;
         uint32_t o[32];
         if (valid) {
           const float gm = __ldg(g.cq_absmax + n * g.nbk + gi);
