@@ -502,8 +502,9 @@ def run_ours(args):
             "roofline": {"bound": "tensor", "kernel": kname, "achieved": round(achieved, 1),
                          "peak": tc_sus, "unit": "TFLOP/s", "frac": round(achieved / tc_sus, 3),
                          "peak_kind": f"{peak_kind} bf16 sustained",
-                         "traffic": tr * (kfl / K / sum(2.0 * M_TOK * N * K for N, K in shapes))
-                         if tr else None},
+                         # dram bytes per algorithmic FLOP (ncu, gate-shaped launch) x the
+                         # average FLOPs of one of this kernel's launches in the step
+                         "traffic": round(tr * kfl / (K * len(shapes))) if tr else None},
             "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": int(n1 - n0),
