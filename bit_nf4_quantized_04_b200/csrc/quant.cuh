@@ -51,39 +51,63 @@ QNF4_DEV float lds_f32(uint32_t addr) {
 
 constexpr int kQChunkBlocks = 128;  // 64-element blocks per streamed chunk (16 KB of bf16)
 constexpr int kQStages = 4;         // chunks in flight per CTA
-constexpr int kQThreads = 256;
+constexpr int kQWorkers = 8;        // worker warps; one more warp issues the copies
+constexpr int kQThreads = 32 * (kQWorkers + 1);
 constexpr uint32_t kQChunkBytes = kQChunkBlocks * 128u;
 constexpr size_t kQSmem = kQStages * kQChunkBytes + 128;
 
+// Spin on a phase with a bound, in every lane of a warp, then agree: the result is
+// the same in all lanes (all observed the phase, or the warp gives up together).
+QNF4_DEV bool warp_wait(uint64_t* bar, uint32_t parity, unsigned long long wait_ns,
+                        volatile int* abort_flag, unsigned int site) {
+  bool ok = mbar_try_wait(bar, parity);
+  if (!ok) {
+    const uint64_t t0 = globaltimer();
+    while (!(ok = mbar_try_wait(bar, parity))) {
+      if (*abort_flag) break;
+      if (globaltimer() - t0 > wait_ns) {
+        set_err(site);
+        *abort_flag = 1;
+        break;
+      }
+    }
+  }
+  return __all_sync(0xffffffffu, ok);
+}
+
 // Blockwise NF4 quantization, streamed: each CTA walks its chunks (chunk c holds
-// blocks [128 c, 128 c + 128)) through a ring of shared-memory stages filled by
-// cp.async.bulk. Inside a chunk, a group of 8 threads takes one 64-element block
-// (each thread 8 consecutive elements, one 16-byte shared load) and writes 4
-// packed bytes. Optional outputs: WRITE -> packed codes and fp32 absmax; SSE ->
-// per-CTA float64 partial sums of the single-level squared round-trip error.
+// blocks [128 c, 128 c + 128)) through a ring of shared-memory stages. One warp
+// fills the ring with cp.async.bulk; eight worker warps consume it, each releasing a
+// stage with one arrival when done, so no warp waits for the others. Inside a
+// chunk, a group of 8 threads takes one 64-element block (each thread 8 consecutive
+// elements, one 16-byte shared load) and writes 4 packed bytes. Optional outputs:
+// WRITE -> packed codes and fp32 absmax; SSE -> per-CTA float64 partial sums of the
+// single-level squared round-trip error.
 //
 // Code search (see Nf4Tables), for a block with absmax c > 0: the bin
 // k = round(w H/c + H) comes from one fused multiply-add with a magic constant
 // (1.5 * 2^23, whose low mantissa bits then hold k); the table entry t_k carries
 // c_k + 1 in its low mantissa bits; d = fma(-c, t_k, w) = w - c t_k rounded once,
-// so its sign is exactly that of w/c - t_k, and code = c_k + 1 - [d < 0]. Within
-// 2^-18 c of t_k the block falls back to the exact IEEE quotient and the full count.
-// Non-finite weights are outside the method: the table index is masked, so they
-// cannot read outside it, but their codes are unspecified.
+// so its sign is exactly that of w/c - t_k, and code = c_k + 1 - [d < 0]. If any of a
+// thread's 8 values lies within 2^-18 c of its t_k, those 8 take the exact IEEE
+// quotient and the full count. Non-finite weights are outside the method: the table
+// index is masked, so they cannot read outside it, but their codes are unspecified.
 template <bool WRITE, bool SSE>
 __global__ void __launch_bounds__(kQThreads, 2)
     k_nf4_quant(const uint16_t* __restrict__ W, int64_t nblocks, uint32_t* __restrict__ packed,
                 float* __restrict__ absmax, double* __restrict__ sse_part, QuantTab tab,
                 unsigned long long wait_ns) {
   extern __shared__ uint8_t qsm_raw[];
-  __shared__ __align__(8) uint64_t full[kQStages];
+  __shared__ __align__(8) uint64_t full[kQStages], empty[kQStages];
   __shared__ float s_thr[16];
   __shared__ float s_lv[16];
   __shared__ float s_tc[2 * kMaxHalfBins + 1];
-  __shared__ double s_red[kQThreads / 32];
+  __shared__ double s_red[kQWorkers];
+  __shared__ volatile int s_abort;
   uint8_t* qsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(qsm_raw) + 127) &
                                             ~static_cast<uintptr_t>(127));
   const int tid = threadIdx.x;
+  const int warp = tid >> 5;
   for (int i = tid; i < 16; i += kQThreads) {
     s_thr[i] = tab.thr[i];
     s_lv[i] = tab.levels[i];
@@ -92,130 +116,154 @@ __global__ void __launch_bounds__(kQThreads, 2)
   const int64_t nchunks = (nblocks + kQChunkBlocks - 1) / kQChunkBlocks;
   const int64_t my = blockIdx.x < nchunks ? (nchunks - 1 - blockIdx.x) / gridDim.x + 1 : 0;
   if (tid == 0) {
-    for (int i = 0; i < kQStages; ++i) mbar_init(&full[i], 1);
+    for (int i = 0; i < kQStages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], kQWorkers);
+    }
+    s_abort = 0;
     fence_mbar_init();
   }
   __syncthreads();
-  auto issue = [&](int64_t j) {
-    const int64_t c = blockIdx.x + j * gridDim.x;
-    const int64_t nb = min(static_cast<int64_t>(kQChunkBlocks), nblocks - c * kQChunkBlocks);
-    const uint32_t bytes = static_cast<uint32_t>(nb) * 128u;
-    uint64_t* bar = &full[j % kQStages];
-    mbar_expect_tx(bar, bytes);
-    bulk_load(qsm + (j % kQStages) * kQChunkBytes, W + c * kQChunkBlocks * 64, bytes, bar);
-  };
-  int64_t issued = 0;
-  if (tid == 0) {
-    for (; issued < min(static_cast<int64_t>(kQStages), my); ++issued) issue(issued);
-  }
 
-  const int H = tab.bin_h;
-  const float hf = static_cast<float>(H);
-  const float magic = hf + 12582912.0f;
-  const uint32_t tc_base = smem_u32(s_tc);
-  const int lane8 = tid & 7;
-  const int grp = tid >> 3;  // 32 groups of 8 threads
   double acc = 0.0;
-  bool aborted = false;
-
-  for (int64_t j = 0; j < my; ++j) {
-    const int st = static_cast<int>(j % kQStages);
-    const bool ok = mbar_wait(&full[st], static_cast<uint32_t>((j / kQStages) & 1), wait_ns, 51);
-    if (!__syncthreads_and(ok)) {
-      aborted = true;
-      break;
-    }
-    const int64_t c0 = (blockIdx.x + j * gridDim.x) * kQChunkBlocks;
-    const int nb = static_cast<int>(min(static_cast<int64_t>(kQChunkBlocks), nblocks - c0));
-    const uint8_t* chunk = qsm + st * kQChunkBytes;
-#pragma unroll
-    for (int u = 0; u < kQChunkBlocks / 32; ++u) {
-      const int bl = grp + 32 * u;  // block within the chunk
-      const bool valid = bl < nb;   // groups past a partial chunk's end work on zeros
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (valid) v = *reinterpret_cast<const uint4*>(chunk + bl * 128 + lane8 * 16);
-      float w[8];
-      const uint32_t words[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        w[2 * e] = bf16lo(words[e]);
-        w[2 * e + 1] = bf16hi(words[e]);
-      }
-      float m = 0.f;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(w[e]));
-      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
-      const float c = m;
-      int code[8];
-      if (c == 0.f) {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) code[e] = 7;  // the exact-zero level
-      } else {
-        const float hr = hf * rcp_approx(c);
-        const float cw = c * 0x1p-18f;
-        bool amb = (H == 0) || !(c >= 0x1p-100f);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const uint32_t kb = __float_as_uint(fmaf(w[e], hr, magic));
-          const float tk = lds_f32(tc_base + ((kb & 0xFFu) << 2));
-          const float d = fmaf(-c, tk, w[e]);
-          code[e] = (__float_as_int(tk) & 31) + (__float_as_int(d) >> 31);
-          amb = amb || (fabsf(d) <= cw);
+  if (warp == kQWorkers) {
+    // ---------------------------------------------------------------- producer
+    if ((tid & 31) == 0) {
+      int st = 0;
+      uint32_t ph = 0;
+      int64_t issued = 0;
+      for (int64_t j = 0; j < my; ++j) {
+        if (!mbar_try_wait(&empty[st], ph ^ 1u)) {
+          const uint64_t t0 = globaltimer();
+          bool ok = false;
+          while (!(ok = mbar_try_wait(&empty[st], ph ^ 1u))) {
+            if (s_abort) break;
+            if (globaltimer() - t0 > wait_ns) {
+              set_err(53);
+              s_abort = 1;
+              break;
+            }
+          }
+          if (!ok) break;
         }
-        if (amb) {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) code[e] = nf4_code_exact(w[e], c, s_thr);
+        const int64_t c = blockIdx.x + j * gridDim.x;
+        const int64_t nb = min(static_cast<int64_t>(kQChunkBlocks), nblocks - c * kQChunkBlocks);
+        const uint32_t bytes = static_cast<uint32_t>(nb) * 128u;
+        mbar_expect_tx(&full[st], bytes);
+        bulk_load(qsm + st * kQChunkBytes, W + c * kQChunkBlocks * 64, bytes, &full[st]);
+        issued = j + 1;
+        if (++st == kQStages) {
+          st = 0;
+          ph ^= 1u;
         }
       }
-      const int64_t b = c0 + bl;
-      if (WRITE && valid) {
-        uint32_t word = 0;
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-          word |= static_cast<uint32_t>((code[2 * e] << 4) | code[2 * e + 1]) << (8 * e);
-        packed[b * 8 + lane8] = word;
-        if (lane8 == 0) absmax[b] = c;
-      }
-      if (SSE) {
-        float sse = 0.f;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float r = fmaf(-c, s_lv[code[e]], w[e]);
-          sse = fmaf(r, r, sse);
+      // Drain: every copy issued must land before the CTA exits (one deadline).
+      const uint64_t t0 = globaltimer();
+      for (int64_t jj = max(static_cast<int64_t>(0), issued - kQStages); jj < issued; ++jj) {
+        while (!mbar_try_wait(&full[jj % kQStages], static_cast<uint32_t>((jj / kQStages) & 1))) {
+          if (globaltimer() - t0 > wait_ns) {
+            set_err(52);
+            break;
+          }
         }
-        sse += __shfl_xor_sync(0xffffffffu, sse, 1);
-        sse += __shfl_xor_sync(0xffffffffu, sse, 2);
-        sse += __shfl_xor_sync(0xffffffffu, sse, 4);
-        if (lane8 == 0 && valid) acc += static_cast<double>(sse);
       }
     }
-    __syncthreads();  // every thread is done with this stage
-    if (tid == 0 && issued < my) issue(issued++);
-  }
-  if (aborted && tid == 0) {
-    // Drain: copies issued but not yet consumed must land before the CTA exits.
-    const uint64_t t0 = globaltimer();
-    for (int64_t jj = max(static_cast<int64_t>(0), issued - kQStages); jj < issued; ++jj) {
-      while (!mbar_try_wait(&full[jj % kQStages], static_cast<uint32_t>((jj / kQStages) & 1))) {
-        if (globaltimer() - t0 > wait_ns) {
-          set_err(52);
-          break;
+  } else {
+    // ---------------------------------------------------------------- workers
+    const int H = tab.bin_h;
+    const float hf = static_cast<float>(H);
+    const float magic = hf + 12582912.0f;
+    const uint32_t tc_base = smem_u32(s_tc);
+    const uint32_t lv_base = smem_u32(s_lv);
+    const int lane8 = tid & 7;
+    const int grp = tid >> 3;  // 32 groups of 8 threads
+    int st = 0;
+    uint32_t ph = 0;
+    for (int64_t j = 0; j < my; ++j) {
+      if (!warp_wait(&full[st], ph, wait_ns, &s_abort, 51)) break;
+      const int64_t c0 = (blockIdx.x + j * gridDim.x) * kQChunkBlocks;
+      const int nb = static_cast<int>(min(static_cast<int64_t>(kQChunkBlocks), nblocks - c0));
+      const uint8_t* chunk = qsm + st * kQChunkBytes;
+#pragma unroll
+      for (int u = 0; u < kQChunkBlocks / 32; ++u) {
+        const int bl = grp + 32 * u;  // block within the chunk
+        const bool valid = bl < nb;   // groups past a partial chunk's end work on zeros
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (valid) v = *reinterpret_cast<const uint4*>(chunk + bl * 128 + lane8 * 16);
+        float w[8];
+        const uint32_t words[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          w[2 * e] = bf16lo(words[e]);
+          w[2 * e + 1] = bf16hi(words[e]);
         }
+        float m = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(w[e]));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+        const float c = m;
+        uint32_t code[8];
+        if (c == 0.f) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) code[e] = 7u;  // the exact-zero level
+        } else {
+          const float hr = hf * rcp_approx(c);
+          float dmin = 3.0e38f;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const uint32_t kb = __float_as_uint(fmaf(w[e], hr, magic));
+            const float tk = lds_f32(tc_base + ((kb & 0xFFu) << 2));
+            const float d = fmaf(-c, tk, w[e]);
+            code[e] = static_cast<uint32_t>((__float_as_int(tk) & 31) + (__float_as_int(d) >> 31));
+            dmin = fminf(dmin, fabsf(d));
+          }
+          if (!(dmin > c * 0x1p-18f) || H == 0 || !(c >= 0x1p-100f)) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) code[e] = static_cast<uint32_t>(nf4_code_exact(w[e], c, s_thr));
+          }
+        }
+        const int64_t b = c0 + bl;
+        if (WRITE && valid) {
+          // element 2e in the high nibble of byte e
+          const uint32_t b0 = code[0] * 16u + code[1], b1 = code[2] * 16u + code[3];
+          const uint32_t b2 = code[4] * 16u + code[5], b3 = code[6] * 16u + code[7];
+          const uint32_t word = __byte_perm(__byte_perm(b0, b1, 0x1140), __byte_perm(b2, b3, 0x1140), 0x5410);
+          packed[b * 8 + lane8] = word;
+          if (lane8 == 0) absmax[b] = c;
+        }
+        if (SSE) {
+          float sse = 0.f;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float r = fmaf(-c, lds_f32(lv_base + (code[e] << 2)), w[e]);
+            sse = fmaf(r, r, sse);
+          }
+          sse += __shfl_xor_sync(0xffffffffu, sse, 1);
+          sse += __shfl_xor_sync(0xffffffffu, sse, 2);
+          sse += __shfl_xor_sync(0xffffffffu, sse, 4);
+          if (lane8 == 0 && valid) acc += static_cast<double>(sse);
+        }
+      }
+      __syncwarp();
+      if ((tid & 31) == 0) mbar_arrive(&empty[st]);  // this warp is done with the stage
+      if (++st == kQStages) {
+        st = 0;
+        ph ^= 1u;
       }
     }
   }
   if (SSE) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if ((tid & 31) == 0) s_red[tid >> 5] = acc;
-    __syncthreads();
-    if (tid == 0) {
-      double t = 0.0;
-      for (int i = 0; i < kQThreads / 32; ++i) t += s_red[i];
-      sse_part[blockIdx.x] = t;
-    }
+    if ((tid & 31) == 0 && warp < kQWorkers) s_red[warp] = acc;
+  }
+  __syncthreads();
+  if (SSE && tid == 0) {
+    double t = 0.0;
+    for (int i = 0; i < kQWorkers; ++i) t += s_red[i];
+    sse_part[blockIdx.x] = t;
   }
 }
 
