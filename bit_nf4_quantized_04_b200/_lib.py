@@ -40,6 +40,7 @@ SIGNATURES = {
     "qnf4_double_quant": (ST, [P, I64, I32, P, P, P, P, SZ, P]),
     "qnf4_dequant": (ST, [C.POINTER(Qnf4Weight), P, I32, P]),
     "qnf4_qlora_linear_fwd": (ST, [C.POINTER(Qnf4Weight), P, I64, P, P, I32, F32, P, P, SZ, P]),
+    "qnf4_qlora_linear_fwd_noalloc": (ST, [C.POINTER(Qnf4Weight), P, I64, P, P, I32, F32, P, P]),
     "qnf4_qlora_linear_bwd": (ST, [C.POINTER(Qnf4Weight), P, P, I64, P, P, I32, F32, P, P, P, P,
                                    SZ, P]),
     "qnf4_nf4_recon_error": (ST, [P, I64, I64, I32, P, P, SZ, P]),

@@ -623,6 +623,34 @@ qnf4_status check_linear_args(int64_t N, int64_t K, int64_t M, int r, bool bwd,
   return QNF4_OK;
 }
 
+
+// ---------------------------------------------------------------------------
+// Workspace for the allocation-free forward (qnf4_qlora_linear_fwd_noalloc). A
+// file-scope device array: every GPU that loads the library holds it until exit.
+// ---------------------------------------------------------------------------
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;  // 8 MiB
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of the array on the current device, looked up once per device
+// (cudaGetSymbolAddress with that device current); nullptr and a message on failure.
+void* noalloc_scratch_ptr() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+  static std::mutex mu;
+  static std::vector<void*> cache;
+  std::lock_guard<std::mutex> lk(mu);
+  if (static_cast<int>(cache.size()) <= dev) cache.resize(dev + 1, nullptr);
+  if (!cache[dev]) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) {
+      fail(QNF4_ERR_CUDA, "scratch address: %s", cudaGetErrorString(e));
+      return nullptr;
+    }
+    cache[dev] = p;
+  }
+  return cache[dev];
+}
 }  // namespace
 }  // namespace qnf4
 
@@ -838,6 +866,25 @@ qnf4_status qnf4_qlora_linear_fwd(const qnf4_weight* w, const void* x, int64_t M
   src.N = w->N;
   src.K = w->K;
   return linear_fwd(src, x, M, A, B, r, scale, h, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+qnf4_status qnf4_qlora_linear_fwd_noalloc(const qnf4_weight* w, const void* x, int64_t M,
+                                          const void* A, const void* B, int32_t r, float scale,
+                                          void* h, void* stream) {
+  qnf4_status st = check_weight(w);
+  if (st != QNF4_OK) return st;
+  st = check_linear_args(w->N, w->K, M, r, false, {x, A, B, h});
+  if (st != QNF4_OK) return st;
+  if (M == 0) return QNF4_OK;
+  const size_t need = qnf4_workspace_size(QNF4_OP_FWD, w->N, w->K, M, r);
+  if (need > kNoAllocScratchBytes)
+    return fail(QNF4_ERR_WORKSPACE,
+                "this shape needs %zu bytes of workspace; the built-in scratch holds %zu "
+                "(use qnf4_qlora_linear_fwd with a caller-provided workspace)",
+                need, kNoAllocScratchBytes);
+  void* ws = noalloc_scratch_ptr();
+  if (!ws) return QNF4_ERR_CUDA;
+  return qnf4_qlora_linear_fwd(w, x, M, A, B, r, scale, h, ws, kNoAllocScratchBytes, stream);
 }
 
 qnf4_status qnf4_qlora_linear_bwd(const qnf4_weight* w, const void* x, const void* dY, int64_t M,

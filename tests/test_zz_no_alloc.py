@@ -1,0 +1,50 @@
+"""The allocation-free forward entry point, through the C ABI.
+
+Callers that cannot allocate device memory (an allocator callback, a pre-planned
+engine's host hook, a caller without a device allocator of its own) use
+qnf4_qlora_linear_fwd_noalloc, which takes its workspace from an array built into the
+library. Its output must match the regular entry point (caller-provided workspace)
+within the GEMM tolerance, on two calls in a row (the second reuses the array's
+leftover contents). This file sorts last so a run that stops at the first failure
+has run every other test first.
+"""
+import ctypes as C
+
+import pytest
+import torch
+
+import synth
+
+from helpers import assert_close, f64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("N,K,M,r", [(4096, 4096, 16, 16), (384, 640, 130, 8)])
+def test_noalloc_forward_matches_workspace_forward(N, K, M, r):
+    import bit_nf4_quantized_04_b200 as q
+    W = synth.llama_weight((N, K), 77 + N)
+    x = synth.normal_bf16((M, K), 1.0, 78).cuda()
+    A = synth.normal_bf16((r, K), 0.01, 79).cuda()
+    B = synth.normal_bf16((N, r), 0.01, 80).cuda()
+    s = 2.0
+    w = q.quantize_weight(W.cuda())
+    ref = q.qlora_linear_fwd(w, x, A, B, s)
+    cw = w.c()
+    stream = torch.cuda.current_stream().cuda_stream
+    for _ in range(2):
+        h = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+        st = q.lib.qnf4_qlora_linear_fwd_noalloc(C.byref(cw), x.data_ptr(), M, A.data_ptr(),
+                                                 B.data_ptr(), r, s, h.data_ptr(), stream)
+        assert st == 0, q.lib.qnf4_last_error()
+        torch.cuda.synchronize()
+        assert_close(f64(h.cpu()), f64(ref.cpu()), "no-alloc forward")
+
+
+def test_noalloc_forward_rejects_oversized_shapes():
+    import bit_nf4_quantized_04_b200 as q
+    fake = 1 << 20  # rejected on the host before anything is launched or dereferenced
+    w = q.Qnf4Weight(4096, 4096, 64, 256, fake, fake, fake, fake)
+    st = q.lib.qnf4_qlora_linear_fwd_noalloc(C.byref(w), fake, 1 << 20, fake, fake, 16, 1.0,
+                                             fake, None)
+    assert st == 6 and b"built-in scratch" in q.lib.qnf4_last_error()
