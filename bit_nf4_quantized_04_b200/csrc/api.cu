@@ -243,9 +243,11 @@ GemmPlan plan_gemm(int asrc, int64_t rows, int64_t cols, int64_t contraction, in
   // as fit in one wave, at least two steps each.
   const int64_t tiles = p.tiles();
   const int64_t slots = static_cast<int64_t>(nsm) * p.ctas_per_sm;
+  // Each split costs its partial tile and one more term in the last CTA's reduction,
+  // so keep at least four steps per split.
   int best = 1;
   if (tiles < slots && p.nsteps > 1) {
-    const int max_splits = std::max(1, p.nsteps / 2);
+    const int max_splits = std::max(1, p.nsteps / 4);
     best = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(max_splits, slots / tiles)));
   }
   p.steps_per_split = (p.nsteps + best - 1) / best;

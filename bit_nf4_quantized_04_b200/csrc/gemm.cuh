@@ -733,9 +733,22 @@ __global__ void __launch_bounds__(gemm_threads(NSET), MINB)
             float v[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) v[j] = 0.f;
-            for (int zz = 0; zz < g.splits; ++zz) {
+            // Partials in split order (deterministic), four splits' loads in flight at
+            // a time so the reduction costs one L2 round trip per four splits.
+            for (int zz = 0; zz < g.splits; zz += 4) {
+              float t[4][16];
 #pragma unroll
-              for (int j = 0; j < 16; ++j) v[j] += __ldcg(all + zz * tsz + (c0 + j) * 128 + rl);
+              for (int u = 0; u < 4; ++u) {
+                const bool in = zz + u < g.splits;
+                const float* src = all + (zz + u) * tsz + c0 * 128 + rl;
+#pragma unroll
+                for (int j = 0; j < 16; ++j) t[u][j] = in ? __ldcg(src + j * 128) : 0.f;
+              }
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+#pragma unroll
+                for (int j = 0; j < 16; ++j) v[j] += t[u][j];
+              }
             }
             epi_store(g, row, col0 + c0, v, 16);
           }
