@@ -217,7 +217,6 @@ GemmPlan plan_gemm(int asrc, int64_t rows, int64_t cols, int64_t contraction, in
   p.nset = src_deq(asrc) ? (thin ? QNF4_NSET_THIN : (src_tmem_a(asrc) ? QNF4_NSET_WIDE_TMEM
                                                                        : QNF4_NSET_WIDE_SMEM))
                          : 1;
-  if (asrc == A_CHANQ_K) p.nset = thin ? 1 : 2;
   if (src_tmem_a(asrc)) {
     // TMEM A stages. Each is reusable only after the MMA that read it has completed,
     // so the ring depth bounds the steps in flight per MMA round trip: as deep as the

@@ -16,7 +16,8 @@
 //              = output features (backward dX = dY W). Same converter, MN-major tile.
 //   A_DENSE_K  bf16 matrix by TMA, K-major (dense layers, x for u = x A^T, dY for v).
 //   A_DENSE_MN bf16 matrix by TMA, MN-major (dense dX, x^T for dA, dY^T for dB).
-//   A_CHANQ_K  per-output-channel 1/2/4-bit codes with per-row mapping tables.
+//   A_CHANQ_K  per-output-channel 1/2/4-bit codes with per-row mapping tables,
+//              widened to the 4-bit layout and looked up like NF4 (A in tensor memory).
 //
 // The extra chunk adds sum_j Aext[row, j] * Bext[col, j] over j < r into the same
 // TMEM accumulator: the rank-r adapter term of "QLoRA: Efficient Finetuning of
@@ -27,8 +28,8 @@
 // takes the steps i with i % NSET == h, one 64-element NF4 block per thread and
 // step) and then run the epilogue (tcgen05.ld from TMEM, optional split-K reduction
 // in the last-arriving CTA). For A_NF4_K the dequantized operand goes straight into
-// tensor memory with tcgen05.st and the MMA reads A from there; the other sources
-// stage A in shared memory. Every wait is bounded; on timeout the kernel records an
+// tensor memory with tcgen05.st and the MMA reads A from there (likewise for
+// A_CHANQ_K); the other sources stage A in shared memory. Every wait is bounded; on timeout the kernel records an
 // error, stops, drains its own copies and MMAs, frees TMEM and returns.
 #pragma once
 #include "common.cuh"
@@ -44,7 +45,6 @@ constexpr uint32_t kATile = 128u * 128u;  // 128 rows x 64 bf16 (or 2 x 64 x 64 
 constexpr uint32_t kPTile = 4096u;         // packed NF4 bytes of one step
 constexpr int kMaxS1 = 16;
 constexpr int kMaxS2 = 8;
-constexpr uint32_t kCqStride = 17;  // floats per row of the chanq table (padding vs conflicts)
 
 __host__ __device__ constexpr bool src_deq(int a) {
   return a == A_NF4_K || a == A_NF4_MN || a == A_CHANQ_K;
@@ -56,7 +56,9 @@ __host__ __device__ constexpr bool src_packed_tma(int a) { return a == A_NF4_K |
 #ifndef QNF4_NF4K_TMEM_A
 #define QNF4_NF4K_TMEM_A 1
 #endif
-__host__ __device__ constexpr bool src_tmem_a(int a) { return QNF4_NF4K_TMEM_A && a == A_NF4_K; }
+__host__ __device__ constexpr bool src_tmem_a(int a) {
+  return QNF4_NF4K_TMEM_A && (a == A_NF4_K || a == A_CHANQ_K);
+}
 __host__ __device__ constexpr int gemm_threads(int nset) { return 64 + 128 * nset; }
 
 // TMEM columns: the fp32 accumulator (a power of two >= tn, at least 32), then
@@ -133,7 +135,7 @@ __host__ __device__ inline SmemPlan smem_plan(int asrc, int tn, int s1, int s2, 
   p.ring2 = static_cast<uint32_t>(s1) * p.slot1;
   p.ext = p.ring2 + static_cast<uint32_t>(s2) * p.slot2;
   p.cq = p.ext + (has_ext ? kATile : 0u);
-  p.total = p.cq + (asrc == A_CHANQ_K ? 128u * kCqStride * 4u : 0u);
+  p.total = p.cq + (asrc == A_CHANQ_K ? 256u * 4u : 0u);
   return p;
 }
 
@@ -246,34 +248,6 @@ QNF4_DEV void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
       "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
       "r"(r[29]), "r"(r[30]), "r"(r[31])
       : "memory");
-}
-
-// One 64-element group of a per-channel row with B-bit codes (MSB first).
-template <int B>
-QNF4_DEV void chanq_group_to_bf16(const uint8_t* src, float g, const float* tab,
-                                  uint32_t (&o)[32]) {
-  constexpr int NW = 2 * B;  // 32-bit words holding 64 codes
-  uint32_t w[NW];
-#pragma unroll
-  for (int i = 0; i < NW / 2; ++i) {
-    const uint2 v = __ldg(reinterpret_cast<const uint2*>(src) + i);
-    w[2 * i] = v.x;
-    w[2 * i + 1] = v.y;
-  }
-  constexpr uint32_t mask = (1u << B) - 1u;
-#pragma unroll
-  for (int e = 0; e < 64; e += 2) {
-    uint32_t c[2];
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int bit = (e + h) * B;           // position in the MSB-first stream
-      const int byte = bit >> 3;
-      const int sh = 8 - B - (bit & 7);      // shift inside that byte
-      const uint32_t by = (w[byte >> 2] >> (8 * (byte & 3))) & 0xFFu;
-      c[h] = (by >> sh) & mask;
-    }
-    o[e >> 1] = pack_bf16x2(tab[c[0]] * g, tab[c[1]] * g);
-  }
 }
 
 QNF4_DEV uint16_t f2bf(float f) {
@@ -642,39 +616,96 @@ __global__ void __launch_bounds__(gemm_threads(NSET), MINB)
         mbar_arrive(&full2[s2]);
       }
     } else if constexpr (ASRC == A_CHANQ_K) {
-      const int64_t n = row0 + t;
+      // Row slot = the TMEM lane this warp may access; the row's 2^b mapping values
+      // live in registers (unused entries 0), and each 64-element group's codes are
+      // widened to the 4-bit layout of NF4 so the same register lookup applies.
+      const int slot = q * 32 + lane;
+      const int64_t n = row0 + slot;
       const bool valid = n < g.wN;
+      uint32_t* s_t1 = reinterpret_cast<uint32_t*>(base + sp.cq);  // 1-bit byte -> nibble word
+      if (set == 0) {
+        for (int e = t; e < 256; e += 128) {
+          uint32_t word = 0;
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            const uint32_t hi = (static_cast<uint32_t>(e) >> (7 - 2 * m)) & 1u;
+            const uint32_t lo = (static_cast<uint32_t>(e) >> (6 - 2 * m)) & 1u;
+            word |= ((hi << 4) | lo) << (8 * m);
+          }
+          s_t1[e] = word;
+        }
+      }
+      named_sync(2, NCONV);  // the table is read by every converter set
       int bits = 1;
       const uint8_t* prow = nullptr;
-      float* tab = reinterpret_cast<float*>(base + sp.cq) + t * kCqStride;
-      if (valid && set == 0) {
-        const int64_t mo = g.cq_map_off[n];
-        for (int c = 0; c < (1 << g.cq_bits[n]); ++c) tab[c] = g.cq_map[mo + c];
+      float mp[16];
+      {
+        int64_t mo = 0;
+        if (valid) {
+          bits = g.cq_bits[n];
+          prow = g.cq_packed + g.cq_row_off[n];
+          mo = g.cq_map_off[n];
+        }
+        const int nmap = valid ? (1 << bits) : 0;
+#pragma unroll
+        for (int c = 0; c < 16; ++c) mp[c] = c < nmap ? g.cq_map[mo + c] : 0.f;
       }
-      if (valid) {
-        bits = g.cq_bits[n];
-        prow = g.cq_packed + g.cq_row_off[n];
-      }
-      if (NSET > 1) named_sync(2, NCONV);  // the tables are shared by both sets
       for (ConvCursor cur(set); cur.i < nst; cur.next(NSET, S1, S2)) {
         const int i = cur.i;
         const int s2 = cur.s2;
         const int gi = step0 + i;
+        // the group's codes and scale (issued before the waits)
+        uint32_t cw[8];
+        float gm = 0.f;
+        if (valid) {
+          gm = __ldg(g.cq_absmax + n * g.nbk + gi);
+          // A row holds K b / 8 bytes (a multiple of 8, not of 16, e.g. K = 448) and a
+          // group 8 b bytes, so only 8-byte loads are aligned for every shape.
+          const uint2* src = reinterpret_cast<const uint2*>(prow + static_cast<int64_t>(gi) * 8 * bits);
+          if (bits == 4) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const uint2 a = __ldg(src + k);
+              cw[2 * k] = a.x;
+              cw[2 * k + 1] = a.y;
+            }
+          } else if (bits == 2) {
+            const uint2 a0 = __ldg(src), a1 = __ldg(src + 1);
+            const uint32_t in[4] = {a0.x, a0.y, a1.x, a1.y};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              // byte x = c0 c1 c2 c3 (2 bits each, first at the top) -> (c0 c1), (c2 c3)
+              const uint32_t w = in[k];
+              const uint32_t hi = ((w >> 2) & 0x30303030u) | ((w >> 4) & 0x03030303u);
+              const uint32_t lo = ((w << 2) & 0x30303030u) | (w & 0x03030303u);
+              cw[2 * k] = __byte_perm(hi, lo, 0x5140);
+              cw[2 * k + 1] = __byte_perm(hi, lo, 0x7362);
+            }
+          } else {
+            const uint2 a = __ldg(src);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) cw[k] = s_t1[((k < 4 ? a.x : a.y) >> (8 * (k & 3))) & 0xFFu];
+          }
+        } else {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) cw[k] = 0u;
+        }
         if (!wait_or_abort(&full1[cur.s], cur.ph, g.wait_ns, &s_abort, 33)) break;
         if (i >= S2 && !wait_or_abort(&empty1[cur.sj], cur.phj, g.wait_ns, &s_abort, 34)) break;
         uint32_t o[32];
-        if (valid) {
-          const float gm = __ldg(g.cq_absmax + n * g.nbk + gi);
-          const uint8_t* src = prow + static_cast<int64_t>(gi) * 8 * bits;
-          if (bits == 4) chanq_group_to_bf16<4>(src, gm, tab, o);
-          else if (bits == 2) chanq_group_to_bf16<2>(src, gm, tab, o);
-          else chanq_group_to_bf16<1>(src, gm, tab, o);
-        } else {
+        Nf4Planes P;
+        nf4_planes(mp, gm, P);
 #pragma unroll
-          for (int c = 0; c < 32; ++c) o[c] = 0u;
+        for (int k = 0; k < 8; ++k) nf4_lookup8(cw[k], P, &o[4 * k]);
+        if (TMA_A) {
+          tc_fence_after();
+          tmem_st32(tmem + (static_cast<uint32_t>(q * 32) << 16) + a_col + 32u * s2, o);
+          tmem_wait_st();
+          tc_fence_before();
+        } else {
+          store_row_sw128(base + sp.ring2 + s2 * sp.slot2, slot, o);
+          fence_proxy_async();
         }
-        store_row_sw128(base + sp.ring2 + s2 * sp.slot2, t, o);
-        fence_proxy_async();
         mbar_arrive(&full2[s2]);
       }
     }
