@@ -108,5 +108,10 @@ def test_workspace_sizes_are_positive_and_monotone(q):
     a = q.workspace_size(q._lib.OP_FWD, 4096, 4096, 16, 16)
     b = q.workspace_size(q._lib.OP_FWD, 4096, 4096, 4096, 16)
     c = q.workspace_size(q._lib.OP_BWD, 4096, 4096, 4096, 16)
-    assert 0 < a < b < c
+    assert 0 < a and 0 < b < c
+    # the decode path (M <= 16) fits the allocation-free forward's 8 MiB scratch on
+    # every Llama-2-7B layer shape
+    for N, K in [(4096, 4096), (11008, 4096), (4096, 11008)]:
+        for M in (1, 8, 9, 16):
+            assert 0 < q.workspace_size(q._lib.OP_FWD, N, K, M, 64) <= 8 << 20
     assert q.workspace_size(q._lib.OP_QUANTIZE, 4096, 4096) > 0
