@@ -17,7 +17,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libqnf4.so")
 SOURCES = ["api.cu", "codebook.cpp"]
-HEADERS = ["common.cuh", "quant.cuh", "chanq.cuh", "gemm.cuh", "decode.cuh", "tables.h"]
+HEADERS = ["common.cuh", "quant.cuh", "chanq.cuh", "gemm.cuh", "tables.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

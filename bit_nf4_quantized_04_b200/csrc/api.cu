@@ -17,7 +17,6 @@
 #include "../../include/qnf4.h"
 #include "chanq.cuh"
 #include "common.cuh"
-#include "decode.cuh"
 #include "gemm.cuh"
 #include "quant.cuh"
 #include "tables.h"
@@ -80,9 +79,9 @@ QuantTab make_tab() {
 constexpr int kQuantMaxGrid = 1024;
 
 int quant_grid(int64_t nblocks) {
-  // persistent: two streaming CTAs per SM, never more CTAs than chunks
+  // persistent: kQCtasPerSm streaming CTAs per SM, never more CTAs than chunks
   const int64_t chunks = (nblocks + kQChunkBlocks - 1) / kQChunkBlocks;
-  return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(chunks, num_sms() * 2)));
+  return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(chunks, num_sms() * kQCtasPerSm)));
 }
 
 bool g_quant_smem_set[64] = {};
@@ -493,178 +492,6 @@ qnf4_status linear_fwd(const BaseSrc& src, const void* x, int64_t M, const void*
   return st;
 }
 
-// ---------------------------------------------------------------------------
-// Decode forward (M <= 16 tokens): adapter kernel + streaming dequant/mma.sync kernel.
-// ---------------------------------------------------------------------------
-struct DecPlan {
-  int64_t T = 0;
-  int KB = 0, G = 0, nchunks = 0, jmax = 1, grid = 0;
-  int xrows = 0;
-  int gb[kDecMaxChunks + 1] = {};
-  int cb[kDecMaxChunks + 1] = {};
-  size_t smem = 0;
-  size_t off_u = 0, off_cnt = 0, off_part = 0, total = 0;
-  bool fits = false;  // every warp's run touches at most kDecMaxFin tiles
-  bool usable() const { return nchunks >= 1 && nchunks <= kDecMaxChunks && fits; }
-};
-
-DecPlan plan_dec(int64_t N, int64_t K, int64_t M, int nsm) {
-  DecPlan D;
-  D.T = (N + kDecRows - 1) / kDecRows;
-  D.KB = static_cast<int>(K / 64);
-  D.G = (D.KB + 3) / 4;
-  D.xrows = static_cast<int>(M) + (M < kDecMaxTok ? 1 : 0);       // tokens, plus a zero row
-  const int gmax = kDecSmem / (D.xrows * 4 * 128);  // 256-column groups per x window
-  D.nchunks = (D.G + gmax - 1) / gmax;
-  if (D.nchunks < 1 || D.nchunks > kDecMaxChunks) return D;
-  if (N * (K / 2) >= (int64_t(1) << 31)) return D;  // 32-bit code offsets
-  const int gc = (D.G + D.nchunks - 1) / D.nchunks;
-  for (int c = 0; c < D.nchunks; ++c) D.gb[c] = std::min(D.G, c * gc);
-  D.gb[D.nchunks] = D.G;
-  // one CTA per SM, shared between the chunks in proportion to their columns; the
-  // prep kernel's SMs stay free, so that its cluster runs beside the main grid
-  const int64_t ctas = nsm > 2 * kDecPrepCtas ? nsm - kDecPrepCtas : nsm;
-  D.cb[0] = 0;
-  for (int c = 0; c < D.nchunks; ++c) {
-    const int64_t g = D.gb[c + 1] - D.gb[c];
-    int64_t n = (ctas * g + D.G - 1) / D.G;
-    n = std::min(n, (D.T * g + kDecWarps - 1) / kDecWarps);
-    D.cb[c + 1] = D.cb[c] + static_cast<int>(std::max<int64_t>(1, n));
-  }
-  D.grid = D.cb[D.nchunks];
-  D.jmax = 1;
-  D.fits = true;
-  for (int c = 0; c < D.nchunks; ++c) {
-    const DecSplit sp = dec_split(D.T, D.gb[c], D.gb[c + 1], D.cb[c + 1] - D.cb[c]);
-    for (int64_t p = 0; p < D.T; ++p) D.jmax = std::max(D.jmax, sp.ncon(p));
-    const int64_t maxlen = (sp.items + sp.tw - 1) / sp.tw;
-    if ((2 * sp.gc - 2 + maxlen) / sp.gc > kDecMaxFin) D.fits = false;
-    if (sp.items > (int64_t(1) << 26) || sp.tw > (int64_t(1) << 24)) D.fits = false;  // exact divisions
-  }
-  D.smem = kDecRingBytes + 128 + static_cast<size_t>(D.xrows) * (4 * gc) * 128;
-  size_t o = 0;
-  D.off_u = o;
-  o = align256(o + static_cast<size_t>(kDecUShare) * sizeof(float));
-  D.off_cnt = o;
-  o = align256(o + static_cast<size_t>(D.T) * sizeof(unsigned int));
-  D.off_part = o;
-  o = align256(o + static_cast<size_t>(D.T) * D.nchunks * D.jmax * kDecSlot * sizeof(float));
-  D.total = o;
-  return D;
-}
-
-bool g_dec_smem_set[3][64] = {};
-
-qnf4_status launch_dec_main(const DecPlan& D, const DecArgs& a, cudaStream_t s) {
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !g_dec_smem_set[1][dev]) {
-    for (auto k : {k_dec<false>, k_dec<true>}) {
-      const cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 kDecRingBytes + 128 + kDecSmem);
-      if (e != cudaSuccess) return fail(QNF4_ERR_CUDA, "smem attribute: %s", cudaGetErrorString(e));
-    }
-    g_dec_smem_set[1][dev] = true;
-  }
-  cudaLaunchConfig_t cfg;
-  std::memset(&cfg, 0, sizeof(cfg));
-  cfg.gridDim = dim3(D.grid, 1, 1);
-  cfg.blockDim = dim3(kDecThreads, 1, 1);
-  cfg.dynamicSmemBytes = D.smem;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  const cudaError_t e = a.M > 8 ? cudaLaunchKernelEx(&cfg, k_dec<true>, a) : cudaLaunchKernelEx(&cfg, k_dec<false>, a);
-  if (e != cudaSuccess) {
-    g_launches.fetch_add(1, std::memory_order_relaxed);
-    cudaGetLastError();
-    return fail(QNF4_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
-  }
-  return launched("decode");
-}
-
-qnf4_status linear_fwd_dec(const qnf4_weight* w, const void* x, int64_t M, const void* A,
-                           const void* B, int r, float scale, void* h, void* ws, size_t ws_bytes,
-                           cudaStream_t s) {
-  const DecPlan D = plan_dec(w->N, w->K, M, num_sms());
-  if (!ws || ws_bytes < D.total) return fail(QNF4_ERR_WORKSPACE, "workspace too small (%zu < %zu)", ws_bytes, D.total);
-  if (!al16(ws)) return fail(QNF4_ERR_ALIGN, "the workspace must be 16-byte aligned");
-  uint8_t* w8 = static_cast<uint8_t*>(ws);
-  unsigned int* cnt = reinterpret_cast<unsigned int*>(w8 + D.off_cnt);
-  float* u = reinterpret_cast<float*>(w8 + D.off_u);
-  {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 64 && !g_dec_smem_set[0][dev]) {
-      const cudaError_t e = cudaFuncSetAttribute(k_dec_prep, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 kDecPrepWarps * kDecUShare * 4);
-      if (e != cudaSuccess) return fail(QNF4_ERR_CUDA, "smem attribute: %s", cudaGetErrorString(e));
-      g_dec_smem_set[0][dev] = true;
-    }
-    cudaLaunchConfig_t cfg;
-    std::memset(&cfg, 0, sizeof(cfg));
-    cfg.gridDim = dim3(kDecPrepCtas, 1, 1);
-    cfg.blockDim = dim3(kDecPrepThreads, 1, 1);
-    cfg.dynamicSmemBytes = static_cast<size_t>(kDecPrepWarps) * kDecUShare * 4;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[2];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = kDecPrepCtas;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[1].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 2;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, k_dec_prep, static_cast<const uint16_t*>(x),
-                                             static_cast<const uint16_t*>(A), static_cast<int>(M),
-                                             w->K, r, u, cnt, D.T);
-    if (e != cudaSuccess) {
-      g_launches.fetch_add(1, std::memory_order_relaxed);
-      cudaGetLastError();
-      return fail(QNF4_ERR_CUDA, "decode prep launch: %s", cudaGetErrorString(e));
-    }
-    launched("decode prep");
-  }
-  DecArgs a;
-  std::memset(&a, 0, sizeof(a));
-  a.packed = w->packed;
-  a.code2 = w->code2;
-  a.scale2 = w->scale2;
-  a.mean = w->mean;
-  a.x = static_cast<const uint16_t*>(x);
-  a.A = static_cast<const uint16_t*>(A);
-  a.B = static_cast<const uint16_t*>(B);
-  a.u = u;
-  a.scale = scale;
-  a.h = static_cast<uint16_t*>(h);
-  a.part = reinterpret_cast<float*>(w8 + D.off_part);
-  a.cnt = cnt;
-  a.xrows = D.xrows;
-  a.N = w->N;
-  a.K = w->K;
-  a.T = D.T;
-  a.M = static_cast<int>(M);
-  a.r = r;
-  a.KB = D.KB;
-  a.jmax = D.jmax;
-  a.nchunks = D.nchunks;
-  std::memcpy(a.gb, D.gb, sizeof(a.gb));
-  std::memcpy(a.cb, D.cb, sizeof(a.cb));
-  std::memcpy(a.levels, nf4_tables().levels, sizeof(a.levels));
-  if (g_ev_start) cudaEventRecord(g_ev_start, s);
-  const qnf4_status st = launch_dec_main(D, a, s);
-  if (g_ev_stop) cudaEventRecord(g_ev_stop, s);
-  return st;
-}
-
-bool use_dec(int64_t N, int64_t K, int64_t M) {
-  return M >= 1 && M <= kDecMaxTok && plan_dec(N, K, M, 1).usable();
-}
-
 qnf4_status linear_bwd(const BaseSrc& src, const void* x, const void* dY, int64_t M, const void* A,
                        const void* B, int r, float scale, void* dX, float* dA, float* dB, void* ws,
                        size_t ws_bytes, cudaStream_t s) {
@@ -888,9 +715,7 @@ size_t qnf4_workspace_size(int32_t op, int64_t N, int64_t K, int64_t M, int32_t 
   switch (op) {
     case QNF4_OP_QUANTIZE: return kQuantMaxGrid * sizeof(double);
     case QNF4_OP_DOUBLE_QUANT: return kDqPartials * sizeof(double);
-    case QNF4_OP_FWD:
-      if (use_dec(N, K, M)) return plan_dec(N, K, M, num_sms()).total;
-      return plan_linear(A_NF4_K, N, K, M, r, false, num_sms()).total;
+    case QNF4_OP_FWD: return plan_linear(A_NF4_K, N, K, M, r, false, num_sms()).total;
     case QNF4_OP_BWD: return plan_linear(A_NF4_MN, N, K, M, r, true, num_sms()).total;
     case QNF4_OP_CHANQ_FWD: return plan_linear(A_CHANQ_K, N, K, M, r, false, num_sms()).total;
     default: return 0;
@@ -1036,8 +861,6 @@ qnf4_status qnf4_qlora_linear_fwd(const qnf4_weight* w, const void* x, int64_t M
   st = check_linear_args(w->N, w->K, M, r, false, {x, A, B, h});
   if (st != QNF4_OK) return st;
   if (M == 0) return QNF4_OK;
-  if (use_dec(w->N, w->K, M))
-    return linear_fwd_dec(w, x, M, A, B, r, scale, h, ws, ws_bytes, static_cast<cudaStream_t>(stream));
   BaseSrc src;
   src.kind = A_NF4_K;
   src.w = w;
