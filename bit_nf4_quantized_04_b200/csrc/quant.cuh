@@ -43,6 +43,24 @@ QNF4_DEV float rcp_approx(float x) {
   return r;
 }
 
+// Two fp32 lanes in one 64-bit register, and the packed fma of sm_100 (two IEEE
+// single-precision fused multiply-adds, round to nearest even: each lane is fmaf).
+QNF4_DEV uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+QNF4_DEV float2 f2_unpack(uint64_t v) {
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+  return r;
+}
+QNF4_DEV uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+
 QNF4_DEV float lds_f32(uint32_t addr) {
   float v;
   asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
@@ -52,6 +70,7 @@ QNF4_DEV float lds_f32(uint32_t addr) {
 constexpr int kQChunkBlocks = 128;  // 64-element blocks per streamed chunk (16 KB of bf16)
 constexpr int kQStages = 4;         // chunks in flight per CTA
 constexpr int kQWorkers = 8;        // worker warps; one more warp issues the copies
+constexpr int kQCtasPerSm = 3;      // resident CTAs per SM (registers and shared memory allow it)
 constexpr int kQThreads = 32 * (kQWorkers + 1);
 constexpr uint32_t kQChunkBytes = kQChunkBlocks * 128u;
 constexpr size_t kQSmem = kQStages * kQChunkBytes + 128;
@@ -93,7 +112,7 @@ QNF4_DEV bool warp_wait(uint64_t* bar, uint32_t parity, unsigned long long wait_
 // quotient and the full count. Non-finite weights are outside the method: the table
 // index is masked, so they cannot read outside it, but their codes are unspecified.
 template <bool WRITE, bool SSE>
-__global__ void __launch_bounds__(kQThreads, 2)
+__global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
     k_nf4_quant(const uint16_t* __restrict__ W, int64_t nblocks, uint32_t* __restrict__ packed,
                 float* __restrict__ absmax, double* __restrict__ sse_part, QuantTab tab,
                 unsigned long long wait_ns) {
@@ -101,7 +120,7 @@ __global__ void __launch_bounds__(kQThreads, 2)
   __shared__ __align__(8) uint64_t full[kQStages], empty[kQStages];
   __shared__ float s_thr[16];
   __shared__ float s_lv[16];
-  __shared__ float s_tc[2 * kMaxHalfBins + 1];
+  __shared__ __align__(1024) float s_tc[2 * kMaxHalfBins + 1];
   __shared__ double s_red[kQWorkers];
   __shared__ volatile int s_abort;
   uint8_t* qsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(qsm_raw) + 127) &
@@ -172,9 +191,9 @@ __global__ void __launch_bounds__(kQThreads, 2)
     // ---------------------------------------------------------------- workers
     const int H = tab.bin_h;
     const float hf = static_cast<float>(H);
-    const float magic = hf + 12582912.0f;
-    const uint32_t tc_base = smem_u32(s_tc);
-    const uint32_t lv_base = smem_u32(s_lv);
+    const uint64_t mg2 = f2_pack(hf + 12582912.0f, hf + 12582912.0f);
+    // the bin table sits 1024-byte aligned, so entry k is at base | 4 (k & 0xFF)
+    const char* tcb = reinterpret_cast<const char*>(s_tc);
     const int lane8 = tid & 7;
     const int grp = tid >> 3;  // 32 groups of 8 threads
     int st = 0;
@@ -190,38 +209,61 @@ __global__ void __launch_bounds__(kQThreads, 2)
         const bool valid = bl < nb;   // groups past a partial chunk's end work on zeros
         uint4 v = make_uint4(0u, 0u, 0u, 0u);
         if (valid) v = *reinterpret_cast<const uint4*>(chunk + bl * 128 + lane8 * 16);
-        float w[8];
         const uint32_t words[4] = {v.x, v.y, v.z, v.w};
+        float w[8];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           w[2 * e] = bf16lo(words[e]);
           w[2 * e + 1] = bf16hi(words[e]);
         }
-        float m = 0.f;
+        float m = fmaxf(fabsf(w[0]), fabsf(w[1]));
 #pragma unroll
-        for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(w[e]));
+        for (int e = 2; e < 8; ++e) m = fmaxf(m, fabsf(w[e]));
         m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
         m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
         m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
         const float c = m;
         uint32_t code[8];
+        float sse = 0.f;
         if (c == 0.f) {
 #pragma unroll
-          for (int e = 0; e < 8; ++e) code[e] = 7u;  // the exact-zero level
+          for (int e = 0; e < 8; ++e) code[e] = 7u;  // the exact-zero level (error 0)
         } else {
           const float hr = hf * rcp_approx(c);
+          const uint64_t hr2 = f2_pack(hr, hr), nc2 = f2_pack(-c, -c);
+          uint64_t wp[4], dp[4];
+          float tk[8];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            wp[e] = f2_pack(w[2 * e], w[2 * e + 1]);
+            const float2 kb = f2_unpack(f2_fma(wp[e], hr2, mg2));
+            tk[2 * e] = *reinterpret_cast<const float*>(tcb + ((__float_as_uint(kb.x) << 2) & 0x3FCu));
+            tk[2 * e + 1] = *reinterpret_cast<const float*>(tcb + ((__float_as_uint(kb.y) << 2) & 0x3FCu));
+          }
           float dmin = 3.0e38f;
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const uint32_t kb = __float_as_uint(fmaf(w[e], hr, magic));
-            const float tk = lds_f32(tc_base + ((kb & 0xFFu) << 2));
-            const float d = fmaf(-c, tk, w[e]);
-            code[e] = static_cast<uint32_t>((__float_as_int(tk) & 31) + (__float_as_int(d) >> 31));
-            dmin = fminf(dmin, fabsf(d));
+          for (int e = 0; e < 4; ++e) {
+            dp[e] = f2_fma(f2_pack(tk[2 * e], tk[2 * e + 1]), nc2, wp[e]);
+            const float2 d = f2_unpack(dp[e]);
+            code[2 * e] = static_cast<uint32_t>((__float_as_int(tk[2 * e]) & 31) + (__float_as_int(d.x) >> 31));
+            code[2 * e + 1] = static_cast<uint32_t>((__float_as_int(tk[2 * e + 1]) & 31) + (__float_as_int(d.y) >> 31));
+            dmin = fminf(dmin, fminf(fabsf(d.x), fabsf(d.y)));
           }
           if (!(dmin > c * 0x1p-18f) || H == 0 || !(c >= 0x1p-100f)) {
 #pragma unroll
             for (int e = 0; e < 8; ++e) code[e] = static_cast<uint32_t>(nf4_code_exact(w[e], c, s_thr));
+          }
+          if (SSE) {
+            // r = w - c q[code], two running sums of r^2 (even and odd elements)
+            uint64_t acc2 = f2_pack(0.f, 0.f);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const uint64_t q2 = f2_pack(s_lv[code[2 * e]], s_lv[code[2 * e + 1]]);
+              const uint64_t r2 = f2_fma(q2, nc2, wp[e]);
+              acc2 = f2_fma(r2, r2, acc2);
+            }
+            const float2 a2 = f2_unpack(acc2);
+            sse = a2.x + a2.y;
           }
         }
         const int64_t b = c0 + bl;
@@ -234,12 +276,6 @@ __global__ void __launch_bounds__(kQThreads, 2)
           if (lane8 == 0) absmax[b] = c;
         }
         if (SSE) {
-          float sse = 0.f;
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float r = fmaf(-c, lds_f32(lv_base + (code[e] << 2)), w[e]);
-            sse = fmaf(r, r, sse);
-          }
           sse += __shfl_xor_sync(0xffffffffu, sse, 1);
           sse += __shfl_xor_sync(0xffffffffu, sse, 2);
           sse += __shfl_xor_sync(0xffffffffu, sse, 4);
