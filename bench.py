@@ -538,7 +538,29 @@ def run_case(args):
               q.workspace_size(q._lib.OP_QUANTIZE, N, K))
     ws = torch.empty(wsz, dtype=torch.uint8, device=dev)
     h = torch.empty(m, N, dtype=torch.bfloat16, device=dev)
-    if args.case in ("fwd", "decode"):
+    if args.case in ("chanq_quant", "chanq_fwd"):
+        # the per-channel 1/2/4-bit layer of the step (11008 x 4096, 2048 tokens)
+        bits = synth.chan_bits(CQ_N)
+        maps, map_off, thr, thr_off = synth.chan_tables(bits)
+        roff = torch.zeros(CQ_N + 1, dtype=torch.int64)
+        roff[1:] = torch.cumsum(CQ_K * bits.to(torch.int64) // 8, 0)
+        bits, maps, map_off, thr, thr_off, roff = (t.to(dev) for t in (bits, maps, map_off, thr, thr_off, roff))
+        cW = synth.llama_weight((CQ_N, CQ_K), synth.SEED_W + 100, device=dev)
+        cp = torch.empty(int(roff[-1]) + 16, dtype=torch.uint8, device=dev)
+        cg = torch.empty(CQ_N * CQ_K // 64, dtype=torch.float32, device=dev)
+        cx = synth.normal_bf16((CQ_M, CQ_K), 1.0, synth.SEED_X + 50, device=dev)
+        cA = A[:, :CQ_K].contiguous()
+        cB = synth.normal_bf16((CQ_N, RANK), 0.01, synth.SEED_B + 50, device=dev)
+        ch = torch.empty(CQ_M, CQ_N, dtype=torch.bfloat16, device=dev)
+        cws = torch.empty(q.workspace_size(q._lib.OP_CHANQ_FWD, CQ_N, CQ_K, CQ_M, RANK), dtype=torch.uint8, device=dev)
+        q.chanq_quantize(cW, bits, thr, thr_off, roff, packed=cp, absmax=cg)
+        if args.case == "chanq_quant":
+            fn = lambda: q.chanq_quantize(cW, bits, thr, thr_off, roff, packed=cp, absmax=cg)  # noqa: E731
+        else:
+            fn = lambda: q.chanq_linear_fwd(cp, roff, bits, maps, map_off, cg, CQ_N, CQ_K, cx, cA, cB, s,  # noqa: E731
+                                            h=ch, ws=cws)
+        N, K, m = CQ_N, CQ_K, (0 if args.case == "chanq_quant" else CQ_M)
+    elif args.case in ("fwd", "decode"):
         fn = lambda: q.qlora_linear_fwd(w, x, A, B, s, h=h, ws=ws)  # noqa: E731
     elif args.case == "bwd":
         fn = lambda: q.qlora_linear_bwd(w, x, dY, A, B, s, ws=ws)  # noqa: E731
@@ -592,7 +614,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-breakdown", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
-    ap.add_argument("--case", choices=["fwd", "bwd", "decode", "quant"], default=None,
+    ap.add_argument("--case", choices=["fwd", "bwd", "decode", "quant", "chanq_quant", "chanq_fwd"], default=None,
                     help="run one operation on one gate-shaped layer (for ncu captures)")
     args = ap.parse_args()
     if args.case:
