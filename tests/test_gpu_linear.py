@@ -146,6 +146,64 @@ def test_chanq_quantize_bit_exact(q, N, K):
     assert np.array_equal(gp.cpu().numpy()[: packed.size], packed)
 
 
+def _bf16_round(a: np.ndarray) -> np.ndarray:
+    """fp32 -> nearest bf16 value (ties to even), as fp32."""
+    u = a.astype(np.float32).view(np.uint32).astype(np.uint64)
+    r = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16) << 16
+    return r.astype(np.uint32).view(np.float32)
+
+
+def test_chanq_quantize_near_edges(q):
+    # Rows of 4-bit codes whose thresholds are bf16 values, weights in groups with
+    # absmax exactly 1 placed on each threshold and one bf16 step either side of it,
+    # so the normalised value hits or straddles every threshold; a row with two
+    # thresholds in one bin and one whose thresholds defeat the bin table (the exact
+    # path); an all-zero group. Codes must match the oracle bit for bit.
+    K = 256
+    rng = np.random.default_rng(7)
+    rows_thr = []
+    for i in range(6):
+        t = np.sort(rng.uniform(-0.95, 0.95, 15)).astype(np.float32)
+        rows_thr.append(_bf16_round(t))
+    t = rows_thr[0].copy()
+    t[7] = _bf16_round(np.array([t[6] * np.float32(1 + 2.0 ** -7)]))[0]  # two in one bin
+    rows_thr.append(np.sort(t))
+    # five thresholds within 0.004 (< any bin): three share a bin at every density, so
+    # the row takes the exact path throughout
+    close = np.float32(0.3) + np.arange(5, dtype=np.float32) * np.float32(2.0 ** -8)
+    t = np.sort(np.concatenate([close, rng.uniform(-0.9, 0.2, 10).astype(np.float32)]))
+    rows_thr.append(_bf16_round(t))
+    N = len(rows_thr)
+    W = np.zeros((N, K), np.float32)
+    for i, t in enumerate(rows_thr):
+        vals = []
+        for x in t:
+            up = np.nextafter(x, np.float32(2), dtype=np.float32)
+            dn = np.nextafter(x, np.float32(-2), dtype=np.float32)
+            vals += [x, _bf16_round(np.array([up + (up - x) * 2**16]))[0],
+                     _bf16_round(np.array([dn - (x - dn) * 2**16]))[0]]
+        vals = np.array(vals, np.float32)
+        row = np.zeros(K, np.float32)
+        for gsi in range(K // 64 - 1):                           # the last group stays all zero
+            seg = rng.choice(vals, 63)
+            row[gsi * 64: gsi * 64 + 63] = seg
+            row[gsi * 64 + 63] = 1.0 if gsi % 2 == 0 else -1.0   # absmax exactly 1
+        W[i] = row
+    Wt = torch.from_numpy(W).to(torch.bfloat16)
+    assert np.array_equal(f32(Wt), W)
+    bits = torch.full((N,), 4, dtype=torch.uint8)
+    thr = torch.from_numpy(np.concatenate(rows_thr).astype(np.float32))
+    thr_off = torch.arange(0, 15 * N + 1, 15, dtype=torch.int64)
+    roff = torch.from_numpy(ochq.row_offsets(bits.numpy(), K))
+    packed, roff_o, g, _ = chanq_oracle(Wt, bits, thr, thr_off)
+    gp, gg = q.chanq_quantize(Wt.cuda(), bits.cuda(), thr.cuda(), thr_off.cuda(), roff.cuda())
+    torch.cuda.synchronize()
+    assert np.array_equal(gg.cpu().numpy().view(np.uint32), g.view(np.uint32))
+    got = gp.cpu().numpy()[: packed.size]
+    bad = np.nonzero(got != packed)[0]
+    assert bad.size == 0, f"{bad.size} code bytes differ, first at {bad[:5]}"
+
+
 @pytest.mark.parametrize("N,K,M,r", [(40, 128, 5, 8), (200, 448, 70, 16), (1100, 4096, 260, 16)])
 def test_chanq_linear_fwd(q, N, K, M, r):
     W, bits, maps, map_off, thr, thr_off, roff = _chanq_case(N, K, 600 + N)
