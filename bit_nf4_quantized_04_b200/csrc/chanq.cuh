@@ -81,8 +81,11 @@ __global__ void __launch_bounds__(256) k_chanq_quant(const uint16_t* __restrict_
     const unsigned ok = __ballot_sync(0xffffffffu, good) & 0xFu;
     const bool row_exact = ok == 0u;
     const float kH = chanq_h(row_exact ? 0 : __ffs(ok) - 1);
-    // ---- the row's bin table (entries past the range are never indexed by finite x)
-    for (int e = lane; e < kCqTable; e += 32) {
+    // ---- the row's bin table: bins 0 .. 2 H + 1 (finite weights index no others; a
+    // non-finite weight indexes entry 0 and its NaN or infinite residual sends the
+    // group to the exact path)
+    const int nbin = 2 * static_cast<int>(kH) + 2;
+    for (int e = lane; e < nbin; e += 32) {
       const float lo = (static_cast<float>(e) - 0.5f) / kH - 1.f;  // bin e's lower edge
       int cnt = 0;
       float tn = 2.0f, tn2 = 2.0f;
