@@ -157,12 +157,15 @@ bool make_map(CUtensorMap* m, const void* ptr, bool u8, uint64_t inner, uint64_t
 struct GemmPlan {
   int asrc = 0, tn = 16, has_ext = 0;
   int64_t rows = 0, cols = 0;
-  int nsteps = 0, row_tiles = 0, col_tiles = 0, splits = 1, steps_per_split = 0, s1 = 1, s2 = 0;
+  int nsteps = 0, row_tiles = 0, col_tiles = 0, s1 = 1, s2 = 0;
+  // work units: full_tiles whole tiles, then tail_tiles tiles cut into tail_splits
+  // contraction slices of tail_sps steps; grid = persistent CTAs
+  int full_tiles = 0, tail_tiles = 0, tail_splits = 1, tail_sps = 0, units = 0, grid = 1;
   int ctas_per_sm = 1;
   int nset = 1;  // converter warp sets (4 warps each)
   size_t smem = 0;
   size_t part_floats() const {
-    return splits > 1 ? static_cast<size_t>(row_tiles) * col_tiles * splits * tn * 128 : 0;
+    return tail_splits > 1 ? static_cast<size_t>(tail_tiles) * tail_splits * tn * 128 : 0;
   }
   int64_t tiles() const { return static_cast<int64_t>(row_tiles) * col_tiles; }
 };
@@ -238,19 +241,27 @@ GemmPlan plan_gemm(int asrc, int64_t rows, int64_t cols, int64_t contraction, in
     if (p.s2 > p.s1) p.s2 = p.s1;
   }
   p.smem = smem_plan(asrc, tn, p.s1, p.s2, has_ext).total + 1024;
-  // Split the contraction when the output tiles leave CTA slots idle: as many splits
-  // as fit in one wave, at least two steps each.
+  // Persistent CTAs, one per slot, take the tiles in waves. The tiles of a last,
+  // partial wave are cut into contraction slices so that wave is as full as it can
+  // be: as many slices as the idle slots allow, at least four steps each (each slice
+  // costs a partial tile and one more term in the last slice's reduction).
   const int64_t tiles = p.tiles();
   const int64_t slots = static_cast<int64_t>(nsm) * p.ctas_per_sm;
-  // Each split costs its partial tile and one more term in the last CTA's reduction,
-  // so keep at least four steps per split.
+  p.full_tiles = static_cast<int>((tiles / slots) * slots);
+  p.tail_tiles = static_cast<int>(tiles - p.full_tiles);
   int best = 1;
-  if (tiles < slots && p.nsteps > 1) {
+  if (p.tail_tiles > 0 && p.nsteps > 1) {
     const int max_splits = std::max(1, p.nsteps / 4);
-    best = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(max_splits, slots / tiles)));
+    best = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(max_splits, slots / p.tail_tiles)));
   }
-  p.steps_per_split = (p.nsteps + best - 1) / best;
-  p.splits = (p.nsteps + p.steps_per_split - 1) / p.steps_per_split;
+  p.tail_sps = (p.nsteps + best - 1) / best;
+  p.tail_splits = p.tail_sps > 0 ? (p.nsteps + p.tail_sps - 1) / p.tail_sps : 1;
+  p.units = p.full_tiles + p.tail_tiles * p.tail_splits;
+#ifndef QNF4_PERSIST
+#define QNF4_PERSIST 1
+#endif
+  // QNF4_PERSIST=0: one unit per CTA, the hardware scheduler hands out the units
+  p.grid = static_cast<int>(std::max<int64_t>(1, QNF4_PERSIST ? std::min<int64_t>(p.units, slots) : p.units));
   return p;
 }
 
@@ -319,7 +330,7 @@ bool g_smem_set[5][4][3][64] = {};
 
 template <int ASRC, int NSET, int MINB>
 qnf4_status launch_gemm(const GemmPlan& p, const CUtensorMap& a, const CUtensorMap& b,
-                        const CUtensorMap& bx, GemmArgs g, cudaStream_t s) {
+                        const CUtensorMap& bx, const CUtensorMap& o, GemmArgs g, cudaStream_t s) {
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !g_smem_set[ASRC][NSET][MINB][dev]) {
@@ -330,21 +341,28 @@ qnf4_status launch_gemm(const GemmPlan& p, const CUtensorMap& a, const CUtensorM
     g_smem_set[ASRC][NSET][MINB][dev] = true;
   }
   if (p.s1 < 1 || p.s1 > kMaxS1 || p.s2 < 0 || p.s2 > kMaxS2 || p.s2 > p.s1 || p.tn < 16 || p.tn > 256 ||
-      p.tn % 16 || tmem_cols(ASRC, p.tn, p.s2) > (p.ctas_per_sm == 2 ? 256u : 512u))
+      p.tn % 16 || tmem_cols(ASRC, p.tn, p.s2) > (p.ctas_per_sm == 2 ? 256u : 512u) ||
+      (src_deq(ASRC) && NSET > p.s2))
     return fail(QNF4_ERR_ARG, "internal tiling out of range (s1 %d, s2 %d, tn %d)", p.s1, p.s2, p.tn);
   g.rows = p.rows;
   g.cols = p.cols;
   g.nsteps = p.nsteps;
-  g.steps_per_split = p.steps_per_split;
-  g.splits = p.splits;
+  g.row_tiles = p.row_tiles;
+  g.full_tiles = p.full_tiles;
+  g.tail_tiles = p.tail_tiles;
+  g.tail_splits = p.tail_splits;
+  g.tail_sps = p.tail_sps;
+  g.nunits = p.units;
   g.tn = p.tn;
   g.s1 = p.s1;
   g.s2 = p.s2;
   g.has_ext = p.has_ext;
   g.wait_ns = g_wait_ns;
+  if (!p.has_ext) g.stage = 0;  // the staging buffers live in the adapter tile
   cudaLaunchConfig_t cfg;
   std::memset(&cfg, 0, sizeof(cfg));
-  cfg.gridDim = dim3(p.row_tiles, p.col_tiles, p.splits);
+  if (p.units < 1) return QNF4_OK;  // empty D: nothing to compute
+  cfg.gridDim = dim3(p.grid, 1, 1);
   cfg.blockDim = dim3(gemm_threads(NSET), 1, 1);
   cfg.dynamicSmemBytes = p.smem;
   cfg.stream = s;
@@ -353,7 +371,7 @@ qnf4_status launch_gemm(const GemmPlan& p, const CUtensorMap& a, const CUtensorM
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, k_gemm<ASRC, NSET, MINB>, a, b, bx, g);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, k_gemm<ASRC, NSET, MINB>, a, b, bx, o, g);
   if (e != cudaSuccess) {
     g_launches.fetch_add(1, std::memory_order_relaxed);
     cudaGetLastError();
@@ -365,30 +383,32 @@ qnf4_status launch_gemm(const GemmPlan& p, const CUtensorMap& a, const CUtensorM
 // The instantiated (source, converter sets, CTAs per SM) combinations.
 template <int ASRC>
 qnf4_status launch_deq(const GemmPlan& p, const CUtensorMap& a, const CUtensorMap& b,
-                       const CUtensorMap& bx, const GemmArgs& g, cudaStream_t s) {
+                       const CUtensorMap& bx, const CUtensorMap& o, const GemmArgs& g,
+                       cudaStream_t s) {
   const int key = p.nset * 10 + p.ctas_per_sm;
   switch (key) {
-    case 11: return launch_gemm<ASRC, 1, 1>(p, a, b, bx, g, s);
-    case 12: return launch_gemm<ASRC, 1, 2>(p, a, b, bx, g, s);
-    case 21: return launch_gemm<ASRC, 2, 1>(p, a, b, bx, g, s);
-    case 22: return launch_gemm<ASRC, 2, 2>(p, a, b, bx, g, s);
-    case 31: return launch_gemm<ASRC, 3, 1>(p, a, b, bx, g, s);
+    case 11: return launch_gemm<ASRC, 1, 1>(p, a, b, bx, o, g, s);
+    case 12: return launch_gemm<ASRC, 1, 2>(p, a, b, bx, o, g, s);
+    case 21: return launch_gemm<ASRC, 2, 1>(p, a, b, bx, o, g, s);
+    case 22: return launch_gemm<ASRC, 2, 2>(p, a, b, bx, o, g, s);
+    case 31: return launch_gemm<ASRC, 3, 1>(p, a, b, bx, o, g, s);
     default: return fail(QNF4_ERR_ARG, "no kernel for %d converter sets x %d CTAs/SM", p.nset, p.ctas_per_sm);
   }
 }
 
 qnf4_status launch_any(const GemmPlan& p, const CUtensorMap& a, const CUtensorMap& b,
-                       const CUtensorMap& bx, const GemmArgs& g, cudaStream_t s) {
+                       const CUtensorMap& bx, const CUtensorMap& o, const GemmArgs& g,
+                       cudaStream_t s) {
   switch (p.asrc) {
-    case A_NF4_K: return launch_deq<A_NF4_K>(p, a, b, bx, g, s);
-    case A_NF4_MN: return launch_deq<A_NF4_MN>(p, a, b, bx, g, s);
+    case A_NF4_K: return launch_deq<A_NF4_K>(p, a, b, bx, o, g, s);
+    case A_NF4_MN: return launch_deq<A_NF4_MN>(p, a, b, bx, o, g, s);
     case A_DENSE_K:
-      return p.ctas_per_sm == 2 ? launch_gemm<A_DENSE_K, 1, 2>(p, a, b, bx, g, s)
-                                : launch_gemm<A_DENSE_K, 1, 1>(p, a, b, bx, g, s);
+      return p.ctas_per_sm == 2 ? launch_gemm<A_DENSE_K, 1, 2>(p, a, b, bx, o, g, s)
+                                : launch_gemm<A_DENSE_K, 1, 1>(p, a, b, bx, o, g, s);
     case A_DENSE_MN:
-      return p.ctas_per_sm == 2 ? launch_gemm<A_DENSE_MN, 1, 2>(p, a, b, bx, g, s)
-                                : launch_gemm<A_DENSE_MN, 1, 1>(p, a, b, bx, g, s);
-    default: return launch_deq<A_CHANQ_K>(p, a, b, bx, g, s);
+      return p.ctas_per_sm == 2 ? launch_gemm<A_DENSE_MN, 1, 2>(p, a, b, bx, o, g, s)
+                                : launch_gemm<A_DENSE_MN, 1, 1>(p, a, b, bx, o, g, s);
+    default: return launch_deq<A_CHANQ_K>(p, a, b, bx, o, g, s);
   }
 }
 
@@ -414,6 +434,15 @@ struct BaseSrc {
   int64_t N = 0, K = 0;
 };
 
+// Output map of the staged epilogue: bf16 D with rows contiguous (ld elements between
+// columns), stored in boxes of 128 rows x 8 columns. False when the layout does not allow
+// it (row stride not a multiple of 16 bytes); the epilogue then stores element by element.
+bool stage_map(CUtensorMap* m, void* out, int64_t rows, int64_t cols, int64_t ld) {
+  std::memset(m, 0, sizeof(*m));
+  if ((ld * 2) % 16 != 0 || !al16(out)) return false;
+  return make_map(m, out, false, rows, cols, ld, 128, 8, false);
+}
+
 qnf4_status map_fail() { return fail(QNF4_ERR_CUDA, "cuTensorMapEncodeTiled unavailable or refused the layout"); }
 
 // u = x A^T (contraction K), written as bf16(scale u) into up [M, 64] and, when ut is
@@ -432,7 +461,7 @@ qnf4_status run_u(const LinPlan& L, const void* x, const void* A, int64_t M, int
   g.scale = scale;
   g.part = part;
   g.counters = cnt;
-  return launch_any(L.u, ma, mb, none, g, s);
+  return launch_any(L.u, ma, mb, none, none, g, s);
 }
 
 qnf4_status linear_fwd(const BaseSrc& src, const void* x, int64_t M, const void* A, const void* B,
@@ -483,11 +512,13 @@ qnf4_status linear_fwd(const BaseSrc& src, const void* x, int64_t M, const void*
   g.out = h;
   g.o_rs = 1;
   g.o_cs = N;
+  CUtensorMap mo;
+  g.stage = stage_map(&mo, h, N, M, N) ? 1 : 0;
   g.part = part;
   g.counters = cnt;
   g.lazy_dep = 1;  // only the adapter chunk reads what the u kernel writes
   if (g_ev_start) cudaEventRecord(g_ev_start, s);
-  st = launch_any(L.main, ma, mb, mbx, g, s);
+  st = launch_any(L.main, ma, mb, mbx, mo, g, s);
   if (g_ev_stop) cudaEventRecord(g_ev_stop, s);
   return st;
 }
@@ -535,7 +566,7 @@ qnf4_status linear_bwd(const BaseSrc& src, const void* x, const void* dY, int64_
     g.scale = scale;
     g.part = part;
     g.counters = cnt;
-    st = launch_any(L.v, ma, mb, none, g, s);
+    st = launch_any(L.v, ma, mb, none, none, g, s);
     if (st != QNF4_OK) return st;
   }
   // dX = dY W_hat + (scale v) A
@@ -565,10 +596,12 @@ qnf4_status linear_bwd(const BaseSrc& src, const void* x, const void* dY, int64_
     g.out = dX;
     g.o_rs = 1;
     g.o_cs = K;
+    CUtensorMap mo;
+    g.stage = stage_map(&mo, dX, K, M, K) ? 1 : 0;
     g.part = part;
     g.counters = cnt;
     if (g_ev_start) cudaEventRecord(g_ev_start, s);
-    st = launch_any(L.main, ma, mb, mbx, g, s);
+    st = launch_any(L.main, ma, mb, mbx, mo, g, s);
     if (g_ev_stop) cudaEventRecord(g_ev_stop, s);
     if (st != QNF4_OK) return st;
   }
@@ -586,7 +619,7 @@ qnf4_status linear_bwd(const BaseSrc& src, const void* x, const void* dY, int64_
     g.scale = 1.f;
     g.part = part;
     g.counters = cnt;
-    st = launch_any(L.da, ma, mb, none, g, s);
+    st = launch_any(L.da, ma, mb, none, none, g, s);
     if (st != QNF4_OK) return st;
   }
   // dB = dY^T (scale u)  -> [N, r]
@@ -603,7 +636,7 @@ qnf4_status linear_bwd(const BaseSrc& src, const void* x, const void* dY, int64_
     g.scale = 1.f;
     g.part = part;
     g.counters = cnt;
-    st = launch_any(L.db, ma, mb, none, g, s);
+    st = launch_any(L.db, ma, mb, none, none, g, s);
     if (st != QNF4_OK) return st;
   }
   return QNF4_OK;

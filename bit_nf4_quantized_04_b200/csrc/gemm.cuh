@@ -78,8 +78,16 @@ __host__ __device__ inline uint32_t tmem_cols(int asrc, int tn, int s2) {
 struct GemmArgs {
   int64_t rows, cols;     // extents of D
   int nsteps;             // contraction steps of 64 in total
-  int steps_per_split;    // steps per blockIdx.z slice
-  int splits;             // gridDim.z
+  // Work units, taken by CTA b in the order b, b + gridDim.x, ...: units
+  // 0 .. full_tiles-1 are whole tiles (tile t = unit), the following
+  // tail_tiles * tail_splits units are contraction slices of the remaining tiles
+  // (tile full_tiles + v % tail_tiles, slice v / tail_tiles, tail_sps steps each),
+  // reduced by the last slice to finish. Tile t covers row tile t % row_tiles and
+  // column tile t / row_tiles.
+  int row_tiles;
+  int full_tiles;
+  int tail_tiles, tail_splits, tail_sps;
+  int nunits;
   int tn;                 // N tile: multiple of 16, 16..256
   int s1, s2;             // depth of the load ring and of the dequantized-A ring
   int has_ext;            // add the adapter chunk (in split 0)
@@ -109,8 +117,10 @@ struct GemmArgs {
   void* out2;             // EPI_UV: transposed copy, [col][row] with stride o2_ld
   int64_t o2_ld;
   float scale;
-  float* part;            // split-K partial tiles
-  unsigned int* counters; // split-K arrival counters (zero on entry, left zero)
+  int stage;              // EPI_BF16 whole tiles leave through shared memory and the tmO
+                          // tensor map (out rows contiguous, 16-byte row stride, has_ext)
+  float* part;            // partial tiles of the tail slices [tail_tiles][tail_splits][tn][128]
+  unsigned int* counters; // arrival counters per tail tile (zero on entry, left zero)
   unsigned long long wait_ns;
   int lazy_dep;           // programmatic dependent launch: 0 = every thread waits for the
                           // previous grid after the prologue; 1 = only the adapter chunk's
@@ -148,6 +158,19 @@ __host__ __device__ inline SmemPlan smem_plan(int asrc, int tn, int s1, int s2, 
 __device__ unsigned long long g_wait_cycles[64];
 #endif
 
+// Tracing build: clock cycles of a code span, per warp (lane 0), at a wait-stat site.
+#ifdef QNF4_WAIT_STATS
+#define QNF4_TSTAMP(v) const long long v = clock64()
+#define QNF4_TSPAN(site, v)                                                                    \
+  do {                                                                                         \
+    if ((threadIdx.x & 31) == 0)                                                               \
+      atomicAdd(&g_wait_cycles[site], static_cast<unsigned long long>(clock64() - (v)));       \
+  } while (0)
+#else
+#define QNF4_TSTAMP(v)
+#define QNF4_TSPAN(site, v)
+#endif
+
 QNF4_DEV bool wait_or_abort(uint64_t* bar, uint32_t parity, unsigned long long wait_ns,
                             volatile int* abort_flag, unsigned int site) {
   if (mbar_try_wait(bar, parity)) return true;
@@ -173,6 +196,15 @@ QNF4_DEV bool wait_or_abort(uint64_t* bar, uint32_t parity, unsigned long long w
 
 QNF4_DEV void named_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// Barrier of one converter set's 128 threads (ids 3 .. 3 + NSET - 1, immediates so the
+// kernel reserves only the barriers it uses).
+template <int NSET>
+QNF4_DEV void set_sync(int set) {
+  if (NSET == 1 || set == 0) asm volatile("bar.sync 3, 128;" ::: "memory");
+  else if (NSET == 2 || set == 1) asm volatile("bar.sync 4, 128;" ::: "memory");
+  else asm volatile("bar.sync 5, 128;" ::: "memory");
 }
 
 // Write one 128-byte row slot (64 bf16 given as 32 packed words) of a SW128 tile:
@@ -280,16 +312,65 @@ QNF4_DEV void epi_store(const GemmArgs& g, int64_t row, int64_t col0, const floa
   }
 }
 
-// Where a converter set's step i sits in the two rings, advanced without division
-// (NSET < S2 <= S1, so an index wraps at most once per advance): s / ph = load-ring
-// slot and phase of step i, s2 = its A stage, sj / phj = load-ring slot and phase of
-// step i - S2, the last reader of that A stage (valid once i >= S2).
+// One work unit: a tile of D and the contraction steps it covers.
+struct Unit {
+  int64_t row0, col0;  // first row / column of the tile
+  int step0, nst;      // first contraction step and number of steps
+  int z, splits;       // slice index and slices of this tile (1: a whole tile)
+  int pt;              // tail tile index (partials and counter), when splits > 1
+  bool ext;            // the adapter chunk is added here (slice 0)
+};
+
+QNF4_DEV Unit unit_of(const GemmArgs& g, int u) {
+  Unit w;
+  int t;
+  int sps;
+  if (u < g.full_tiles) {
+    t = u;
+    w.z = 0;
+    w.splits = 1;
+    w.pt = 0;
+    sps = g.nsteps;
+  } else {
+    const int v = u - g.full_tiles;
+    w.pt = v % g.tail_tiles;
+    w.z = v / g.tail_tiles;
+    t = g.full_tiles + w.pt;
+    w.splits = g.tail_splits;
+    sps = g.tail_sps;
+  }
+  const int rt = t % g.row_tiles;
+  w.row0 = static_cast<int64_t>(rt) * kRowsTile;
+  w.col0 = static_cast<int64_t>(t / g.row_tiles) * g.tn;
+  w.step0 = w.z * sps;
+  w.nst = max(0, min(g.nsteps - w.step0, sps));
+  w.ext = g.has_ext && w.z == 0;
+  return w;
+}
+
+// Where a converter set's step sits in the two rings, advanced without division
+// (NSET <= S2 <= S1, so an index wraps at most once per advance). Both rings advance
+// once per position, over all units of the CTA: a unit's contraction steps, then its
+// adapter chunk. i = position in the unit, r = ring position, s / ph = load-ring slot
+// and phase, s2 = A stage; sj / phj = load-ring slot and phase of position r - S2,
+// the last user of that A stage (valid once r >= S2): the MMA's release of that slot
+// also releases the stage.
 struct ConvCursor {
-  int i, s, s2, sj;
+  int i, r, s, s2, sj;
   uint32_t ph, phj;
-  QNF4_DEV explicit ConvCursor(int set) : i(set), s(set), s2(set), sj(0), ph(0), phj(0) {}
+  QNF4_DEV ConvCursor(int set, int rbase, int S1, int S2) {
+    i = set;
+    r = rbase + set;
+    s = r % S1;
+    ph = static_cast<uint32_t>(r / S1) & 1u;
+    s2 = r % S2;
+    const int j = r - S2;
+    sj = j >= 0 ? j % S1 : 0;
+    phj = j >= 0 ? (static_cast<uint32_t>(j / S1) & 1u) : 0u;
+  }
   QNF4_DEV void next(int nset, int S1, int S2) {
     i += nset;
+    r += nset;
     s += nset;
     if (s >= S1) {
       s -= S1;
@@ -297,9 +378,9 @@ struct ConvCursor {
     }
     s2 += nset;
     if (s2 >= S2) s2 -= S2;
-    const int j = i - S2;
+    const int j = r - S2;
     if (j >= 0) {
-      if (j < nset) {  // first step with a predecessor: j < nset < S1
+      if (j < nset) {  // first position with a predecessor: j < nset <= S1
         sj = j;
         phj = 0;
       } else {
@@ -313,20 +394,30 @@ struct ConvCursor {
   }
 };
 
+// Converter steps of the next unit staged before the previous unit's epilogue (per
+// CTA, at most S2: those steps wait only for MMAs of earlier units).
+#ifndef QNF4_EPI_AHEAD
+#define QNF4_EPI_AHEAD -1  // -1: one step per converter set
+#endif
+
 // ---------------------------------------------------------------------------
 // the kernel
 // ---------------------------------------------------------------------------
+// Persistent: CTA b runs units b, b + gridDim.x, ... The load and A rings and their
+// phases continue from unit to unit; the accumulator is handed back and forth
+// through acc_bar (MMAs of a unit done) and acc_empty (its epilogue has read TMEM).
 template <int ASRC, int NSET, int MINB>
 __global__ void __launch_bounds__(gemm_threads(NSET), MINB)
     k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-           const __grid_constant__ CUtensorMap tmBx, const GemmArgs g) {
+           const __grid_constant__ CUtensorMap tmBx, const __grid_constant__ CUtensorMap tmO,
+           const GemmArgs g) {
   constexpr bool DEQ = src_deq(ASRC);
   constexpr bool MN = src_mn(ASRC);
   constexpr bool TMA_A = src_tmem_a(ASRC);
   constexpr int NCONV = 128 * NSET;  // converter / epilogue threads
   extern __shared__ uint8_t dsmem[];
   __shared__ __align__(8) uint64_t full1[kMaxS1], empty1[kMaxS1], full2[kMaxS2];
-  __shared__ __align__(8) uint64_t acc_bar, ext_bar, fin_bar;
+  __shared__ __align__(8) uint64_t acc_bar, acc_empty, ext_bar, fin_bar;
   __shared__ uint32_t s_tmem;
   __shared__ volatile int s_abort;
   __shared__ int s_last;
@@ -338,13 +429,8 @@ __global__ void __launch_bounds__(gemm_threads(NSET), MINB)
                                              ~static_cast<uintptr_t>(1023));
   const SmemPlan sp = smem_plan(ASRC, g.tn, g.s1, g.s2, g.has_ext);
   const int S1 = g.s1, S2 = g.s2;
-  const int z = blockIdx.z;
-  const int step0 = z * g.steps_per_split;
-  const int nst = max(0, min(g.nsteps - step0, g.steps_per_split));
-  const bool ext = g.has_ext && z == 0;
-  const int nload = nst + (ext ? 1 : 0);
-  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * kRowsTile;
-  const int64_t col0 = static_cast<int64_t>(blockIdx.y) * g.tn;
+  const int u0 = blockIdx.x;
+  const int ustep = gridDim.x;
   const uint32_t ncols = tmem_cols(ASRC, g.tn, S2);
 #ifdef QNF4_WAIT_STATS
   const long long g_t_start = clock64();
@@ -358,6 +444,7 @@ __global__ void __launch_bounds__(gemm_threads(NSET), MINB)
     }
     for (int i = 0; i < S2; ++i) mbar_init(&full2[i], 128);
     mbar_init(&acc_bar, 1);
+    mbar_init(&acc_empty, NCONV);
     mbar_init(&ext_bar, 128);
     mbar_init(&fin_bar, 1);
     s_abort = 0;
@@ -373,7 +460,8 @@ __global__ void __launch_bounds__(gemm_threads(NSET), MINB)
   if (warp == 0 && lane == 0) {
     if (src_dense(ASRC) || src_packed_tma(ASRC)) tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
-    if (ext) tma_prefetch_desc(&tmBx);
+    if (g.has_ext) tma_prefetch_desc(&tmBx);
+    if (g.stage) tma_prefetch_desc(&tmO);
   }
   __syncthreads();
   tc_fence_after();
@@ -390,36 +478,46 @@ __global__ void __launch_bounds__(gemm_threads(NSET), MINB)
       int issued = 0;
       int s = 0;
       uint32_t ph = 0;
-      int32_t kc = step0 * kStep;
+      bool ok = true, dep = false;
       uint32_t bytes = static_cast<uint32_t>(g.tn) * 128u;
       if (src_dense(ASRC)) bytes += kATile;
       if (src_packed_tma(ASRC)) bytes += kPTile;
-      for (int i = 0; i < nload; ++i) {
-        if (!mbar_try_wait(&empty1[s], ph ^ 1) &&
-            !wait_or_abort(&empty1[s], ph ^ 1, g.wait_ns, &s_abort, 11))
-          break;
-        uint8_t* slot = base + s * sp.slot1;
-        uint64_t* fb = &full1[s];
-        if (i < nst) {
-          mbar_expect_tx(fb, bytes);
-          if (ASRC == A_DENSE_K) tma_load_2d(slot + sp.off_a1, &tmA, fb, kc, (int32_t)row0);
-          if (ASRC == A_DENSE_MN) {
-            tma_load_2d(slot + sp.off_a1, &tmA, fb, (int32_t)row0, kc);
-            tma_load_2d(slot + sp.off_a1 + 8192, &tmA, fb, (int32_t)row0 + 64, kc);
+      for (int u = u0; u < g.nunits && ok; u += ustep) {
+        const Unit w = unit_of(g, u);
+        const int nload = w.nst + (w.ext ? 1 : 0);
+        int32_t kc = w.step0 * kStep;
+        for (int i = 0; i < nload; ++i) {
+          if (!mbar_try_wait(&empty1[s], ph ^ 1) &&
+              !wait_or_abort(&empty1[s], ph ^ 1, g.wait_ns, &s_abort, 11)) {
+            ok = false;
+            break;
           }
-          if (ASRC == A_NF4_K) tma_load_2d(slot + sp.off_p1, &tmA, fb, kc / 2, (int32_t)row0);
-          if (ASRC == A_NF4_MN) tma_load_2d(slot + sp.off_p1, &tmA, fb, (int32_t)(row0 / 2), kc);
-          tma_load_2d(slot + sp.off_b1, &tmB, fb, kc, (int32_t)col0);
-        } else {
-          if (g.lazy_dep) griddep_wait();
-          mbar_expect_tx(fb, static_cast<uint32_t>(g.tn) * 128u);
-          tma_load_2d(slot + sp.off_b1, &tmBx, fb, 0, (int32_t)col0);
-        }
-        issued = i + 1;
-        kc += kStep;
-        if (++s == S1) {
-          s = 0;
-          ph ^= 1;
+          uint8_t* slot = base + s * sp.slot1;
+          uint64_t* fb = &full1[s];
+          if (i < w.nst) {
+            mbar_expect_tx(fb, bytes);
+            if (ASRC == A_DENSE_K) tma_load_2d(slot + sp.off_a1, &tmA, fb, kc, (int32_t)w.row0);
+            if (ASRC == A_DENSE_MN) {
+              tma_load_2d(slot + sp.off_a1, &tmA, fb, (int32_t)w.row0, kc);
+              tma_load_2d(slot + sp.off_a1 + 8192, &tmA, fb, (int32_t)w.row0 + 64, kc);
+            }
+            if (ASRC == A_NF4_K) tma_load_2d(slot + sp.off_p1, &tmA, fb, kc / 2, (int32_t)w.row0);
+            if (ASRC == A_NF4_MN) tma_load_2d(slot + sp.off_p1, &tmA, fb, (int32_t)(w.row0 / 2), kc);
+            tma_load_2d(slot + sp.off_b1, &tmB, fb, kc, (int32_t)w.col0);
+          } else {
+            if (g.lazy_dep && !dep) {
+              griddep_wait();
+              dep = true;
+            }
+            mbar_expect_tx(fb, static_cast<uint32_t>(g.tn) * 128u);
+            tma_load_2d(slot + sp.off_b1, &tmBx, fb, 0, (int32_t)w.col0);
+          }
+          ++issued;
+          kc += kStep;
+          if (++s == S1) {
+            s = 0;
+            ph ^= 1;
+          }
         }
       }
       // Drain: the last copy issued into each slot must land before the CTA exits.
@@ -442,7 +540,7 @@ __global__ void __launch_bounds__(gemm_threads(NSET), MINB)
     // ------------------------------------------------------------ MMA issuer
     // One thread keeps the tensor core fed: the descriptors are built once and only
     // offset per stage, stage indices and phases advance incrementally, and a step
-    // costs one barrier test, four MMAs and one commit (the stage's release).
+    // costs one barrier test, four MMAs and the stage releases.
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16(128, static_cast<uint32_t>(g.tn), MN ? 1u : 0u, 0u);
       const uint64_t bdesc0 = smem_desc(smem_u32(base + sp.off_b1), 16, 1024, kLayoutSW128);
@@ -456,51 +554,76 @@ __global__ void __launch_bounds__(gemm_threads(NSET), MINB)
       bool ok = true;
       int s = 0, s2 = 0;
       uint32_t ph = 0, ph2 = 0;
-      for (int i = 0; i < nst; ++i) {
-        uint64_t* bar = DEQ ? &full2[s2] : &full1[s];
-        const uint32_t pp = DEQ ? ph2 : ph;
-        if (!mbar_try_wait(bar, pp) && !wait_or_abort(bar, pp, g.wait_ns, &s_abort, DEQ ? 22 : 21)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint64_t bd = bdesc0 + static_cast<uint64_t>(static_cast<uint32_t>(s) * b_stride);
-        const uint64_t ad = adesc0 + static_cast<uint64_t>(static_cast<uint32_t>(DEQ ? s2 : s) * a_stride);
-        const uint32_t ta = tmem_a0 + 32u * static_cast<uint32_t>(s2);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
-          if (TMA_A) mma_ts(tmem, ta + 8u * kk, bd + 2u * kk, idesc, acc);
-          else mma_ss(tmem, ad + a_kstep * kk, bd + 2u * kk, idesc, acc);
-        }
-        mma_commit(&empty1[s]);  // frees ring-1 slot s and, S2 steps later, A stage s2
-        if (++s == S1) {
-          s = 0;
-          ph ^= 1;
-        }
-        if (DEQ && ++s2 == S2) {
-          s2 = 0;
-          ph2 ^= 1;
-        }
-      }
-      if (ok && ext) {
-        const int i = nst;
-        const int s = i % S1;
-        if (wait_or_abort(&full1[s], (i / S1) & 1, g.wait_ns, &s_abort, 23) &&
-            wait_or_abort(&ext_bar, 0, g.wait_ns, &s_abort, 24)) {
+      int k = 0, kx = 0;  // units done, adapter chunks done
+      for (int u = u0; u < g.nunits; u += ustep, ++k) {
+        const Unit w = unit_of(g, u);
+        // the previous unit's epilogue must have read the accumulator
+        if (k > 0) {
+          if (!wait_or_abort(&acc_empty, (k - 1) & 1, g.wait_ns, &s_abort, 26)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
+        }
+        for (int i = 0; i < w.nst; ++i) {
+          uint64_t* bar = DEQ ? &full2[s2] : &full1[s];
+          const uint32_t pp = DEQ ? ph2 : ph;
+          if (!mbar_try_wait(bar, pp) && !wait_or_abort(bar, pp, g.wait_ns, &s_abort, DEQ ? 22 : 21)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t bd = bdesc0 + static_cast<uint64_t>(static_cast<uint32_t>(s) * b_stride);
+          const uint64_t ad = adesc0 + static_cast<uint64_t>(static_cast<uint32_t>(DEQ ? s2 : s) * a_stride);
+          const uint32_t ta = tmem_a0 + 32u * static_cast<uint32_t>(s2);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
+            if (TMA_A) mma_ts(tmem, ta + 8u * kk, bd + 2u * kk, idesc, acc);
+            else mma_ss(tmem, ad + a_kstep * kk, bd + 2u * kk, idesc, acc);
+          }
+          // frees load-ring slot s and, for a dequantized A, A stage s2
+          mma_commit(&empty1[s]);
+          if (++s == S1) {
+            s = 0;
+            ph ^= 1;
+          }
+          if (DEQ && ++s2 == S2) {
+            s2 = 0;
+            ph2 ^= 1;
+          }
+        }
+        if (!ok) break;
+        if (w.ext) {
+          // The adapter chunk: one more position of both rings. Its full2 arrival is
+          // bookkeeping only; its B tile and A tile are waited for here.
+          if ((DEQ && !wait_or_abort(&full2[s2], ph2, g.wait_ns, &s_abort, 22)) ||
+              !wait_or_abort(&full1[s], ph, g.wait_ns, &s_abort, 23) ||
+              !wait_or_abort(&ext_bar, kx & 1, g.wait_ns, &s_abort, 24)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t bd = bdesc0 + static_cast<uint64_t>(static_cast<uint32_t>(s) * b_stride);
           const uint32_t aa = smem_u32(base + sp.ext);
-          const uint32_t bb = smem_u32(base + s * sp.slot1 + sp.off_b1);
           for (int kk = 0; kk < g.ext_k16; ++kk) {
             const uint64_t ad = MN ? smem_desc(aa + kk * 2048, 8192, 1024, kLayoutSW128)
                                    : smem_desc(aa + kk * 32, 16, 1024, kLayoutSW128);
-            const uint64_t bd = smem_desc(bb + kk * 32, 16, 1024, kLayoutSW128);
-            mma_ss(tmem, ad, bd, idesc, (nst > 0 || kk > 0) ? 1u : 0u);
+            mma_ss(tmem, ad, bd + 2u * kk, idesc, (w.nst > 0 || kk > 0) ? 1u : 0u);
           }
           mma_commit(&empty1[s]);
+          if (++s == S1) {
+            s = 0;
+            ph ^= 1;
+          }
+          if (DEQ && ++s2 == S2) {
+            s2 = 0;
+            ph2 ^= 1;
+          }
+          ++kx;
         }
+        mma_commit(&acc_bar);
       }
-      mma_commit(&acc_bar);
       // Drain: every MMA of this CTA completes before TMEM and smem are released.
       mma_commit(&fin_bar);
       const uint64_t t0 = globaltimer();
@@ -518,11 +641,15 @@ __global__ void __launch_bounds__(gemm_threads(NSET), MINB)
     const int set = ct >> 7;          // converter set: steps i with i % NSET == set
     const int t = ct & 127;           // row slot 0..127
     const int q = warp & 3;           // TMEM lane quarter this warp may access
-    if (ext && set == 0) {
-      uint32_t w[32];
+    const int lrow = q * 32 + lane;   // the accumulator row (TMEM lane) of this thread
+    bool dead = false;                // a wait of this thread gave up
+
+    // The adapter operand of unit w into the ext tile (converter set 0 only).
+    auto write_ext = [&](const Unit& w) {
+      uint32_t v[32];
       if (!MN) {
         // row slot t = D row (row0 + t): adapter B[row, 0..r), zero padded to 64
-        const int64_t row = row0 + t;
+        const int64_t row = w.row0 + t;
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
           const int j0 = 2 * c;
@@ -531,202 +658,84 @@ __global__ void __launch_bounds__(gemm_threads(NSET), MINB)
             if (j0 < g.ext_r) lo = g.ext_a[row * g.ext_ld + j0];
             if (j0 + 1 < g.ext_r) hi = g.ext_a[row * g.ext_ld + j0 + 1];
           }
-          w[c] = lo | (hi << 16);
+          v[c] = lo | (hi << 16);
         }
       } else {
         // MN-major: row slot t = (atom kb, contraction j); A[j, row0 + 64 kb .. +64)
         const int kb = t >> 6, j = t & 63;
-        const int64_t k0 = row0 + kb * 64;
+        const int64_t k0 = w.row0 + kb * 64;
         if (j < g.ext_r && k0 < g.rows) {
           const uint4* src = reinterpret_cast<const uint4*>(g.ext_a + j * g.ext_ld + k0);
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
-            const uint4 v = src[c];
-            w[4 * c] = v.x; w[4 * c + 1] = v.y; w[4 * c + 2] = v.z; w[4 * c + 3] = v.w;
+            const uint4 x = src[c];
+            v[4 * c] = x.x; v[4 * c + 1] = x.y; v[4 * c + 2] = x.z; v[4 * c + 3] = x.w;
           }
         } else {
 #pragma unroll
-          for (int c = 0; c < 32; ++c) w[c] = 0u;
+          for (int c = 0; c < 32; ++c) v[c] = 0u;
         }
       }
-      store_row_sw128(base + sp.ext, t, w);
+      store_row_sw128(base + sp.ext, t, v);
       fence_proxy_async();
       mbar_arrive(&ext_bar);
-    }
+    };
 
-    if constexpr (ASRC == A_NF4_K || ASRC == A_NF4_MN) {
-      float lv[16];
+    // Epilogue of the k-th unit of this CTA. Every converter thread calls it for the
+    // same units in the same order; it returns false for all of them alike once the
+    // CTA has aborted, so all take the same path through the named barriers.
+    auto epilogue = [&](int u, int k) -> bool {
+      wait_or_abort(&acc_bar, k & 1, g.wait_ns, &s_abort, 41);
+      QNF4_TSTAMP(te0);
+      named_sync(1, NCONV);
+      if (ct == 0) s_last = s_abort ? 0 : 2;
+      named_sync(1, NCONV);
+      const bool have = s_last == 2;
+      named_sync(1, NCONV);
+      QNF4_TSPAN(44, te0);
+      if (!have) return false;
+      tc_fence_after();
+      const Unit w = unit_of(g, u);
+      const int64_t row = w.row0 + lrow;
+      const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16);
+      // the sets split the tile's columns in 16-column chunks
+      const int nchunk = g.tn / 16;
+      if (w.splits == 1 && g.stage) {
+        // 8-column pieces (bf16, [8 columns][128 rows]) through two 2 KB buffers per
+        // set in the adapter tile, which is idle from the unit's last MMA to the next
+        // unit's adapter write; one thread of the set stores each piece by TMA.
+        uint8_t* stg = base + sp.ext + set * 4096;
+        const int npiece = g.tn / 8;
+        int p = set;
+        uint32_t r[8];
+        if (p < npiece) tmem_ld8(taddr + p * 8, r);
+        for (int b = 0; p < npiece; p += NSET, b ^= 1) {
+          tmem_wait_ld();
+          uint32_t v[8];
 #pragma unroll
-      for (int k = 0; k < 16; ++k) lv[k] = s_lv[k];
-      const float mu = *g.mean;
-      // In tensor memory the row slot must be the lane this warp may access.
-      const int slot = TMA_A ? (q * 32 + lane) : t;
-      ConvCursor cur(set);
-      // block index of this slot at step i and its per-step increment
-      int64_t bidx;
-      int64_t bstep;
-      bool rowok;
-      if (ASRC == A_NF4_K) {
-        const int64_t n = row0 + slot;
-        rowok = n < g.wN;
-        bidx = n * g.nbk + step0 + set;
-        bstep = NSET;
-      } else {
-        const int kb = slot >> 6, nr = slot & 63;
-        const int64_t kblk = row0 / 64 + kb;
-        rowok = kblk < g.nbk;
-        bidx = (static_cast<int64_t>(step0 + set) * kStep + nr) * g.nbk + kblk;
-        bstep = static_cast<int64_t>(NSET) * kStep * g.nbk;
-      }
-      const int64_t nb1 = g.wN * g.nbk;
-      // constants of this set's next step, fetched one of its steps ahead
-      int64_t bnext = bidx;
-      bool vnext = rowok && set < nst && bnext < nb1;
-      uint32_t cnext = vnext ? g.code2[bnext] : 0u;
-      float snext = vnext ? __ldg(g.scale2 + (bnext >> 8)) : 0.f;
-      for (; cur.i < nst; cur.next(NSET, S1, S2)) {
-        const int i = cur.i;
-        const int s = cur.s, s2 = cur.s2;
-        const bool valid = vnext;
-        const float ch = valid ? fmaf(e4m3_to_f32(static_cast<uint8_t>(cnext)), snext, mu) : 0.f;
-        bnext += bstep;
-        vnext = rowok && (i + NSET) < nst && bnext < nb1;
-        if (vnext) {
-          cnext = g.code2[bnext];
-          snext = __ldg(g.scale2 + (bnext >> 8));
-        }
-        if (!wait_or_abort(&full1[s], cur.ph, g.wait_ns, &s_abort, 31)) break;
-        // A stage s2 was last read by step i - S2; its commit released load-ring slot
-        // cur.sj in phase cur.phj. Waiting for that phase means the stage is free again.
-        if (i >= S2 && !wait_or_abort(&empty1[cur.sj], cur.phj, g.wait_ns, &s_abort, 32)) break;
-        const uint8_t* pk = base + s * sp.slot1 + sp.off_p1;
-        const uint8_t* src =
-            (ASRC == A_NF4_K) ? pk + slot * 32 : pk + (slot & 63) * 64 + (slot >> 6) * 32;
-        uint32_t o[32];
-        nf4_block_to_bf16(src, ch, lv, o);
-        if (TMA_A) {
-          tc_fence_after();
-          tmem_st32(tmem + (static_cast<uint32_t>(q * 32) << 16) + a_col + 32u * s2, o);
-          tmem_wait_st();
-          tc_fence_before();
-        } else {
-          store_row_sw128(base + sp.ring2 + s2 * sp.slot2, slot, o);
+          for (int j = 0; j < 8; ++j) v[j] = r[j];
+          if (p + NSET < npiece) tmem_ld8(taddr + (p + NSET) * 8, r);  // next piece in flight
+          uint16_t* dst = reinterpret_cast<uint16_t*>(stg + b * 2048) + lrow;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) dst[j * 128] = f2bf(__uint_as_float(v[j]));
           fence_proxy_async();
-        }
-        mbar_arrive(&full2[s2]);
-      }
-    } else if constexpr (ASRC == A_CHANQ_K) {
-      // Row slot = the TMEM lane this warp may access; the row's 2^b mapping values
-      // live in registers (unused entries 0), and each 64-element group's codes are
-      // widened to the 4-bit layout of NF4 so the same register lookup applies.
-      const int slot = q * 32 + lane;
-      const int64_t n = row0 + slot;
-      const bool valid = n < g.wN;
-      uint32_t* s_t1 = reinterpret_cast<uint32_t*>(base + sp.cq);  // 1-bit byte -> nibble word
-      if (set == 0) {
-        for (int e = t; e < 256; e += 128) {
-          uint32_t word = 0;
-#pragma unroll
-          for (int m = 0; m < 4; ++m) {
-            const uint32_t hi = (static_cast<uint32_t>(e) >> (7 - 2 * m)) & 1u;
-            const uint32_t lo = (static_cast<uint32_t>(e) >> (6 - 2 * m)) & 1u;
-            word |= ((hi << 4) | lo) << (8 * m);
+          if (t == 0) bulk_wait_read0();  // the set's previous piece has left buffer b ^ 1
+          set_sync<NSET>(set);
+          if (t == 0) {
+            tma_store_2d(&tmO, stg + b * 2048, static_cast<int32_t>(w.row0),
+                         static_cast<int32_t>(w.col0 + p * 8));
+            bulk_commit();
           }
-          s_t1[e] = word;
         }
-      }
-      named_sync(2, NCONV);  // the table is read by every converter set
-      int bits = 1;
-      const uint8_t* prow = nullptr;
-      float mp[16];
-      {
-        int64_t mo = 0;
-        if (valid) {
-          bits = g.cq_bits[n];
-          prow = g.cq_packed + g.cq_row_off[n];
-          mo = g.cq_map_off[n];
-        }
-        const int nmap = valid ? (1 << bits) : 0;
-#pragma unroll
-        for (int c = 0; c < 16; ++c) mp[c] = c < nmap ? g.cq_map[mo + c] : 0.f;
-      }
-      for (ConvCursor cur(set); cur.i < nst; cur.next(NSET, S1, S2)) {
-        const int i = cur.i;
-        const int s2 = cur.s2;
-        const int gi = step0 + i;
-        // the group's codes and scale (issued before the waits)
-        uint32_t cw[8];
-        float gm = 0.f;
-        if (valid) {
-          gm = __ldg(g.cq_absmax + n * g.nbk + gi);
-          // A row holds K b / 8 bytes (a multiple of 8, not of 16, e.g. K = 448) and a
-          // group 8 b bytes, so only 8-byte loads are aligned for every shape.
-          const uint2* src = reinterpret_cast<const uint2*>(prow + static_cast<int64_t>(gi) * 8 * bits);
-          if (bits == 4) {
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const uint2 a = __ldg(src + k);
-              cw[2 * k] = a.x;
-              cw[2 * k + 1] = a.y;
-            }
-          } else if (bits == 2) {
-            const uint2 a0 = __ldg(src), a1 = __ldg(src + 1);
-            const uint32_t in[4] = {a0.x, a0.y, a1.x, a1.y};
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              // byte x = c0 c1 c2 c3 (2 bits each, first at the top) -> (c0 c1), (c2 c3)
-              const uint32_t w = in[k];
-              const uint32_t hi = ((w >> 2) & 0x30303030u) | ((w >> 4) & 0x03030303u);
-              const uint32_t lo = ((w << 2) & 0x30303030u) | (w & 0x03030303u);
-              cw[2 * k] = __byte_perm(hi, lo, 0x5140);
-              cw[2 * k + 1] = __byte_perm(hi, lo, 0x7362);
-            }
-          } else {
-            const uint2 a = __ldg(src);
-#pragma unroll
-            for (int k = 0; k < 8; ++k) cw[k] = s_t1[((k < 4 ? a.x : a.y) >> (8 * (k & 3))) & 0xFFu];
-          }
-        } else {
-#pragma unroll
-          for (int k = 0; k < 8; ++k) cw[k] = 0u;
-        }
-        if (!wait_or_abort(&full1[cur.s], cur.ph, g.wait_ns, &s_abort, 33)) break;
-        if (i >= S2 && !wait_or_abort(&empty1[cur.sj], cur.phj, g.wait_ns, &s_abort, 34)) break;
-        uint32_t o[32];
-        Nf4Planes P;
-        nf4_planes(mp, gm, P);
-#pragma unroll
-        for (int k = 0; k < 8; ++k) nf4_lookup8(cw[k], P, &o[4 * k]);
-        if (TMA_A) {
-          tc_fence_after();
-          tmem_st32(tmem + (static_cast<uint32_t>(q * 32) << 16) + a_col + 32u * s2, o);
-          tmem_wait_st();
-          tc_fence_before();
-        } else {
-          store_row_sw128(base + sp.ring2 + s2 * sp.slot2, slot, o);
-          fence_proxy_async();
-        }
-        mbar_arrive(&full2[s2]);
-      }
-    }
-
-    // ------------------------------------------------------------ epilogue
-    // The decision to write is taken once, so all converter threads take the same
-    // path through the named barriers below.
-    wait_or_abort(&acc_bar, 0, g.wait_ns, &s_abort, 41);
-    named_sync(1, NCONV);
-    if (ct == 0) s_last = s_abort ? 0 : 2;
-    named_sync(1, NCONV);
-    const bool have = s_last == 2;
-    named_sync(1, NCONV);
-    tc_fence_after();
-    const int rl = q * 32 + lane;
-    const int64_t row = row0 + rl;
-    const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16);
-    // the sets split the tile's columns in 16-column chunks
-    const int nchunk = g.tn / 16;
-    if (have) {
-      if (g.splits == 1) {
+        tc_fence_before();
+        mbar_arrive(&acc_empty);
+        QNF4_TSPAN(42, te0);
+        QNF4_TSTAMP(te1);
+        // the adapter tile is free for its next write once every piece has left it
+        if (t == 0) bulk_wait_read0();
+        named_sync(1, NCONV);
+        QNF4_TSPAN(43, te1);
+      } else if (w.splits == 1) {
         for (int ck = set; ck < nchunk; ck += NSET) {
           const int c0 = ck * 16;
           uint32_t r[16];
@@ -735,58 +744,306 @@ __global__ void __launch_bounds__(gemm_threads(NSET), MINB)
           float v[16];
 #pragma unroll
           for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r[j]);
-          epi_store(g, row, col0 + c0, v, 16);
+          epi_store(g, row, w.col0 + c0, v, 16);
         }
+        tc_fence_before();
+        mbar_arrive(&acc_empty);
       } else {
-        const int64_t tile = static_cast<int64_t>(blockIdx.y) * gridDim.x + blockIdx.x;
         const int64_t tsz = static_cast<int64_t>(g.tn) * 128;
-        float* mine = g.part + (tile * g.splits + z) * tsz;
+        float* mine = g.part + (static_cast<int64_t>(w.pt) * w.splits + w.z) * tsz;
         for (int ck = set; ck < nchunk; ck += NSET) {
           const int c0 = ck * 16;
           uint32_t r[16];
           tmem_ld16(taddr + c0, r);
           tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 16; ++j) __stcg(mine + (c0 + j) * 128 + rl, __uint_as_float(r[j]));
+          for (int j = 0; j < 16; ++j) __stcg(mine + (c0 + j) * 128 + lrow, __uint_as_float(r[j]));
         }
+        tc_fence_before();
+        mbar_arrive(&acc_empty);
         __threadfence();
         named_sync(1, NCONV);
         if (ct == 0) {
-          const unsigned int old = atomicAdd(g.counters + tile, 1u);
-          s_last = (old == static_cast<unsigned int>(g.splits - 1)) ? 1 : 0;
+          const unsigned int old = atomicAdd(g.counters + w.pt, 1u);
+          s_last = (old == static_cast<unsigned int>(w.splits - 1)) ? 1 : 0;
         }
         named_sync(1, NCONV);
         if (s_last) {
           __threadfence();
-          const float* all = g.part + tile * g.splits * tsz;
-          for (int ck = set; ck < nchunk; ck += NSET) {
-            const int c0 = ck * 16;
-            float v[16];
+          const float* all = g.part + static_cast<int64_t>(w.pt) * w.splits * tsz;
+          // 8-column pieces: the next unit's conversion state stays live across the
+          // epilogue, so the reduction keeps few registers
+          for (int ck = set; ck < 2 * nchunk; ck += NSET) {
+            const int c0 = ck * 8;
+            float v[8];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) v[j] = 0.f;
-            // Partials in split order (deterministic), four splits' loads in flight at
-            // a time so the reduction costs one L2 round trip per four splits.
-            for (int zz = 0; zz < g.splits; zz += 4) {
-              float t[4][16];
+            for (int j = 0; j < 8; ++j) v[j] = 0.f;
+            // Partials in slice order (deterministic), four slices' loads in flight
+            // at a time so the reduction costs one L2 round trip per four slices.
+            for (int zz = 0; zz < w.splits; zz += 4) {
+              float tt[4][8];
 #pragma unroll
-              for (int u = 0; u < 4; ++u) {
-                const bool in = zz + u < g.splits;
-                const float* src = all + (zz + u) * tsz + c0 * 128 + rl;
+              for (int uu = 0; uu < 4; ++uu) {
+                const bool in = zz + uu < w.splits;
+                const float* src = all + (zz + uu) * tsz + c0 * 128 + lrow;
 #pragma unroll
-                for (int j = 0; j < 16; ++j) t[u][j] = in ? __ldcg(src + j * 128) : 0.f;
+                for (int j = 0; j < 8; ++j) tt[uu][j] = in ? __ldcg(src + j * 128) : 0.f;
               }
 #pragma unroll
-              for (int u = 0; u < 4; ++u) {
+              for (int uu = 0; uu < 4; ++uu) {
 #pragma unroll
-                for (int j = 0; j < 16; ++j) v[j] += t[u][j];
+                for (int j = 0; j < 8; ++j) v[j] += tt[uu][j];
               }
             }
-            epi_store(g, row, col0 + c0, v, 16);
+            epi_store(g, row, w.col0 + c0, v, 8);
           }
-          if (ct == 0) g.counters[tile] = 0u;
+          if (ct == 0) g.counters[w.pt] = 0u;
         }
       }
+      return true;
+    };
+
+    // Per-source state and one conversion step (A-ring position cur, unit w).
+    // NF4: the 16 levels in registers; block constants fetched one step ahead.
+    float lv[16];
+    float mu = 0.f;
+    const int slot = TMA_A ? lrow : t;  // A row slot (in TMEM: the lane this warp may access)
+    int64_t bnext = 0;
+    bool rowok = false, vnext = false;
+    uint32_t cnext = 0;
+    float snext = 0.f;
+    int64_t bstep = 0;
+    int cn = 0;  // MN-major: contraction index (weight row) of the next step's block
+    // block index of this slot's first step in unit w
+    auto first_block = [&](const Unit& w) -> int64_t {
+      if (ASRC == A_NF4_K) {
+        const int64_t n = w.row0 + slot;
+        rowok = n < g.wN;
+        return n * g.nbk + w.step0 + set;
+      }
+      const int kb = slot >> 6, nr = slot & 63;
+      const int64_t kblk = w.row0 / 64 + kb;
+      rowok = kblk < g.nbk;
+      cn = (w.step0 + set) * kStep + nr;
+      return (static_cast<int64_t>(w.step0 + set) * kStep + nr) * g.nbk + kblk;
+    };
+    // constants of this set's first step in unit un (none past the last unit)
+    auto prefetch_unit = [&](int un) {
+      vnext = false;
+      if (un < g.nunits) {
+        const Unit wn = unit_of(g, un);
+        bnext = first_block(wn);
+        vnext = rowok && set < wn.nst && (ASRC == A_NF4_K || cn < g.wN);
+      }
+      if (vnext) {
+        cnext = g.code2[bnext];
+        snext = __ldg(g.scale2 + (bnext >> 8));
+      }
+    };
+    // per-channel: the row's 2^b mapping values (unused entries 0), codes widened
+    // to the 4-bit layout so the NF4 register lookup applies
+    int cbits = 1;
+    const uint8_t* prow = nullptr;
+    bool cvalid = false;
+    int64_t crow = 0;
+    float mp[16];
+    const uint32_t* s_t1 = reinterpret_cast<const uint32_t*>(base + sp.cq);  // 1-bit byte -> nibble word
+
+    if constexpr (ASRC == A_NF4_K || ASRC == A_NF4_MN) {
+#pragma unroll
+      for (int kq = 0; kq < 16; ++kq) lv[kq] = s_lv[kq];
+      mu = *g.mean;
+      bstep = (ASRC == A_NF4_K) ? static_cast<int64_t>(NSET)
+                                : static_cast<int64_t>(NSET) * kStep * g.nbk;
+      prefetch_unit(u0);
+    } else if constexpr (ASRC == A_CHANQ_K) {
+      if (set == 0) {
+        uint32_t* t1 = reinterpret_cast<uint32_t*>(base + sp.cq);
+        for (int e = t; e < 256; e += 128) {
+          uint32_t word = 0;
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            const uint32_t hi = (static_cast<uint32_t>(e) >> (7 - 2 * m)) & 1u;
+            const uint32_t lo = (static_cast<uint32_t>(e) >> (6 - 2 * m)) & 1u;
+            word |= ((hi << 4) | lo) << (8 * m);
+          }
+          t1[e] = word;
+        }
+      }
+      named_sync(2, NCONV);  // the table is read by every converter set
     }
+
+    // Hand a finished A stage to the MMA.
+    auto publish = [&](const ConvCursor& cur, const uint32_t (&o)[32]) {
+      if (TMA_A) {
+        tc_fence_after();
+        tmem_st32(tmem + (static_cast<uint32_t>(q * 32) << 16) + a_col + 32u * cur.s2, o);
+        tmem_wait_st();
+        tc_fence_before();
+      } else {
+        store_row_sw128(base + sp.ring2 + cur.s2 * sp.slot2, slot, o);
+        fence_proxy_async();
+      }
+      mbar_arrive(&full2[cur.s2]);
+    };
+    // Wait until step cur's packed data has landed and its A stage is free (the MMA
+    // of the position S2 earlier has completed).
+    auto acquire = [&](const ConvCursor& cur, unsigned int site) -> bool {
+      if (!wait_or_abort(&full1[cur.s], cur.ph, g.wait_ns, &s_abort, site)) return false;
+      if (cur.r >= S2 && !wait_or_abort(&empty1[cur.sj], cur.phj, g.wait_ns, &s_abort, site + 1))
+        return false;
+      return true;
+    };
+    // The adapter position writes no A stage, but its full2 arrival must fall in that
+    // stage's next phase: wait for the stage's previous user as a conversion would.
+    auto pass_ext = [&](const ConvCursor& cur) -> bool {
+      if (cur.r >= S2 && !wait_or_abort(&empty1[cur.sj], cur.phj, g.wait_ns, &s_abort, 35))
+        return false;
+      mbar_arrive(&full2[cur.s2]);
+      return true;
+    };
+
+    // One conversion step; false when a wait gave up.
+    auto step = [&](const Unit& w, const ConvCursor& cur, int u) -> bool {
+      if constexpr (ASRC == A_NF4_K || ASRC == A_NF4_MN) {
+        const bool valid = vnext;
+        const float ch = valid ? fmaf(e4m3_to_f32(static_cast<uint8_t>(cnext)), snext, mu) : 0.f;
+        // constants of this set's next step: in this unit, else in the CTA's next unit
+        if (cur.i + NSET < w.nst) {
+          bnext += bstep;
+          cn += NSET * kStep;
+          vnext = rowok && (ASRC == A_NF4_K || cn < g.wN);
+          if (vnext) {
+            cnext = g.code2[bnext];
+            snext = __ldg(g.scale2 + (bnext >> 8));
+          }
+        } else {
+          prefetch_unit(u + ustep);
+        }
+        if (!acquire(cur, 31)) return false;
+        const uint8_t* pk = base + cur.s * sp.slot1 + sp.off_p1;
+        const uint8_t* src =
+            (ASRC == A_NF4_K) ? pk + slot * 32 : pk + (slot & 63) * 64 + (slot >> 6) * 32;
+        uint32_t o[32];
+        nf4_block_to_bf16(src, ch, lv, o);
+        publish(cur, o);
+      } else if constexpr (ASRC == A_CHANQ_K) {
+        const int gi = w.step0 + cur.i;
+        // the group's codes and scale (issued before the waits)
+        uint32_t cw[8];
+        float gm = 0.f;
+        if (cvalid) {
+          gm = __ldg(g.cq_absmax + crow * g.nbk + gi);
+          // A row holds K b / 8 bytes (a multiple of 8, not of 16, e.g. K = 448) and a
+          // group 8 b bytes, so only 8-byte loads are aligned for every shape.
+          const uint2* src = reinterpret_cast<const uint2*>(prow + static_cast<int64_t>(gi) * 8 * cbits);
+          if (cbits == 4) {
+#pragma unroll
+            for (int kq = 0; kq < 4; ++kq) {
+              const uint2 a = __ldg(src + kq);
+              cw[2 * kq] = a.x;
+              cw[2 * kq + 1] = a.y;
+            }
+          } else if (cbits == 2) {
+            const uint2 a0 = __ldg(src), a1 = __ldg(src + 1);
+            const uint32_t in[4] = {a0.x, a0.y, a1.x, a1.y};
+#pragma unroll
+            for (int kq = 0; kq < 4; ++kq) {
+              // byte x = c0 c1 c2 c3 (2 bits each, first at the top) -> (c0 c1), (c2 c3)
+              const uint32_t x = in[kq];
+              const uint32_t hi = ((x >> 2) & 0x30303030u) | ((x >> 4) & 0x03030303u);
+              const uint32_t lo = ((x << 2) & 0x30303030u) | (x & 0x03030303u);
+              cw[2 * kq] = __byte_perm(hi, lo, 0x5140);
+              cw[2 * kq + 1] = __byte_perm(hi, lo, 0x7362);
+            }
+          } else {
+            const uint2 a = __ldg(src);
+#pragma unroll
+            for (int kq = 0; kq < 8; ++kq) cw[kq] = s_t1[((kq < 4 ? a.x : a.y) >> (8 * (kq & 3))) & 0xFFu];
+          }
+        } else {
+#pragma unroll
+          for (int kq = 0; kq < 8; ++kq) cw[kq] = 0u;
+        }
+        if (!acquire(cur, 33)) return false;
+        uint32_t o[32];
+        Nf4Planes P;
+        nf4_planes(mp, gm, P);
+#pragma unroll
+        for (int kq = 0; kq < 8; ++kq) nf4_lookup8(cw[kq], P, &o[4 * kq]);
+        publish(cur, o);
+      }
+      return true;
+    };
+    // per-unit state of the per-channel source: this row's bits, codes and mapping
+    auto unit_rows = [&](const Unit& w) {
+      if constexpr (ASRC == A_CHANQ_K) {
+        crow = w.row0 + slot;
+        cvalid = crow < g.wN;
+        int64_t mo = 0;
+        cbits = 1;
+        if (cvalid) {
+          cbits = g.cq_bits[crow];
+          prow = g.cq_packed + g.cq_row_off[crow];
+          mo = g.cq_map_off[crow];
+        }
+        const int nmap = cvalid ? (1 << cbits) : 0;
+#pragma unroll
+        for (int c = 0; c < 16; ++c) mp[c] = c < nmap ? g.cq_map[mo + c] : 0.f;
+      }
+    };
+
+    // The unit loop. Steps of unit k with i < ahead are converted before the
+    // epilogue of unit k-1 (they wait only for MMAs of earlier units), so the MMA
+    // has work the moment the accumulator is free again.
+    const int ahead = QNF4_EPI_AHEAD >= 0 ? min(QNF4_EPI_AHEAD, S2) : min(NSET, S2);
+    int rbase = 0;  // ring position of the unit's first step
+    int k = 0;
+    bool quit = false;
+    int up = -1;  // the previous unit, while its epilogue is still due
+    for (int u = u0; u < g.nunits; u += ustep, ++k) {
+      const Unit w = unit_of(g, u);
+      if (k == 0 && w.ext && set == 0) write_ext(w);
+      unit_rows(w);
+      if constexpr (ASRC == A_NF4_K || ASRC == A_NF4_MN) {
+        if (set >= w.nst) prefetch_unit(u + ustep);  // no step of this set here
+      }
+      ConvCursor cur(set, rbase, S1, S2);
+      const int nload = w.nst + (w.ext ? 1 : 0);
+      if (up >= 0) {
+        // positions converted before the previous unit's epilogue
+        if (DEQ && !dead) {
+          const int pre = min(ahead, nload);
+          for (; cur.i < pre; cur.next(NSET, S1, S2)) {
+            if (!(cur.i < w.nst ? step(w, cur, u) : pass_ext(cur))) {
+              dead = true;
+              break;
+            }
+          }
+        }
+        const bool more = epilogue(up, k - 1);
+        up = -1;
+        if (!more) {
+          quit = true;
+          break;
+        }
+        if (w.ext && set == 0) write_ext(w);
+      }
+      if (DEQ && !dead) {
+        for (; cur.i < w.nst; cur.next(NSET, S1, S2)) {
+          if (!step(w, cur, u)) {
+            dead = true;
+            break;
+          }
+        }
+        // the adapter position, when it falls to this set
+        if (!dead && cur.i == w.nst && w.ext && !pass_ext(cur)) dead = true;
+      }
+      up = u;
+      rbase += nload;
+    }
+    if (!quit && up >= 0) epilogue(up, k - 1);
+    if (g.stage && t == 0) bulk_wait0();  // the output stores have completed
     tc_fence_before();
   }
 
