@@ -156,6 +156,8 @@ __host__ __device__ inline SmemPlan smem_plan(int asrc, int tn, int s1, int s2, 
 // Tracing build only: clock cycles spent blocked at each wait site (index = site,
 // 0..63), summed over all threads that wait there. Read with qnf4_debug_wait_stats.
 __device__ unsigned long long g_wait_cycles[64];
+// per-CTA partial sums (shared-memory atomics), added to g_wait_cycles once at exit
+__shared__ unsigned long long s_wait_cycles[64];
 #endif
 
 // Tracing build: clock cycles of a code span, per warp (lane 0), at a wait-stat site.
@@ -164,7 +166,7 @@ __device__ unsigned long long g_wait_cycles[64];
 #define QNF4_TSPAN(site, v)                                                                    \
   do {                                                                                         \
     if ((threadIdx.x & 31) == 0)                                                               \
-      atomicAdd(&g_wait_cycles[site], static_cast<unsigned long long>(clock64() - (v)));       \
+      atomicAdd(&s_wait_cycles[site], static_cast<unsigned long long>(clock64() - (v)));       \
   } while (0)
 #else
 #define QNF4_TSTAMP(v)
@@ -179,7 +181,7 @@ QNF4_DEV bool wait_or_abort(uint64_t* bar, uint32_t parity, unsigned long long w
   struct Acc {
     long long c0;
     unsigned int site;
-    QNF4_DEV ~Acc() { atomicAdd(&g_wait_cycles[site & 63], static_cast<unsigned long long>(clock64() - c0)); }
+    QNF4_DEV ~Acc() { atomicAdd(&s_wait_cycles[site & 63], static_cast<unsigned long long>(clock64() - c0)); }
   } acc{c0, site};
 #endif
   const uint64_t t0 = globaltimer();
@@ -452,6 +454,9 @@ __global__ void __launch_bounds__(gemm_threads(NSET), MINB)
     fence_mbar_init();
   }
   if (threadIdx.x < 16) s_lv[threadIdx.x] = g.levels[threadIdx.x];
+#ifdef QNF4_WAIT_STATS
+  if (threadIdx.x < 64) s_wait_cycles[threadIdx.x] = 0;
+#endif
   if (warp == 1) {
     tmem_alloc(&s_tmem, ncols);
     tmem_relinquish();
@@ -1051,10 +1056,14 @@ __global__ void __launch_bounds__(gemm_threads(NSET), MINB)
   if (lane == 0) {
     // per-warp active time: 60 = producer, 61 = MMA, 62 = converters (sum of warps)
     const unsigned int slot = warp == 0 ? 60 : (warp == 1 ? 61 : 62);
-    atomicAdd(&g_wait_cycles[slot], static_cast<unsigned long long>(clock64() - g_t_start));
+    atomicAdd(&s_wait_cycles[slot], static_cast<unsigned long long>(clock64() - g_t_start));
   }
 #endif
   __syncthreads();
+#ifdef QNF4_WAIT_STATS
+  if (threadIdx.x < 64 && s_wait_cycles[threadIdx.x])
+    atomicAdd(&g_wait_cycles[threadIdx.x], s_wait_cycles[threadIdx.x]);
+#endif
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, ncols);
