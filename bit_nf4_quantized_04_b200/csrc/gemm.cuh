@@ -776,31 +776,33 @@ __global__ void __launch_bounds__(gemm_threads(NSET), MINB)
         if (s_last) {
           __threadfence();
           const float* all = g.part + static_cast<int64_t>(w.pt) * w.splits * tsz;
-          // 8-column pieces: the next unit's conversion state stays live across the
-          // epilogue, so the reduction keeps few registers
-          for (int ck = set; ck < 2 * nchunk; ck += NSET) {
-            const int c0 = ck * 8;
-            float v[8];
+          // Pieces of RW columns: in the dequantizing kernels the next unit's conversion
+          // state stays live across the epilogue, so their reduction keeps fewer
+          // registers (8 columns); the dense ones take 16 (half the round trips).
+          constexpr int RW = DEQ ? 8 : 16;
+          for (int ck = set; ck < nchunk * (16 / RW); ck += NSET) {
+            const int c0 = ck * RW;
+            float v[RW];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) v[j] = 0.f;
+            for (int j = 0; j < RW; ++j) v[j] = 0.f;
             // Partials in slice order (deterministic), four slices' loads in flight
             // at a time so the reduction costs one L2 round trip per four slices.
             for (int zz = 0; zz < w.splits; zz += 4) {
-              float tt[4][8];
+              float tt[4][RW];
 #pragma unroll
               for (int uu = 0; uu < 4; ++uu) {
                 const bool in = zz + uu < w.splits;
                 const float* src = all + (zz + uu) * tsz + c0 * 128 + lrow;
 #pragma unroll
-                for (int j = 0; j < 8; ++j) tt[uu][j] = in ? __ldcg(src + j * 128) : 0.f;
+                for (int j = 0; j < RW; ++j) tt[uu][j] = in ? __ldcg(src + j * 128) : 0.f;
               }
 #pragma unroll
               for (int uu = 0; uu < 4; ++uu) {
 #pragma unroll
-                for (int j = 0; j < 8; ++j) v[j] += tt[uu][j];
+                for (int j = 0; j < RW; ++j) v[j] += tt[uu][j];
               }
             }
-            epi_store(g, row, w.col0 + c0, v, 8);
+            epi_store(g, row, w.col0 + c0, v, RW);
           }
           if (ct == 0) g.counters[w.pt] = 0u;
         }
