@@ -182,6 +182,9 @@ constexpr size_t kSmemLimit = 227 * 1024;
 #ifndef QNF4_S2_THIN_TMEM
 #define QNF4_S2_THIN_TMEM 7
 #endif
+#ifndef QNF4_MIN_SPLIT_STEPS
+#define QNF4_MIN_SPLIT_STEPS 4
+#endif
 #ifndef QNF4_NSET_THIN
 #define QNF4_NSET_THIN 1
 #endif
@@ -251,7 +254,7 @@ GemmPlan plan_gemm(int asrc, int64_t rows, int64_t cols, int64_t contraction, in
   p.tail_tiles = static_cast<int>(tiles - p.full_tiles);
   int best = 1;
   if (p.tail_tiles > 0 && p.nsteps > 1) {
-    const int max_splits = std::max(1, p.nsteps / 4);
+    const int max_splits = std::max(1, p.nsteps / QNF4_MIN_SPLIT_STEPS);
     best = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(max_splits, slots / p.tail_tiles)));
   }
   p.tail_sps = (p.nsteps + best - 1) / best;
@@ -546,13 +549,11 @@ qnf4_status linear_bwd(const BaseSrc& src, const void* x, const void* dY, int64_
     qnf4_status st = launched("transpose_b");
     if (st != QNF4_OK) return st;
   }
-  // (scale u)^T for dB
-  qnf4_status st = run_u(L, x, A, M, K, r, scale, nullptr, ut,
-                         reinterpret_cast<float*>(w8 + L.off_upart),
-                         reinterpret_cast<unsigned*>(w8 + L.off_ucnt), s);
-  if (st != QNF4_OK) return st;
+  qnf4_status st = QNF4_OK;
   CUtensorMap none;
   std::memset(&none, 0, sizeof(none));
+  // Order: v and u, then dA and dB while x and dY are still in L2 (both are
+  // HBM-bound), then dX (tensor-bound).
   // v = dY B  ->  vp = bf16(scale v) [M, 64], vt = its transpose [r16, ldm]
   {
     CUtensorMap ma, mb;
@@ -567,6 +568,45 @@ qnf4_status linear_bwd(const BaseSrc& src, const void* x, const void* dY, int64_
     g.part = part;
     g.counters = cnt;
     st = launch_any(L.v, ma, mb, none, none, g, s);
+    if (st != QNF4_OK) return st;
+  }
+  // (scale u)^T for dB
+  st = run_u(L, x, A, M, K, r, scale, nullptr, ut,
+                         reinterpret_cast<float*>(w8 + L.off_upart),
+                         reinterpret_cast<unsigned*>(w8 + L.off_ucnt), s);
+  if (st != QNF4_OK) return st;
+  // dA = (scale v)^T x  -> [r, K]
+  {
+    CUtensorMap ma, mb;
+    if (!make_map(&ma, x, false, K, M, K, 64, 64, true)) return map_fail();
+    if (!make_map(&mb, vt, false, M, L.r16, L.ldm, 64, L.r16, true)) return map_fail();
+    GemmArgs g = base_args();
+    g.epi = EPI_F32;
+    g.out = dA;
+    g.o_rs = 1;
+    g.o_cs = K;
+    g.out_cols = r;
+    g.scale = 1.f;
+    g.part = part;
+    g.counters = cnt;
+    st = launch_any(L.da, ma, mb, none, none, g, s);
+    if (st != QNF4_OK) return st;
+  }
+  // dB = dY^T (scale u)  -> [N, r]
+  {
+    CUtensorMap ma, mb;
+    if (!make_map(&ma, dY, false, N, M, N, 64, 64, true)) return map_fail();
+    if (!make_map(&mb, ut, false, M, L.r16, L.ldm, 64, L.r16, true)) return map_fail();
+    GemmArgs g = base_args();
+    g.epi = EPI_F32;
+    g.out = dB;
+    g.o_rs = r;
+    g.o_cs = 1;
+    g.out_cols = r;
+    g.scale = 1.f;
+    g.part = part;
+    g.counters = cnt;
+    st = launch_any(L.db, ma, mb, none, none, g, s);
     if (st != QNF4_OK) return st;
   }
   // dX = dY W_hat + (scale v) A
@@ -603,40 +643,6 @@ qnf4_status linear_bwd(const BaseSrc& src, const void* x, const void* dY, int64_
     if (g_ev_start) cudaEventRecord(g_ev_start, s);
     st = launch_any(L.main, ma, mb, mbx, mo, g, s);
     if (g_ev_stop) cudaEventRecord(g_ev_stop, s);
-    if (st != QNF4_OK) return st;
-  }
-  // dA = (scale v)^T x  -> [r, K]
-  {
-    CUtensorMap ma, mb;
-    if (!make_map(&ma, x, false, K, M, K, 64, 64, true)) return map_fail();
-    if (!make_map(&mb, vt, false, M, L.r16, L.ldm, 64, L.r16, true)) return map_fail();
-    GemmArgs g = base_args();
-    g.epi = EPI_F32;
-    g.out = dA;
-    g.o_rs = 1;
-    g.o_cs = K;
-    g.out_cols = r;
-    g.scale = 1.f;
-    g.part = part;
-    g.counters = cnt;
-    st = launch_any(L.da, ma, mb, none, none, g, s);
-    if (st != QNF4_OK) return st;
-  }
-  // dB = dY^T (scale u)  -> [N, r]
-  {
-    CUtensorMap ma, mb;
-    if (!make_map(&ma, dY, false, N, M, N, 64, 64, true)) return map_fail();
-    if (!make_map(&mb, ut, false, M, L.r16, L.ldm, 64, L.r16, true)) return map_fail();
-    GemmArgs g = base_args();
-    g.epi = EPI_F32;
-    g.out = dB;
-    g.o_rs = r;
-    g.o_cs = 1;
-    g.out_cols = r;
-    g.scale = 1.f;
-    g.part = part;
-    g.counters = cnt;
-    st = launch_any(L.db, ma, mb, none, none, g, s);
     if (st != QNF4_OK) return st;
   }
   return QNF4_OK;
