@@ -1005,22 +1005,23 @@ __global__ void __launch_bounds__(gemm_threads(NSET), MINB)
     // has work the moment the accumulator is free again.
     const int ahead = QNF4_EPI_AHEAD >= 0 ? min(QNF4_EPI_AHEAD, S2) : min(NSET, S2);
     int rbase = 0;  // ring position of the unit's first step
-    int k = 0;
-    bool quit = false;
-    int up = -1;  // the previous unit, while its epilogue is still due
-    for (int u = u0; u < g.nunits; u += ustep, ++k) {
-      const Unit w = unit_of(g, u);
-      if (k == 0 && w.ext && set == 0) write_ext(w);
-      unit_rows(w);
-      if constexpr (ASRC == A_NF4_K || ASRC == A_NF4_MN) {
-        if (set >= w.nst) prefetch_unit(u + ustep);  // no step of this set here
-      }
-      ConvCursor cur(set, rbase, S1, S2);
-      const int nload = w.nst + (w.ext ? 1 : 0);
-      if (up >= 0) {
+    int up = -1;    // the previous unit, while its epilogue is still due
+    // One pass per unit of this CTA and a last one for the final epilogue; the
+    // epilogue and the adapter write each have a single call site (smaller code).
+    for (int k = 0;; ++k) {
+      const int u = u0 + k * ustep;
+      const bool live = u < g.nunits;  // a unit to convert (else only the last epilogue)
+      // (dense sources have no A ring: the cursor gets a dummy depth)
+      ConvCursor cur(set, rbase, S1, DEQ ? S2 : 1);
+      if (live) {
+        const Unit w = unit_of(g, u);
+        unit_rows(w);
+        if constexpr (ASRC == A_NF4_K || ASRC == A_NF4_MN) {
+          if (set >= w.nst) prefetch_unit(u + ustep);  // no step of this set here
+        }
         // positions converted before the previous unit's epilogue
-        if (DEQ && !dead) {
-          const int pre = min(ahead, nload);
+        if (DEQ && up >= 0 && !dead) {
+          const int pre = min(ahead, w.nst + (w.ext ? 1 : 0));
           for (; cur.i < pre; cur.next(NSET, S1, S2)) {
             if (!(cur.i < w.nst ? step(w, cur, u) : pass_ext(cur))) {
               dead = true;
@@ -1028,14 +1029,16 @@ __global__ void __launch_bounds__(gemm_threads(NSET), MINB)
             }
           }
         }
+      }
+      if (up >= 0) {
         const bool more = epilogue(up, k - 1);
         up = -1;
-        if (!more) {
-          quit = true;
-          break;
-        }
-        if (w.ext && set == 0) write_ext(w);
+        if (!more) break;
       }
+      if (!live) break;
+      const Unit w = unit_of(g, u);  // recomputed: not kept live across the epilogue
+      const int nload = w.nst + (w.ext ? 1 : 0);
+      if (w.ext && set == 0) write_ext(w);
       if (DEQ && !dead) {
         for (; cur.i < w.nst; cur.next(NSET, S1, S2)) {
           if (!step(w, cur, u)) {
@@ -1049,7 +1052,6 @@ __global__ void __launch_bounds__(gemm_threads(NSET), MINB)
       up = u;
       rbase += nload;
     }
-    if (!quit && up >= 0) epilogue(up, k - 1);
     if (g.stage && t == 0) bulk_wait0();  // the output stores have completed
     tc_fence_before();
   }
