@@ -776,10 +776,11 @@ __global__ void __launch_bounds__(gemm_threads(NSET), MINB)
         if (s_last) {
           __threadfence();
           const float* all = g.part + static_cast<int64_t>(w.pt) * w.splits * tsz;
-          // Pieces of RW columns: in the dequantizing kernels the next unit's conversion
-          // state stays live across the epilogue, so their reduction keeps fewer
-          // registers (8 columns); the dense ones take 16 (half the round trips).
-          constexpr int RW = DEQ ? 8 : 16;
+          // Pieces of RW columns: in the wide dequantizing kernels the next unit's
+          // conversion state stays live across the epilogue within a tight register
+          // budget, so their reduction takes 8 columns; the others take 16 (half the
+          // L2 round trips of the last slice).
+          constexpr int RW = (DEQ && NSET > 1) ? 8 : 16;
           for (int ck = set; ck < nchunk * (16 / RW); ck += NSET) {
             const int c0 = ck * RW;
             float v[RW];
