@@ -229,8 +229,14 @@ class Workload:
             x=synth.normal_bf16((CQ_M, CQ_K), 1.0, synth.SEED_X + 50, device=dev),
             A=synth.normal_bf16((RANK, CQ_K), 0.01, synth.SEED_A + 50, device=dev),
             B=synth.normal_bf16((CQ_N, RANK), 0.01, synth.SEED_B + 50, device=dev),
-            h=torch.empty(CQ_M, CQ_N, dtype=torch.bfloat16, device=dev))
-        wsz = max(wsz, q.workspace_size(q._lib.OP_CHANQ_FWD, CQ_N, CQ_K, CQ_M, RANK))
+            h=torch.empty(CQ_M, CQ_N, dtype=torch.bfloat16, device=dev),
+            # backward through the per-channel base (a breakdown row, not in the step)
+            dY=synth.normal_bf16((CQ_M, CQ_N), 1.0, synth.SEED_DY + 50, device=dev),
+            dX=torch.empty(CQ_M, CQ_K, dtype=torch.bfloat16, device=dev),
+            dA=torch.empty(RANK, CQ_K, dtype=torch.float32, device=dev),
+            dB=torch.empty(CQ_N, RANK, dtype=torch.float32, device=dev))
+        wsz = max(wsz, q.workspace_size(q._lib.OP_CHANQ_FWD, CQ_N, CQ_K, CQ_M, RANK),
+                  q.workspace_size(q._lib.OP_CHANQ_BWD, CQ_N, CQ_K, CQ_M, RANK))
         self.ws = torch.empty(wsz, dtype=torch.uint8, device=dev)
 
     # the pieces of one step
@@ -337,6 +343,12 @@ def breakdown(wl, q, hbm, tc_sus):
                                              c["map_off"], c["absmax"], CQ_N, CQ_K, c["x"], c["A"],
                                              c["B"], wl.s, h=c["h"], ws=wl.ws), 5, st)
     out["chanq_fwd"] = {"TFLOPs": round(cf / t / 1e12, 1), "frac_tc": round(cf / t / 1e12 / tc_sus, 3)}
+    cb = bwd_flops(CQ_N, CQ_K, CQ_M, RANK)
+    t = time_loop(lambda: q.chanq_linear_bwd(c["packed"], c["roff"], c["bits"], c["maps"],
+                                             c["map_off"], c["absmax"], CQ_N, CQ_K, c["x"], c["dY"],
+                                             c["A"], c["B"], wl.s, dX=c["dX"], dA=c["dA"],
+                                             dB=c["dB"], ws=wl.ws), 5, st)
+    out["chanq_bwd"] = {"TFLOPs": round(cb / t / 1e12, 1), "frac_tc": round(cb / t / 1e12 / tc_sus, 3)}
     # decode (memory-bound): rotate over weight copies whose total exceeds L2 twice over
     l2 = torch.cuda.get_device_properties(wl.dev).L2_cache_size
     wbytes = sum(L["w"].nbytes() for L in wl.layers)
@@ -538,7 +550,7 @@ def run_case(args):
               q.workspace_size(q._lib.OP_QUANTIZE, N, K))
     ws = torch.empty(wsz, dtype=torch.uint8, device=dev)
     h = torch.empty(m, N, dtype=torch.bfloat16, device=dev)
-    if args.case in ("chanq_quant", "chanq_fwd"):
+    if args.case in ("chanq_quant", "chanq_fwd", "chanq_bwd"):
         # the per-channel 1/2/4-bit layer of the step (11008 x 4096, 2048 tokens)
         bits = synth.chan_bits(CQ_N)
         maps, map_off, thr, thr_off = synth.chan_tables(bits)
@@ -552,10 +564,16 @@ def run_case(args):
         cA = A[:, :CQ_K].contiguous()
         cB = synth.normal_bf16((CQ_N, RANK), 0.01, synth.SEED_B + 50, device=dev)
         ch = torch.empty(CQ_M, CQ_N, dtype=torch.bfloat16, device=dev)
-        cws = torch.empty(q.workspace_size(q._lib.OP_CHANQ_FWD, CQ_N, CQ_K, CQ_M, RANK), dtype=torch.uint8, device=dev)
+        cws = torch.empty(max(q.workspace_size(q._lib.OP_CHANQ_FWD, CQ_N, CQ_K, CQ_M, RANK),
+                              q.workspace_size(q._lib.OP_CHANQ_BWD, CQ_N, CQ_K, CQ_M, RANK)),
+                          dtype=torch.uint8, device=dev)
         q.chanq_quantize(cW, bits, thr, thr_off, roff, packed=cp, absmax=cg)
         if args.case == "chanq_quant":
             fn = lambda: q.chanq_quantize(cW, bits, thr, thr_off, roff, packed=cp, absmax=cg)  # noqa: E731
+        elif args.case == "chanq_bwd":
+            cdY = synth.normal_bf16((CQ_M, CQ_N), 1.0, synth.SEED_DY + 50, device=dev)
+            fn = lambda: q.chanq_linear_bwd(cp, roff, bits, maps, map_off, cg, CQ_N, CQ_K, cx, cdY,  # noqa: E731
+                                            cA, cB, s, ws=cws)
         else:
             fn = lambda: q.chanq_linear_fwd(cp, roff, bits, maps, map_off, cg, CQ_N, CQ_K, cx, cA, cB, s,  # noqa: E731
                                             h=ch, ws=cws)
@@ -614,7 +632,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-breakdown", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
-    ap.add_argument("--case", choices=["fwd", "bwd", "decode", "quant", "chanq_quant", "chanq_fwd"], default=None,
+    ap.add_argument("--case", choices=["fwd", "bwd", "decode", "quant", "chanq_quant", "chanq_fwd", "chanq_bwd"], default=None,
                     help="run one operation on one gate-shaped layer (for ncu captures)")
     args = ap.parse_args()
     if args.case:

@@ -25,7 +25,7 @@ BLOCK2 = 256
 __all__ = [
     "Nf4Weight", "nf4_codebook", "nf4_quantize", "double_quant", "dequant", "quantize_weight",
     "qlora_linear_fwd", "qlora_linear_bwd", "nf4_recon_error", "rank_topk",
-    "dense_linear_fwd", "dense_linear_bwd", "chanq_quantize", "chanq_linear_fwd",
+    "dense_linear_fwd", "dense_linear_bwd", "chanq_quantize", "chanq_linear_fwd", "chanq_linear_bwd",
     "workspace_size", "check", "set_wait_timeout_ns", "Qnf4Error",
 ]
 
@@ -255,6 +255,24 @@ def chanq_linear_fwd(packed, row_off, bits, maps, map_off, absmax, N: int, K: in
               A.data_ptr(), B.data_ptr(), r, float(scale), h.data_ptr(), wsb.data_ptr(),
               wsb.numel(), _stream(x))
     return h
+
+
+def chanq_linear_bwd(packed, row_off, bits, maps, map_off, absmax, N: int, K: int, x, dY, A, B,
+                     scale: float, dX=None, dA=None, dB=None, ws=None):
+    """(dX bf16 [M, K], dA fp32 [r, K], dB fp32 [N, r]) through the frozen per-channel base."""
+    for t, nm in ((x, "x"), (dY, "dY"), (A, "A"), (B, "B")):
+        _req(t, torch.bfloat16, nm)
+    M, r = x.shape[0], A.shape[0]
+    dev = x.device
+    dX = dX if dX is not None else torch.empty(M, K, dtype=torch.bfloat16, device=dev)
+    dA = dA if dA is not None else torch.empty(r, K, dtype=torch.float32, device=dev)
+    dB = dB if dB is not None else torch.empty(N, r, dtype=torch.float32, device=dev)
+    wsb = _ws(workspace_size(_lib.OP_CHANQ_BWD, N, K, M, r), x, ws)
+    _lib.call("qnf4_chanq_linear_bwd", packed.data_ptr(), row_off.data_ptr(), bits.data_ptr(),
+              maps.data_ptr(), map_off.data_ptr(), absmax.data_ptr(), N, K, x.data_ptr(),
+              dY.data_ptr(), M, A.data_ptr(), B.data_ptr(), r, float(scale), dX.data_ptr(),
+              dA.data_ptr(), dB.data_ptr(), wsb.data_ptr(), wsb.numel(), _stream(x))
+    return dX, dA, dB
 
 
 def check(stream: int | None = None) -> None:

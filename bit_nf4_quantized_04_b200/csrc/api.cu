@@ -329,11 +329,12 @@ LinPlan plan_linear(int main_src, int64_t N, int64_t K, int64_t M, int r, bool b
   return L;
 }
 
-bool g_smem_set[5][4][3][64] = {};
+bool g_smem_set[6][4][3][64] = {};
 
 template <int ASRC, int NSET, int MINB>
 qnf4_status launch_gemm(const GemmPlan& p, const CUtensorMap& a, const CUtensorMap& b,
-                        const CUtensorMap& bx, const CUtensorMap& o, GemmArgs g, cudaStream_t s) {
+                        const CUtensorMap& bx, const CUtensorMap& o, const CUtensorMap& t, GemmArgs g,
+                        cudaStream_t s) {
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !g_smem_set[ASRC][NSET][MINB][dev]) {
@@ -374,7 +375,7 @@ qnf4_status launch_gemm(const GemmPlan& p, const CUtensorMap& a, const CUtensorM
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, k_gemm<ASRC, NSET, MINB>, a, b, bx, o, g);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, k_gemm<ASRC, NSET, MINB>, a, b, bx, o, t, g);
   if (e != cudaSuccess) {
     g_launches.fetch_add(1, std::memory_order_relaxed);
     cudaGetLastError();
@@ -386,32 +387,33 @@ qnf4_status launch_gemm(const GemmPlan& p, const CUtensorMap& a, const CUtensorM
 // The instantiated (source, converter sets, CTAs per SM) combinations.
 template <int ASRC>
 qnf4_status launch_deq(const GemmPlan& p, const CUtensorMap& a, const CUtensorMap& b,
-                       const CUtensorMap& bx, const CUtensorMap& o, const GemmArgs& g,
-                       cudaStream_t s) {
+                       const CUtensorMap& bx, const CUtensorMap& o, const CUtensorMap& t,
+                       const GemmArgs& g, cudaStream_t s) {
   const int key = p.nset * 10 + p.ctas_per_sm;
   switch (key) {
-    case 11: return launch_gemm<ASRC, 1, 1>(p, a, b, bx, o, g, s);
-    case 12: return launch_gemm<ASRC, 1, 2>(p, a, b, bx, o, g, s);
-    case 21: return launch_gemm<ASRC, 2, 1>(p, a, b, bx, o, g, s);
-    case 22: return launch_gemm<ASRC, 2, 2>(p, a, b, bx, o, g, s);
-    case 31: return launch_gemm<ASRC, 3, 1>(p, a, b, bx, o, g, s);
+    case 11: return launch_gemm<ASRC, 1, 1>(p, a, b, bx, o, t, g, s);
+    case 12: return launch_gemm<ASRC, 1, 2>(p, a, b, bx, o, t, g, s);
+    case 21: return launch_gemm<ASRC, 2, 1>(p, a, b, bx, o, t, g, s);
+    case 22: return launch_gemm<ASRC, 2, 2>(p, a, b, bx, o, t, g, s);
+    case 31: return launch_gemm<ASRC, 3, 1>(p, a, b, bx, o, t, g, s);
     default: return fail(QNF4_ERR_ARG, "no kernel for %d converter sets x %d CTAs/SM", p.nset, p.ctas_per_sm);
   }
 }
 
 qnf4_status launch_any(const GemmPlan& p, const CUtensorMap& a, const CUtensorMap& b,
-                       const CUtensorMap& bx, const CUtensorMap& o, const GemmArgs& g,
-                       cudaStream_t s) {
+                       const CUtensorMap& bx, const CUtensorMap& o, const CUtensorMap& t,
+                       const GemmArgs& g, cudaStream_t s) {
   switch (p.asrc) {
-    case A_NF4_K: return launch_deq<A_NF4_K>(p, a, b, bx, o, g, s);
-    case A_NF4_MN: return launch_deq<A_NF4_MN>(p, a, b, bx, o, g, s);
+    case A_NF4_K: return launch_deq<A_NF4_K>(p, a, b, bx, o, t, g, s);
+    case A_NF4_MN: return launch_deq<A_NF4_MN>(p, a, b, bx, o, t, g, s);
     case A_DENSE_K:
-      return p.ctas_per_sm == 2 ? launch_gemm<A_DENSE_K, 1, 2>(p, a, b, bx, o, g, s)
-                                : launch_gemm<A_DENSE_K, 1, 1>(p, a, b, bx, o, g, s);
+      return p.ctas_per_sm == 2 ? launch_gemm<A_DENSE_K, 1, 2>(p, a, b, bx, o, t, g, s)
+                                : launch_gemm<A_DENSE_K, 1, 1>(p, a, b, bx, o, t, g, s);
     case A_DENSE_MN:
-      return p.ctas_per_sm == 2 ? launch_gemm<A_DENSE_MN, 1, 2>(p, a, b, bx, o, g, s)
-                                : launch_gemm<A_DENSE_MN, 1, 1>(p, a, b, bx, o, g, s);
-    default: return launch_deq<A_CHANQ_K>(p, a, b, bx, o, g, s);
+      return p.ctas_per_sm == 2 ? launch_gemm<A_DENSE_MN, 1, 2>(p, a, b, bx, o, t, g, s)
+                                : launch_gemm<A_DENSE_MN, 1, 1>(p, a, b, bx, o, t, g, s);
+    case A_CHANQ_MN: return launch_deq<A_CHANQ_MN>(p, a, b, bx, o, t, g, s);
+    default: return launch_deq<A_CHANQ_K>(p, a, b, bx, o, t, g, s);
   }
 }
 
@@ -434,6 +436,10 @@ struct BaseSrc {
   const float* cq_map = nullptr;
   const int64_t* cq_map_off = nullptr;
   const float* cq_absmax = nullptr;
+  // per-channel backward: the codes widened to the NF4 nibble layout [N, K/2] and the
+  // rows' 16-entry tables [N, 16], made in the workspace by k_chanq_widen
+  uint8_t* cq_wide = nullptr;
+  float* cq_tab = nullptr;
   int64_t N = 0, K = 0;
 };
 
@@ -444,6 +450,28 @@ bool stage_map(CUtensorMap* m, void* out, int64_t rows, int64_t cols, int64_t ld
   std::memset(m, 0, sizeof(*m));
   if ((ld * 2) % 16 != 0 || !al16(out)) return false;
   return make_map(m, out, false, rows, cols, ld, 128, 8, false);
+}
+
+// Workspace after the backward's own: the widened codes [N, K/2] and the tables [N, 16].
+size_t chanq_wide_bytes(int64_t N, int64_t K) {
+  return align256(static_cast<size_t>(N) * static_cast<size_t>(K / 2)) +
+         align256(static_cast<size_t>(N) * 16 * sizeof(float));
+}
+
+// 2-D fp32 tensor [outer, inner] (row stride ld elements), no swizzle.
+bool make_map_f32(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint64_t ld,
+                  uint32_t box_in, uint32_t box_out) {
+  std::memset(m, 0, sizeof(*m));
+  EncodeFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {ld * 4};
+  cuuint32_t box[2] = {box_in, box_out};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(ptr), dims, strides,
+                        box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
 }
 
 qnf4_status map_fail() { return fail(QNF4_ERR_CUDA, "cuTensorMapEncodeTiled unavailable or refused the layout"); }
@@ -464,7 +492,7 @@ qnf4_status run_u(const LinPlan& L, const void* x, const void* A, int64_t M, int
   g.scale = scale;
   g.part = part;
   g.counters = cnt;
-  return launch_any(L.u, ma, mb, none, none, g, s);
+  return launch_any(L.u, ma, mb, none, none, none, g, s);
 }
 
 qnf4_status linear_fwd(const BaseSrc& src, const void* x, int64_t M, const void* A, const void* B,
@@ -482,7 +510,8 @@ qnf4_status linear_fwd(const BaseSrc& src, const void* x, int64_t M, const void*
                          reinterpret_cast<float*>(w8 + L.off_upart),
                          reinterpret_cast<unsigned*>(w8 + L.off_ucnt), s);
   if (st != QNF4_OK) return st;
-  CUtensorMap ma, mb, mbx;
+  CUtensorMap ma, mb, mbx, none;
+  std::memset(&none, 0, sizeof(none));
   std::memset(&ma, 0, sizeof(ma));
   const int tn = L.main.tn;
   if (src.kind == A_NF4_K) {
@@ -521,7 +550,7 @@ qnf4_status linear_fwd(const BaseSrc& src, const void* x, int64_t M, const void*
   g.counters = cnt;
   g.lazy_dep = 1;  // only the adapter chunk reads what the u kernel writes
   if (g_ev_start) cudaEventRecord(g_ev_start, s);
-  st = launch_any(L.main, ma, mb, mbx, mo, g, s);
+  st = launch_any(L.main, ma, mb, mbx, mo, none, g, s);
   if (g_ev_stop) cudaEventRecord(g_ev_stop, s);
   return st;
 }
@@ -530,7 +559,8 @@ qnf4_status linear_bwd(const BaseSrc& src, const void* x, const void* dY, int64_
                        const void* B, int r, float scale, void* dX, float* dA, float* dB, void* ws,
                        size_t ws_bytes, cudaStream_t s) {
   const int64_t N = src.N, K = src.K;
-  const int main_src = src.kind == A_NF4_K ? A_NF4_MN : A_DENSE_MN;
+  const int main_src =
+      src.kind == A_NF4_K ? A_NF4_MN : (src.kind == A_CHANQ_K ? A_CHANQ_MN : A_DENSE_MN);
   const LinPlan L = plan_linear(main_src, N, K, M, r, true, num_sms());
   if (!ws || ws_bytes < L.total) return fail(QNF4_ERR_WORKSPACE, "workspace too small (%zu < %zu)", ws_bytes, L.total);
   uint8_t* w8 = static_cast<uint8_t*>(ws);
@@ -567,7 +597,7 @@ qnf4_status linear_bwd(const BaseSrc& src, const void* x, const void* dY, int64_
     g.scale = scale;
     g.part = part;
     g.counters = cnt;
-    st = launch_any(L.v, ma, mb, none, none, g, s);
+    st = launch_any(L.v, ma, mb, none, none, none, g, s);
     if (st != QNF4_OK) return st;
   }
   // (scale u)^T for dB
@@ -589,7 +619,7 @@ qnf4_status linear_bwd(const BaseSrc& src, const void* x, const void* dY, int64_
     g.scale = 1.f;
     g.part = part;
     g.counters = cnt;
-    st = launch_any(L.da, ma, mb, none, none, g, s);
+    st = launch_any(L.da, ma, mb, none, none, none, g, s);
     if (st != QNF4_OK) return st;
   }
   // dB = dY^T (scale u)  -> [N, r]
@@ -606,15 +636,19 @@ qnf4_status linear_bwd(const BaseSrc& src, const void* x, const void* dY, int64_
     g.scale = 1.f;
     g.part = part;
     g.counters = cnt;
-    st = launch_any(L.db, ma, mb, none, none, g, s);
+    st = launch_any(L.db, ma, mb, none, none, none, g, s);
     if (st != QNF4_OK) return st;
   }
   // dX = dY W_hat + (scale v) A
   {
-    CUtensorMap ma, mb, mbx;
+    CUtensorMap ma, mb, mbx, mt;
+    std::memset(&mt, 0, sizeof(mt));
     const int tn = L.main.tn;
     if (main_src == A_NF4_MN) {
       if (!make_map(&ma, src.w->packed, true, K / 2, N, K / 2, 64, 64, false)) return map_fail();
+    } else if (main_src == A_CHANQ_MN) {
+      if (!make_map(&ma, src.cq_wide, true, K / 2, N, K / 2, 64, 64, false)) return map_fail();
+      if (!make_map_f32(&mt, src.cq_tab, 16, N, 16, 16, 64)) return map_fail();
     } else {
       if (!make_map(&ma, src.Wd, false, K, N, K, 64, 64, true)) return map_fail();
     }
@@ -631,6 +665,8 @@ qnf4_status linear_bwd(const BaseSrc& src, const void* x, const void* dY, int64_
       g.code2 = src.w->code2;
       g.scale2 = src.w->scale2;
       g.mean = src.w->mean;
+    } else if (main_src == A_CHANQ_MN) {
+      g.cq_absmax = src.cq_absmax;
     }
     g.epi = EPI_BF16;
     g.out = dX;
@@ -641,7 +677,7 @@ qnf4_status linear_bwd(const BaseSrc& src, const void* x, const void* dY, int64_
     g.part = part;
     g.counters = cnt;
     if (g_ev_start) cudaEventRecord(g_ev_start, s);
-    st = launch_any(L.main, ma, mb, mbx, mo, g, s);
+    st = launch_any(L.main, ma, mb, mbx, mo, mt, g, s);
     if (g_ev_stop) cudaEventRecord(g_ev_stop, s);
     if (st != QNF4_OK) return st;
   }
@@ -757,6 +793,10 @@ size_t qnf4_workspace_size(int32_t op, int64_t N, int64_t K, int64_t M, int32_t 
     case QNF4_OP_FWD: return plan_linear(A_NF4_K, N, K, M, r, false, num_sms()).total;
     case QNF4_OP_BWD: return plan_linear(A_NF4_MN, N, K, M, r, true, num_sms()).total;
     case QNF4_OP_CHANQ_FWD: return plan_linear(A_CHANQ_K, N, K, M, r, false, num_sms()).total;
+    case QNF4_OP_CHANQ_BWD: {
+      const size_t t = plan_linear(A_CHANQ_MN, N, K, M, r, true, num_sms()).total;
+      return t + chanq_wide_bytes(N, K);
+    }
     default: return 0;
   }
 }
@@ -1001,6 +1041,45 @@ qnf4_status qnf4_chanq_linear_fwd(const uint8_t* packed, const int64_t* row_off,
   src.N = N;
   src.K = K;
   return linear_fwd(src, x, M, A, B, r, scale, h, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+qnf4_status qnf4_chanq_linear_bwd(const uint8_t* packed, const int64_t* row_off, const uint8_t* bits,
+                                  const float* map, const int64_t* map_off, const float* absmax,
+                                  int64_t N, int64_t K, const void* x, const void* dY, int64_t M,
+                                  const void* A, const void* B, int32_t r, float scale, void* dX,
+                                  float* dA, float* dB, void* ws, size_t ws_bytes, void* stream) {
+  qnf4_status st = check_linear_args(N, K, M, r, true,
+                                     {packed, row_off, bits, map, map_off, absmax, x, dY, A, B, dX, dA, dB});
+  if (st != QNF4_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (M == 0) {
+    cudaMemsetAsync(dA, 0, sizeof(float) * r * K, s);
+    cudaMemsetAsync(dB, 0, sizeof(float) * r * N, s);
+    return launched("bwd(M=0)", 0);
+  }
+  const size_t own = plan_linear(A_CHANQ_MN, N, K, M, r, true, num_sms()).total;
+  if (!ws || ws_bytes < own + chanq_wide_bytes(N, K))
+    return fail(QNF4_ERR_WORKSPACE, "workspace too small (%zu < %zu)", ws_bytes, own + chanq_wide_bytes(N, K));
+  BaseSrc src;
+  src.kind = A_CHANQ_K;
+  src.cq_packed = packed;
+  src.cq_row_off = row_off;
+  src.cq_bits = bits;
+  src.cq_map = map;
+  src.cq_map_off = map_off;
+  src.cq_absmax = absmax;
+  src.cq_wide = static_cast<uint8_t*>(ws) + own;
+  src.cq_tab = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + own +
+                                        align256(static_cast<size_t>(N) * static_cast<size_t>(K / 2)));
+  src.N = N;
+  src.K = K;
+  {
+    const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((N + 7) / 8, num_sms() * 8)));
+    k_chanq_widen<<<grid, 256, 0, s>>>(packed, row_off, bits, map, map_off, N, K, src.cq_wide, src.cq_tab);
+    st = launched("chanq_widen");
+    if (st != QNF4_OK) return st;
+  }
+  return linear_bwd(src, x, dY, M, A, B, r, scale, dX, dA, dB, ws, own, s);
 }
 
 }  // extern "C"

@@ -161,4 +161,48 @@ __global__ void __launch_bounds__(256) k_chanq_quant(const uint16_t* __restrict_
   }
 }
 
+
+// Widen a per-channel weight into the NF4 storage layout for the transposed
+// (backward dX) GEMM, which reads it like an NF4 weight: row n's codes (bits[n] in
+// {1, 2, 4}, MSB-first at packed + row_off[n]) become 4-bit codes, element 2j in the
+// high nibble of byte j (wide [N, K/2]); its 2^b mapping values become a 16-entry fp32
+// table with the unused entries 0 (tab [N, 16]). One warp per row. Row offsets are
+// multiples of K b / 8, a multiple of 8 bytes, so a 4-bit row's words are aligned.
+__global__ void __launch_bounds__(256) k_chanq_widen(const uint8_t* __restrict__ packed,
+                                                     const int64_t* __restrict__ row_off,
+                                                     const uint8_t* __restrict__ bits,
+                                                     const float* __restrict__ map,
+                                                     const int64_t* __restrict__ map_off, int64_t N,
+                                                     int64_t K, uint8_t* __restrict__ wide,
+                                                     float* __restrict__ tab) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  for (int64_t n = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; n < N;
+       n += warps) {
+    const int b = bits[n];
+    const uint8_t* src = packed + row_off[n];
+    uint32_t* dst = reinterpret_cast<uint32_t*>(wide + n * (K / 2));
+    for (int64_t wi = lane; wi < K / 8; wi += 32) {  // one output word = 8 codes
+      uint32_t word = 0;
+      if (b == 4) {
+        word = *reinterpret_cast<const uint32_t*>(src + 4 * wi);
+      } else {
+        // code k of the 8 at bit (w - b (k + 1)) of the big-endian field of width w
+        const uint32_t x = b == 2 ? ((static_cast<uint32_t>(src[2 * wi]) << 8) | src[2 * wi + 1])
+                                  : static_cast<uint32_t>(src[wi]);
+        const int w = 8 * b;
+        const uint32_t m = (1u << b) - 1u;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint32_t hi = (x >> (w - b * (2 * j + 1))) & m;
+          const uint32_t lo = (x >> (w - b * (2 * j + 2))) & m;
+          word |= ((hi << 4) | lo) << (8 * j);
+        }
+      }
+      dst[wi] = word;
+    }
+    if (lane < 16) tab[n * 16 + lane] = lane < (1 << b) ? map[map_off[n] + lane] : 0.f;
+  }
+}
+
 }  // namespace qnf4

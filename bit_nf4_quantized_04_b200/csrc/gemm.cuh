@@ -18,6 +18,9 @@
 //   A_DENSE_MN bf16 matrix by TMA, MN-major (dense dX, x^T for dA, dY^T for dB).
 //   A_CHANQ_K  per-output-channel 1/2/4-bit codes with per-row mapping tables,
 //              widened to the 4-bit layout and looked up like NF4 (A in tensor memory).
+//   A_CHANQ_MN the same weight read transposed (backward dX), from codes widened to
+//              the NF4 nibble layout beforehand: TMA brings each step's code tile and
+//              its 64 rows' 16-entry tables; the converters look up like A_NF4_MN.
 //
 // The extra chunk adds sum_j Aext[row, j] * Bext[col, j] over j < r into the same
 // TMEM accumulator: the rank-r adapter term of "QLoRA: Efficient Finetuning of
@@ -36,7 +39,7 @@
 
 namespace qnf4 {
 
-enum : int { A_NF4_K = 0, A_NF4_MN = 1, A_DENSE_K = 2, A_DENSE_MN = 3, A_CHANQ_K = 4 };
+enum : int { A_NF4_K = 0, A_NF4_MN = 1, A_DENSE_K = 2, A_DENSE_MN = 3, A_CHANQ_K = 4, A_CHANQ_MN = 5 };
 enum : int { EPI_BF16 = 0, EPI_F32 = 1, EPI_UV = 2 };
 
 constexpr int kRowsTile = 128;
@@ -47,11 +50,18 @@ constexpr int kMaxS1 = 16;
 constexpr int kMaxS2 = 8;
 
 __host__ __device__ constexpr bool src_deq(int a) {
-  return a == A_NF4_K || a == A_NF4_MN || a == A_CHANQ_K;
+  return a == A_NF4_K || a == A_NF4_MN || a == A_CHANQ_K || a == A_CHANQ_MN;
 }
-__host__ __device__ constexpr bool src_mn(int a) { return a == A_NF4_MN || a == A_DENSE_MN; }
+__host__ __device__ constexpr bool src_mn(int a) {
+  return a == A_NF4_MN || a == A_DENSE_MN || a == A_CHANQ_MN;
+}
 __host__ __device__ constexpr bool src_dense(int a) { return a == A_DENSE_K || a == A_DENSE_MN; }
-__host__ __device__ constexpr bool src_packed_tma(int a) { return a == A_NF4_K || a == A_NF4_MN; }
+__host__ __device__ constexpr bool src_packed_tma(int a) {
+  return a == A_NF4_K || a == A_NF4_MN || a == A_CHANQ_MN;
+}
+// a per-step tile of 64 rows' 16-entry fp32 mapping tables (4 KB) rides in the load ring
+__host__ __device__ constexpr bool src_table_tma(int a) { return a == A_CHANQ_MN; }
+constexpr uint32_t kTTile = 64u * 16u * 4u;
 // A operand staged in tensor memory (written by tcgen05.st) instead of shared memory
 #ifndef QNF4_NF4K_TMEM_A
 #define QNF4_NF4K_TMEM_A 1
@@ -128,7 +138,7 @@ struct GemmArgs {
 };
 
 struct SmemPlan {
-  uint32_t off_a1, off_b1, off_p1, slot1, slot2, ring2, ext, cq, total;
+  uint32_t off_a1, off_b1, off_p1, off_t1, slot1, slot2, ring2, ext, cq, total;
 };
 
 __host__ __device__ inline SmemPlan smem_plan(int asrc, int tn, int s1, int s2, int has_ext) {
@@ -140,6 +150,8 @@ __host__ __device__ inline SmemPlan smem_plan(int asrc, int tn, int s1, int s2, 
   o += static_cast<uint32_t>(tn) * 128u;
   p.off_p1 = o;
   if (src_packed_tma(asrc)) o += kPTile;
+  p.off_t1 = o;
+  if (src_table_tma(asrc)) o += kTTile;
   p.slot1 = (o + 1023u) & ~1023u;
   p.slot2 = (src_deq(asrc) && !src_tmem_a(asrc)) ? kATile : 0u;
   p.ring2 = static_cast<uint32_t>(s1) * p.slot1;
@@ -412,6 +424,7 @@ template <int ASRC, int NSET, int MINB>
 __global__ void __launch_bounds__(gemm_threads(NSET), MINB)
     k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
            const __grid_constant__ CUtensorMap tmBx, const __grid_constant__ CUtensorMap tmO,
+           const __grid_constant__ CUtensorMap tmT,
            const GemmArgs g) {
   constexpr bool DEQ = src_deq(ASRC);
   constexpr bool MN = src_mn(ASRC);
@@ -467,6 +480,7 @@ __global__ void __launch_bounds__(gemm_threads(NSET), MINB)
     tma_prefetch_desc(&tmB);
     if (g.has_ext) tma_prefetch_desc(&tmBx);
     if (g.stage) tma_prefetch_desc(&tmO);
+    if (src_table_tma(ASRC)) tma_prefetch_desc(&tmT);
   }
   __syncthreads();
   tc_fence_after();
@@ -487,6 +501,7 @@ __global__ void __launch_bounds__(gemm_threads(NSET), MINB)
       uint32_t bytes = static_cast<uint32_t>(g.tn) * 128u;
       if (src_dense(ASRC)) bytes += kATile;
       if (src_packed_tma(ASRC)) bytes += kPTile;
+      if (src_table_tma(ASRC)) bytes += kTTile;
       for (int u = u0; u < g.nunits && ok; u += ustep) {
         const Unit w = unit_of(g, u);
         const int nload = w.nst + (w.ext ? 1 : 0);
@@ -507,7 +522,10 @@ __global__ void __launch_bounds__(gemm_threads(NSET), MINB)
               tma_load_2d(slot + sp.off_a1 + 8192, &tmA, fb, (int32_t)w.row0 + 64, kc);
             }
             if (ASRC == A_NF4_K) tma_load_2d(slot + sp.off_p1, &tmA, fb, kc / 2, (int32_t)w.row0);
-            if (ASRC == A_NF4_MN) tma_load_2d(slot + sp.off_p1, &tmA, fb, (int32_t)(w.row0 / 2), kc);
+            if (ASRC == A_NF4_MN || ASRC == A_CHANQ_MN)
+              tma_load_2d(slot + sp.off_p1, &tmA, fb, (int32_t)(w.row0 / 2), kc);
+            // the tables of this step's 64 contraction rows
+            if (ASRC == A_CHANQ_MN) tma_load_2d(slot + sp.off_t1, &tmT, fb, 0, kc);
             tma_load_2d(slot + sp.off_b1, &tmB, fb, kc, (int32_t)w.col0);
           } else {
             if (g.lazy_dep && !dep) {
@@ -844,8 +862,12 @@ __global__ void __launch_bounds__(gemm_threads(NSET), MINB)
         vnext = rowok && set < wn.nst && (ASRC == A_NF4_K || cn < g.wN);
       }
       if (vnext) {
-        cnext = g.code2[bnext];
-        snext = __ldg(g.scale2 + (bnext >> 8));
+        if (ASRC == A_CHANQ_MN) {
+          snext = __ldg(g.cq_absmax + bnext);  // the group's absmax is its constant
+        } else {
+          cnext = g.code2[bnext];
+          snext = __ldg(g.scale2 + (bnext >> 8));
+        }
       }
     };
     // per-channel: the row's 2^b mapping values (unused entries 0), codes widened
@@ -863,6 +885,9 @@ __global__ void __launch_bounds__(gemm_threads(NSET), MINB)
       mu = *g.mean;
       bstep = (ASRC == A_NF4_K) ? static_cast<int64_t>(NSET)
                                 : static_cast<int64_t>(NSET) * kStep * g.nbk;
+      prefetch_unit(u0);
+    } else if constexpr (ASRC == A_CHANQ_MN) {
+      bstep = static_cast<int64_t>(NSET) * kStep * g.nbk;
       prefetch_unit(u0);
     } else if constexpr (ASRC == A_CHANQ_K) {
       if (set == 0) {
@@ -913,17 +938,23 @@ __global__ void __launch_bounds__(gemm_threads(NSET), MINB)
 
     // One conversion step; false when a wait gave up.
     auto step = [&](const Unit& w, const ConvCursor& cur, int u) -> bool {
-      if constexpr (ASRC == A_NF4_K || ASRC == A_NF4_MN) {
+      if constexpr (ASRC == A_NF4_K || ASRC == A_NF4_MN || ASRC == A_CHANQ_MN) {
         const bool valid = vnext;
-        const float ch = valid ? fmaf(e4m3_to_f32(static_cast<uint8_t>(cnext)), snext, mu) : 0.f;
+        const float ch = !valid ? 0.f
+                         : (ASRC == A_CHANQ_MN ? snext
+                                               : fmaf(e4m3_to_f32(static_cast<uint8_t>(cnext)), snext, mu));
         // constants of this set's next step: in this unit, else in the CTA's next unit
         if (cur.i + NSET < w.nst) {
           bnext += bstep;
           cn += NSET * kStep;
           vnext = rowok && (ASRC == A_NF4_K || cn < g.wN);
           if (vnext) {
-            cnext = g.code2[bnext];
-            snext = __ldg(g.scale2 + (bnext >> 8));
+            if (ASRC == A_CHANQ_MN) {
+              snext = __ldg(g.cq_absmax + bnext);
+            } else {
+              cnext = g.code2[bnext];
+              snext = __ldg(g.scale2 + (bnext >> 8));
+            }
           }
         } else {
           prefetch_unit(u + ustep);
@@ -933,7 +964,21 @@ __global__ void __launch_bounds__(gemm_threads(NSET), MINB)
         const uint8_t* src =
             (ASRC == A_NF4_K) ? pk + slot * 32 : pk + (slot & 63) * 64 + (slot >> 6) * 32;
         uint32_t o[32];
-        nf4_block_to_bf16(src, ch, lv, o);
+        if constexpr (ASRC == A_CHANQ_MN) {
+          // this step's contraction row (slot & 63): its 16 mapping values from the
+          // table tile that came with the codes (unused entries 0)
+          const float4* tb = reinterpret_cast<const float4*>(base + cur.s * sp.slot1 + sp.off_t1 +
+                                                             (slot & 63) * 64);
+          float tv[16];
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const float4 f = tb[q4];
+            tv[4 * q4] = f.x; tv[4 * q4 + 1] = f.y; tv[4 * q4 + 2] = f.z; tv[4 * q4 + 3] = f.w;
+          }
+          nf4_block_to_bf16(src, ch, tv, o);
+        } else {
+          nf4_block_to_bf16(src, ch, lv, o);
+        }
         publish(cur, o);
       } else if constexpr (ASRC == A_CHANQ_K) {
         const int gi = w.step0 + cur.i;
@@ -1017,7 +1062,7 @@ __global__ void __launch_bounds__(gemm_threads(NSET), MINB)
       if (live) {
         const Unit w = unit_of(g, u);
         unit_rows(w);
-        if constexpr (ASRC == A_NF4_K || ASRC == A_NF4_MN) {
+        if constexpr (ASRC == A_NF4_K || ASRC == A_NF4_MN || ASRC == A_CHANQ_MN) {
           if (set >= w.nst) prefetch_unit(u + ustep);  // no step of this set here
         }
         // positions converted before the previous unit's epilogue

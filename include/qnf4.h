@@ -68,7 +68,8 @@ enum {
   QNF4_OP_DOUBLE_QUANT = 1, /* qnf4_double_quant                                    */
   QNF4_OP_FWD = 2,          /* qnf4_qlora_linear_fwd, qnf4_dense_linear_fwd          */
   QNF4_OP_BWD = 3,          /* qnf4_qlora_linear_bwd, qnf4_dense_linear_bwd          */
-  QNF4_OP_CHANQ_FWD = 4     /* qnf4_chanq_linear_fwd                                 */
+  QNF4_OP_CHANQ_FWD = 4,    /* qnf4_chanq_linear_fwd                                 */
+  QNF4_OP_CHANQ_BWD = 5     /* qnf4_chanq_linear_bwd                                 */
 };
 
 /* A double-quantized NF4 weight [QLoRA 贡献一/贡献二]. All pointers are device
@@ -212,6 +213,24 @@ QNF4_API qnf4_status qnf4_chanq_linear_fwd(const uint8_t* packed, const int64_t*
                                   const float* absmax, int64_t N, int64_t K, const void* x,
                                   int64_t M, const void* A, const void* B, int32_t r, float scale,
                                   void* h, void* ws, size_t ws_bytes, void* stream);
+
+/* [LowRA §3 (the per-channel dequantization used in fine-tuning), QLoRA's
+ * backward through the frozen base] Backward of the linear layer over a per-channel
+ * quantized base (the same inputs as qnf4_chanq_linear_fwd, plus dY [M, N] bf16):
+ *   v  = dY B,
+ *   dX = dY bf16(w_hat) + scale v A        bf16 [M, K]
+ *   dA = scale v^T x                       fp32 [r, K]
+ *   dB = scale dY^T (x A^T)                fp32 [N, r]
+ * with w_hat as in qnf4_chanq_linear_fwd; no gradient for the frozen base. N must be
+ * a multiple of 8. The workspace (qnf4_workspace_size with QNF4_OP_CHANQ_BWD) also
+ * holds the codes widened to 4 bits and the rows' 16-entry tables, rebuilt each call.
+ * dA and dB are written, not accumulated; M = 0 writes them as zeros. */
+QNF4_API qnf4_status qnf4_chanq_linear_bwd(const uint8_t* packed, const int64_t* row_off,
+                                  const uint8_t* bits, const float* map, const int64_t* map_off,
+                                  const float* absmax, int64_t N, int64_t K, const void* x,
+                                  const void* dY, int64_t M, const void* A, const void* B,
+                                  int32_t r, float scale, void* dX, float* dA, float* dB,
+                                  void* ws, size_t ws_bytes, void* stream);
 
 /* Bytes of device workspace an operation needs for these sizes (0 if none). */
 QNF4_API size_t qnf4_workspace_size(int32_t op, int64_t N, int64_t K, int64_t M, int32_t r);

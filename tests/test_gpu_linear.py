@@ -219,3 +219,64 @@ def test_chanq_linear_fwd(q, N, K, M, r):
     h = q.chanq_linear_fwd(dev(pk), roff.cuda(), bits.cuda(), maps.cuda(), map_off.cuda(),
                            dev(g), N, K, x.cuda(), A.cuda(), B.cuda(), s)
     assert_close(f64(h.cpu()), href, "chanq h")
+
+
+@pytest.mark.parametrize("N,K,M,r", [
+    (40, 128, 5, 8),        # thin token tile, one row tile
+    (200, 448, 70, 16),     # ragged N, K = 448 (7 groups, rows of 56 b bytes)
+    (1104, 4096, 260, 16),  # two token tiles, contraction slices on the last wave
+    (512, 8192, 600, 24),   # more tiles than CTAs: several units per CTA
+])
+def test_chanq_linear_bwd(q, N, K, M, r):
+    # dX = dY w_hat + s v A, dA = s v^T x, dB = s dY^T (x A^T) against the float64 oracle on
+    # the oracle's dequantized per-channel weight
+    W, bits, maps, map_off, thr, thr_off, roff = _chanq_case(N, K, 900 + N)
+    packed, roff_o, g, _ = chanq_oracle(W, bits, thr, thr_off)
+    x = synth.normal_bf16((M, K), 1.0, 81)
+    A = synth.normal_bf16((r, K), 0.01, 82)
+    B = synth.normal_bf16((N, r), 0.01, 83)
+    dY = synth.normal_bf16((M, N), 1.0, 84)
+    s = 16.0 / r
+    wh = ochq.dequant(packed, roff_o, bits.numpy(), maps.numpy(), map_off.numpy(), g, N, K)
+    rdX, rdA, rdB = olin.backward(f64(x), f64(dY), olin.base_bf16(wh), f64(A), f64(B), s)
+    pk = np.zeros(max(packed.size, 16), np.uint8)
+    pk[: packed.size] = packed
+    dX, dA, dB = q.chanq_linear_bwd(dev(pk), roff.cuda(), bits.cuda(), maps.cuda(), map_off.cuda(),
+                                    dev(g), N, K, x.cuda(), dY.cuda(), A.cuda(), B.cuda(), s)
+    assert_close(f64(dX.cpu()), rdX, "chanq dX")
+    assert_close(dA.cpu().double().numpy(), rdA, "chanq dA")
+    assert_close(dB.cpu().double().numpy(), rdB, "chanq dB")
+
+
+def test_chanq_linear_bwd_matches_nf4_special_case(q):
+    # 4-bit rows with the NF4 levels as every row's map and each group's absmax as its
+    # scale give a single-level NF4 weight; the per-channel backward must then agree with
+    # the dense backward on that weight dequantized by the oracle
+    N, K, M, r = 256, 512, 130, 8
+    W = synth.llama_weight((N, K), 95, std=0.02)
+    from oracle import nf4 as onf4
+    lv = onf4.codebook().astype(np.float32)
+    bits = torch.full((N,), 4, dtype=torch.uint8)
+    thr_row = np.nextafter(onf4.thresholds().astype(np.float32), np.float32(-2), dtype=np.float32)
+    thr = torch.from_numpy(np.tile(thr_row, N).astype(np.float32))
+    thr_off = torch.arange(0, 15 * N + 1, 15, dtype=torch.int64)
+    maps = torch.from_numpy(np.tile(lv, N).astype(np.float32))
+    map_off = torch.arange(0, 16 * N + 1, 16, dtype=torch.int64)
+    roff = torch.from_numpy(ochq.row_offsets(bits.numpy(), K))
+    packed, roff_o, g, _ = chanq_oracle(W, bits, thr, thr_off)
+    wh = ochq.dequant(packed, roff_o, bits.numpy(), maps.numpy(), map_off.numpy(), g, N, K)
+    Wd = torch.from_numpy(olin.base_bf16(wh).astype(np.float32)).to(torch.bfloat16)
+    x = synth.normal_bf16((M, K), 1.0, 96)
+    A = synth.normal_bf16((r, K), 0.01, 97)
+    B = synth.normal_bf16((N, r), 0.01, 98)
+    dY = synth.normal_bf16((M, N), 1.0, 99)
+    pk = np.zeros(max(packed.size, 16), np.uint8)
+    pk[: packed.size] = packed
+    got = q.chanq_linear_bwd(dev(pk), roff.cuda(), bits.cuda(), maps.cuda(), map_off.cuda(), dev(g),
+                             N, K, x.cuda(), dY.cuda(), A.cuda(), B.cuda(), 2.0)
+    ref = q.dense_linear_bwd(Wd.cuda(), x.cuda(), dY.cuda(), A.cuda(), B.cuda(), 2.0)
+    torch.cuda.synchronize()
+    # same bf16 weight, same kernels downstream of the operand: identical results
+    for a, b, nm in zip(got, ref, ("dX", "dA", "dB")):
+        assert torch.equal(a, b), nm
+
