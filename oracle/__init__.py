@@ -20,11 +20,12 @@ CDF. Sources, cited by page title and section:
     blocks of the flattened weight.
   * "LowRA" article (cloud.tencent.com.cn), §4.1 (per-output-channel quantization,
     64-element absmax group normalisation, thresholds = bin edges, mappings =
-    representative values, Fig. 3).
+    representative values, Fig. 3), 第五部分 (weighted Lloyd-Max learner of the
+    mappings and thresholds).
 
 Parity status of each function is listed in its docstring. Conventions the pages
 leave open (tail probability of the NF4 grid, nibble order, tie rules, the 8-bit
 float format for double quantization) are self-consistent readings and marked
 "parity unpinned" where no page fixes them.
 """
-from . import numerics, nf4, linear, chanq, rank  # noqa: F401
+from . import numerics, nf4, linear, chanq, rank, lloyd  # noqa: F401
