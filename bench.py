@@ -314,6 +314,19 @@ def time_loop(fn, iters, stream):
     return s.elapsed_time(e) / 1e3 / iters
 
 
+def lloyd_t0(bits: int):
+    """Initial thresholds of the learner: 0.0 for 1 bit, the NormalFloat midpoints for
+    2 and 4 bits (the page's initialisation), from the library's host-side codebook for
+    4 bits and fixed values for 2 bits."""
+    if bits == 1:
+        return [0.0]
+    if bits == 2:
+        return [-0.5, 0.21790908, 0.7179091]
+    import bit_nf4_quantized_04_b200 as q
+    lv = q.nf4_codebook()[0]
+    return [float((float(lv[k]) + float(lv[k + 1])) * 0.5) for k in range(15)]
+
+
 def breakdown(wl, q, hbm, tc_sus):
     """Per-row throughput, each timed alone (short loops, L2-exceeding inputs)."""
     st = torch.cuda.current_stream()
@@ -349,6 +362,13 @@ def breakdown(wl, q, hbm, tc_sus):
                                              c["A"], c["B"], wl.s, dX=c["dX"], dA=c["dA"],
                                              dB=c["dB"], ws=wl.ws), 5, st)
     out["chanq_bwd"] = {"TFLOPs": round(cb / t / 1e12, 1), "frac_tc": round(cb / t / 1e12 / tc_sus, 3)}
+    # the weighted Lloyd-Max learner of that layer's tables at 1, 2 and 4 bits (8
+    # iterations each), e.g. for the precision allocation's per-channel errors; bound by
+    # float64 arithmetic, reported as weight bytes read per second and time per layer
+    t0s = {b: torch.tensor(lloyd_t0(b)) for b in (1, 2, 4)}
+    t = time_loop(lambda: [q.chanq_learn(c["W"], b, t0s[b], 8) for b in (1, 2, 4)], 3, st)
+    out["chanq_learn"] = {"GBps": round(3 * CQ_N * CQ_K * 2 / t / 1e9, 1), "ms": round(t * 1e3, 3),
+                          "bound": "fp64 alu"}
     # decode (memory-bound): rotate over weight copies whose total exceeds L2 twice over
     l2 = torch.cuda.get_device_properties(wl.dev).L2_cache_size
     wbytes = sum(L["w"].nbytes() for L in wl.layers)

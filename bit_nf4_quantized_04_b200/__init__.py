@@ -25,7 +25,7 @@ BLOCK2 = 256
 __all__ = [
     "Nf4Weight", "nf4_codebook", "nf4_quantize", "double_quant", "dequant", "quantize_weight",
     "qlora_linear_fwd", "qlora_linear_bwd", "nf4_recon_error", "rank_topk",
-    "dense_linear_fwd", "dense_linear_bwd", "chanq_quantize", "chanq_linear_fwd", "chanq_linear_bwd",
+    "dense_linear_fwd", "dense_linear_bwd", "chanq_quantize", "chanq_linear_fwd", "chanq_linear_bwd", "chanq_learn",
     "workspace_size", "check", "set_wait_timeout_ns", "Qnf4Error",
 ]
 
@@ -273,6 +273,23 @@ def chanq_linear_bwd(packed, row_off, bits, maps, map_off, absmax, N: int, K: in
               dY.data_ptr(), M, A.data_ptr(), B.data_ptr(), r, float(scale), dX.data_ptr(),
               dA.data_ptr(), dB.data_ptr(), wsb.data_ptr(), wsb.numel(), _stream(x))
     return dX, dA, dB
+
+
+def chanq_learn(W: torch.Tensor, bits: int, thr0: torch.Tensor, iters: int = 8):
+    """Weighted Lloyd-Max tables of every row at one bit width: (map fp32 [N, 2^b],
+    thr fp32 [N, 2^b - 1], err float64 [N], iterations int32 [N])."""
+    _req(W, torch.bfloat16, "W")
+    N, K = W.shape
+    L = 1 << bits
+    dev = W.device
+    thr0 = thr0.to(device=dev, dtype=torch.float32).contiguous()
+    mp = torch.empty(N, L, dtype=torch.float32, device=dev)
+    th = torch.empty(N, L - 1, dtype=torch.float32, device=dev)
+    err = torch.empty(N, dtype=torch.float64, device=dev)
+    it = torch.empty(N, dtype=torch.int32, device=dev)
+    _lib.call("qnf4_chanq_learn", W.data_ptr(), N, K, bits, thr0.data_ptr(), iters, mp.data_ptr(),
+              th.data_ptr(), err.data_ptr(), it.data_ptr(), _stream(W))
+    return mp, th, err, it
 
 
 def check(stream: int | None = None) -> None:

@@ -52,6 +52,7 @@ SIGNATURES = {
                                    P]),
     "qnf4_chanq_linear_bwd": (ST, [P, P, P, P, P, P, I64, I64, P, P, I64, P, P, I32, F32, P, P,
                                    P, P, SZ, P]),
+    "qnf4_chanq_learn": (ST, [P, I64, I64, I32, P, I32, P, P, P, P, P]),
     "qnf4_workspace_size": (SZ, [I32, I64, I64, I64, I32]),
     "qnf4_check": (ST, [P]),
     "qnf4_set_wait_timeout_ns": (ST, [C.c_uint64]),

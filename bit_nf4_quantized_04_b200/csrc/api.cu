@@ -1043,6 +1043,35 @@ qnf4_status qnf4_chanq_linear_fwd(const uint8_t* packed, const int64_t* row_off,
   return linear_fwd(src, x, M, A, B, r, scale, h, ws, ws_bytes, static_cast<cudaStream_t>(stream));
 }
 
+qnf4_status qnf4_chanq_learn(const void* W_bf16, int64_t N, int64_t K, int32_t bits,
+                             const float* thr0, int32_t iters, float* map, float* thr,
+                             double* err, int32_t* iters_done, void* stream) {
+  for (const void* p : {W_bf16, static_cast<const void*>(thr0), static_cast<const void*>(map),
+                        static_cast<const void*>(thr), static_cast<const void*>(err)}) {
+    if (!p) return fail(QNF4_ERR_ARG, "NULL buffer");
+    if (!al16(p)) return fail(QNF4_ERR_ALIGN, "buffers must be 16-byte aligned");
+  }
+  if (bits != 1 && bits != 2 && bits != 4) return fail(QNF4_ERR_ARG, "bits must be 1, 2 or 4 (got %d)", bits);
+  if (iters < 1) return fail(QNF4_ERR_ARG, "iters must be >= 1");
+  if (N < 0 || K <= 0 || K % 64) return fail(QNF4_ERR_SHAPE, "K must be a positive multiple of 64");
+  if (K > 32768) return fail(QNF4_ERR_SHAPE, "K at most 32768 (the row lives in shared memory)");
+  if (N == 0) return QNF4_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t smem = static_cast<size_t>(K) * 4 + static_cast<size_t>(K / 64) * 4;
+  const int grid = static_cast<int>(std::min<int64_t>(N, static_cast<int64_t>(num_sms()) * 4));
+  auto go = [&](auto kern) -> qnf4_status {
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
+      return fail(QNF4_ERR_CUDA, "shared memory attribute refused");
+    kern<<<grid, kLearnThreads, smem, s>>>(static_cast<const uint16_t*>(W_bf16), N, K, thr0, iters, map,
+                                           thr, err, iters_done);
+    return launched("chanq_learn");
+  };
+  if (bits == 1) return go(k_chanq_learn<2>);
+  if (bits == 2) return go(k_chanq_learn<4>);
+  return go(k_chanq_learn<16>);
+}
+
 qnf4_status qnf4_chanq_linear_bwd(const uint8_t* packed, const int64_t* row_off, const uint8_t* bits,
                                   const float* map, const int64_t* map_off, const float* absmax,
                                   int64_t N, int64_t K, const void* x, const void* dY, int64_t M,

@@ -205,4 +205,173 @@ __global__ void __launch_bounds__(256) k_chanq_widen(const uint8_t* __restrict__
   }
 }
 
+
+// ---------------------------------------------------------------------------
+// Weighted Lloyd-Max learner of a row's mapping and thresholds ("LowRA", 第五部分
+// 映射与阈值学习器, with the §4.1 group normalisation). One CTA per row, L = 2^b levels.
+// Values x = fp32(w / g) (0 in an all-zero group), weight g = the 64-group absmax.
+// Each iteration: bin = #{k : x > t_k}; per bin S0 = sum g, S1 = sum g x in float64
+// (the products of two fp32 values are exact there, so only the summation order, which
+// is fixed here, differs from a sequential sum); centre m_k = fp32(S1 / S0) or the
+// previous value for an empty bin; thresholds fp32((m_k + m_{k+1}) / 2); error
+// E = (sum (g x) x - sum_k (2 m_k S1_k - m_k^2 S0_k)) / sum g, evaluated with explicit
+// roundings (no contraction); from the second iteration on, E not below the previous
+// one stops after that iteration. Initial centres: -1, midpoints of the initial
+// thresholds, +1. Output: the last tables, the iterations run, and the mean over the
+// row of (w - fp32(m[c] g))^2 (float64) with c from the output thresholds.
+// ---------------------------------------------------------------------------
+constexpr int kLearnThreads = 256;
+
+// Fixed-order block sum of NV doubles per thread: warp butterflies, then the warps'
+// results in warp order; the sums land in s_out[0..NV). Every thread of the block calls it.
+template <int NV, int NW>
+QNF4_DEV void learn_block_sum(double (&v)[NV], double* s_red, double* s_out) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+#pragma unroll
+    for (int o = 16; o; o >>= 1) v[i] = __dadd_rn(v[i], __shfl_xor_sync(0xffffffffu, v[i], o));
+  }
+  if (lane == 0) {
+#pragma unroll
+    for (int i = 0; i < NV; ++i) s_red[warp * NV + i] = v[i];
+  }
+  __syncthreads();
+  if (tid < NV) {
+    double a = 0.0;
+    for (int w = 0; w < NW; ++w) a = __dadd_rn(a, s_red[w * NV + tid]);
+    s_out[tid] = a;
+  }
+  __syncthreads();
+}
+
+template <int L>
+__global__ void __launch_bounds__(kLearnThreads) k_chanq_learn(
+    const uint16_t* __restrict__ W, int64_t N, int64_t K, const float* __restrict__ thr0, int iters,
+    float* __restrict__ map_out, float* __restrict__ thr_out, double* __restrict__ err_out,
+    int* __restrict__ done_out) {
+  constexpr int NW = kLearnThreads / 32;
+  extern __shared__ float lsm[];
+  float* sx = lsm;          // normalised values [K]
+  float* sg = lsm + K;      // group absmax [K / 64]
+  __shared__ double s_red[NW * 2 * L];
+  __shared__ double s_S[2 * L];
+  __shared__ double s_tot[2];
+  __shared__ double s_term[L];
+  __shared__ float s_t[L], s_m[L];
+  __shared__ int s_stop;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+  for (int64_t n = blockIdx.x; n < N; n += gridDim.x) {
+    const uint16_t* wr = W + n * K;
+    // values and weights: a warp per 64-group, two elements per lane
+    for (int64_t grp = warp; grp < K / 64; grp += NW) {
+      const uint32_t pr = *reinterpret_cast<const uint32_t*>(wr + grp * 64 + 2 * lane);
+      const float a = bf16lo(pr), b = bf16hi(pr);
+      float mx = fmaxf(fabsf(a), fabsf(b));
+#pragma unroll
+      for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      sx[grp * 64 + 2 * lane] = mx > 0.f ? __fdiv_rn(a, mx) : 0.f;
+      sx[grp * 64 + 2 * lane + 1] = mx > 0.f ? __fdiv_rn(b, mx) : 0.f;
+      if (lane == 0) sg[grp] = mx;
+    }
+    __syncthreads();
+    {
+      double v[2] = {0.0, 0.0};  // sum g, sum (g x) x
+      for (int64_t j = tid; j < K; j += kLearnThreads) {
+        const double gg = sg[j >> 6], xx = sx[j];
+        v[0] = __dadd_rn(v[0], gg);
+        v[1] = __dadd_rn(v[1], __dmul_rn(__dmul_rn(gg, xx), xx));
+      }
+      learn_block_sum<2, NW>(v, s_red, s_S);
+      if (tid == 0) {
+        s_tot[0] = s_S[0];
+        s_tot[1] = s_S[1];
+      }
+    }
+    if (tid < L - 1) s_t[tid] = thr0[tid];
+    __syncthreads();
+    if (tid < L)
+      s_m[tid] = tid == 0 ? -1.f
+               : tid == L - 1 ? 1.f
+                              : __double2float_rn(__dmul_rn(__dadd_rn(static_cast<double>(s_t[tid - 1]),
+                                                                      static_cast<double>(s_t[tid])), 0.5));
+    if (tid == 0) s_stop = 0;
+    __syncthreads();
+    double eprev = 0.0;  // thread 0
+    int done = 0;
+    for (int it = 0; it < iters; ++it) {
+      float tr[L - 1];
+#pragma unroll
+      for (int k = 0; k < L - 1; ++k) tr[k] = s_t[k];
+      // every bin's sums in registers, predicated (only bin c gains; the others add
+      // exact zeros)
+      double v[2 * L];
+#pragma unroll
+      for (int k = 0; k < 2 * L; ++k) v[k] = 0.0;
+      for (int64_t j = tid; j < K; j += kLearnThreads) {
+        const float xx = sx[j];
+        int c = 0;
+#pragma unroll
+        for (int k = 0; k < L - 1; ++k) c += xx > tr[k] ? 1 : 0;
+        const double gg = sg[j >> 6];
+        const double gx = __dmul_rn(gg, static_cast<double>(xx));
+#pragma unroll
+        for (int k = 0; k < L; ++k) {
+          v[k] = __dadd_rn(v[k], c == k ? gg : 0.0);
+          v[L + k] = __dadd_rn(v[L + k], c == k ? gx : 0.0);
+        }
+      }
+      learn_block_sum<2 * L, NW>(v, s_red, s_S);
+      // centre k and its error term on thread k; thresholds on threads 0..L-2; the
+      // terms summed in bin order on thread 0
+      if (tid < L) {
+        const double S0 = s_S[tid], S1 = s_S[L + tid];
+        if (S0 > 0.0) s_m[tid] = __double2float_rn(__ddiv_rn(S1, S0));
+        const double mk = s_m[tid];
+        s_term[tid] = __dsub_rn(__dmul_rn(__dmul_rn(2.0, mk), S1), __dmul_rn(__dmul_rn(mk, mk), S0));
+      }
+      __syncthreads();
+      if (tid < L - 1)
+        s_t[tid] = __double2float_rn(__dmul_rn(__dadd_rn(static_cast<double>(s_m[tid]),
+                                                         static_cast<double>(s_m[tid + 1])), 0.5));
+      if (tid == 0) {
+        double acc = 0.0;
+        for (int k = 0; k < L; ++k) acc = __dadd_rn(acc, s_term[k]);
+        const double E = s_tot[0] > 0.0 ? __ddiv_rn(__dsub_rn(s_tot[1], acc), s_tot[0]) : 0.0;
+        if (it > 0 && E >= eprev) s_stop = 1;
+        eprev = E;
+      }
+      done = it + 1;
+      __syncthreads();
+      if (s_stop) break;
+    }
+    // the error of the quantization the output tables give
+    {
+      float tr[L - 1];
+#pragma unroll
+      for (int k = 0; k < L - 1; ++k) tr[k] = s_t[k];
+      double v[1] = {0.0};
+      for (int64_t j = tid; j < K; j += kLearnThreads) {
+        const float xx = sx[j];
+        int c = 0;
+#pragma unroll
+        for (int k = 0; k < L - 1; ++k) c += xx > tr[k] ? 1 : 0;
+        const float deq = __fmul_rn(s_m[c], sg[j >> 6]);
+        const float wv = __uint_as_float(static_cast<uint32_t>(wr[j]) << 16);
+        const double d = __dsub_rn(static_cast<double>(wv), static_cast<double>(deq));
+        v[0] = __dadd_rn(v[0], __dmul_rn(d, d));
+      }
+      learn_block_sum<1, NW>(v, s_red, s_S);
+      if (tid == 0) {
+        err_out[n] = __ddiv_rn(s_S[0], static_cast<double>(K));
+        if (done_out) done_out[n] = done;
+      }
+    }
+    if (tid < L) map_out[n * L + tid] = s_m[tid];
+    if (tid < L - 1) thr_out[n * (L - 1) + tid] = s_t[tid];
+    __syncthreads();  // the next row reuses the shared arrays
+  }
+}
+
 }  // namespace qnf4

@@ -232,6 +232,23 @@ QNF4_API qnf4_status qnf4_chanq_linear_bwd(const uint8_t* packed, const int64_t*
                                   int32_t r, float scale, void* dX, float* dA, float* dB,
                                   void* ws, size_t ws_bytes, void* stream);
 
+/* [LowRA 第五部分 (the mapping and threshold learner), with the §4.1 group normalisation]
+ * Weighted Lloyd-Max learning of every row's mapping and thresholds at one bit width.
+ * W_bf16 [N, K] (K a multiple of 64, at most 32768); bits in {1, 2, 4}; thr0 the 2^b - 1
+ * initial thresholds shared by all rows (device, fp32, ascending: 0.0 for 1 bit, the
+ * NormalFloat midpoints for 2 and 4 bits in the page's scheme); iters >= 1 the cap.
+ * Per row, values x = fp32(w / g) weighted by their 64-group absmax g; each iteration
+ * assigns x to bin #{k : x > t_k}, sets each centre to its bin's weighted mean (float64
+ * sums, rounded to fp32; an empty bin keeps its centre) and each threshold to the fp32
+ * midpoint of its neighbours, and the learner stops once the weighted error no longer
+ * decreases. Outputs (device): map fp32 [N, 2^b], thr fp32 [N, 2^b - 1] (the last
+ * tables), err float64 [N] = mean over the row of (w - fp32(map[c] g))^2 with c from
+ * thr (the channel's quantization error, e.g. for a precision allocation), and
+ * iters_done int32 [N] (or NULL). Deterministic. */
+QNF4_API qnf4_status qnf4_chanq_learn(const void* W_bf16, int64_t N, int64_t K, int32_t bits,
+                             const float* thr0, int32_t iters, float* map, float* thr,
+                             double* err, int32_t* iters_done, void* stream);
+
 /* Bytes of device workspace an operation needs for these sizes (0 if none). */
 QNF4_API size_t qnf4_workspace_size(int32_t op, int64_t N, int64_t K, int64_t M, int32_t r);
 
