@@ -467,10 +467,8 @@ def run_ours(args):
         torch.distributed.barrier()
     elapsed = t_start.elapsed_time(t_stop) / 1e3
     q.check()
-    if ws_ > 1:
-        tt = torch.tensor([elapsed], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        elapsed = float(tt.item())
+    from bit_nf4_quantized_04_b200.dist import max_over_ranks
+    elapsed = max_over_ranks(elapsed, dev)
     # dominant kernel: the fwd h GEMM or the bwd dX GEMM, whichever took longer
     tf = sum(a.elapsed_time(b) for a, b in evf) / 1e3
     tb = sum(a.elapsed_time(b) for a, b in evb) / 1e3
@@ -507,11 +505,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     if ws_ > 1:
         torch.distributed.barrier()
-    te = time_loop(e2e_step, ke, stream)
-    if ws_ > 1:
-        tt = torch.tensor([te], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        te = float(tt.item())
+    te = max_over_ranks(time_loop(e2e_step, ke, stream), dev)
     e2e_value = flops * ws_ / te / 1e12
     cpu = None
     if rank == 0 and ws_ == 1 and not args.no_cpu:

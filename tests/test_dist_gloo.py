@@ -1,0 +1,113 @@
+"""The multi-rank paths on CPU: two processes over gloo (world size 2), the exchanges of
+bit_nf4_quantized_04_b200.dist checked against the single-process oracle.
+
+* sharded profiling pass ("AQLoRA", §3.1 and the §3.2 layer choice): each rank computes the
+  NF4 reconstruction SSE of its own layers (here with the oracle), the SSEs are all-gathered
+  and both ranks must rank the same top-K as the oracle on all layers;
+* token data parallelism (QLoRA's adapter training): each rank's dA, dB over its token
+  shard, all-reduced, must equal the full-batch gradients;
+* the benchmark's timing rule: the maximum over ranks.
+"""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as tdist
+import torch.multiprocessing as mp
+
+import synth
+
+WORLD = 2
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _layers():
+    # six layers of different shapes and spreads (so the ranking is not trivial)
+    shapes = [(64, 128), (128, 64), (96, 192), (64, 256), (192, 64), (128, 128)]
+    return [synth.llama_weight(sh, 700 + i, std=0.01 * (1 + (i * 7) % 5)) for i, sh in enumerate(shapes)]
+
+
+def _grads(x, dY, Wb, A, B, s):
+    from oracle import linear as olin
+    _, dA, dB = olin.backward(x, dY, Wb, A, B, s)
+    return dA.astype(np.float32), dB.astype(np.float32)
+
+
+def _case():
+    M, N, K, r = 12, 48, 64, 4
+    x = synth.normal_bf16((M, K), 1.0, 801).float().numpy().astype(np.float64)
+    dY = synth.normal_bf16((M, N), 1.0, 802).float().numpy().astype(np.float64)
+    Wb = synth.normal_bf16((N, K), 0.02, 803).float().numpy().astype(np.float64)
+    A = synth.normal_bf16((r, K), 0.01, 804).float().numpy().astype(np.float64)
+    B = synth.normal_bf16((N, r), 0.01, 805).float().numpy().astype(np.float64)
+    return x, dY, Wb, A, B, 2.0
+
+
+def _worker(rank, port, out_dir):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    tdist.init_process_group("gloo", rank=rank, world_size=WORLD)
+    try:
+        from bit_nf4_quantized_04_b200 import dist
+        from oracle import nf4 as onf4
+        from oracle import rank as orank
+        layers = _layers()
+        top, sse = dist.sharded_profile_topk(
+            layers, 3, sse_fn=lambda W: onf4.recon_sse(W.float().numpy()),
+            rank_fn=lambda s, n, k: orank.top_k(s, n, k), device=torch.device("cpu"))
+        x, dY, Wb, A, B, s = _case()
+        sl = slice(rank, None, WORLD)          # this rank's tokens
+        dA, dB = _grads(x[sl], dY[sl], Wb, A, B, s)
+        tA, tB = torch.from_numpy(dA), torch.from_numpy(dB)
+        dist.allreduce_adapter_grads(tA, tB)
+        mx = dist.max_over_ranks(1.0 + rank)
+        np.savez(os.path.join(out_dir, f"r{rank}.npz"), top=np.array(top), sse=sse.numpy(),
+                 dA=tA.numpy(), dB=tB.numpy(), mx=np.array(mx))
+    finally:
+        tdist.barrier()
+        tdist.destroy_process_group()
+
+
+def test_two_ranks_over_gloo(tmp_path):
+    mp.spawn(_worker, args=(_free_port(), str(tmp_path)), nprocs=WORLD, join=True)
+    res = [np.load(tmp_path / f"r{r}.npz") for r in range(WORLD)]
+    from oracle import nf4 as onf4
+    from oracle import rank as orank
+    layers = _layers()
+    sse_ref = np.array([onf4.recon_sse(W.float().numpy()) for W in layers])
+    top_ref = orank.top_k(list(sse_ref), [int(W.numel()) for W in layers], 3)
+    x, dY, Wb, A, B, s = _case()
+    dA_ref, dB_ref = _grads(x, dY, Wb, A, B, s)
+    for r in range(WORLD):
+        assert np.array_equal(res[r]["sse"], sse_ref)          # each SSE computed once, gathered
+        assert list(res[r]["top"]) == list(top_ref)
+        np.testing.assert_allclose(res[r]["dA"], dA_ref, rtol=1e-5, atol=1e-6)
+        np.testing.assert_allclose(res[r]["dB"], dB_ref, rtol=1e-5, atol=1e-6)
+        assert float(res[r]["mx"]) == float(WORLD)
+    # both ranks hold bit-identical gradients after the all-reduce
+    assert np.array_equal(res[0]["dA"], res[1]["dA"]) and np.array_equal(res[0]["dB"], res[1]["dB"])
+
+
+def test_shard_covers_every_item_once():
+    from bit_nf4_quantized_04_b200.dist import shard
+    for n in (0, 1, 5, 6, 7):
+        for world in (1, 2, 3, 4):
+            got = sorted(i for r in range(world) for i in shard(n, world, r))
+            assert got == list(range(n))
+
+
+def test_single_process_reduces_to_local():
+    from bit_nf4_quantized_04_b200 import dist
+    from oracle import nf4 as onf4
+    layers = _layers()[:3]
+    sse = dist.sharded_layer_errors(layers, sse_fn=lambda W: onf4.recon_sse(W.float().numpy()),
+                                    device=torch.device("cpu"))
+    assert np.array_equal(sse.numpy(), [onf4.recon_sse(W.float().numpy()) for W in layers])
+    assert dist.max_over_ranks(3.5) == 3.5
