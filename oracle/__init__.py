@@ -28,4 +28,4 @@ leave open (tail probability of the NF4 grid, nibble order, tie rules, the 8-bit
 float format for double quantization) are self-consistent readings and marked
 "parity unpinned" where no page fixes them.
 """
-from . import numerics, nf4, linear, chanq, rank, lloyd  # noqa: F401
+from . import numerics, nf4, linear, chanq, rank, lloyd, loftq  # noqa: F401
