@@ -369,6 +369,14 @@ def breakdown(wl, q, hbm, tc_sus):
     t = time_loop(lambda: [q.chanq_learn(c["W"], b, t0s[b], 8) for b in (1, 2, 4)], 3, st)
     out["chanq_learn"] = {"GBps": round(3 * CQ_N * CQ_K * 2 / t / 1e9, 1), "ms": round(t * 1e3, 3),
                           "bound": "fp64 alu"}
+    # LoftQ-style initialisation of that layer over the NF4 base (five alternating steps at
+    # the adapter rank): time per layer; the Gram matrix and its eigensolve are library calls
+    lws = torch.empty(q.workspace_size(q._lib.OP_LOFTQ, CQ_N, CQ_K, 0, RANK), dtype=torch.uint8,
+                      device=wl.dev)
+    q.loftq_nf4(c["W"], RANK, 5, ws=lws)
+    t = time_loop(lambda: q.loftq_nf4(c["W"], RANK, 5, ws=lws), 2, st)
+    out["loftq_init"] = {"ms": round(t * 1e3, 2), "steps": 5, "rank": RANK}
+    del lws
     # decode (memory-bound): rotate over weight copies whose total exceeds L2 twice over
     l2 = torch.cuda.get_device_properties(wl.dev).L2_cache_size
     wbytes = sum(L["w"].nbytes() for L in wl.layers)

@@ -292,6 +292,27 @@ def chanq_learn(W: torch.Tensor, bits: int, thr0: torch.Tensor, iters: int = 8):
     return mp, th, err, it
 
 
+def loftq_nf4(W: torch.Tensor, r: int, steps: int = 5, ws=None):
+    """LoftQ-style initialisation over the NF4 base: (the last step's ``Nf4Weight``,
+    A fp32 [r, K], B fp32 [N, r], objectives ||W - Q - B A||_F^2 float64 [steps])."""
+    _req(W, torch.bfloat16, "W")
+    N, K = W.shape
+    dev = W.device
+    n = N * K
+    packed = torch.empty(n // 2, dtype=torch.uint8, device=dev)
+    code2 = torch.empty(n // BLOCK1, dtype=torch.uint8, device=dev)
+    scale2 = torch.empty((n // BLOCK1 + BLOCK2 - 1) // BLOCK2, dtype=torch.float32, device=dev)
+    mean = torch.empty(4, dtype=torch.float32, device=dev)
+    A = torch.empty(r, K, dtype=torch.float32, device=dev)
+    B = torch.empty(N, r, dtype=torch.float32, device=dev)
+    errs = torch.empty(steps, dtype=torch.float64, device=dev)
+    wsb = _ws(workspace_size(_lib.OP_LOFTQ, N, K, 0, r), W, ws)
+    _lib.call("qnf4_loftq_nf4", W.data_ptr(), N, K, r, steps, packed.data_ptr(), code2.data_ptr(),
+              scale2.data_ptr(), mean.data_ptr(), A.data_ptr(), B.data_ptr(), errs.data_ptr(),
+              wsb.data_ptr(), wsb.numel(), _stream(W))
+    return Nf4Weight(N, K, packed, code2, scale2, mean[:1]), A, B, errs
+
+
 def check(stream: int | None = None) -> None:
     """Synchronise the stream and raise if a kernel's bounded wait gave up."""
     _lib.call("qnf4_check", torch.cuda.current_stream().cuda_stream if stream is None else stream)

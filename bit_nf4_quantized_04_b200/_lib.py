@@ -16,7 +16,7 @@ QNF4_OK = 0
 STATUS_NAMES = {0: "OK", 1: "ERR_ARG", 2: "ERR_SHAPE", 3: "ERR_ALIGN", 4: "ERR_CUDA",
                 5: "ERR_TIMEOUT", 6: "ERR_WORKSPACE"}
 OUT_F32, OUT_BF16 = 0, 1
-OP_QUANTIZE, OP_DOUBLE_QUANT, OP_FWD, OP_BWD, OP_CHANQ_FWD, OP_CHANQ_BWD = 0, 1, 2, 3, 4, 5
+OP_QUANTIZE, OP_DOUBLE_QUANT, OP_FWD, OP_BWD, OP_CHANQ_FWD, OP_CHANQ_BWD, OP_LOFTQ = 0, 1, 2, 3, 4, 5, 6
 
 
 class Qnf4Weight(C.Structure):
@@ -53,6 +53,7 @@ SIGNATURES = {
     "qnf4_chanq_linear_bwd": (ST, [P, P, P, P, P, P, I64, I64, P, P, I64, P, P, I32, F32, P, P,
                                    P, P, SZ, P]),
     "qnf4_chanq_learn": (ST, [P, I64, I64, I32, P, I32, P, P, P, P, P]),
+    "qnf4_loftq_nf4": (ST, [P, I64, I64, I32, I32, P, P, P, P, P, P, P, P, SZ, P]),
     "qnf4_workspace_size": (SZ, [I32, I64, I64, I64, I32]),
     "qnf4_check": (ST, [P]),
     "qnf4_set_wait_timeout_ns": (ST, [C.c_uint64]),

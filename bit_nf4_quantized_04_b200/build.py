@@ -17,7 +17,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libqnf4.so")
 SOURCES = ["api.cu", "codebook.cpp"]
-HEADERS = ["common.cuh", "quant.cuh", "chanq.cuh", "gemm.cuh", "tables.h"]
+HEADERS = ["common.cuh", "quant.cuh", "chanq.cuh", "gemm.cuh", "loftq.cuh", "tables.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
@@ -47,7 +47,7 @@ def build(force: bool = False, verbose: bool = False, extra: list[str] | None = 
            "-Xcompiler", "-fvisibility=hidden", "--expt-relaxed-constexpr",
            "-I", os.path.join(ROOT, "include"),
            *(extra or []),
-           *[os.path.join(CSRC, f) for f in SOURCES], "-o", tmp]
+           *[os.path.join(CSRC, f) for f in SOURCES], "-ldl", "-o", tmp]
     if verbose:
         print(" ".join(cmd), flush=True)
     res = subprocess.run(cmd, capture_output=True, text=True)

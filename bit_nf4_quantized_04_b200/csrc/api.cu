@@ -4,6 +4,9 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
+#include <cublas_v2.h>
+#include <cusolverDn.h>
+#include <dlfcn.h>
 
 #include <algorithm>
 #include <atomic>
@@ -18,6 +21,7 @@
 #include "chanq.cuh"
 #include "common.cuh"
 #include "gemm.cuh"
+#include "loftq.cuh"
 #include "quant.cuh"
 #include "tables.h"
 
@@ -727,6 +731,103 @@ void* noalloc_scratch_ptr() {
   }
   return cache[dev];
 }
+// ---------------------------------------------------------------------------
+// Dense linear algebra for the LoftQ initialisation's truncated SVD: cuBLAS (sgemm) and
+// cuSOLVER (syevd), loaded at first use by soname (torch's copies when torch has loaded
+// them, else the toolkit's), so the library still loads where they are absent.
+// ---------------------------------------------------------------------------
+struct LinAlgLib {
+  bool ok = false;
+  decltype(&cublasCreate_v2) blas_create = nullptr;
+  decltype(&cublasSetStream_v2) blas_stream = nullptr;
+  decltype(&cublasSgemm_v2) sgemm = nullptr;
+  decltype(&cusolverDnCreate) sol_create = nullptr;
+  decltype(&cusolverDnSetStream) sol_stream = nullptr;
+  decltype(&cusolverDnSsyevd_bufferSize) syevd_size = nullptr;
+  decltype(&cusolverDnSsyevd) syevd = nullptr;
+};
+
+const LinAlgLib& linalg_lib() {
+  static const LinAlgLib lib = [] {
+    LinAlgLib l;
+    auto open = [](std::initializer_list<const char*> names) -> void* {
+      for (const char* n : names)
+        if (void* h = dlopen(n, RTLD_NOW | RTLD_GLOBAL)) return h;
+      return nullptr;
+    };
+    void* hb = open({"libcublas.so.12", "/usr/local/cuda/lib64/libcublas.so.12", "libcublas.so"});
+    void* hs = open({"libcusolver.so.11", "/usr/local/cuda/lib64/libcusolver.so.11", "libcusolver.so"});
+    if (!hb || !hs) return l;
+    l.blas_create = reinterpret_cast<decltype(l.blas_create)>(dlsym(hb, "cublasCreate_v2"));
+    l.blas_stream = reinterpret_cast<decltype(l.blas_stream)>(dlsym(hb, "cublasSetStream_v2"));
+    l.sgemm = reinterpret_cast<decltype(l.sgemm)>(dlsym(hb, "cublasSgemm_v2"));
+    l.sol_create = reinterpret_cast<decltype(l.sol_create)>(dlsym(hs, "cusolverDnCreate"));
+    l.sol_stream = reinterpret_cast<decltype(l.sol_stream)>(dlsym(hs, "cusolverDnSetStream"));
+    l.syevd_size = reinterpret_cast<decltype(l.syevd_size)>(dlsym(hs, "cusolverDnSsyevd_bufferSize"));
+    l.syevd = reinterpret_cast<decltype(l.syevd)>(dlsym(hs, "cusolverDnSsyevd"));
+    l.ok = l.blas_create && l.blas_stream && l.sgemm && l.sol_create && l.sol_stream &&
+           l.syevd_size && l.syevd;
+    return l;
+  }();
+  return lib;
+}
+
+// One cuBLAS and one cuSOLVER handle per device, kept for the process.
+bool linalg_handles(cublasHandle_t* hb, cusolverDnHandle_t* hs) {
+  const LinAlgLib& L = linalg_lib();
+  if (!L.ok) return false;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return false;
+  static std::mutex mu;
+  static cublasHandle_t b[64] = {};
+  static cusolverDnHandle_t so[64] = {};
+  std::lock_guard<std::mutex> lk(mu);
+  if (!b[dev] && L.blas_create(&b[dev]) != CUBLAS_STATUS_SUCCESS) return false;
+  if (!so[dev] && L.sol_create(&so[dev]) != CUSOLVER_STATUS_SUCCESS) return false;
+  *hb = b[dev];
+  *hs = so[dev];
+  return true;
+}
+
+// Floats of syevd workspace for an m x m Gram matrix: the library's own query when a GPU
+// and cuSOLVER are at hand, and never below the LAPACK bound 1 + 6m + 2m^2.
+size_t loftq_lwork(int64_t m) {
+  size_t need = 1 + 6 * static_cast<size_t>(m) + 2 * static_cast<size_t>(m) * static_cast<size_t>(m);
+  cublasHandle_t hb;
+  cusolverDnHandle_t hs;
+  if (linalg_handles(&hb, &hs)) {
+    int lw = 0;
+    if (linalg_lib().syevd_size(hs, CUSOLVER_EIG_MODE_VECTOR, CUBLAS_FILL_MODE_LOWER, static_cast<int>(m),
+                                nullptr, static_cast<int>(m), nullptr, &lw) == CUSOLVER_STATUS_SUCCESS)
+      need = std::max(need, static_cast<size_t>(lw));
+  }
+  return need;
+}
+
+struct LoftqLayout {
+  size_t tgt, q, absmax, dq, gram, eig, p, info, work, total;
+  int64_t m;
+  size_t lwork;
+};
+
+LoftqLayout loftq_layout(int64_t N, int64_t K, int r) {
+  LoftqLayout l{};
+  l.m = std::min(N, K);
+  l.lwork = loftq_lwork(l.m);
+  size_t o = 0;
+  l.tgt = o;    o = align256(o + static_cast<size_t>(N) * K * 2);
+  l.q = o;      o = align256(o + static_cast<size_t>(N) * K * 4);
+  l.absmax = o; o = align256(o + static_cast<size_t>(N) * K / 64 * 4);
+  l.dq = o;     o = align256(o + qnf4_workspace_size(QNF4_OP_DOUBLE_QUANT, 0, 0, 0, 0));
+  l.gram = o;   o = align256(o + static_cast<size_t>(l.m) * l.m * 4);
+  l.eig = o;    o = align256(o + static_cast<size_t>(l.m) * 4);
+  l.p = o;      o = align256(o + static_cast<size_t>(l.m) * r * 4);
+  l.info = o;   o = align256(o + 16);
+  l.work = o;   o = align256(o + l.lwork * 4);
+  l.total = o;
+  return l;
+}
+
 }  // namespace
 }  // namespace qnf4
 
@@ -793,6 +894,7 @@ size_t qnf4_workspace_size(int32_t op, int64_t N, int64_t K, int64_t M, int32_t 
     case QNF4_OP_FWD: return plan_linear(A_NF4_K, N, K, M, r, false, num_sms()).total;
     case QNF4_OP_BWD: return plan_linear(A_NF4_MN, N, K, M, r, true, num_sms()).total;
     case QNF4_OP_CHANQ_FWD: return plan_linear(A_CHANQ_K, N, K, M, r, false, num_sms()).total;
+    case QNF4_OP_LOFTQ: return loftq_layout(N, K, r).total;
     case QNF4_OP_CHANQ_BWD: {
       const size_t t = plan_linear(A_CHANQ_MN, N, K, M, r, true, num_sms()).total;
       return t + chanq_wide_bytes(N, K);
@@ -1070,6 +1172,90 @@ qnf4_status qnf4_chanq_learn(const void* W_bf16, int64_t N, int64_t K, int32_t b
   if (bits == 1) return go(k_chanq_learn<2>);
   if (bits == 2) return go(k_chanq_learn<4>);
   return go(k_chanq_learn<16>);
+}
+
+qnf4_status qnf4_loftq_nf4(const void* W_bf16, int64_t N, int64_t K, int32_t r, int32_t steps,
+                           uint8_t* packed, uint8_t* code2, float* scale2, float* mean, float* A,
+                           float* B, double* errs, void* ws, size_t ws_bytes, void* stream) {
+  for (const void* p : {W_bf16, static_cast<const void*>(packed), static_cast<const void*>(code2),
+                        static_cast<const void*>(scale2), static_cast<const void*>(mean),
+                        static_cast<const void*>(A), static_cast<const void*>(B),
+                        static_cast<const void*>(errs)}) {
+    if (!p) return fail(QNF4_ERR_ARG, "NULL buffer");
+    if (!al16(p)) return fail(QNF4_ERR_ALIGN, "buffers must be 16-byte aligned");
+  }
+  if (N <= 0 || K <= 0 || K % 64) return fail(QNF4_ERR_SHAPE, "N > 0 and K a positive multiple of 64");
+  if (r < 1 || r > std::min(N, K)) return fail(QNF4_ERR_ARG, "r must be in [1, min(N, K)]");
+  if (steps < 1) return fail(QNF4_ERR_ARG, "steps must be >= 1");
+  if (std::min(N, K) > 16384) return fail(QNF4_ERR_SHAPE, "min(N, K) at most 16384 (the Gram matrix)");
+  cublasHandle_t hb;
+  cusolverDnHandle_t hs;
+  if (!linalg_handles(&hb, &hs)) return fail(QNF4_ERR_CUDA, "cuBLAS / cuSOLVER unavailable");
+  const LoftqLayout l = loftq_layout(N, K, r);
+  if (!ws || ws_bytes < l.total) return fail(QNF4_ERR_WORKSPACE, "workspace too small (%zu < %zu)", ws_bytes, l.total);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const LinAlgLib& L = linalg_lib();
+  if (L.blas_stream(hb, s) != CUBLAS_STATUS_SUCCESS || L.sol_stream(hs, s) != CUSOLVER_STATUS_SUCCESS)
+    return fail(QNF4_ERR_CUDA, "cuBLAS / cuSOLVER stream");
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  uint16_t* tgt = reinterpret_cast<uint16_t*>(w8 + l.tgt);
+  float* Q = reinterpret_cast<float*>(w8 + l.q);
+  float* absmax = reinterpret_cast<float*>(w8 + l.absmax);
+  float* G = reinterpret_cast<float*>(w8 + l.gram);
+  float* eig = reinterpret_cast<float*>(w8 + l.eig);
+  float* P = reinterpret_cast<float*>(w8 + l.p);
+  int* info = reinterpret_cast<int*>(w8 + l.info);
+  float* work = reinterpret_cast<float*>(w8 + l.work);
+  const int64_t m = l.m;
+  const bool gram_k = N >= K;  // Gram R^T R (K x K) when N >= K, else R R^T (N x N)
+  cudaMemsetAsync(A, 0, sizeof(float) * r * K, s);
+  cudaMemsetAsync(B, 0, sizeof(float) * N * r, s);
+  qnf4_weight wq{N, K, 64, 256, packed, code2, scale2, mean};
+  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((N * K + 255) / 256, num_sms() * 8)));
+  const float one = 1.f, zero = 0.f;
+  for (int t = 0; t < steps; ++t) {
+    k_loftq_target<<<grid, 256, 0, s>>>(static_cast<const uint16_t*>(W_bf16), B, A, N, K, r, tgt);
+    qnf4_status st = launched("loftq_target");
+    if (st != QNF4_OK) return st;
+    st = qnf4_nf4_quantize(tgt, N, K, 64, packed, absmax, nullptr, nullptr, 0, stream);
+    if (st != QNF4_OK) return st;
+    st = qnf4_double_quant(absmax, N * K / 64, 256, code2, scale2, mean, w8 + l.dq,
+                           qnf4_workspace_size(QNF4_OP_DOUBLE_QUANT, 0, 0, 0, 0), stream);
+    if (st != QNF4_OK) return st;
+    st = qnf4_dequant(&wq, Q, QNF4_OUT_F32, stream);
+    if (st != QNF4_OK) return st;
+    k_loftq_residual<<<grid, 256, 0, s>>>(static_cast<const uint16_t*>(W_bf16), Q, N * K);
+    st = launched("loftq_residual");
+    if (st != QNF4_OK) return st;
+    // R row-major [N, K] is column-major K x N with leading dimension K
+    const cublasStatus_t g1 =
+        gram_k ? L.sgemm(hb, CUBLAS_OP_N, CUBLAS_OP_T, static_cast<int>(K), static_cast<int>(K),
+                         static_cast<int>(N), &one, Q, static_cast<int>(K), Q, static_cast<int>(K), &zero, G,
+                         static_cast<int>(K))
+               : L.sgemm(hb, CUBLAS_OP_T, CUBLAS_OP_N, static_cast<int>(N), static_cast<int>(N),
+                         static_cast<int>(K), &one, Q, static_cast<int>(K), Q, static_cast<int>(K), &zero, G,
+                         static_cast<int>(N));
+    if (g1 != CUBLAS_STATUS_SUCCESS) return fail(QNF4_ERR_CUDA, "cuBLAS sgemm (Gram) failed");
+    if (L.syevd(hs, CUSOLVER_EIG_MODE_VECTOR, CUBLAS_FILL_MODE_LOWER, static_cast<int>(m), G,
+                static_cast<int>(m), eig, work, static_cast<int>(l.lwork), info) != CUSOLVER_STATUS_SUCCESS)
+      return fail(QNF4_ERR_CUDA, "cuSOLVER syevd failed");
+    const int fg = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((m * r + 255) / 256, num_sms() * 4)));
+    // top-r eigenvectors: Gram on the K side gives V (A = rho V^T, B = R V / rho), on the
+    // N side U (B = rho U, A^T = R^T U / rho)
+    k_loftq_factor<<<fg, 256, 0, s>>>(G, eig, m, r, P, gram_k ? A : B, gram_k ? 0 : 1);
+    st = launched("loftq_factor");
+    if (st != QNF4_OK) return st;
+    const cublasStatus_t g2 =
+        gram_k ? L.sgemm(hb, CUBLAS_OP_T, CUBLAS_OP_N, r, static_cast<int>(N), static_cast<int>(K), &one, P,
+                         static_cast<int>(K), Q, static_cast<int>(K), &zero, B, r)
+               : L.sgemm(hb, CUBLAS_OP_N, CUBLAS_OP_N, static_cast<int>(K), r, static_cast<int>(N), &one, Q,
+                         static_cast<int>(K), P, static_cast<int>(N), &zero, A, static_cast<int>(K));
+    if (g2 != CUBLAS_STATUS_SUCCESS) return fail(QNF4_ERR_CUDA, "cuBLAS sgemm (factor) failed");
+    k_loftq_err<<<1, 256, 0, s>>>(eig, m, r, info, errs + t);
+    st = launched("loftq_err");
+    if (st != QNF4_OK) return st;
+  }
+  return QNF4_OK;
 }
 
 qnf4_status qnf4_chanq_linear_bwd(const uint8_t* packed, const int64_t* row_off, const uint8_t* bits,

@@ -69,7 +69,8 @@ enum {
   QNF4_OP_FWD = 2,          /* qnf4_qlora_linear_fwd, qnf4_dense_linear_fwd          */
   QNF4_OP_BWD = 3,          /* qnf4_qlora_linear_bwd, qnf4_dense_linear_bwd          */
   QNF4_OP_CHANQ_FWD = 4,    /* qnf4_chanq_linear_fwd                                 */
-  QNF4_OP_CHANQ_BWD = 5     /* qnf4_chanq_linear_bwd                                 */
+  QNF4_OP_CHANQ_BWD = 5,    /* qnf4_chanq_linear_bwd                                 */
+  QNF4_OP_LOFTQ = 6         /* qnf4_loftq_nf4                                        */
 };
 
 /* A double-quantized NF4 weight [QLoRA 贡献一/贡献二]. All pointers are device
@@ -248,6 +249,21 @@ QNF4_API qnf4_status qnf4_chanq_linear_bwd(const uint8_t* packed, const int64_t*
 QNF4_API qnf4_status qnf4_chanq_learn(const void* W_bf16, int64_t N, int64_t K, int32_t bits,
                              const float* thr0, int32_t iters, float* map, float* thr,
                              double* err, int32_t* iters_done, void* stream);
+
+/* [LowRA workflow: quantize, take the quantization error, initialise the low-rank tensors
+ * with LoftQ, five alternating steps; QLoRA's NF4 + double quantization as the quantizer]
+ * With A = 0, B = 0 at the start, each step: Q = dequant(NF4 + double quant(bf16(W - B A)))
+ * into packed / code2 / scale2 / mean (the qnf4_weight layout of qnf4_nf4_quantize and
+ * qnf4_double_quant); R = W - Q; B = U S^(1/2), A = S^(1/2) V^T from the rank-r truncated
+ * SVD U S V^T of R; errs[t] = ||W - Q - B A||_F^2 (float64, the discarded squared singular
+ * values). The SVD goes through the Gram matrix of R in fp32 (cuBLAS sgemm, cuSOLVER syevd,
+ * loaded at first use: QNF4_ERR_CUDA if they are absent). W_bf16 [N, K], K a multiple of 64,
+ * 1 <= r <= min(N, K), min(N, K) <= 16384, steps >= 1. Outputs (device): the last step's
+ * quantized base, A fp32 [r, K], B fp32 [N, r], errs [steps]. Workspace: QNF4_OP_LOFTQ. */
+QNF4_API qnf4_status qnf4_loftq_nf4(const void* W_bf16, int64_t N, int64_t K, int32_t r,
+                           int32_t steps, uint8_t* packed, uint8_t* code2, float* scale2,
+                           float* mean, float* A, float* B, double* errs, void* ws,
+                           size_t ws_bytes, void* stream);
 
 /* Bytes of device workspace an operation needs for these sizes (0 if none). */
 QNF4_API size_t qnf4_workspace_size(int32_t op, int64_t N, int64_t K, int64_t M, int32_t r);
