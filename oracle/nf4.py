@@ -2,7 +2,8 @@
 
 TEST INFRASTRUCTURE ONLY (see the package docstring). Source: "QLoRA: Efficient
 Finetuning of Quantized LLMs" (Heng's Blog), sections 贡献一 4-bit NormalFloat (NF4)
-and 贡献二 Double Quantization; "AQLoRA", §3.1 for the reconstruction error.
+and 贡献二 Double Quantization; "AQLoRA", §3.1 for the reconstruction error and the
+sparsity of a layer.
 
 Readings of points the page leaves open (each is a convention, self-consistent on
 both sides of the parity tests):
@@ -217,6 +218,23 @@ def recon_sse(w: np.ndarray, block1: int = BLOCK1) -> float:
 def recon_error(w: np.ndarray, block1: int = BLOCK1) -> float:
     """epsilon_l = SSE_l / |W_l|."""
     return recon_sse(w, block1) / np.asarray(w).size
+
+
+# AQLoRA §3.1: the layer's sparsity s_l = Pr[|W_ij| < tau] with tau = 0.01. The threshold
+# is taken as the fp32 value of tau (the form the kernels receive); for bf16 weights that
+# is the same test as against the real 0.01, since no bf16 value lies between the two.
+SPARSITY_TAU = np.float32(0.01)
+
+
+def below_count(w: np.ndarray, tau=SPARSITY_TAU) -> int:
+    """#{elements with |w| < tau}, tau given as fp32."""
+    a = np.abs(np.asarray(w, dtype=np.float64).reshape(-1))
+    return int(np.count_nonzero(a < float(np.float32(tau))))
+
+
+def sparsity(w: np.ndarray, tau=SPARSITY_TAU) -> float:
+    """s_l = below_count / |W_l|."""
+    return below_count(w, tau) / np.asarray(w).size
 
 
 # ---------------------------------------------------------------------------

@@ -87,6 +87,12 @@ def test_tiny_layer_fwd_bwd(q):
     (256, 256, 1, 64),     # single token, largest rank
     (128, 1024, 300, 24),
     (264, 320, 64, 8),
+    # several token tiles with ragged token rows, v's contraction N = 1000 (not a multiple
+    # of the 64-wide step), ranks padded to 16, 32, 48 and 64 columns
+    (1000, 256, 700, 5),
+    (520, 640, 512, 20),
+    (264, 192, 530, 40),
+    (136, 384, 600, 64),
 ])
 def test_ragged_shapes(q, N, K, M, r):
     _run_nf4(q, N, K, M, r, seed=N * 7 + K + M + r)

@@ -5,6 +5,7 @@ page prints (tests/golden), closed forms, brute force on small inputs, or a libr
 routine (math.erfc, torch's fp8 / bf16 casts) that the oracle does not use.
 """
 import math
+from fractions import Fraction
 import os
 
 import numpy as np
@@ -290,3 +291,35 @@ def test_recon_error_zero_on_grid_and_bruteforce():
     _, c = nf4.quantize(w)
     hg = float(np.max(np.diff(q.astype(np.float64)))) / 2
     assert nf4.recon_sse(w) <= w.size * hg ** 2 * float(np.max(c)) ** 2
+
+
+# ---------------------------------------------------------------------------
+# AQLoRA §3.1 sparsity s_l = Pr[|W_ij| < tau], tau = 0.01
+# ---------------------------------------------------------------------------
+def _below_exact(vals, tau=Fraction(1, 100)):
+    # brute force against the real number 0.01, each value taken exactly
+    return sum(1 for v in vals if abs(Fraction(float(v))) < tau)
+
+
+def test_sparsity_brute_force_against_real_tau():
+    W = torch.randn(48, 128, generator=torch.Generator().manual_seed(5)) * 0.02
+    Wb = W.to(torch.bfloat16).float().numpy()
+    assert nf4.below_count(Wb) == _below_exact(Wb.reshape(-1))
+    assert nf4.sparsity(Wb) == _below_exact(Wb.reshape(-1)) / Wb.size
+
+
+def test_sparsity_at_the_bf16_neighbours_of_tau():
+    # bf16 values in [2^-7, 2^-6) are multiples of 2^-14: 163 * 2^-14 < 0.01 < 164 * 2^-14
+    lo, hi = 163 * 2.0 ** -14, 164 * 2.0 ** -14
+    assert lo < 0.01 < hi
+    vals = np.array([lo, -lo, hi, -hi, 0.0, -0.0, 0.01, 1.0], dtype=np.float32)
+    vals = torch.from_numpy(vals).to(torch.bfloat16).float().numpy()
+    assert vals[0] == np.float32(lo) and vals[2] == np.float32(hi)
+    # lo, -lo, +0, -0 are below; hi, -hi, bf16(0.01) = hi, 1.0 are not
+    assert nf4.below_count(vals) == 4 == _below_exact(vals)
+
+
+def test_sparsity_special_cases():
+    assert nf4.sparsity(np.zeros((4, 64), np.float32)) == 1.0
+    assert nf4.sparsity(np.full((4, 64), 0.5, np.float32)) == 0.0
+    assert nf4.sparsity(np.full((4, 64), -0.01, np.float32)) == 0.0  # |w| = tau is not below
