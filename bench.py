@@ -210,7 +210,7 @@ class Workload:
             L["dX"] = torch.empty(M_TOK, K, dtype=torch.bfloat16, device=dev)
             L["dA"] = torch.empty(RANK, K, dtype=torch.float32, device=dev)
             L["dB"] = torch.empty(N, RANK, dtype=torch.float32, device=dev)
-            for op, m in ((q._lib.OP_QUANTIZE, 0), (q._lib.OP_DOUBLE_QUANT, 0),
+            for op, m in ((q._lib.OP_QUANTIZE, 0), (q._lib.OP_DOUBLE_QUANT, 0), (q._lib.OP_LAYER_STATS, 0),
                           (q._lib.OP_FWD, M_TOK), (q._lib.OP_BWD, M_TOK)):
                 wsz = max(wsz, q.workspace_size(op, N, K, m, RANK))
             self.layers.append(L)
@@ -340,6 +340,11 @@ def breakdown(wl, q, hbm, tc_sus):
                   10, st)
     gbs = nparam * 2 / t / 1e9
     out["recon_error"] = {"GBps": round(gbs, 1), "frac_hbm": round(gbs / hbm, 3)}
+    # the same pass with the AQLoRA sparsity count beside the error (one read of W)
+    lso = torch.empty(4, dtype=torch.float64, device=wl.dev)
+    t = time_loop(lambda: [q.nf4_layer_stats(L["W"], out=lso, ws=wl.ws) for L in wl.layers], 10, st)
+    gbs = nparam * 2 / t / 1e9
+    out["layer_stats"] = {"GBps": round(gbs, 1), "frac_hbm": round(gbs / hbm, 3)}
     ff = sum(fwd_flops(N, K, M_TOK, RANK) for N, K in layer_shapes())
     bf = sum(bwd_flops(N, K, M_TOK, RANK) for N, K in layer_shapes())
     t = time_loop(wl.fwd, 5, st)

@@ -183,6 +183,19 @@ def nf4_recon_error(W: torch.Tensor, sse=None, ws=None) -> torch.Tensor:
     return sse[:1]
 
 
+def nf4_layer_stats(W: torch.Tensor, tau: float = 0.01, out=None, ws=None):
+    """The AQLoRA profiling statistics of a bf16 [N, K] weight in one pass: float64 [2] =
+    (NF4 reconstruction SSE, #{|w| < tau}); epsilon and the sparsity are these / (N K)."""
+    _req(W, torch.bfloat16, "W")
+    N, K = W.shape
+    o = out if out is not None else torch.empty(4, dtype=torch.float64, device=W.device)
+    wsb = _ws(workspace_size(_lib.OP_LAYER_STATS, N, K), W, ws)
+    # the two doubles 16 bytes apart (the ABI wants 16-byte aligned outputs)
+    _lib.call("qnf4_nf4_layer_stats", W.data_ptr(), N, K, float(tau), o.data_ptr(),
+              o.data_ptr() + 16, wsb.data_ptr(), wsb.numel(), _stream(W))
+    return o[0::2]
+
+
 def rank_topk(sse, n_params, k: int) -> list[int]:
     """Host ranking: indices of the k layers with the largest sse/n, ties to the lower index."""
     s = [float(v) for v in sse]

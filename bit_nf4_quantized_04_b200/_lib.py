@@ -17,6 +17,7 @@ STATUS_NAMES = {0: "OK", 1: "ERR_ARG", 2: "ERR_SHAPE", 3: "ERR_ALIGN", 4: "ERR_C
                 5: "ERR_TIMEOUT", 6: "ERR_WORKSPACE"}
 OUT_F32, OUT_BF16 = 0, 1
 OP_QUANTIZE, OP_DOUBLE_QUANT, OP_FWD, OP_BWD, OP_CHANQ_FWD, OP_CHANQ_BWD, OP_LOFTQ = 0, 1, 2, 3, 4, 5, 6
+OP_LAYER_STATS = 7
 
 
 class Qnf4Weight(C.Structure):
@@ -44,6 +45,7 @@ SIGNATURES = {
     "qnf4_qlora_linear_bwd": (ST, [C.POINTER(Qnf4Weight), P, P, I64, P, P, I32, F32, P, P, P, P,
                                    SZ, P]),
     "qnf4_nf4_recon_error": (ST, [P, I64, I64, I32, P, P, SZ, P]),
+    "qnf4_nf4_layer_stats": (ST, [P, I64, I64, F32, P, P, P, SZ, P]),
     "qnf4_rank_topk": (ST, [P, P, I32, I32, P]),
     "qnf4_dense_linear_fwd": (ST, [P, I64, I64, P, I64, P, P, I32, F32, P, P, SZ, P]),
     "qnf4_dense_linear_bwd": (ST, [P, I64, I64, P, P, I64, P, P, I32, F32, P, P, P, P, SZ, P]),

@@ -9,6 +9,7 @@
 #include <dlfcn.h>
 
 #include <algorithm>
+#include <cmath>
 #include <atomic>
 #include <cstdarg>
 #include <cstdio>
@@ -94,7 +95,8 @@ qnf4_status quant_smem_attr() {
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !g_quant_smem_set[dev]) {
-    for (auto fn : {k_nf4_quant<true, true>, k_nf4_quant<true, false>, k_nf4_quant<false, true>}) {
+    for (auto fn : {k_nf4_quant<true, true>, k_nf4_quant<true, false>, k_nf4_quant<false, true>,
+                    k_nf4_quant<false, true, true>}) {
       const cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                  static_cast<int>(kQSmem));
       if (e != cudaSuccess) return fail(QNF4_ERR_CUDA, "smem attribute: %s", cudaGetErrorString(e));
@@ -890,6 +892,7 @@ qnf4_status qnf4_check(void* stream) {
 size_t qnf4_workspace_size(int32_t op, int64_t N, int64_t K, int64_t M, int32_t r) {
   switch (op) {
     case QNF4_OP_QUANTIZE: return kQuantMaxGrid * sizeof(double);
+    case QNF4_OP_LAYER_STATS: return 2 * kQuantMaxGrid * sizeof(double);
     case QNF4_OP_DOUBLE_QUANT: return kDqPartials * sizeof(double);
     case QNF4_OP_FWD: return plan_linear(A_NF4_K, N, K, M, r, false, num_sms()).total;
     case QNF4_OP_BWD: return plan_linear(A_NF4_MN, N, K, M, r, true, num_sms()).total;
@@ -959,6 +962,34 @@ qnf4_status qnf4_nf4_recon_error(const void* W, int64_t N, int64_t K, int32_t bl
                                                           make_tab(), g_wait_ns);
   k_sum_partials<<<1, 256, 0, s>>>(static_cast<const double*>(ws), grid, sse);
   return launched("nf4_recon_error", 2);
+}
+
+qnf4_status qnf4_nf4_layer_stats(const void* W, int64_t N, int64_t K, float tau, double* sse,
+                                 double* below, void* ws, size_t ws_bytes, void* stream) {
+  if (N < 0 || K <= 0) return fail(QNF4_ERR_SHAPE, "bad shape");
+  if (K % 64) return fail(QNF4_ERR_SHAPE, "K must be a multiple of 64");
+  if (!W || !sse || !below) return fail(QNF4_ERR_ARG, "NULL buffer");
+  if (!al16(W) || !al16(sse) || !al16(below)) return fail(QNF4_ERR_ALIGN, "buffers must be 16-byte aligned");
+  if (!(tau >= 0.f) || std::isinf(tau)) return fail(QNF4_ERR_ARG, "tau must be finite and >= 0");
+  if (!ws || ws_bytes < qnf4_workspace_size(QNF4_OP_LAYER_STATS, N, K, 0, 0))
+    return fail(QNF4_ERR_WORKSPACE, "workspace too small");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t nblocks = N * K / 64;
+  if (nblocks == 0) {
+    cudaMemsetAsync(sse, 0, sizeof(double), s);
+    cudaMemsetAsync(below, 0, sizeof(double), s);
+    return launched("layer_stats(empty)", 0);
+  }
+  qnf4_status st = quant_smem_attr();
+  if (st != QNF4_OK) return st;
+  const int grid = quant_grid(nblocks);
+  double* part = static_cast<double*>(ws);
+  k_nf4_quant<false, true, true><<<grid, kQThreads, kQSmem, s>>>(
+      static_cast<const uint16_t*>(W), nblocks, nullptr, nullptr, part, make_tab(), g_wait_ns, tau,
+      part + kQuantMaxGrid);
+  k_sum_partials<<<1, 256, 0, s>>>(part, grid, sse);
+  k_sum_partials<<<1, 256, 0, s>>>(part + kQuantMaxGrid, grid, below);
+  return launched("nf4_layer_stats", 3);
 }
 
 qnf4_status qnf4_double_quant(const float* absmax, int64_t nb1, int32_t block2, uint8_t* code2,

@@ -101,7 +101,8 @@ QNF4_DEV bool warp_wait(uint64_t* bar, uint32_t parity, unsigned long long wait_
 // chunk, a group of 8 threads takes one 64-element block (each thread 8 consecutive
 // elements, one 16-byte shared load) and writes 4 packed bytes. Optional outputs:
 // WRITE -> packed codes and fp32 absmax; SSE -> per-CTA float64 partial sums of the
-// single-level squared round-trip error.
+// single-level squared round-trip error; CNT -> per-CTA float64 counts of the elements
+// with |w| < tau (the sparsity of "AQLoRA" §3.1), exact integers.
 //
 // Code search (see Nf4Tables), for a block with absmax c > 0: the bin
 // k = round(w H/c + H) comes from one fused multiply-add with a magic constant
@@ -111,17 +112,18 @@ QNF4_DEV bool warp_wait(uint64_t* bar, uint32_t parity, unsigned long long wait_
 // thread's 8 values lies within 2^-18 c of its t_k, those 8 take the exact IEEE
 // quotient and the full count. Non-finite weights are outside the method: the table
 // index is masked, so they cannot read outside it, but their codes are unspecified.
-template <bool WRITE, bool SSE>
+template <bool WRITE, bool SSE, bool CNT = false>
 __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
     k_nf4_quant(const uint16_t* __restrict__ W, int64_t nblocks, uint32_t* __restrict__ packed,
                 float* __restrict__ absmax, double* __restrict__ sse_part, QuantTab tab,
-                unsigned long long wait_ns) {
+                unsigned long long wait_ns, float tau = 0.f, double* __restrict__ cnt_part = nullptr) {
   extern __shared__ uint8_t qsm_raw[];
   __shared__ __align__(8) uint64_t full[kQStages], empty[kQStages];
   __shared__ float s_thr[16];
   __shared__ float s_lv[16];
   __shared__ __align__(1024) float s_tc[2 * kMaxHalfBins + 1];
   __shared__ double s_red[kQWorkers];
+  __shared__ unsigned long long s_cnt[kQWorkers];
   __shared__ volatile int s_abort;
   uint8_t* qsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(qsm_raw) + 127) &
                                             ~static_cast<uintptr_t>(127));
@@ -145,6 +147,7 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
   __syncthreads();
 
   double acc = 0.0;
+  unsigned int below = 0;  // this thread's elements with |w| < tau (CNT)
   if (warp == kQWorkers) {
     // ---------------------------------------------------------------- producer
     if ((tid & 31) == 0) {
@@ -215,6 +218,10 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
         for (int e = 0; e < 4; ++e) {
           w[2 * e] = bf16lo(words[e]);
           w[2 * e + 1] = bf16hi(words[e]);
+        }
+        if (CNT && valid) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) below += fabsf(w[e]) < tau ? 1u : 0u;
         }
         float m = fmaxf(fabsf(w[0]), fabsf(w[1]));
 #pragma unroll
@@ -295,11 +302,22 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
     if ((tid & 31) == 0 && warp < kQWorkers) s_red[warp] = acc;
   }
+  if (CNT) {
+    unsigned long long b = below;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) b += __shfl_xor_sync(0xffffffffu, b, o);
+    if ((tid & 31) == 0 && warp < kQWorkers) s_cnt[warp] = b;
+  }
   __syncthreads();
   if (SSE && tid == 0) {
     double t = 0.0;
     for (int i = 0; i < kQWorkers; ++i) t += s_red[i];
     sse_part[blockIdx.x] = t;
+  }
+  if (CNT && tid == 0) {
+    unsigned long long t = 0;
+    for (int i = 0; i < kQWorkers; ++i) t += s_cnt[i];
+    cnt_part[blockIdx.x] = static_cast<double>(t);  // exact below 2^53
   }
 }
 

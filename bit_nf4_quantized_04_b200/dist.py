@@ -9,6 +9,8 @@ GPUs) for the exchanges the path really has.
   Quantized LLMs" (only A and B are trained): dA and dB are sums over tokens, so a rank
   that ran the backward on its share of the tokens all-reduces them (sum) to obtain the
   full-batch gradients; the frozen NF4 base needs no exchange.
+* The same pass with the layer's sparsity s = Pr[|w| < 0.01] beside the error
+  (sharded_layer_stats: two float64 per layer gathered).
 * max_over_ranks: the timing rule of the benchmark (the slowest rank's time).
 
 Every rank must call these functions in the same order with the same arguments' shapes.
@@ -58,6 +60,37 @@ def sharded_layer_errors(layers: Sequence[torch.Tensor],
     parts = [torch.empty_like(local) for _ in range(world)]
     tdist.all_gather(parts, local, group=group)
     out = torch.empty(n, dtype=torch.float64, device=dev)
+    for r in range(world):
+        for i, li in enumerate(shard(n, world, r)):
+            out[li] = parts[r][i]
+    return out
+
+
+def sharded_layer_stats(layers: Sequence[torch.Tensor],
+                        stats_fn: Callable[[torch.Tensor], Sequence[float]] | None = None,
+                        group=None, device: torch.device | None = None) -> torch.Tensor:
+    """Both statistics of the AQLoRA profiling pass for every layer, float64 [L, 2] =
+    (reconstruction SSE, #{|w| < 0.01}), identical on all ranks, each layer computed by
+    exactly one rank. `stats_fn` maps a bf16 weight to the pair; by default the library's
+    one-pass GPU kernel (qnf4_nf4_layer_stats)."""
+    world, rank = _world(group)
+    if stats_fn is None:
+        from . import nf4_layer_stats
+
+        def stats_fn(W):
+            return nf4_layer_stats(W).tolist()
+    n = len(layers)
+    mine = shard(n, world, rank)
+    per = (n + world - 1) // world
+    dev = device if device is not None else (layers[0].device if n else torch.device("cpu"))
+    local = torch.zeros(per, 2, dtype=torch.float64, device=dev)
+    for i, li in enumerate(mine):
+        local[i] = torch.tensor([float(v) for v in stats_fn(layers[li])], dtype=torch.float64)
+    if world == 1:
+        return local[:n].clone()
+    parts = [torch.empty_like(local) for _ in range(world)]
+    tdist.all_gather(parts, local, group=group)
+    out = torch.empty(n, 2, dtype=torch.float64, device=dev)
     for r in range(world):
         for i, li in enumerate(shard(n, world, r)):
             out[li] = parts[r][i]

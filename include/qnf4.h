@@ -70,7 +70,8 @@ enum {
   QNF4_OP_BWD = 3,          /* qnf4_qlora_linear_bwd, qnf4_dense_linear_bwd          */
   QNF4_OP_CHANQ_FWD = 4,    /* qnf4_chanq_linear_fwd                                 */
   QNF4_OP_CHANQ_BWD = 5,    /* qnf4_chanq_linear_bwd                                 */
-  QNF4_OP_LOFTQ = 6         /* qnf4_loftq_nf4                                        */
+  QNF4_OP_LOFTQ = 6,        /* qnf4_loftq_nf4                                        */
+  QNF4_OP_LAYER_STATS = 7   /* qnf4_nf4_layer_stats                                  */
 };
 
 /* A double-quantized NF4 weight [QLoRA 贡献一/贡献二]. All pointers are device
@@ -174,6 +175,15 @@ QNF4_API qnf4_status qnf4_qlora_linear_bwd(const qnf4_weight* w, const void* x, 
  * The caller divides by N*K for epsilon and ranks layers (qnf4_rank_topk). */
 QNF4_API qnf4_status qnf4_nf4_recon_error(const void* W_bf16, int64_t N, int64_t K, int32_t block1,
                                  double* sse, void* ws, size_t ws_bytes, void* stream);
+
+/* [AQLoRA §3.1] Both statistics of the profiling pass in one read of a bf16 weight [N, K]:
+ * sse (device, 1 double) exactly as qnf4_nf4_recon_error, and below (device, 1 double) =
+ * #{elements with |w| < tau}, an exact integer; the layer's sparsity is below / (N K).
+ * The page's tau is 0.01: pass 0.01f (for bf16 weights the same test as the real 0.01).
+ * K a multiple of 64, tau finite and >= 0. Workspace: QNF4_OP_LAYER_STATS. */
+QNF4_API qnf4_status qnf4_nf4_layer_stats(const void* W, int64_t N, int64_t K, float tau,
+                                 double* sse, double* below, void* ws, size_t ws_bytes,
+                                 void* stream);
 
 /* [AQLoRA abstract, §3.1] Host helper: indices of the k layers with the largest
  * epsilon = sse[i] / n_params[i], in descending order, ties to the lower index.

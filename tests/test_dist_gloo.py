@@ -2,8 +2,9 @@
 bit_nf4_quantized_04_b200.dist checked against the single-process oracle.
 
 * sharded profiling pass ("AQLoRA", §3.1 and the §3.2 layer choice): each rank computes the
-  NF4 reconstruction SSE of its own layers (here with the oracle), the SSEs are all-gathered
-  and both ranks must rank the same top-K as the oracle on all layers;
+  NF4 reconstruction SSE (and the sparsity count) of its own layers (here with the oracle),
+  the results are all-gathered and both ranks must rank the same top-K as the oracle on all
+  layers;
 * token data parallelism (QLoRA's adapter training): each rank's dA, dB over its token
   shard, all-reduced, must equal the full-batch gradients;
 * the benchmark's timing rule: the maximum over ranks.
@@ -62,13 +63,16 @@ def _worker(rank, port, out_dir):
         top, sse = dist.sharded_profile_topk(
             layers, 3, sse_fn=lambda W: onf4.recon_sse(W.float().numpy()),
             rank_fn=lambda s, n, k: orank.top_k(s, n, k), device=torch.device("cpu"))
+        stats = dist.sharded_layer_stats(
+            layers, stats_fn=lambda W: (onf4.recon_sse(W.float().numpy()), onf4.below_count(W.float().numpy())),
+            device=torch.device("cpu"))
         x, dY, Wb, A, B, s = _case()
         sl = slice(rank, None, WORLD)          # this rank's tokens
         dA, dB = _grads(x[sl], dY[sl], Wb, A, B, s)
         tA, tB = torch.from_numpy(dA), torch.from_numpy(dB)
         dist.allreduce_adapter_grads(tA, tB)
         mx = dist.max_over_ranks(1.0 + rank)
-        np.savez(os.path.join(out_dir, f"r{rank}.npz"), top=np.array(top), sse=sse.numpy(),
+        np.savez(os.path.join(out_dir, f"r{rank}.npz"), top=np.array(top), sse=sse.numpy(), stats=stats.numpy(),
                  dA=tA.numpy(), dB=tB.numpy(), mx=np.array(mx))
     finally:
         tdist.barrier()
@@ -88,6 +92,9 @@ def test_two_ranks_over_gloo(tmp_path):
     for r in range(WORLD):
         assert np.array_equal(res[r]["sse"], sse_ref)          # each SSE computed once, gathered
         assert list(res[r]["top"]) == list(top_ref)
+        # the sparsity counts travel with the errors ("AQLoRA" §3.1), each computed once
+        assert np.array_equal(res[r]["stats"][:, 0], sse_ref)
+        assert np.array_equal(res[r]["stats"][:, 1], [onf4.below_count(W.float().numpy()) for W in layers])
         np.testing.assert_allclose(res[r]["dA"], dA_ref, rtol=1e-5, atol=1e-6)
         np.testing.assert_allclose(res[r]["dB"], dB_ref, rtol=1e-5, atol=1e-6)
         assert float(res[r]["mx"]) == float(WORLD)

@@ -151,3 +151,34 @@ def test_recon_error(q, N, K):
     # the same figure from the quantize pass with its SSE output on
     _, _, s = q.nf4_quantize(W.cuda(), sse=True)
     assert abs(s.item() - ref) <= 1e-5 * ref
+
+
+@pytest.mark.parametrize("N,K", [(256, 512), (33, 320), (4096, 11008)])
+def test_layer_stats(q, N, K):
+    # AQLoRA §3.1 in one pass: the SSE bit-identical to the reconstruction-error kernel's,
+    # the count of |w| < 0.01 exact
+    W = synth.llama_weight((N, K), 199 + N, std=0.013)
+    st = q.nf4_layer_stats(W.cuda()).cpu().numpy()
+    assert st[0] == q.nf4_recon_error(W.cuda()).item()
+    assert st[1] == onf4.below_count(f32(W))
+    ref = onf4.recon_sse(f32(W))
+    assert abs(st[0] - ref) <= 1e-5 * ref
+
+
+def test_layer_stats_crafted_and_degenerate(q):
+    # the bf16 neighbours of tau, signed zeros, a whole zero row (its blocks all below),
+    # and a partial last chunk of the streamed kernel (N * K / 64 not a multiple of 128)
+    lo, hi = 163 * 2.0 ** -14, 164 * 2.0 ** -14
+    W = synth.llama_weight((3, 192), 7, std=0.02).float()
+    W[0, :8] = torch.tensor([lo, -lo, hi, -hi, 0.0, -0.0, 0.01, -0.01])
+    W[1] = 0.0
+    Wb = W.to(torch.bfloat16)
+    st = q.nf4_layer_stats(Wb.cuda()).cpu().numpy()
+    assert st[1] == onf4.below_count(f32(Wb))
+    assert abs(st[0] - onf4.recon_sse(f32(Wb))) <= 1e-5 * onf4.recon_sse(f32(Wb))
+    z = torch.zeros(5, 128, dtype=torch.bfloat16, device="cuda")
+    stz = q.nf4_layer_stats(z).cpu().numpy()
+    assert stz[0] == 0.0 and stz[1] == z.numel()
+    # another threshold: every element with |w| < 1 counts
+    st1 = q.nf4_layer_stats(Wb.cuda(), tau=1.0).cpu().numpy()
+    assert st1[1] == onf4.below_count(f32(Wb), np.float32(1.0)) == Wb.numel()
