@@ -159,9 +159,17 @@ def double_quant(absmax: np.ndarray, block2: int = BLOCK2):
     round-to-nearest-even. Returns (code2 uint8 [nb1], scale2 fp32 [nb2], mean fp32).
     """
     c = np.asarray(absmax, dtype=np.float32)
+    return double_quant_with_mean(c, dq_mean(c), block2)
+
+
+def double_quant_with_mean(absmax: np.ndarray, mu, block2: int = BLOCK2):
+    """The encoding step of double_quant with the tensor mean given: what one shard of a
+    matrix split across processes does once the mean of all its constants is known (its
+    first constant on a 256-block boundary)."""
+    c = np.asarray(absmax, dtype=np.float32)
+    mu = np.float32(mu)
     nb1 = c.size
     nb2 = (nb1 + block2 - 1) // block2
-    mu = dq_mean(c)
     cc = (c - mu).astype(np.float32)  # fp32 subtraction
     code2 = np.zeros(nb1, dtype=np.uint8)
     s2 = np.zeros(nb2, dtype=np.float32)

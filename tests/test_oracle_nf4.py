@@ -323,3 +323,22 @@ def test_sparsity_special_cases():
     assert nf4.sparsity(np.zeros((4, 64), np.float32)) == 1.0
     assert nf4.sparsity(np.full((4, 64), 0.5, np.float32)) == 0.0
     assert nf4.sparsity(np.full((4, 64), -0.01, np.float32)) == 0.0  # |w| = tau is not below
+
+
+def test_double_quant_sharded_on_256_block_boundaries_is_bit_identical():
+    # a matrix split by rows across processes: each shard's constants start on a 256-block
+    # boundary, the float64 sums of the shards add up exactly (bf16-derived constants), so
+    # encoding each shard with the global mean reproduces the whole-matrix result
+    W = torch.randn(24, 4096, generator=torch.Generator().manual_seed(11)) * 0.02
+    flat = W.to(torch.bfloat16).float().numpy().reshape(-1)
+    _, c = nf4.quantize(flat)
+    code2, s2, mu = nf4.double_quant(c)
+    cuts = [0, 4 * 64, 12 * 64, c.size]  # rows 0-3, 4-11, 12-23 (K / 64 = 64 constants per row)
+    parts = [c[a:b] for a, b in zip(cuts[:-1], cuts[1:])]
+    total = sum(math.fsum(p.astype(np.float64).tolist()) for p in parts)
+    assert total == math.fsum(c.astype(np.float64).tolist())
+    mu_g = np.float32(total / c.size)
+    assert mu_g == mu
+    got = [nf4.double_quant_with_mean(p, mu_g) for p in parts]
+    assert np.array_equal(np.concatenate([g[0] for g in got]), code2)
+    assert np.array_equal(np.concatenate([g[1] for g in got]), s2)
