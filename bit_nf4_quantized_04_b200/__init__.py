@@ -121,6 +121,33 @@ def double_quant(absmax: torch.Tensor, code2=None, scale2=None, mean=None, ws=No
     return code2, scale2, mean[:1]
 
 
+def dq_sum(absmax: torch.Tensor, out=None, ws=None) -> torch.Tensor:
+    """Float64 sum of a (shard's) first-level constants, device tensor [1]."""
+    _req(absmax, torch.float32, "absmax")
+    o = out if out is not None else torch.empty(2, dtype=torch.float64, device=absmax.device)
+    wsb = _ws(workspace_size(_lib.OP_DOUBLE_QUANT, 0, 0), absmax, ws)
+    _lib.call("qnf4_dq_sum", absmax.data_ptr(), absmax.numel(), o.data_ptr(), wsb.data_ptr(),
+              wsb.numel(), _stream(absmax))
+    return o[:1]
+
+
+def double_quant_shard(absmax: torch.Tensor, total_sum: torch.Tensor, total_count: int,
+                       code2=None, scale2=None, mean=None):
+    """Double quantization of one row shard's constants with the whole matrix's constant
+    sum (float64 device tensor, 16-byte aligned) and count: (code2, scale2, mean)."""
+    _req(absmax, torch.float32, "absmax")
+    nb1 = absmax.numel()
+    nb2 = (nb1 + BLOCK2 - 1) // BLOCK2
+    dev = absmax.device
+    code2 = code2 if code2 is not None else torch.empty(nb1, dtype=torch.uint8, device=dev)
+    scale2 = scale2 if scale2 is not None else torch.empty(nb2, dtype=torch.float32, device=dev)
+    mean = mean if mean is not None else torch.empty(4, dtype=torch.float32, device=dev)
+    _lib.call("qnf4_double_quant_shard", absmax.data_ptr(), nb1, BLOCK2, total_sum.data_ptr(),
+              int(total_count), code2.data_ptr(), scale2.data_ptr(), mean.data_ptr(),
+              _stream(absmax))
+    return code2, scale2, mean[:1]
+
+
 def quantize_weight(W: torch.Tensor) -> Nf4Weight:
     """NF4 + double quantization of a bf16 [N, K] weight into an ``Nf4Weight``."""
     N, K = W.shape

@@ -39,6 +39,8 @@ SIGNATURES = {
     "qnf4_nf4_codebook": (ST, [P, P]),
     "qnf4_nf4_quantize": (ST, [P, I64, I64, I32, P, P, P, P, SZ, P]),
     "qnf4_double_quant": (ST, [P, I64, I32, P, P, P, P, SZ, P]),
+    "qnf4_dq_sum": (ST, [P, I64, P, P, SZ, P]),
+    "qnf4_double_quant_shard": (ST, [P, I64, I32, P, I64, P, P, P, P]),
     "qnf4_dequant": (ST, [C.POINTER(Qnf4Weight), P, I32, P]),
     "qnf4_qlora_linear_fwd": (ST, [C.POINTER(Qnf4Weight), P, I64, P, P, I32, F32, P, P, SZ, P]),
     "qnf4_qlora_linear_fwd_noalloc": (ST, [C.POINTER(Qnf4Weight), P, I64, P, P, I32, F32, P, P]),

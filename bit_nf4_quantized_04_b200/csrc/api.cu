@@ -1007,8 +1007,38 @@ qnf4_status qnf4_double_quant(const float* absmax, int64_t nb1, int32_t block2, 
   const int64_t nb2 = (nb1 + 255) / 256;
   int grid = static_cast<int>(std::min<int64_t>((nb2 + 7) / 8, num_sms() * 4));
   grid = std::max(grid, 1);
-  k_dq_encode<<<grid, 256, 0, s>>>(absmax, nb1, part, kDqPartials, code2, scale2, mean);
+  k_dq_encode<<<grid, 256, 0, s>>>(absmax, nb1, part, kDqPartials, nb1, code2, scale2, mean);
   return launched("double_quant", 2);
+}
+
+qnf4_status qnf4_dq_sum(const float* absmax, int64_t nb1, double* sum, void* ws, size_t ws_bytes,
+                        void* stream) {
+  if (nb1 <= 0) return fail(QNF4_ERR_SHAPE, "nb1 must be positive");
+  if (!absmax || !sum) return fail(QNF4_ERR_ARG, "NULL buffer");
+  if (!al16(absmax) || !al16(sum)) return fail(QNF4_ERR_ALIGN, "buffers must be 16-byte aligned");
+  if (!ws || ws_bytes < qnf4_workspace_size(QNF4_OP_DOUBLE_QUANT, 0, 0, 0, 0))
+    return fail(QNF4_ERR_WORKSPACE, "workspace too small");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  double* part = static_cast<double*>(ws);
+  k_dq_partial<<<kDqPartials, 256, 0, s>>>(absmax, nb1, part);
+  k_sum_partials<<<1, 256, 0, s>>>(part, kDqPartials, sum);
+  return launched("dq_sum", 2);
+}
+
+qnf4_status qnf4_double_quant_shard(const float* absmax, int64_t nb1, int32_t block2,
+                                    const double* total_sum, int64_t total_count, uint8_t* code2,
+                                    float* scale2, float* mean, void* stream) {
+  if (block2 != 256) return fail(QNF4_ERR_ARG, "block2 must be 256");
+  if (nb1 <= 0) return fail(QNF4_ERR_SHAPE, "nb1 must be positive");
+  if (total_count < nb1) return fail(QNF4_ERR_SHAPE, "total_count must be >= nb1");
+  if (!absmax || !total_sum || !code2 || !scale2 || !mean) return fail(QNF4_ERR_ARG, "NULL buffer");
+  if (!al16(absmax) || !al16(total_sum) || !al16(code2) || !al16(scale2) || !al16(mean))
+    return fail(QNF4_ERR_ALIGN, "buffers must be 16-byte aligned");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t nb2 = (nb1 + 255) / 256;
+  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((nb2 + 7) / 8, num_sms() * 4)));
+  k_dq_encode<<<grid, 256, 0, s>>>(absmax, nb1, total_sum, 1, total_count, code2, scale2, mean);
+  return launched("dq_encode_shard");
 }
 
 qnf4_status qnf4_dequant(const qnf4_weight* w, void* out, int32_t out_dtype, void* stream) {

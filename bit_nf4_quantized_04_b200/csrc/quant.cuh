@@ -363,9 +363,11 @@ __global__ void __launch_bounds__(256) k_dq_partial(const float* __restrict__ c,
 // exactly in float64, so the mean is independent of the summation order), then one
 // warp per 256-block: subtract the mean, block absmax, scale = absmax / 448 (IEEE
 // division), code = E4M3 round-to-nearest-even with saturation of (c - mean)/scale.
+// count is the number of constants behind the partials: nb1 for a whole matrix, the
+// matrix's total for one row shard of it (whose partial is then the all-reduced sum).
 __global__ void __launch_bounds__(256) k_dq_encode(const float* __restrict__ c, int64_t nb1,
                                                    const double* __restrict__ part, int npart,
-                                                   uint8_t* __restrict__ code2,
+                                                   int64_t count, uint8_t* __restrict__ code2,
                                                    float* __restrict__ scale2,
                                                    float* __restrict__ mean_out) {
   __shared__ float s_mu;
@@ -376,7 +378,7 @@ __global__ void __launch_bounds__(256) k_dq_encode(const float* __restrict__ c, 
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
     if (lane == 0) {
-      const float mu = static_cast<float>(t / static_cast<double>(nb1));
+      const float mu = static_cast<float>(t / static_cast<double>(count));
       s_mu = mu;
       if (blockIdx.x == 0) *mean_out = mu;
     }

@@ -11,6 +11,10 @@ GPUs) for the exchanges the path really has.
   full-batch gradients; the frozen NF4 base needs no exchange.
 * The same pass with the layer's sparsity s = Pr[|w| < 0.01] beside the error
   (sharded_layer_stats: two float64 per layer gathered).
+* One matrix quantized as row shards ("QLoRA", 贡献二): NF4 is blockwise and local; the
+  double-quantization mean needs the float64 sum of all the matrix's constants, one exact
+  all-reduce of a scalar, after which each shard encodes its own constants
+  (sharded_quantize_weight), bit-identical to one process.
 * max_over_ranks: the timing rule of the benchmark (the slowest rank's time).
 
 Every rank must call these functions in the same order with the same arguments' shapes.
@@ -19,6 +23,7 @@ they reduce to the local computation.
 """
 from __future__ import annotations
 
+import math
 from typing import Callable, Sequence
 
 import torch
@@ -109,6 +114,47 @@ def sharded_profile_topk(layers: Sequence[torch.Tensor], k: int,
         from . import rank_topk as rank_fn
     n_params = [int(W.numel()) for W in layers]
     return rank_fn(sse.cpu().tolist(), n_params, k), sse
+
+
+def shard_rows(N: int, K: int, world: int, rank: int) -> tuple[int, int]:
+    """Rows [r0, r1) of an [N, K] weight for `rank` when it is quantized as row shards: as
+    even as possible in units of 256 / gcd(256, K / 64) rows, so that every shard's block
+    constants start on a 256-constant (double-quantization block) boundary."""
+    unit = 256 // math.gcd(256, K // 64)
+    units = (N + unit - 1) // unit
+    lo = (units * rank) // world
+    hi = (units * (rank + 1)) // world
+    return min(N, lo * unit), min(N, hi * unit)
+
+
+def sharded_double_quant(absmax: torch.Tensor, total_count: int, group=None,
+                         sum_fn: Callable | None = None, encode_fn: Callable | None = None):
+    """Double quantization of this rank's row shard of one matrix ("QLoRA", 贡献二): the
+    shard's float64 constant sum is all-reduced (exact: bf16-derived constants sum exactly
+    in float64, so the mean is bit-identical to one process), then the shard is encoded
+    with the matrix's mean. `sum_fn(absmax)` -> float64 tensor [1], `encode_fn(absmax,
+    total_sum, total_count)` -> (code2, scale2, mean); by default the library's qnf4_dq_sum
+    and qnf4_double_quant_shard."""
+    world, _ = _world(group)
+    if sum_fn is None:
+        from . import dq_sum as sum_fn
+    if encode_fn is None:
+        from . import double_quant_shard as encode_fn
+    total = sum_fn(absmax)
+    if world > 1:
+        tdist.all_reduce(total, op=tdist.ReduceOp.SUM, group=group)
+    return encode_fn(absmax, total, total_count)
+
+
+def sharded_quantize_weight(W_rows: torch.Tensor, N: int, group=None):
+    """NF4 + double quantization of this rank's rows (shard_rows) of an [N, K] bf16 weight:
+    the rank's ``Nf4Weight`` slice (packed codes of its rows, its constants' code2 / scale2
+    slices and the matrix's mean). NF4 needs no exchange; the mean needs one scalar."""
+    from . import Nf4Weight, nf4_quantize
+    rows, K = W_rows.shape
+    packed, absmax = nf4_quantize(W_rows)
+    code2, scale2, mean = sharded_double_quant(absmax, N * K // 64, group)
+    return Nf4Weight(rows, K, packed, code2, scale2, mean)
 
 
 def allreduce_adapter_grads(dA: torch.Tensor, dB: torch.Tensor, group=None) -> None:

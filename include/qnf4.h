@@ -127,6 +127,20 @@ QNF4_API qnf4_status qnf4_double_quant(const float* absmax, int64_t nb1, int32_t
                               uint8_t* code2, float* scale2, float* mean,
                               void* ws, size_t ws_bytes, void* stream);
 
+/* [QLoRA 贡献二] A matrix quantized as row shards (one per process): the tensor mean needs
+ * the float64 sum of all its constants. qnf4_dq_sum writes this shard's sum to *sum (device,
+ * 1 double; workspace QNF4_OP_DOUBLE_QUANT); the caller adds the shards' sums (an exact
+ * all-reduce: bf16-derived constants sum exactly in float64) and passes the total and the
+ * matrix's constant count to qnf4_double_quant_shard, which encodes this shard's nb1
+ * constants exactly as qnf4_double_quant encodes them inside the whole matrix, provided the
+ * shard starts on a 256-constant boundary (its rows a multiple of 256 / gcd(256, K / 64)).
+ * Outputs are the shard's slices of code2 / scale2, and the (global) mean. */
+QNF4_API qnf4_status qnf4_dq_sum(const float* absmax, int64_t nb1, double* sum, void* ws,
+                        size_t ws_bytes, void* stream);
+QNF4_API qnf4_status qnf4_double_quant_shard(const float* absmax, int64_t nb1, int32_t block2,
+                                    const double* total_sum, int64_t total_count,
+                                    uint8_t* code2, float* scale2, float* mean, void* stream);
+
 /* [QLoRA opening formula, 贡献二] Two-level dequantization of a whole weight to
  * out [N, K] as fp32 (out_dtype QNF4_OUT_F32) or bf16 round-to-nearest-even
  * (QNF4_OUT_BF16). Meant for tests and export: the linear layer never writes the

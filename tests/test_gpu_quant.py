@@ -182,3 +182,27 @@ def test_layer_stats_crafted_and_degenerate(q):
     # another threshold: every element with |w| < 1 counts
     st1 = q.nf4_layer_stats(Wb.cuda(), tau=1.0).cpu().numpy()
     assert st1[1] == onf4.below_count(f32(Wb), np.float32(1.0)) == Wb.numel()
+
+
+@pytest.mark.parametrize("N,K,world", [(150, 11008, 2), (4096, 4096, 3), (33, 320, 4)])
+def test_row_sharded_quantization_is_bit_identical(q, N, K, world):
+    # one matrix quantized as row shards (one per process in production; here in turn on
+    # one GPU): NF4 codes and constants per shard, float64 constant sums added (what the
+    # all-reduce does), each shard encoded with the matrix's sum and count
+    from bit_nf4_quantized_04_b200 import dist
+    W = synth.llama_weight((N, K), 300 + N, std=0.02).cuda()
+    whole = q.quantize_weight(W)
+    spans = [dist.shard_rows(N, K, world, r) for r in range(world)]
+    parts = [q.nf4_quantize(W[a:b].contiguous()) for a, b in spans if b > a]
+    total = torch.zeros(2, dtype=torch.float64, device="cuda")
+    for _, absmax in parts:
+        total[:1] += q.dq_sum(absmax)
+    enc = [q.double_quant_shard(absmax, total, N * K // 64) for _, absmax in parts]
+    torch.cuda.synchronize()
+    assert torch.equal(torch.cat([p for p, _ in parts]), whole.packed)
+    assert torch.equal(torch.cat([e[0] for e in enc]), whole.code2)
+    assert torch.equal(torch.cat([e[1] for e in enc]), whole.scale2)
+    assert all(torch.equal(e[2], whole.mean) for e in enc)
+    # one process: the dist entry point reduces to the whole-matrix quantization
+    w1 = dist.sharded_quantize_weight(W, N)
+    assert torch.equal(w1.code2, whole.code2) and torch.equal(w1.mean, whole.mean)
