@@ -279,6 +279,25 @@ class Workload:
         self.bwd(evb)
         self.chanq()
 
+    def layer_step(self, L):
+        """One layer's share of the step (quantize + double quant, fwd, bwd): the unit the
+        end-to-end run pipelines behind that layer's host-to-device copies."""
+        q = self.q
+        q.nf4_quantize(L["W"], sse=True, packed=L["packed"], absmax=L["absmax"], sse_out=L["sse"],
+                       ws=self.ws)
+        q.double_quant(L["absmax"], code2=L["code2"], scale2=L["scale2"], mean=L["mean"], ws=self.ws)
+        q.qlora_linear_fwd(L["w"], L["x"], L["A"], L["B"], self.s, h=L["h"], ws=self.ws)
+        q.qlora_linear_bwd(L["w"], L["x"], L["dY"], L["A"], L["B"], self.s, dX=L["dX"], dA=L["dA"],
+                           dB=L["dB"], ws=self.ws)
+
+    def input_groups(self):
+        """inputs(), grouped by the unit that first needs them: one group per layer, then
+        the per-channel layer's."""
+        c = self.cq
+        return [[L["W"], L["x"], L["A"], L["B"], L["dY"]] for L in self.layers] + \
+            [[c["W"], c["bits"], c["thr"], c["thr_off"], c["roff"], c["maps"], c["map_off"],
+              c["x"], c["A"], c["B"]]]
+
     def inputs(self):
         """Every tensor the step reads from outside (for the end-to-end copies)."""
         out = []
@@ -500,18 +519,34 @@ def run_ours(args):
     if not args.no_breakdown:
         extra = breakdown(wl, q, hbm, tc_sus)
     clocks.stop()
-    # end to end through the public API: pinned host inputs in, gradients out, per step
-    ins = wl.inputs()
-    host_in = [t.cpu().pin_memory() for t in ins]
+    # end to end through the public API: pinned host inputs in, gradients out, per step.
+    # The host-to-device copies run on a side stream in the order the layers need them;
+    # each layer's kernels wait only for that layer's copies, so later copies overlap
+    # earlier layers' compute. A step's copies start once the previous step's kernels are
+    # done (the device buffers are reused).
+    groups = wl.input_groups()
+    ins = [t for g in groups for t in g]
+    assert nbytes(ins) == nbytes(wl.inputs())
+    host_groups = [[t.cpu().pin_memory() for t in g] for g in groups]
     res = wl.results()
     host_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in res]
     h2d, d2h = nbytes(ins), nbytes(res)
     ke = max(1, min(K, 5))
+    copy_stream = torch.cuda.Stream(device=dev)
+    landed = [torch.cuda.Event() for _ in groups]
 
     def e2e_step():
-        for d, h in zip(ins, host_in):
-            d.copy_(h, non_blocking=True)
-        wl.step()
+        copy_stream.wait_stream(stream)
+        with torch.cuda.stream(copy_stream):
+            for g, hg, ev in zip(groups, host_groups, landed):
+                for d, h in zip(g, hg):
+                    d.copy_(h, non_blocking=True)
+                ev.record(copy_stream)
+        for L, ev in zip(wl.layers, landed):
+            stream.wait_event(ev)
+            wl.layer_step(L)
+        stream.wait_event(landed[-1])
+        wl.chanq()
         for h, d in zip(host_out, res):
             h.copy_(d, non_blocking=True)
     e2e_step()
