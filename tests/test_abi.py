@@ -104,6 +104,34 @@ def test_argument_checks_fail_before_any_launch(q):
     assert b"positive" in q.lib.qnf4_last_error()
 
 
+def test_argument_checks_of_the_next_rows(q):
+    fake = 1 << 20  # never dereferenced: every call below fails its host-side checks
+    nan = float("nan")
+    # layer statistics (error + sparsity): shape, NULL, alignment, tau, workspace
+    assert _st(q, "qnf4_nf4_layer_stats", fake, 4, 100, 0.01, fake, fake, fake, 1 << 20, None) == 2
+    assert _st(q, "qnf4_nf4_layer_stats", fake, 4, 64, 0.01, fake, None, fake, 1 << 20, None) == 1
+    assert _st(q, "qnf4_nf4_layer_stats", fake, 4, 64, 0.01, fake, fake + 8, fake, 1 << 20, None) == 3
+    assert _st(q, "qnf4_nf4_layer_stats", fake, 4, 64, -1.0, fake, fake, fake, 1 << 20, None) == 1
+    assert _st(q, "qnf4_nf4_layer_stats", fake, 4, 64, nan, fake, fake, fake, 1 << 20, None) == 1
+    assert _st(q, "qnf4_nf4_layer_stats", fake, 4, 64, 0.01, fake, fake, fake, 16, None) == 6
+    # row-sharded double quantization
+    assert _st(q, "qnf4_dq_sum", fake, 0, fake, fake, 1 << 20, None) == 2
+    assert _st(q, "qnf4_dq_sum", fake, 10, None, fake, 1 << 20, None) == 1
+    assert _st(q, "qnf4_dq_sum", fake, 10, fake, fake, 8, None) == 6
+    assert _st(q, "qnf4_double_quant_shard", fake, 10, 128, fake, 10, fake, fake, fake, None) == 1
+    assert _st(q, "qnf4_double_quant_shard", fake, 10, 256, fake, 9, fake, fake, fake, None) == 2
+    assert _st(q, "qnf4_double_quant_shard", fake, 10, 256, None, 10, fake, fake, fake, None) == 1
+    # LoftQ initialisation: shape, rank, steps, the Gram-matrix size limit
+    args = (fake, fake, fake, fake, fake, fake, fake, fake, 1 << 30, None)
+    assert _st(q, "qnf4_loftq_nf4", fake, 32, 100, 4, 5, *args) == 2
+    assert _st(q, "qnf4_loftq_nf4", fake, 32, 128, 0, 5, *args) == 1
+    assert _st(q, "qnf4_loftq_nf4", fake, 32, 128, 33, 5, *args) == 1
+    assert _st(q, "qnf4_loftq_nf4", fake, 32, 128, 4, 0, *args) == 1
+    assert _st(q, "qnf4_loftq_nf4", fake, 20000, 20032, 4, 5, *args) == 2
+    # per-channel table learner: bit width
+    assert _st(q, "qnf4_chanq_learn", fake, 4, 128, 3, fake, 8, fake, fake, fake, fake, None) == 1
+
+
 def test_workspace_sizes_are_positive_and_monotone(q):
     a = q.workspace_size(q._lib.OP_FWD, 4096, 4096, 16, 16)
     b = q.workspace_size(q._lib.OP_FWD, 4096, 4096, 4096, 16)
@@ -115,3 +143,7 @@ def test_workspace_sizes_are_positive_and_monotone(q):
         for M in (1, 8, 9, 16):
             assert 0 < q.workspace_size(q._lib.OP_FWD, N, K, M, 64) <= 8 << 20
     assert q.workspace_size(q._lib.OP_QUANTIZE, 4096, 4096) > 0
+    assert q.workspace_size(q._lib.OP_LAYER_STATS, 4096, 4096) > q.workspace_size(q._lib.OP_QUANTIZE, 4096, 4096)
+    # LoftQ: at least the bf16 target, the fp32 residual and the Gram matrix
+    N, K, r = 11008, 4096, 16
+    assert q.workspace_size(q._lib.OP_LOFTQ, N, K, 0, r) >= N * K * 6 + K * K * 4
