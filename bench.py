@@ -211,6 +211,7 @@ class Workload:
             L["dA"] = torch.empty(RANK, K, dtype=torch.float32, device=dev)
             L["dB"] = torch.empty(N, RANK, dtype=torch.float32, device=dev)
             for op, m in ((q._lib.OP_QUANTIZE, 0), (q._lib.OP_DOUBLE_QUANT, 0), (q._lib.OP_LAYER_STATS, 0),
+                          (q._lib.OP_QUANTIZE_WEIGHT, 0),
                           (q._lib.OP_FWD, M_TOK), (q._lib.OP_BWD, M_TOK)):
                 wsz = max(wsz, q.workspace_size(op, N, K, m, RANK))
             self.layers.append(L)
@@ -241,12 +242,12 @@ class Workload:
 
     # the pieces of one step
     def quantize(self):
+        # NF4 codes, constants, double quantization and the reconstruction SSE: two
+        # launches per layer (qnf4_quantize_weight)
         q = self.q
         for L in self.layers:
-            q.nf4_quantize(L["W"], sse=True, packed=L["packed"], absmax=L["absmax"],
-                           sse_out=L["sse"], ws=self.ws)
-            q.double_quant(L["absmax"], code2=L["code2"], scale2=L["scale2"], mean=L["mean"],
-                           ws=self.ws)
+            q.quantize_weight(L["W"], sse=True, out=L["w"], absmax=L["absmax"], sse_out=L["sse"],
+                              ws=self.ws)
 
     def fwd(self, ev=None):
         for i, L in enumerate(self.layers):
@@ -283,9 +284,8 @@ class Workload:
         """One layer's share of the step (quantize + double quant, fwd, bwd): the unit the
         end-to-end run pipelines behind that layer's host-to-device copies."""
         q = self.q
-        q.nf4_quantize(L["W"], sse=True, packed=L["packed"], absmax=L["absmax"], sse_out=L["sse"],
-                       ws=self.ws)
-        q.double_quant(L["absmax"], code2=L["code2"], scale2=L["scale2"], mean=L["mean"], ws=self.ws)
+        q.quantize_weight(L["W"], sse=True, out=L["w"], absmax=L["absmax"], sse_out=L["sse"],
+                          ws=self.ws)
         q.qlora_linear_fwd(L["w"], L["x"], L["A"], L["B"], self.s, h=L["h"], ws=self.ws)
         q.qlora_linear_bwd(L["w"], L["x"], L["dY"], L["A"], L["B"], self.s, dX=L["dX"], dA=L["dA"],
                            dB=L["dB"], ws=self.ws)

@@ -148,12 +148,29 @@ def double_quant_shard(absmax: torch.Tensor, total_sum: torch.Tensor, total_coun
     return code2, scale2, mean[:1]
 
 
-def quantize_weight(W: torch.Tensor) -> Nf4Weight:
-    """NF4 + double quantization of a bf16 [N, K] weight into an ``Nf4Weight``."""
+def quantize_weight(W: torch.Tensor, sse: bool = False, out: Nf4Weight | None = None,
+                    absmax=None, sse_out=None, ws=None):
+    """NF4 + double quantization of a bf16 [N, K] weight into an ``Nf4Weight`` (two
+    launches, qnf4_quantize_weight); with sse=True also the reconstruction SSE (float64
+    [1]): returns (weight, sse) then."""
+    _req(W, torch.bfloat16, "W")
     N, K = W.shape
-    packed, absmax = nf4_quantize(W)
-    code2, scale2, mean = double_quant(absmax)
-    return Nf4Weight(N, K, packed, code2, scale2, mean)
+    n = N * K
+    dev = W.device
+    if out is None:
+        out = Nf4Weight(N, K, torch.empty(n // 2, dtype=torch.uint8, device=dev),
+                        torch.empty(n // BLOCK1, dtype=torch.uint8, device=dev),
+                        torch.empty((n // BLOCK1 + BLOCK2 - 1) // BLOCK2, dtype=torch.float32, device=dev),
+                        torch.empty(4, dtype=torch.float32, device=dev)[:1])
+    absmax = absmax if absmax is not None else torch.empty(n // BLOCK1, dtype=torch.float32, device=dev)
+    s = None
+    if sse:
+        s = sse_out if sse_out is not None else torch.empty(2, dtype=torch.float64, device=dev)
+    wsb = _ws(workspace_size(_lib.OP_QUANTIZE_WEIGHT, N, K), W, ws)
+    _lib.call("qnf4_quantize_weight", W.data_ptr(), N, K, out.packed.data_ptr(), absmax.data_ptr(),
+              out.code2.data_ptr(), out.scale2.data_ptr(), out.mean.data_ptr(), _p(s),
+              wsb.data_ptr(), wsb.numel(), _stream(W))
+    return (out, s[:1]) if sse else out
 
 
 def dequant(w: Nf4Weight, dtype: torch.dtype = torch.float32, out=None) -> torch.Tensor:

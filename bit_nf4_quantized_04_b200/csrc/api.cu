@@ -893,6 +893,7 @@ size_t qnf4_workspace_size(int32_t op, int64_t N, int64_t K, int64_t M, int32_t 
   switch (op) {
     case QNF4_OP_QUANTIZE: return kQuantMaxGrid * sizeof(double);
     case QNF4_OP_LAYER_STATS: return 2 * kQuantMaxGrid * sizeof(double);
+    case QNF4_OP_QUANTIZE_WEIGHT: return 2 * kQuantMaxGrid * sizeof(double);
     case QNF4_OP_DOUBLE_QUANT: return kDqPartials * sizeof(double);
     case QNF4_OP_FWD: return plan_linear(A_NF4_K, N, K, M, r, false, num_sms()).total;
     case QNF4_OP_BWD: return plan_linear(A_NF4_MN, N, K, M, r, true, num_sms()).total;
@@ -937,6 +938,43 @@ qnf4_status qnf4_nf4_quantize(const void* W, int64_t N, int64_t K, int32_t block
       static_cast<const uint16_t*>(W), nblocks, reinterpret_cast<uint32_t*>(packed), absmax,
       nullptr, tab, g_wait_ns);
   return launched("nf4_quantize");
+}
+
+qnf4_status qnf4_quantize_weight(const void* W, int64_t N, int64_t K, uint8_t* packed, float* absmax,
+                                 uint8_t* code2, float* scale2, float* mean, double* sse, void* ws,
+                                 size_t ws_bytes, void* stream) {
+  if (N <= 0 || K <= 0) return fail(QNF4_ERR_SHAPE, "N and K must be positive");
+  if (K % 64) return fail(QNF4_ERR_SHAPE, "K must be a multiple of 64");
+  if (!W || !packed || !absmax || !code2 || !scale2 || !mean) return fail(QNF4_ERR_ARG, "NULL buffer");
+  for (const void* p : {W, static_cast<const void*>(packed), static_cast<const void*>(absmax),
+                        static_cast<const void*>(code2), static_cast<const void*>(scale2),
+                        static_cast<const void*>(mean)})
+    if (!al16(p)) return fail(QNF4_ERR_ALIGN, "buffers must be 16-byte aligned");
+  if (sse && !al16(sse)) return fail(QNF4_ERR_ALIGN, "buffers must be 16-byte aligned");
+  if (!ws || ws_bytes < qnf4_workspace_size(QNF4_OP_QUANTIZE_WEIGHT, N, K, 0, 0))
+    return fail(QNF4_ERR_WORKSPACE, "workspace too small");
+  qnf4_status st = quant_smem_attr();
+  if (st != QNF4_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t nblocks = N * K / 64;
+  const int grid = quant_grid(nblocks);
+  double* asum = static_cast<double*>(ws);
+  double* ssep = asum + kQuantMaxGrid;
+  const QuantTab tab = make_tab();
+  if (sse) {
+    k_nf4_quant<true, true><<<grid, kQThreads, kQSmem, s>>>(
+        static_cast<const uint16_t*>(W), nblocks, reinterpret_cast<uint32_t*>(packed), absmax, ssep,
+        tab, g_wait_ns, 0.f, nullptr, asum);
+  } else {
+    k_nf4_quant<true, false><<<grid, kQThreads, kQSmem, s>>>(
+        static_cast<const uint16_t*>(W), nblocks, reinterpret_cast<uint32_t*>(packed), absmax,
+        nullptr, tab, g_wait_ns, 0.f, nullptr, asum);
+  }
+  const int64_t nb2 = (nblocks + 255) / 256;
+  const int egrid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((nb2 + 7) / 8, num_sms() * 4)));
+  k_dq_encode<<<egrid, 256, 0, s>>>(absmax, nblocks, asum, grid, nblocks, code2, scale2, mean,
+                                    sse ? ssep : nullptr, grid, sse);
+  return launched("quantize_weight", 2);
 }
 
 qnf4_status qnf4_nf4_recon_error(const void* W, int64_t N, int64_t K, int32_t block1, double* sse,

@@ -102,7 +102,9 @@ QNF4_DEV bool warp_wait(uint64_t* bar, uint32_t parity, unsigned long long wait_
 // elements, one 16-byte shared load) and writes 4 packed bytes. Optional outputs:
 // WRITE -> packed codes and fp32 absmax; SSE -> per-CTA float64 partial sums of the
 // single-level squared round-trip error; CNT -> per-CTA float64 counts of the elements
-// with |w| < tau (the sparsity of "AQLoRA" §3.1), exact integers.
+// with |w| < tau (the sparsity of "AQLoRA" §3.1), exact integers; asum_part (optional,
+// with WRITE) -> per-CTA float64 sums of the block constants, the partials of the double
+// quantization's tensor mean.
 //
 // Code search (see Nf4Tables), for a block with absmax c > 0: the bin
 // k = round(w H/c + H) comes from one fused multiply-add with a magic constant
@@ -116,7 +118,8 @@ template <bool WRITE, bool SSE, bool CNT = false>
 __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
     k_nf4_quant(const uint16_t* __restrict__ W, int64_t nblocks, uint32_t* __restrict__ packed,
                 float* __restrict__ absmax, double* __restrict__ sse_part, QuantTab tab,
-                unsigned long long wait_ns, float tau = 0.f, double* __restrict__ cnt_part = nullptr) {
+                unsigned long long wait_ns, float tau = 0.f, double* __restrict__ cnt_part = nullptr,
+                double* __restrict__ asum_part = nullptr) {
   extern __shared__ uint8_t qsm_raw[];
   __shared__ __align__(8) uint64_t full[kQStages], empty[kQStages];
   __shared__ float s_thr[16];
@@ -124,6 +127,7 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
   __shared__ __align__(1024) float s_tc[2 * kMaxHalfBins + 1];
   __shared__ double s_red[kQWorkers];
   __shared__ unsigned long long s_cnt[kQWorkers];
+  __shared__ double s_asum[kQWorkers];
   __shared__ volatile int s_abort;
   uint8_t* qsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(qsm_raw) + 127) &
                                             ~static_cast<uintptr_t>(127));
@@ -147,6 +151,7 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
   __syncthreads();
 
   double acc = 0.0;
+  double asum = 0.0;       // this thread's block constants (asum_part; group leaders only)
   unsigned int below = 0;  // this thread's elements with |w| < tau (CNT)
   if (warp == kQWorkers) {
     // ---------------------------------------------------------------- producer
@@ -280,7 +285,10 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
           const uint32_t b2 = code[4] * 16u + code[5], b3 = code[6] * 16u + code[7];
           const uint32_t word = __byte_perm(__byte_perm(b0, b1, 0x1140), __byte_perm(b2, b3, 0x1140), 0x5410);
           packed[b * 8 + lane8] = word;
-          if (lane8 == 0) absmax[b] = c;
+          if (lane8 == 0) {
+            absmax[b] = c;
+            asum += static_cast<double>(c);
+          }
         }
         if (SSE) {
           sse += __shfl_xor_sync(0xffffffffu, sse, 1);
@@ -308,7 +316,17 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
     for (int o = 16; o > 0; o >>= 1) b += __shfl_xor_sync(0xffffffffu, b, o);
     if ((tid & 31) == 0 && warp < kQWorkers) s_cnt[warp] = b;
   }
+  if (WRITE && asum_part) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) asum += __shfl_xor_sync(0xffffffffu, asum, o);
+    if ((tid & 31) == 0 && warp < kQWorkers) s_asum[warp] = asum;
+  }
   __syncthreads();
+  if (WRITE && asum_part && tid == 0) {
+    double t = 0.0;
+    for (int i = 0; i < kQWorkers; ++i) t += s_asum[i];
+    asum_part[blockIdx.x] = t;  // exact: bf16-derived constants sum exactly in float64
+  }
   if (SSE && tid == 0) {
     double t = 0.0;
     for (int i = 0; i < kQWorkers; ++i) t += s_red[i];
@@ -321,9 +339,9 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
   }
 }
 
-// Sum n float64 partials in a fixed order (one CTA of 256 threads) into *out.
-__global__ void __launch_bounds__(256) k_sum_partials(const double* __restrict__ part, int n,
-                                                      double* __restrict__ out) {
+// Sum n float64 partials in a fixed order with the 256 threads of a CTA (all must call
+// it); the result is valid in thread 0.
+QNF4_DEV double block_sum_partials(const double* __restrict__ part, int n) {
   __shared__ double s[256];
   double t = 0.0;
   for (int i = threadIdx.x; i < n; i += 256) t += part[i];
@@ -333,7 +351,14 @@ __global__ void __launch_bounds__(256) k_sum_partials(const double* __restrict__
     if (threadIdx.x < o) s[threadIdx.x] += s[threadIdx.x + o];
     __syncthreads();
   }
-  if (threadIdx.x == 0) *out = s[0];
+  return s[0];
+}
+
+// Sum n float64 partials in a fixed order (one CTA of 256 threads) into *out.
+__global__ void __launch_bounds__(256) k_sum_partials(const double* __restrict__ part, int n,
+                                                      double* __restrict__ out) {
+  const double t = block_sum_partials(part, n);
+  if (threadIdx.x == 0) *out = t;
 }
 
 // ---------------------------------------------------------------------------
@@ -369,9 +394,17 @@ __global__ void __launch_bounds__(256) k_dq_encode(const float* __restrict__ c, 
                                                    const double* __restrict__ part, int npart,
                                                    int64_t count, uint8_t* __restrict__ code2,
                                                    float* __restrict__ scale2,
-                                                   float* __restrict__ mean_out) {
+                                                   float* __restrict__ mean_out,
+                                                   const double* __restrict__ sse_part = nullptr,
+                                                   int nsse = 0, double* __restrict__ sse_out = nullptr) {
   __shared__ float s_mu;
   const int lane = threadIdx.x & 31;
+  // (fused quantize path) CTA 0 also folds the quantizer's SSE partials, in the same
+  // order as k_sum_partials
+  if (sse_out && blockIdx.x == 0) {
+    const double t = block_sum_partials(sse_part, nsse);
+    if (threadIdx.x == 0) *sse_out = t;
+  }
   if (threadIdx.x < 32) {
     double t = 0.0;
     for (int i = lane; i < npart; i += 32) t += part[i];

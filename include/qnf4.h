@@ -71,7 +71,8 @@ enum {
   QNF4_OP_CHANQ_FWD = 4,    /* qnf4_chanq_linear_fwd                                 */
   QNF4_OP_CHANQ_BWD = 5,    /* qnf4_chanq_linear_bwd                                 */
   QNF4_OP_LOFTQ = 6,        /* qnf4_loftq_nf4                                        */
-  QNF4_OP_LAYER_STATS = 7   /* qnf4_nf4_layer_stats                                  */
+  QNF4_OP_LAYER_STATS = 7,  /* qnf4_nf4_layer_stats                                  */
+  QNF4_OP_QUANTIZE_WEIGHT = 8 /* qnf4_quantize_weight                                */
 };
 
 /* A double-quantized NF4 weight [QLoRA 贡献一/贡献二]. All pointers are device
@@ -126,6 +127,16 @@ QNF4_API qnf4_status qnf4_nf4_quantize(const void* W_bf16, int64_t N, int64_t K,
 QNF4_API qnf4_status qnf4_double_quant(const float* absmax, int64_t nb1, int32_t block2,
                               uint8_t* code2, float* scale2, float* mean,
                               void* ws, size_t ws_bytes, void* stream);
+
+/* [QLoRA 贡献一 + 贡献二; AQLoRA §3.1] The whole quantization of a bf16 weight [N, K] in two
+ * launches: packed NF4 codes and fp32 absmax (as qnf4_nf4_quantize), code2 / scale2 / mean
+ * (as qnf4_double_quant, bit for bit: the tensor mean's float64 sum is exact) and, when sse
+ * is not NULL, the reconstruction SSE (as qnf4_nf4_quantize's, bit for bit). The quantizer
+ * hands the constant sums to the encoder, which also folds the SSE. N, K > 0, K a multiple
+ * of 64. Workspace: QNF4_OP_QUANTIZE_WEIGHT. */
+QNF4_API qnf4_status qnf4_quantize_weight(const void* W_bf16, int64_t N, int64_t K, uint8_t* packed,
+                                 float* absmax, uint8_t* code2, float* scale2, float* mean,
+                                 double* sse, void* ws, size_t ws_bytes, void* stream);
 
 /* [QLoRA 贡献二] A matrix quantized as row shards (one per process): the tensor mean needs
  * the float64 sum of all its constants. qnf4_dq_sum writes this shard's sum to *sum (device,

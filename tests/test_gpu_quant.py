@@ -206,3 +206,38 @@ def test_row_sharded_quantization_is_bit_identical(q, N, K, world):
     # one process: the dist entry point reduces to the whole-matrix quantization
     w1 = dist.sharded_quantize_weight(W, N)
     assert torch.equal(w1.code2, whole.code2) and torch.equal(w1.mean, whole.mean)
+
+
+@pytest.mark.parametrize("N,K", [(33, 320), (4096, 11008), (300, 4096)])
+def test_fused_quantize_weight_matches_the_separate_calls(q, N, K):
+    # qnf4_quantize_weight (two launches: the quantizer hands its constant sums to the
+    # encoder, which also folds the SSE) against qnf4_nf4_quantize + qnf4_double_quant,
+    # bit for bit, and against the oracle
+    W = synth.llama_weight((N, K), 500 + N, std=0.02)
+    if N == 300:
+        W[7] = 0  # an all-zero row (zero constants) inside the tensor
+    Wc = W.cuda()
+    w, sse = q.quantize_weight(Wc, sse=True)
+    packed, absmax, sse2 = q.nf4_quantize(Wc, sse=True)
+    code2, scale2, mean = q.double_quant(absmax)
+    torch.cuda.synchronize()
+    assert torch.equal(w.packed, packed)
+    assert torch.equal(w.code2, code2) and torch.equal(w.scale2, scale2)
+    assert torch.equal(w.mean, mean)
+    assert sse.item() == sse2.item()
+    oq = oracle_quant(W)
+    assert np.array_equal(w.code2.cpu().numpy(), oq["code2"])
+    ref = onf4.recon_sse(f32(W))
+    assert abs(sse.item() - ref) <= 1e-5 * ref
+    # without the SSE output
+    w2 = q.quantize_weight(Wc)
+    assert torch.equal(w2.packed, packed) and torch.equal(w2.code2, code2)
+
+
+def test_fused_quantize_weight_all_zero(q):
+    z = torch.zeros(8, 256, dtype=torch.bfloat16, device="cuda")
+    w, sse = q.quantize_weight(z, sse=True)
+    torch.cuda.synchronize()
+    assert sse.item() == 0.0 and w.mean.item() == 0.0
+    assert torch.all(w.code2 == 0) and torch.all(w.scale2 == 0)
+    assert torch.all(w.packed == 0x77)
