@@ -110,6 +110,22 @@ def test_llama7b_prefill_q_proj_sampled(q):
     _run_nf4(q, 4096, 4096, 4096, 16, seed=1000, bwd=True, rows=rows)
 
 
+def test_llama7b_prefill_gate_and_down_sampled(q):
+    # the bench's launch configuration on the two other 7B shapes: gate (11008 x 4096: the
+    # last wave's tiles cut into contraction slices) and down (4096 x 11008: a contraction
+    # of 172 blocks, the backward's over N = 4096), fwd + bwd at 4096 tokens, r = 16
+    rows = np.array([0, 1, 255, 256, 1000, 2047, 3071, 4095])
+    _run_nf4(q, 11008, 4096, 4096, 16, seed=1001, bwd=True, rows=rows)
+    _run_nf4(q, 4096, 11008, 4096, 16, seed=1006, bwd=True, rows=rows)
+
+
+def test_llama13b_prefill_r64_sampled(q):
+    # the 13B-shaped configuration's attention projection at 8192 tokens, r = 64 (the
+    # adapter chunk spans four K = 16 sub-steps)
+    rows = np.array([0, 129, 4095, 4096, 8191])
+    _run_nf4(q, 5120, 5120, 8192, 64, seed=1300, bwd=True, rows=rows)
+
+
 def test_zero_adapter_is_base_only(q):
     N, K, M, r = 256, 512, 40, 8
     W, x, A, B, _ = _inputs(N, K, M, r, 31)
@@ -225,6 +241,35 @@ def test_chanq_linear_fwd(q, N, K, M, r):
     h = q.chanq_linear_fwd(dev(pk), roff.cuda(), bits.cuda(), maps.cuda(), map_off.cuda(),
                            dev(g), N, K, x.cuda(), A.cuda(), B.cuda(), s)
     assert_close(f64(h.cpu()), href, "chanq h")
+
+
+def test_chanq_linear_full_size_sampled(q):
+    # the per-channel configuration in the bench's launch configuration: 11008 x 4096 at
+    # 1/2/4 bits, 2048 tokens, r = 16; forward and backward on sampled token rows (dA, dB
+    # over all tokens)
+    N, K, M, r = 11008, 4096, 2048, 16
+    W, bits, maps, map_off, thr, thr_off, roff = _chanq_case(N, K, 610)
+    packed, roff_o, g, _ = chanq_oracle(W, bits, thr, thr_off)
+    x = synth.normal_bf16((M, K), 1.0, 611)
+    A = synth.normal_bf16((r, K), 0.01, 612)
+    B = synth.normal_bf16((N, r), 0.01, 613)
+    dY = synth.normal_bf16((M, N), 1.0, 614)
+    s = 2.0
+    wb = olin.base_bf16(ochq.dequant(packed, roff_o, bits.numpy(), maps.numpy(), map_off.numpy(),
+                                     g, N, K))
+    sel = np.array([0, 1, 127, 128, 1000, 2047])
+    xs, dYs = f64(x), f64(dY)
+    pk = np.zeros(max(packed.size, 16), np.uint8)
+    pk[: packed.size] = packed
+    args = (dev(pk), roff.cuda(), bits.cuda(), maps.cuda(), map_off.cuda(), dev(g), N, K)
+    h = q.chanq_linear_fwd(*args, x.cuda(), A.cuda(), B.cuda(), s)
+    assert_close(f64(h.cpu())[sel], olin.forward(xs[sel], wb, f64(A), f64(B), s), "chanq h (full)")
+    dX, dA, dB = q.chanq_linear_bwd(*args, x.cuda(), dY.cuda(), A.cuda(), B.cuda(), s)
+    torch.cuda.synchronize()
+    v = dYs @ f64(B)
+    assert_close(f64(dX.cpu())[sel], dYs[sel] @ wb + s * (v[sel] @ f64(A)), "chanq dX (full)")
+    assert_close(dA.cpu().double().numpy(), s * (v.T @ xs), "chanq dA (full)")
+    assert_close(dB.cpu().double().numpy(), s * (dYs.T @ (xs @ f64(A).T)), "chanq dB (full)")
 
 
 @pytest.mark.parametrize("N,K,M,r", [
