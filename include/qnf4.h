@@ -292,7 +292,9 @@ QNF4_API qnf4_status qnf4_chanq_learn(const void* W_bf16, int64_t N, int64_t K, 
  * qnf4_double_quant); R = W - Q; B = U S^(1/2), A = S^(1/2) V^T from the rank-r truncated
  * SVD U S V^T of R; errs[t] = ||W - Q - B A||_F^2 (float64, the discarded squared singular
  * values). The SVD goes through the Gram matrix of R in fp32 (cuBLAS sgemm, cuSOLVER syevd,
- * loaded at first use: QNF4_ERR_CUDA if they are absent). W_bf16 [N, K], K a multiple of 64,
+ * loaded at first use: QNF4_ERR_CUDA if they are absent; the first call on a device creates
+ * one handle of each, owned by the library for the process, and sets them to `stream`, so
+ * concurrent calls on different streams must not overlap). W_bf16 [N, K], K a multiple of 64,
  * 1 <= r <= min(N, K), min(N, K) <= 16384, steps >= 1. Outputs (device): the last step's
  * quantized base, A fp32 [r, K], B fp32 [N, r], errs [steps]. Workspace: QNF4_OP_LOFTQ. */
 QNF4_API qnf4_status qnf4_loftq_nf4(const void* W_bf16, int64_t N, int64_t K, int32_t r,
