@@ -884,6 +884,7 @@ qnf4_status qnf4_check(void* stream) {
   if (flag) {
     const unsigned int zero = 0;
     cudaMemcpyToSymbol(g_qnf4_err, &zero, sizeof(zero));
+    if (flag == kErrEigensolve) return fail(QNF4_ERR_CUDA, "LoftQ eigensolve failed (cuSOLVER info != 0)");
     return fail(QNF4_ERR_TIMEOUT, "a kernel wait gave up (site %u)", flag);
   }
   return QNF4_OK;

@@ -13,6 +13,9 @@
 
 namespace qnf4 {
 
+// Device error code of a failed eigensolve (qnf4_check reports it as a CUDA error).
+constexpr unsigned int kErrEigensolve = 90;
+
 // target[n, k] = bf16(fp32(W[n, k] - sum_j B[n, j] A[j, k])), the sum in float64.
 __global__ void __launch_bounds__(256) k_loftq_target(const uint16_t* __restrict__ W,
                                                       const float* __restrict__ B,
@@ -78,7 +81,7 @@ __global__ void k_loftq_err(const float* __restrict__ w, int64_t m, int r,
   }
   if (threadIdx.x == 0) {
     *err = part[0];
-    if (*info != 0) set_err(90);
+    if (*info != 0) set_err(kErrEigensolve);
   }
 }
 

@@ -14,7 +14,8 @@
  * Conventions shared by every entry point:
  *   - All buffers are allocated and owned by the caller. The library never
  *     allocates or frees device memory and never synchronises the stream, except
- *     qnf4_check(), which synchronises to read the device error flag.
+ *     qnf4_check(), which synchronises to read the device error flag, and
+ *     qnf4_loftq_nf4(), whose first call on a device creates cuBLAS / cuSOLVER handles.
  *   - Pointers are device pointers unless the comment says "host".
  *   - Every device pointer must be 16-byte aligned (QNF4_ERR_ALIGN otherwise).
  *   - Matrices are row-major. W0 is [N, K] (N output features, K input features),
@@ -307,7 +308,8 @@ QNF4_API size_t qnf4_workspace_size(int32_t op, int64_t N, int64_t K, int64_t M,
 
 /* Synchronise `stream`, then report and clear the device error flag: QNF4_OK, or
  * QNF4_ERR_TIMEOUT if a bounded wait inside a kernel gave up since the last check,
- * or QNF4_ERR_CUDA if the stream holds a CUDA error. */
+ * or QNF4_ERR_CUDA if the stream holds a CUDA error or a LoftQ eigensolve reported
+ * failure (cuSOLVER info != 0). */
 QNF4_API qnf4_status qnf4_check(void* stream);
 
 /* Upper bound, in nanoseconds, on any single wait inside a kernel before it gives
