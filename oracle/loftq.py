@@ -15,8 +15,9 @@ The alternating steps, as the page's description reads plainly (A = 0, B = 0 at 
   3. B = U_r S_r^(1/2), A = S_r^(1/2) V_r^T.
 The objective after step t is e_t = ||W - Q_t - B A||_F^2 = sum_{i > r} s_i^2 (Eckart-Young).
 Readings (the page gives neither): W - B A enters the quantizer rounded to bf16 (the
-quantizer's input type), the SVD is of the float64 residual, and the outputs are the last
-step's quantized base and adapters. Parity of the GPU path is by properties (objectives
+quantizer's input type; parity unpinned for this rounding: no pin tells it from an
+unrounded target), the SVD is of the float64 residual, and the outputs are the last step's
+quantized base and adapters. Parity of the GPU path is by properties (objectives
 within a tolerance, codes equal on all but a tiny fraction), not bit-exact: its SVD works in
 fp32 through the Gram matrix.
 """
