@@ -178,34 +178,20 @@ struct GemmPlan {
 
 constexpr size_t kSmemLimit = 227 * 1024;
 
-// Tiling defaults (converter warp sets per CTA, CTAs per SM for thin N tiles).
-#ifndef QNF4_NSET_WIDE_TMEM
-#define QNF4_NSET_WIDE_TMEM 3
-#endif
-#ifndef QNF4_NSET_WIDE_SMEM
-#define QNF4_NSET_WIDE_SMEM 3
-#endif
-#ifndef QNF4_S2_THIN_TMEM
-#define QNF4_S2_THIN_TMEM 7
-#endif
-#ifndef QNF4_MIN_SPLIT_STEPS
-#define QNF4_MIN_SPLIT_STEPS 4
-#endif
-#ifndef QNF4_NSET_THIN
-#define QNF4_NSET_THIN 1
-#endif
-#ifndef QNF4_CTAS_THIN
-#define QNF4_CTAS_THIN 2
-#endif
+// Tiling (measured on the Llama shapes): three converter sets for wide tiles, one set
+// and two CTAs per SM for thin tiles, a 7-deep TMEM A ring for thin tiles, and
+// contraction slices of at least four steps.
+constexpr int kNsetWide = 3;
+constexpr int kNsetThin = 1;
+constexpr int kCtasThin = 2;
+constexpr int kS2ThinTmem = 7;
+constexpr int kMinSplitSteps = 4;
 
-#ifndef QNF4_TN_MAX
-#define QNF4_TN_MAX 256
-#endif
 int tn_for_tokens(int64_t M) {
   if (M <= 16) return 16;
   if (M <= 32) return 32;
   if (M <= 64) return 64;
-  if (M <= 128 || QNF4_TN_MAX == 128) return 128;
+  if (M <= 128) return 128;
   return 256;
 }
 
@@ -223,18 +209,16 @@ GemmPlan plan_gemm(int asrc, int64_t rows, int64_t cols, int64_t contraction, in
   // Thin N tiles (decode, rank-r GEMMs) are latency bound: give them two CTAs per SM
   // and a shallower dequant ring; wide tiles take the whole shared memory.
   const bool thin = tn <= 32;
-  p.ctas_per_sm = thin ? QNF4_CTAS_THIN : 1;
+  p.ctas_per_sm = thin ? kCtasThin : 1;
   // Wide tiles need several converter sets to keep the tensor core fed; thin tiles
   // run more CTAs per SM instead.
-  p.nset = src_deq(asrc) ? (thin ? QNF4_NSET_THIN : (src_tmem_a(asrc) ? QNF4_NSET_WIDE_TMEM
-                                                                       : QNF4_NSET_WIDE_SMEM))
-                         : 1;
+  p.nset = src_deq(asrc) ? (thin ? kNsetThin : kNsetWide) : 1;
   if (src_tmem_a(asrc)) {
     // TMEM A stages. Each is reusable only after the MMA that read it has completed,
     // so the ring depth bounds the steps in flight per MMA round trip: as deep as the
     // accumulator leaves room for (256 columns per CTA at two CTAs per SM, 512 at one).
     const int room = static_cast<int>(((p.ctas_per_sm == 2 ? 256u : 512u) - acc_cols(tn)) / 32u);
-    p.s2 = std::min(room, thin ? QNF4_S2_THIN_TMEM : 8);
+    p.s2 = std::min(room, thin ? kS2ThinTmem : 8);
     if (p.s2 > kMaxS2) p.s2 = kMaxS2;
   } else {
     p.s2 = src_deq(asrc) ? ((thin ? 2 : 4)) : 0;
@@ -260,17 +244,13 @@ GemmPlan plan_gemm(int asrc, int64_t rows, int64_t cols, int64_t contraction, in
   p.tail_tiles = static_cast<int>(tiles - p.full_tiles);
   int best = 1;
   if (p.tail_tiles > 0 && p.nsteps > 1) {
-    const int max_splits = std::max(1, p.nsteps / QNF4_MIN_SPLIT_STEPS);
+    const int max_splits = std::max(1, p.nsteps / kMinSplitSteps);
     best = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(max_splits, slots / p.tail_tiles)));
   }
   p.tail_sps = (p.nsteps + best - 1) / best;
   p.tail_splits = p.tail_sps > 0 ? (p.nsteps + p.tail_sps - 1) / p.tail_sps : 1;
   p.units = p.full_tiles + p.tail_tiles * p.tail_splits;
-#ifndef QNF4_PERSIST
-#define QNF4_PERSIST 1
-#endif
-  // QNF4_PERSIST=0: one unit per CTA, the hardware scheduler hands out the units
-  p.grid = static_cast<int>(std::max<int64_t>(1, QNF4_PERSIST ? std::min<int64_t>(p.units, slots) : p.units));
+  p.grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(p.units, slots)));
   return p;
 }
 
@@ -709,29 +689,42 @@ qnf4_status check_linear_args(int64_t N, int64_t K, int64_t M, int r, bool bwd,
 // ---------------------------------------------------------------------------
 // Workspace for the allocation-free forward (qnf4_qlora_linear_fwd_noalloc). A
 // file-scope device array: every GPU that loads the library holds it until exit.
+// 32 MiB covers the forward's split-K partial tiles at their largest (one 256-column
+// tile slice per CTA slot: 148 x 256 x 128 fp32 on a B200, 19.4 MB), the adapter
+// projection's partials and the bf16 (s u) rows (128 bytes per token) up to 65536
+// tokens, for every N, K and r <= 64.
 // ---------------------------------------------------------------------------
-constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;  // 8 MiB
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
-// Device address of the array on the current device, looked up once per device
-// (cudaGetSymbolAddress with that device current); nullptr and a message on failure.
+// Device address of the array on each device, looked up once per device with that
+// device current (cudaGetSymbolAddress); later calls read the cached address without
+// taking the lock. nullptr and a message on failure.
 void* noalloc_scratch_ptr() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+  constexpr int kMaxDev = 64;
+  static std::atomic<void*> cache[kMaxDev] = {};
   static std::mutex mu;
-  static std::vector<void*> cache;
-  std::lock_guard<std::mutex> lk(mu);
-  if (static_cast<int>(cache.size()) <= dev) cache.resize(dev + 1, nullptr);
-  if (!cache[dev]) {
-    void* p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess) {
-      fail(QNF4_ERR_CUDA, "scratch address: %s", cudaGetErrorString(e));
-      return nullptr;
-    }
-    cache[dev] = p;
+  int dev = 0;
+  const cudaError_t ge = cudaGetDevice(&dev);
+  if (ge != cudaSuccess) {
+    fail(QNF4_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(ge));
+    return nullptr;
   }
-  return cache[dev];
+  if (dev < 0 || dev >= kMaxDev) {
+    fail(QNF4_ERR_CUDA, "device %d out of range for the built-in scratch (at most %d devices)", dev, kMaxDev);
+    return nullptr;
+  }
+  if (void* p = cache[dev].load(std::memory_order_acquire)) return p;
+  std::lock_guard<std::mutex> lk(mu);
+  if (void* p = cache[dev].load(std::memory_order_relaxed)) return p;
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+  if (e != cudaSuccess) {
+    fail(QNF4_ERR_CUDA, "scratch address: %s", cudaGetErrorString(e));
+    return nullptr;
+  }
+  cache[dev].store(p, std::memory_order_release);
+  return p;
 }
 // ---------------------------------------------------------------------------
 // Dense linear algebra for the LoftQ initialisation's truncated SVD: cuBLAS (sgemm) and
@@ -848,18 +841,6 @@ const char* qnf4_last_error(void) { return g_last.c_str(); }
 
 unsigned long long qnf4_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
-#ifdef QNF4_WAIT_STATS
-// Tracing builds only (not declared in the public header): copy and clear the
-// per-site wait-cycle counters of the GEMM kernel.
-extern "C" QNF4_API int qnf4_debug_wait_stats(unsigned long long out[64]) {
-  cudaDeviceSynchronize();
-  if (cudaMemcpyFromSymbol(out, g_wait_cycles, 64 * sizeof(unsigned long long)) != cudaSuccess)
-    return 1;
-  static const unsigned long long zero[64] = {};
-  cudaMemcpyToSymbol(g_wait_cycles, zero, sizeof(zero));
-  return 0;
-}
-#endif
 
 qnf4_status qnf4_set_timing_events(void* start, void* stop) {
   if ((start == nullptr) != (stop == nullptr)) return fail(QNF4_ERR_ARG, "give both events or neither");

@@ -18,6 +18,14 @@ __device__ unsigned int g_qnf4_err = 0;
 
 QNF4_DEV void set_err(unsigned int code) { atomicCAS(&g_qnf4_err, 0u, code); }
 
+// Deadline of a drain: once a kernel gives up, it still waits for its own copies and
+// MMAs in flight before it frees shared and tensor memory, however short the caller's
+// wait limit; those always finish unless the hardware itself has stopped.
+constexpr unsigned long long kDrainFloorNs = 1000000000ull;
+QNF4_DEV unsigned long long drain_ns(unsigned long long wait_ns) {
+  return wait_ns > kDrainFloorNs ? wait_ns : kDrainFloorNs;
+}
+
 QNF4_DEV uint64_t globaltimer() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

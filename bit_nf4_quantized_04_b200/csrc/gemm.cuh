@@ -63,12 +63,7 @@ __host__ __device__ constexpr bool src_packed_tma(int a) {
 __host__ __device__ constexpr bool src_table_tma(int a) { return a == A_CHANQ_MN; }
 constexpr uint32_t kTTile = 64u * 16u * 4u;
 // A operand staged in tensor memory (written by tcgen05.st) instead of shared memory
-#ifndef QNF4_NF4K_TMEM_A
-#define QNF4_NF4K_TMEM_A 1
-#endif
-__host__ __device__ constexpr bool src_tmem_a(int a) {
-  return QNF4_NF4K_TMEM_A && (a == A_NF4_K || a == A_CHANQ_K);
-}
+__host__ __device__ constexpr bool src_tmem_a(int a) { return a == A_NF4_K || a == A_CHANQ_K; }
 __host__ __device__ constexpr int gemm_threads(int nset) { return 64 + 128 * nset; }
 
 // TMEM columns: the fp32 accumulator (a power of two >= tn, at least 32), then
@@ -164,38 +159,9 @@ __host__ __device__ inline SmemPlan smem_plan(int asrc, int tn, int s1, int s2, 
 // ---------------------------------------------------------------------------
 // device helpers
 // ---------------------------------------------------------------------------
-#ifdef QNF4_WAIT_STATS
-// Tracing build only: clock cycles spent blocked at each wait site (index = site,
-// 0..63), summed over all threads that wait there. Read with qnf4_debug_wait_stats.
-__device__ unsigned long long g_wait_cycles[64];
-// per-CTA partial sums (shared-memory atomics), added to g_wait_cycles once at exit
-__shared__ unsigned long long s_wait_cycles[64];
-#endif
-
-// Tracing build: clock cycles of a code span, per warp (lane 0), at a wait-stat site.
-#ifdef QNF4_WAIT_STATS
-#define QNF4_TSTAMP(v) const long long v = clock64()
-#define QNF4_TSPAN(site, v)                                                                    \
-  do {                                                                                         \
-    if ((threadIdx.x & 31) == 0)                                                               \
-      atomicAdd(&s_wait_cycles[site], static_cast<unsigned long long>(clock64() - (v)));       \
-  } while (0)
-#else
-#define QNF4_TSTAMP(v)
-#define QNF4_TSPAN(site, v)
-#endif
-
 QNF4_DEV bool wait_or_abort(uint64_t* bar, uint32_t parity, unsigned long long wait_ns,
                             volatile int* abort_flag, unsigned int site) {
   if (mbar_try_wait(bar, parity)) return true;
-#ifdef QNF4_WAIT_STATS
-  const long long c0 = clock64();
-  struct Acc {
-    long long c0;
-    unsigned int site;
-    QNF4_DEV ~Acc() { atomicAdd(&s_wait_cycles[site & 63], static_cast<unsigned long long>(clock64() - c0)); }
-  } acc{c0, site};
-#endif
   const uint64_t t0 = globaltimer();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -408,12 +374,6 @@ struct ConvCursor {
   }
 };
 
-// Converter steps of the next unit staged before the previous unit's epilogue (per
-// CTA, at most S2: those steps wait only for MMAs of earlier units).
-#ifndef QNF4_EPI_AHEAD
-#define QNF4_EPI_AHEAD -1  // -1: one step per converter set
-#endif
-
 // ---------------------------------------------------------------------------
 // the kernel
 // ---------------------------------------------------------------------------
@@ -447,9 +407,6 @@ __global__ void __launch_bounds__(gemm_threads(NSET), MINB)
   const int u0 = blockIdx.x;
   const int ustep = gridDim.x;
   const uint32_t ncols = tmem_cols(ASRC, g.tn, S2);
-#ifdef QNF4_WAIT_STATS
-  const long long g_t_start = clock64();
-#endif
   const uint32_t a_col = acc_cols(g.tn);  // first TMEM column of the A stages
 
   if (threadIdx.x == 0) {
@@ -467,9 +424,6 @@ __global__ void __launch_bounds__(gemm_threads(NSET), MINB)
     fence_mbar_init();
   }
   if (threadIdx.x < 16) s_lv[threadIdx.x] = g.levels[threadIdx.x];
-#ifdef QNF4_WAIT_STATS
-  if (threadIdx.x < 64) s_wait_cycles[threadIdx.x] = 0;
-#endif
   if (warp == 1) {
     tmem_alloc(&s_tmem, ncols);
     tmem_relinquish();
@@ -551,7 +505,7 @@ __global__ void __launch_bounds__(gemm_threads(NSET), MINB)
       for (int s = 0; s < nslots && !late; ++s) {
         const int j = s + S1 * ((issued - 1 - s) / S1);
         while (!mbar_try_wait(&full1[s], (j / S1) & 1)) {
-          if (globaltimer() - t0 > g.wait_ns) {
+          if (globaltimer() - t0 > drain_ns(g.wait_ns)) {
             set_err(12);
             late = true;
             break;
@@ -651,7 +605,7 @@ __global__ void __launch_bounds__(gemm_threads(NSET), MINB)
       mma_commit(&fin_bar);
       const uint64_t t0 = globaltimer();
       while (!mbar_try_wait(&fin_bar, 0)) {
-        if (globaltimer() - t0 > g.wait_ns) {
+        if (globaltimer() - t0 > drain_ns(g.wait_ns)) {
           set_err(25);
           break;
         }
@@ -709,13 +663,11 @@ __global__ void __launch_bounds__(gemm_threads(NSET), MINB)
     // CTA has aborted, so all take the same path through the named barriers.
     auto epilogue = [&](int u, int k) -> bool {
       wait_or_abort(&acc_bar, k & 1, g.wait_ns, &s_abort, 41);
-      QNF4_TSTAMP(te0);
       named_sync(1, NCONV);
       if (ct == 0) s_last = s_abort ? 0 : 2;
       named_sync(1, NCONV);
       const bool have = s_last == 2;
       named_sync(1, NCONV);
-      QNF4_TSPAN(44, te0);
       if (!have) return false;
       tc_fence_after();
       const Unit w = unit_of(g, u);
@@ -752,12 +704,9 @@ __global__ void __launch_bounds__(gemm_threads(NSET), MINB)
         }
         tc_fence_before();
         mbar_arrive(&acc_empty);
-        QNF4_TSPAN(42, te0);
-        QNF4_TSTAMP(te1);
         // the adapter tile is free for its next write once every piece has left it
         if (t == 0) bulk_wait_read0();
         named_sync(1, NCONV);
-        QNF4_TSPAN(43, te1);
       } else if (w.splits == 1) {
         for (int ck = set; ck < nchunk; ck += NSET) {
           const int c0 = ck * 16;
@@ -1046,10 +995,10 @@ __global__ void __launch_bounds__(gemm_threads(NSET), MINB)
       }
     };
 
-    // The unit loop. Steps of unit k with i < ahead are converted before the
-    // epilogue of unit k-1 (they wait only for MMAs of earlier units), so the MMA
-    // has work the moment the accumulator is free again.
-    const int ahead = QNF4_EPI_AHEAD >= 0 ? min(QNF4_EPI_AHEAD, S2) : min(NSET, S2);
+    // The unit loop. Each set converts its first step of unit k before the epilogue
+    // of unit k-1 (those steps wait only for MMAs of earlier units), so the MMA has
+    // work the moment the accumulator is free again.
+    const int ahead = min(NSET, S2);
     int rbase = 0;  // ring position of the unit's first step
     int up = -1;    // the previous unit, while its epilogue is still due
     // One pass per unit of this CTA and a last one for the final epilogue; the
@@ -1102,18 +1051,7 @@ __global__ void __launch_bounds__(gemm_threads(NSET), MINB)
     tc_fence_before();
   }
 
-#ifdef QNF4_WAIT_STATS
-  if (lane == 0) {
-    // per-warp active time: 60 = producer, 61 = MMA, 62 = converters (sum of warps)
-    const unsigned int slot = warp == 0 ? 60 : (warp == 1 ? 61 : 62);
-    atomicAdd(&s_wait_cycles[slot], static_cast<unsigned long long>(clock64() - g_t_start));
-  }
-#endif
   __syncthreads();
-#ifdef QNF4_WAIT_STATS
-  if (threadIdx.x < 64 && s_wait_cycles[threadIdx.x])
-    atomicAdd(&g_wait_cycles[threadIdx.x], s_wait_cycles[threadIdx.x]);
-#endif
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, ncols);

@@ -188,7 +188,7 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
       const uint64_t t0 = globaltimer();
       for (int64_t jj = max(static_cast<int64_t>(0), issued - kQStages); jj < issued; ++jj) {
         while (!mbar_try_wait(&full[jj % kQStages], static_cast<uint32_t>((jj / kQStages) & 1))) {
-          if (globaltimer() - t0 > wait_ns) {
+          if (globaltimer() - t0 > drain_ns(wait_ns)) {
             set_err(52);
             break;
           }

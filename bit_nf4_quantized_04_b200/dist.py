@@ -130,9 +130,14 @@ def shard_rows(N: int, K: int, world: int, rank: int) -> tuple[int, int]:
 def sharded_double_quant(absmax: torch.Tensor, total_count: int, group=None,
                          sum_fn: Callable | None = None, encode_fn: Callable | None = None):
     """Double quantization of this rank's row shard of one matrix ("QLoRA", 贡献二): the
-    shard's float64 constant sum is all-reduced (exact: bf16-derived constants sum exactly
-    in float64, so the mean is bit-identical to one process), then the shard is encoded
-    with the matrix's mean. `sum_fn(absmax)` -> float64 tensor [1], `encode_fn(absmax,
+    shard's float64 constant sum is all-reduced, then the shard is encoded with the
+    matrix's mean. The result is bit-identical to one process when every float64 partial
+    sum is exact, which holds when the constants' binades span at most
+    53 - 8 - ceil(log2(count)) (8 significant bits per bf16 constant, log2(count) carry
+    bits): 25 binades at 13B-layer size, far more than trained or synthetic Llama
+    weights span. A matrix with both tiny and normal nonzero block maxima beyond that
+    span may round its mean differently depending on the all-reduce order (all-zero
+    blocks add exact zeros and do not count). `sum_fn(absmax)` -> float64 tensor [1], `encode_fn(absmax,
     total_sum, total_count)` -> (code2, scale2, mean); by default the library's qnf4_dq_sum
     and qnf4_double_quant_shard."""
     world, _ = _world(group)

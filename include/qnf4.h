@@ -171,14 +171,17 @@ QNF4_API qnf4_status qnf4_qlora_linear_fwd(const qnf4_weight* w, const void* x, 
  * device memory: code that runs where cudaMalloc is unavailable or forbidden (an
  * allocator callback, a host hook inside a pre-planned inference engine, a caller
  * that owns no device allocator). The pages have no counterpart; this is a library
- * convenience. The workspace is a file-scope device array of 8 MiB in this library,
+ * convenience. The workspace is a file-scope device array of 32 MiB in this library,
  * held by every GPU that loads it until the process exits. Shapes whose workspace
- * (qnf4_workspace_size(QNF4_OP_FWD, N, K, M, r)) exceeds 8 MiB are rejected with
- * QNF4_ERR_WORKSPACE before any launch. The first call on a device looks up the
+ * (qnf4_workspace_size(QNF4_OP_FWD, N, K, M, r)) exceeds 32 MiB are rejected with
+ * QNF4_ERR_WORKSPACE before any launch; on a 148-SM B200 every N, K and r <= 64 fits
+ * up to M = 65536 tokens (the split-K partial tiles take at most 19.4 MB, the bf16
+ * adapter projection 128 bytes per token). The first call on a device looks up the
  * array's device address (once per device); make that first call before any stream
  * capture. All calls share the one array and it keeps the last call's contents, so
  * calls that overlap on the GPU (concurrent streams, or devices sharing a context)
- * race; calls ordered on one stream are safe. Results equal qnf4_qlora_linear_fwd. */
+ * race; calls ordered on one stream are safe. It runs the same kernels with the same
+ * tiling as qnf4_qlora_linear_fwd, so its results are bit-identical to that call's. */
 QNF4_API qnf4_status qnf4_qlora_linear_fwd_noalloc(const qnf4_weight* w, const void* x, int64_t M,
                                                    const void* A, const void* B, int32_t r,
                                                    float scale, void* h, void* stream);
