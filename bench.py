@@ -16,8 +16,10 @@ with every other piece of the step inside the timed region.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-Multi-GPU (torchrun): each rank runs its own copy of the step (independent layer
-sets, no collective on the data path: weak scaling); the time is the max over ranks.
+Multi-GPU: ``--gpus N`` without a torchrun environment relaunches itself under
+torch.distributed.run with N ranks on this node (127.0.0.1); each rank runs its own copy
+of the step (independent layer sets, no collective on the data path: weak scaling) and
+the time is the max over ranks.
 --impl reference times the CPU oracle (the plain NumPy restatement of the pages) on
 a bounded sample of the same step on the host cores.
 """
@@ -176,6 +178,21 @@ def oracle_sample(rows: int = 4096, m: int = 128):
             f"error + dequant, then fwd+bwd on {m} of 4096 tokens (r={r}); "
             "TFLOP/s = sample fwd+bwd FLOPs / time")
     return flops / dt / 1e12, dt, desc, flops
+
+
+ORACLE_ROWS = 512  # the bounded sample both the reference arm and cpu_baseline time
+
+
+def oracle_repeated(seconds: float):
+    """The oracle on the step's bounded sample (ORACLE_ROWS rows of q_proj, 128 tokens),
+    repeated until `seconds` have passed: (TFLOP/s, seconds, description, repeats)."""
+    tot, fl, n, desc = 0.0, 0.0, 0, ""
+    while tot < seconds or n == 0:
+        _, dt, desc, f = oracle_sample(rows=ORACLE_ROWS)
+        tot += dt
+        fl += f
+        n += 1
+    return fl / tot / 1e12, tot, desc, n
 
 
 # ------------------------------------------------------------------------------ GPU arm
@@ -346,8 +363,10 @@ def lloyd_t0(bits: int):
     return [float((float(lv[k]) + float(lv[k + 1])) * 0.5) for k in range(15)]
 
 
-def breakdown(wl, q, hbm, tc_sus):
-    """Per-row throughput, each timed alone (short loops, L2-exceeding inputs)."""
+def breakdown(wl, q, hbm, tc):
+    """Per-row throughput, each timed alone (short loops, L2-exceeding inputs). Tensor
+    rows are fractions of `tc`, the burst bf16 peak (each loop runs well under a second at
+    full clock)."""
     st = torch.cuda.current_stream()
     out = {}
     nparam = sum(N * K for N, K in layer_shapes())
@@ -367,9 +386,9 @@ def breakdown(wl, q, hbm, tc_sus):
     ff = sum(fwd_flops(N, K, M_TOK, RANK) for N, K in layer_shapes())
     bf = sum(bwd_flops(N, K, M_TOK, RANK) for N, K in layer_shapes())
     t = time_loop(wl.fwd, 5, st)
-    out["fwd_prefill"] = {"TFLOPs": round(ff / t / 1e12, 1), "frac_tc": round(ff / t / 1e12 / tc_sus, 3)}
+    out["fwd_prefill"] = {"TFLOPs": round(ff / t / 1e12, 1), "frac_tc": round(ff / t / 1e12 / tc, 3)}
     t = time_loop(wl.bwd, 5, st)
-    out["bwd_prefill"] = {"TFLOPs": round(bf / t / 1e12, 1), "frac_tc": round(bf / t / 1e12 / tc_sus, 3)}
+    out["bwd_prefill"] = {"TFLOPs": round(bf / t / 1e12, 1), "frac_tc": round(bf / t / 1e12 / tc, 3)}
     c = wl.cq
     t = time_loop(lambda: q.chanq_quantize(c["W"], c["bits"], c["thr"], c["thr_off"], c["roff"],
                                            packed=c["packed"], absmax=c["absmax"]), 10, st)
@@ -379,13 +398,13 @@ def breakdown(wl, q, hbm, tc_sus):
     t = time_loop(lambda: q.chanq_linear_fwd(c["packed"], c["roff"], c["bits"], c["maps"],
                                              c["map_off"], c["absmax"], CQ_N, CQ_K, c["x"], c["A"],
                                              c["B"], wl.s, h=c["h"], ws=wl.ws), 5, st)
-    out["chanq_fwd"] = {"TFLOPs": round(cf / t / 1e12, 1), "frac_tc": round(cf / t / 1e12 / tc_sus, 3)}
+    out["chanq_fwd"] = {"TFLOPs": round(cf / t / 1e12, 1), "frac_tc": round(cf / t / 1e12 / tc, 3)}
     cb = bwd_flops(CQ_N, CQ_K, CQ_M, RANK)
     t = time_loop(lambda: q.chanq_linear_bwd(c["packed"], c["roff"], c["bits"], c["maps"],
                                              c["map_off"], c["absmax"], CQ_N, CQ_K, c["x"], c["dY"],
                                              c["A"], c["B"], wl.s, dX=c["dX"], dA=c["dA"],
                                              dB=c["dB"], ws=wl.ws), 5, st)
-    out["chanq_bwd"] = {"TFLOPs": round(cb / t / 1e12, 1), "frac_tc": round(cb / t / 1e12 / tc_sus, 3)}
+    out["chanq_bwd"] = {"TFLOPs": round(cb / t / 1e12, 1), "frac_tc": round(cb / t / 1e12 / tc, 3)}
     # the weighted Lloyd-Max learner of that layer's tables at 1, 2 and 4 bits (8
     # iterations each), e.g. for the precision allocation's per-channel errors; bound by
     # float64 arithmetic, reported as weight bytes read per second and time per layer
@@ -401,10 +420,10 @@ def breakdown(wl, q, hbm, tc_sus):
     t = time_loop(lambda: q.loftq_nf4(c["W"], RANK, 5, ws=lws), 2, st)
     out["loftq_init"] = {"ms": round(t * 1e3, 2), "steps": 5, "rank": RANK}
     del lws
-    # decode (memory-bound): rotate over weight copies whose total exceeds L2 twice over
+    # decode (memory-bound): rotate over weight copies totalling at least 4x the L2
     l2 = torch.cuda.get_device_properties(wl.dev).L2_cache_size
     wbytes = sum(L["w"].nbytes() for L in wl.layers)
-    copies = max(2, int(2 * l2 // wbytes) + 1)
+    copies = max(2, -(-4 * l2 // wbytes))
     pool = [[q.Nf4Weight(L["N"], L["K"], L["packed"].clone(), L["code2"].clone(),
                          L["scale2"].clone(), L["mean"].clone()[:1]) for L in wl.layers]
             for _ in range(copies)]
@@ -439,6 +458,176 @@ def breakdown(wl, q, hbm, tc_sus):
     out["decode_fwd"]["pool_copies"] = copies
     out["decode_fwd"]["launch"] = "CUDA graph of all copies x 7 layers, PDL edges"
     q.check()
+    return out
+
+
+def graphed(fn):
+    """fn captured once into a CUDA graph (after one eager call, so every lazy set-up of
+    the library and of torch has happened); returns the graph's replay."""
+    fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    g.replay()
+    torch.cuda.synchronize()
+    return g.replay
+
+
+def arm_seconds(fn, seconds, stream):
+    """Seconds per call of fn over a region of at least `seconds` (the iteration count is
+    taken from one calibration call)."""
+    t1 = time_loop(fn, 1, stream)
+    iters = max(1, int(-(-seconds // max(t1, 1e-7))))
+    return time_loop(fn, iters, stream), iters
+
+
+def protocol(wl, q, hbm, tc_burst, tc_sus, dev, seconds=2.0, sessions=3):
+    """The timing protocol of the AQLoRA page's speed measurements: every arm runs for a
+    fixed duration (>= `seconds`), a duplicate of the step arm measures the noise floor,
+    and the whole session of arms is repeated `sessions` times; per arm the median and
+    the spread (max - min) / median over sessions. Quantize, forward, backward and decode
+    arms replay CUDA graphs; the decode arm rotates over weight copies totalling >= 4x L2."""
+    st = torch.cuda.current_stream()
+    nparam = sum(N * K for N, K in layer_shapes())
+    ff = sum(fwd_flops(N, K, M_TOK, RANK) for N, K in layer_shapes())
+    bf = sum(bwd_flops(N, K, M_TOK, RANK) for N, K in layer_shapes())
+    quant = graphed(wl.quantize)
+    fwd = graphed(wl.fwd)
+    bwd = graphed(wl.bwd)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    wbytes = sum(L["w"].nbytes() for L in wl.layers)
+    copies = max(2, -(-4 * l2 // wbytes))
+    pool = [[q.Nf4Weight(L["N"], L["K"], L["packed"].clone(), L["code2"].clone(),
+                         L["scale2"].clone(), L["mean"].clone()[:1]) for L in wl.layers]
+            for _ in range(copies)]
+    xs = [L["x"][:16].contiguous() for L in wl.layers]
+    hs = [torch.empty(16, L["N"], dtype=torch.bfloat16, device=dev) for L in wl.layers]
+
+    def dec_all():
+        for ws_ in pool:
+            for i, L in enumerate(wl.layers):
+                q.qlora_linear_fwd(ws_[i], xs[i], L["A"], L["B"], wl.s, h=hs[i], ws=wl.ws)
+    dec = graphed(dec_all)
+    dbytes = sum(N * K * (0.5 + 1 / 64 + 4 / 16384) + 16 * K * 2 + RANK * (N + K) * 2 + 16 * N * 2
+                 for N, K in layer_shapes())
+    sf = step_flops()
+    arms = {
+        "step": (wl.step, lambda t: sf / t / 1e12, "TFLOP/s"),
+        "step_dup": (wl.step, lambda t: sf / t / 1e12, "TFLOP/s"),
+        "quant_dq_sse": (quant, lambda t: nparam * 2.5159 / t / 1e9, "GB/s"),
+        "fwd_prefill": (fwd, lambda t: ff / t / 1e12, "TFLOP/s"),
+        "bwd_prefill": (bwd, lambda t: bf / t / 1e12, "TFLOP/s"),
+        "decode_M16": (dec, lambda t: dbytes * copies / t / 1e9, "GB/s"),
+    }
+    vals = {k: [] for k in arms}
+    clocks = Clocks(dev.index if dev.index is not None else 0)
+    for _ in range(sessions):
+        for k, (fn, conv, _) in arms.items():
+            t, _ = arm_seconds(fn, seconds, st)
+            vals[k].append(conv(t))
+    clocks.stop()
+    q.check()
+    out = {"seconds_per_arm": seconds, "sessions": sessions, "clocks": clocks.summary(),
+           "decode_pool_copies": copies, "arms": {}}
+    for k, (_, _, unit) in arms.items():
+        v = vals[k]
+        med = statistics.median(v)
+        row = {"median": round(med, 2), "unit": unit,
+               "spread": round((max(v) - min(v)) / med, 4), "sessions": [round(x, 2) for x in v]}
+        if unit == "GB/s":
+            row["frac_hbm"] = round(med / hbm, 3)
+        else:
+            row["frac_tc_burst"] = round(med / tc_burst, 3)
+            row["frac_tc_sustained"] = round(med / tc_sus, 3)
+        out["arms"][k] = row
+    out["noise_floor"] = round(statistics.median(
+        [abs(a - b) / a for a, b in zip(vals["step"], vals["step_dup"])]), 4)
+    return out
+
+
+def stack13b(q, dev, hbm, tc, seconds=2.0):
+    """The Llama-2-13B-shaped stack (40 layers x {5120^2 x4, 13824x5120 x2, 5120x13824},
+    280 matrices, 12.69 B parameters, per-matrix std drawn from U[0.01, 0.04]): the
+    AQLoRA profiling pass over the whole stack (NF4 + double quantization + the NF4
+    reconstruction SSE of every matrix, qnf4_quantize_weight), the ranking that keeps the
+    top-8 matrices by SSE per parameter in 16-bit, then forward + backward of every
+    matrix at 8192 tokens with r = 64, alpha = 128, the 8 protected ones through the dense
+    path. Timed: the profiling pass (GB/s at 2.5159 B/param) and the fwd + bwd pass
+    (TFLOP/s), each over a region of at least `seconds`."""
+    import synth
+    st = torch.cuda.current_stream()
+    shapes = synth.llama13b_stack()
+    stds = synth.llama13b_stds()
+    M, r, alpha, topk = 8192, 64, 128.0, 8
+    s = alpha / r
+    Ws, wq = [], []
+    for i, sh in enumerate(shapes):
+        Ws.append(synth.llama_weight((sh.N, sh.K), synth.SEED_W + 300 + i, std=float(stds[i]),
+                                     device=dev))
+        n = sh.N * sh.K
+        wq.append(q.Nf4Weight(sh.N, sh.K, torch.empty(n // 2, dtype=torch.uint8, device=dev),
+                              torch.empty(n // 64, dtype=torch.uint8, device=dev),
+                              torch.empty((n // 64 + 255) // 256, dtype=torch.float32, device=dev),
+                              torch.empty(4, dtype=torch.float32, device=dev)[:1]))
+    nmax = max(sh.N * sh.K for sh in shapes)
+    absmax = torch.empty(nmax // 64, dtype=torch.float32, device=dev)
+    sse = torch.zeros(len(shapes), 2, dtype=torch.float64, device=dev)
+    kinds = sorted({(sh.N, sh.K) for sh in shapes})
+    io = {}
+    wsz = q.workspace_size(q._lib.OP_QUANTIZE_WEIGHT, nmax, 64)
+    for j, (N, K) in enumerate(kinds):
+        io[(N, K)] = dict(
+            x=synth.normal_bf16((M, K), 1.0, synth.SEED_X + 300 + j, device=dev),
+            dY=synth.normal_bf16((M, N), 1.0, synth.SEED_DY + 300 + j, device=dev),
+            A=synth.normal_bf16((r, K), 0.01, synth.SEED_A + 300 + j, device=dev),
+            B=synth.normal_bf16((N, r), 0.01, synth.SEED_B + 300 + j, device=dev),
+            h=torch.empty(M, N, dtype=torch.bfloat16, device=dev),
+            dX=torch.empty(M, K, dtype=torch.bfloat16, device=dev),
+            dA=torch.empty(r, K, dtype=torch.float32, device=dev),
+            dB=torch.empty(N, r, dtype=torch.float32, device=dev))
+        wsz = max(wsz, q.workspace_size(q._lib.OP_FWD, N, K, M, r),
+                  q.workspace_size(q._lib.OP_BWD, N, K, M, r))
+    ws = torch.empty(wsz, dtype=torch.uint8, device=dev)
+
+    def profile_pass():
+        for i, W in enumerate(Ws):
+            q.quantize_weight(W, sse=True, out=wq[i], absmax=absmax, sse_out=sse[i], ws=ws)
+    profile = graphed(profile_pass)
+    nparams = [sh.N * sh.K for sh in shapes]
+    protected = q.rank_topk(sse[:, 0].cpu().tolist(), nparams, topk)
+    prot = set(protected)
+
+    def train_pass():
+        for i, sh in enumerate(shapes):
+            d = io[(sh.N, sh.K)]
+            if i in prot:
+                q.dense_linear_fwd(Ws[i], d["x"], d["A"], d["B"], s, h=d["h"], ws=ws)
+                q.dense_linear_bwd(Ws[i], d["x"], d["dY"], d["A"], d["B"], s, dX=d["dX"],
+                                   dA=d["dA"], dB=d["dB"], ws=ws)
+            else:
+                q.qlora_linear_fwd(wq[i], d["x"], d["A"], d["B"], s, h=d["h"], ws=ws)
+                q.qlora_linear_bwd(wq[i], d["x"], d["dY"], d["A"], d["B"], s, dX=d["dX"],
+                                   dA=d["dA"], dB=d["dB"], ws=ws)
+    train_pass()
+    torch.cuda.synchronize()
+    tp, ip = arm_seconds(profile, seconds, st)
+    tt, it = arm_seconds(train_pass, seconds, st)
+    q.check()
+    ptot = sum(nparams)
+    fl = sum(fwd_flops(sh.N, sh.K, M, r) + bwd_flops(sh.N, sh.K, M, r) for sh in shapes)
+    gbs = ptot * 2.5159 / tp / 1e9
+    tfs = fl / tt / 1e12
+    out = {"matrices": len(shapes), "params": ptot, "tokens": M, "r": r, "alpha": alpha,
+           "profile_pass": {"GBps": round(gbs, 1), "frac_hbm": round(gbs / hbm, 3),
+                            "ms": round(tp * 1e3, 2), "passes": ip,
+                            "launch": "CUDA graph of 280 x qnf4_quantize_weight"},
+           "protected_top8": protected,
+           "fwd_bwd": {"TFLOPs": round(tfs, 1), "frac_tc": round(tfs / tc, 3),
+                       "tflop_per_pass": round(fl / 1e12, 2), "ms": round(tt * 1e3, 1),
+                       "passes": it}}
+    del Ws, wq, io, ws, absmax
+    torch.cuda.empty_cache()
     return out
 
 
@@ -479,10 +668,13 @@ def run_ours(args):
         a.record(stream)
         b.record(stream)
     torch.cuda.synchronize()
+    # clock samples (every 200 ms) from the warm-up through the timed region and the
+    # per-row breakdown that follows it
+    clocks = Clocks(local)
+    time.sleep(0.5)
     for _ in range(W):
         wl.step()
     q.check()
-    clocks = Clocks(local)
     if ws_ > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
@@ -505,20 +697,41 @@ def run_ours(args):
     tf = sum(a.elapsed_time(b) for a, b in evf) / 1e3
     tb = sum(a.elapsed_time(b) for a, b in evb) / 1e3
     shapes = layer_shapes()
-    fl_f = sum(2.0 * M_TOK * N * K + 2.0 * M_TOK * RANK * N for N, K in shapes) * K
-    fl_b = sum(2.0 * M_TOK * N * K + 2.0 * M_TOK * RANK * K for N, K in shapes) * K
+    per_f = sum(2.0 * M_TOK * N * Kk + 2.0 * M_TOK * RANK * N for N, Kk in shapes)
+    per_b = sum(2.0 * M_TOK * N * Kk + 2.0 * M_TOK * RANK * Kk for N, Kk in shapes)
     if tf >= tb:
-        kname, kt, kfl = "k_gemm<A_NF4_K> (fwd h = x W^T + LoRA)", tf, fl_f
+        kname, evs, per = "k_gemm<A_NF4_K> (fwd h = x W^T + LoRA)", evf, per_f
     else:
-        kname, kt, kfl = "k_gemm<A_NF4_MN> (bwd dX = dY W + LoRA)", tb, fl_b
-    achieved = kfl / kt / 1e12
+        kname, evs, per = "k_gemm<A_NF4_MN> (bwd dX = dY W + LoRA)", evb, per_b
+    kt = sum(a.elapsed_time(b) for a, b in evs) / 1e3
+    achieved = per * K / kt / 1e12
+    # per-step achieved rate of that kernel (7 launches a step): its spread over the steps
+    per_step = [per / (sum(a.elapsed_time(b) for a, b in evs[7 * k:7 * k + 7]) / 1e3) / 1e12
+                for k in range(K)]
     tr = traffic_for("k_gemm<A_NF4_K>" if tf >= tb else "k_gemm<A_NF4_MN>")
     flops = step_flops()
     value = flops * K * ws_ / elapsed / 1e12
     extra = {}
-    if not args.no_breakdown:
-        extra = breakdown(wl, q, hbm, tc_sus)
+    if ws_ == 1 and not args.no_breakdown:
+        extra = breakdown(wl, q, hbm, tc_burst)
+    else:
+        time.sleep(0.5)
     clocks.stop()
+    clk = clocks.summary()
+    # The burst bf16 peak applies to a kernel timed in a short region at full clock; a
+    # region of seconds under the power cap (SM clock held well below max) takes the
+    # sustained one.
+    smhz, smax = clk.get("sm_mhz"), clk.get("sm_max_mhz")
+    long_region = elapsed >= 2.0 or (smhz is not None and smax and smhz < 0.9 * smax)
+    tc_peak = tc_sus if long_region else tc_burst
+    peak_kind = f"{peak_kind} bf16 {'sustained' if long_region else 'burst'}"
+    proto = None
+    stack = None
+    if ws_ == 1 and not args.no_breakdown:
+        if not args.no_stack:
+            stack = stack13b(q, dev, hbm, tc_burst)
+        if not args.no_protocol:
+            proto = protocol(wl, q, hbm, tc_burst, tc_sus, dev)
     # end to end through the public API: pinned host inputs in, gradients out, per step.
     # The host-to-device copies run on a side stream in the order the layers need them;
     # each layer's kernels wait only for that layer's copies, so later copies overlap
@@ -557,9 +770,9 @@ def run_ours(args):
     e2e_value = flops * ws_ / te / 1e12
     cpu = None
     if rank == 0 and ws_ == 1 and not args.no_cpu:
-        v, dt, desc, _ = oracle_sample()
+        v, dt, desc, n = oracle_repeated(10.0)
         cpu = {"value": round(v, 6), "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
-               "sample": desc, "seconds": round(dt, 2)}
+               "sample": desc + f"; repeated {n} times", "seconds": round(dt, 2)}
     if rank == 0:
         l2 = torch.cuda.get_device_properties(dev).L2_cache_size
         touched = sum(nbytes([L["W"], L["x"], L["dY"], L["h"], L["dX"], L["packed"]]) for L in wl.layers)
@@ -574,18 +787,25 @@ def run_ours(args):
                        "l2": f"inputs larger than L2: {touched / 1e9:.2f} GB touched per step "
                              f"vs {l2 / 1e6:.0f} MB L2"},
             "roofline": {"bound": "tensor", "kernel": kname, "achieved": round(achieved, 1),
-                         "peak": tc_sus, "unit": "TFLOP/s", "frac": round(achieved / tc_sus, 3),
-                         "peak_kind": f"{peak_kind} bf16 sustained",
+                         "peak": tc_peak, "unit": "TFLOP/s", "frac": round(achieved / tc_peak, 3),
+                         "peak_kind": peak_kind,
+                         "timed_region_s": round(elapsed, 4),
+                         "spread": round((max(per_step) - min(per_step)) / statistics.median(per_step), 4),
+                         "achieved_per_step_median": round(statistics.median(per_step), 1),
                          # dram bytes per algorithmic FLOP (ncu, gate-shaped launch) x the
                          # average FLOPs of one of this kernel's launches in the step
-                         "traffic": round(tr * kfl / (K * len(shapes))) if tr else None},
+                         "traffic": round(tr * per / len(shapes)) if tr else None},
             "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": int(n1 - n0),
-            "clocks": clocks.summary(),
+            "clocks": clk,
             "cpu_baseline": cpu,
             "breakdown": extra,
         }
+        if stack is not None:
+            line["stack13b"] = stack
+        if proto is not None:
+            line["protocol"] = proto
         print(json.dumps(line), flush=True)
     if ws_ > 1:
         torch.distributed.barrier()
@@ -661,12 +881,12 @@ def run_reference(args):
     K, W = args.steps, args.warmup
     # each step: a ~1 s sample of the step (512 weight rows, 128 tokens)
     for _ in range(W):
-        oracle_sample(rows=512)
+        oracle_sample(rows=ORACLE_ROWS)
     times = []
     desc = ""
     flops = 0.0
     for _ in range(K):
-        _, dt, desc, flops = oracle_sample(rows=512)
+        _, dt, desc, flops = oracle_sample(rows=ORACLE_ROWS)
         times.append(dt)
     tot = sum(times)
     value = flops * K / tot / 1e12
@@ -686,6 +906,18 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def relaunch(n: int) -> int:
+    """Run this command again as n ranks of torch.distributed.run on this node."""
+    import socket
+    with socket.socket() as so:
+        so.bind(("127.0.0.1", 0))
+        port = so.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr", "127.0.0.1", f"--master-port={port}", os.path.abspath(__file__),
+           *sys.argv[1:]]
+    return subprocess.run(cmd).returncode
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -694,9 +926,13 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-breakdown", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-stack", action="store_true", help="skip the 13B-stack row")
+    ap.add_argument("--no-protocol", action="store_true", help="skip the 2 s x 3 session arms")
     ap.add_argument("--case", choices=["fwd", "bwd", "decode", "quant", "chanq_quant", "chanq_fwd", "chanq_bwd"], default=None,
                     help="run one operation on one gate-shaped layer (for ncu captures)")
     args = ap.parse_args()
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        sys.exit(relaunch(args.gpus))
     if args.case:
         run_case(args)
         return

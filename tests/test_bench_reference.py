@@ -35,3 +35,18 @@ def test_reference_arm_other_ranks_do_no_work():
     res = _run(1, 2)
     assert res.returncode == 0, res.stderr[-2000:]
     assert not [l for l in res.stdout.splitlines() if l.startswith("{")]
+
+
+def test_gpus_flag_starts_the_ranks_itself():
+    # without a torchrun environment, --gpus N relaunches the command as N ranks of
+    # torch.distributed.run on this node; rank 0 alone prints the contract line
+    env = {k: v for k, v in os.environ.items()
+           if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT")}
+    res = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--gpus", "2",
+                          "--steps", "1", "--warmup", "0"], cwd=ROOT, env=env,
+                         capture_output=True, text=True, timeout=900)
+    assert res.returncode == 0, res.stderr[-2000:]
+    lines = [l for l in res.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1, res.stdout[-2000:]
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["n_gpus"] == 2
