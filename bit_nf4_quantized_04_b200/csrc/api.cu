@@ -169,6 +169,7 @@ struct GemmPlan {
   int full_tiles = 0, tail_tiles = 0, tail_splits = 1, tail_sps = 0, units = 0, grid = 1;
   int ctas_per_sm = 1;
   int nset = 1;  // converter warp sets (4 warps each)
+  int lut = 0;   // NF4 dequantization through the shared-memory pair table
   size_t smem = 0;
   size_t part_floats() const {
     return tail_splits > 1 ? static_cast<size_t>(tail_tiles) * tail_splits * tn * 128 : 0;
@@ -223,17 +224,22 @@ GemmPlan plan_gemm(int asrc, int64_t rows, int64_t cols, int64_t contraction, in
   } else {
     p.s2 = src_deq(asrc) ? ((thin ? 2 : 4)) : 0;
   }
+  // Thin NF4 tiles (decode) dequantize through the shared-memory pair table (32 copies):
+  // their converters are bound by integer issue, which the table moves to the load and
+  // fma pipes.
+  const bool nf4 = asrc == A_NF4_K || asrc == A_NF4_MN;
+  p.lut = (nf4 && thin) ? 32 : 0;
   // 1 KB to align the dynamic buffer, 1 KB for static shared data, per CTA
   const size_t budget = (p.ctas_per_sm == 2 ? (kSmemLimit / 2 - 2048) : kSmemLimit) - 2048;
   for (int pass = 0; pass < 2; ++pass) {
-    const SmemPlan one = smem_plan(asrc, tn, 1, p.s2, has_ext);
+    const SmemPlan one = smem_plan(asrc, tn, 1, p.s2, has_ext, p.lut);
     const size_t fixed = one.total - one.slot1;
     p.s1 = static_cast<int>(std::min<size_t>(kMaxS1, (budget - fixed) / one.slot1));
     // the dequantized-A ring may not be deeper than the load ring (its stages are
     // released through the load ring's barriers)
     if (p.s2 > p.s1) p.s2 = p.s1;
   }
-  p.smem = smem_plan(asrc, tn, p.s1, p.s2, has_ext).total + 1024;
+  p.smem = smem_plan(asrc, tn, p.s1, p.s2, has_ext, p.lut).total + 1024;
   // Persistent CTAs, one per slot, take the tiles in waves. The tiles of a last,
   // partial wave are cut into contraction slices so that wave is as full as it can
   // be: as many slices as the idle slots allow, at least four steps each (each slice
@@ -347,6 +353,7 @@ qnf4_status launch_gemm(const GemmPlan& p, const CUtensorMap& a, const CUtensorM
   g.s1 = p.s1;
   g.s2 = p.s2;
   g.has_ext = p.has_ext;
+  g.lut = p.lut;
   g.wait_ns = g_wait_ns;
   if (!p.has_ext) g.stage = 0;  // the staging buffers live in the adapter tile
   cudaLaunchConfig_t cfg;
@@ -518,6 +525,7 @@ qnf4_status linear_fwd(const BaseSrc& src, const void* x, int64_t M, const void*
     g.code2 = src.w->code2;
     g.scale2 = src.w->scale2;
     g.mean = src.w->mean;
+    g.packed = src.w->packed;
   } else if (src.kind == A_CHANQ_K) {
     g.cq_packed = src.cq_packed;
     g.cq_row_off = src.cq_row_off;

@@ -137,7 +137,7 @@ void build(Nf4Tables& t) {
       const float tk = c < 15 ? t.thr[c] : 2.0f;
       uint32_t bits;
       std::memcpy(&bits, &tk, 4);
-      bits = (bits & ~31u) | static_cast<uint32_t>(c + 1);
+      bits = (bits & ~15u) | static_cast<uint32_t>((14 - c) & 15);
       std::memcpy(&t.bin_tc[b], &bits, 4);
     }
     break;

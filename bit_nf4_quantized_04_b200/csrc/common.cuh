@@ -110,6 +110,10 @@ QNF4_DEV void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "mem
 QNF4_DEV void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
+// Bulk prefetch of a global range into L2 (16-byte aligned address, size a multiple of 16).
+QNF4_DEV void prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
 // 1-D bulk copy global -> shared (16-byte aligned addresses, size multiple of 16).
 QNF4_DEV void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile(

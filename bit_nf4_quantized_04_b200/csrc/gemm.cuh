@@ -127,16 +127,26 @@ struct GemmArgs {
   float* part;            // partial tiles of the tail slices [tail_tiles][tail_splits][tn][128]
   unsigned int* counters; // arrival counters per tail tile (zero on entry, left zero)
   unsigned long long wait_ns;
+  const uint8_t* packed;  // A_NF4_K: the packed codes [wN, nbk * 32] (for the L2 prefetch)
+  int lut;                // NF4 sources: copies of the shared-memory pair table (16 or 32;
+                          // nf4_block_lut), 0 = the register byte planes
   int lazy_dep;           // programmatic dependent launch: 0 = every thread waits for the
                           // previous grid after the prologue; 1 = only the adapter chunk's
                           // copy waits (its operand is the one the previous grid writes)
 };
 
 struct SmemPlan {
-  uint32_t off_a1, off_b1, off_p1, off_t1, slot1, slot2, ring2, ext, cq, total;
+  uint32_t off_a1, off_b1, off_p1, off_t1, slot1, slot2, ring2, ext, cq, lut, total;
 };
 
-__host__ __device__ inline SmemPlan smem_plan(int asrc, int tn, int s1, int s2, int has_ext) {
+// Shared-memory NF4 lookup table: one entry per packed byte value (the two bf16 levels
+// the byte's nibbles select), replicated `copies` times (16 or 32) with lane l reading
+// copy l mod copies: 32 copies never share a bank within a warp, 16 copies at most two
+// lanes per bank (8 or 16 KB less shared memory).
+__host__ __device__ constexpr uint32_t lut_bytes(int copies) { return 256u * static_cast<uint32_t>(copies) * 4u; }
+
+__host__ __device__ inline SmemPlan smem_plan(int asrc, int tn, int s1, int s2, int has_ext,
+                                              int lut = 0) {
   SmemPlan p{};
   uint32_t o = 0;
   p.off_a1 = o;
@@ -152,7 +162,8 @@ __host__ __device__ inline SmemPlan smem_plan(int asrc, int tn, int s1, int s2, 
   p.ring2 = static_cast<uint32_t>(s1) * p.slot1;
   p.ext = p.ring2 + static_cast<uint32_t>(s2) * p.slot2;
   p.cq = p.ext + (has_ext ? kATile : 0u);
-  p.total = p.cq + (asrc == A_CHANQ_K ? 256u * 4u : 0u);
+  p.lut = p.cq + (asrc == A_CHANQ_K ? 256u * 4u : 0u);
+  p.total = p.lut + ((lut && (asrc == A_NF4_K || asrc == A_NF4_MN)) ? lut_bytes(lut) : 0u);
   return p;
 }
 
@@ -247,6 +258,44 @@ QNF4_DEV void nf4_block_to_bf16(const uint8_t* src, float c, const float (&lv)[1
   const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
   for (int i = 0; i < 8; ++i) nf4_lookup8(w[i], P, &o[4 * i]);
+}
+
+// Dequantize one NF4 block through the shared-memory pair table: each packed byte
+// (element 2j in the high nibble) indexes the table entry holding bf16(q[hi]) and
+// bf16(q[lo]); one packed bf16 multiply by the block constant c2 = (bf16(c), bf16(c))
+// then gives bf16(bf16(q) bf16(c)) for both elements. The lane's table copy starts at
+// shared address tb. Per two codes: one byte extract, one shared load, one multiply
+// (the register byte-plane lookup spends about five integer operations there).
+QNF4_DEV uint32_t lds_u32(uint32_t addr) {  // read-only table: not volatile
+  uint32_t v;
+  asm("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+QNF4_DEV uint32_t hmul2_bf16(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+QNF4_DEV void nf4_block_lut(const uint8_t* src, uint32_t c2, uint32_t tb, uint32_t sh,
+                            uint32_t (&o)[32]) {
+  const uint4 a = *reinterpret_cast<const uint4*>(src);
+  const uint4 b = *reinterpret_cast<const uint4*>(src + 16);
+  const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t beta = __byte_perm(w[i], 0u, 0x4440u | static_cast<uint32_t>(j));
+      o[4 * i + j] = hmul2_bf16(lds_u32(tb + (beta << sh)), c2);
+    }
+  }
+}
+// Fill the table (every thread of the CTA takes part; a CTA barrier must follow).
+QNF4_DEV void lut_fill(uint32_t* tab, const float* s_lv, int copies, int tid, int nthreads) {
+  for (int i = tid; i < 256 * copies; i += nthreads) {
+    const int beta = i / copies;
+    tab[i] = pack_bf16x2(s_lv[beta >> 4], s_lv[beta & 15]);
+  }
 }
 
 QNF4_DEV void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
@@ -402,7 +451,7 @@ __global__ void __launch_bounds__(gemm_threads(NSET), MINB)
   const int lane = threadIdx.x & 31;
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  const SmemPlan sp = smem_plan(ASRC, g.tn, g.s1, g.s2, g.has_ext);
+  const SmemPlan sp = smem_plan(ASRC, g.tn, g.s1, g.s2, g.has_ext, g.lut);
   const int S1 = g.s1, S2 = g.s2;
   const int u0 = blockIdx.x;
   const int ustep = gridDim.x;
@@ -436,6 +485,8 @@ __global__ void __launch_bounds__(gemm_threads(NSET), MINB)
     if (g.stage) tma_prefetch_desc(&tmO);
     if (src_table_tma(ASRC)) tma_prefetch_desc(&tmT);
   }
+  if ((ASRC == A_NF4_K || ASRC == A_NF4_MN) && g.lut)
+    lut_fill(reinterpret_cast<uint32_t*>(base + sp.lut), g.levels, g.lut, threadIdx.x, blockDim.x);
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s_tmem;
@@ -447,6 +498,22 @@ __global__ void __launch_bounds__(gemm_threads(NSET), MINB)
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
+    // Decode tiles read 32 bytes of each of 128 rows per step, rows K/2 bytes apart:
+    // first the whole warp asks L2 for every unit's row slices of this CTA (contiguous
+    // per row), so DRAM streams whole row ranges instead of scattered 32-byte pieces.
+    if (ASRC == A_NF4_K && g.tn <= 32 && g.packed) {
+      for (int u = u0; u < g.nunits; u += ustep) {
+        const Unit w = unit_of(g, u);
+        if (w.nst <= 0) continue;
+        for (int r = lane; r < kRowsTile; r += 32) {
+          const int64_t row = w.row0 + r;
+          if (row < g.wN)
+            prefetch_l2(g.packed + row * g.nbk * 32 + static_cast<int64_t>(w.step0) * 32,
+                        static_cast<uint32_t>(w.nst) * 32u);
+        }
+      }
+      __syncwarp();
+    }
     if (lane == 0) {
       int issued = 0;
       int s = 0;
@@ -779,7 +846,11 @@ __global__ void __launch_bounds__(gemm_threads(NSET), MINB)
     };
 
     // Per-source state and one conversion step (A-ring position cur, unit w).
-    // NF4: the 16 levels in registers; block constants fetched one step ahead.
+    // NF4: the 16 levels in registers (or this lane's copy of the pair table); block
+    // constants fetched one step ahead.
+    const uint32_t lut_tb =
+        smem_u32(base + sp.lut) + (static_cast<uint32_t>(lane & (g.lut > 0 ? g.lut - 1 : 0)) << 2);
+    const uint32_t lut_sh = g.lut == 16 ? 6u : 7u;  // bytes per table entry row: 4 x copies
     float lv[16];
     float mu = 0.f;
     const int slot = TMA_A ? lrow : t;  // A row slot (in TMEM: the lane this warp may access)
@@ -925,6 +996,8 @@ __global__ void __launch_bounds__(gemm_threads(NSET), MINB)
             tv[4 * q4] = f.x; tv[4 * q4 + 1] = f.y; tv[4 * q4 + 2] = f.z; tv[4 * q4 + 3] = f.w;
           }
           nf4_block_to_bf16(src, ch, tv, o);
+        } else if (g.lut) {
+          nf4_block_lut(src, pack_bf16x2(ch, ch), lut_tb, lut_sh, o);
         } else {
           nf4_block_to_bf16(src, ch, lv, o);
         }

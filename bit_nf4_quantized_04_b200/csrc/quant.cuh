@@ -61,9 +61,16 @@ QNF4_DEV uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
   return d;
 }
 
+// Shared loads of read-only tables (filled before a CTA barrier); not volatile, so the
+// compiler may schedule them freely.
+QNF4_DEV uint32_t lds_u32q(uint32_t addr) {
+  uint32_t v;
+  asm("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
 QNF4_DEV float lds_f32(uint32_t addr) {
   float v;
-  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+  asm("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
   return v;
 }
 
@@ -94,26 +101,45 @@ QNF4_DEV bool warp_wait(uint64_t* bar, uint32_t parity, unsigned long long wait_
   return __all_sync(0xffffffffu, ok);
 }
 
+// max(|a|, |b|) per bf16 lane, NaN if either lane is NaN; the sign bits of the result
+// are not the absolute value's (xorsign), so callers mask them.
+QNF4_DEV uint32_t bmax_abs2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.NaN.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+// (d >> 31) + t: the sign bit of d added to t's bits
+QNF4_DEV uint32_t sign_add(uint32_t d, uint32_t t) {
+  uint32_t r;
+  asm("mad.hi.u32 %0, %1, 2, %2;" : "=r"(r) : "r"(d), "r"(t));
+  return r;
+}
+
 // Blockwise NF4 quantization, streamed: each CTA walks its chunks (chunk c holds
 // blocks [128 c, 128 c + 128)) through a ring of shared-memory stages. One warp
 // fills the ring with cp.async.bulk; eight worker warps consume it, each releasing a
-// stage with one arrival when done, so no warp waits for the others. Inside a
-// chunk, a group of 8 threads takes one 64-element block (each thread 8 consecutive
-// elements, one 16-byte shared load) and writes 4 packed bytes. Optional outputs:
-// WRITE -> packed codes and fp32 absmax; SSE -> per-CTA float64 partial sums of the
-// single-level squared round-trip error; CNT -> per-CTA float64 counts of the elements
-// with |w| < tau (the sparsity of "AQLoRA" §3.1), exact integers; asum_part (optional,
-// with WRITE) -> per-CTA float64 sums of the block constants, the partials of the double
-// quantization's tensor mean.
+// stage with one arrival when done, so no warp waits for the others. Inside a chunk,
+// four threads take one 64-element block, each 16 consecutive elements as two 16-byte
+// shared loads (the first piece alternates between neighbouring blocks, so a quarter
+// warp's loads hit eight different bank groups), and write 8 packed bytes. Optional
+// outputs: WRITE -> packed codes and fp32 absmax; SSE -> per-CTA float64 partial sums
+// of the single-level squared round-trip error (fp32 over a thread's 16 elements);
+// CNT -> per-CTA float64 counts of the elements with |w| < tau (the sparsity of
+// "AQLoRA" §3.1), exact integers; asum_part (optional, with WRITE) -> per-CTA float64
+// sums of the block constants, the partials of the double quantization's tensor mean.
 //
+// absmax: max of |w| on the bf16 bit patterns, two elements per instruction; a block
+// holding a NaN or an infinity has magnitude bits >= 0x7F80 and takes the exact path.
 // Code search (see Nf4Tables), for a block with absmax c > 0: the bin
 // k = round(w H/c + H) comes from one fused multiply-add with a magic constant
-// (1.5 * 2^23, whose low mantissa bits then hold k); the table entry t_k carries
-// c_k + 1 in its low mantissa bits; d = fma(-c, t_k, w) = w - c t_k rounded once,
-// so its sign is exactly that of w/c - t_k, and code = c_k + 1 - [d < 0]. If any of a
-// thread's 8 values lies within 2^-18 c of its t_k, those 8 take the exact IEEE
-// quotient and the full count. Non-finite weights are outside the method: the table
-// index is masked, so they cannot read outside it, but their codes are unspecified.
+// (1.5 * 2^23, whose low mantissa bits then hold k), so the table entry's shared
+// address is one multiply-add of those bits; the entry t_k carries (14 - c_k) mod 16 in
+// its low mantissa bits; d = fma(-c, t_k, w) = w - c t_k rounded once, so its sign is
+// exactly that of w/c - t_k, and adding d's sign bit to t_k's bits leaves 15 - code in
+// the low 4 bits (the packed word is complemented once at the end). If any of a
+// thread's 16 values lies within 2^-18 c of its t_k, those 16 take the exact IEEE
+// quotient and the full count. The residual of the error is w - c q[code], one fma
+// with the level read by the (complemented) code.
 template <bool WRITE, bool SSE, bool CNT = false>
 __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
     k_nf4_quant(const uint16_t* __restrict__ W, int64_t nblocks, uint32_t* __restrict__ packed,
@@ -124,7 +150,8 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
   __shared__ __align__(8) uint64_t full[kQStages], empty[kQStages];
   __shared__ float s_thr[16];
   __shared__ float s_lv[16];
-  __shared__ __align__(1024) float s_tc[2 * kMaxHalfBins + 1];
+  __shared__ float s_lvc[16];  // levels by complemented code: s_lvc[i] = q[15 - i]
+  __shared__ __align__(16) float s_tc[2 * kMaxHalfBins + 1];
   __shared__ double s_red[kQWorkers];
   __shared__ unsigned long long s_cnt[kQWorkers];
   __shared__ double s_asum[kQWorkers];
@@ -136,6 +163,7 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
   for (int i = tid; i < 16; i += kQThreads) {
     s_thr[i] = tab.thr[i];
     s_lv[i] = tab.levels[i];
+    s_lvc[i] = tab.levels[15 - i];
   }
   for (int i = tid; i <= 2 * kMaxHalfBins; i += kQThreads) s_tc[i] = tab.bin_tc[i];
   const int64_t nchunks = (nblocks + kQChunkBlocks - 1) / kQChunkBlocks;
@@ -151,7 +179,7 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
   __syncthreads();
 
   double acc = 0.0;
-  double asum = 0.0;       // this thread's block constants (asum_part; group leaders only)
+  double asum = 0.0;       // this thread's block constants (asum_part; block leaders only)
   unsigned int below = 0;  // this thread's elements with |w| < tau (CNT)
   if (warp == kQWorkers) {
     // ---------------------------------------------------------------- producer
@@ -200,10 +228,14 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
     const int H = tab.bin_h;
     const float hf = static_cast<float>(H);
     const uint64_t mg2 = f2_pack(hf + 12582912.0f, hf + 12582912.0f);
-    // the bin table sits 1024-byte aligned, so entry k is at base | 4 (k & 0xFF)
-    const char* tcb = reinterpret_cast<const char*>(s_tc);
-    const int lane8 = tid & 7;
-    const int grp = tid >> 3;  // 32 groups of 8 threads
+    // bin k's entry sits at shared address kb * 4 + toff, kb = 0x4B400000 + k being the
+    // bits of the magic fma's result (32-bit wrap-around)
+    const uint32_t toff = smem_u32(s_tc) - 0x4B400000u * 4u;
+    const uint32_t lvoff = smem_u32(s_lvc);
+    const int l4 = tid & 3;     // elements 16 l4 .. 16 l4 + 15 of the block
+    const int grp = tid >> 2;   // 64 groups of four threads
+    const int sw = grp & 1;     // which 16-byte piece this thread loads first
+    const int p0 = 2 * l4 + sw, p1 = 2 * l4 + 1 - sw;
     int st = 0;
     uint32_t ph = 0;
     for (int64_t j = 0; j < my; ++j) {
@@ -211,66 +243,57 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
       const int64_t c0 = (blockIdx.x + j * gridDim.x) * kQChunkBlocks;
       const int nb = static_cast<int>(min(static_cast<int64_t>(kQChunkBlocks), nblocks - c0));
       const uint8_t* chunk = qsm + st * kQChunkBytes;
-#pragma unroll
-      for (int u = 0; u < kQChunkBlocks / 32; ++u) {
-        const int bl = grp + 32 * u;  // block within the chunk
+#pragma unroll 1
+      for (int u = 0; u < kQChunkBlocks / 64; ++u) {
+        const int bl = grp + 64 * u;  // block within the chunk
         const bool valid = bl < nb;   // groups past a partial chunk's end work on zeros
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (valid) v = *reinterpret_cast<const uint4*>(chunk + bl * 128 + lane8 * 16);
-        const uint32_t words[4] = {v.x, v.y, v.z, v.w};
-        float w[8];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          w[2 * e] = bf16lo(words[e]);
-          w[2 * e + 1] = bf16hi(words[e]);
+        uint4 va = make_uint4(0u, 0u, 0u, 0u), vb = va;
+        if (valid) {
+          va = *reinterpret_cast<const uint4*>(chunk + bl * 128 + p0 * 16);
+          vb = *reinterpret_cast<const uint4*>(chunk + bl * 128 + p1 * 16);
         }
+        const uint32_t wd[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
         if (CNT && valid) {
 #pragma unroll
-          for (int e = 0; e < 8; ++e) below += fabsf(w[e]) < tau ? 1u : 0u;
+          for (int e = 0; e < 8; ++e)
+            below += (fabsf(bf16lo(wd[e])) < tau ? 1u : 0u) + (fabsf(bf16hi(wd[e])) < tau ? 1u : 0u);
         }
-        float m = fmaxf(fabsf(w[0]), fabsf(w[1]));
-#pragma unroll
-        for (int e = 2; e < 8; ++e) m = fmaxf(m, fabsf(w[e]));
-        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
-        const float c = m;
-        uint32_t code[8];
+        uint32_t m2 = bmax_abs2(bmax_abs2(bmax_abs2(wd[0], wd[1]), bmax_abs2(wd[2], wd[3])),
+                                bmax_abs2(bmax_abs2(wd[4], wd[5]), bmax_abs2(wd[6], wd[7])));
+        uint32_t cb = max(m2 & 0x7FFFu, (m2 >> 16) & 0x7FFFu);
+        cb = max(cb, __shfl_xor_sync(0xffffffffu, cb, 1));
+        cb = max(cb, __shfl_xor_sync(0xffffffffu, cb, 2));
+        const float c = __uint_as_float(cb << 16);
+        uint32_t mc[16];  // 15 - code of the thread's elements: pieces p0 (0..7), p1 (8..15)
         float sse = 0.f;
-        if (c == 0.f) {
+        bool exact = cb >= 0x7F80u || H == 0 || !(c >= 0x1p-100f);
+        if (cb == 0u) {
 #pragma unroll
-          for (int e = 0; e < 8; ++e) code[e] = 7u;  // the exact-zero level (error 0)
-        } else {
+          for (int e = 0; e < 16; ++e) mc[e] = 8u;  // the exact-zero level (error 0)
+          exact = false;
+        } else if (!exact) {
           const float hr = hf * rcp_approx(c);
           const uint64_t hr2 = f2_pack(hr, hr), nc2 = f2_pack(-c, -c);
-          uint64_t wp[4], dp[4];
-          float tk[8];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            wp[e] = f2_pack(w[2 * e], w[2 * e + 1]);
-            const float2 kb = f2_unpack(f2_fma(wp[e], hr2, mg2));
-            tk[2 * e] = *reinterpret_cast<const float*>(tcb + ((__float_as_uint(kb.x) << 2) & 0x3FCu));
-            tk[2 * e + 1] = *reinterpret_cast<const float*>(tcb + ((__float_as_uint(kb.y) << 2) & 0x3FCu));
-          }
+          uint64_t wp[8];
           float dmin = 3.0e38f;
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            dp[e] = f2_fma(f2_pack(tk[2 * e], tk[2 * e + 1]), nc2, wp[e]);
-            const float2 d = f2_unpack(dp[e]);
-            code[2 * e] = static_cast<uint32_t>((__float_as_int(tk[2 * e]) & 31) + (__float_as_int(d.x) >> 31));
-            code[2 * e + 1] = static_cast<uint32_t>((__float_as_int(tk[2 * e + 1]) & 31) + (__float_as_int(d.y) >> 31));
+          for (int e = 0; e < 8; ++e) {
+            wp[e] = f2_pack(bf16lo(wd[e]), bf16hi(wd[e]));
+            const float2 kb = f2_unpack(f2_fma(wp[e], hr2, mg2));
+            const uint32_t ta = lds_u32q(__float_as_uint(kb.x) * 4u + toff);
+            const uint32_t tb = lds_u32q(__float_as_uint(kb.y) * 4u + toff);
+            const float2 d = f2_unpack(f2_fma(f2_pack(__uint_as_float(ta), __uint_as_float(tb)), nc2, wp[e]));
             dmin = fminf(dmin, fminf(fabsf(d.x), fabsf(d.y)));
+            mc[2 * e] = sign_add(__float_as_uint(d.x), ta) & 15u;
+            mc[2 * e + 1] = sign_add(__float_as_uint(d.y), tb) & 15u;
           }
-          if (!(dmin > c * 0x1p-18f) || H == 0 || !(c >= 0x1p-100f)) {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) code[e] = static_cast<uint32_t>(nf4_code_exact(w[e], c, s_thr));
-          }
-          if (SSE) {
+          exact = !(dmin > c * 0x1p-18f);
+          if (SSE && !exact) {
             // r = w - c q[code], two running sums of r^2 (even and odd elements)
             uint64_t acc2 = f2_pack(0.f, 0.f);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const uint64_t q2 = f2_pack(s_lv[code[2 * e]], s_lv[code[2 * e + 1]]);
+            for (int e = 0; e < 8; ++e) {
+              const uint64_t q2 = f2_pack(lds_f32(lvoff + 4u * mc[2 * e]), lds_f32(lvoff + 4u * mc[2 * e + 1]));
               const uint64_t r2 = f2_fma(q2, nc2, wp[e]);
               acc2 = f2_fma(r2, r2, acc2);
             }
@@ -278,24 +301,47 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
             sse = a2.x + a2.y;
           }
         }
-        const int64_t b = c0 + bl;
+        if (exact) {
+          // out of line: the IEEE quotient and the full threshold count (values near a
+          // threshold, tiny or non-finite absmax, or no bin table)
+          float a = 0.f, b = 0.f;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float w0 = bf16lo(wd[e]), w1 = bf16hi(wd[e]);
+            const int k0 = nf4_code_exact(w0, c, s_thr), k1 = nf4_code_exact(w1, c, s_thr);
+            mc[2 * e] = static_cast<uint32_t>(15 - k0);
+            mc[2 * e + 1] = static_cast<uint32_t>(15 - k1);
+            if (SSE) {
+              const float r0 = fmaf(s_lv[k0], -c, w0), r1 = fmaf(s_lv[k1], -c, w1);
+              a = fmaf(r0, r0, a);
+              b = fmaf(r1, r1, b);
+            }
+          }
+          sse = a + b;
+        }
+        const int64_t blk = c0 + bl;
         if (WRITE && valid) {
-          // element 2e in the high nibble of byte e
-          const uint32_t b0 = code[0] * 16u + code[1], b1 = code[2] * 16u + code[3];
-          const uint32_t b2 = code[4] * 16u + code[5], b3 = code[6] * 16u + code[7];
-          const uint32_t word = __byte_perm(__byte_perm(b0, b1, 0x1140), __byte_perm(b2, b3, 0x1140), 0x5410);
-          packed[b * 8 + lane8] = word;
-          if (lane8 == 0) {
-            absmax[b] = c;
+          // element 2i in the high nibble of byte i; the complemented nibbles are
+          // packed, then the word is complemented once
+          uint32_t pw[2];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const uint32_t b0 = mc[8 * h + 0] * 16u + mc[8 * h + 1];
+            const uint32_t b1 = mc[8 * h + 2] * 16u + mc[8 * h + 3];
+            const uint32_t b2 = mc[8 * h + 4] * 16u + mc[8 * h + 5];
+            const uint32_t b3 = mc[8 * h + 6] * 16u + mc[8 * h + 7];
+            pw[h] = ~__byte_perm(__byte_perm(b0, b1, 0x0040), __byte_perm(b2, b3, 0x0040), 0x5410);
+          }
+          uint2 out;
+          out.x = sw ? pw[1] : pw[0];  // piece 2 l4
+          out.y = sw ? pw[0] : pw[1];  // piece 2 l4 + 1
+          reinterpret_cast<uint2*>(packed)[blk * 4 + l4] = out;
+          if (l4 == 0) {
+            absmax[blk] = c;
             asum += static_cast<double>(c);
           }
         }
-        if (SSE) {
-          sse += __shfl_xor_sync(0xffffffffu, sse, 1);
-          sse += __shfl_xor_sync(0xffffffffu, sse, 2);
-          sse += __shfl_xor_sync(0xffffffffu, sse, 4);
-          if (lane8 == 0 && valid) acc += static_cast<double>(sse);
-        }
+        if (SSE && valid) acc += static_cast<double>(sse);
       }
       __syncwarp();
       if ((tid & 31) == 0) mbar_arrive(&empty[st]);  // this warp is done with the stage

@@ -11,9 +11,10 @@ constexpr int kMaxHalfBins = 128;
 // [(k - 0.5)/H - 1, (k + 0.5)/H - 1). H is chosen so that every bin holds at most one
 // decision threshold and every threshold lies at least 2^-16 from a bin edge; then
 // code(x) = c_k + (x >= t_k), where c_k counts the thresholds below the bin and t_k is
-// the next threshold (2.0 past the last). bin_tc[k] stores t_k with c_k + 1 written
-// into its 5 lowest mantissa bits (a shift of at most 31 ulp, inside the kernels'
-// 2^-18 ambiguity window, within which they fall back to the exact count).
+// the next threshold (2.0 past the last). bin_tc[k] stores t_k with (14 - c_k) mod 16
+// written into its 4 lowest mantissa bits (a shift of at most 15 ulp, inside the
+// kernels' 2^-18 ambiguity window, within which they fall back to the exact count), so
+// that adding the sign bit of w - c t_k to its bits leaves 15 - code in the low 4 bits.
 struct Nf4Tables {
   float levels[16];      // sorted NF4 levels, exact 0 at index 7, -1 / +1 at the ends
   float thr[16];         // 15 decision thresholds, thr[15] = +inf sentinel
