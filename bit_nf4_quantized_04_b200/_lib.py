@@ -10,11 +10,14 @@ import ctypes as C
 import os
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libqnf4.so")
+# QNF4_LIB=checked selects the checked build (index checks in the kernels, reported as
+# QNF4_ERR_BOUNDS), for tests; anything else, or unset, the library itself.
+LIB_PATH = os.path.join(HERE, "libqnf4_checked.so" if os.environ.get("QNF4_LIB") == "checked"
+                        else "libqnf4.so")
 
 QNF4_OK = 0
 STATUS_NAMES = {0: "OK", 1: "ERR_ARG", 2: "ERR_SHAPE", 3: "ERR_ALIGN", 4: "ERR_CUDA",
-                5: "ERR_TIMEOUT", 6: "ERR_WORKSPACE"}
+                5: "ERR_TIMEOUT", 6: "ERR_WORKSPACE", 7: "ERR_BOUNDS"}
 OUT_F32, OUT_BF16 = 0, 1
 OP_QUANTIZE, OP_DOUBLE_QUANT, OP_FWD, OP_BWD, OP_CHANQ_FWD, OP_CHANQ_BWD, OP_LOFTQ = 0, 1, 2, 3, 4, 5, 6
 OP_LAYER_STATS, OP_QUANTIZE_WEIGHT = 7, 8

@@ -16,6 +16,9 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libqnf4.so")
+# The checked build: the same library with index checks in the kernels (-DQNF4_CHECKED);
+# an index outside its buffer is skipped and reported by qnf4_check as QNF4_ERR_BOUNDS.
+LIB_CHECKED = os.path.join(HERE, "libqnf4_checked.so")
 SOURCES = ["api.cu", "codebook.cpp"]
 HEADERS = ["common.cuh", "quant.cuh", "chanq.cuh", "gemm.cuh", "loftq.cuh", "tables.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -28,39 +31,54 @@ def _nvcc() -> str:
     raise RuntimeError("nvcc not found: the CUDA toolkit is required to build libqnf4.so")
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
+def _stale(lib: str) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = [os.path.join(CSRC, f) for f in SOURCES + HEADERS]
     deps.append(os.path.join(ROOT, "include", "qnf4.h"))
     deps.append(os.path.abspath(__file__))
     return any(os.path.getmtime(d) > t for d in deps if os.path.exists(d))
 
 
-def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None) -> str:
-    """Compile libqnf4.so if any source is newer than it; return its path."""
-    if not force and not _stale():
-        return LIB
-    tmp = LIB + ".tmp"
-    cmd = [_nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-shared", "-Xcompiler", "-fPIC",
-           "-Xcompiler", "-fvisibility=hidden", "--expt-relaxed-constexpr",
-           "-I", os.path.join(ROOT, "include"),
-           *(extra or []),
-           *[os.path.join(CSRC, f) for f in SOURCES], "-ldl", "-o", tmp]
-    if verbose:
-        print(" ".join(cmd), flush=True)
-    res = subprocess.run(cmd, capture_output=True, text=True)
-    if res.returncode != 0:
-        sys.stderr.write(res.stdout + res.stderr)
-        raise RuntimeError("nvcc failed building libqnf4.so")
-    if verbose and (res.stdout or res.stderr):
-        sys.stderr.write(res.stdout + res.stderr)
-    os.replace(tmp, LIB)
+def _cmd(lib: str, extra: list[str]) -> list[str]:
+    return [_nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-shared", "-Xcompiler", "-fPIC",
+            "-Xcompiler", "-fvisibility=hidden", "--expt-relaxed-constexpr",
+            "-I", os.path.join(ROOT, "include"), *extra,
+            *[os.path.join(CSRC, f) for f in SOURCES], "-ldl", "-o", lib + ".tmp"]
+
+
+def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None,
+          checked: bool = True) -> str:
+    """Compile libqnf4.so (and, with checked=True, libqnf4_checked.so) if any source is
+    newer; the two compilations run in parallel. Returns the main library's path."""
+    jobs = []
+    if force or _stale(LIB):
+        jobs.append((LIB, _cmd(LIB, list(extra or []))))
+    if checked and (force or _stale(LIB_CHECKED)):
+        jobs.append((LIB_CHECKED, _cmd(LIB_CHECKED, ["-DQNF4_CHECKED", *(extra or [])])))
+    procs = []
+    for lib, cmd in jobs:
+        if verbose:
+            print(" ".join(cmd), flush=True)
+        procs.append((lib, subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.PIPE,
+                                            text=True)))
+    failed = []
+    for lib, pr in procs:
+        out, err = pr.communicate()
+        if pr.returncode != 0:
+            sys.stderr.write(out + err)
+            failed.append(os.path.basename(lib))
+        else:
+            if verbose and (out or err):
+                sys.stderr.write(out + err)
+            os.replace(lib + ".tmp", lib)
+    if failed:
+        raise RuntimeError("nvcc failed building " + ", ".join(failed))
     return LIB
 
 
 if __name__ == "__main__":
     force = "--force" in sys.argv
     extra = ["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else None
-    print(build(force=force, verbose=True, extra=extra))
+    print(build(force=force, verbose=True, extra=extra, checked="--no-checked" not in sys.argv))

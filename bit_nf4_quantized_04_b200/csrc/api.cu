@@ -81,8 +81,6 @@ QuantTab make_tab() {
   return q;
 }
 
-constexpr int kQuantMaxGrid = 1024;
-
 int quant_grid(int64_t nblocks) {
   // persistent: kQCtasPerSm streaming CTAs per SM, never more CTAs than chunks
   const int64_t chunks = (nblocks + kQChunkBlocks - 1) / kQChunkBlocks;
@@ -354,6 +352,8 @@ qnf4_status launch_gemm(const GemmPlan& p, const CUtensorMap& a, const CUtensorM
   g.s2 = p.s2;
   g.has_ext = p.has_ext;
   g.lut = p.lut;
+  g.part_elems = static_cast<int64_t>(p.part_floats());
+  g.cnt_elems = p.tail_tiles;
   g.wait_ns = g_wait_ns;
   if (!p.has_ext) g.stage = 0;  // the staging buffers live in the adapter tile
   cudaLaunchConfig_t cfg;
@@ -415,6 +415,8 @@ GemmArgs base_args() {
   std::memset(&g, 0, sizeof(g));
   const Nf4Tables& t = nf4_tables();
   std::memcpy(g.levels, t.levels, sizeof(g.levels));
+  // extents for the checked build's index tests: unbounded until a caller narrows them
+  g.out_elems = g.out2_elems = g.part_elems = g.cnt_elems = g.cst_elems = INT64_MAX;
   return g;
 }
 
@@ -482,6 +484,8 @@ qnf4_status run_u(const LinPlan& L, const void* x, const void* A, int64_t M, int
   g.out = up;
   g.out2 = ut;
   g.o2_ld = L.ldm;
+  g.out_elems = M * 64;
+  g.out2_elems = static_cast<int64_t>(L.r16) * L.ldm;
   g.scale = scale;
   g.part = part;
   g.counters = cnt;
@@ -538,6 +542,8 @@ qnf4_status linear_fwd(const BaseSrc& src, const void* x, int64_t M, const void*
   g.out = h;
   g.o_rs = 1;
   g.o_cs = N;
+  g.out_elems = M * N;
+  if (src.kind == A_NF4_K) g.cst_elems = N * (K / 64);
   CUtensorMap mo;
   g.stage = stage_map(&mo, h, N, M, N) ? 1 : 0;
   g.part = part;
@@ -588,6 +594,8 @@ qnf4_status linear_bwd(const BaseSrc& src, const void* x, const void* dY, int64_
     g.out = vp;
     g.out2 = vt;
     g.o2_ld = L.ldm;
+    g.out_elems = M * 64;
+    g.out2_elems = static_cast<int64_t>(L.r16) * L.ldm;
     g.scale = scale;
     g.part = part;
     g.counters = cnt;
@@ -610,6 +618,7 @@ qnf4_status linear_bwd(const BaseSrc& src, const void* x, const void* dY, int64_
     g.o_rs = 1;
     g.o_cs = K;
     g.out_cols = r;
+    g.out_elems = static_cast<int64_t>(r) * K;
     g.scale = 1.f;
     g.part = part;
     g.counters = cnt;
@@ -627,6 +636,7 @@ qnf4_status linear_bwd(const BaseSrc& src, const void* x, const void* dY, int64_
     g.o_rs = r;
     g.o_cs = 1;
     g.out_cols = r;
+    g.out_elems = N * r;
     g.scale = 1.f;
     g.part = part;
     g.counters = cnt;
@@ -666,6 +676,8 @@ qnf4_status linear_bwd(const BaseSrc& src, const void* x, const void* dY, int64_
     g.out = dX;
     g.o_rs = 1;
     g.o_cs = K;
+    g.out_elems = M * K;
+    if (main_src == A_NF4_MN || main_src == A_CHANQ_MN) g.cst_elems = N * (K / 64);
     CUtensorMap mo;
     g.stage = stage_map(&mo, dX, K, M, K) ? 1 : 0;
     g.part = part;
@@ -874,6 +886,8 @@ qnf4_status qnf4_check(void* stream) {
     const unsigned int zero = 0;
     cudaMemcpyToSymbol(g_qnf4_err, &zero, sizeof(zero));
     if (flag == kErrEigensolve) return fail(QNF4_ERR_CUDA, "LoftQ eigensolve failed (cuSOLVER info != 0)");
+    if (flag >= kErrBoundsBase)
+      return fail(QNF4_ERR_BOUNDS, "a kernel index fell outside its buffer (site %u)", flag - kErrBoundsBase);
     return fail(QNF4_ERR_TIMEOUT, "a kernel wait gave up (site %u)", flag);
   }
   return QNF4_OK;

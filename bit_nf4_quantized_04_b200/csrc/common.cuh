@@ -18,6 +18,20 @@ __device__ unsigned int g_qnf4_err = 0;
 
 QNF4_DEV void set_err(unsigned int code) { atomicCAS(&g_qnf4_err, 0u, code); }
 
+// Index checks of the checked build (compiled with -DQNF4_CHECKED, libqnf4_checked.so): an
+// access whose index falls outside its buffer records kErrBoundsBase + site in the device
+// flag and is skipped, so a planning or indexing mistake shows as QNF4_ERR_BOUNDS instead
+// of a fault. The default build compiles no check (the condition is dead code).
+constexpr unsigned int kErrBoundsBase = 1000;
+#ifdef QNF4_CHECKED
+QNF4_DEV bool in_bounds(bool ok, unsigned int site) {
+  if (!ok) set_err(kErrBoundsBase + site);
+  return ok;
+}
+#else
+QNF4_DEV bool in_bounds(bool, unsigned int) { return true; }
+#endif
+
 // Deadline of a drain: once a kernel gives up, it still waits for its own copies and
 // MMAs in flight before it frees shared and tensor memory, however short the caller's
 // wait limit; those always finish unless the hardware itself has stopped.
@@ -58,6 +72,7 @@ QNF4_DEV void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
                "r"(bytes)
                : "memory");
 }
+// Test for the completion of the phase with the given parity (returns at once).
 QNF4_DEV bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -69,6 +84,24 @@ QNF4_DEV bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// The same test for long waits (a producer waiting for a free slot, an epilogue waiting
+// for a whole tile's MMAs, a drain): a thread whose phase has not completed is suspended
+// by the hardware until it completes or kWaitHintNs pass, so these loops poll rarely
+// instead of taking issue slots from the working warps. Latency-critical hand-offs (data
+// landed, a stage converted) poll with mbar_try_wait, which measured faster there.
+constexpr uint32_t kWaitHintNs = 10000;
+QNF4_DEV bool mbar_try_wait_long(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(kWaitHintNs)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait for the phase with the given parity to complete, at most wait_ns.
 // Returns false (and records `code`) on timeout.
 QNF4_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned long long wait_ns,

@@ -127,6 +127,9 @@ struct GemmArgs {
   float* part;            // partial tiles of the tail slices [tail_tiles][tail_splits][tn][128]
   unsigned int* counters; // arrival counters per tail tile (zero on entry, left zero)
   unsigned long long wait_ns;
+  // extents the checked build tests indices against (elements): out, out2, the partial
+  // tiles, the arrival counters and the block constants (code2 or per-channel absmax)
+  int64_t out_elems, out2_elems, part_elems, cnt_elems, cst_elems;
   const uint8_t* packed;  // A_NF4_K: the packed codes [wN, nbk * 32] (for the L2 prefetch)
   int lut;                // NF4 sources: copies of the shared-memory pair table (16 or 32;
                           // nf4_block_lut), 0 = the register byte planes
@@ -170,12 +173,14 @@ __host__ __device__ inline SmemPlan smem_plan(int asrc, int tn, int s1, int s2, 
 // ---------------------------------------------------------------------------
 // device helpers
 // ---------------------------------------------------------------------------
+// Bounded wait; `lng` marks a long wait (producer slots, whole-tile MMAs), which lets
+// the hardware suspend the thread between polls.
 QNF4_DEV bool wait_or_abort(uint64_t* bar, uint32_t parity, unsigned long long wait_ns,
-                            volatile int* abort_flag, unsigned int site) {
+                            volatile int* abort_flag, unsigned int site, bool lng = false) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (lng ? mbar_try_wait_long(bar, parity) : mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
     if (globaltimer() - t0 > wait_ns) {
       set_err(site);
@@ -321,13 +326,15 @@ QNF4_DEV void epi_store(const GemmArgs& g, int64_t row, int64_t col0, const floa
     uint16_t* o = static_cast<uint16_t*>(g.out);
     for (int j = 0; j < n; ++j) {
       const int64_t col = col0 + j;
-      if (col < g.cols) o[row * g.o_rs + col * g.o_cs] = f2bf(v[j]);
+      const int64_t at = row * g.o_rs + col * g.o_cs;
+      if (col < g.cols && in_bounds(at < g.out_elems, 21)) o[at] = f2bf(v[j]);
     }
   } else if (g.epi == EPI_F32) {
     float* o = static_cast<float*>(g.out);
     for (int j = 0; j < n; ++j) {
       const int64_t col = col0 + j;
-      if (col < g.out_cols) o[row * g.o_rs + col * g.o_cs] = v[j] * g.scale;
+      const int64_t at = row * g.o_rs + col * g.o_cs;
+      if (col < g.out_cols && in_bounds(at < g.out_elems, 21)) o[at] = v[j] * g.scale;
     }
   } else {  // EPI_UV: rows are tokens, cols the adapter rank (padded)
     uint16_t* p = static_cast<uint16_t*>(g.out);
@@ -335,8 +342,8 @@ QNF4_DEV void epi_store(const GemmArgs& g, int64_t row, int64_t col0, const floa
     for (int j = 0; j < n; ++j) {
       const int64_t col = col0 + j;
       const uint16_t b = f2bf(v[j] * g.scale);
-      if (p) p[row * 64 + col] = b;
-      if (pt) pt[col * g.o2_ld + row] = b;
+      if (p && in_bounds(row * 64 + col < g.out_elems, 22)) p[row * 64 + col] = b;
+      if (pt && in_bounds(col * g.o2_ld + row < g.out2_elems, 23)) pt[col * g.o2_ld + row] = b;
     }
   }
 }
@@ -529,7 +536,7 @@ __global__ void __launch_bounds__(gemm_threads(NSET), MINB)
         int32_t kc = w.step0 * kStep;
         for (int i = 0; i < nload; ++i) {
           if (!mbar_try_wait(&empty1[s], ph ^ 1) &&
-              !wait_or_abort(&empty1[s], ph ^ 1, g.wait_ns, &s_abort, 11)) {
+              !wait_or_abort(&empty1[s], ph ^ 1, g.wait_ns, &s_abort, 11, true)) {
             ok = false;
             break;
           }
@@ -571,7 +578,7 @@ __global__ void __launch_bounds__(gemm_threads(NSET), MINB)
       bool late = false;
       for (int s = 0; s < nslots && !late; ++s) {
         const int j = s + S1 * ((issued - 1 - s) / S1);
-        while (!mbar_try_wait(&full1[s], (j / S1) & 1)) {
+        while (!mbar_try_wait_long(&full1[s], (j / S1) & 1)) {
           if (globaltimer() - t0 > drain_ns(g.wait_ns)) {
             set_err(12);
             late = true;
@@ -603,7 +610,7 @@ __global__ void __launch_bounds__(gemm_threads(NSET), MINB)
         const Unit w = unit_of(g, u);
         // the previous unit's epilogue must have read the accumulator
         if (k > 0) {
-          if (!wait_or_abort(&acc_empty, (k - 1) & 1, g.wait_ns, &s_abort, 26)) {
+          if (!wait_or_abort(&acc_empty, (k - 1) & 1, g.wait_ns, &s_abort, 26, true)) {
             ok = false;
             break;
           }
@@ -671,7 +678,7 @@ __global__ void __launch_bounds__(gemm_threads(NSET), MINB)
       // Drain: every MMA of this CTA completes before TMEM and smem are released.
       mma_commit(&fin_bar);
       const uint64_t t0 = globaltimer();
-      while (!mbar_try_wait(&fin_bar, 0)) {
+      while (!mbar_try_wait_long(&fin_bar, 0)) {
         if (globaltimer() - t0 > drain_ns(g.wait_ns)) {
           set_err(25);
           break;
@@ -729,7 +736,7 @@ __global__ void __launch_bounds__(gemm_threads(NSET), MINB)
     // same units in the same order; it returns false for all of them alike once the
     // CTA has aborted, so all take the same path through the named barriers.
     auto epilogue = [&](int u, int k) -> bool {
-      wait_or_abort(&acc_bar, k & 1, g.wait_ns, &s_abort, 41);
+      wait_or_abort(&acc_bar, k & 1, g.wait_ns, &s_abort, 41, true);
       named_sync(1, NCONV);
       if (ct == 0) s_last = s_abort ? 0 : 2;
       named_sync(1, NCONV);
@@ -789,27 +796,35 @@ __global__ void __launch_bounds__(gemm_threads(NSET), MINB)
         mbar_arrive(&acc_empty);
       } else {
         const int64_t tsz = static_cast<int64_t>(g.tn) * 128;
-        float* mine = g.part + (static_cast<int64_t>(w.pt) * w.splits + w.z) * tsz;
+        const int64_t mine_at = (static_cast<int64_t>(w.pt) * w.splits + w.z) * tsz;
+        float* mine = g.part + mine_at;
+        const bool part_ok = in_bounds(mine_at + tsz <= g.part_elems, 24);
         for (int ck = set; ck < nchunk; ck += NSET) {
           const int c0 = ck * 16;
           uint32_t r[16];
           tmem_ld16(taddr + c0, r);
           tmem_wait_ld();
+          if (part_ok) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) __stcg(mine + (c0 + j) * 128 + lrow, __uint_as_float(r[j]));
+            for (int j = 0; j < 16; ++j) __stcg(mine + (c0 + j) * 128 + lrow, __uint_as_float(r[j]));
+          }
         }
         tc_fence_before();
         mbar_arrive(&acc_empty);
         __threadfence();
         named_sync(1, NCONV);
         if (ct == 0) {
-          const unsigned int old = atomicAdd(g.counters + w.pt, 1u);
-          s_last = (old == static_cast<unsigned int>(w.splits - 1)) ? 1 : 0;
+          s_last = 0;
+          if (in_bounds(w.pt < g.cnt_elems, 25)) {
+            const unsigned int old = atomicAdd(g.counters + w.pt, 1u);
+            s_last = (old == static_cast<unsigned int>(w.splits - 1)) ? 1 : 0;
+          }
         }
         named_sync(1, NCONV);
         if (s_last) {
           __threadfence();
           const float* all = g.part + static_cast<int64_t>(w.pt) * w.splits * tsz;
+          in_bounds((static_cast<int64_t>(w.pt) + 1) * w.splits * tsz <= g.part_elems, 26);
           // Pieces of RW columns: in the wide dequantizing kernels the next unit's
           // conversion state stays live across the epilogue within a tight register
           // budget, so their reduction takes 8 columns; the others take 16 (half the
@@ -881,6 +896,7 @@ __global__ void __launch_bounds__(gemm_threads(NSET), MINB)
         bnext = first_block(wn);
         vnext = rowok && set < wn.nst && (ASRC == A_NF4_K || cn < g.wN);
       }
+      if (vnext && !in_bounds(bnext < g.cst_elems, 27)) vnext = false;
       if (vnext) {
         if (ASRC == A_CHANQ_MN) {
           snext = __ldg(g.cq_absmax + bnext);  // the group's absmax is its constant
@@ -968,6 +984,7 @@ __global__ void __launch_bounds__(gemm_threads(NSET), MINB)
           bnext += bstep;
           cn += NSET * kStep;
           vnext = rowok && (ASRC == A_NF4_K || cn < g.wN);
+          if (vnext && !in_bounds(bnext < g.cst_elems, 27)) vnext = false;
           if (vnext) {
             if (ASRC == A_CHANQ_MN) {
               snext = __ldg(g.cq_absmax + bnext);

@@ -43,37 +43,8 @@ QNF4_DEV float rcp_approx(float x) {
   return r;
 }
 
-// Two fp32 lanes in one 64-bit register, and the packed fma of sm_100 (two IEEE
-// single-precision fused multiply-adds, round to nearest even: each lane is fmaf).
-QNF4_DEV uint64_t f2_pack(float lo, float hi) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
-}
-QNF4_DEV float2 f2_unpack(uint64_t v) {
-  float2 r;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
-  return r;
-}
-QNF4_DEV uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
 
-// Shared loads of read-only tables (filled before a CTA barrier); not volatile, so the
-// compiler may schedule them freely.
-QNF4_DEV uint32_t lds_u32q(uint32_t addr) {
-  uint32_t v;
-  asm("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
-  return v;
-}
-QNF4_DEV float lds_f32(uint32_t addr) {
-  float v;
-  asm("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
-  return v;
-}
-
+constexpr int kQuantMaxGrid = 1024;  // most quantize CTAs; the workspace holds that many partials
 constexpr int kQChunkBlocks = 128;  // 64-element blocks per streamed chunk (16 KB of bf16)
 constexpr int kQStages = 4;         // chunks in flight per CTA
 constexpr int kQWorkers = 8;        // worker warps; one more warp issues the copies
@@ -101,18 +72,31 @@ QNF4_DEV bool warp_wait(uint64_t* bar, uint32_t parity, unsigned long long wait_
   return __all_sync(0xffffffffu, ok);
 }
 
+// Shared loads of read-only tables (filled before a CTA barrier), by 32-bit shared address;
+// not volatile, so the compiler may schedule them freely.
+QNF4_DEV uint32_t lds_u32q(uint32_t addr) {
+  uint32_t v;
+  asm("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+QNF4_DEV float lds_f32q(uint32_t addr) {
+  float v;
+  asm("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+  return v;
+}
+// (d >> 31) + t: the sign bit of d added to t's bits (one multiply-add)
+QNF4_DEV uint32_t sign_add(uint32_t d, uint32_t t) {
+  uint32_t r;
+  asm("mad.hi.u32 %0, %1, 2, %2;" : "=r"(r) : "r"(d), "r"(t));
+  return r;
+}
+
 // max(|a|, |b|) per bf16 lane, NaN if either lane is NaN; the sign bits of the result
 // are not the absolute value's (xorsign), so callers mask them.
 QNF4_DEV uint32_t bmax_abs2(uint32_t a, uint32_t b) {
   uint32_t d;
   asm("max.NaN.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
   return d;
-}
-// (d >> 31) + t: the sign bit of d added to t's bits
-QNF4_DEV uint32_t sign_add(uint32_t d, uint32_t t) {
-  uint32_t r;
-  asm("mad.hi.u32 %0, %1, 2, %2;" : "=r"(r) : "r"(d), "r"(t));
-  return r;
 }
 
 // Blockwise NF4 quantization, streamed: each CTA walks its chunks (chunk c holds
@@ -191,7 +175,7 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
         if (!mbar_try_wait(&empty[st], ph ^ 1u)) {
           const uint64_t t0 = globaltimer();
           bool ok = false;
-          while (!(ok = mbar_try_wait(&empty[st], ph ^ 1u))) {
+          while (!(ok = mbar_try_wait_long(&empty[st], ph ^ 1u))) {
             if (s_abort) break;
             if (globaltimer() - t0 > wait_ns) {
               set_err(53);
@@ -204,6 +188,7 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
         const int64_t c = blockIdx.x + j * gridDim.x;
         const int64_t nb = min(static_cast<int64_t>(kQChunkBlocks), nblocks - c * kQChunkBlocks);
         const uint32_t bytes = static_cast<uint32_t>(nb) * 128u;
+        if (!in_bounds(nb > 0 && c * kQChunkBlocks + nb <= nblocks, 1)) break;
         mbar_expect_tx(&full[st], bytes);
         bulk_load(qsm + st * kQChunkBytes, W + c * kQChunkBlocks * 64, bytes, &full[st]);
         issued = j + 1;
@@ -215,7 +200,7 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
       // Drain: every copy issued must land before the CTA exits (one deadline).
       const uint64_t t0 = globaltimer();
       for (int64_t jj = max(static_cast<int64_t>(0), issued - kQStages); jj < issued; ++jj) {
-        while (!mbar_try_wait(&full[jj % kQStages], static_cast<uint32_t>((jj / kQStages) & 1))) {
+        while (!mbar_try_wait_long(&full[jj % kQStages], static_cast<uint32_t>((jj / kQStages) & 1))) {
           if (globaltimer() - t0 > drain_ns(wait_ns)) {
             set_err(52);
             break;
@@ -227,9 +212,9 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
     // ---------------------------------------------------------------- workers
     const int H = tab.bin_h;
     const float hf = static_cast<float>(H);
-    const uint64_t mg2 = f2_pack(hf + 12582912.0f, hf + 12582912.0f);
+    const float2 mg2 = make_float2(hf + 12582912.0f, hf + 12582912.0f);
     // bin k's entry sits at shared address kb * 4 + toff, kb = 0x4B400000 + k being the
-    // bits of the magic fma's result (32-bit wrap-around)
+    // bits of the magic fma's result (32-bit wrap-around): one multiply-add
     const uint32_t toff = smem_u32(s_tc) - 0x4B400000u * 4u;
     const uint32_t lvoff = smem_u32(s_lvc);
     const int l4 = tid & 3;     // elements 16 l4 .. 16 l4 + 15 of the block
@@ -273,32 +258,33 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
           exact = false;
         } else if (!exact) {
           const float hr = hf * rcp_approx(c);
-          const uint64_t hr2 = f2_pack(hr, hr), nc2 = f2_pack(-c, -c);
-          uint64_t wp[8];
+          const float2 hr2 = make_float2(hr, hr), nc2 = make_float2(-c, -c);
+          float2 wp[8];
           float dmin = 3.0e38f;
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            wp[e] = f2_pack(bf16lo(wd[e]), bf16hi(wd[e]));
-            const float2 kb = f2_unpack(f2_fma(wp[e], hr2, mg2));
+            wp[e] = make_float2(bf16lo(wd[e]), bf16hi(wd[e]));
+            const float2 kb = __ffma2_rn(wp[e], hr2, mg2);
             const uint32_t ta = lds_u32q(__float_as_uint(kb.x) * 4u + toff);
             const uint32_t tb = lds_u32q(__float_as_uint(kb.y) * 4u + toff);
-            const float2 d = f2_unpack(f2_fma(f2_pack(__uint_as_float(ta), __uint_as_float(tb)), nc2, wp[e]));
-            dmin = fminf(dmin, fminf(fabsf(d.x), fabsf(d.y)));
-            mc[2 * e] = sign_add(__float_as_uint(d.x), ta) & 15u;
-            mc[2 * e + 1] = sign_add(__float_as_uint(d.y), tb) & 15u;
+            const float dx = fmaf(-c, __uint_as_float(ta), wp[e].x);
+            const float dy = fmaf(-c, __uint_as_float(tb), wp[e].y);
+            dmin = fminf(dmin, fminf(fabsf(dx), fabsf(dy)));
+            mc[2 * e] = sign_add(__float_as_uint(dx), ta) & 15u;
+            mc[2 * e + 1] = sign_add(__float_as_uint(dy), tb) & 15u;
           }
           exact = !(dmin > c * 0x1p-18f);
           if (SSE && !exact) {
             // r = w - c q[code], two running sums of r^2 (even and odd elements)
-            uint64_t acc2 = f2_pack(0.f, 0.f);
+            float2 acc2 = make_float2(0.f, 0.f);
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-              const uint64_t q2 = f2_pack(lds_f32(lvoff + 4u * mc[2 * e]), lds_f32(lvoff + 4u * mc[2 * e + 1]));
-              const uint64_t r2 = f2_fma(q2, nc2, wp[e]);
-              acc2 = f2_fma(r2, r2, acc2);
+              const float2 r2 = __ffma2_rn(make_float2(lds_f32q(lvoff + 4u * mc[2 * e]),
+                                                       lds_f32q(lvoff + 4u * mc[2 * e + 1])),
+                                           nc2, wp[e]);
+              acc2 = __ffma2_rn(r2, r2, acc2);
             }
-            const float2 a2 = f2_unpack(acc2);
-            sse = a2.x + a2.y;
+            sse = acc2.x + acc2.y;
           }
         }
         if (exact) {
@@ -335,8 +321,8 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
           uint2 out;
           out.x = sw ? pw[1] : pw[0];  // piece 2 l4
           out.y = sw ? pw[0] : pw[1];  // piece 2 l4 + 1
-          reinterpret_cast<uint2*>(packed)[blk * 4 + l4] = out;
-          if (l4 == 0) {
+          if (in_bounds(blk < nblocks, 2)) reinterpret_cast<uint2*>(packed)[blk * 4 + l4] = out;
+          if (l4 == 0 && in_bounds(blk < nblocks, 2)) {
             absmax[blk] = c;
             asum += static_cast<double>(c);
           }
@@ -368,17 +354,17 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
     if ((tid & 31) == 0 && warp < kQWorkers) s_asum[warp] = asum;
   }
   __syncthreads();
-  if (WRITE && asum_part && tid == 0) {
+  if (WRITE && asum_part && tid == 0 && in_bounds(blockIdx.x < kQuantMaxGrid, 3)) {
     double t = 0.0;
     for (int i = 0; i < kQWorkers; ++i) t += s_asum[i];
     asum_part[blockIdx.x] = t;  // exact: bf16-derived constants sum exactly in float64
   }
-  if (SSE && tid == 0) {
+  if (SSE && tid == 0 && in_bounds(blockIdx.x < kQuantMaxGrid, 3)) {
     double t = 0.0;
     for (int i = 0; i < kQWorkers; ++i) t += s_red[i];
     sse_part[blockIdx.x] = t;
   }
-  if (CNT && tid == 0) {
+  if (CNT && tid == 0 && in_bounds(blockIdx.x < kQuantMaxGrid, 3)) {
     unsigned long long t = 0;
     for (int i = 0; i < kQWorkers; ++i) t += s_cnt[i];
     cnt_part[blockIdx.x] = static_cast<double>(t);  // exact below 2^53
@@ -427,7 +413,7 @@ __global__ void __launch_bounds__(256) k_dq_partial(const float* __restrict__ c,
     if (threadIdx.x < o) s[threadIdx.x] += s[threadIdx.x + o];
     __syncthreads();
   }
-  if (threadIdx.x == 0) part[blockIdx.x] = s[0];
+  if (threadIdx.x == 0 && in_bounds(blockIdx.x < kDqPartials, 4)) part[blockIdx.x] = s[0];
 }
 
 // Each CTA reduces the partials to the tensor mean (bf16-derived constants sum
@@ -488,7 +474,7 @@ __global__ void __launch_bounds__(256) k_dq_encode(const float* __restrict__ c, 
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     const float s = (m == 0.f) ? 0.f : __fdiv_rn(m, 448.f);
-    if (lane == 0) scale2[j] = s;
+    if (lane == 0 && in_bounds(j < nb2, 5)) scale2[j] = s;
     uint8_t q[8];
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
@@ -525,6 +511,7 @@ __global__ void __launch_bounds__(256) k_dequant(const uint32_t* __restrict__ pa
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t b = i >> 3;  // 8 groups of 8 weights per 64-block
+    if (!in_bounds(b < (n8 >> 3), 6)) continue;
     const float ch = fmaf(e4m3_to_f32(code2[b]), scale2[b >> 8], mu);
     const uint32_t word = packed[i];
     float o[8];

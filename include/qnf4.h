@@ -57,7 +57,9 @@ typedef enum {
   QNF4_ERR_ALIGN = 3,
   QNF4_ERR_CUDA = 4,
   QNF4_ERR_TIMEOUT = 5,
-  QNF4_ERR_WORKSPACE = 6
+  QNF4_ERR_WORKSPACE = 6,
+  QNF4_ERR_BOUNDS = 7   /* checked build (libqnf4_checked.so) only: a kernel index was
+                           outside its buffer; the access was skipped (see qnf4_check) */
 } qnf4_status;
 
 /* Output dtype selector for qnf4_dequant. */
@@ -311,6 +313,7 @@ QNF4_API size_t qnf4_workspace_size(int32_t op, int64_t N, int64_t K, int64_t M,
 
 /* Synchronise `stream`, then report and clear the device error flag: QNF4_OK, or
  * QNF4_ERR_TIMEOUT if a bounded wait inside a kernel gave up since the last check,
+ * QNF4_ERR_BOUNDS (checked build only) if a kernel index fell outside its buffer,
  * or QNF4_ERR_CUDA if the stream holds a CUDA error or a LoftQ eigensolve reported
  * failure (cuSOLVER info != 0). */
 QNF4_API qnf4_status qnf4_check(void* stream);

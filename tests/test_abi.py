@@ -47,6 +47,11 @@ def test_library_exports_every_declared_symbol(q):
     # nothing else leaks out under the qnf4_ prefix, and every binding signature exists
     assert exported == declared
     assert set(q._lib.SIGNATURES) == declared
+    # the checked build (index checks compiled into the kernels) exports the same ABI
+    checked = os.path.join(os.path.dirname(q._lib.LIB_PATH), "libqnf4_checked.so")
+    out = subprocess.run(["nm", "-D", "--defined-only", checked], capture_output=True,
+                         text=True, check=True).stdout
+    assert set(re.findall(r"\bT (qnf4_\w+)", out)) == declared
 
 
 def test_host_codebook_matches_oracle_bit_exactly(q):
