@@ -77,19 +77,23 @@ QuantTab make_tab() {
   std::memcpy(q.thr, t.thr, sizeof(q.thr));
   std::memcpy(q.levels, t.levels, sizeof(q.levels));
   q.bin_h = t.bin_h;
-  std::memcpy(q.bin_tc, t.bin_tc, sizeof(q.bin_tc));
+  std::memcpy(q.bin_th, t.bin_th, sizeof(q.bin_th));
   return q;
 }
 
 int quant_grid(int64_t nblocks) {
-  // persistent: kQCtasPerSm streaming CTAs per SM, never more CTAs than chunks
+  // persistent: kQCtasPerSm streaming CTAs per SM, never more warps than chunks
   const int64_t chunks = (nblocks + kQChunkBlocks - 1) / kQChunkBlocks;
-  return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(chunks, num_sms() * kQCtasPerSm)));
+  const int64_t ctas = (chunks + kQWorkers - 1) / kQWorkers;
+  return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(ctas, num_sms() * kQCtasPerSm)));
 }
 
 bool g_quant_smem_set[64] = {};
 
 qnf4_status quant_smem_attr() {
+  // the quantizer's code search needs the bin table (always found for the NF4 levels)
+  if (nf4_tables().bin_h < 1 || nf4_tables().bin_h > kQMaxH)
+    return fail(QNF4_ERR_ARG, "internal: no NF4 bin table the quantizer can hold");
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !g_quant_smem_set[dev]) {
@@ -156,6 +160,13 @@ bool make_map(CUtensorMap* m, const void* ptr, bool u8, uint64_t inner, uint64_t
                         sw128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+// The quantizer's view of a weight: a [nblocks, 64] bf16 matrix, loaded in boxes of
+// kQChunkBlocks rows with the 128-byte swizzle.
+bool quant_map(CUtensorMap* m, const void* W, int64_t nblocks) {
+  if (nblocks > INT32_MAX) return false;  // the row coordinate is a 32-bit integer
+  return make_map(m, W, false, 64, static_cast<uint64_t>(nblocks), 64, 64, kQChunkBlocks, true);
 }
 
 struct GemmPlan {
@@ -930,16 +941,18 @@ qnf4_status qnf4_nf4_quantize(const void* W, int64_t N, int64_t K, int32_t block
   qnf4_status st = quant_smem_attr();
   if (st != QNF4_OK) return st;
   const int grid = quant_grid(nblocks);
+  CUtensorMap wmap;
+  if (!quant_map(&wmap, W, nblocks)) return map_fail();
   const QuantTab tab = make_tab();
   if (sse) {
     k_nf4_quant<true, true><<<grid, kQThreads, kQSmem, s>>>(
-        static_cast<const uint16_t*>(W), nblocks, reinterpret_cast<uint32_t*>(packed), absmax,
+        wmap, nblocks, reinterpret_cast<uint32_t*>(packed), absmax,
         static_cast<double*>(ws), tab, g_wait_ns);
     k_sum_partials<<<1, 256, 0, s>>>(static_cast<const double*>(ws), grid, sse);
     return launched("nf4_quantize", 2);
   }
   k_nf4_quant<true, false><<<grid, kQThreads, kQSmem, s>>>(
-      static_cast<const uint16_t*>(W), nblocks, reinterpret_cast<uint32_t*>(packed), absmax,
+      wmap, nblocks, reinterpret_cast<uint32_t*>(packed), absmax,
       nullptr, tab, g_wait_ns);
   return launched("nf4_quantize");
 }
@@ -962,16 +975,18 @@ qnf4_status qnf4_quantize_weight(const void* W, int64_t N, int64_t K, uint8_t* p
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int64_t nblocks = N * K / 64;
   const int grid = quant_grid(nblocks);
+  CUtensorMap wmap;
+  if (!quant_map(&wmap, W, nblocks)) return map_fail();
   double* asum = static_cast<double*>(ws);
   double* ssep = asum + kQuantMaxGrid;
   const QuantTab tab = make_tab();
   if (sse) {
     k_nf4_quant<true, true><<<grid, kQThreads, kQSmem, s>>>(
-        static_cast<const uint16_t*>(W), nblocks, reinterpret_cast<uint32_t*>(packed), absmax, ssep,
+        wmap, nblocks, reinterpret_cast<uint32_t*>(packed), absmax, ssep,
         tab, g_wait_ns, 0.f, nullptr, asum);
   } else {
     k_nf4_quant<true, false><<<grid, kQThreads, kQSmem, s>>>(
-        static_cast<const uint16_t*>(W), nblocks, reinterpret_cast<uint32_t*>(packed), absmax,
+        wmap, nblocks, reinterpret_cast<uint32_t*>(packed), absmax,
         nullptr, tab, g_wait_ns, 0.f, nullptr, asum);
   }
   const int64_t nb2 = (nblocks + 255) / 256;
@@ -999,7 +1014,9 @@ qnf4_status qnf4_nf4_recon_error(const void* W, int64_t N, int64_t K, int32_t bl
   qnf4_status st = quant_smem_attr();
   if (st != QNF4_OK) return st;
   const int grid = quant_grid(nblocks);
-  k_nf4_quant<false, true><<<grid, kQThreads, kQSmem, s>>>(static_cast<const uint16_t*>(W), nblocks,
+  CUtensorMap wmap;
+  if (!quant_map(&wmap, W, nblocks)) return map_fail();
+  k_nf4_quant<false, true><<<grid, kQThreads, kQSmem, s>>>(wmap, nblocks,
                                                           nullptr, nullptr, static_cast<double*>(ws),
                                                           make_tab(), g_wait_ns);
   k_sum_partials<<<1, 256, 0, s>>>(static_cast<const double*>(ws), grid, sse);
@@ -1025,9 +1042,11 @@ qnf4_status qnf4_nf4_layer_stats(const void* W, int64_t N, int64_t K, float tau,
   qnf4_status st = quant_smem_attr();
   if (st != QNF4_OK) return st;
   const int grid = quant_grid(nblocks);
+  CUtensorMap wmap;
+  if (!quant_map(&wmap, W, nblocks)) return map_fail();
   double* part = static_cast<double*>(ws);
   k_nf4_quant<false, true, true><<<grid, kQThreads, kQSmem, s>>>(
-      static_cast<const uint16_t*>(W), nblocks, nullptr, nullptr, part, make_tab(), g_wait_ns, tau,
+      wmap, nblocks, nullptr, nullptr, part, make_tab(), g_wait_ns, tau,
       part + kQuantMaxGrid);
   k_sum_partials<<<1, 256, 0, s>>>(part, grid, sse);
   k_sum_partials<<<1, 256, 0, s>>>(part + kQuantMaxGrid, grid, below);

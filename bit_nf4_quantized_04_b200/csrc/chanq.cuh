@@ -136,7 +136,7 @@ __global__ void __launch_bounds__(256) k_chanq_quant(const uint16_t* __restrict_
         code[j] = (__float_as_int(tk.x) & 31) + (__float_as_int(d) >> 31) + 1 + (__float_as_int(d2) >> 31);
         dmin = fminf(dmin, fminf(fabsf(d), fabsf(d2)));
       }
-      if (row_exact || !(dmin > m * 0x1p-17f) || !(m >= 0x1p-100f)) {
+      if (row_exact || !(dmin > m * 0x1p-17f) || !(m >= 0x1p-100f && m < 0x1p64f)) {
 #pragma unroll
         for (int j = 0; j < 8; ++j) code[j] = chanq_code_exact(w[j], m, s_t[wib], nt);
       }

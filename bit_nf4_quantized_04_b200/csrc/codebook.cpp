@@ -135,10 +135,22 @@ void build(Nf4Tables& t) {
       int c = 0;
       for (int k = 0; k < 15; ++k) c += static_cast<double>(t.thr[k]) <= lo ? 1 : 0;
       const float tk = c < 15 ? t.thr[c] : 2.0f;
-      uint32_t bits;
-      std::memcpy(&bits, &tk, 4);
-      bits = (bits & ~15u) | static_cast<uint32_t>((14 - c) & 15);
-      std::memcpy(&t.bin_tc[b], &bits, 4);
+      // entry = (t_k exactly, h'_k): h_k is half the fp32 spacing below t_k, so that
+      // t_k - h_k is the midpoint under which RN(w / c) rounds below t_k; h'_k moves it by
+      // 2^-15 h_k towards the side an exact tie rounds to (up when t_k's mantissa is even,
+      // round half to even), and carries (c_k + 1) mod 16 in its 4 lowest mantissa bits
+      // (a shift of at most 15 ulp, far inside that 2^-15 move)
+      const double h = (static_cast<double>(tk) -
+                        static_cast<double>(std::nextafter(tk, -std::numeric_limits<float>::infinity()))) * 0.5;
+      uint32_t tbits;
+      std::memcpy(&tbits, &tk, 4);
+      const bool even = (tbits & 1u) == 0;
+      const float hp = static_cast<float>(even ? h * (1.0 + 0x1p-15) : h * (1.0 - 0x1p-15));
+      uint32_t hbits;
+      std::memcpy(&hbits, &hp, 4);
+      hbits = (hbits & ~15u) | static_cast<uint32_t>((c + 1) & 15);
+      t.bin_th[2 * b] = tk;
+      std::memcpy(&t.bin_th[2 * b + 1], &hbits, 4);
     }
     break;
   }

@@ -40,11 +40,16 @@ QNF4_DEV unsigned long long drain_ns(unsigned long long wait_ns) {
   return wait_ns > kDrainFloorNs ? wait_ns : kDrainFloorNs;
 }
 
-QNF4_DEV uint64_t globaltimer() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
+// Clock of the bounded waits: the SM's cycle counter, a cheap register read. (Reading
+// %globaltimer is a slow special-register access; many warps polling it measured 97-98 %
+// busy on the SM's special-function / conversion pipe, which then throttled everything
+// else that pipe serves.) Limits given in nanoseconds count as 2 cycles per ns (clocks up
+// to 2 GHz), so a wait never gives up before its limit.
+QNF4_DEV long long wait_clock() { return clock64(); }
+QNF4_DEV long long ns_cycles(unsigned long long ns) {
+  return static_cast<long long>(ns < (1ull << 61) ? ns : (1ull << 61)) * 2;
 }
+
 
 // Programmatic dependent launch (PDL) controls.
 QNF4_DEV void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
@@ -107,10 +112,10 @@ QNF4_DEV bool mbar_try_wait_long(uint64_t* bar, uint32_t parity) {
 QNF4_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned long long wait_ns,
                         unsigned int code) {
   if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer();
+  const long long t0 = wait_clock();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (globaltimer() - t0 > wait_ns) {
+    if (wait_clock() - t0 > ns_cycles(wait_ns)) {
       set_err(code);
       return false;
     }

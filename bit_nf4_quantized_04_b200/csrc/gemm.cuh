@@ -178,11 +178,11 @@ __host__ __device__ inline SmemPlan smem_plan(int asrc, int tn, int s1, int s2, 
 QNF4_DEV bool wait_or_abort(uint64_t* bar, uint32_t parity, unsigned long long wait_ns,
                             volatile int* abort_flag, unsigned int site, bool lng = false) {
   if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer();
+  const long long t0 = wait_clock();
   while (true) {
     if (lng ? mbar_try_wait_long(bar, parity) : mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (globaltimer() - t0 > wait_ns) {
+    if (wait_clock() - t0 > ns_cycles(wait_ns)) {
       set_err(site);
       *abort_flag = 1;
       return false;
@@ -574,12 +574,12 @@ __global__ void __launch_bounds__(gemm_threads(NSET), MINB)
       // Drain: the last copy issued into each slot must land before the CTA exits.
       // One deadline covers the whole drain.
       const int nslots = min(issued, S1);
-      const uint64_t t0 = globaltimer();
+      const long long t0 = wait_clock();
       bool late = false;
       for (int s = 0; s < nslots && !late; ++s) {
         const int j = s + S1 * ((issued - 1 - s) / S1);
         while (!mbar_try_wait_long(&full1[s], (j / S1) & 1)) {
-          if (globaltimer() - t0 > drain_ns(g.wait_ns)) {
+          if (wait_clock() - t0 > ns_cycles(drain_ns(g.wait_ns))) {
             set_err(12);
             late = true;
             break;
@@ -677,9 +677,9 @@ __global__ void __launch_bounds__(gemm_threads(NSET), MINB)
       }
       // Drain: every MMA of this CTA completes before TMEM and smem are released.
       mma_commit(&fin_bar);
-      const uint64_t t0 = globaltimer();
+      const long long t0 = wait_clock();
       while (!mbar_try_wait_long(&fin_bar, 0)) {
-        if (globaltimer() - t0 > drain_ns(g.wait_ns)) {
+        if (wait_clock() - t0 > ns_cycles(drain_ns(g.wait_ns))) {
           set_err(25);
           break;
         }

@@ -15,27 +15,8 @@ struct QuantTab {
   float thr[16];
   float levels[16];
   int bin_h;
-  float bin_tc[2 * kMaxHalfBins + 1];
+  float bin_th[2 * (2 * kMaxHalfBins + 1)];
 };
-
-QNF4_DEV uint4 ld_stream_u4(const void* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
-}
-
-// Exact code of w in a block with absolute maximum c > 0: x = RN(w / c) by IEEE
-// division, code = #{k : x >= thr[k]}. Kept out of line: it runs only for values
-// within 2^-19 of a decision threshold (or for blocks with a tiny absmax).
-__device__ __noinline__ int nf4_code_exact(float w, float c, const float* s_thr) {
-  const float x = __fdiv_rn(w, c);
-  int code = 0;
-#pragma unroll
-  for (int k = 0; k < 15; ++k) code += (x >= s_thr[k]) ? 1 : 0;
-  return code;
-}
 
 QNF4_DEV float rcp_approx(float x) {
   float r;
@@ -45,13 +26,15 @@ QNF4_DEV float rcp_approx(float x) {
 
 
 constexpr int kQuantMaxGrid = 1024;  // most quantize CTAs; the workspace holds that many partials
-constexpr int kQChunkBlocks = 128;  // 64-element blocks per streamed chunk (16 KB of bf16)
-constexpr int kQStages = 4;         // chunks in flight per CTA
-constexpr int kQWorkers = 8;        // worker warps; one more warp issues the copies
+constexpr int kQChunkBlocks = 32;   // 64-element blocks per streamed chunk: one per lane
+constexpr int kQStages = 2;         // chunks in flight per warp
+constexpr int kQWorkers = 8;        // warps per CTA, each streaming its own chunks
 constexpr int kQCtasPerSm = 3;      // resident CTAs per SM (registers and shared memory allow it)
-constexpr int kQThreads = 32 * (kQWorkers + 1);
-constexpr uint32_t kQChunkBytes = kQChunkBlocks * 128u;
-constexpr size_t kQSmem = kQStages * kQChunkBytes + 128;
+constexpr int kQThreads = 32 * kQWorkers;
+constexpr uint32_t kQChunkBytes = kQChunkBlocks * 128u;  // 4 KB of bf16
+constexpr int kQMaxH = 16;          // largest bin count H the kernels' table holds
+constexpr int kQTabCopies = 16;     // table copies, one per lane of a half warp
+constexpr size_t kQSmem = static_cast<size_t>(kQWorkers) * kQStages * kQChunkBytes + 1024;
 
 // Spin on a phase with a bound, in every lane of a warp, then agree: the result is
 // the same in all lanes (all observed the phase, or the warp gives up together).
@@ -59,10 +42,10 @@ QNF4_DEV bool warp_wait(uint64_t* bar, uint32_t parity, unsigned long long wait_
                         volatile int* abort_flag, unsigned int site) {
   bool ok = mbar_try_wait(bar, parity);
   if (!ok) {
-    const uint64_t t0 = globaltimer();
+    const long long t0 = wait_clock();
     while (!(ok = mbar_try_wait(bar, parity))) {
       if (*abort_flag) break;
-      if (globaltimer() - t0 > wait_ns) {
+      if (wait_clock() - t0 > ns_cycles(wait_ns)) {
         set_err(site);
         *abort_flag = 1;
         break;
@@ -74,20 +57,28 @@ QNF4_DEV bool warp_wait(uint64_t* bar, uint32_t parity, unsigned long long wait_
 
 // Shared loads of read-only tables (filled before a CTA barrier), by 32-bit shared address;
 // not volatile, so the compiler may schedule them freely.
-QNF4_DEV uint32_t lds_u32q(uint32_t addr) {
-  uint32_t v;
-  asm("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
-  return v;
-}
 QNF4_DEV float lds_f32q(uint32_t addr) {
   float v;
   asm("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
   return v;
 }
-// (d >> 31) + t: the sign bit of d added to t's bits (one multiply-add)
-QNF4_DEV uint32_t sign_add(uint32_t d, uint32_t t) {
+QNF4_DEV float2 lds_f32x2q(uint32_t addr) {
+  float2 v;
+  asm("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr));
+  return v;
+}
+// A 16-byte stage load; volatile and ordered after the mbarrier wait that published it.
+QNF4_DEV uint4 lds_u4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr));
+  return v;
+}
+// t - [s < 0]: the sign of s (as a signed integer) taken from t's bits, one multiply-add
+QNF4_DEV uint32_t sign_sub(uint32_t s, uint32_t t) {
   uint32_t r;
-  asm("mad.hi.u32 %0, %1, 2, %2;" : "=r"(r) : "r"(d), "r"(t));
+  asm("mad.hi.s32 %0, %1, 2, %2;" : "=r"(r) : "r"(s), "r"(t));
   return r;
 }
 
@@ -99,259 +90,253 @@ QNF4_DEV uint32_t bmax_abs2(uint32_t a, uint32_t b) {
   return d;
 }
 
-// Blockwise NF4 quantization, streamed: each CTA walks its chunks (chunk c holds
-// blocks [128 c, 128 c + 128)) through a ring of shared-memory stages. One warp
-// fills the ring with cp.async.bulk; eight worker warps consume it, each releasing a
-// stage with one arrival when done, so no warp waits for the others. Inside a chunk,
-// four threads take one 64-element block, each 16 consecutive elements as two 16-byte
-// shared loads (the first piece alternates between neighbouring blocks, so a quarter
-// warp's loads hit eight different bank groups), and write 8 packed bytes. Optional
-// outputs: WRITE -> packed codes and fp32 absmax; SSE -> per-CTA float64 partial sums
-// of the single-level squared round-trip error (fp32 over a thread's 16 elements);
-// CNT -> per-CTA float64 counts of the elements with |w| < tau (the sparsity of
-// "AQLoRA" §3.1), exact integers; asum_part (optional, with WRITE) -> per-CTA float64
-// sums of the block constants, the partials of the double quantization's tensor mean.
+// Codes of one 64-element block with finite absmax c > 0 (see k_nf4_quant): pw[u] gets
+// the packed bytes of elements 8u .. 8u + 7, acc the squared residuals (SSE). SCALED
+// decides on w f and c f instead (f a power of two), and acc then holds the residuals
+// of the scaled values.
+template <bool SCALED, bool SSE>
+QNF4_DEV void nf4_block_codes(const uint4 (&v)[8], float c, float f, float hf, float2 mg2,
+                              uint32_t toff, uint32_t lvb, uint32_t (&pw)[8], float2& acc) {
+  const float cd = SCALED ? c * f : c;
+  const float hr = hf * rcp_approx(cd);
+  const float2 hr2 = make_float2(hr, hr), nc2 = make_float2(-cd, -cd);
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    const uint32_t wd[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+    uint32_t by[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float2 wp = make_float2(bf16lo(wd[i]), bf16hi(wd[i]));
+      if (SCALED) wp = __fmul2_rn(wp, make_float2(f, f));
+      const float2 kb = __ffma2_rn(wp, hr2, mg2);
+      const float2 ta = lds_f32x2q(__float_as_uint(kb.x) * (8u * kQTabCopies) + toff);
+      const float2 tb = lds_f32x2q(__float_as_uint(kb.y) * (8u * kQTabCopies) + toff);
+      const float sx = fmaf(cd, ta.y, fmaf(-cd, ta.x, wp.x));
+      const float sy = fmaf(cd, tb.y, fmaf(-cd, tb.x, wp.y));
+      const uint32_t ux = sign_sub(__float_as_uint(sx), __float_as_uint(ta.y));  // code in bits 0-3
+      const uint32_t uy = sign_sub(__float_as_uint(sy), __float_as_uint(tb.y));
+      by[i] = ((ux << 4) & 0xF0u) | (uy & 0x0Fu);  // element 2i in the high nibble
+      if (SSE) {
+        const float2 r2 = __ffma2_rn(make_float2(lds_f32q(lvb + 4u * (ux & 15u)),
+                                                 lds_f32q(lvb + 4u * (uy & 15u))),
+                                     nc2, wp);
+        acc = __ffma2_rn(r2, r2, acc);
+      }
+    }
+    pw[u] = __byte_perm(__byte_perm(by[0], by[1], 0x0040), __byte_perm(by[2], by[3], 0x0040), 0x5410);
+  }
+}
+
+// Blockwise NF4 quantization, one 64-element block per lane. Warp g of the grid takes
+// the 32-block chunks g, g + G, ... (G = warps in the grid) through its own ring of
+// kQStages shared-memory stages: its lane 0 issues one TMA tile load per chunk (the
+// weight seen as a [blocks, 64] bf16 matrix, 128-byte swizzle, rows past the end
+// zero-filled) as soon as the warp has finished the chunk that stage held; no copy warp
+// and no barrier between warps. The swizzle puts 16-byte piece u of row r at piece
+// u ^ (r mod 8), so the lanes' reads of piece u fall in eight different bank groups per
+// quarter warp. Optional outputs: WRITE -> packed codes (32 bytes per block) and fp32
+// absmax; SSE -> per-CTA float64 partial sums of the single-level squared round-trip
+// error (fp32 within a block); CNT -> per-CTA float64 counts of the elements with
+// |w| < tau (the sparsity of "AQLoRA" §3.1), exact integers; asum_part (optional, with
+// WRITE) -> per-CTA float64 sums of the block constants, the partials of the double
+// quantization's tensor mean.
 //
-// absmax: max of |w| on the bf16 bit patterns, two elements per instruction; a block
-// holding a NaN or an infinity has magnitude bits >= 0x7F80 and takes the exact path.
-// Code search (see Nf4Tables), for a block with absmax c > 0: the bin
+// absmax: max of |w| on the bf16 bit patterns, two elements per instruction.
+// Code search (see Nf4Tables), for a block with finite absmax c > 0: the bin
 // k = round(w H/c + H) comes from one fused multiply-add with a magic constant
 // (1.5 * 2^23, whose low mantissa bits then hold k), so the table entry's shared
-// address is one multiply-add of those bits; the entry t_k carries (14 - c_k) mod 16 in
-// its low mantissa bits; d = fma(-c, t_k, w) = w - c t_k rounded once, so its sign is
-// exactly that of w/c - t_k, and adding d's sign bit to t_k's bits leaves 15 - code in
-// the low 4 bits (the packed word is complemented once at the end). If any of a
-// thread's 16 values lies within 2^-18 c of its t_k, those 16 take the exact IEEE
-// quotient and the full count. The residual of the error is w - c q[code], one fma
-// with the level read by the (complemented) code.
+// address is one multiply-add of those bits. The entry (t_k, h'_k) gives the decision
+// without a division: d = fma(-c, t_k, w), s = fma(c, h'_k, d); s < 0 exactly when the
+// IEEE quotient RN(w / c) lies below t_k, and subtracting [s < 0] from h'_k's bits
+// leaves the code in the low 4 bits. Blocks with c < 2^-64 or c >= 2^64 decide on w and
+// c scaled by 2^64 or 2^-64 (the same quotient, every intermediate a normal float). An
+// all-zero block takes code 7 (the exact zero level); a block holding an infinity or a
+// NaN takes the code of the IEEE quotient: 7 for a finite w over an infinite c, 0
+// (every comparison false) for the NaN quotients. The residual of the error is
+// w - c q[code], one fma with the level read by the code.
 template <bool WRITE, bool SSE, bool CNT = false>
 __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
-    k_nf4_quant(const uint16_t* __restrict__ W, int64_t nblocks, uint32_t* __restrict__ packed,
-                float* __restrict__ absmax, double* __restrict__ sse_part, QuantTab tab,
-                unsigned long long wait_ns, float tau = 0.f, double* __restrict__ cnt_part = nullptr,
+    k_nf4_quant(const __grid_constant__ CUtensorMap wmap, int64_t nblocks,
+                uint32_t* __restrict__ packed, float* __restrict__ absmax,
+                double* __restrict__ sse_part, QuantTab tab, unsigned long long wait_ns,
+                float tau = 0.f, double* __restrict__ cnt_part = nullptr,
                 double* __restrict__ asum_part = nullptr) {
   extern __shared__ uint8_t qsm_raw[];
-  __shared__ __align__(8) uint64_t full[kQStages], empty[kQStages];
-  __shared__ float s_thr[16];
+  __shared__ __align__(8) uint64_t full[kQWorkers][kQStages];
   __shared__ float s_lv[16];
-  __shared__ float s_lvc[16];  // levels by complemented code: s_lvc[i] = q[15 - i]
-  __shared__ __align__(16) float s_tc[2 * kMaxHalfBins + 1];
+  // entry k of copy j at (k kQTabCopies + j): a half warp's lanes read different copies
+  __shared__ __align__(16) float2 s_th[(2 * kQMaxH + 1) * kQTabCopies];
   __shared__ double s_red[kQWorkers];
   __shared__ unsigned long long s_cnt[kQWorkers];
   __shared__ double s_asum[kQWorkers];
   __shared__ volatile int s_abort;
-  uint8_t* qsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(qsm_raw) + 127) &
-                                            ~static_cast<uintptr_t>(127));
+  uint8_t* qsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(qsm_raw) + 1023) &
+                                            ~static_cast<uintptr_t>(1023));
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
-  for (int i = tid; i < 16; i += kQThreads) {
-    s_thr[i] = tab.thr[i];
-    s_lv[i] = tab.levels[i];
-    s_lvc[i] = tab.levels[15 - i];
+  const int lane = tid & 31;
+  const int H = tab.bin_h;
+  for (int i = tid; i < 16; i += kQThreads) s_lv[i] = tab.levels[i];
+  for (int i = tid; i < (2 * H + 1) * kQTabCopies; i += kQThreads) {
+    const int k = i / kQTabCopies;
+    s_th[i] = make_float2(tab.bin_th[2 * k], tab.bin_th[2 * k + 1]);
   }
-  for (int i = tid; i <= 2 * kMaxHalfBins; i += kQThreads) s_tc[i] = tab.bin_tc[i];
-  const int64_t nchunks = (nblocks + kQChunkBlocks - 1) / kQChunkBlocks;
-  const int64_t my = blockIdx.x < nchunks ? (nchunks - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  if (lane == 0) {
+    for (int i = 0; i < kQStages; ++i) mbar_init(&full[warp][i], 1);
+  }
   if (tid == 0) {
-    for (int i = 0; i < kQStages; ++i) {
-      mbar_init(&full[i], 1);
-      mbar_init(&empty[i], kQWorkers);
-    }
     s_abort = 0;
-    fence_mbar_init();
+    tma_prefetch_desc(&wmap);
   }
+  fence_mbar_init();
   __syncthreads();
 
+  const int64_t nchunks = (nblocks + kQChunkBlocks - 1) / kQChunkBlocks;
+  const int64_t gw = static_cast<int64_t>(blockIdx.x) * kQWorkers + warp;  // this warp
+  const int64_t GW = static_cast<int64_t>(gridDim.x) * kQWorkers;
+  const int64_t my = gw < nchunks ? (nchunks - 1 - gw) / GW + 1 : 0;      // its chunks
+  uint8_t* ring = qsm + warp * (kQStages * kQChunkBytes);
+  uint64_t* fb = full[warp];
+  // lane 0 streams chunk j of this warp into stage j % kQStages (the whole box counts
+  // towards the transaction bytes, zero-filled rows included)
+  auto issue = [&](int64_t j) {
+    const int64_t c = gw + j * GW;
+    if (!in_bounds(c < nchunks, 1)) return;
+    uint64_t* bar = &fb[j % kQStages];
+    mbar_expect_tx(bar, kQChunkBytes);
+    tma_load_2d(ring + (j % kQStages) * kQChunkBytes, &wmap, bar, 0,
+                static_cast<int32_t>(c * kQChunkBlocks));
+  };
+  if (lane == 0) {
+    for (int64_t j = 0; j < min(my, static_cast<int64_t>(kQStages)); ++j) issue(j);
+  }
+
   double acc = 0.0;
-  double asum = 0.0;       // this thread's block constants (asum_part; block leaders only)
-  unsigned int below = 0;  // this thread's elements with |w| < tau (CNT)
-  if (warp == kQWorkers) {
-    // ---------------------------------------------------------------- producer
-    if ((tid & 31) == 0) {
-      int st = 0;
-      uint32_t ph = 0;
-      int64_t issued = 0;
-      for (int64_t j = 0; j < my; ++j) {
-        if (!mbar_try_wait(&empty[st], ph ^ 1u)) {
-          const uint64_t t0 = globaltimer();
-          bool ok = false;
-          while (!(ok = mbar_try_wait_long(&empty[st], ph ^ 1u))) {
-            if (s_abort) break;
-            if (globaltimer() - t0 > wait_ns) {
-              set_err(53);
-              s_abort = 1;
-              break;
-            }
-          }
-          if (!ok) break;
-        }
-        const int64_t c = blockIdx.x + j * gridDim.x;
-        const int64_t nb = min(static_cast<int64_t>(kQChunkBlocks), nblocks - c * kQChunkBlocks);
-        const uint32_t bytes = static_cast<uint32_t>(nb) * 128u;
-        if (!in_bounds(nb > 0 && c * kQChunkBlocks + nb <= nblocks, 1)) break;
-        mbar_expect_tx(&full[st], bytes);
-        bulk_load(qsm + st * kQChunkBytes, W + c * kQChunkBlocks * 64, bytes, &full[st]);
-        issued = j + 1;
-        if (++st == kQStages) {
-          st = 0;
-          ph ^= 1u;
-        }
-      }
-      // Drain: every copy issued must land before the CTA exits (one deadline).
-      const uint64_t t0 = globaltimer();
-      for (int64_t jj = max(static_cast<int64_t>(0), issued - kQStages); jj < issued; ++jj) {
-        while (!mbar_try_wait_long(&full[jj % kQStages], static_cast<uint32_t>((jj / kQStages) & 1))) {
-          if (globaltimer() - t0 > drain_ns(wait_ns)) {
-            set_err(52);
-            break;
-          }
+  double asum = 0.0;       // this lane's block constants (asum_part)
+  unsigned int below = 0;  // this lane's elements with |w| < tau (CNT)
+  const uint32_t taub = __float_as_uint(tau);
+  const float hf = static_cast<float>(H);
+  const float2 mg2 = make_float2(hf + 12582912.0f, hf + 12582912.0f);
+  // bin k's entry of this lane's copy sits at shared address kb * 8 kQTabCopies + toff,
+  // kb = 0x4B400000 + k being the bits of the magic fma's result (32-bit wrap-around)
+  const uint32_t toff = smem_u32(s_th) + (lane & (kQTabCopies - 1)) * 8u -
+                        0x4B400000u * (8u * kQTabCopies);
+  const uint32_t lvb = smem_u32(s_lv);
+  int64_t done = 0;  // chunks consumed (their copies have landed)
+  for (int64_t j = 0; j < my; ++j) {
+    if (!warp_wait(&fb[j % kQStages], static_cast<uint32_t>((j / kQStages) & 1), wait_ns, &s_abort, 51))
+      break;
+    done = j + 1;
+    const int64_t blk = (gw + j * GW) * kQChunkBlocks + lane;
+    const bool valid = blk < nblocks;
+    // this lane's row; piece u at row ^ (u << 4) (the swizzle)
+    const uint32_t row = smem_u32(ring + (j % kQStages) * kQChunkBytes) + lane * 128u +
+                         ((lane & 7u) << 4);
+    uint4 v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) v[u] = lds_u4(row ^ (static_cast<uint32_t>(u) << 4));
+    uint32_t m2[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      m2[u] = bmax_abs2(bmax_abs2(bmax_abs2(v[u].x, v[u].y), bmax_abs2(v[u].z, v[u].w)),
+                        bmax_abs2(bmax_abs2(v[u + 4].x, v[u + 4].y), bmax_abs2(v[u + 4].z, v[u + 4].w)));
+    const uint32_t mm = bmax_abs2(bmax_abs2(m2[0], m2[1]), bmax_abs2(m2[2], m2[3]));
+    const uint32_t cb = max(mm & 0x7FFFu, (mm >> 16) & 0x7FFFu);
+    const float c = __uint_as_float(cb << 16);
+    if (CNT && valid) {
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const uint32_t wd[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          // |w| < tau on the magnitude bits (a NaN never counts)
+          below += ((wd[i] << 16) & 0x7FFF0000u) < taub ? 1u : 0u;
+          below += (wd[i] & 0x7FFF0000u) < taub ? 1u : 0u;
         }
       }
     }
-  } else {
-    // ---------------------------------------------------------------- workers
-    const int H = tab.bin_h;
-    const float hf = static_cast<float>(H);
-    const float2 mg2 = make_float2(hf + 12582912.0f, hf + 12582912.0f);
-    // bin k's entry sits at shared address kb * 4 + toff, kb = 0x4B400000 + k being the
-    // bits of the magic fma's result (32-bit wrap-around): one multiply-add
-    const uint32_t toff = smem_u32(s_tc) - 0x4B400000u * 4u;
-    const uint32_t lvoff = smem_u32(s_lvc);
-    const int l4 = tid & 3;     // elements 16 l4 .. 16 l4 + 15 of the block
-    const int grp = tid >> 2;   // 64 groups of four threads
-    const int sw = grp & 1;     // which 16-byte piece this thread loads first
-    const int p0 = 2 * l4 + sw, p1 = 2 * l4 + 1 - sw;
-    int st = 0;
-    uint32_t ph = 0;
-    for (int64_t j = 0; j < my; ++j) {
-      if (!warp_wait(&full[st], ph, wait_ns, &s_abort, 51)) break;
-      const int64_t c0 = (blockIdx.x + j * gridDim.x) * kQChunkBlocks;
-      const int nb = static_cast<int>(min(static_cast<int64_t>(kQChunkBlocks), nblocks - c0));
-      const uint8_t* chunk = qsm + st * kQChunkBytes;
-#pragma unroll 1
-      for (int u = 0; u < kQChunkBlocks / 64; ++u) {
-        const int bl = grp + 64 * u;  // block within the chunk
-        const bool valid = bl < nb;   // groups past a partial chunk's end work on zeros
-        uint4 va = make_uint4(0u, 0u, 0u, 0u), vb = va;
-        if (valid) {
-          va = *reinterpret_cast<const uint4*>(chunk + bl * 128 + p0 * 16);
-          vb = *reinterpret_cast<const uint4*>(chunk + bl * 128 + p1 * 16);
-        }
-        const uint32_t wd[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
-        if (CNT && valid) {
-#pragma unroll
-          for (int e = 0; e < 8; ++e)
-            below += (fabsf(bf16lo(wd[e])) < tau ? 1u : 0u) + (fabsf(bf16hi(wd[e])) < tau ? 1u : 0u);
-        }
-        uint32_t m2 = bmax_abs2(bmax_abs2(bmax_abs2(wd[0], wd[1]), bmax_abs2(wd[2], wd[3])),
-                                bmax_abs2(bmax_abs2(wd[4], wd[5]), bmax_abs2(wd[6], wd[7])));
-        uint32_t cb = max(m2 & 0x7FFFu, (m2 >> 16) & 0x7FFFu);
-        cb = max(cb, __shfl_xor_sync(0xffffffffu, cb, 1));
-        cb = max(cb, __shfl_xor_sync(0xffffffffu, cb, 2));
-        const float c = __uint_as_float(cb << 16);
-        uint32_t mc[16];  // 15 - code of the thread's elements: pieces p0 (0..7), p1 (8..15)
-        float sse = 0.f;
-        bool exact = cb >= 0x7F80u || H == 0 || !(c >= 0x1p-100f);
-        if (cb == 0u) {
-#pragma unroll
-          for (int e = 0; e < 16; ++e) mc[e] = 8u;  // the exact-zero level (error 0)
-          exact = false;
-        } else if (!exact) {
-          const float hr = hf * rcp_approx(c);
-          const float2 hr2 = make_float2(hr, hr), nc2 = make_float2(-c, -c);
-          float2 wp[8];
-          float dmin = 3.0e38f;
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            wp[e] = make_float2(bf16lo(wd[e]), bf16hi(wd[e]));
-            const float2 kb = __ffma2_rn(wp[e], hr2, mg2);
-            const uint32_t ta = lds_u32q(__float_as_uint(kb.x) * 4u + toff);
-            const uint32_t tb = lds_u32q(__float_as_uint(kb.y) * 4u + toff);
-            const float dx = fmaf(-c, __uint_as_float(ta), wp[e].x);
-            const float dy = fmaf(-c, __uint_as_float(tb), wp[e].y);
-            dmin = fminf(dmin, fminf(fabsf(dx), fabsf(dy)));
-            mc[2 * e] = sign_add(__float_as_uint(dx), ta) & 15u;
-            mc[2 * e + 1] = sign_add(__float_as_uint(dy), tb) & 15u;
-          }
-          exact = !(dmin > c * 0x1p-18f);
-          if (SSE && !exact) {
-            // r = w - c q[code], two running sums of r^2 (even and odd elements)
-            float2 acc2 = make_float2(0.f, 0.f);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const float2 r2 = __ffma2_rn(make_float2(lds_f32q(lvoff + 4u * mc[2 * e]),
-                                                       lds_f32q(lvoff + 4u * mc[2 * e + 1])),
-                                           nc2, wp[e]);
-              acc2 = __ffma2_rn(r2, r2, acc2);
-            }
-            sse = acc2.x + acc2.y;
-          }
-        }
-        if (exact) {
-          // out of line: the IEEE quotient and the full threshold count (values near a
-          // threshold, tiny or non-finite absmax, or no bin table)
-          float a = 0.f, b = 0.f;
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float w0 = bf16lo(wd[e]), w1 = bf16hi(wd[e]);
-            const int k0 = nf4_code_exact(w0, c, s_thr), k1 = nf4_code_exact(w1, c, s_thr);
-            mc[2 * e] = static_cast<uint32_t>(15 - k0);
-            mc[2 * e + 1] = static_cast<uint32_t>(15 - k1);
-            if (SSE) {
-              const float r0 = fmaf(s_lv[k0], -c, w0), r1 = fmaf(s_lv[k1], -c, w1);
-              a = fmaf(r0, r0, a);
-              b = fmaf(r1, r1, b);
-            }
-          }
-          sse = a + b;
-        }
-        const int64_t blk = c0 + bl;
-        if (WRITE && valid) {
-          // element 2i in the high nibble of byte i; the complemented nibbles are
-          // packed, then the word is complemented once
-          uint32_t pw[2];
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const uint32_t b0 = mc[8 * h + 0] * 16u + mc[8 * h + 1];
-            const uint32_t b1 = mc[8 * h + 2] * 16u + mc[8 * h + 3];
-            const uint32_t b2 = mc[8 * h + 4] * 16u + mc[8 * h + 5];
-            const uint32_t b3 = mc[8 * h + 6] * 16u + mc[8 * h + 7];
-            pw[h] = ~__byte_perm(__byte_perm(b0, b1, 0x0040), __byte_perm(b2, b3, 0x0040), 0x5410);
-          }
-          uint2 out;
-          out.x = sw ? pw[1] : pw[0];  // piece 2 l4
-          out.y = sw ? pw[0] : pw[1];  // piece 2 l4 + 1
-          if (in_bounds(blk < nblocks, 2)) reinterpret_cast<uint2*>(packed)[blk * 4 + l4] = out;
-          if (l4 == 0 && in_bounds(blk < nblocks, 2)) {
-            absmax[blk] = c;
-            asum += static_cast<double>(c);
-          }
-        }
-        if (SSE && valid) acc += static_cast<double>(sse);
+    uint32_t pw[8];
+    float2 acc2 = make_float2(0.f, 0.f);
+    float ssq = 1.f;  // a scaled block's residuals times ssq are the true ones
+    if (cb - 1u < 0x7F7Fu) {  // 0 < c < inf
+      if (cb >= 0x1F80u && cb < 0x5F80u) {
+        nf4_block_codes<false, SSE>(v, c, 1.f, hf, mg2, toff, lvb, pw, acc2);
+      } else {
+        // c < 2^-64 or c >= 2^64: decide on (w f) / (c f), f = 2^64 or 2^-64, which has
+        // the same quotient and keeps c f, 1 / (c f) and the residuals normal floats (a
+        // w f that lands below them is so far from every threshold that its rounding
+        // cannot change a decision)
+        const bool tiny = cb < 0x1F80u;
+        nf4_block_codes<true, SSE>(v, c, tiny ? 0x1p64f : 0x1p-64f, hf, mg2, toff, lvb, pw, acc2);
+        ssq = tiny ? 0x1p-64f : 0x1p64f;
       }
-      __syncwarp();
-      if ((tid & 31) == 0) mbar_arrive(&empty[st]);  // this warp is done with the stage
-      if (++st == kQStages) {
-        st = 0;
-        ph ^= 1u;
+    } else {
+      // c = 0 (all zeros: code 7) or a non-finite block: code 7 where the quotient is
+      // a signed zero (finite w, infinite c), else 0 (a NaN quotient)
+      const float2 nc2 = make_float2(-c, -c);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const uint32_t wd[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+        uint32_t by[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint32_t kx = (cb > 0x7F80u || (wd[i] & 0x7FFFu) >= 0x7F80u) ? 0u : 7u;
+          const uint32_t ky = (cb > 0x7F80u || (wd[i] & 0x7FFF0000u) >= 0x7F800000u) ? 0u : 7u;
+          by[i] = (kx << 4) | ky;
+          if (SSE) {
+            const float2 r2 = __ffma2_rn(make_float2(s_lv[kx], s_lv[ky]), nc2,
+                                         make_float2(bf16lo(wd[i]), bf16hi(wd[i])));
+            acc2 = __ffma2_rn(r2, r2, acc2);
+          }
+        }
+        pw[u] = __byte_perm(__byte_perm(by[0], by[1], 0x0040), __byte_perm(by[2], by[3], 0x0040), 0x5410);
+      }
+    }
+    if (WRITE && valid && in_bounds(blk < nblocks, 2)) {
+      uint4* dst = reinterpret_cast<uint4*>(packed) + blk * 2;
+      dst[0] = make_uint4(pw[0], pw[1], pw[2], pw[3]);
+      dst[1] = make_uint4(pw[4], pw[5], pw[6], pw[7]);
+      absmax[blk] = c;
+      asum += static_cast<double>(c);
+    }
+    if (SSE && valid) acc += static_cast<double>((acc2.x + acc2.y) * ssq * ssq);
+    // the warp is done with this stage: refill it with the chunk kQStages ahead (the
+    // proxy fence orders the lanes' shared reads before the copy engine's writes)
+    __syncwarp();
+    if (lane == 0 && j + kQStages < my) {
+      fence_proxy_async();
+      issue(j + kQStages);
+    }
+  }
+  // Drain: after a give-up, the copies this warp issued but did not consume must land
+  // before the CTA exits (one deadline).
+  if (lane == 0 && done < my) {
+    const int64_t issued = min(my, done + static_cast<int64_t>(kQStages));
+    const long long t0 = wait_clock();
+    for (int64_t jj = done; jj < issued; ++jj) {
+      while (!mbar_try_wait_long(&fb[jj % kQStages], static_cast<uint32_t>((jj / kQStages) & 1))) {
+        if (wait_clock() - t0 > ns_cycles(drain_ns(wait_ns))) {
+          set_err(52);
+          break;
+        }
       }
     }
   }
   if (SSE) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if ((tid & 31) == 0 && warp < kQWorkers) s_red[warp] = acc;
+    if (lane == 0) s_red[warp] = acc;
   }
   if (CNT) {
     unsigned long long b = below;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) b += __shfl_xor_sync(0xffffffffu, b, o);
-    if ((tid & 31) == 0 && warp < kQWorkers) s_cnt[warp] = b;
+    if (lane == 0) s_cnt[warp] = b;
   }
   if (WRITE && asum_part) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) asum += __shfl_xor_sync(0xffffffffu, asum, o);
-    if ((tid & 31) == 0 && warp < kQWorkers) s_asum[warp] = asum;
+    if (lane == 0) s_asum[warp] = asum;
   }
   __syncthreads();
   if (WRITE && asum_part && tid == 0 && in_bounds(blockIdx.x < kQuantMaxGrid, 3)) {

@@ -45,9 +45,9 @@ def _crafted(N, K, seed):
     if flat.numel() >= 128:
         flat[64:128] = 0.03125                # identical values
     if flat.numel() >= 192:
-        flat[128:160] = -1e-30                # tiny constants: one block through the
-        flat[130] = 1e-30                     # reciprocal shortcut, one through the
-        flat[160:192] = 3e-33                 # exact-division path (absmax < 2^-100)
+        flat[128:160] = -1e-30                # tiny constants (absmax < 2^-64: the
+        flat[130] = 1e-30                     # kernels decide on scaled values)
+        flat[160:192] = 3e-33
     if flat.numel() >= 256:
         q = torch.tensor(onf4.codebook())     # values on the grid and at midpoints
         mid = (q[1:] + q[:-1]) / 2
@@ -58,8 +58,8 @@ def _crafted(N, K, seed):
 
 def _near_threshold_blocks(nblocks, seed):
     """bf16 blocks whose normalised values w / absmax fall within 2^-19 of an NF4
-    decision threshold (found by search over the bf16 grid), so the kernels' exact
-    fallback runs, mixed with values at the thresholds' bf16 neighbours."""
+    decision threshold (found by search over the bf16 grid): the values where a
+    rounding slip in the kernels' division-free decision would show."""
     T = onf4.thresholds().astype(np.float64)
     rng = np.random.default_rng(seed)
     mant = np.arange(128, dtype=np.uint32)
@@ -88,6 +88,66 @@ def test_quantize_near_thresholds(q):
     W = _near_threshold_blocks(64, 11)
     assert np.array_equal(f32(W), f32(W).astype(np.float32))
     _check_quant(q, W)
+
+
+def _exhaustive_blocks(cbits_list):
+    """For each bf16 block constant c (given by its bit pattern), every bf16 value w with
+    |w| <= c, both signs and zero, in blocks of 63 such values plus c itself."""
+    blocks = []
+    for cb in cbits_list:
+        mags = np.arange(1, cb + 1, dtype=np.uint32)
+        ws = np.concatenate([mags, mags | 0x8000, [0]]).astype(np.uint32)
+        ws = (ws << 16).view(np.float32)
+        pad = (-ws.size) % 63
+        ws = np.concatenate([ws, np.zeros(pad, np.float32)]).reshape(-1, 63)
+        c = np.full((ws.shape[0], 1), (np.uint32(cb) << 16).view(np.float32))
+        blk = np.concatenate([ws, c], axis=1)
+        for i in range(blk.shape[0]):  # move c around the block
+            j = i % 64
+            blk[i, [j, 63]] = blk[i, [63, j]]
+        blocks.append(blk)
+    out = np.concatenate(blocks)
+    if out.shape[0] % 2:
+        out = np.concatenate([out, np.zeros((1, 64), np.float32)])
+    return torch.from_numpy(out.reshape(-1, 128)).to(torch.bfloat16)
+
+
+def test_quantize_every_bf16_value_under_chosen_constants(q):
+    """Brute force over the bf16 grid: under each block constant c below, every value
+    |w| <= c is coded, and the codes must equal the oracle's IEEE division and threshold
+    count. The constants span subnormals, the scaling edges at 2^-64 and 2^64, 1, and
+    the largest finite bf16, plus random patterns."""
+    rng = np.random.default_rng(123)
+    cbits = [0x0001, 0x0055, 0x0080, 0x0D2B, 0x1F7F, 0x1F80, 0x1F81, 0x3C80, 0x3D4C, 0x3F80,
+             0x3FC0, 0x4000, 0x5F7F, 0x5F80, 0x5FFF, 0x7E80, 0x7F00, 0x7F7F]
+    cbits += [int(v) for v in rng.integers(1, 0x7F80, 14)]
+    W = _exhaustive_blocks(cbits)
+    assert np.array_equal(f32(W), f32(W).astype(np.float32))
+    _check_quant(q, W)
+
+
+def test_quantize_non_finite_blocks(q):
+    """Blocks holding an infinity or a NaN: the codes are those of the IEEE quotient
+    (a finite w over an infinite constant gives a signed zero, code 7; inf / inf and NaN
+    give code 0), the block constant is the infinity or a NaN."""
+    g = torch.Generator().manual_seed(5)
+    w = (torch.randn(8, 64, generator=g) * 0.5)
+    w[0, 3] = float("inf")
+    w[1, 0] = float("-inf")
+    w[2, 10], w[2, 20] = float("inf"), float("-inf")
+    w[3, 7] = float("nan")
+    w[4, :] = float("nan")
+    w[5, 63] = float("inf")
+    w[5, 0] = float("nan")
+    W = w.reshape(4, 128).to(torch.bfloat16)
+    codes, b = onf4.quantize(f32(W))
+    packed, absmax = q.nf4_quantize(W.cuda())
+    torch.cuda.synchronize()
+    assert np.array_equal(packed.cpu().numpy(), onf4.pack(codes))
+    a = absmax.cpu().numpy()
+    assert np.array_equal(np.isnan(a), np.isnan(b))
+    ok = ~np.isnan(b)
+    assert np.array_equal(a[ok].view(np.uint32), b[ok].view(np.uint32))
 
 
 def test_quantize_tiny_layer(q):

@@ -8,10 +8,12 @@ frees its memory and returns, so the context stays usable; qnf4_check then repor
 QNF4_ERR_TIMEOUT with the site.
 
 Here the limit is set far below the time the work needs (100 ns: a 4096-token forward
-holds an accumulator for tens of microseconds, and a quantize worker waits hundreds of
-nanoseconds for its first copy), so waits run out on purpose. Nothing is faulted,
-trapped or left hanging: the kernels end by themselves. After restoring the default
-limit, the next calls must give exactly the results of calls that never timed out.
+holds an accumulator for tens of microseconds), so waits run out on purpose. Nothing is
+faulted, trapped or left hanging: the kernels end by themselves. After restoring the
+default limit, the next calls must give exactly the results of calls that never timed
+out. The quantization kernel is not among the cases: its only waits are each warp's
+waits for its own copies, which one suspended mbarrier poll outlasts, so no limit makes
+them run out.
 """
 import pytest
 import torch
@@ -75,18 +77,3 @@ def test_backward_wait_timeout_reports_and_recovers(q):
     q.check()
     for g, rf in zip(got, ref):
         assert torch.equal(g, rf)
-
-
-def test_quantize_wait_timeout_reports_and_recovers(q):
-    W = synth.llama_weight((11008, 4096), 921, device="cuda")
-    ref, ref_sse = q.quantize_weight(W, sse=True)
-    q.check()
-    q.set_wait_timeout_ns(100)
-    q.quantize_weight(W, sse=True)
-    _expect_timeout(q)
-    q.set_wait_timeout_ns(DEFAULT_NS)
-    got, sse = q.quantize_weight(W, sse=True)
-    q.check()
-    for a, b in ((got.packed, ref.packed), (got.code2, ref.code2), (got.scale2, ref.scale2),
-                 (got.mean, ref.mean), (sse, ref_sse)):
-        assert torch.equal(a, b)
