@@ -20,7 +20,7 @@ LIB = os.path.join(HERE, "libqnf4.so")
 # an index outside its buffer is skipped and reported by qnf4_check as QNF4_ERR_BOUNDS.
 LIB_CHECKED = os.path.join(HERE, "libqnf4_checked.so")
 SOURCES = ["api.cu", "codebook.cpp"]
-HEADERS = ["common.cuh", "quant.cuh", "chanq.cuh", "gemm.cuh", "loftq.cuh", "tables.h"]
+HEADERS = ["common.cuh", "quant.cuh", "chanq.cuh", "gemm.cuh", "decode.cuh", "loftq.cuh", "tables.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -21,6 +21,7 @@
 #include "../../include/qnf4.h"
 #include "chanq.cuh"
 #include "common.cuh"
+#include "decode.cuh"
 #include "gemm.cuh"
 #include "loftq.cuh"
 #include "quant.cuh"
@@ -167,6 +168,38 @@ bool make_map(CUtensorMap* m, const void* ptr, bool u8, uint64_t inner, uint64_t
 bool quant_map(CUtensorMap* m, const void* W, int64_t nblocks) {
   if (nblocks > INT32_MAX) return false;  // the row coordinate is a 32-bit integer
   return make_map(m, W, false, 64, static_cast<uint64_t>(nblocks), 64, 64, kQChunkBlocks, true);
+}
+
+// x [M, K] bf16 seen as [K/64][M][64]: box = 16 column blocks x rows x 64 columns
+// (128-byte swizzle on the 128-byte rows).
+bool make_map_xblocks(CUtensorMap* m, const void* x, uint64_t K, uint64_t M, uint32_t rows) {
+  std::memset(m, 0, sizeof(*m));
+  EncodeFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {64, M, K / 64};
+  cuuint64_t strides[2] = {K * 2, 128};
+  cuuint32_t box[3] = {64, rows, 16};
+  cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(x), dims, strides,
+                        box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// packed [N, K/2] bytes seen as [N][K/256][128] (K a multiple of 256): box = rows x 4
+// column groups x 128 bytes, each row's 512 bytes in order (128-byte swizzle).
+bool make_map_wcols(CUtensorMap* m, const void* packed, uint64_t K, uint64_t N, uint32_t rows) {
+  std::memset(m, 0, sizeof(*m));
+  EncodeFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {128, K / 256, N};
+  cuuint64_t strides[2] = {128, K / 2};
+  cuuint32_t box[3] = {128, 4, rows};
+  cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(packed), dims, strides,
+                        box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
 }
 
 struct GemmPlan {
@@ -501,6 +534,124 @@ qnf4_status run_u(const LinPlan& L, const void* x, const void* A, int64_t M, int
   g.part = part;
   g.counters = cnt;
   return launch_any(L.u, ma, mb, none, none, none, g, s);
+}
+
+// ---------------------------------------------------------------------------
+// Decode-size forward (M <= 16 tokens): k_lora_u, then k_nf4_decode (see decode.cuh)
+// ---------------------------------------------------------------------------
+constexpr int64_t kDecodeMaxTokens = 16;
+
+struct DecodePlan {
+  int Q = 1, P = 1, ks = 1;
+  int64_t rbs = 0;
+  size_t off_up = 0, total = 0;
+};
+
+// One CTA per SM, each holding at most kDecMaxRb row blocks (more CTAs than SMs only
+// when N > 16 kDecMaxRb SMs rows).
+DecodePlan plan_decode(int64_t N, int64_t K, int64_t M, int r, int sms) {
+  DecodePlan d;
+  d.Q = M <= 8 ? 1 : 2;
+  d.rbs = (N + 15) / 16;
+  const int64_t need = (d.rbs + kDecMaxRb - 1) / kDecMaxRb;
+  d.P = static_cast<int>(std::max<int64_t>(need, std::min<int64_t>(sms, d.rbs)));
+  d.ks = static_cast<int>((K + kDecUChunk - 1) / kDecUChunk);
+  size_t o = 0;
+  d.off_up = o;
+  o = align256(o + static_cast<size_t>(d.ks) * r * M * sizeof(float));
+  d.total = o;
+  return d;
+}
+
+bool g_dec_smem_set[2][64] = {};
+
+template <int Q>
+cudaError_t launch_decode(const CUtensorMap& mw0, const CUtensorMap& mw1, const CUtensorMap& mx,
+                          const DecodeArgs& a, int rlo, int w3d, int P, cudaStream_t s) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !g_dec_smem_set[Q - 1][dev]) {
+    const cudaError_t e = cudaFuncSetAttribute(k_nf4_decode<Q>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               static_cast<int>(kDecSmem));
+    if (e != cudaSuccess) return e;
+    g_dec_smem_set[Q - 1][dev] = true;
+  }
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(P);
+  cfg.blockDim = dim3(kDecBlockThreads);
+  cfg.dynamicSmemBytes = kDecSmem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k_nf4_decode<Q>, mw0, mw1, mx, a, rlo, w3d, g_wait_ns);
+}
+
+qnf4_status decode_fwd(const qnf4_weight* w, const void* x, int64_t M, const void* A, const void* B,
+                       int r, float scale, void* h, void* ws, size_t ws_bytes, cudaStream_t s) {
+  const int64_t N = w->N, K = w->K;
+  const DecodePlan d = plan_decode(N, K, M, r, num_sms());
+  if (!ws || ws_bytes < d.total) return fail(QNF4_ERR_WORKSPACE, "workspace too small (%zu < %zu)", ws_bytes, d.total);
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  float* upart = reinterpret_cast<float*>(w8 + d.off_up);
+  DecodeArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.N = N;
+  a.K = K;
+  a.M = static_cast<int>(M);
+  a.r = r;
+  a.nkb = static_cast<int>(K / 64);
+  a.ks = d.ks;
+  a.rbs = d.rbs;
+  a.scale = scale;
+  std::memcpy(a.levels, nf4_tables().levels, sizeof(a.levels));
+  a.code2 = w->code2;
+  a.scale2 = w->scale2;
+  a.mean = w->mean;
+  a.Bm = static_cast<const uint16_t*>(B);
+  a.upart = upart;
+  a.h = static_cast<uint16_t*>(h);
+  a.nb2 = (N * (K / 64) + 255) / 256;
+  if (g_ev_start) cudaEventRecord(g_ev_start, s);
+  {
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(r, d.ks);
+    cfg.blockDim = dim3(128);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, k_lora_u, static_cast<const uint16_t*>(x),
+                                             static_cast<const uint16_t*>(A), K, static_cast<int>(M), r,
+                                             upart);
+    if (e != cudaSuccess) return fail(QNF4_ERR_CUDA, "k_lora_u launch: %s", cudaGetErrorString(e));
+  }
+  // CTAs hold rlo or rlo + 1 row blocks; one packed-weight map per box height, as
+  // [K/256][N][128] (one box of four 128-byte columns) when K is a multiple of 256
+  const int rlo = static_cast<int>(d.rbs / d.P);
+  const int rhi = std::min(rlo + 1, kDecMaxRb);
+  const int w3d = K % 256 == 0 ? 1 : 0;
+  CUtensorMap mw0, mw1, mx;
+  if (w3d) {
+    if (!make_map_wcols(&mw0, w->packed, K, N, 16 * rlo) || !make_map_wcols(&mw1, w->packed, K, N, 16 * rhi))
+      return map_fail();
+  } else {
+    if (!make_map(&mw0, w->packed, true, K / 2, N, K / 2, 128, 16 * rlo, true) ||
+        !make_map(&mw1, w->packed, true, K / 2, N, K / 2, 128, 16 * rhi, true))
+      return map_fail();
+  }
+  if (!make_map_xblocks(&mx, x, K, M, static_cast<uint32_t>(M))) return map_fail();
+  const cudaError_t e = d.Q == 1 ? launch_decode<1>(mw0, mw1, mx, a, rlo, w3d, d.P, s)
+                                 : launch_decode<2>(mw0, mw1, mx, a, rlo, w3d, d.P, s);
+  if (e != cudaSuccess) return fail(QNF4_ERR_CUDA, "k_nf4_decode launch: %s", cudaGetErrorString(e));
+  if (g_ev_stop) cudaEventRecord(g_ev_stop, s);
+  return launched("decode_fwd", 2);
 }
 
 qnf4_status linear_fwd(const BaseSrc& src, const void* x, int64_t M, const void* A, const void* B,
@@ -910,7 +1061,10 @@ size_t qnf4_workspace_size(int32_t op, int64_t N, int64_t K, int64_t M, int32_t 
     case QNF4_OP_LAYER_STATS: return 2 * kQuantMaxGrid * sizeof(double);
     case QNF4_OP_QUANTIZE_WEIGHT: return 2 * kQuantMaxGrid * sizeof(double);
     case QNF4_OP_DOUBLE_QUANT: return kDqPartials * sizeof(double);
-    case QNF4_OP_FWD: return plan_linear(A_NF4_K, N, K, M, r, false, num_sms()).total;
+    case QNF4_OP_FWD: {
+      const size_t t = plan_linear(A_NF4_K, N, K, M, r, false, num_sms()).total;
+      return M <= kDecodeMaxTokens ? std::max(t, plan_decode(N, K, M, r, num_sms()).total) : t;
+    }
     case QNF4_OP_BWD: return plan_linear(A_NF4_MN, N, K, M, r, true, num_sms()).total;
     case QNF4_OP_CHANQ_FWD: return plan_linear(A_CHANQ_K, N, K, M, r, false, num_sms()).total;
     case QNF4_OP_LOFTQ: return loftq_layout(N, K, r).total;
@@ -1164,6 +1318,8 @@ qnf4_status qnf4_qlora_linear_fwd(const qnf4_weight* w, const void* x, int64_t M
   st = check_linear_args(w->N, w->K, M, r, false, {x, A, B, h});
   if (st != QNF4_OK) return st;
   if (M == 0) return QNF4_OK;
+  if (M <= kDecodeMaxTokens)
+    return decode_fwd(w, x, M, A, B, r, scale, h, ws, ws_bytes, static_cast<cudaStream_t>(stream));
   BaseSrc src;
   src.kind = A_NF4_K;
   src.w = w;

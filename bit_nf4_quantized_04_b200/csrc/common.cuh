@@ -122,6 +122,25 @@ QNF4_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned long long wait_
   }
 }
 
+// Spin on a phase with a bound, in every lane of a warp, then agree: the result is
+// the same in all lanes (all observed the phase, or the warp gives up together).
+QNF4_DEV bool warp_wait(uint64_t* bar, uint32_t parity, unsigned long long wait_ns,
+                        volatile int* abort_flag, unsigned int site) {
+  bool ok = mbar_try_wait(bar, parity);
+  if (!ok) {
+    const long long t0 = wait_clock();
+    while (!(ok = mbar_try_wait(bar, parity))) {
+      if (*abort_flag) break;
+      if (wait_clock() - t0 > ns_cycles(wait_ns)) {
+        set_err(site);
+        *abort_flag = 1;
+        break;
+      }
+    }
+  }
+  return __all_sync(0xffffffffu, ok);
+}
+
 // ----------------------------------------------------------------------------
 // TMA (bulk tensor copies global -> shared, completion on an mbarrier)
 // ----------------------------------------------------------------------------
@@ -131,6 +150,14 @@ QNF4_DEV void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int3
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+QNF4_DEV void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int32_t x,
+                          int32_t y, int32_t z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
       : "memory");
 }
 // Tile shared -> global (bulk async group of the issuing thread; out-of-range

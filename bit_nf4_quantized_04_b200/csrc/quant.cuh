@@ -36,25 +36,6 @@ constexpr int kQMaxH = 16;          // largest bin count H the kernels' table ho
 constexpr int kQTabCopies = 16;     // table copies, one per lane of a half warp
 constexpr size_t kQSmem = static_cast<size_t>(kQWorkers) * kQStages * kQChunkBytes + 1024;
 
-// Spin on a phase with a bound, in every lane of a warp, then agree: the result is
-// the same in all lanes (all observed the phase, or the warp gives up together).
-QNF4_DEV bool warp_wait(uint64_t* bar, uint32_t parity, unsigned long long wait_ns,
-                        volatile int* abort_flag, unsigned int site) {
-  bool ok = mbar_try_wait(bar, parity);
-  if (!ok) {
-    const long long t0 = wait_clock();
-    while (!(ok = mbar_try_wait(bar, parity))) {
-      if (*abort_flag) break;
-      if (wait_clock() - t0 > ns_cycles(wait_ns)) {
-        set_err(site);
-        *abort_flag = 1;
-        break;
-      }
-    }
-  }
-  return __all_sync(0xffffffffu, ok);
-}
-
 // Shared loads of read-only tables (filled before a CTA barrier), by 32-bit shared address;
 // not volatile, so the compiler may schedule them freely.
 QNF4_DEV float lds_f32q(uint32_t addr) {
@@ -103,7 +84,7 @@ QNF4_DEV void nf4_block_codes(const uint4 (&v)[8], float c, float f, float hf, f
 #pragma unroll
   for (int u = 0; u < 8; ++u) {
     const uint32_t wd[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-    uint32_t by[4];
+    uint32_t ue[4], uo[4];  // codes (bits 0-3) of elements 8u + 2i and 8u + 2i + 1
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       float2 wp = make_float2(bf16lo(wd[i]), bf16hi(wd[i]));
@@ -113,17 +94,19 @@ QNF4_DEV void nf4_block_codes(const uint4 (&v)[8], float c, float f, float hf, f
       const float2 tb = lds_f32x2q(__float_as_uint(kb.y) * (8u * kQTabCopies) + toff);
       const float sx = fmaf(cd, ta.y, fmaf(-cd, ta.x, wp.x));
       const float sy = fmaf(cd, tb.y, fmaf(-cd, tb.x, wp.y));
-      const uint32_t ux = sign_sub(__float_as_uint(sx), __float_as_uint(ta.y));  // code in bits 0-3
-      const uint32_t uy = sign_sub(__float_as_uint(sy), __float_as_uint(tb.y));
-      by[i] = ((ux << 4) & 0xF0u) | (uy & 0x0Fu);  // element 2i in the high nibble
+      ue[i] = sign_sub(__float_as_uint(sx), __float_as_uint(ta.y));
+      uo[i] = sign_sub(__float_as_uint(sy), __float_as_uint(tb.y));
       if (SSE) {
-        const float2 r2 = __ffma2_rn(make_float2(lds_f32q(lvb + 4u * (ux & 15u)),
-                                                 lds_f32q(lvb + 4u * (uy & 15u))),
+        const float2 r2 = __ffma2_rn(make_float2(lds_f32q(lvb + 4u * (ue[i] & 15u)),
+                                                 lds_f32q(lvb + 4u * (uo[i] & 15u))),
                                      nc2, wp);
         acc = __ffma2_rn(r2, r2, acc);
       }
     }
-    pw[u] = __byte_perm(__byte_perm(by[0], by[1], 0x0040), __byte_perm(by[2], by[3], 0x0040), 0x5410);
+    // byte i of each word from the i-th code; even elements into the high nibbles
+    const uint32_t ev = __byte_perm(__byte_perm(ue[0], ue[1], 0x0040), __byte_perm(ue[2], ue[3], 0x0040), 0x5410);
+    const uint32_t od = __byte_perm(__byte_perm(uo[0], uo[1], 0x0040), __byte_perm(uo[2], uo[3], 0x0040), 0x5410);
+    pw[u] = ((ev << 4) & 0xF0F0F0F0u) | (od & 0x0F0F0F0Fu);
   }
 }
 
