@@ -197,6 +197,30 @@ def qlora_linear_fwd(w: Nf4Weight, x: torch.Tensor, A: torch.Tensor, B: torch.Te
     return h
 
 
+def qlora_linear_fwd_group(ws_: list, xs: list, As: list, Bs: list, scale: float, hs=None,
+                           ws=None) -> list:
+    """The decode-size forward (1..16 tokens) of up to 8 independent layers in one launch:
+    h[l] = x[l] dequant(W_l)^T + scale (x[l] A[l]^T) B[l]^T; every layer has the same
+    token count and rank."""
+    n = len(ws_)
+    if not (len(xs) == len(As) == len(Bs) == n):
+        raise ValueError("one x, A and B per layer")
+    for i in range(n):
+        for t, nm in ((xs[i], "x"), (As[i], "A"), (Bs[i], "B")):
+            _req(t, torch.bfloat16, nm)
+    M = xs[0].shape[0]
+    r = As[0].shape[0]
+    dev = xs[0].device
+    hs = hs if hs is not None else [torch.empty(M, w.N, dtype=torch.bfloat16, device=dev) for w in ws_]
+    need = sum(workspace_size(_lib.OP_FWD, w.N, w.K, M, r) for w in ws_)
+    wsb = _ws(need, xs[0], ws)
+    arr = (_lib.Qnf4Weight * n)(*[w.c() for w in ws_])
+    ptrs = lambda ts: (C.c_void_p * n)(*[t.data_ptr() for t in ts])  # noqa: E731
+    _lib.call("qnf4_qlora_linear_fwd_group", n, arr, ptrs(xs), M, ptrs(As), ptrs(Bs), r, float(scale),
+              ptrs(hs), wsb.data_ptr(), wsb.numel(), _stream(xs[0]))
+    return hs
+
+
 def qlora_linear_bwd(w: Nf4Weight, x: torch.Tensor, dY: torch.Tensor, A: torch.Tensor,
                      B: torch.Tensor, scale: float, dX=None, dA=None, dB=None, ws=None):
     """(dX bf16 [M, K], dA fp32 [r, K], dB fp32 [N, r]) through the frozen NF4 base."""

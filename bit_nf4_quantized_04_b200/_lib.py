@@ -48,6 +48,8 @@ SIGNATURES = {
     "qnf4_dequant": (ST, [C.POINTER(Qnf4Weight), P, I32, P]),
     "qnf4_qlora_linear_fwd": (ST, [C.POINTER(Qnf4Weight), P, I64, P, P, I32, F32, P, P, SZ, P]),
     "qnf4_qlora_linear_fwd_noalloc": (ST, [C.POINTER(Qnf4Weight), P, I64, P, P, I32, F32, P, P]),
+    "qnf4_qlora_linear_fwd_group": (ST, [I32, C.POINTER(Qnf4Weight), C.POINTER(P), I64, C.POINTER(P),
+                                         C.POINTER(P), I32, F32, C.POINTER(P), P, SZ, P]),
     "qnf4_qlora_linear_bwd": (ST, [C.POINTER(Qnf4Weight), P, P, I64, P, P, I32, F32, P, P, P, P,
                                    SZ, P]),
     "qnf4_nf4_recon_error": (ST, [P, I64, I64, I32, P, P, SZ, P]),

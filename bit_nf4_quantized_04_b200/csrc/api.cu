@@ -50,11 +50,38 @@ std::atomic<unsigned long long> g_launches{0};
 thread_local cudaEvent_t g_ev_start = nullptr, g_ev_stop = nullptr;
 
 // Check the last launch(es) and count `n` kernels of this library as launched.
+// first failure of a cudaLaunchKernelEx launch since the last launched() check
+thread_local cudaError_t g_launch_err = cudaSuccess;
+
 qnf4_status launched(const char* what, int n = 1) {
   g_launches.fetch_add(static_cast<unsigned long long>(n), std::memory_order_relaxed);
-  const cudaError_t e = cudaGetLastError();
+  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) e = g_launch_err;
+  g_launch_err = cudaSuccess;
   if (e != cudaSuccess) return fail(QNF4_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
   return QNF4_OK;
+}
+
+// Launch as a programmatic dependent of the previous kernel in the stream: the kernel
+// may start (and run its prologue) while that kernel finishes; every kernel launched
+// this way calls griddepcontrol.wait before it touches global memory.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       Args... args) {
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+  if (e != cudaSuccess && g_launch_err == cudaSuccess) g_launch_err = e;
+  return e;
 }
 
 int num_sms() {
@@ -541,33 +568,16 @@ qnf4_status run_u(const LinPlan& L, const void* x, const void* A, int64_t M, int
 // ---------------------------------------------------------------------------
 constexpr int64_t kDecodeMaxTokens = 16;
 
-struct DecodePlan {
-  int Q = 1, P = 1, ks = 1;
-  int64_t rbs = 0;
-  size_t off_up = 0, total = 0;
-};
-
-// One CTA per SM, each holding at most kDecMaxRb row blocks (more CTAs than SMs only
-// when N > 16 kDecMaxRb SMs rows).
-DecodePlan plan_decode(int64_t N, int64_t K, int64_t M, int r, int sms) {
-  DecodePlan d;
-  d.Q = M <= 8 ? 1 : 2;
-  d.rbs = (N + 15) / 16;
-  const int64_t need = (d.rbs + kDecMaxRb - 1) / kDecMaxRb;
-  d.P = static_cast<int>(std::max<int64_t>(need, std::min<int64_t>(sms, d.rbs)));
-  d.ks = static_cast<int>((K + kDecUChunk - 1) / kDecUChunk);
-  size_t o = 0;
-  d.off_up = o;
-  o = align256(o + static_cast<size_t>(d.ks) * r * M * sizeof(float));
-  d.total = o;
-  return d;
+// Workspace of one decode-size layer: its adapter projection partials, 256-aligned.
+size_t decode_ws_bytes(int64_t K, int64_t M, int r) {
+  const int64_t ks = (K + kDecUChunk - 1) / kDecUChunk;
+  return align256(static_cast<size_t>(ks) * r * M * sizeof(float));
 }
 
 bool g_dec_smem_set[2][64] = {};
 
 template <int Q>
-cudaError_t launch_decode(const CUtensorMap& mw0, const CUtensorMap& mw1, const CUtensorMap& mx,
-                          const DecodeArgs& a, int rlo, int w3d, int P, cudaStream_t s) {
+cudaError_t launch_decode(const DecodeArgs& a, int P, cudaStream_t s) {
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !g_dec_smem_set[Q - 1][dev]) {
@@ -576,82 +586,87 @@ cudaError_t launch_decode(const CUtensorMap& mw0, const CUtensorMap& mw1, const 
     if (e != cudaSuccess) return e;
     g_dec_smem_set[Q - 1][dev] = true;
   }
-  cudaLaunchConfig_t cfg;
-  std::memset(&cfg, 0, sizeof(cfg));
-  cfg.gridDim = dim3(P);
-  cfg.blockDim = dim3(kDecBlockThreads);
-  cfg.dynamicSmemBytes = kDecSmem;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, k_nf4_decode<Q>, mw0, mw1, mx, a, rlo, w3d, g_wait_ns);
+  return launch_pdl(k_nf4_decode<Q>, dim3(P), dim3(kDecBlockThreads), kDecSmem, s, a, g_wait_ns);
+}
+
+// Decode-size forward of n independent layers in one launch pair (k_lora_u, then
+// k_nf4_decode); the layers share M, r and scale. Arguments are checked by the caller.
+qnf4_status decode_group(int n, const qnf4_weight* w, const void* const* xs, int64_t M,
+                         const void* const* As, const void* const* Bs, int r, float scale,
+                         void* const* hs, void* ws, size_t ws_bytes, cudaStream_t s) {
+  static thread_local DecodeArgs a;  // about 10 KB: kept off the stack
+  std::memset(&a, 0, sizeof(a));
+  a.n = n;
+  a.M = static_cast<int>(M);
+  a.r = r;
+  a.scale = scale;
+  std::memcpy(a.levels, nf4_tables().levels, sizeof(a.levels));
+  size_t need = 0;
+  int64_t units = 0, kmax = 0;
+  double total = 0.0;  // work = units x K (bytes per unit are 8 K)
+  for (int l = 0; l < n; ++l) {
+    const int64_t N = w[l].N, K = w[l].K;
+    DecLayer& L = a.L[l];
+    L.N = N;
+    L.K = K;
+    L.nkb = static_cast<int>(K / 64);
+    L.ks = static_cast<int>((K + kDecUChunk - 1) / kDecUChunk);
+    L.w3d = K % 256 == 0 ? 1 : 0;
+    L.unit0 = units;
+    L.nb2 = (N * (K / 64) + 255) / 256;
+    L.code2 = w[l].code2;
+    L.scale2 = w[l].scale2;
+    L.mean = w[l].mean;
+    L.x = static_cast<const uint16_t*>(xs[l]);
+    L.A = static_cast<const uint16_t*>(As[l]);
+    L.Bm = static_cast<const uint16_t*>(Bs[l]);
+    L.h = static_cast<uint16_t*>(hs[l]);
+    L.upart = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + need);
+    need += decode_ws_bytes(K, M, r);
+    for (int i = 0; i < kDecMaxRb; ++i) {
+      const uint32_t rows = 16u * (i + 1);
+      const bool ok = L.w3d ? make_map_wcols(&a.wmap[l][i], w[l].packed, K, N, rows)
+                            : make_map(&a.wmap[l][i], w[l].packed, true, K / 2, N, K / 2, 128, rows, true);
+      if (!ok) return map_fail();
+    }
+    if (!make_map_xblocks(&a.xmap[l], xs[l], K, M, static_cast<uint32_t>(M))) return map_fail();
+    const int64_t rbs = (N + 15) / 16;
+    units += rbs;
+    total += static_cast<double>(rbs) * static_cast<double>(K);
+    kmax = std::max(kmax, K);
+  }
+  if (!ws || ws_bytes < need) return fail(QNF4_ERR_WORKSPACE, "workspace too small (%zu < %zu)", ws_bytes, need);
+  a.units = units;
+  // CTA p takes the units from the first one whose start lies at or past p / P of the
+  // total work (units x K), so every CTA streams about the same number of bytes
+  const int P = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>({num_sms(), units, kDecMaxCta})));
+  {
+    int p = 0;
+    double cum = 0.0;
+    int64_t u = 0;
+    a.cta_unit[0] = 0;
+    for (int l = 0; l < n; ++l) {
+      const int64_t rbs = (w[l].N + 15) / 16;
+      for (int64_t b = 0; b < rbs; ++b, ++u) {
+        while (p + 1 < P && cum >= total * (p + 1) / P) a.cta_unit[++p] = u;
+        cum += static_cast<double>(w[l].K);
+      }
+    }
+    while (p < P) a.cta_unit[++p] = units;
+  }
+  if (g_ev_start) cudaEventRecord(g_ev_start, s);
+  const int ksmax = static_cast<int>((kmax + kDecUChunk - 1) / kDecUChunk);
+  cudaError_t e = launch_pdl(k_lora_u, dim3(r, ksmax, n), dim3(128), 0, s, a);
+  if (e != cudaSuccess) return fail(QNF4_ERR_CUDA, "k_lora_u launch: %s", cudaGetErrorString(e));
+  e = M <= 8 ? launch_decode<1>(a, P, s) : launch_decode<2>(a, P, s);
+  if (e != cudaSuccess) return fail(QNF4_ERR_CUDA, "k_nf4_decode launch: %s", cudaGetErrorString(e));
+  if (g_ev_stop) cudaEventRecord(g_ev_stop, s);
+  return launched("decode_fwd", 2);
 }
 
 qnf4_status decode_fwd(const qnf4_weight* w, const void* x, int64_t M, const void* A, const void* B,
                        int r, float scale, void* h, void* ws, size_t ws_bytes, cudaStream_t s) {
-  const int64_t N = w->N, K = w->K;
-  const DecodePlan d = plan_decode(N, K, M, r, num_sms());
-  if (!ws || ws_bytes < d.total) return fail(QNF4_ERR_WORKSPACE, "workspace too small (%zu < %zu)", ws_bytes, d.total);
-  uint8_t* w8 = static_cast<uint8_t*>(ws);
-  float* upart = reinterpret_cast<float*>(w8 + d.off_up);
-  DecodeArgs a;
-  std::memset(&a, 0, sizeof(a));
-  a.N = N;
-  a.K = K;
-  a.M = static_cast<int>(M);
-  a.r = r;
-  a.nkb = static_cast<int>(K / 64);
-  a.ks = d.ks;
-  a.rbs = d.rbs;
-  a.scale = scale;
-  std::memcpy(a.levels, nf4_tables().levels, sizeof(a.levels));
-  a.code2 = w->code2;
-  a.scale2 = w->scale2;
-  a.mean = w->mean;
-  a.Bm = static_cast<const uint16_t*>(B);
-  a.upart = upart;
-  a.h = static_cast<uint16_t*>(h);
-  a.nb2 = (N * (K / 64) + 255) / 256;
-  if (g_ev_start) cudaEventRecord(g_ev_start, s);
-  {
-    cudaLaunchConfig_t cfg;
-    std::memset(&cfg, 0, sizeof(cfg));
-    cfg.gridDim = dim3(r, d.ks);
-    cfg.blockDim = dim3(128);
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, k_lora_u, static_cast<const uint16_t*>(x),
-                                             static_cast<const uint16_t*>(A), K, static_cast<int>(M), r,
-                                             upart);
-    if (e != cudaSuccess) return fail(QNF4_ERR_CUDA, "k_lora_u launch: %s", cudaGetErrorString(e));
-  }
-  // CTAs hold rlo or rlo + 1 row blocks; one packed-weight map per box height, as
-  // [K/256][N][128] (one box of four 128-byte columns) when K is a multiple of 256
-  const int rlo = static_cast<int>(d.rbs / d.P);
-  const int rhi = std::min(rlo + 1, kDecMaxRb);
-  const int w3d = K % 256 == 0 ? 1 : 0;
-  CUtensorMap mw0, mw1, mx;
-  if (w3d) {
-    if (!make_map_wcols(&mw0, w->packed, K, N, 16 * rlo) || !make_map_wcols(&mw1, w->packed, K, N, 16 * rhi))
-      return map_fail();
-  } else {
-    if (!make_map(&mw0, w->packed, true, K / 2, N, K / 2, 128, 16 * rlo, true) ||
-        !make_map(&mw1, w->packed, true, K / 2, N, K / 2, 128, 16 * rhi, true))
-      return map_fail();
-  }
-  if (!make_map_xblocks(&mx, x, K, M, static_cast<uint32_t>(M))) return map_fail();
-  const cudaError_t e = d.Q == 1 ? launch_decode<1>(mw0, mw1, mx, a, rlo, w3d, d.P, s)
-                                 : launch_decode<2>(mw0, mw1, mx, a, rlo, w3d, d.P, s);
-  if (e != cudaSuccess) return fail(QNF4_ERR_CUDA, "k_nf4_decode launch: %s", cudaGetErrorString(e));
-  if (g_ev_stop) cudaEventRecord(g_ev_stop, s);
-  return launched("decode_fwd", 2);
+  return decode_group(1, w, &x, M, &A, &B, r, scale, &h, ws, ws_bytes, s);
 }
 
 qnf4_status linear_fwd(const BaseSrc& src, const void* x, int64_t M, const void* A, const void* B,
@@ -1063,7 +1078,7 @@ size_t qnf4_workspace_size(int32_t op, int64_t N, int64_t K, int64_t M, int32_t 
     case QNF4_OP_DOUBLE_QUANT: return kDqPartials * sizeof(double);
     case QNF4_OP_FWD: {
       const size_t t = plan_linear(A_NF4_K, N, K, M, r, false, num_sms()).total;
-      return M <= kDecodeMaxTokens ? std::max(t, plan_decode(N, K, M, r, num_sms()).total) : t;
+      return M <= kDecodeMaxTokens ? std::max(t, decode_ws_bytes(K, M, r)) : t;
     }
     case QNF4_OP_BWD: return plan_linear(A_NF4_MN, N, K, M, r, true, num_sms()).total;
     case QNF4_OP_CHANQ_FWD: return plan_linear(A_CHANQ_K, N, K, M, r, false, num_sms()).total;
@@ -1099,15 +1114,15 @@ qnf4_status qnf4_nf4_quantize(const void* W, int64_t N, int64_t K, int32_t block
   if (!quant_map(&wmap, W, nblocks)) return map_fail();
   const QuantTab tab = make_tab();
   if (sse) {
-    k_nf4_quant<true, true><<<grid, kQThreads, kQSmem, s>>>(
+    launch_pdl(k_nf4_quant<true, true>, dim3(grid), dim3(kQThreads), kQSmem, s, 
         wmap, nblocks, reinterpret_cast<uint32_t*>(packed), absmax,
-        static_cast<double*>(ws), tab, g_wait_ns);
-    k_sum_partials<<<1, 256, 0, s>>>(static_cast<const double*>(ws), grid, sse);
+        static_cast<double*>(ws), tab, g_wait_ns, 0.f, nullptr, nullptr);
+    launch_pdl(k_sum_partials, dim3(1), dim3(256), 0, s, static_cast<const double*>(ws), grid, sse);
     return launched("nf4_quantize", 2);
   }
-  k_nf4_quant<true, false><<<grid, kQThreads, kQSmem, s>>>(
+  launch_pdl(k_nf4_quant<true, false>, dim3(grid), dim3(kQThreads), kQSmem, s, 
       wmap, nblocks, reinterpret_cast<uint32_t*>(packed), absmax,
-      nullptr, tab, g_wait_ns);
+      nullptr, tab, g_wait_ns, 0.f, nullptr, nullptr);
   return launched("nf4_quantize");
 }
 
@@ -1135,17 +1150,17 @@ qnf4_status qnf4_quantize_weight(const void* W, int64_t N, int64_t K, uint8_t* p
   double* ssep = asum + kQuantMaxGrid;
   const QuantTab tab = make_tab();
   if (sse) {
-    k_nf4_quant<true, true><<<grid, kQThreads, kQSmem, s>>>(
+    launch_pdl(k_nf4_quant<true, true>, dim3(grid), dim3(kQThreads), kQSmem, s, 
         wmap, nblocks, reinterpret_cast<uint32_t*>(packed), absmax, ssep,
         tab, g_wait_ns, 0.f, nullptr, asum);
   } else {
-    k_nf4_quant<true, false><<<grid, kQThreads, kQSmem, s>>>(
+    launch_pdl(k_nf4_quant<true, false>, dim3(grid), dim3(kQThreads), kQSmem, s, 
         wmap, nblocks, reinterpret_cast<uint32_t*>(packed), absmax,
         nullptr, tab, g_wait_ns, 0.f, nullptr, asum);
   }
   const int64_t nb2 = (nblocks + 255) / 256;
   const int egrid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((nb2 + 7) / 8, num_sms() * 4)));
-  k_dq_encode<<<egrid, 256, 0, s>>>(absmax, nblocks, asum, grid, nblocks, code2, scale2, mean,
+  launch_pdl(k_dq_encode, dim3(egrid), dim3(256), 0, s, absmax, nblocks, asum, grid, nblocks, code2, scale2, mean,
                                     sse ? ssep : nullptr, grid, sse);
   return launched("quantize_weight", 2);
 }
@@ -1170,10 +1185,10 @@ qnf4_status qnf4_nf4_recon_error(const void* W, int64_t N, int64_t K, int32_t bl
   const int grid = quant_grid(nblocks);
   CUtensorMap wmap;
   if (!quant_map(&wmap, W, nblocks)) return map_fail();
-  k_nf4_quant<false, true><<<grid, kQThreads, kQSmem, s>>>(wmap, nblocks,
+  launch_pdl(k_nf4_quant<false, true>, dim3(grid), dim3(kQThreads), kQSmem, s, wmap, nblocks,
                                                           nullptr, nullptr, static_cast<double*>(ws),
-                                                          make_tab(), g_wait_ns);
-  k_sum_partials<<<1, 256, 0, s>>>(static_cast<const double*>(ws), grid, sse);
+                                                          make_tab(), g_wait_ns, 0.f, nullptr, nullptr);
+  launch_pdl(k_sum_partials, dim3(1), dim3(256), 0, s, static_cast<const double*>(ws), grid, sse);
   return launched("nf4_recon_error", 2);
 }
 
@@ -1199,11 +1214,11 @@ qnf4_status qnf4_nf4_layer_stats(const void* W, int64_t N, int64_t K, float tau,
   CUtensorMap wmap;
   if (!quant_map(&wmap, W, nblocks)) return map_fail();
   double* part = static_cast<double*>(ws);
-  k_nf4_quant<false, true, true><<<grid, kQThreads, kQSmem, s>>>(
+  launch_pdl(k_nf4_quant<false, true, true>, dim3(grid), dim3(kQThreads), kQSmem, s, 
       wmap, nblocks, nullptr, nullptr, part, make_tab(), g_wait_ns, tau,
-      part + kQuantMaxGrid);
-  k_sum_partials<<<1, 256, 0, s>>>(part, grid, sse);
-  k_sum_partials<<<1, 256, 0, s>>>(part + kQuantMaxGrid, grid, below);
+      part + kQuantMaxGrid, nullptr);
+  launch_pdl(k_sum_partials, dim3(1), dim3(256), 0, s, part, grid, sse);
+  launch_pdl(k_sum_partials, dim3(1), dim3(256), 0, s, part + kQuantMaxGrid, grid, below);
   return launched("nf4_layer_stats", 3);
 }
 
@@ -1222,7 +1237,7 @@ qnf4_status qnf4_double_quant(const float* absmax, int64_t nb1, int32_t block2, 
   const int64_t nb2 = (nb1 + 255) / 256;
   int grid = static_cast<int>(std::min<int64_t>((nb2 + 7) / 8, num_sms() * 4));
   grid = std::max(grid, 1);
-  k_dq_encode<<<grid, 256, 0, s>>>(absmax, nb1, part, kDqPartials, nb1, code2, scale2, mean);
+  launch_pdl(k_dq_encode, dim3(grid), dim3(256), 0, s, absmax, nb1, part, kDqPartials, nb1, code2, scale2, mean, nullptr, 0, nullptr);
   return launched("double_quant", 2);
 }
 
@@ -1236,7 +1251,7 @@ qnf4_status qnf4_dq_sum(const float* absmax, int64_t nb1, double* sum, void* ws,
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   double* part = static_cast<double*>(ws);
   k_dq_partial<<<kDqPartials, 256, 0, s>>>(absmax, nb1, part);
-  k_sum_partials<<<1, 256, 0, s>>>(part, kDqPartials, sum);
+  launch_pdl(k_sum_partials, dim3(1), dim3(256), 0, s, part, kDqPartials, sum);
   return launched("dq_sum", 2);
 }
 
@@ -1252,7 +1267,7 @@ qnf4_status qnf4_double_quant_shard(const float* absmax, int64_t nb1, int32_t bl
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int64_t nb2 = (nb1 + 255) / 256;
   const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((nb2 + 7) / 8, num_sms() * 4)));
-  k_dq_encode<<<grid, 256, 0, s>>>(absmax, nb1, total_sum, 1, total_count, code2, scale2, mean);
+  launch_pdl(k_dq_encode, dim3(grid), dim3(256), 0, s, absmax, nb1, total_sum, 1, total_count, code2, scale2, mean, nullptr, 0, nullptr);
   return launched("dq_encode_shard");
 }
 
@@ -1326,6 +1341,27 @@ qnf4_status qnf4_qlora_linear_fwd(const qnf4_weight* w, const void* x, int64_t M
   src.N = w->N;
   src.K = w->K;
   return linear_fwd(src, x, M, A, B, r, scale, h, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+qnf4_status qnf4_qlora_linear_fwd_group(int32_t n, const qnf4_weight* w, const void* const* x,
+                                        int64_t M, const void* const* A, const void* const* B,
+                                        int32_t r, float scale, void* const* h, void* ws,
+                                        size_t ws_bytes, void* stream) {
+  if (n < 1 || n > kDecMaxGroup) return fail(QNF4_ERR_ARG, "n must be in [1, %d] (got %d)", kDecMaxGroup, n);
+  if (!w || !x || !A || !B || !h) return fail(QNF4_ERR_ARG, "NULL array");
+  if (M < 1 || M > kDecodeMaxTokens)
+    return fail(QNF4_ERR_SHAPE, "the grouped forward takes 1 to %lld tokens (got %lld)",
+                static_cast<long long>(kDecodeMaxTokens), static_cast<long long>(M));
+  size_t need = 0;
+  for (int l = 0; l < n; ++l) {
+    qnf4_status st = check_weight(&w[l]);
+    if (st != QNF4_OK) return st;
+    st = check_linear_args(w[l].N, w[l].K, M, r, false, {x[l], A[l], B[l], h[l]});
+    if (st != QNF4_OK) return st;
+    need += decode_ws_bytes(w[l].K, M, r);
+  }
+  if (!ws || ws_bytes < need) return fail(QNF4_ERR_WORKSPACE, "workspace too small (%zu < %zu)", ws_bytes, need);
+  return decode_group(n, w, x, M, A, B, r, scale, h, ws, ws_bytes, static_cast<cudaStream_t>(stream));
 }
 
 qnf4_status qnf4_qlora_linear_fwd_noalloc(const qnf4_weight* w, const void* x, int64_t M,

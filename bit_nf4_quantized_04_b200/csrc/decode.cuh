@@ -53,15 +53,17 @@ constexpr int kDecMaxRb = 5;      // 16-row blocks a CTA holds at most
 constexpr int kDecMaxRows = 16 * kDecMaxRb;
 constexpr int kDecMaxStages = 4;
 constexpr int kDecSbBlocks = 16;            // column blocks per stage (one per warp)
-constexpr uint32_t kDecRingBytes = 168u * 1024u;
+constexpr uint32_t kDecRingBytes = 152u * 1024u;
 constexpr int kDecLutCopies = 32;
 constexpr int kDecRedSlots = 4;
 constexpr int kDecRedRow = 84;   // floats per token row of a reduction slot (padded)
 constexpr uint32_t kDecLutBytes = 256u * kDecLutCopies * 4u;                 // 32 KB
-constexpr uint32_t kDecRedBytes = kDecRedSlots * 16u * kDecRedRow * 4u;      // 21 KB (in the ring)
+constexpr uint32_t kDecRedBytes = kDecRedSlots * 16u * kDecRedRow * 4u;      // 21 KB
 constexpr uint32_t kDecCsBytes = kDecWarps * kDecMaxRows * 4u;               // 5 KB
 constexpr uint32_t kDecBsBytes = kDecMaxRows * 64u * 2u;                     // 10 KB: B rows, r <= 64
-constexpr size_t kDecSmem = 1024 + kDecRingBytes + kDecLutBytes + kDecCsBytes + kDecBsBytes;
+constexpr uint32_t kDecUsBytes = 64u * 16u * 4u;                             // 4 KB: u [r][M]
+constexpr size_t kDecSmem =
+    1024 + kDecRingBytes + kDecLutBytes + kDecCsBytes + kDecBsBytes + kDecRedBytes + kDecUsBytes;
 // stage = the token box (16 blocks x M rows x 128 B), then 4 packed boxes (16R rows x
 // 128 B); every box starts on a 1024-byte boundary
 __host__ __device__ constexpr uint32_t dec_stage_bytes(int R, int M) {
@@ -73,23 +75,40 @@ __host__ __device__ constexpr int dec_stages(int R, int M) {
              : kDecMaxStages;
 }
 static_assert(dec_stages(kDecMaxRb, 16) >= 2, "the ring must hold two stages of the largest tile");
-static_assert(kDecRedBytes + 64u * 16u * 4u <= kDecRingBytes, "reduction buffers and u live in the ring");
 constexpr int kDecUChunk = 1024;  // contraction columns per k_lora_u partial (128 threads x 8)
 constexpr int kDecMaxUParts = 64;  // partials (K <= 65536)
 
-struct DecodeArgs {
+constexpr int kDecMaxGroup = 8;    // layers per launch
+constexpr int kDecMaxCta = 256;    // CTAs per launch (one per SM)
+
+// One layer of a launch.
+struct DecLayer {
   int64_t N, K;
-  int M, r, nkb, ks;       // tokens, rank, 64-blocks per row, adapter partials
-  int64_t rbs;             // 16-row blocks
-  float scale;
-  float levels[16];
+  int nkb, ks, w3d;          // 64-blocks per row, adapter partials, packed boxes are 3-D
+  int64_t unit0;             // first unit (16-row block) of this layer in the launch
+  int64_t nb2;               // scale2 entries
   const uint8_t* code2;
   const float* scale2;
   const float* mean;
-  const uint16_t* Bm;      // [N, r] bf16
-  const float* upart;      // [ks][r][M] fp32
-  uint16_t* h;             // [M, N] bf16
-  int64_t nb2;             // scale2 entries
+  const uint16_t* x;         // [M, K] bf16
+  const uint16_t* A;         // [r, K] bf16
+  const uint16_t* Bm;        // [N, r] bf16
+  float* upart;              // [ks][r][M] fp32
+  uint16_t* h;               // [M, N] bf16
+};
+
+struct DecodeArgs {
+  // wmap[l][i]: layer l's packed weight in boxes of 16 (i + 1) rows, as [N][K/256][128]
+  // bytes in boxes of rows x 4 x 128 (w3d) or as [N, K/2] bytes in boxes of 128 x rows;
+  // xmap[l]: x as [K/64][M][64] in boxes of 16 blocks x M rows x 64 columns
+  CUtensorMap wmap[kDecMaxGroup][kDecMaxRb];
+  CUtensorMap xmap[kDecMaxGroup];
+  DecLayer L[kDecMaxGroup];
+  int n, M, r;
+  float scale;
+  float levels[16];
+  int64_t units;                  // 16-row blocks of all layers
+  int64_t cta_unit[kDecMaxCta + 1];  // CTA p holds units [cta_unit[p], cta_unit[p + 1])
 };
 
 QNF4_DEV uint4 lds_u4d(uint32_t addr) {
@@ -123,26 +142,29 @@ QNF4_DEV void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a
         "f"(c[3]));
 }
 
-// The adapter projection u = A x^T in partial sums over contraction chunks of 1024:
-// CTA (j, c) writes upart[c][j][m] for every token m (fixed-order reduction over its
-// four warps). Launched as a programmatic dependent of whatever ran before: it first
-// waits for that grid, then lets its own dependent (the main kernel) start.
-__global__ void __launch_bounds__(128) k_lora_u(const uint16_t* __restrict__ x,
-                                                const uint16_t* __restrict__ A, int64_t K, int M,
-                                                int r, float* __restrict__ upart) {
+// The adapter projections u_l = A_l x_l^T in partial sums over contraction chunks of
+// 1024: CTA (j, c, l) writes layer l's upart[c][j][m] for every token m (fixed-order
+// reduction over its four warps). Launched as a programmatic dependent of whatever ran
+// before: it first waits for that grid, then lets its own dependent (the main kernel)
+// start.
+__global__ void __launch_bounds__(128) k_lora_u(const __grid_constant__ DecodeArgs g) {
   griddep_wait();
   griddep_launch_dependents();
   __shared__ float s_red[4][16];
-  const int j = blockIdx.x, c = blockIdx.y;
+  const int j = blockIdx.x, c = blockIdx.y, l = blockIdx.z;
+  const DecLayer& L = g.L[l];
+  const int M = g.M, r = g.r;
+  const int64_t K = L.K;
+  if (c >= L.ks) return;
   const int64_t k0 = static_cast<int64_t>(c) * kDecUChunk + threadIdx.x * 8;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const bool in = k0 < K;  // K is a multiple of 64, so k0 + 7 < K too
   uint4 av = make_uint4(0u, 0u, 0u, 0u);
   uint4 xv[16];
-  if (in) av = *reinterpret_cast<const uint4*>(A + j * K + k0);
+  if (in) av = *reinterpret_cast<const uint4*>(L.A + j * K + k0);
 #pragma unroll
   for (int m = 0; m < 16; ++m)
-    xv[m] = (in && m < M) ? *reinterpret_cast<const uint4*>(x + m * K + k0) : make_uint4(0u, 0u, 0u, 0u);
+    xv[m] = (in && m < M) ? *reinterpret_cast<const uint4*>(L.x + m * K + k0) : make_uint4(0u, 0u, 0u, 0u);
   const uint32_t aw[4] = {av.x, av.y, av.z, av.w};
   float vm[16];
 #pragma unroll
@@ -169,7 +191,7 @@ __global__ void __launch_bounds__(128) k_lora_u(const uint16_t* __restrict__ x,
   if (threadIdx.x < M) {
     const float v = ((s_red[0][threadIdx.x] + s_red[1][threadIdx.x]) + s_red[2][threadIdx.x]) + s_red[3][threadIdx.x];
     const int64_t o = (static_cast<int64_t>(c) * r + j) * M + threadIdx.x;
-    if (in_bounds(c < (K + kDecUChunk - 1) / kDecUChunk, 76)) upart[o] = v;
+    L.upart[o] = v;
   }
 }
 
@@ -184,15 +206,10 @@ QNF4_DEV void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
 QNF4_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 QNF4_DEV void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
-// Q token groups of 8 (Q = 1: M <= 8; Q = 2: M <= 16). wmap0 / wmap1: the packed
-// weight in boxes of 16 rlo / 16 (rlo + 1) rows, either as [N][K/256][128] bytes in
-// boxes of rows x 4 x 128 (w3d) or as [N, K/2] bytes in boxes of 128 x rows; xmap: x as
-// [K/64][M][64] in boxes of 16 blocks x M rows x 64 columns.
+// Q token groups of 8 (Q = 1: M <= 8; Q = 2: M <= 16).
 template <int Q>
 __global__ void __launch_bounds__(kDecBlockThreads, 1)
-    k_nf4_decode(const __grid_constant__ CUtensorMap wmap0, const __grid_constant__ CUtensorMap wmap1,
-                 const __grid_constant__ CUtensorMap xmap, DecodeArgs a, int rlo, int w3d,
-                 unsigned long long wait_ns) {
+    k_nf4_decode(const __grid_constant__ DecodeArgs g, unsigned long long wait_ns) {
   extern __shared__ uint8_t dsm_raw[];
   __shared__ __align__(8) uint64_t full[kDecMaxStages];
   __shared__ __align__(8) uint64_t empty[kDecMaxStages];
@@ -203,26 +220,26 @@ __global__ void __launch_bounds__(kDecBlockThreads, 1)
   uint32_t* lut = reinterpret_cast<uint32_t*>(base + kDecRingBytes);
   float* cs_all = reinterpret_cast<float*>(base + kDecRingBytes + kDecLutBytes);
   uint16_t* bs = reinterpret_cast<uint16_t*>(base + kDecRingBytes + kDecLutBytes + kDecCsBytes);
-  // after the main loop the ring holds the reduction slots and u [r][M]
-  float* red = reinterpret_cast<float*>(ring);
+  float* red = reinterpret_cast<float*>(base + kDecRingBytes + kDecLutBytes + kDecCsBytes + kDecBsBytes);
   float* us = red + kDecRedBytes / 4;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int g = lane >> 2, t = lane & 3;
-  const int pg = 2 * (g & 3) + (g >> 2);  // packed row of mma row g within 8
-
-  // this CTA's rows [row0, row0 + 16 R)
-  const int64_t P = gridDim.x;
-  const int64_t rb0 = static_cast<int64_t>(blockIdx.x) * a.rbs / P;
-  const int R = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * a.rbs / P - rb0);
-  const int64_t row0 = rb0 * 16;
-  const CUtensorMap* wm = R == rlo ? &wmap0 : &wmap1;
-  const int nkb = a.nkb;
-  const int nsb = (nkb + kDecSbBlocks - 1) / kDecSbBlocks;  // stages in all
-  const int M = a.M;
-  const uint32_t stb = dec_stage_bytes(R, M);
-  const int nst = dec_stages(R, M);
+  const int g8 = lane >> 2, t = lane & 3;
+  const int pg = 2 * (g8 & 3) + (g8 >> 2);  // packed row of mma row g8 within 8
+  const int M = g.M;
+  const uint32_t stb = dec_stage_bytes(kDecMaxRb, M);
+  const int nst = dec_stages(kDecMaxRb, M);
   const uint32_t woff = 2048u * M;
   const bool producer = warp == kDecWarps;
+  const int64_t u_begin = g.cta_unit[blockIdx.x], u_end = g.cta_unit[blockIdx.x + 1];
+  // the segment starting at unit u: layer l, its first row block rb, R <= kDecMaxRb blocks
+  auto seg_of = [&](int64_t u, int& l, int64_t& rb, int& R) {
+    l = 0;
+    while (l + 1 < g.n && g.L[l + 1].unit0 <= u) ++l;
+    rb = u - g.L[l].unit0;
+    const int64_t lend = l + 1 < g.n ? g.L[l + 1].unit0 : g.units;
+    const int64_t e = u_end < lend ? u_end : lend;
+    R = static_cast<int>(e - u < kDecMaxRb ? e - u : kDecMaxRb);
+  };
   if (tid == 0) {
     s_abort = 0;
     s_issued = -1;
@@ -233,205 +250,320 @@ __global__ void __launch_bounds__(kDecBlockThreads, 1)
     fence_mbar_init();
   }
   __syncthreads();
-  // the producer fills stage j: the token box and the packed boxes (blocks and columns
-  // past the end are zero-filled)
-  auto issue = [&](int j) {
-    uint8_t* st = ring + (j % nst) * stb;
-    uint64_t* bar = &full[j % nst];
-    const int kb0 = j * kDecSbBlocks;
-    mbar_expect_tx(bar, 16u * M * 128u + 4u * 16u * R * 128u);
-    tma_load_3d(st, &xmap, bar, 0, 0, kb0);
-    if (w3d) {
-      tma_load_3d(st + woff, wm, bar, 0, kb0 / 4, static_cast<int32_t>(row0));
-    } else {
-      for (int b = 0; b < 4; ++b)
-        tma_load_2d(st + woff + b * (16u * R * 128u), wm, bar, kb0 * 32 + b * 128,
-                    static_cast<int32_t>(row0));
-    }
-  };
+
   if (producer) {
-    // fill the ring, then refill each stage once the 16 compute warps have released its
-    // previous use; then leave (the compute warps synchronise among themselves)
+    // stream the CTA's segments: stage gs (a global count) goes into slot gs mod nst
+    // once the 16 compute warps have released that slot's previous use; then leave
     if (lane == 0) {
-      tma_prefetch_desc(wm);
-      tma_prefetch_desc(&xmap);
-      int j = 0;
-      for (; j < nsb; ++j) {
-        if (j >= nst) {
-          const long long t0 = wait_clock();
-          bool freed = true;
-          while (!mbar_try_wait(&empty[j % nst], static_cast<uint32_t>((j / nst - 1) & 1))) {
-            if (s_abort) {
-              freed = false;
-              break;
+      int64_t gs = 0;
+      bool stop = false;
+      for (int64_t u = u_begin; u < u_end && !stop;) {
+        int l, R;
+        int64_t rb;
+        seg_of(u, l, rb, R);
+        const DecLayer& L = g.L[l];
+        const CUtensorMap* wm = &g.wmap[l][R - 1];
+        const int nsb = (L.nkb + kDecSbBlocks - 1) / kDecSbBlocks;
+        const int32_t row0 = static_cast<int32_t>(rb * 16);
+        for (int j = 0; j < nsb; ++j) {
+          if (gs >= nst) {
+            const long long t0 = wait_clock();
+            while (!mbar_try_wait(&empty[gs % nst], static_cast<uint32_t>((gs / nst - 1) & 1))) {
+              if (s_abort) {
+                stop = true;
+                break;
+              }
+              if (wait_clock() - t0 > ns_cycles(wait_ns)) {
+                set_err(63);
+                s_abort = 1;
+                stop = true;
+                break;
+              }
             }
-            if (wait_clock() - t0 > ns_cycles(wait_ns)) {
-              set_err(63);
-              s_abort = 1;
-              freed = false;
-              break;
-            }
+            if (stop) break;
+            fence_proxy_async();
           }
-          if (!freed) break;
-          fence_proxy_async();
+          if (s_abort) {
+            stop = true;
+            break;
+          }
+          uint8_t* st = ring + (gs % nst) * stb;
+          uint64_t* bar = &full[gs % nst];
+          const int kb0 = j * kDecSbBlocks;
+          mbar_expect_tx(bar, 16u * M * 128u + 4u * 16u * R * 128u);
+          tma_load_3d(st, &g.xmap[l], bar, 0, 0, kb0);
+          if (L.w3d) {
+            tma_load_3d(st + woff, wm, bar, 0, kb0 / 4, row0);
+          } else {
+            for (int b = 0; b < 4; ++b)
+              tma_load_2d(st + woff + b * (16u * R * 128u), wm, bar, kb0 * 32 + b * 128, row0);
+          }
+          ++gs;
         }
-        if (s_abort) break;
-        issue(j);
+        u += R;
       }
-      s_issued = j;
+      s_issued = static_cast<int>(gs);
     }
     return;
   }
-  const float mu = __ldg(a.mean);
-  // this CTA's rows of B (bf16 [16R, r]) for the epilogue: asynchronous 16-byte copies
-  // when the rows are 16-byte aligned (r a multiple of 8), else plain loads
-  const bool bvec = (a.r & 7) == 0;
-  if (bvec) {
-    const int np = 16 * R * a.r / 8;
-    for (int i = tid; i < np; i += kDecThreads) {
-      const int64_t n = row0 + (i * 8) / a.r;
-      const bool in = n < a.N;
-      cp_async16(smem_u32(bs + i * 8), in ? a.Bm + row0 * a.r + i * 8 : a.Bm, in ? 16u : 0u);
-    }
-    cp_async_commit();
-  } else {
-    for (int i = tid; i < 16 * R * a.r; i += kDecThreads) {
-      const int64_t n = row0 + i / a.r;
-      bs[i] = n < a.N ? a.Bm[n * a.r + i % a.r] : static_cast<uint16_t>(0);
-    }
-  }
+
   // pair table: entry b, copy j at word b * 32 + j
   for (int i = tid; i < 256 * kDecLutCopies; i += kDecThreads) {
     const int b = i / kDecLutCopies;
-    lut[i] = pack_bf16x2(a.levels[b >> 4], a.levels[b & 15]);
+    lut[i] = pack_bf16x2(g.levels[b >> 4], g.levels[b & 15]);
   }
+  compute_sync();
 
   const uint32_t lutb = smem_u32(lut) + lane * 4u;
   float* cs = cs_all + warp * kDecMaxRows;
-  float acc[kDecMaxRb][Q][4];
-#pragma unroll
-  for (int rb = 0; rb < kDecMaxRb; ++rb)
-#pragma unroll
-    for (int q = 0; q < Q; ++q)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) acc[rb][q][e] = 0.f;
-  // block constants (code2 byte, scale2) of rows lane + 32 c for this warp's block of
-  // stage j, loaded one stage ahead of their use
-  constexpr int kCpl = (kDecMaxRows + 31) / 32;  // rows per lane
-  auto cload = [&](int j, uint32_t (&q)[kCpl], float (&sc)[kCpl]) {
-    const int kb = j * kDecSbBlocks + warp;
-#pragma unroll
-    for (int c = 0; c < kCpl; ++c) {
-      q[c] = 0u;
-      sc[c] = 0.f;
-      const int rr = lane + 32 * c;
-      const int64_t n = row0 + rr;
-      if (j < nsb && kb < nkb && rr < 16 * R && n < a.N) {
-        const int64_t blk = n * nkb + kb;
-        if (in_bounds((blk >> 8) < a.nb2, 71)) {
-          q[c] = a.code2[blk];
-          sc[c] = a.scale2[blk >> 8];
-        }
+  constexpr int kCpl = (kDecMaxRows + 31) / 32;  // rows per lane for the block constants
+  bool ok = true, waited = false;
+  int ul = -1;  // layer whose u is in us
+  int64_t gs = 0;
+  for (int64_t u = u_begin; u < u_end;) {
+    int l, R;
+    int64_t rb;
+    seg_of(u, l, rb, R);
+    u += R;
+    const DecLayer& L = g.L[l];
+    const int64_t row0 = rb * 16, N = L.N;
+    const int nkb = L.nkb;
+    const int nsb = (nkb + kDecSbBlocks - 1) / kDecSbBlocks;
+    const float mu = __ldg(L.mean);
+    // this segment's rows of B (bf16 [16R, r]) for its epilogue: asynchronous 16-byte
+    // copies when the rows are 16-byte aligned (r a multiple of 8), else plain loads
+    const int r = g.r;
+    if ((r & 7) == 0) {
+      const int np = 16 * R * r / 8;
+      for (int i = tid; i < np; i += kDecThreads) {
+        const int64_t n = row0 + (i * 8) / r;
+        const bool in = n < N;
+        cp_async16(smem_u32(bs + i * 8), in ? L.Bm + row0 * r + i * 8 : L.Bm, in ? 16u : 0u);
+      }
+      cp_async_commit();
+    } else {
+      for (int i = tid; i < 16 * R * r; i += kDecThreads) {
+        const int64_t n = row0 + i / r;
+        bs[i] = n < N ? L.Bm[n * r + i % r] : static_cast<uint16_t>(0);
       }
     }
-  };
-  uint32_t pq[kCpl];
-  float psc[kCpl];
-  cload(0, pq, psc);
-  compute_sync();  // the tables and B rows are ready
-  bool ok = true;
-
-  for (int j = 0; j < nsb; ++j) {
-    const int kb = j * kDecSbBlocks + warp;
-    if (ok) ok = warp_wait(&full[j % nst], static_cast<uint32_t>((j / nst) & 1), wait_ns, &s_abort, 61);
-    if (!ok) continue;  // after a give-up no stage is released: the producer stops
-    if (kb >= nkb) {
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[j % nst]);
-      continue;
-    }
-    const uint32_t sb = smem_u32(ring + (j % nst) * stb);
-    // c of the CTA's rows for block kb, exchanged through the warp's scratch: packed
-    // row rr at word (rr mod 8) * 2 kDecMaxRb + rr / 8, so thread (g, t) reads its rows
-    // pg + 8 i at pg * 2 kDecMaxRb + i
+    // block constants (code2 byte, scale2) of rows lane + 32 c for this warp's block of
+    // stage j, loaded one stage ahead of their use
+    auto cload = [&](int j, uint32_t (&q)[kCpl], float (&sc)[kCpl]) {
+      const int kb = j * kDecSbBlocks + warp;
 #pragma unroll
-    for (int c = 0; c < kCpl; ++c) {
-      const int rr = lane + 32 * c;
-      if (rr < kDecMaxRows)
-        cs[(rr & 7) * (2 * kDecMaxRb) + (rr >> 3)] =
-            fmaf(e4m3_to_f32(static_cast<uint8_t>(pq[c])), psc[c], mu);
-    }
-    cload(j + 1, pq, psc);  // the next stage's constants land while the tensor cores work
-    __syncwarp();
-    float ch[2 * kDecMaxRb];
-#pragma unroll
-    for (int jj = 0; jj < kDecMaxRb; ++jj) {
-      const float2 v = *reinterpret_cast<const float2*>(cs + pg * (2 * kDecMaxRb) + 2 * jj);
-      ch[2 * jj] = v.x;
-      ch[2 * jj + 1] = v.y;
-    }
-    // token fragments: row g (+ 8), columns 16 t .. 16 t + 15 of this warp's block
-    // (row rho = warp M + row of the box, pieces 2t, 2t+1 swizzled by rho mod 8)
-    uint4 xa[Q], xb[Q];
-#pragma unroll
-    for (int q = 0; q < Q; ++q) {
-      const int tr = g + 8 * q < M ? g + 8 * q : M - 1;
-      const uint32_t rho = static_cast<uint32_t>(warp * M + tr);
-      const uint32_t rowa = sb + rho * 128u;
-      xa[q] = lds_u4d(rowa + ((static_cast<uint32_t>(2 * t) ^ (rho & 7u)) << 4));
-      xb[q] = lds_u4d(rowa + ((static_cast<uint32_t>(2 * t + 1) ^ (rho & 7u)) << 4));
-    }
-    // this warp's 32 packed bytes of a row: 128-byte group warp / 4, pieces 2 (warp mod 4)
-    // and + 1, swizzled by the 128-byte line: line = r * 4 + group (w3d) or
-    // group * 16R + r (four 2-D boxes)
-    const uint32_t gg = warp >> 2;
-    const uint32_t u0 = 2u * (warp & 3) + (t >> 1);
-    auto wline = [&](int r) { return w3d ? static_cast<uint32_t>(r) * 4u + gg : gg * 16u * R + r; };
-    const float z[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int rb = 0; rb < kDecMaxRb; ++rb) {
-      if (rb < R) {
-        const uint32_t la = wline(rb * 16 + pg), lb = wline(rb * 16 + 8 + pg);
-        const uint2 wa = lds_u2d(sb + woff + la * 128u + (((u0 ^ (la & 7u)) << 4) | ((t & 1) << 3)));
-        const uint2 wb = lds_u2d(sb + woff + lb * 128u + (((u0 ^ (lb & 7u)) << 4) | ((t & 1) << 3)));
-        float d[Q][4];
-#pragma unroll
-        for (int k4 = 0; k4 < 4; ++k4) {
-          const uint32_t wlo = k4 < 2 ? wa.x : wa.y, whi = k4 < 2 ? wb.x : wb.y;
-          const int i0 = (2 * k4) & 3;
-          const uint32_t a0 = lut_pair(lutb, wlo, i0), a2 = lut_pair(lutb, wlo, i0 + 1);
-          const uint32_t a1 = lut_pair(lutb, whi, i0), a3 = lut_pair(lutb, whi, i0 + 1);
-#pragma unroll
-          for (int q = 0; q < Q; ++q) {
-            const uint4& xv = k4 < 2 ? xa[q] : xb[q];
-            const uint32_t b0 = (k4 & 1) ? xv.z : xv.x, b1 = (k4 & 1) ? xv.w : xv.y;
-            if (k4 == 0)
-              mma_bf16_16816(d[q], a0, a1, a2, a3, b0, b1, z);
-            else
-              mma_bf16_16816(d[q], a0, a1, a2, a3, b0, b1, d[q]);
+      for (int c = 0; c < kCpl; ++c) {
+        q[c] = 0u;
+        sc[c] = 0.f;
+        const int rr = lane + 32 * c;
+        const int64_t n = row0 + rr;
+        if (j < nsb && kb < nkb && rr < 16 * R && n < N) {
+          const int64_t blk = n * nkb + kb;
+          if (in_bounds((blk >> 8) < L.nb2, 71)) {
+            q[c] = L.code2[blk];
+            sc[c] = L.scale2[blk >> 8];
           }
         }
+      }
+    };
+    uint32_t pq[kCpl];
+    float psc[kCpl];
+    cload(0, pq, psc);
+    float acc[kDecMaxRb][Q][4];
 #pragma unroll
-        for (int q = 0; q < Q; ++q) {
-          acc[rb][q][0] = fmaf(ch[2 * rb], d[q][0], acc[rb][q][0]);
-          acc[rb][q][1] = fmaf(ch[2 * rb], d[q][1], acc[rb][q][1]);
-          acc[rb][q][2] = fmaf(ch[2 * rb + 1], d[q][2], acc[rb][q][2]);
-          acc[rb][q][3] = fmaf(ch[2 * rb + 1], d[q][3], acc[rb][q][3]);
+    for (int b = 0; b < kDecMaxRb; ++b)
+#pragma unroll
+      for (int q = 0; q < Q; ++q)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[b][q][e] = 0.f;
+    const uint32_t gg = warp >> 2;
+    const uint32_t u0 = 2u * (warp & 3) + (t >> 1);
+    // this warp's 32 packed bytes of row rr: 128-byte group warp / 4, pieces 2 (warp mod
+    // 4) and + 1, swizzled by the 128-byte line: line = rr * 4 + group (3-D boxes) or
+    // group * 16R + rr (four 2-D boxes)
+    auto wline = [&](int rr) {
+      return L.w3d ? static_cast<uint32_t>(rr) * 4u + gg : gg * 16u * R + static_cast<uint32_t>(rr);
+    };
+    for (int j = 0; j < nsb; ++j, ++gs) {
+      if (ok) ok = warp_wait(&full[gs % nst], static_cast<uint32_t>((gs / nst) & 1), wait_ns, &s_abort, 61);
+      if (!ok) continue;  // after a give-up no stage is released: the producer stops
+      const int kb = j * kDecSbBlocks + warp;
+      if (kb >= nkb) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[gs % nst]);
+        continue;
+      }
+      const uint32_t sb = smem_u32(ring + (gs % nst) * stb);
+      // c of the segment's rows for block kb, exchanged through the warp's scratch:
+      // packed row rr at word (rr mod 8) * 2 kDecMaxRb + rr / 8, so thread (g8, t) reads
+      // its rows pg + 8 i at pg * 2 kDecMaxRb + i
+#pragma unroll
+      for (int c = 0; c < kCpl; ++c) {
+        const int rr = lane + 32 * c;
+        if (rr < kDecMaxRows)
+          cs[(rr & 7) * (2 * kDecMaxRb) + (rr >> 3)] =
+              fmaf(e4m3_to_f32(static_cast<uint8_t>(pq[c])), psc[c], mu);
+      }
+      cload(j + 1, pq, psc);  // the next stage's constants land while the tensor cores work
+      __syncwarp();
+      float ch[2 * kDecMaxRb];
+#pragma unroll
+      for (int i = 0; i < kDecMaxRb; ++i) {
+        const float2 v = *reinterpret_cast<const float2*>(cs + pg * (2 * kDecMaxRb) + 2 * i);
+        ch[2 * i] = v.x;
+        ch[2 * i + 1] = v.y;
+      }
+      // token fragments: row g8 (+ 8), columns 16 t .. 16 t + 15 of this warp's block
+      // (row rho = warp M + row of the box, pieces 2t, 2t+1 swizzled by rho mod 8)
+      uint4 xa[Q], xb[Q];
+#pragma unroll
+      for (int q = 0; q < Q; ++q) {
+        const int tr = g8 + 8 * q < M ? g8 + 8 * q : M - 1;
+        const uint32_t rho = static_cast<uint32_t>(warp * M + tr);
+        const uint32_t rowa = sb + rho * 128u;
+        xa[q] = lds_u4d(rowa + ((static_cast<uint32_t>(2 * t) ^ (rho & 7u)) << 4));
+        xb[q] = lds_u4d(rowa + ((static_cast<uint32_t>(2 * t + 1) ^ (rho & 7u)) << 4));
+      }
+      const float z[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int b = 0; b < kDecMaxRb; ++b) {
+        if (b < R) {
+          const uint32_t la = wline(b * 16 + pg), lb = wline(b * 16 + 8 + pg);
+          const uint2 wa = lds_u2d(sb + woff + la * 128u + (((u0 ^ (la & 7u)) << 4) | ((t & 1) << 3)));
+          const uint2 wb = lds_u2d(sb + woff + lb * 128u + (((u0 ^ (lb & 7u)) << 4) | ((t & 1) << 3)));
+          float d[Q][4];
+#pragma unroll
+          for (int k4 = 0; k4 < 4; ++k4) {
+            const uint32_t wlo = k4 < 2 ? wa.x : wa.y, whi = k4 < 2 ? wb.x : wb.y;
+            const int i0 = (2 * k4) & 3;
+            const uint32_t a0 = lut_pair(lutb, wlo, i0), a2 = lut_pair(lutb, wlo, i0 + 1);
+            const uint32_t a1 = lut_pair(lutb, whi, i0), a3 = lut_pair(lutb, whi, i0 + 1);
+#pragma unroll
+            for (int q = 0; q < Q; ++q) {
+              const uint4& xv = k4 < 2 ? xa[q] : xb[q];
+              const uint32_t b0 = (k4 & 1) ? xv.z : xv.x, b1 = (k4 & 1) ? xv.w : xv.y;
+              if (k4 == 0)
+                mma_bf16_16816(d[q], a0, a1, a2, a3, b0, b1, z);
+              else
+                mma_bf16_16816(d[q], a0, a1, a2, a3, b0, b1, d[q]);
+            }
+          }
+#pragma unroll
+          for (int q = 0; q < Q; ++q) {
+            acc[b][q][0] = fmaf(ch[2 * b], d[q][0], acc[b][q][0]);
+            acc[b][q][1] = fmaf(ch[2 * b], d[q][1], acc[b][q][1]);
+            acc[b][q][2] = fmaf(ch[2 * b + 1], d[q][2], acc[b][q][2]);
+            acc[b][q][3] = fmaf(ch[2 * b + 1], d[q][3], acc[b][q][3]);
+          }
         }
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[gs % nst]);  // this warp is done with the stage
     }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[j % nst]);  // this warp is done with the stage
+    if (!ok) break;
+
+    // ---- segment end: u of this layer (once the adapter kernel has finished), the
+    // fixed-order sum of the 16 warps' partials (warp w adds into slot w % 4, warps 0-3
+    // first, then 4-7, 8-11, 12-15; slots [token][row], rows padded to kDecRedRow) ----
+    if (!waited) {
+      griddep_wait();
+      waited = true;
+    }
+    const int nu = r * M;
+    const bool newu = l != ul;
+    float up[kDecMaxUParts / 4];
+    if (newu) {
+#pragma unroll
+      for (int c = 0; c < kDecMaxUParts / 4; ++c)
+        up[c] = (tid < nu && c < L.ks) ? __ldcg(L.upart + static_cast<int64_t>(c) * nu + tid) : 0.f;
+    }
+    float* slot = red + (warp % kDecRedSlots) * (16 * kDecRedRow);
+#pragma unroll
+    for (int round = 0; round < kDecWarps / kDecRedSlots; ++round) {
+      if (warp / kDecRedSlots == round) {
+#pragma unroll
+        for (int b = 0; b < kDecMaxRb; ++b) {
+          if (b < R) {
+#pragma unroll
+            for (int q = 0; q < Q; ++q) {
+              const int rw = b * 16 + pg, tk = 8 * q + 2 * t;  // the packed row of mma row g8
+              float* p = slot + tk * kDecRedRow + rw;
+              if (round == 0) {
+                p[0] = acc[b][q][0];
+                p[kDecRedRow] = acc[b][q][1];
+                p[8] = acc[b][q][2];
+                p[kDecRedRow + 8] = acc[b][q][3];
+              } else {
+                p[0] += acc[b][q][0];
+                p[kDecRedRow] += acc[b][q][1];
+                p[8] += acc[b][q][2];
+                p[kDecRedRow + 8] += acc[b][q][3];
+              }
+            }
+          }
+        }
+      }
+      compute_sync();
+    }
+    if (newu) {
+      for (int i = tid; i < nu; i += kDecThreads) {
+        float v = 0.f;
+        if (i == tid) {
+#pragma unroll
+          for (int c = 0; c < kDecMaxUParts / 4; ++c) v += up[c];
+        } else {
+          for (int c = 0; c < kDecMaxUParts / 4 && c < L.ks; ++c)
+            v += __ldcg(L.upart + static_cast<int64_t>(c) * nu + i);
+        }
+        for (int c = kDecMaxUParts / 4; c < L.ks; ++c) v += __ldcg(L.upart + static_cast<int64_t>(c) * nu + i);
+        us[i] = v;
+      }
+      ul = l;
+    }
+    cp_async_wait_all();  // the B rows
+    compute_sync();
+    // outputs o = m * 16 R + row: h[m, row0 + row] = sum of the slots + s B u
+    const int nrows = 16 * R;
+    const int nout = nrows * M;
+    for (int o = tid; o < nout; o += kDecThreads) {
+      const int rl = o % nrows, m = o / nrows;
+      const int64_t n = row0 + rl;
+      if (n >= N) continue;
+      float v = 0.f;
+#pragma unroll
+      for (int sl = 0; sl < kDecRedSlots; ++sl) v += red[sl * (16 * kDecRedRow) + m * kDecRedRow + rl];
+      const uint16_t* brow = bs + rl * r;
+      float lr = 0.f;
+      if ((r & 7) == 0) {
+        for (int j = 0; j < r; j += 8) {
+          const uint4 bv = *reinterpret_cast<const uint4*>(brow + j);
+          const float* uj = us + j * M + m;
+          lr = fmaf(bf16lo(bv.x), uj[0], lr);
+          lr = fmaf(bf16hi(bv.x), uj[M], lr);
+          lr = fmaf(bf16lo(bv.y), uj[2 * M], lr);
+          lr = fmaf(bf16hi(bv.y), uj[3 * M], lr);
+          lr = fmaf(bf16lo(bv.z), uj[4 * M], lr);
+          lr = fmaf(bf16hi(bv.z), uj[5 * M], lr);
+          lr = fmaf(bf16lo(bv.w), uj[6 * M], lr);
+          lr = fmaf(bf16hi(bv.w), uj[7 * M], lr);
+        }
+      } else {
+        for (int j = 0; j < r; ++j) lr = fmaf(bf16lo(brow[j]), us[j * M + m], lr);
+      }
+      const float out = fmaf(g.scale, lr, v);
+      if (in_bounds(m < M, 74))
+        L.h[static_cast<int64_t>(m) * N + n] = static_cast<uint16_t>(pack_bf16x2(out, 0.f) & 0xFFFFu);
+    }
+    compute_sync();  // red, us and bs are reused by the next segment
   }
   // Drain: after a give-up, the stages issued but not waited for must land before the
-  // ring is reused or the CTA exits (one deadline). At most nst stages can be in
-  // flight, each in its own buffer; the waits below return at once for those that landed.
+  // CTA exits (one deadline). At most nst stages can be in flight, each in its own slot.
   compute_sync();
   if (tid == 0 && s_abort) {
     const long long t0 = wait_clock();
     while (s_issued < 0 && wait_clock() - t0 <= ns_cycles(drain_ns(wait_ns))) {
     }
-    const int issued = s_issued < 0 ? nsb : s_issued;
+    const int issued = s_issued < 0 ? 0 : s_issued;
     for (int jj = issued - nst > 0 ? issued - nst : 0; jj < issued; ++jj) {
       while (!mbar_try_wait_long(&full[jj % nst], static_cast<uint32_t>((jj / nst) & 1))) {
         if (wait_clock() - t0 > ns_cycles(drain_ns(wait_ns))) {
@@ -441,94 +573,7 @@ __global__ void __launch_bounds__(kDecBlockThreads, 1)
       }
     }
   }
-  cp_async_wait_all();  // the B rows
-  compute_sync();  // every warp is done with the ring, which now holds the reduction
-
-  // u once the adapter kernel has finished: entry i = j M + m sums its ks partials in
-  // order; the loads go out before the warps' reduction, which hides their latency
-  griddep_wait();
-  const int nu = a.r * a.M;
-  float up[kDecMaxUParts / 4];
-  const bool uact = tid < nu;  // nu <= 1024: threads tid and tid + 512 (second pass below)
-#pragma unroll
-  for (int c = 0; c < kDecMaxUParts / 4; ++c)
-    up[c] = (uact && c < a.ks) ? __ldcg(a.upart + static_cast<int64_t>(c) * nu + tid) : 0.f;
-  // ---- fixed-order sum of the 16 warps' partials: warp w adds into slot w % 4, warps
-  // 0-3 first, then 4-7, 8-11, 12-15; slot layout [token][row], rows padded to 84 ----
-  float* slot = red + (warp % kDecRedSlots) * (16 * kDecRedRow);
-#pragma unroll
-  for (int round = 0; round < kDecWarps / kDecRedSlots; ++round) {
-    if (warp / kDecRedSlots == round) {
-#pragma unroll
-      for (int rb = 0; rb < kDecMaxRb; ++rb) {
-        if (rb < R) {
-#pragma unroll
-          for (int q = 0; q < Q; ++q) {
-            const int rw = rb * 16 + pg, tk = 8 * q + 2 * t;  // the packed row of mma row g
-            float* p = slot + tk * kDecRedRow + rw;
-            const float v[4] = {acc[rb][q][0], acc[rb][q][1], acc[rb][q][2], acc[rb][q][3]};
-            if (round == 0) {
-              p[0] = v[0];
-              p[kDecRedRow] = v[1];
-              p[8] = v[2];
-              p[kDecRedRow + 8] = v[3];
-            } else {
-              p[0] += v[0];
-              p[kDecRedRow] += v[1];
-              p[8] += v[2];
-              p[kDecRedRow + 8] += v[3];
-            }
-          }
-        }
-      }
-    }
-    compute_sync();
-  }
-  for (int i = tid; i < nu; i += kDecThreads) {
-    float v = 0.f;
-    if (i == tid) {
-#pragma unroll
-      for (int c = 0; c < kDecMaxUParts / 4; ++c) v += up[c];
-    } else {
-      for (int c = 0; c < kDecMaxUParts / 4 && c < a.ks; ++c) v += __ldcg(a.upart + static_cast<int64_t>(c) * nu + i);
-    }
-    for (int c = kDecMaxUParts / 4; c < a.ks; ++c) v += __ldcg(a.upart + static_cast<int64_t>(c) * nu + i);
-    us[i] = v;
-  }
-  compute_sync();
-  // outputs o = m * 16 R + row: h[m, row0 + row] = sum of the slots + s B u
-  const int nrows = 16 * R;
-  const int nout = nrows * a.M;
-  const bool vec = (a.r & 7) == 0;
-  for (int o = tid; o < nout; o += kDecThreads) {
-    const int rl = o % nrows, m = o / nrows;
-    const int64_t n = row0 + rl;
-    if (n >= a.N) continue;
-    float v = 0.f;
-#pragma unroll
-    for (int sl = 0; sl < kDecRedSlots; ++sl) v += red[sl * (16 * kDecRedRow) + m * kDecRedRow + rl];
-    const uint16_t* brow = bs + rl * a.r;
-    float l = 0.f;
-    if (vec) {
-      for (int j = 0; j < a.r; j += 8) {
-        const uint4 bv = *reinterpret_cast<const uint4*>(brow + j);
-        const float* uj = us + j * a.M + m;
-        l = fmaf(bf16lo(bv.x), uj[0], l);
-        l = fmaf(bf16hi(bv.x), uj[a.M], l);
-        l = fmaf(bf16lo(bv.y), uj[2 * a.M], l);
-        l = fmaf(bf16hi(bv.y), uj[3 * a.M], l);
-        l = fmaf(bf16lo(bv.z), uj[4 * a.M], l);
-        l = fmaf(bf16hi(bv.z), uj[5 * a.M], l);
-        l = fmaf(bf16lo(bv.w), uj[6 * a.M], l);
-        l = fmaf(bf16hi(bv.w), uj[7 * a.M], l);
-      }
-    } else {
-      for (int j = 0; j < a.r; ++j) l = fmaf(bf16lo(brow[j]), us[j * a.M + m], l);
-    }
-    const float out = fmaf(a.scale, l, v);
-    if (in_bounds(m < a.M, 74))
-      a.h[static_cast<int64_t>(m) * a.N + n] = static_cast<uint16_t>(pack_bf16x2(out, 0.f) & 0xFFFFu);
-  }
+  cp_async_wait_all();
 }
 
 }  // namespace qnf4

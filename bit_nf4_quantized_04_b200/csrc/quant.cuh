@@ -173,6 +173,10 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
   }
   fence_mbar_init();
   __syncthreads();
+  // launched as a programmatic dependent: the prologue above overlapped the previous
+  // kernel; wait for it before touching global memory, and let the next kernel start
+  griddep_wait();
+  griddep_launch_dependents();
 
   const int64_t nchunks = (nblocks + kQChunkBlocks - 1) / kQChunkBlocks;
   const int64_t gw = static_cast<int64_t>(blockIdx.x) * kQWorkers + warp;  // this warp
@@ -357,6 +361,8 @@ QNF4_DEV double block_sum_partials(const double* __restrict__ part, int n) {
 // Sum n float64 partials in a fixed order (one CTA of 256 threads) into *out.
 __global__ void __launch_bounds__(256) k_sum_partials(const double* __restrict__ part, int n,
                                                       double* __restrict__ out) {
+  griddep_wait();  // (programmatic dependent of the kernel that wrote the partials)
+  griddep_launch_dependents();
   const double t = block_sum_partials(part, n);
   if (threadIdx.x == 0) *out = t;
 }
@@ -398,6 +404,8 @@ __global__ void __launch_bounds__(256) k_dq_encode(const float* __restrict__ c, 
                                                    const double* __restrict__ sse_part = nullptr,
                                                    int nsse = 0, double* __restrict__ sse_out = nullptr) {
   __shared__ float s_mu;
+  griddep_wait();  // (programmatic dependent of the kernel that wrote the constants)
+  griddep_launch_dependents();
   const int lane = threadIdx.x & 31;
   // (fused quantize path) CTA 0 also folds the quantizer's SSE partials, in the same
   // order as k_sum_partials

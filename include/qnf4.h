@@ -169,6 +169,23 @@ QNF4_API qnf4_status qnf4_qlora_linear_fwd(const qnf4_weight* w, const void* x, 
                                   const void* A, const void* B, int32_t r, float scale,
                                   void* h, void* ws, size_t ws_bytes, void* stream);
 
+/* [QLoRA opening formula] The forward of n (1..8) independent layers at decode sizes
+ * (1 <= M <= 16 tokens) in one launch pair: layer l computes h[l] = x[l] bf16(W_hat_l)^T
+ * + scale (x[l] A[l]^T) B[l]^T exactly as qnf4_qlora_linear_fwd does for it (each row's
+ * arithmetic is the same, so the results are bit-identical to n separate calls). All
+ * layers share M, r and scale; w is an array of n weights, x, A, B and h host arrays of
+ * n device pointers with each layer's own shapes (as for the single call). The launch
+ * spreads the layers' weight rows over the SMs by bytes, so small layers do not leave
+ * SMs idle. ws must hold the sum over the layers of
+ * qnf4_workspace_size(QNF4_OP_FWD, N_l, K_l, M, r). Errors: QNF4_ERR_ARG for n outside
+ * 1..8 or NULL arrays, QNF4_ERR_SHAPE for M outside 1..16, and each layer's checks of the
+ * single call. */
+QNF4_API qnf4_status qnf4_qlora_linear_fwd_group(int32_t n, const qnf4_weight* w,
+                                                 const void* const* x, int64_t M,
+                                                 const void* const* A, const void* const* B,
+                                                 int32_t r, float scale, void* const* h,
+                                                 void* ws, size_t ws_bytes, void* stream);
+
 /* The forward above without a workspace argument, for callers that cannot allocate
  * device memory: code that runs where cudaMalloc is unavailable or forbidden (an
  * allocator callback, a host hook inside a pre-planned inference engine, a caller

@@ -32,7 +32,8 @@ def _declared():
 def test_header_declares_the_abi():
     names = _declared()
     for n in ("qnf4_nf4_codebook", "qnf4_nf4_quantize", "qnf4_double_quant", "qnf4_dequant",
-              "qnf4_qlora_linear_fwd", "qnf4_qlora_linear_bwd", "qnf4_nf4_recon_error",
+              "qnf4_qlora_linear_fwd", "qnf4_qlora_linear_fwd_group", "qnf4_qlora_linear_bwd",
+              "qnf4_nf4_recon_error",
               "qnf4_chanq_quantize", "qnf4_chanq_linear_fwd", "qnf4_workspace_size",
               "qnf4_last_error"):
         assert n in names
@@ -107,6 +108,19 @@ def test_argument_checks_fail_before_any_launch(q):
     assert _st(q, "qnf4_rank_topk", None, None, 3, 1, None) == 1
     assert _st(q, "qnf4_set_wait_timeout_ns", 0) == 1
     assert b"positive" in q.lib.qnf4_last_error()
+    # grouped forward: n in 1..8, M in 1..16, per-layer checks as for the single call
+    arr = (q.Qnf4Weight * 2)(w, w)
+    ptrs = (C.c_void_p * 2)(fake, fake)
+    assert _st(q, "qnf4_qlora_linear_fwd_group", 0, arr, ptrs, 4, ptrs, ptrs, 8, 1.0, ptrs, fake,
+               1 << 20, None) == 1
+    assert _st(q, "qnf4_qlora_linear_fwd_group", 9, arr, ptrs, 4, ptrs, ptrs, 8, 1.0, ptrs, fake,
+               1 << 20, None) == 1
+    assert _st(q, "qnf4_qlora_linear_fwd_group", 2, arr, ptrs, 17, ptrs, ptrs, 8, 1.0, ptrs, fake,
+               1 << 20, None) == 2
+    assert _st(q, "qnf4_qlora_linear_fwd_group", 2, arr, ptrs, 4, ptrs, ptrs, 65, 1.0, ptrs, fake,
+               1 << 20, None) == 1
+    assert _st(q, "qnf4_qlora_linear_fwd_group", 2, arr, ptrs, 4, ptrs, ptrs, 8, 1.0, ptrs, fake,
+               16, None) == 6
 
 
 def test_argument_checks_of_the_next_rows(q):

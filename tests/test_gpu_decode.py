@@ -96,3 +96,39 @@ def test_decode_long_k(q):
     w = weight_from_oracle(q, oq, N, K)
     h = q.qlora_linear_fwd(w, x.cuda(), A.cuda(), B.cuda(), s)
     assert_close(f64(h.cpu()), href, "h at K = 16640")
+
+
+def test_group_matches_single_calls_bit_exactly(q):
+    """n independent layers in one grouped launch give exactly the single calls' outputs
+    (each row's arithmetic is the same), and one layer is checked against the oracle."""
+    shapes = [(520, 2048), (40, 448), (1000, 4096), (264, 960), (200, 192), (136, 1024), (16, 64)]
+    for M in (1, 5, 16):
+        cases = [_case(N, K, M, 16, seed=900 + 7 * i + M) for i, (N, K) in enumerate(shapes)]
+        ws_ = [weight_from_oracle(q, c[0], N, K) for c, (N, K) in zip(cases, shapes)]
+        xs = [c[1].cuda() for c in cases]
+        As = [c[2].cuda() for c in cases]
+        Bs = [c[3].cuda() for c in cases]
+        s = cases[0][4]
+        single = [q.qlora_linear_fwd(w, x, A, B, s) for w, x, A, B in zip(ws_, xs, As, Bs)]
+        group = q.qlora_linear_fwd_group(ws_, xs, As, Bs, s)
+        torch.cuda.synchronize()
+        for i, (a, b) in enumerate(zip(single, group)):
+            assert torch.equal(a, b), f"layer {i} M={M}: grouped output differs from the single call"
+        assert_close(f64(group[2].cpu()), cases[2][5], f"group layer 2 M={M}")
+
+
+def test_group_llama7b_layer_set(q):
+    """The 7B layer set (q, k, v, o, gate, up, down) at 4 tokens in one launch against
+    the single calls, bit for bit."""
+    ws_, xs, As, Bs = [], [], [], []
+    for i, s_ in enumerate(synth.LLAMA7B_SET):
+        W = synth.llama_weight((s_.N, s_.K), 3100 + i, device="cuda")
+        ws_.append(q.quantize_weight(W))
+        xs.append(synth.normal_bf16((4, s_.K), 1.0, 3200 + i, device="cuda"))
+        As.append(synth.normal_bf16((16, s_.K), 0.01, 3300 + i, device="cuda"))
+        Bs.append(synth.normal_bf16((s_.N, 16), 0.01, 3400 + i, device="cuda"))
+    single = [q.qlora_linear_fwd(w, x, A, B, 2.0) for w, x, A, B in zip(ws_, xs, As, Bs)]
+    group = q.qlora_linear_fwd_group(ws_, xs, As, Bs, 2.0)
+    torch.cuda.synchronize()
+    for i, (a, b) in enumerate(zip(single, group)):
+        assert torch.equal(a, b), f"layer {i}"
