@@ -433,30 +433,43 @@ def breakdown(wl, q, hbm, tc):
         hs = [torch.empty(m, L["N"], dtype=torch.bfloat16, device=wl.dev) for L in wl.layers]
         ctr = [0]
 
-        def run():
+        As = [L["A"] for L in wl.layers]
+        Bs = [L["B"] for L in wl.layers]
+
+        def run_group():  # the 7 layers in one grouped launch pair
+            ws_ = pool[ctr[0] % copies]
+            ctr[0] += 1
+            q.qlora_linear_fwd_group(ws_, xs, As, Bs, wl.s, hs=hs, ws=wl.ws)
+
+        def run_single():  # one call per layer
             ws_ = pool[ctr[0] % copies]
             ctr[0] += 1
             for i, L in enumerate(wl.layers):
                 q.qlora_linear_fwd(ws_[i], xs[i], L["A"], L["B"], wl.s, h=hs[i], ws=wl.ws)
-        run()
-        torch.cuda.synchronize()
-        # one decode pass is a few microseconds of GPU work per layer, far below the
-        # host's per-call cost: capture the 7-layer passes over every weight copy in
-        # one CUDA graph and time its replays
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph):
-            for _ in range(copies):
-                run()
-        graph.replay()
-        torch.cuda.synchronize()
-        t = time_loop(graph.replay, 3, torch.cuda.current_stream()) / copies
         byt = sum(N * K * (0.5 + 1 / 64 + 4 / 16384) + m * K * 2 + RANK * (N + K) * 2 + m * N * 2
                   for N, K in layer_shapes())
-        dec[f"M{m}"] = {"GBps": round(byt / t / 1e9, 1), "frac_hbm": round(byt / t / 1e9 / hbm, 3),
-                        "us": round(t * 1e6, 1)}
+        res = {}
+        for nm, run in (("group", run_group), ("single_calls", run_single)):
+            run()
+            torch.cuda.synchronize()
+            # one decode pass is a few microseconds of GPU work per layer, far below the
+            # host's per-call cost: capture the 7-layer passes over every weight copy in
+            # one CUDA graph and time its replays
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                for _ in range(copies):
+                    run()
+            graph.replay()
+            torch.cuda.synchronize()
+            t = time_loop(graph.replay, 3, torch.cuda.current_stream()) / copies
+            res[nm] = {"GBps": round(byt / t / 1e9, 1), "frac_hbm": round(byt / t / 1e9 / hbm, 3),
+                       "us": round(t * 1e6, 1)}
+            del graph
+        dec[f"M{m}"] = dict(res["group"], single_calls=res["single_calls"])
     out["decode_fwd"] = dec
     out["decode_fwd"]["pool_copies"] = copies
-    out["decode_fwd"]["launch"] = "CUDA graph of all copies x 7 layers, PDL edges"
+    out["decode_fwd"]["launch"] = ("CUDA graph of all copies; per copy one qnf4_qlora_linear_fwd_group "
+                                   "call over the 7 layers (single_calls: one call per layer)")
     q.check()
     return out
 
@@ -504,10 +517,12 @@ def protocol(wl, q, hbm, tc_burst, tc_sus, dev, seconds=2.0, sessions=3):
     xs = [L["x"][:16].contiguous() for L in wl.layers]
     hs = [torch.empty(16, L["N"], dtype=torch.bfloat16, device=dev) for L in wl.layers]
 
+    As = [L["A"] for L in wl.layers]
+    Bs = [L["B"] for L in wl.layers]
+
     def dec_all():
         for ws_ in pool:
-            for i, L in enumerate(wl.layers):
-                q.qlora_linear_fwd(ws_[i], xs[i], L["A"], L["B"], wl.s, h=hs[i], ws=wl.ws)
+            q.qlora_linear_fwd_group(ws_, xs, As, Bs, wl.s, hs=hs, ws=wl.ws)
     dec = graphed(dec_all)
     dbytes = sum(N * K * (0.5 + 1 / 64 + 4 / 16384) + 16 * K * 2 + RANK * (N + K) * 2 + 16 * N * 2
                  for N, K in layer_shapes())

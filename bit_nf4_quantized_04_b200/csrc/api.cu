@@ -205,7 +205,7 @@ bool make_map_xblocks(CUtensorMap* m, const void* x, uint64_t K, uint64_t M, uin
   if (!fn) return false;
   cuuint64_t dims[3] = {64, M, K / 64};
   cuuint64_t strides[2] = {K * 2, 128};
-  cuuint32_t box[3] = {64, rows, 16};
+  cuuint32_t box[3] = {64, rows, kDecSbBlocks};
   cuuint32_t estr[3] = {1, 1, 1};
   const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(x), dims, strides,
                         box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -221,7 +221,7 @@ bool make_map_wcols(CUtensorMap* m, const void* packed, uint64_t K, uint64_t N, 
   if (!fn) return false;
   cuuint64_t dims[3] = {128, K / 256, N};
   cuuint64_t strides[2] = {128, K / 2};
-  cuuint32_t box[3] = {128, 4, rows};
+  cuuint32_t box[3] = {128, kDecGroups, rows};
   cuuint32_t estr[3] = {1, 1, 1};
   const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(packed), dims, strides,
                         box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,

@@ -46,13 +46,15 @@
 
 namespace qnf4 {
 
-constexpr int kDecWarps = 16;                  // compute warps
+constexpr int kDecWarps = 12;                  // compute warps
 constexpr int kDecThreads = 32 * kDecWarps;
 constexpr int kDecBlockThreads = kDecThreads + 32;  // plus the producer warp
 constexpr int kDecMaxRb = 5;      // 16-row blocks a CTA holds at most
 constexpr int kDecMaxRows = 16 * kDecMaxRb;
 constexpr int kDecMaxStages = 4;
-constexpr int kDecSbBlocks = 16;            // column blocks per stage (one per warp)
+constexpr int kDecSbBlocks = kDecWarps;     // column blocks per stage (one per warp)
+constexpr int kDecGroups = kDecSbBlocks / 4;  // 128-byte packed groups per stage row
+static_assert(kDecSbBlocks % 4 == 0, "a stage holds whole 128-byte packed groups");
 constexpr uint32_t kDecRingBytes = 152u * 1024u;
 constexpr int kDecLutCopies = 32;
 constexpr int kDecRedSlots = 4;
@@ -64,10 +66,13 @@ constexpr uint32_t kDecBsBytes = kDecMaxRows * 64u * 2u;                     // 
 constexpr uint32_t kDecUsBytes = 64u * 16u * 4u;                             // 4 KB: u [r][M]
 constexpr size_t kDecSmem =
     1024 + kDecRingBytes + kDecLutBytes + kDecCsBytes + kDecBsBytes + kDecRedBytes + kDecUsBytes;
-// stage = the token box (16 blocks x M rows x 128 B), then 4 packed boxes (16R rows x
-// 128 B); every box starts on a 1024-byte boundary
+// stage = the token box (kDecSbBlocks blocks x M rows x 128 B), then the packed rows
+// (kDecGroups x 16R rows x 128 B); both start on a 1024-byte boundary (the swizzle's)
+__host__ __device__ constexpr uint32_t dec_x_bytes(int M) {
+  return (128u * kDecSbBlocks * M + 1023u) & ~1023u;
+}
 __host__ __device__ constexpr uint32_t dec_stage_bytes(int R, int M) {
-  return 2048u * M + 8192u * R;
+  return dec_x_bytes(M) + ((2048u * kDecGroups * R + 1023u) & ~1023u);
 }
 __host__ __device__ constexpr int dec_stages(int R, int M) {
   return static_cast<int>(kDecRingBytes / dec_stage_bytes(R, M)) < kDecMaxStages
@@ -228,7 +233,7 @@ __global__ void __launch_bounds__(kDecBlockThreads, 1)
   const int M = g.M;
   const uint32_t stb = dec_stage_bytes(kDecMaxRb, M);
   const int nst = dec_stages(kDecMaxRb, M);
-  const uint32_t woff = 2048u * M;
+  const uint32_t woff = dec_x_bytes(M);
   const bool producer = warp == kDecWarps;
   const int64_t u_begin = g.cta_unit[blockIdx.x], u_end = g.cta_unit[blockIdx.x + 1];
   // the segment starting at unit u: layer l, its first row block rb, R <= kDecMaxRb blocks
@@ -290,12 +295,12 @@ __global__ void __launch_bounds__(kDecBlockThreads, 1)
           uint8_t* st = ring + (gs % nst) * stb;
           uint64_t* bar = &full[gs % nst];
           const int kb0 = j * kDecSbBlocks;
-          mbar_expect_tx(bar, 16u * M * 128u + 4u * 16u * R * 128u);
+          mbar_expect_tx(bar, 128u * kDecSbBlocks * M + kDecGroups * 16u * R * 128u);
           tma_load_3d(st, &g.xmap[l], bar, 0, 0, kb0);
           if (L.w3d) {
             tma_load_3d(st + woff, wm, bar, 0, kb0 / 4, row0);
           } else {
-            for (int b = 0; b < 4; ++b)
+            for (int b = 0; b < kDecGroups; ++b)
               tma_load_2d(st + woff + b * (16u * R * 128u), wm, bar, kb0 * 32 + b * 128, row0);
           }
           ++gs;
@@ -330,6 +335,9 @@ __global__ void __launch_bounds__(kDecBlockThreads, 1)
     const int nkb = L.nkb;
     const int nsb = (nkb + kDecSbBlocks - 1) / kDecSbBlocks;
     const float mu = __ldg(L.mean);
+    const bool w3d = L.w3d != 0;
+    const uint8_t* __restrict__ code2 = L.code2;
+    const float* __restrict__ scale2 = L.scale2;
     // this segment's rows of B (bf16 [16R, r]) for its epilogue: asynchronous 16-byte
     // copies when the rows are 16-byte aligned (r a multiple of 8), else plain loads
     const int r = g.r;
@@ -349,20 +357,23 @@ __global__ void __launch_bounds__(kDecBlockThreads, 1)
     }
     // block constants (code2 byte, scale2) of rows lane + 32 c for this warp's block of
     // stage j, loaded one stage ahead of their use
+    // the block index of this lane's rows at block 0 (or -1 past the rows)
+    int64_t cblk[kCpl];
+#pragma unroll
+    for (int c = 0; c < kCpl; ++c) {
+      const int rr = lane + 32 * c;
+      cblk[c] = (rr < 16 * R && row0 + rr < N) ? (row0 + rr) * nkb + warp : -1;
+    }
     auto cload = [&](int j, uint32_t (&q)[kCpl], float (&sc)[kCpl]) {
-      const int kb = j * kDecSbBlocks + warp;
+      const bool live = j < nsb && j * kDecSbBlocks + warp < nkb;
 #pragma unroll
       for (int c = 0; c < kCpl; ++c) {
         q[c] = 0u;
         sc[c] = 0.f;
-        const int rr = lane + 32 * c;
-        const int64_t n = row0 + rr;
-        if (j < nsb && kb < nkb && rr < 16 * R && n < N) {
-          const int64_t blk = n * nkb + kb;
-          if (in_bounds((blk >> 8) < L.nb2, 71)) {
-            q[c] = L.code2[blk];
-            sc[c] = L.scale2[blk >> 8];
-          }
+        const int64_t blk = cblk[c] + j * kDecSbBlocks;
+        if (live && cblk[c] >= 0 && in_bounds((blk >> 8) < L.nb2, 71)) {
+          q[c] = code2[blk];
+          sc[c] = scale2[blk >> 8];
         }
       }
     };
@@ -380,10 +391,21 @@ __global__ void __launch_bounds__(kDecBlockThreads, 1)
     const uint32_t u0 = 2u * (warp & 3) + (t >> 1);
     // this warp's 32 packed bytes of row rr: 128-byte group warp / 4, pieces 2 (warp mod
     // 4) and + 1, swizzled by the 128-byte line: line = rr * 4 + group (3-D boxes) or
-    // group * 16R + rr (four 2-D boxes)
-    auto wline = [&](int rr) {
-      return L.w3d ? static_cast<uint32_t>(rr) * 4u + gg : gg * 16u * R + static_cast<uint32_t>(rr);
-    };
+    // group * 16R + rr (four 2-D boxes). Rows pg + 16 b (+ 8) share the line's swizzle
+    // key, so row block b sits at a fixed stride from row block 0.
+    const uint32_t la0 = w3d ? static_cast<uint32_t>(pg) * kDecGroups + gg : gg * 16u * R + static_cast<uint32_t>(pg);
+    const uint32_t woffa = woff + la0 * 128u + (((u0 ^ (la0 & 7u)) << 4) | ((t & 1) << 3));
+    const uint32_t bstride = w3d ? 16u * kDecGroups * 128u : 16u * 128u;  // bytes per row block
+    const uint32_t hstride = bstride / 2;                          // rows + 8
+    // token fragment offsets (rows g8, g8 + 8 of this warp's block, the last row past M)
+    uint32_t xoffa[Q], xoffb[Q];
+#pragma unroll
+    for (int q = 0; q < Q; ++q) {
+      const int tr = g8 + 8 * q < M ? g8 + 8 * q : M - 1;
+      const uint32_t rho = static_cast<uint32_t>(warp * M + tr);
+      xoffa[q] = rho * 128u + ((static_cast<uint32_t>(2 * t) ^ (rho & 7u)) << 4);
+      xoffb[q] = rho * 128u + ((static_cast<uint32_t>(2 * t + 1) ^ (rho & 7u)) << 4);
+    }
     for (int j = 0; j < nsb; ++j, ++gs) {
       if (ok) ok = warp_wait(&full[gs % nst], static_cast<uint32_t>((gs / nst) & 1), wait_ns, &s_abort, 61);
       if (!ok) continue;  // after a give-up no stage is released: the producer stops
@@ -418,19 +440,16 @@ __global__ void __launch_bounds__(kDecBlockThreads, 1)
       uint4 xa[Q], xb[Q];
 #pragma unroll
       for (int q = 0; q < Q; ++q) {
-        const int tr = g8 + 8 * q < M ? g8 + 8 * q : M - 1;
-        const uint32_t rho = static_cast<uint32_t>(warp * M + tr);
-        const uint32_t rowa = sb + rho * 128u;
-        xa[q] = lds_u4d(rowa + ((static_cast<uint32_t>(2 * t) ^ (rho & 7u)) << 4));
-        xb[q] = lds_u4d(rowa + ((static_cast<uint32_t>(2 * t + 1) ^ (rho & 7u)) << 4));
+        xa[q] = lds_u4d(sb + xoffa[q]);
+        xb[q] = lds_u4d(sb + xoffb[q]);
       }
+      const uint32_t wbase = sb + woffa;
       const float z[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int b = 0; b < kDecMaxRb; ++b) {
         if (b < R) {
-          const uint32_t la = wline(b * 16 + pg), lb = wline(b * 16 + 8 + pg);
-          const uint2 wa = lds_u2d(sb + woff + la * 128u + (((u0 ^ (la & 7u)) << 4) | ((t & 1) << 3)));
-          const uint2 wb = lds_u2d(sb + woff + lb * 128u + (((u0 ^ (lb & 7u)) << 4) | ((t & 1) << 3)));
+          const uint2 wa = lds_u2d(wbase + b * bstride);
+          const uint2 wb = lds_u2d(wbase + b * bstride + hstride);
           float d[Q][4];
 #pragma unroll
           for (int k4 = 0; k4 < 4; ++k4) {
