@@ -8,26 +8,30 @@
 //
 // At M <= 16 the layer is bound by the stream of packed weights (about 4.13 bits per
 // parameter), and every weight element is used by at most 16 tokens. The kernel gives
-// each warp its own weight tiles and tensor-core work, with no hand-off between warps:
+// each warp its own weight tiles and tensor-core work, with no hand-off between warps.
+// One launch serves 1 to 8 independent layers (the single-layer forward is n = 1):
 //
-// * Work: CTA p of P holds the 16-row blocks [p RB / P, (p + 1) RB / P) of the RB row
-//   blocks (at most kDecMaxRb), over the whole contraction, so no two CTAs share an
-//   output and the CTAs' byte counts differ by at most one row block. Its 16 warps
-//   split the 64-column blocks: warp w takes blocks w, w + 16, ... for all the CTA's
-//   rows, so each token fragment it loads serves every one of those rows.
-// * Loads: the CTA streams its rows through a ring of stages in shared memory (as many
-//   as fit, 2 to 4), one stage per 16 column blocks (1024 columns), each filled by TMA
-//   tile copies from a producer warp of its own (warp 16), which refills a stage as
-//   soon as the 16 compute warps have released it (an "empty" barrier per stage; no
+// * Work: the layers' 16-row blocks form one list of units; CTA p takes a contiguous run
+//   of units carrying about 1 / P of the packed bytes, and works through it in segments
+//   of at most kDecMaxRb blocks of one layer, each over that layer's whole contraction,
+//   so no two CTAs share an output. The 12 compute warps split the 64-column blocks of
+//   a segment: warp w takes blocks w, w + 12, ... for all the segment's rows, so each
+//   token fragment it loads serves every one of those rows.
+// * Loads: the CTA streams its segments through a ring of stages in shared memory (as
+//   many as fit, 2 to 4), one stage per 12 column blocks (768 columns), each filled by
+//   TMA tile copies from a producer warp of its own (warp 12), which refills a stage as
+//   soon as the 12 compute warps have released it (an "empty" barrier per stage; no
 //   CTA-wide barrier in the loop; the producer issues only after the CTA has set up its
 //   barriers, and leaves once everything is issued): the packed rows as one box of a
 //   3-D view [row][128-byte group][128 bytes] when K is a multiple of 256 (each row's
-//   512 bytes requested in order), else as four 128-byte-wide boxes, and the M token
+//   384 bytes requested in order), else as three 128-byte-wide boxes, and the M token
 //   rows as one box of a 3-D view of x, [column block][token row][64 columns]; every
 //   box uses the 128-byte swizzle. Warp w works on block w of the stage; token columns
 //   past M read row M - 1 (they only feed output columns that are never stored).
 // * Rows: within each 16-row block, mma row g reads packed row 2 (g mod 4) + g / 4 (and
 //   that + 8), which spreads a quarter warp's 8-byte reads over the swizzled pieces.
+//   Twelve compute warps (not 16) keep four warps per SM sub-partition, so each thread
+//   can hold 128 registers and keep more table lookups in flight.
 // * Math: mma.sync m16n8k16 (bf16 in, fp32 out) with the weight rows as the M side and
 //   the tokens as N. Within a block the contraction order is permuted, identically for
 //   both operands, so that thread t of a quad holds columns 16t .. 16t + 15: its weight
@@ -36,8 +40,9 @@
 //   its token fragment is 32 consecutive bytes of each of its token rows. The block's
 //   partial sums (unscaled levels) are multiplied by the block constant c in fp32 and
 //   added to the accumulator.
-// * Reduction: the 16 warps' accumulators are summed in shared memory in a fixed order;
-//   the epilogue adds s B u and writes bf16.
+// * Reduction: at the end of a segment the 12 warps' accumulators are summed in shared
+//   memory in a fixed order; the epilogue adds s B u and writes bf16. The producer keeps
+//   streaming the next segment meanwhile.
 // * Adapter: u = A x^T comes from k_lora_u, launched just before as the primary of a
 //   programmatic dependent launch: the main kernel streams its weights while u is
 //   computed, and waits for it (griddepcontrol.wait) only before its epilogue.
@@ -200,7 +205,7 @@ __global__ void __launch_bounds__(128) k_lora_u(const __grid_constant__ DecodeAr
   }
 }
 
-// barrier of the 16 compute warps only (the producer warp has left)
+// barrier of the compute warps only (the producer warp has left)
 QNF4_DEV void compute_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kDecThreads) : "memory"); }
 
 // 16-byte asynchronous copy global -> shared; src_bytes = 0 writes zeros and reads nothing
@@ -258,7 +263,7 @@ __global__ void __launch_bounds__(kDecBlockThreads, 1)
 
   if (producer) {
     // stream the CTA's segments: stage gs (a global count) goes into slot gs mod nst
-    // once the 16 compute warps have released that slot's previous use; then leave
+    // once the compute warps have released that slot's previous use; then leave
     if (lane == 0) {
       int64_t gs = 0;
       bool stop = false;
@@ -482,8 +487,8 @@ __global__ void __launch_bounds__(kDecBlockThreads, 1)
     if (!ok) break;
 
     // ---- segment end: u of this layer (once the adapter kernel has finished), the
-    // fixed-order sum of the 16 warps' partials (warp w adds into slot w % 4, warps 0-3
-    // first, then 4-7, 8-11, 12-15; slots [token][row], rows padded to kDecRedRow) ----
+    // fixed-order sum of the compute warps' partials (warp w adds into slot w % 4, warps 0-3
+    // first, then 4-7 and 8-11; slots [token][row], rows padded to kDecRedRow) ----
     if (!waited) {
       griddep_wait();
       waited = true;
