@@ -13,39 +13,46 @@
 //
 // * Work: the layers' 16-row blocks form one list of units; CTA p takes a contiguous run
 //   of units carrying about 1 / P of the packed bytes, and works through it in segments
-//   of at most kDecMaxRb blocks of one layer, each over that layer's whole contraction,
-//   so no two CTAs share an output. The 12 compute warps split the 64-column blocks of
-//   a segment: warp w takes blocks w, w + 12, ... for all the segment's rows, so each
-//   token fragment it loads serves every one of those rows.
+//   of at most 5 blocks of one layer (4 with two token groups, whose accumulators and
+//   token fragments are twice as many), each over that layer's whole contraction, so no
+//   two CTAs share an output. The 12 compute warps split the 64-column blocks of a
+//   segment: warp w takes blocks w, w + 12, ... for all the segment's rows, so each token
+//   fragment it loads serves every one of those rows. The row-block count of a segment is
+//   a compile-time constant of its loop (one instance per count), so the row blocks'
+//   table lookups interleave without branches.
 // * Loads: the CTA streams its segments through a ring of stages in shared memory (as
-//   many as fit, 2 to 4), one stage per 12 column blocks (768 columns), each filled by
-//   TMA tile copies from a producer warp of its own (warp 12), which refills a stage as
-//   soon as the 12 compute warps have released it (an "empty" barrier per stage; no
-//   CTA-wide barrier in the loop; the producer issues only after the CTA has set up its
-//   barriers, and leaves once everything is issued): the packed rows as one box of a
-//   3-D view [row][128-byte group][128 bytes] when K is a multiple of 256 (each row's
-//   384 bytes requested in order), else as three 128-byte-wide boxes, and the M token
-//   rows as one box of a 3-D view of x, [column block][token row][64 columns]; every
-//   box uses the 128-byte swizzle. Warp w works on block w of the stage; token columns
-//   past M read row M - 1 (they only feed output columns that are never stored).
+//   many as fit, 2 to 4), one stage per 12 column blocks (768 columns). Two producer
+//   warps walk the same stages and refill a slot as soon as the 12 compute warps have
+//   released it (an "empty" barrier per stage; no CTA-wide barrier in the loop). Warp 12
+//   issues the TMA tile copies: the packed rows as one box of a 3-D view [row][128-byte
+//   group][128 bytes] when K is a multiple of 256 (each row's 384 bytes requested in
+//   order), else as three 128-byte-wide boxes, and the M token rows as one box of a 3-D
+//   view of x, [column block][token row][64 columns]; every box uses the 128-byte
+//   swizzle. Warp 13 copies the stage's block constants (per row, the code2 bytes of its
+//   12 blocks and the two scale2 words they can use) with 4-byte asynchronous copies and
+//   arrives on the stage's barrier when they land, so the tile copies never queue behind
+//   those small ones. Warp w works on block w of the stage; token columns past M read
+//   row M - 1 (they only feed output columns that are never stored).
 // * Rows: within each 16-row block, mma row g reads packed row 2 (g mod 4) + g / 4 (and
 //   that + 8), which spreads a quarter warp's 8-byte reads over the swizzled pieces.
-//   Twelve compute warps (not 16) keep four warps per SM sub-partition, so each thread
-//   can hold 128 registers and keep more table lookups in flight.
+//   Twelve compute warps (not 16) keep at most four warps per SM sub-partition, so each
+//   thread can hold 128 registers and keep more table lookups in flight.
 // * Math: mma.sync m16n8k16 (bf16 in, fp32 out) with the weight rows as the M side and
 //   the tokens as N. Within a block the contraction order is permuted, identically for
 //   both operands, so that thread t of a quad holds columns 16t .. 16t + 15: its weight
 //   fragment is 8 consecutive packed bytes of each of its two rows, turned into bf16
 //   pairs by a 256-entry table (one copy per lane, so the lookups never conflict), and
 //   its token fragment is 32 consecutive bytes of each of its token rows. The block's
-//   partial sums (unscaled levels) are multiplied by the block constant c in fp32 and
-//   added to the accumulator.
+//   partial sums (unscaled levels) are multiplied by the block constant c (computed per
+//   stage from the staged code2 and scale2) in fp32 and added to the accumulator.
 // * Reduction: at the end of a segment the 12 warps' accumulators are summed in shared
-//   memory in a fixed order; the epilogue adds s B u and writes bf16. The producer keeps
-//   streaming the next segment meanwhile.
+//   memory in a fixed order and written as bf16. Warp 0 first adds the adapter term
+//   s B u to its accumulators with the same tensor-core instruction (B rows and bf16 s u
+//   in shared memory, the rank padded to a multiple of 16 with zeros). The producers
+//   keep streaming the next segment meanwhile.
 // * Adapter: u = A x^T comes from k_lora_u, launched just before as the primary of a
 //   programmatic dependent launch: the main kernel streams its weights while u is
-//   computed, and waits for it (griddepcontrol.wait) only before its epilogue.
+//   computed, and waits for it (griddepcontrol.wait) only before its first epilogue.
 #pragma once
 #include "common.cuh"
 
@@ -53,7 +60,7 @@ namespace qnf4 {
 
 constexpr int kDecWarps = 12;                  // compute warps
 constexpr int kDecThreads = 32 * kDecWarps;
-constexpr int kDecBlockThreads = kDecThreads + 32;  // plus the producer warp
+constexpr int kDecBlockThreads = kDecThreads + 64;  // plus the two producer warps
 constexpr int kDecMaxRb = 5;      // 16-row blocks a CTA holds at most
 constexpr int kDecMaxRows = 16 * kDecMaxRb;
 constexpr int kDecMaxStages = 4;
@@ -66,18 +73,29 @@ constexpr int kDecRedSlots = 4;
 constexpr int kDecRedRow = 84;   // floats per token row of a reduction slot (padded)
 constexpr uint32_t kDecLutBytes = 256u * kDecLutCopies * 4u;                 // 32 KB
 constexpr uint32_t kDecRedBytes = kDecRedSlots * 16u * kDecRedRow * 4u;      // 21 KB
-constexpr uint32_t kDecCsBytes = kDecWarps * kDecMaxRows * 4u;               // 5 KB
+constexpr uint32_t kDecCsBytes = kDecWarps * kDecMaxRows * 4u;               // 4 KB
 constexpr uint32_t kDecBsBytes = kDecMaxRows * 64u * 2u;                     // 10 KB: B rows, r <= 64
-constexpr uint32_t kDecUsBytes = 64u * 16u * 4u;                             // 4 KB: u [r][M]
+constexpr uint32_t kDecUsBytes = 16u * 64u * 2u;                             // 2 KB: bf16 s u [token][r]
 constexpr size_t kDecSmem =
     1024 + kDecRingBytes + kDecLutBytes + kDecCsBytes + kDecBsBytes + kDecRedBytes + kDecUsBytes;
-// stage = the token box (kDecSbBlocks blocks x M rows x 128 B), then the packed rows
-// (kDecGroups x 16R rows x 128 B); both start on a 1024-byte boundary (the swizzle's)
+// Block constants of a stage, copied by the producer warp: for each of the 16R rows the
+// 16 code2 bytes from its first block's byte rounded down to 4 (the stage's 12 blocks lie
+// inside), then the two scale2 words its 12 blocks can fall into.
+constexpr uint32_t kDecCodeRow = 16u;
+constexpr uint32_t kDecCstScale = kDecMaxRows * kDecCodeRow;                 // 1280
+constexpr uint32_t kDecCstBytes = 2048u;
+static_assert(kDecCstScale + kDecMaxRows * 8u <= kDecCstBytes, "constants area");
+// stage = the token box (kDecSbBlocks blocks x M rows x 128 B), the packed rows
+// (kDecGroups x 16R rows x 128 B), then the block constants; the boxes start on a
+// 1024-byte boundary (the swizzle's)
 __host__ __device__ constexpr uint32_t dec_x_bytes(int M) {
   return (128u * kDecSbBlocks * M + 1023u) & ~1023u;
 }
+__host__ __device__ constexpr uint32_t dec_w_bytes(int R) {
+  return (2048u * kDecGroups * R + 1023u) & ~1023u;
+}
 __host__ __device__ constexpr uint32_t dec_stage_bytes(int R, int M) {
-  return dec_x_bytes(M) + ((2048u * kDecGroups * R + 1023u) & ~1023u);
+  return dec_x_bytes(M) + dec_w_bytes(R) + kDecCstBytes;
 }
 __host__ __device__ constexpr int dec_stages(int R, int M) {
   return static_cast<int>(kDecRingBytes / dec_stage_bytes(R, M)) < kDecMaxStages
@@ -213,8 +231,33 @@ QNF4_DEV void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
                : "memory");
 }
+// 4-byte asynchronous copy global -> shared of src_bytes (0..4) bytes, the rest zeros
+QNF4_DEV void cp_async4(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+               : "memory");
+}
 QNF4_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 QNF4_DEV void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+// one arrival on the barrier once this thread's earlier cp.async copies have landed
+// (counted among the barrier's expected arrivals)
+QNF4_DEV void cp_async_mbar_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+QNF4_DEV uint32_t lds_u8d(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u8 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+QNF4_DEV float lds_f32d(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+  return v;
+}
+
+template <int V>
+struct DecRows {
+  static constexpr int value = V;
+};
 
 // Q token groups of 8 (Q = 1: M <= 8; Q = 2: M <= 16).
 template <int Q>
@@ -231,30 +274,34 @@ __global__ void __launch_bounds__(kDecBlockThreads, 1)
   float* cs_all = reinterpret_cast<float*>(base + kDecRingBytes + kDecLutBytes);
   uint16_t* bs = reinterpret_cast<uint16_t*>(base + kDecRingBytes + kDecLutBytes + kDecCsBytes);
   float* red = reinterpret_cast<float*>(base + kDecRingBytes + kDecLutBytes + kDecCsBytes + kDecBsBytes);
-  float* us = red + kDecRedBytes / 4;
+  uint16_t* us = reinterpret_cast<uint16_t*>(red + kDecRedBytes / 4);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g8 = lane >> 2, t = lane & 3;
   const int pg = 2 * (g8 & 3) + (g8 >> 2);  // packed row of mma row g8 within 8
   const int M = g.M;
-  const uint32_t stb = dec_stage_bytes(kDecMaxRb, M);
-  const int nst = dec_stages(kDecMaxRb, M);
+  // row blocks per segment: two token groups keep fewer (their accumulators and token
+  // fragments are twice as many), which also leaves room for a third stage
+  constexpr int kRb = Q == 2 ? 4 : kDecMaxRb;
+  const uint32_t stb = dec_stage_bytes(kRb, M);
+  const int nst = dec_stages(kRb, M);
   const uint32_t woff = dec_x_bytes(M);
-  const bool producer = warp == kDecWarps;
+  const uint32_t coff = woff + dec_w_bytes(kRb);  // block constants of a stage
+  const bool producer = warp >= kDecWarps;
   const int64_t u_begin = g.cta_unit[blockIdx.x], u_end = g.cta_unit[blockIdx.x + 1];
-  // the segment starting at unit u: layer l, its first row block rb, R <= kDecMaxRb blocks
+  // the segment starting at unit u: layer l, its first row block rb, R <= kRb blocks
   auto seg_of = [&](int64_t u, int& l, int64_t& rb, int& R) {
     l = 0;
     while (l + 1 < g.n && g.L[l + 1].unit0 <= u) ++l;
     rb = u - g.L[l].unit0;
     const int64_t lend = l + 1 < g.n ? g.L[l + 1].unit0 : g.units;
     const int64_t e = u_end < lend ? u_end : lend;
-    R = static_cast<int>(e - u < kDecMaxRb ? e - u : kDecMaxRb);
+    R = static_cast<int>(e - u < kRb ? e - u : kRb);
   };
   if (tid == 0) {
     s_abort = 0;
     s_issued = -1;
     for (int i = 0; i < kDecMaxStages; ++i) {
-      mbar_init(&full[i], 1);
+      mbar_init(&full[i], 1 + 32);  // the TMA transaction + the producer lanes' copies
       mbar_init(&empty[i], kDecWarps);
     }
     fence_mbar_init();
@@ -263,43 +310,43 @@ __global__ void __launch_bounds__(kDecBlockThreads, 1)
 
   if (producer) {
     // stream the CTA's segments: stage gs (a global count) goes into slot gs mod nst
-    // once the compute warps have released that slot's previous use; then leave
-    if (lane == 0) {
-      int64_t gs = 0;
-      bool stop = false;
-      for (int64_t u = u_begin; u < u_end && !stop;) {
-        int l, R;
-        int64_t rb;
-        seg_of(u, l, rb, R);
-        const DecLayer& L = g.L[l];
-        const CUtensorMap* wm = &g.wmap[l][R - 1];
-        const int nsb = (L.nkb + kDecSbBlocks - 1) / kDecSbBlocks;
-        const int32_t row0 = static_cast<int32_t>(rb * 16);
-        for (int j = 0; j < nsb; ++j) {
-          if (gs >= nst) {
-            const long long t0 = wait_clock();
-            while (!mbar_try_wait(&empty[gs % nst], static_cast<uint32_t>((gs / nst - 1) & 1))) {
-              if (s_abort) {
-                stop = true;
-                break;
-              }
-              if (wait_clock() - t0 > ns_cycles(wait_ns)) {
-                set_err(63);
-                s_abort = 1;
-                stop = true;
-                break;
-              }
-            }
-            if (stop) break;
-            fence_proxy_async();
-          }
-          if (s_abort) {
+    // once the compute warps have released that slot's previous use. Both producer warps
+    // walk the same stages: lane 0 of warp 12 issues the tile copies, the lanes of warp
+    // 13 copy the block constants and arrive on the stage's barrier when they have
+    // landed (so the tile copies never queue behind the many small ones).
+    const bool tma_warp = warp == kDecWarps;
+    int64_t gs = 0;
+    bool stop = false;
+    for (int64_t u = u_begin; u < u_end && !stop;) {
+      int l, R;
+      int64_t rb;
+      seg_of(u, l, rb, R);
+      const DecLayer& L = g.L[l];
+      const CUtensorMap* wm = &g.wmap[l][R - 1];
+      const int nkb = L.nkb;
+      const int nsb = (nkb + kDecSbBlocks - 1) / kDecSbBlocks;
+      const int32_t row0 = static_cast<int32_t>(rb * 16);
+      const int64_t c2len = L.N * nkb;  // code2 bytes
+      int64_t crow[(kDecMaxRows + 31) / 32];  // block index of this lane's rows at column 0
+#pragma unroll
+      for (int c = 0; c < (kDecMaxRows + 31) / 32; ++c) crow[c] = (row0 + lane + 32 * c) * static_cast<int64_t>(nkb);
+      for (int j = 0; j < nsb; ++j) {
+        const int slot = static_cast<int>(gs % nst);
+        if (gs >= nst) {
+          if (!warp_wait(&empty[slot], static_cast<uint32_t>((gs / nst - 1) & 1), wait_ns, &s_abort, 63)) {
             stop = true;
             break;
           }
-          uint8_t* st = ring + (gs % nst) * stb;
-          uint64_t* bar = &full[gs % nst];
-          const int kb0 = j * kDecSbBlocks;
+          fence_proxy_async();
+        }
+        if (__shfl_sync(0xffffffffu, s_abort, 0)) {
+          stop = true;
+          break;
+        }
+        uint8_t* st = ring + slot * stb;
+        uint64_t* bar = &full[slot];
+        const int kb0 = j * kDecSbBlocks;
+        if (tma_warp && lane == 0) {
           mbar_expect_tx(bar, 128u * kDecSbBlocks * M + kDecGroups * 16u * R * 128u);
           tma_load_3d(st, &g.xmap[l], bar, 0, 0, kb0);
           if (L.w3d) {
@@ -308,12 +355,43 @@ __global__ void __launch_bounds__(kDecBlockThreads, 1)
             for (int b = 0; b < kDecGroups; ++b)
               tma_load_2d(st + woff + b * (16u * R * 128u), wm, bar, kb0 * 32 + b * 128, row0);
           }
-          ++gs;
         }
-        u += R;
+        if (!tma_warp) {
+          // block constants: lane handles rows lane + 32 c: 4 code2 words from the row's
+          // first block rounded down to 4 bytes (the last word of code2 may be partial), then
+          // scale2 words s0 and s0 + 1
+          const uint32_t cdst = smem_u32(st + coff);
+#pragma unroll
+          for (int c = 0; c < (kDecMaxRows + 31) / 32; ++c) {
+            const int rr = lane + 32 * c;
+            if (rr < 16 * R) {
+              const bool live = row0 + rr < L.N;
+              const int64_t a = crow[c] + kb0;
+              const int64_t w0 = a & ~static_cast<int64_t>(3);
+              const int64_t left = live ? c2len - w0 : 0;
+              const uint32_t d = cdst + rr * kDecCodeRow;
+#pragma unroll
+              for (int v = 0; v < 4; ++v) {
+                const int64_t lv = left - 4 * v;
+                const uint32_t nb = lv >= 4 ? 4u : (lv > 0 ? static_cast<uint32_t>(lv) : 0u);
+                cp_async4(d + 4 * v, nb ? L.code2 + w0 + 4 * v : L.code2, nb);
+              }
+              const int64_t s0 = a >> 8;
+              const uint32_t ds = cdst + kDecCstScale + rr * 8;
+              cp_async4(ds, live ? L.scale2 + s0 : L.scale2, live ? 4u : 0u);
+              const bool ok1 = live && s0 + 1 < L.nb2;
+              cp_async4(ds + 4, ok1 ? L.scale2 + s0 + 1 : L.scale2, ok1 ? 4u : 0u);
+              in_bounds(!live || (w0 >= 0 && s0 < L.nb2), 75);
+            }
+          }
+          cp_async_mbar_arrive(bar);
+        }
+        ++gs;
       }
-      s_issued = static_cast<int>(gs);
+      u += R;
     }
+    if (tma_warp && lane == 0) s_issued = static_cast<int>(gs);
+    cp_async_wait_all();
     return;
   }
 
@@ -327,67 +405,48 @@ __global__ void __launch_bounds__(kDecBlockThreads, 1)
   const uint32_t lutb = smem_u32(lut) + lane * 4u;
   float* cs = cs_all + warp * kDecMaxRows;
   constexpr int kCpl = (kDecMaxRows + 31) / 32;  // rows per lane for the block constants
+  const int r = g.r;
+  const int r16 = (r + 15) & ~15;  // the adapter's contraction, padded with zeros
   bool ok = true, waited = false;
-  int ul = -1;  // layer whose u is in us
+  int ul = -1;  // layer whose s u is in us
   int64_t gs = 0;
-  for (int64_t u = u_begin; u < u_end;) {
-    int l, R;
-    int64_t rb;
-    seg_of(u, l, rb, R);
-    u += R;
+  // one segment of R row blocks (R a compile-time constant, so the row-block loops
+  // unroll without branches and their table lookups interleave)
+  auto segment = [&](auto Rc, int l, int64_t rb) {
+    constexpr int R = decltype(Rc)::value;
     const DecLayer& L = g.L[l];
     const int64_t row0 = rb * 16, N = L.N;
     const int nkb = L.nkb;
     const int nsb = (nkb + kDecSbBlocks - 1) / kDecSbBlocks;
     const float mu = __ldg(L.mean);
     const bool w3d = L.w3d != 0;
-    const uint8_t* __restrict__ code2 = L.code2;
-    const float* __restrict__ scale2 = L.scale2;
-    // this segment's rows of B (bf16 [16R, r]) for its epilogue: asynchronous 16-byte
-    // copies when the rows are 16-byte aligned (r a multiple of 8), else plain loads
-    const int r = g.r;
+    // this segment's rows of B as bf16 [16R][r16] (zero past r and past N) for the
+    // adapter product: 16-byte asynchronous copies when rows are 16-byte aligned
     if ((r & 7) == 0) {
-      const int np = 16 * R * r / 8;
-      for (int i = tid; i < np; i += kDecThreads) {
-        const int64_t n = row0 + (i * 8) / r;
-        const bool in = n < N;
-        cp_async16(smem_u32(bs + i * 8), in ? L.Bm + row0 * r + i * 8 : L.Bm, in ? 16u : 0u);
+      const int pr = r16 / 8;
+      for (int i = tid; i < 16 * R * pr; i += kDecThreads) {
+        const int rl = i / pr, p = i - pr * (i / pr);
+        const int64_t n = row0 + rl;
+        const bool in = n < N && 8 * p < r;
+        cp_async16(smem_u32(bs + rl * r16 + 8 * p), in ? L.Bm + n * r + 8 * p : L.Bm, in ? 16u : 0u);
       }
       cp_async_commit();
     } else {
-      for (int i = tid; i < 16 * R * r; i += kDecThreads) {
-        const int64_t n = row0 + i / r;
-        bs[i] = n < N ? L.Bm[n * r + i % r] : static_cast<uint16_t>(0);
+      for (int i = tid; i < 16 * R * r16; i += kDecThreads) {
+        const int rl = i / r16, jj = i - r16 * (i / r16);
+        const int64_t n = row0 + rl;
+        bs[i] = (n < N && jj < r) ? L.Bm[n * r + jj] : static_cast<uint16_t>(0);
       }
     }
-    // block constants (code2 byte, scale2) of rows lane + 32 c for this warp's block of
-    // stage j, loaded one stage ahead of their use
-    // the block index of this lane's rows at block 0 (or -1 past the rows)
-    int64_t cblk[kCpl];
+    // low 8 bits of the block index of this lane's rows (lane + 32 c) at column 0: they
+    // give, per stage, the row's byte in the staged code2 window and its scale2 word
+    uint32_t alo[kCpl];
 #pragma unroll
-    for (int c = 0; c < kCpl; ++c) {
-      const int rr = lane + 32 * c;
-      cblk[c] = (rr < 16 * R && row0 + rr < N) ? (row0 + rr) * nkb + warp : -1;
-    }
-    auto cload = [&](int j, uint32_t (&q)[kCpl], float (&sc)[kCpl]) {
-      const bool live = j < nsb && j * kDecSbBlocks + warp < nkb;
+    for (int c = 0; c < kCpl; ++c)
+      alo[c] = static_cast<uint32_t>(((row0 + lane + 32 * c) * nkb) & 255);
+    float acc[R][Q][4];
 #pragma unroll
-      for (int c = 0; c < kCpl; ++c) {
-        q[c] = 0u;
-        sc[c] = 0.f;
-        const int64_t blk = cblk[c] + j * kDecSbBlocks;
-        if (live && cblk[c] >= 0 && in_bounds((blk >> 8) < L.nb2, 71)) {
-          q[c] = code2[blk];
-          sc[c] = scale2[blk >> 8];
-        }
-      }
-    };
-    uint32_t pq[kCpl];
-    float psc[kCpl];
-    cload(0, pq, psc);
-    float acc[kDecMaxRb][Q][4];
-#pragma unroll
-    for (int b = 0; b < kDecMaxRb; ++b)
+    for (int b = 0; b < R; ++b)
 #pragma unroll
       for (int q = 0; q < Q; ++q)
 #pragma unroll
@@ -421,21 +480,24 @@ __global__ void __launch_bounds__(kDecBlockThreads, 1)
         continue;
       }
       const uint32_t sb = smem_u32(ring + (gs % nst) * stb);
-      // c of the segment's rows for block kb, exchanged through the warp's scratch:
-      // packed row rr at word (rr mod 8) * 2 kDecMaxRb + rr / 8, so thread (g8, t) reads
-      // its rows pg + 8 i at pg * 2 kDecMaxRb + i
+      // c of the segment's rows for block kb from the staged constants, exchanged through
+      // the warp's scratch: packed row rr at word (rr mod 8) * 2 kDecMaxRb + rr / 8, so
+      // thread (g8, t) reads its rows pg + 8 i at pg * 2 kDecMaxRb + i
+      const uint32_t cst = sb + coff;
 #pragma unroll
       for (int c = 0; c < kCpl; ++c) {
         const int rr = lane + 32 * c;
-        if (rr < kDecMaxRows)
-          cs[(rr & 7) * (2 * kDecMaxRb) + (rr >> 3)] =
-              fmaf(e4m3_to_f32(static_cast<uint8_t>(pq[c])), psc[c], mu);
+        if (rr < 16 * R) {
+          const uint32_t a = (alo[c] + static_cast<uint32_t>(j * kDecSbBlocks)) & 255u;
+          const uint32_t code = lds_u8d(cst + rr * kDecCodeRow + (a & 3u) + warp);
+          const float s2 = lds_f32d(cst + kDecCstScale + rr * 8 + (((a + warp) >> 8) << 2));
+          cs[(rr & 7) * (2 * kDecMaxRb) + (rr >> 3)] = fmaf(e4m3_to_f32(static_cast<uint8_t>(code)), s2, mu);
+        }
       }
-      cload(j + 1, pq, psc);  // the next stage's constants land while the tensor cores work
       __syncwarp();
-      float ch[2 * kDecMaxRb];
+      float ch[2 * R];
 #pragma unroll
-      for (int i = 0; i < kDecMaxRb; ++i) {
+      for (int i = 0; i < R; ++i) {
         const float2 v = *reinterpret_cast<const float2*>(cs + pg * (2 * kDecMaxRb) + 2 * i);
         ch[2 * i] = v.x;
         ch[2 * i + 1] = v.y;
@@ -451,134 +513,145 @@ __global__ void __launch_bounds__(kDecBlockThreads, 1)
       const uint32_t wbase = sb + woffa;
       const float z[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int b = 0; b < kDecMaxRb; ++b) {
-        if (b < R) {
-          const uint2 wa = lds_u2d(wbase + b * bstride);
-          const uint2 wb = lds_u2d(wbase + b * bstride + hstride);
-          float d[Q][4];
+      for (int b = 0; b < R; ++b) {
+        const uint2 wa = lds_u2d(wbase + b * bstride);
+        const uint2 wb = lds_u2d(wbase + b * bstride + hstride);
+        float d[Q][4];
 #pragma unroll
-          for (int k4 = 0; k4 < 4; ++k4) {
-            const uint32_t wlo = k4 < 2 ? wa.x : wa.y, whi = k4 < 2 ? wb.x : wb.y;
-            const int i0 = (2 * k4) & 3;
-            const uint32_t a0 = lut_pair(lutb, wlo, i0), a2 = lut_pair(lutb, wlo, i0 + 1);
-            const uint32_t a1 = lut_pair(lutb, whi, i0), a3 = lut_pair(lutb, whi, i0 + 1);
-#pragma unroll
-            for (int q = 0; q < Q; ++q) {
-              const uint4& xv = k4 < 2 ? xa[q] : xb[q];
-              const uint32_t b0 = (k4 & 1) ? xv.z : xv.x, b1 = (k4 & 1) ? xv.w : xv.y;
-              if (k4 == 0)
-                mma_bf16_16816(d[q], a0, a1, a2, a3, b0, b1, z);
-              else
-                mma_bf16_16816(d[q], a0, a1, a2, a3, b0, b1, d[q]);
-            }
-          }
+        for (int k4 = 0; k4 < 4; ++k4) {
+          const uint32_t wlo = k4 < 2 ? wa.x : wa.y, whi = k4 < 2 ? wb.x : wb.y;
+          const int i0 = (2 * k4) & 3;
+          const uint32_t a0 = lut_pair(lutb, wlo, i0), a2 = lut_pair(lutb, wlo, i0 + 1);
+          const uint32_t a1 = lut_pair(lutb, whi, i0), a3 = lut_pair(lutb, whi, i0 + 1);
 #pragma unroll
           for (int q = 0; q < Q; ++q) {
-            acc[b][q][0] = fmaf(ch[2 * b], d[q][0], acc[b][q][0]);
-            acc[b][q][1] = fmaf(ch[2 * b], d[q][1], acc[b][q][1]);
-            acc[b][q][2] = fmaf(ch[2 * b + 1], d[q][2], acc[b][q][2]);
-            acc[b][q][3] = fmaf(ch[2 * b + 1], d[q][3], acc[b][q][3]);
+            const uint4& xv = k4 < 2 ? xa[q] : xb[q];
+            const uint32_t b0 = (k4 & 1) ? xv.z : xv.x, b1 = (k4 & 1) ? xv.w : xv.y;
+            if (k4 == 0)
+              mma_bf16_16816(d[q], a0, a1, a2, a3, b0, b1, z);
+            else
+              mma_bf16_16816(d[q], a0, a1, a2, a3, b0, b1, d[q]);
           }
+        }
+#pragma unroll
+        for (int q = 0; q < Q; ++q) {
+          acc[b][q][0] = fmaf(ch[2 * b], d[q][0], acc[b][q][0]);
+          acc[b][q][1] = fmaf(ch[2 * b], d[q][1], acc[b][q][1]);
+          acc[b][q][2] = fmaf(ch[2 * b + 1], d[q][2], acc[b][q][2]);
+          acc[b][q][3] = fmaf(ch[2 * b + 1], d[q][3], acc[b][q][3]);
         }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[gs % nst]);  // this warp is done with the stage
     }
-    if (!ok) break;
+    if (!ok) return;
 
-    // ---- segment end: u of this layer (once the adapter kernel has finished), the
-    // fixed-order sum of the compute warps' partials (warp w adds into slot w % 4, warps 0-3
-    // first, then 4-7 and 8-11; slots [token][row], rows padded to kDecRedRow) ----
+    // ---- segment end: s u of this layer as bf16 [token][r16] (once the adapter kernel
+    // has finished; partials summed in a fixed order), then the fixed-order sum of the
+    // compute warps' partials (warp w adds into slot w % 4, warps 0-3 first, then 4-7
+    // and 8-11; slots [token][row], rows padded to kDecRedRow). Warp 0 first adds the
+    // adapter term s B u to its accumulators with the tensor cores. ----
     if (!waited) {
       griddep_wait();
       waited = true;
     }
-    const int nu = r * M;
-    const bool newu = l != ul;
-    float up[kDecMaxUParts / 4];
-    if (newu) {
+    if (l != ul) {
+      const int nu = r * M;
+      for (int i = tid; i < 16 * r16; i += kDecThreads) {
+        const int m = i / r16, jj = i - r16 * (i / r16);
+        float v = 0.f;
+        if (m < M && jj < r) {
+          const float* p = L.upart + jj * M + m;
+          constexpr int kPre = 8;  // partials loaded together
+          for (int c0 = 0; c0 < L.ks; c0 += kPre) {
+            float up[kPre];
 #pragma unroll
-      for (int c = 0; c < kDecMaxUParts / 4; ++c)
-        up[c] = (tid < nu && c < L.ks) ? __ldcg(L.upart + static_cast<int64_t>(c) * nu + tid) : 0.f;
+            for (int c = 0; c < kPre; ++c)
+              up[c] = c0 + c < L.ks ? __ldcg(p + static_cast<int64_t>(c0 + c) * nu) : 0.f;
+#pragma unroll
+            for (int c = 0; c < kPre; ++c)
+              if (c0 + c < L.ks) v += up[c];
+          }
+        }
+        us[i] = static_cast<uint16_t>(pack_bf16x2(g.scale * v, 0.f) & 0xFFFFu);
+      }
+      ul = l;
+    }
+    cp_async_wait_all();  // the B rows
+    compute_sync();
+    if (warp == 0) {
+      const uint32_t bsa = smem_u32(bs), usa = smem_u32(us);
+      for (int kc = 0; kc < r16; kc += 16) {
+        uint32_t bu[Q][2];
+#pragma unroll
+        for (int q = 0; q < Q; ++q) {
+          const uint32_t o = ((8 * q + g8) * r16 + kc + 2 * t) * 2;
+          bu[q][0] = lds_u32d(usa + o);
+          bu[q][1] = lds_u32d(usa + o + 16);
+        }
+#pragma unroll
+        for (int b = 0; b < R; ++b) {
+          const uint32_t o0 = ((b * 16 + pg) * r16 + kc + 2 * t) * 2;
+          const uint32_t o1 = o0 + 8 * r16 * 2;
+          const uint32_t a0 = lds_u32d(bsa + o0), a2 = lds_u32d(bsa + o0 + 16);
+          const uint32_t a1 = lds_u32d(bsa + o1), a3 = lds_u32d(bsa + o1 + 16);
+#pragma unroll
+          for (int q = 0; q < Q; ++q) mma_bf16_16816(acc[b][q], a0, a1, a2, a3, bu[q][0], bu[q][1], acc[b][q]);
+        }
+      }
     }
     float* slot = red + (warp % kDecRedSlots) * (16 * kDecRedRow);
 #pragma unroll
     for (int round = 0; round < kDecWarps / kDecRedSlots; ++round) {
       if (warp / kDecRedSlots == round) {
 #pragma unroll
-        for (int b = 0; b < kDecMaxRb; ++b) {
-          if (b < R) {
+        for (int b = 0; b < R; ++b) {
 #pragma unroll
-            for (int q = 0; q < Q; ++q) {
-              const int rw = b * 16 + pg, tk = 8 * q + 2 * t;  // the packed row of mma row g8
-              float* p = slot + tk * kDecRedRow + rw;
-              if (round == 0) {
-                p[0] = acc[b][q][0];
-                p[kDecRedRow] = acc[b][q][1];
-                p[8] = acc[b][q][2];
-                p[kDecRedRow + 8] = acc[b][q][3];
-              } else {
-                p[0] += acc[b][q][0];
-                p[kDecRedRow] += acc[b][q][1];
-                p[8] += acc[b][q][2];
-                p[kDecRedRow + 8] += acc[b][q][3];
-              }
+          for (int q = 0; q < Q; ++q) {
+            const int rw = b * 16 + pg, tk = 8 * q + 2 * t;  // the packed row of mma row g8
+            float* p = slot + tk * kDecRedRow + rw;
+            if (round == 0) {
+              p[0] = acc[b][q][0];
+              p[kDecRedRow] = acc[b][q][1];
+              p[8] = acc[b][q][2];
+              p[kDecRedRow + 8] = acc[b][q][3];
+            } else {
+              p[0] += acc[b][q][0];
+              p[kDecRedRow] += acc[b][q][1];
+              p[8] += acc[b][q][2];
+              p[kDecRedRow + 8] += acc[b][q][3];
             }
           }
         }
       }
       compute_sync();
     }
-    if (newu) {
-      for (int i = tid; i < nu; i += kDecThreads) {
-        float v = 0.f;
-        if (i == tid) {
-#pragma unroll
-          for (int c = 0; c < kDecMaxUParts / 4; ++c) v += up[c];
-        } else {
-          for (int c = 0; c < kDecMaxUParts / 4 && c < L.ks; ++c)
-            v += __ldcg(L.upart + static_cast<int64_t>(c) * nu + i);
-        }
-        for (int c = kDecMaxUParts / 4; c < L.ks; ++c) v += __ldcg(L.upart + static_cast<int64_t>(c) * nu + i);
-        us[i] = v;
-      }
-      ul = l;
-    }
-    cp_async_wait_all();  // the B rows
-    compute_sync();
-    // outputs o = m * 16 R + row: h[m, row0 + row] = sum of the slots + s B u
-    const int nrows = 16 * R;
-    const int nout = nrows * M;
-    for (int o = tid; o < nout; o += kDecThreads) {
+    // outputs o = m * 16 R + row: h[m, row0 + row] = the slots' sum
+    constexpr int nrows = 16 * R;
+    for (int o = tid; o < nrows * M; o += kDecThreads) {
       const int rl = o % nrows, m = o / nrows;
       const int64_t n = row0 + rl;
       if (n >= N) continue;
-      float v = 0.f;
-#pragma unroll
-      for (int sl = 0; sl < kDecRedSlots; ++sl) v += red[sl * (16 * kDecRedRow) + m * kDecRedRow + rl];
-      const uint16_t* brow = bs + rl * r;
-      float lr = 0.f;
-      if ((r & 7) == 0) {
-        for (int j = 0; j < r; j += 8) {
-          const uint4 bv = *reinterpret_cast<const uint4*>(brow + j);
-          const float* uj = us + j * M + m;
-          lr = fmaf(bf16lo(bv.x), uj[0], lr);
-          lr = fmaf(bf16hi(bv.x), uj[M], lr);
-          lr = fmaf(bf16lo(bv.y), uj[2 * M], lr);
-          lr = fmaf(bf16hi(bv.y), uj[3 * M], lr);
-          lr = fmaf(bf16lo(bv.z), uj[4 * M], lr);
-          lr = fmaf(bf16hi(bv.z), uj[5 * M], lr);
-          lr = fmaf(bf16lo(bv.w), uj[6 * M], lr);
-          lr = fmaf(bf16hi(bv.w), uj[7 * M], lr);
-        }
-      } else {
-        for (int j = 0; j < r; ++j) lr = fmaf(bf16lo(brow[j]), us[j * M + m], lr);
-      }
-      const float out = fmaf(g.scale, lr, v);
+      const float* p = red + m * kDecRedRow + rl;
+      const float v = ((p[0] + p[16 * kDecRedRow]) + p[2 * 16 * kDecRedRow]) + p[3 * 16 * kDecRedRow];
       if (in_bounds(m < M, 74))
-        L.h[static_cast<int64_t>(m) * N + n] = static_cast<uint16_t>(pack_bf16x2(out, 0.f) & 0xFFFFu);
+        L.h[static_cast<int64_t>(m) * N + n] = static_cast<uint16_t>(pack_bf16x2(v, 0.f) & 0xFFFFu);
     }
     compute_sync();  // red, us and bs are reused by the next segment
+  };
+  static_assert(kDecMaxRb == 5 && kDecRedSlots == 4, "segment dispatch and slot sum");
+  for (int64_t u = u_begin; u < u_end && ok;) {
+    int l, R;
+    int64_t rb;
+    seg_of(u, l, rb, R);
+    u += R;
+    switch (R) {
+      case 1: segment(DecRows<1>{}, l, rb); break;
+      case 2: segment(DecRows<2>{}, l, rb); break;
+      case 3: segment(DecRows<3>{}, l, rb); break;
+      case 4: segment(DecRows<4>{}, l, rb); break;
+      default: segment(DecRows<kRb>{}, l, rb); break;
+    }
   }
   // Drain: after a give-up, the stages issued but not waited for must land before the
   // CTA exits (one deadline). At most nst stages can be in flight, each in its own slot.
