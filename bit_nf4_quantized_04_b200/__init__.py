@@ -173,6 +173,39 @@ def quantize_weight(W: torch.Tensor, sse: bool = False, out: Nf4Weight | None = 
     return (out, s[:1]) if sse else out
 
 
+def quantize_weight_group(Ws: list, sse: bool = False, outs=None, absmax=None, sse_out=None,
+                          ws=None):
+    """quantize_weight for up to 8 bf16 weights in two launches (qnf4_quantize_weight_group):
+    returns the list of ``Nf4Weight``, and with sse=True also the list of float64 [1] SSEs.
+    outs, absmax and sse_out, when given, are lists with one entry per weight."""
+    n = len(Ws)
+    for W in Ws:
+        _req(W, torch.bfloat16, "W")
+    dev = Ws[0].device
+    if outs is None:
+        outs = []
+        for W in Ws:
+            m = W.shape[0] * W.shape[1]
+            outs.append(Nf4Weight(W.shape[0], W.shape[1], torch.empty(m // 2, dtype=torch.uint8, device=dev),
+                                  torch.empty(m // BLOCK1, dtype=torch.uint8, device=dev),
+                                  torch.empty((m // BLOCK1 + BLOCK2 - 1) // BLOCK2, dtype=torch.float32,
+                                              device=dev),
+                                  torch.empty(4, dtype=torch.float32, device=dev)[:1]))
+    if absmax is None:
+        absmax = [torch.empty(W.shape[0] * W.shape[1] // BLOCK1, dtype=torch.float32, device=dev) for W in Ws]
+    ss = None
+    if sse:
+        ss = sse_out if sse_out is not None else [torch.empty(2, dtype=torch.float64, device=dev) for _ in Ws]
+    wsb = _ws(workspace_size(_lib.OP_QUANTIZE_WEIGHT_GROUP, 0, 0), Ws[0], ws)
+    ptrs = lambda ts: (C.c_void_p * n)(*[t.data_ptr() for t in ts])  # noqa: E731
+    i64 = lambda v: (C.c_int64 * n)(*v)  # noqa: E731
+    _lib.call("qnf4_quantize_weight_group", n, ptrs(Ws), i64([W.shape[0] for W in Ws]),
+              i64([W.shape[1] for W in Ws]), ptrs([o.packed for o in outs]), ptrs(absmax),
+              ptrs([o.code2 for o in outs]), ptrs([o.scale2 for o in outs]), ptrs([o.mean for o in outs]),
+              ptrs(ss) if sse else None, wsb.data_ptr(), wsb.numel(), _stream(Ws[0]))
+    return (outs, [t[:1] for t in ss]) if sse else outs
+
+
 def dequant(w: Nf4Weight, dtype: torch.dtype = torch.float32, out=None) -> torch.Tensor:
     """Two-level dequantization to an [N, K] fp32 or bf16 tensor (test/export path)."""
     code = {torch.float32: _lib.OUT_F32, torch.bfloat16: _lib.OUT_BF16}[dtype]

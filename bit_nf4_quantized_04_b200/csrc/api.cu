@@ -109,12 +109,12 @@ QuantTab make_tab() {
   return q;
 }
 
-int quant_grid(int64_t nblocks) {
+int quant_grid_chunks(int64_t chunks) {
   // persistent: kQCtasPerSm streaming CTAs per SM, never more warps than chunks
-  const int64_t chunks = (nblocks + kQChunkBlocks - 1) / kQChunkBlocks;
   const int64_t ctas = (chunks + kQWorkers - 1) / kQWorkers;
   return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(ctas, num_sms() * kQCtasPerSm)));
 }
+int quant_grid(int64_t nblocks) { return quant_grid_chunks((nblocks + kQChunkBlocks - 1) / kQChunkBlocks); }
 
 bool g_quant_smem_set[64] = {};
 
@@ -195,6 +195,47 @@ bool make_map(CUtensorMap* m, const void* ptr, bool u8, uint64_t inner, uint64_t
 bool quant_map(CUtensorMap* m, const void* W, int64_t nblocks) {
   if (nblocks > INT32_MAX) return false;  // the row coordinate is a 32-bit integer
   return make_map(m, W, false, 64, static_cast<uint64_t>(nblocks), 64, 64, kQChunkBlocks, true);
+}
+
+// One weight as the only job of a quantize launch (false if its map cannot be made).
+bool one_quant_job(QuantJobs* j, const void* W, int64_t nblocks, uint8_t* packed, float* absmax) {
+  std::memset(j, 0, sizeof(*j));
+  j->n = 1;
+  j->nblocks[0] = nblocks;
+  j->chunk0[0] = 0;
+  j->chunk0[1] = (nblocks + kQChunkBlocks - 1) / kQChunkBlocks;
+  j->packed[0] = reinterpret_cast<uint32_t*>(packed);
+  j->absmax[0] = absmax;
+  return quant_map(&j->map[0], W, nblocks);
+}
+
+// CTAs of a double-quantization launch over nb2 256-blocks, each a contiguous run.
+int dq_grid(DqJobs* d, int64_t nb2) {
+  const int64_t P = std::max<int64_t>(1, std::min<int64_t>((nb2 + 7) / 8, num_sms() * 4));
+  d->per_cta = std::max<int64_t>(1, (nb2 + P - 1) / P);
+  return static_cast<int>(std::max<int64_t>(1, (nb2 + d->per_cta - 1) / d->per_cta));
+}
+
+// One tensor as the only job of a double-quantization launch; returns the grid.
+int one_dq_job(DqJobs* d, const float* c, int64_t nb1, const double* part, int npart, int64_t count,
+               uint8_t* code2, float* scale2, float* mean, const double* sse_part, int nsse,
+               double* sse_out) {
+  std::memset(d, 0, sizeof(*d));
+  d->n = 1;
+  d->c[0] = c;
+  d->nb1[0] = nb1;
+  d->count[0] = count;
+  d->part[0] = part;
+  d->npart = npart;
+  d->code2[0] = code2;
+  d->scale2[0] = scale2;
+  d->mean[0] = mean;
+  d->sse_part[0] = sse_part;
+  d->nsse = nsse;
+  d->sse_out[0] = sse_out;
+  d->b2_0[0] = 0;
+  d->b2_0[1] = (nb1 + 255) / 256;
+  return dq_grid(d, d->b2_0[1]);
 }
 
 // x [M, K] bf16 seen as [K/64][M][64]: box = 16 column blocks x rows x 64 columns
@@ -1075,6 +1116,7 @@ size_t qnf4_workspace_size(int32_t op, int64_t N, int64_t K, int64_t M, int32_t 
     case QNF4_OP_QUANTIZE: return kQuantMaxGrid * sizeof(double);
     case QNF4_OP_LAYER_STATS: return 2 * kQuantMaxGrid * sizeof(double);
     case QNF4_OP_QUANTIZE_WEIGHT: return 2 * kQuantMaxGrid * sizeof(double);
+    case QNF4_OP_QUANTIZE_WEIGHT_GROUP: return 2 * kQMaxJobs * kQuantMaxGrid * sizeof(double);
     case QNF4_OP_DOUBLE_QUANT: return kDqPartials * sizeof(double);
     case QNF4_OP_FWD: {
       const size_t t = plan_linear(A_NF4_K, N, K, M, r, false, num_sms()).total;
@@ -1110,19 +1152,19 @@ qnf4_status qnf4_nf4_quantize(const void* W, int64_t N, int64_t K, int32_t block
   qnf4_status st = quant_smem_attr();
   if (st != QNF4_OK) return st;
   const int grid = quant_grid(nblocks);
-  CUtensorMap wmap;
-  if (!quant_map(&wmap, W, nblocks)) return map_fail();
+  static thread_local QuantJobs jobs;
+  if (!one_quant_job(&jobs, W, nblocks, packed, absmax)) return map_fail();
   const QuantTab tab = make_tab();
   if (sse) {
-    launch_pdl(k_nf4_quant<true, true>, dim3(grid), dim3(kQThreads), kQSmem, s, 
-        wmap, nblocks, reinterpret_cast<uint32_t*>(packed), absmax,
-        static_cast<double*>(ws), tab, g_wait_ns, 0.f, nullptr, nullptr);
+    launch_pdl(k_nf4_quant<true, true>, dim3(grid), dim3(kQThreads), kQSmem, s, jobs,
+               static_cast<double*>(ws), tab, g_wait_ns, 0.f, static_cast<double*>(nullptr),
+               static_cast<double*>(nullptr));
     launch_pdl(k_sum_partials, dim3(1), dim3(256), 0, s, static_cast<const double*>(ws), grid, sse);
     return launched("nf4_quantize", 2);
   }
-  launch_pdl(k_nf4_quant<true, false>, dim3(grid), dim3(kQThreads), kQSmem, s, 
-      wmap, nblocks, reinterpret_cast<uint32_t*>(packed), absmax,
-      nullptr, tab, g_wait_ns, 0.f, nullptr, nullptr);
+  launch_pdl(k_nf4_quant<true, false>, dim3(grid), dim3(kQThreads), kQSmem, s, jobs,
+             static_cast<double*>(nullptr), tab, g_wait_ns, 0.f, static_cast<double*>(nullptr),
+             static_cast<double*>(nullptr));
   return launched("nf4_quantize");
 }
 
@@ -1144,25 +1186,85 @@ qnf4_status qnf4_quantize_weight(const void* W, int64_t N, int64_t K, uint8_t* p
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int64_t nblocks = N * K / 64;
   const int grid = quant_grid(nblocks);
-  CUtensorMap wmap;
-  if (!quant_map(&wmap, W, nblocks)) return map_fail();
+  static thread_local QuantJobs jobs;
+  if (!one_quant_job(&jobs, W, nblocks, packed, absmax)) return map_fail();
   double* asum = static_cast<double*>(ws);
   double* ssep = asum + kQuantMaxGrid;
   const QuantTab tab = make_tab();
   if (sse) {
-    launch_pdl(k_nf4_quant<true, true>, dim3(grid), dim3(kQThreads), kQSmem, s, 
-        wmap, nblocks, reinterpret_cast<uint32_t*>(packed), absmax, ssep,
-        tab, g_wait_ns, 0.f, nullptr, asum);
+    launch_pdl(k_nf4_quant<true, true>, dim3(grid), dim3(kQThreads), kQSmem, s, jobs, ssep, tab,
+               g_wait_ns, 0.f, static_cast<double*>(nullptr), asum);
   } else {
-    launch_pdl(k_nf4_quant<true, false>, dim3(grid), dim3(kQThreads), kQSmem, s, 
-        wmap, nblocks, reinterpret_cast<uint32_t*>(packed), absmax,
-        nullptr, tab, g_wait_ns, 0.f, nullptr, asum);
+    launch_pdl(k_nf4_quant<true, false>, dim3(grid), dim3(kQThreads), kQSmem, s, jobs,
+               static_cast<double*>(nullptr), tab, g_wait_ns, 0.f, static_cast<double*>(nullptr), asum);
   }
-  const int64_t nb2 = (nblocks + 255) / 256;
-  const int egrid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((nb2 + 7) / 8, num_sms() * 4)));
-  launch_pdl(k_dq_encode, dim3(egrid), dim3(256), 0, s, absmax, nblocks, asum, grid, nblocks, code2, scale2, mean,
-                                    sse ? ssep : nullptr, grid, sse);
+  static thread_local DqJobs dq;
+  const int egrid = one_dq_job(&dq, absmax, nblocks, asum, grid, nblocks, code2, scale2, mean,
+                               sse ? ssep : nullptr, grid, sse);
+  launch_pdl(k_dq_encode, dim3(egrid), dim3(256), 0, s, dq);
   return launched("quantize_weight", 2);
+}
+
+qnf4_status qnf4_quantize_weight_group(int32_t n, const void* const* W, const int64_t* N,
+                                       const int64_t* K, uint8_t* const* packed, float* const* absmax,
+                                       uint8_t* const* code2, float* const* scale2, float* const* mean,
+                                       double* const* sse, void* ws, size_t ws_bytes, void* stream) {
+  if (n < 1 || n > kQMaxJobs) return fail(QNF4_ERR_ARG, "n must be in [1, %d] (got %d)", kQMaxJobs, n);
+  if (!W || !N || !K || !packed || !absmax || !code2 || !scale2 || !mean) return fail(QNF4_ERR_ARG, "NULL array");
+  for (int l = 0; l < n; ++l) {
+    if (N[l] <= 0 || K[l] <= 0) return fail(QNF4_ERR_SHAPE, "weight %d: N and K must be positive", l);
+    if (K[l] % 64) return fail(QNF4_ERR_SHAPE, "weight %d: K must be a multiple of 64", l);
+    if (!W[l] || !packed[l] || !absmax[l] || !code2[l] || !scale2[l] || !mean[l] || (sse && !sse[l]))
+      return fail(QNF4_ERR_ARG, "weight %d: NULL buffer", l);
+    for (const void* p : {W[l], static_cast<const void*>(packed[l]), static_cast<const void*>(absmax[l]),
+                          static_cast<const void*>(code2[l]), static_cast<const void*>(scale2[l]),
+                          static_cast<const void*>(mean[l]), static_cast<const void*>(sse ? sse[l] : nullptr)})
+      if (p && !al16(p)) return fail(QNF4_ERR_ALIGN, "buffers must be 16-byte aligned");
+  }
+  if (!ws || ws_bytes < qnf4_workspace_size(QNF4_OP_QUANTIZE_WEIGHT_GROUP, 0, 0, 0, 0))
+    return fail(QNF4_ERR_WORKSPACE, "workspace too small");
+  qnf4_status st = quant_smem_attr();
+  if (st != QNF4_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  static thread_local QuantJobs jobs;
+  static thread_local DqJobs dq;
+  std::memset(&jobs, 0, sizeof(jobs));
+  std::memset(&dq, 0, sizeof(dq));
+  jobs.n = dq.n = n;
+  jobs.chunk0[0] = dq.b2_0[0] = 0;
+  double* asum = static_cast<double*>(ws);
+  double* ssep = asum + kQMaxJobs * kQuantMaxGrid;
+  for (int l = 0; l < n; ++l) {
+    const int64_t nb = N[l] * K[l] / 64;
+    jobs.nblocks[l] = nb;
+    jobs.chunk0[l + 1] = jobs.chunk0[l] + (nb + kQChunkBlocks - 1) / kQChunkBlocks;
+    jobs.packed[l] = reinterpret_cast<uint32_t*>(packed[l]);
+    jobs.absmax[l] = absmax[l];
+    if (!quant_map(&jobs.map[l], W[l], nb)) return map_fail();
+    dq.c[l] = absmax[l];
+    dq.nb1[l] = nb;
+    dq.count[l] = nb;
+    dq.part[l] = asum + l * kQuantMaxGrid;
+    dq.code2[l] = code2[l];
+    dq.scale2[l] = scale2[l];
+    dq.mean[l] = mean[l];
+    dq.sse_part[l] = ssep + l * kQuantMaxGrid;
+    dq.sse_out[l] = sse ? sse[l] : nullptr;
+    dq.b2_0[l + 1] = dq.b2_0[l] + (nb + 255) / 256;
+  }
+  const int grid = quant_grid_chunks(jobs.chunk0[n]);
+  dq.npart = dq.nsse = grid;
+  const QuantTab tab = make_tab();
+  if (sse) {
+    launch_pdl(k_nf4_quant<true, true>, dim3(grid), dim3(kQThreads), kQSmem, s, jobs, ssep, tab,
+               g_wait_ns, 0.f, static_cast<double*>(nullptr), asum);
+  } else {
+    launch_pdl(k_nf4_quant<true, false>, dim3(grid), dim3(kQThreads), kQSmem, s, jobs,
+               static_cast<double*>(nullptr), tab, g_wait_ns, 0.f, static_cast<double*>(nullptr), asum);
+  }
+  const int egrid = std::max(dq_grid(&dq, dq.b2_0[n]), n);  // CTA l < n folds weight l's SSE
+  launch_pdl(k_dq_encode, dim3(egrid), dim3(256), 0, s, dq);
+  return launched("quantize_weight_group", 2);
 }
 
 qnf4_status qnf4_nf4_recon_error(const void* W, int64_t N, int64_t K, int32_t block1, double* sse,
@@ -1183,11 +1285,11 @@ qnf4_status qnf4_nf4_recon_error(const void* W, int64_t N, int64_t K, int32_t bl
   qnf4_status st = quant_smem_attr();
   if (st != QNF4_OK) return st;
   const int grid = quant_grid(nblocks);
-  CUtensorMap wmap;
-  if (!quant_map(&wmap, W, nblocks)) return map_fail();
-  launch_pdl(k_nf4_quant<false, true>, dim3(grid), dim3(kQThreads), kQSmem, s, wmap, nblocks,
-                                                          nullptr, nullptr, static_cast<double*>(ws),
-                                                          make_tab(), g_wait_ns, 0.f, nullptr, nullptr);
+  static thread_local QuantJobs jobs;
+  if (!one_quant_job(&jobs, W, nblocks, nullptr, nullptr)) return map_fail();
+  launch_pdl(k_nf4_quant<false, true>, dim3(grid), dim3(kQThreads), kQSmem, s, jobs,
+             static_cast<double*>(ws), make_tab(), g_wait_ns, 0.f, static_cast<double*>(nullptr),
+             static_cast<double*>(nullptr));
   launch_pdl(k_sum_partials, dim3(1), dim3(256), 0, s, static_cast<const double*>(ws), grid, sse);
   return launched("nf4_recon_error", 2);
 }
@@ -1211,12 +1313,11 @@ qnf4_status qnf4_nf4_layer_stats(const void* W, int64_t N, int64_t K, float tau,
   qnf4_status st = quant_smem_attr();
   if (st != QNF4_OK) return st;
   const int grid = quant_grid(nblocks);
-  CUtensorMap wmap;
-  if (!quant_map(&wmap, W, nblocks)) return map_fail();
+  static thread_local QuantJobs jobs;
+  if (!one_quant_job(&jobs, W, nblocks, nullptr, nullptr)) return map_fail();
   double* part = static_cast<double*>(ws);
-  launch_pdl(k_nf4_quant<false, true, true>, dim3(grid), dim3(kQThreads), kQSmem, s, 
-      wmap, nblocks, nullptr, nullptr, part, make_tab(), g_wait_ns, tau,
-      part + kQuantMaxGrid, nullptr);
+  launch_pdl(k_nf4_quant<false, true, true>, dim3(grid), dim3(kQThreads), kQSmem, s, jobs, part,
+             make_tab(), g_wait_ns, tau, part + kQuantMaxGrid, static_cast<double*>(nullptr));
   launch_pdl(k_sum_partials, dim3(1), dim3(256), 0, s, part, grid, sse);
   launch_pdl(k_sum_partials, dim3(1), dim3(256), 0, s, part + kQuantMaxGrid, grid, below);
   return launched("nf4_layer_stats", 3);
@@ -1234,10 +1335,9 @@ qnf4_status qnf4_double_quant(const float* absmax, int64_t nb1, int32_t block2, 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   double* part = static_cast<double*>(ws);
   k_dq_partial<<<kDqPartials, 256, 0, s>>>(absmax, nb1, part);
-  const int64_t nb2 = (nb1 + 255) / 256;
-  int grid = static_cast<int>(std::min<int64_t>((nb2 + 7) / 8, num_sms() * 4));
-  grid = std::max(grid, 1);
-  launch_pdl(k_dq_encode, dim3(grid), dim3(256), 0, s, absmax, nb1, part, kDqPartials, nb1, code2, scale2, mean, nullptr, 0, nullptr);
+  static thread_local DqJobs dq;
+  const int grid = one_dq_job(&dq, absmax, nb1, part, kDqPartials, nb1, code2, scale2, mean, nullptr, 0, nullptr);
+  launch_pdl(k_dq_encode, dim3(grid), dim3(256), 0, s, dq);
   return launched("double_quant", 2);
 }
 
@@ -1265,9 +1365,9 @@ qnf4_status qnf4_double_quant_shard(const float* absmax, int64_t nb1, int32_t bl
   if (!al16(absmax) || !al16(total_sum) || !al16(code2) || !al16(scale2) || !al16(mean))
     return fail(QNF4_ERR_ALIGN, "buffers must be 16-byte aligned");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int64_t nb2 = (nb1 + 255) / 256;
-  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((nb2 + 7) / 8, num_sms() * 4)));
-  launch_pdl(k_dq_encode, dim3(grid), dim3(256), 0, s, absmax, nb1, total_sum, 1, total_count, code2, scale2, mean, nullptr, 0, nullptr);
+  static thread_local DqJobs dq;
+  const int grid = one_dq_job(&dq, absmax, nb1, total_sum, 1, total_count, code2, scale2, mean, nullptr, 0, nullptr);
+  launch_pdl(k_dq_encode, dim3(grid), dim3(256), 0, s, dq);
   return launched("dq_encode_shard");
 }
 

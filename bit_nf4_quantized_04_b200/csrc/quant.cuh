@@ -35,6 +35,19 @@ constexpr uint32_t kQChunkBytes = kQChunkBlocks * 128u;  // 4 KB of bf16
 constexpr int kQMaxH = 16;          // largest bin count H the kernels' table holds
 constexpr int kQTabCopies = 16;     // table copies, one per lane of a half warp
 constexpr size_t kQSmem = static_cast<size_t>(kQWorkers) * kQStages * kQChunkBytes + 1024;
+constexpr int kQMaxJobs = 8;        // weights one launch quantizes
+
+// The weights of one quantize launch: their chunks form one list (job l's chunks are
+// [chunk0[l], chunk0[l + 1])), so a group of weights streams as one. A job's partial
+// sums go to part[l * kQuantMaxGrid + CTA].
+struct QuantJobs {
+  CUtensorMap map[kQMaxJobs];   // weight l as [nblocks, 64] bf16, boxes of kQChunkBlocks rows
+  int64_t nblocks[kQMaxJobs];
+  int64_t chunk0[kQMaxJobs + 1];
+  uint32_t* packed[kQMaxJobs];
+  float* absmax[kQMaxJobs];
+  int n;
+};
 
 // Shared loads of read-only tables (filled before a CTA barrier), by 32-bit shared address;
 // not volatile, so the compiler may schedule them freely.
@@ -110,8 +123,9 @@ QNF4_DEV void nf4_block_codes(const uint4 (&v)[8], float c, float f, float hf, f
   }
 }
 
-// Blockwise NF4 quantization, one 64-element block per lane. Warp g of the grid takes
-// the 32-block chunks g, g + G, ... (G = warps in the grid) through its own ring of
+// Blockwise NF4 quantization, one 64-element block per lane, of one or more weights
+// (jobs) whose 32-block chunks form one list. Warp g of the grid takes the chunks
+// g, g + G, ... (G = warps in the grid) through its own ring of
 // kQStages shared-memory stages: its lane 0 issues one TMA tile load per chunk (the
 // weight seen as a [blocks, 64] bf16 matrix, 128-byte swizzle, rows past the end
 // zero-filled) as soon as the warp has finished the chunk that stage held; no copy warp
@@ -122,7 +136,8 @@ QNF4_DEV void nf4_block_codes(const uint4 (&v)[8], float c, float f, float hf, f
 // error (fp32 within a block); CNT -> per-CTA float64 counts of the elements with
 // |w| < tau (the sparsity of "AQLoRA" §3.1), exact integers; asum_part (optional, with
 // WRITE) -> per-CTA float64 sums of the block constants, the partials of the double
-// quantization's tensor mean.
+// quantization's tensor mean. Partials are per job: a warp's chunks run through the
+// jobs in order, and it adds its sums into the CTA's slot of a job when it leaves it.
 //
 // absmax: max of |w| on the bf16 bit patterns, two elements per instruction.
 // Code search (see Nf4Tables), for a block with finite absmax c > 0: the bin
@@ -139,8 +154,7 @@ QNF4_DEV void nf4_block_codes(const uint4 (&v)[8], float c, float f, float hf, f
 // w - c q[code], one fma with the level read by the code.
 template <bool WRITE, bool SSE, bool CNT = false>
 __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
-    k_nf4_quant(const __grid_constant__ CUtensorMap wmap, int64_t nblocks,
-                uint32_t* __restrict__ packed, float* __restrict__ absmax,
+    k_nf4_quant(const __grid_constant__ QuantJobs jobs,
                 double* __restrict__ sse_part, QuantTab tab, unsigned long long wait_ns,
                 float tau = 0.f, double* __restrict__ cnt_part = nullptr,
                 double* __restrict__ asum_part = nullptr) {
@@ -149,9 +163,9 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
   __shared__ float s_lv[16];
   // entry k of copy j at (k kQTabCopies + j): a half warp's lanes read different copies
   __shared__ __align__(16) float2 s_th[(2 * kQMaxH + 1) * kQTabCopies];
-  __shared__ double s_red[kQWorkers];
-  __shared__ unsigned long long s_cnt[kQWorkers];
-  __shared__ double s_asum[kQWorkers];
+  __shared__ double s_red[kQWorkers][kQMaxJobs];
+  __shared__ unsigned long long s_cnt[kQWorkers][kQMaxJobs];
+  __shared__ double s_asum[kQWorkers][kQMaxJobs];
   __shared__ volatile int s_abort;
   uint8_t* qsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(qsm_raw) + 1023) &
                                             ~static_cast<uintptr_t>(1023));
@@ -167,10 +181,13 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
   if (lane == 0) {
     for (int i = 0; i < kQStages; ++i) mbar_init(&full[warp][i], 1);
   }
-  if (tid == 0) {
-    s_abort = 0;
-    tma_prefetch_desc(&wmap);
+  if (lane < kQMaxJobs) {
+    s_red[warp][lane] = 0.0;
+    s_cnt[warp][lane] = 0ull;
+    s_asum[warp][lane] = 0.0;
   }
+  if (tid < jobs.n) tma_prefetch_desc(&jobs.map[tid]);
+  if (tid == 0) s_abort = 0;
   fence_mbar_init();
   __syncthreads();
   // launched as a programmatic dependent: the prologue above overlapped the previous
@@ -178,7 +195,13 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
   griddep_wait();
   griddep_launch_dependents();
 
-  const int64_t nchunks = (nblocks + kQChunkBlocks - 1) / kQChunkBlocks;
+  const int64_t nchunks = jobs.chunk0[jobs.n];
+  // the job of chunk c
+  auto job_of = [&](int64_t c) {
+    int l = 0;
+    while (l + 1 < jobs.n && c >= jobs.chunk0[l + 1]) ++l;
+    return l;
+  };
   const int64_t gw = static_cast<int64_t>(blockIdx.x) * kQWorkers + warp;  // this warp
   const int64_t GW = static_cast<int64_t>(gridDim.x) * kQWorkers;
   const int64_t my = gw < nchunks ? (nchunks - 1 - gw) / GW + 1 : 0;      // its chunks
@@ -189,10 +212,11 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
   auto issue = [&](int64_t j) {
     const int64_t c = gw + j * GW;
     if (!in_bounds(c < nchunks, 1)) return;
+    const int l = job_of(c);
     uint64_t* bar = &fb[j % kQStages];
     mbar_expect_tx(bar, kQChunkBytes);
-    tma_load_2d(ring + (j % kQStages) * kQChunkBytes, &wmap, bar, 0,
-                static_cast<int32_t>(c * kQChunkBlocks));
+    tma_load_2d(ring + (j % kQStages) * kQChunkBytes, &jobs.map[l], bar, 0,
+                static_cast<int32_t>((c - jobs.chunk0[l]) * kQChunkBlocks));
   };
   if (lane == 0) {
     for (int64_t j = 0; j < min(my, static_cast<int64_t>(kQStages)); ++j) issue(j);
@@ -209,12 +233,42 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
   const uint32_t toff = smem_u32(s_th) + (lane & (kQTabCopies - 1)) * 8u -
                         0x4B400000u * (8u * kQTabCopies);
   const uint32_t lvb = smem_u32(s_lv);
+  // add this warp's sums for job l into the CTA's slots and restart them (all lanes)
+  auto flush = [&](int l) {
+    if (SSE) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (lane == 0) s_red[warp][l] += acc;
+    }
+    if (CNT) {
+      unsigned long long b = below;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) b += __shfl_xor_sync(0xffffffffu, b, o);
+      if (lane == 0) s_cnt[warp][l] += b;
+    }
+    if (WRITE && asum_part) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) asum += __shfl_xor_sync(0xffffffffu, asum, o);
+      if (lane == 0) s_asum[warp][l] += asum;
+    }
+    acc = 0.0;
+    asum = 0.0;
+    below = 0;
+  };
+  int cur = -1;      // job of the warp's running sums
   int64_t done = 0;  // chunks consumed (their copies have landed)
   for (int64_t j = 0; j < my; ++j) {
     if (!warp_wait(&fb[j % kQStages], static_cast<uint32_t>((j / kQStages) & 1), wait_ns, &s_abort, 51))
       break;
     done = j + 1;
-    const int64_t blk = (gw + j * GW) * kQChunkBlocks + lane;
+    const int64_t cj = gw + j * GW;
+    const int l = job_of(cj);
+    if (l != cur) {
+      if (cur >= 0) flush(cur);
+      cur = l;
+    }
+    const int64_t nblocks = jobs.nblocks[l];
+    const int64_t blk = (cj - jobs.chunk0[l]) * kQChunkBlocks + lane;
     const bool valid = blk < nblocks;
     // this lane's row; piece u at row ^ (u << 4) (the swizzle)
     const uint32_t row = smem_u32(ring + (j % kQStages) * kQChunkBytes) + lane * 128u +
@@ -280,10 +334,10 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
       }
     }
     if (WRITE && valid && in_bounds(blk < nblocks, 2)) {
-      uint4* dst = reinterpret_cast<uint4*>(packed) + blk * 2;
+      uint4* dst = reinterpret_cast<uint4*>(jobs.packed[l]) + blk * 2;
       dst[0] = make_uint4(pw[0], pw[1], pw[2], pw[3]);
       dst[1] = make_uint4(pw[4], pw[5], pw[6], pw[7]);
-      absmax[blk] = c;
+      jobs.absmax[l][blk] = c;
       asum += static_cast<double>(c);
     }
     if (SSE && valid) acc += static_cast<double>((acc2.x + acc2.y) * ssq * ssq);
@@ -309,37 +363,26 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
       }
     }
   }
-  if (SSE) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (lane == 0) s_red[warp] = acc;
-  }
-  if (CNT) {
-    unsigned long long b = below;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) b += __shfl_xor_sync(0xffffffffu, b, o);
-    if (lane == 0) s_cnt[warp] = b;
-  }
-  if (WRITE && asum_part) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) asum += __shfl_xor_sync(0xffffffffu, asum, o);
-    if (lane == 0) s_asum[warp] = asum;
-  }
+  if (cur >= 0) flush(cur);
   __syncthreads();
-  if (WRITE && asum_part && tid == 0 && in_bounds(blockIdx.x < kQuantMaxGrid, 3)) {
-    double t = 0.0;
-    for (int i = 0; i < kQWorkers; ++i) t += s_asum[i];
-    asum_part[blockIdx.x] = t;  // exact: bf16-derived constants sum exactly in float64
-  }
-  if (SSE && tid == 0 && in_bounds(blockIdx.x < kQuantMaxGrid, 3)) {
-    double t = 0.0;
-    for (int i = 0; i < kQWorkers; ++i) t += s_red[i];
-    sse_part[blockIdx.x] = t;
-  }
-  if (CNT && tid == 0 && in_bounds(blockIdx.x < kQuantMaxGrid, 3)) {
-    unsigned long long t = 0;
-    for (int i = 0; i < kQWorkers; ++i) t += s_cnt[i];
-    cnt_part[blockIdx.x] = static_cast<double>(t);  // exact below 2^53
+  // thread l writes job l's partials of this CTA (the warps' sums in a fixed order)
+  if (tid < jobs.n && in_bounds(blockIdx.x < kQuantMaxGrid, 3)) {
+    const int64_t o = static_cast<int64_t>(tid) * kQuantMaxGrid + blockIdx.x;
+    if (WRITE && asum_part) {
+      double t = 0.0;
+      for (int i = 0; i < kQWorkers; ++i) t += s_asum[i][tid];
+      asum_part[o] = t;  // exact: bf16-derived constants sum exactly in float64
+    }
+    if (SSE) {
+      double t = 0.0;
+      for (int i = 0; i < kQWorkers; ++i) t += s_red[i][tid];
+      sse_part[o] = t;
+    }
+    if (CNT) {
+      unsigned long long t = 0;
+      for (int i = 0; i < kQWorkers; ++i) t += s_cnt[i][tid];
+      cnt_part[o] = static_cast<double>(t);  // exact below 2^53
+    }
   }
 }
 
@@ -390,46 +433,71 @@ __global__ void __launch_bounds__(256) k_dq_partial(const float* __restrict__ c,
   if (threadIdx.x == 0 && in_bounds(blockIdx.x < kDqPartials, 4)) part[blockIdx.x] = s[0];
 }
 
-// Each CTA reduces the partials to the tensor mean (bf16-derived constants sum
-// exactly in float64, so the mean is independent of the summation order), then one
-// warp per 256-block: subtract the mean, block absmax, scale = absmax / 448 (IEEE
-// division), code = E4M3 round-to-nearest-even with saturation of (c - mean)/scale.
-// count is the number of constants behind the partials: nb1 for a whole matrix, the
-// matrix's total for one row shard of it (whose partial is then the all-reduced sum).
-__global__ void __launch_bounds__(256) k_dq_encode(const float* __restrict__ c, int64_t nb1,
-                                                   const double* __restrict__ part, int npart,
-                                                   int64_t count, uint8_t* __restrict__ code2,
-                                                   float* __restrict__ scale2,
-                                                   float* __restrict__ mean_out,
-                                                   const double* __restrict__ sse_part = nullptr,
-                                                   int nsse = 0, double* __restrict__ sse_out = nullptr) {
-  __shared__ float s_mu;
+// The tensors of one double-quantization launch: their 256-blocks form one list (job
+// l's are [b2_0[l], b2_0[l + 1])), which the CTAs take in contiguous runs of per_cta.
+struct DqJobs {
+  const float* c[kQMaxJobs];         // first-level constants [nb1]
+  int64_t nb1[kQMaxJobs];
+  int64_t count[kQMaxJobs];          // constants behind the mean's partials
+  const double* part[kQMaxJobs];     // the mean's float64 partials, npart per job
+  uint8_t* code2[kQMaxJobs];
+  float* scale2[kQMaxJobs];
+  float* mean[kQMaxJobs];
+  const double* sse_part[kQMaxJobs];  // (fused quantize path) SSE partials, nsse per job
+  double* sse_out[kQMaxJobs];         // or NULL
+  int64_t b2_0[kQMaxJobs + 1];
+  int64_t per_cta;
+  int npart, nsse, n;
+};
+
+// Each CTA reduces the partials of the jobs it touches to their tensor means
+// (bf16-derived constants sum exactly in float64, so a mean is independent of the
+// summation order), then one warp per 256-block: subtract the mean, block absmax,
+// scale = absmax / 448 (IEEE division), code = E4M3 round-to-nearest-even with
+// saturation of (c - mean)/scale. A job's count is the number of constants behind its
+// partials: nb1 for a whole matrix, the matrix's total for one row shard of it (whose
+// partial is then the all-reduced sum). CTA l (l < n) writes job l's mean and, on the
+// fused quantize path, folds its SSE partials in k_sum_partials' order.
+__global__ void __launch_bounds__(256) k_dq_encode(const __grid_constant__ DqJobs d) {
+  __shared__ float s_mu[kQMaxJobs];
   griddep_wait();  // (programmatic dependent of the kernel that wrote the constants)
   griddep_launch_dependents();
-  const int lane = threadIdx.x & 31;
-  // (fused quantize path) CTA 0 also folds the quantizer's SSE partials, in the same
-  // order as k_sum_partials
-  if (sse_out && blockIdx.x == 0) {
-    const double t = block_sum_partials(sse_part, nsse);
-    if (threadIdx.x == 0) *sse_out = t;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int64_t lo = static_cast<int64_t>(blockIdx.x) * d.per_cta;
+  const int64_t hi = min(d.b2_0[d.n], lo + d.per_cta);
+  auto job_of = [&](int64_t j) {
+    int l = 0;
+    while (l + 1 < d.n && j >= d.b2_0[l + 1]) ++l;
+    return l;
+  };
+  const int llo = lo < hi ? job_of(lo) : d.n, lhi = lo < hi ? job_of(hi - 1) : -1;
+  const int own = static_cast<int>(blockIdx.x) < d.n ? static_cast<int>(blockIdx.x) : -1;
+  if (own >= 0 && d.sse_out[own]) {
+    const double t = block_sum_partials(d.sse_part[own], d.nsse);
+    if (threadIdx.x == 0) *d.sse_out[own] = t;
   }
-  if (threadIdx.x < 32) {
+  // warp w computes job w's mean if this CTA needs it
+  static_assert(kQMaxJobs <= 256 / 32, "one warp per job");
+  if (wid < d.n && ((wid >= llo && wid <= lhi) || wid == own)) {
     double t = 0.0;
-    for (int i = lane; i < npart; i += 32) t += part[i];
+    for (int i = lane; i < d.npart; i += 32) t += d.part[wid][i];
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
     if (lane == 0) {
-      const float mu = static_cast<float>(t / static_cast<double>(count));
-      s_mu = mu;
-      if (blockIdx.x == 0) *mean_out = mu;
+      const float mu = static_cast<float>(t / static_cast<double>(d.count[wid]));
+      s_mu[wid] = mu;
+      if (wid == own) *d.mean[wid] = mu;
     }
   }
   __syncthreads();
-  const float mu = s_mu;
-  const int64_t nb2 = (nb1 + 255) / 256;
-  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-  for (int64_t j = warp; j < nb2; j += nwarps) {
+  for (int64_t jg = lo + wid; jg < hi; jg += 8) {
+    const int l = job_of(jg);
+    const int64_t j = jg - d.b2_0[l];
+    const float mu = s_mu[l];
+    const float* __restrict__ c = d.c[l];
+    const int64_t nb1 = d.nb1[l], nb2 = (nb1 + 255) / 256;
+    uint8_t* __restrict__ code2 = d.code2[l];
+    float* __restrict__ scale2 = d.scale2[l];
     const int64_t e0 = j * 256 + lane * 8;
     float v[8];
     if (e0 + 8 <= nb1) {

@@ -75,7 +75,8 @@ enum {
   QNF4_OP_CHANQ_BWD = 5,    /* qnf4_chanq_linear_bwd                                 */
   QNF4_OP_LOFTQ = 6,        /* qnf4_loftq_nf4                                        */
   QNF4_OP_LAYER_STATS = 7,  /* qnf4_nf4_layer_stats                                  */
-  QNF4_OP_QUANTIZE_WEIGHT = 8 /* qnf4_quantize_weight                                */
+  QNF4_OP_QUANTIZE_WEIGHT = 8, /* qnf4_quantize_weight                               */
+  QNF4_OP_QUANTIZE_WEIGHT_GROUP = 9 /* qnf4_quantize_weight_group (any shapes)        */
 };
 
 /* A double-quantized NF4 weight [QLoRA 贡献一/贡献二]. All pointers are device
@@ -140,6 +141,19 @@ QNF4_API qnf4_status qnf4_double_quant(const float* absmax, int64_t nb1, int32_t
 QNF4_API qnf4_status qnf4_quantize_weight(const void* W_bf16, int64_t N, int64_t K, uint8_t* packed,
                                  float* absmax, uint8_t* code2, float* scale2, float* mean,
                                  double* sse, void* ws, size_t ws_bytes, void* stream);
+
+/* [QLoRA 贡献一 + 贡献二; AQLoRA §3.1] qnf4_quantize_weight for n (1..8) independent weights
+ * in two launches, whose work forms one list (so a set of layers streams as one matrix
+ * would). Host arrays of n entries: W[l] (bf16 [N[l], K[l]], device), N[l], K[l] (> 0, K[l]
+ * a multiple of 64), the device outputs packed[l], absmax[l], code2[l], scale2[l], mean[l]
+ * as qnf4_quantize_weight's, and sse (NULL for none, else n device pointers to one double
+ * each). Every output but the SSE equals qnf4_quantize_weight's bit for bit; each SSE is the
+ * same float64 sum of fp32 block sums, grouped differently (equal up to float64 rounding).
+ * Workspace: qnf4_workspace_size(QNF4_OP_QUANTIZE_WEIGHT_GROUP, 0, 0, 0, 0). */
+QNF4_API qnf4_status qnf4_quantize_weight_group(int32_t n, const void* const* W, const int64_t* N,
+                                       const int64_t* K, uint8_t* const* packed, float* const* absmax,
+                                       uint8_t* const* code2, float* const* scale2, float* const* mean,
+                                       double* const* sse, void* ws, size_t ws_bytes, void* stream);
 
 /* [QLoRA 贡献二] A matrix quantized as row shards (one per process): the tensor mean needs
  * the float64 sum of all its constants. qnf4_dq_sum writes this shard's sum to *sum (device,

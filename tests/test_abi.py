@@ -33,6 +33,7 @@ def test_header_declares_the_abi():
     names = _declared()
     for n in ("qnf4_nf4_codebook", "qnf4_nf4_quantize", "qnf4_double_quant", "qnf4_dequant",
               "qnf4_qlora_linear_fwd", "qnf4_qlora_linear_fwd_group", "qnf4_qlora_linear_bwd",
+              "qnf4_quantize_weight", "qnf4_quantize_weight_group",
               "qnf4_nf4_recon_error",
               "qnf4_chanq_quantize", "qnf4_chanq_linear_fwd", "qnf4_workspace_size",
               "qnf4_last_error"):
@@ -121,6 +122,21 @@ def test_argument_checks_fail_before_any_launch(q):
                1 << 20, None) == 1
     assert _st(q, "qnf4_qlora_linear_fwd_group", 2, arr, ptrs, 4, ptrs, ptrs, 8, 1.0, ptrs, fake,
                16, None) == 6
+    # grouped quantization: n in 1..8, per-weight shape, NULL and alignment checks, workspace
+    i64 = lambda *v: (C.c_int64 * len(v))(*v)  # noqa: E731
+    N2, K2 = i64(4, 8), i64(64, 128)
+    gq = lambda n, N, K, p, ws_bytes: _st(q, "qnf4_quantize_weight_group", n, p, N, K, p, p, p, p, p,  # noqa: E731
+                                          None, fake, ws_bytes, None)
+    assert gq(0, N2, K2, ptrs, 1 << 20) == 1
+    assert gq(9, N2, K2, ptrs, 1 << 20) == 1
+    assert gq(2, N2, i64(64, 100), ptrs, 1 << 20) == 2
+    assert gq(2, i64(4, 0), K2, ptrs, 1 << 20) == 2
+    assert gq(2, N2, K2, (C.c_void_p * 2)(fake, None), 1 << 20) == 1
+    assert gq(2, N2, K2, (C.c_void_p * 2)(fake, fake + 8), 1 << 20) == 3
+    assert gq(2, N2, K2, ptrs, 16) == 6
+    assert _st(q, "qnf4_quantize_weight_group", 2, None, N2, K2, ptrs, ptrs, ptrs, ptrs, ptrs, None,
+               fake, 1 << 20, None) == 1
+    assert q.workspace_size(q._lib.OP_QUANTIZE_WEIGHT_GROUP, 0, 0) >= 2 * 8 * 1024 * 8
 
 
 def test_argument_checks_of_the_next_rows(q):

@@ -301,3 +301,35 @@ def test_fused_quantize_weight_all_zero(q):
     assert sse.item() == 0.0 and w.mean.item() == 0.0
     assert torch.all(w.code2 == 0) and torch.all(w.scale2 == 0)
     assert torch.all(w.packed == 0x77)
+
+
+@pytest.mark.parametrize("shapes", [
+    [(33, 320)],                                              # one weight (the single call's grid)
+    [(33, 320), (4096, 11008), (300, 4096), (8, 64)],         # ragged chunk and 256-block ends
+    [(16, 64 * k) for k in range(1, 9)],                      # eight tiny weights: CTAs span several
+])
+def test_quantize_weight_group_matches_single_calls(q, shapes):
+    # qnf4_quantize_weight_group: codes, constants, code2, scale2 and mean equal the
+    # single call's bit for bit; each SSE equals it up to float64 rounding (the per-CTA
+    # partials group the same fp32 block sums differently) and matches the oracle
+    Ws = []
+    for i, (N, K) in enumerate(shapes):
+        W = synth.llama_weight((N, K), 900 + 7 * i + N, std=0.02)
+        if N == 300:
+            W[5] = 0
+        Ws.append(W.cuda())
+    outs, sses = q.quantize_weight_group(Ws, sse=True)
+    plain = q.quantize_weight_group(Ws)
+    torch.cuda.synchronize()
+    for i, W in enumerate(Ws):
+        w, sse = q.quantize_weight(W, sse=True)
+        torch.cuda.synchronize()
+        for a, b in ((outs[i].packed, w.packed), (outs[i].code2, w.code2), (outs[i].scale2, w.scale2),
+                     (outs[i].mean, w.mean), (plain[i].packed, w.packed), (plain[i].code2, w.code2)):
+            assert torch.equal(a, b), f"weight {i} {shapes[i]}"
+        assert abs(sses[i].item() - sse.item()) <= 1e-12 * max(sse.item(), 1e-300)
+    # one weight of the mixed set against the oracle
+    oq = oracle_quant(Ws[-1].cpu())
+    assert np.array_equal(outs[-1].code2.cpu().numpy(), oq["code2"])
+    ref = onf4.recon_sse(f32(Ws[-1].cpu()))
+    assert abs(sses[-1].item() - ref) <= 1e-5 * ref
