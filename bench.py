@@ -228,7 +228,7 @@ class Workload:
             L["dA"] = torch.empty(RANK, K, dtype=torch.float32, device=dev)
             L["dB"] = torch.empty(N, RANK, dtype=torch.float32, device=dev)
             for op, m in ((q._lib.OP_QUANTIZE, 0), (q._lib.OP_DOUBLE_QUANT, 0), (q._lib.OP_LAYER_STATS, 0),
-                          (q._lib.OP_QUANTIZE_WEIGHT, 0),
+                          (q._lib.OP_QUANTIZE_WEIGHT, 0), (q._lib.OP_QUANTIZE_WEIGHT_GROUP, 0),
                           (q._lib.OP_FWD, M_TOK), (q._lib.OP_BWD, M_TOK)):
                 wsz = max(wsz, q.workspace_size(op, N, K, m, RANK))
             self.layers.append(L)
@@ -259,12 +259,12 @@ class Workload:
 
     # the pieces of one step
     def quantize(self):
-        # NF4 codes, constants, double quantization and the reconstruction SSE: two
-        # launches per layer (qnf4_quantize_weight)
-        q = self.q
-        for L in self.layers:
-            q.quantize_weight(L["W"], sse=True, out=L["w"], absmax=L["absmax"], sse_out=L["sse"],
-                              ws=self.ws)
+        # NF4 codes, constants, double quantization and the reconstruction SSE of the 7
+        # layers: two launches for the set (qnf4_quantize_weight_group)
+        L = self.layers
+        self.q.quantize_weight_group([x["W"] for x in L], sse=True, outs=[x["w"] for x in L],
+                                     absmax=[x["absmax"] for x in L], sse_out=[x["sse"] for x in L],
+                                     ws=self.ws)
 
     def fwd(self, ev=None):
         for i, L in enumerate(self.layers):
@@ -586,11 +586,11 @@ def stack13b(q, dev, hbm, tc, seconds=2.0):
                               torch.empty((n // 64 + 255) // 256, dtype=torch.float32, device=dev),
                               torch.empty(4, dtype=torch.float32, device=dev)[:1]))
     nmax = max(sh.N * sh.K for sh in shapes)
-    absmax = torch.empty(nmax // 64, dtype=torch.float32, device=dev)
+    absmax = [torch.empty(nmax // 64, dtype=torch.float32, device=dev) for _ in range(8)]
     sse = torch.zeros(len(shapes), 2, dtype=torch.float64, device=dev)
     kinds = sorted({(sh.N, sh.K) for sh in shapes})
     io = {}
-    wsz = q.workspace_size(q._lib.OP_QUANTIZE_WEIGHT, nmax, 64)
+    wsz = q.workspace_size(q._lib.OP_QUANTIZE_WEIGHT_GROUP, 0, 0)
     for j, (N, K) in enumerate(kinds):
         io[(N, K)] = dict(
             x=synth.normal_bf16((M, K), 1.0, synth.SEED_X + 300 + j, device=dev),
@@ -606,8 +606,13 @@ def stack13b(q, dev, hbm, tc, seconds=2.0):
     ws = torch.empty(wsz, dtype=torch.uint8, device=dev)
 
     def profile_pass():
-        for i, W in enumerate(Ws):
-            q.quantize_weight(W, sse=True, out=wq[i], absmax=absmax, sse_out=sse[i], ws=ws)
+        # groups of 8 matrices, two launches per group (qnf4_quantize_weight_group); the
+        # group's first-level constants go to per-matrix slices of one buffer
+        for g0 in range(0, len(Ws), 8):
+            ids = range(g0, min(g0 + 8, len(Ws)))
+            q.quantize_weight_group([Ws[i] for i in ids], sse=True, outs=[wq[i] for i in ids],
+                                    absmax=[absmax[k] for k in range(len(ids))],
+                                    sse_out=[sse[i] for i in ids], ws=ws)
     profile = graphed(profile_pass)
     nparams = [sh.N * sh.K for sh in shapes]
     protected = q.rank_topk(sse[:, 0].cpu().tolist(), nparams, topk)
@@ -636,7 +641,7 @@ def stack13b(q, dev, hbm, tc, seconds=2.0):
     out = {"matrices": len(shapes), "params": ptot, "tokens": M, "r": r, "alpha": alpha,
            "profile_pass": {"GBps": round(gbs, 1), "frac_hbm": round(gbs / hbm, 3),
                             "ms": round(tp * 1e3, 2), "passes": ip,
-                            "launch": "CUDA graph of 280 x qnf4_quantize_weight"},
+                            "launch": "CUDA graph of 35 x qnf4_quantize_weight_group (8 matrices each)"},
            "protected_top8": protected,
            "fwd_bwd": {"TFLOPs": round(tfs, 1), "frac_tc": round(tfs / tc, 3),
                        "tflop_per_pass": round(fl / 1e12, 2), "ms": round(tt * 1e3, 1),
@@ -828,11 +833,35 @@ def run_ours(args):
 
 
 def run_case(args):
-    """One operation on one gate-shaped layer (11008x4096 NF4 weight), warmup + steps
-    launches and nothing else: the small, L2-exceeding case for ncu captures."""
+    """One operation on one gate-shaped layer (11008x4096 NF4 weight), or a grouped call
+    over the 7-layer set (quant_group, decode_group), warmup + steps calls and nothing
+    else: the small, L2-exceeding case for ncu captures."""
     import synth
     import bit_nf4_quantized_04_b200 as q
     dev = torch.device("cuda", 0)
+    if args.case in ("quant_group", "decode_group"):
+        shapes = layer_shapes()
+        Ws = [synth.llama_weight((N, K), synth.SEED_W + i, device=dev) for i, (N, K) in enumerate(shapes)]
+        gws = torch.empty(1 << 26, dtype=torch.uint8, device=dev)
+        if args.case == "quant_group":
+            outs, sses = q.quantize_weight_group(Ws, sse=True, ws=gws)
+            fn = lambda: q.quantize_weight_group(Ws, sse=True, outs=outs, sse_out=sses, ws=gws)  # noqa: E731
+            m = 0
+        else:
+            m = 16
+            wq = q.quantize_weight_group(Ws, ws=gws)
+            xs = [synth.normal_bf16((m, K), 1.0, synth.SEED_X + i, device=dev) for i, (N, K) in enumerate(shapes)]
+            As = [synth.normal_bf16((RANK, K), 0.01, synth.SEED_A + i, device=dev) for i, (N, K) in enumerate(shapes)]
+            Bs = [synth.normal_bf16((N, RANK), 0.01, synth.SEED_B + i, device=dev) for i, (N, K) in enumerate(shapes)]
+            hs = [torch.empty(m, N, dtype=torch.bfloat16, device=dev) for N, K in shapes]
+            fn = lambda: q.qlora_linear_fwd_group(wq, xs, As, Bs, ALPHA / RANK, hs=hs, ws=gws)  # noqa: E731
+        for _ in range(args.warmup):
+            fn()
+        t = time_loop(fn, args.steps, torch.cuda.current_stream())
+        q.check()
+        print(json.dumps({"case": args.case, "layers": len(shapes), "M": m,
+                          "calls": args.warmup + args.steps, "us_per_call": round(t * 1e6, 2)}))
+        return
     N, K = 11008, 4096
     m = {"fwd": M_TOK, "bwd": M_TOK, "decode": 16}.get(args.case, M_TOK)
     W = synth.llama_weight((N, K), synth.SEED_W + 4, device=dev)
@@ -880,7 +909,7 @@ def run_case(args):
     elif args.case == "bwd":
         fn = lambda: q.qlora_linear_bwd(w, x, dY, A, B, s, ws=ws)  # noqa: E731
     else:  # quant
-        fn = lambda: q.quantize_weight(W, sse=True, ws=ws)  # noqa: E731  (as the step runs it)
+        fn = lambda: q.quantize_weight(W, sse=True, ws=ws)  # noqa: E731  (one weight alone)
     for _ in range(args.warmup):
         fn()
     t = time_loop(fn, args.steps, torch.cuda.current_stream())
@@ -943,7 +972,8 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-stack", action="store_true", help="skip the 13B-stack row")
     ap.add_argument("--no-protocol", action="store_true", help="skip the 2 s x 3 session arms")
-    ap.add_argument("--case", choices=["fwd", "bwd", "decode", "quant", "chanq_quant", "chanq_fwd", "chanq_bwd"], default=None,
+    ap.add_argument("--case", choices=["fwd", "bwd", "decode", "quant", "chanq_quant", "chanq_fwd", "chanq_bwd",
+                                       "quant_group", "decode_group"], default=None,
                     help="run one operation on one gate-shaped layer (for ncu captures)")
     args = ap.parse_args()
     if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
