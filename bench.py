@@ -366,21 +366,22 @@ def lloyd_t0(bits: int):
 def breakdown(wl, q, hbm, tc):
     """Per-row throughput, each timed alone (short loops, L2-exceeding inputs). Tensor
     rows are fractions of `tc`, the burst bf16 peak (each loop runs well under a second at
-    full clock)."""
+    full clock). The HBM-bound rows over the layer set replay a CUDA graph of their calls
+    (as the protocol arms do), so the host's launch work does not leave the GPU idle."""
     st = torch.cuda.current_stream()
     out = {}
     nparam = sum(N * K for N, K in layer_shapes())
-    t = time_loop(wl.quantize, 10, st)
+    t = time_loop(graphed(wl.quantize), 10, st)
     gbs = nparam * (2 + 0.5 + 1 / 64 + 4 / 16384) / t / 1e9
     out["quant_dq_sse"] = {"GBps": round(gbs, 1), "frac_hbm": round(gbs / hbm, 3),
                            "bytes_per_param": 2.5159}
-    t = time_loop(lambda: [q.nf4_recon_error(L["W"], sse=L["sse"], ws=wl.ws) for L in wl.layers],
+    t = time_loop(graphed(lambda: [q.nf4_recon_error(L["W"], sse=L["sse"], ws=wl.ws) for L in wl.layers]),
                   10, st)
     gbs = nparam * 2 / t / 1e9
     out["recon_error"] = {"GBps": round(gbs, 1), "frac_hbm": round(gbs / hbm, 3)}
     # the same pass with the AQLoRA sparsity count beside the error (one read of W)
     lso = torch.empty(4, dtype=torch.float64, device=wl.dev)
-    t = time_loop(lambda: [q.nf4_layer_stats(L["W"], out=lso, ws=wl.ws) for L in wl.layers], 10, st)
+    t = time_loop(graphed(lambda: [q.nf4_layer_stats(L["W"], out=lso, ws=wl.ws) for L in wl.layers]), 10, st)
     gbs = nparam * 2 / t / 1e9
     out["layer_stats"] = {"GBps": round(gbs, 1), "frac_hbm": round(gbs / hbm, 3)}
     ff = sum(fwd_flops(N, K, M_TOK, RANK) for N, K in layer_shapes())
