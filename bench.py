@@ -229,6 +229,7 @@ class Workload:
             L["dB"] = torch.empty(N, RANK, dtype=torch.float32, device=dev)
             for op, m in ((q._lib.OP_QUANTIZE, 0), (q._lib.OP_DOUBLE_QUANT, 0), (q._lib.OP_LAYER_STATS, 0),
                           (q._lib.OP_QUANTIZE_WEIGHT, 0), (q._lib.OP_QUANTIZE_WEIGHT_GROUP, 0),
+                          (q._lib.OP_LAYER_STATS_GROUP, 0),
                           (q._lib.OP_FWD, M_TOK), (q._lib.OP_BWD, M_TOK)):
                 wsz = max(wsz, q.workspace_size(op, N, K, m, RANK))
             self.layers.append(L)
@@ -375,13 +376,15 @@ def breakdown(wl, q, hbm, tc):
     gbs = nparam * (2 + 0.5 + 1 / 64 + 4 / 16384) / t / 1e9
     out["quant_dq_sse"] = {"GBps": round(gbs, 1), "frac_hbm": round(gbs / hbm, 3),
                            "bytes_per_param": 2.5159}
-    t = time_loop(graphed(lambda: [q.nf4_recon_error(L["W"], sse=L["sse"], ws=wl.ws) for L in wl.layers]),
-                  10, st)
+    # the AQLoRA profiling pass over the layer set in one quantizer launch
+    # (qnf4_nf4_layer_stats_group): the error alone, then with the sparsity count beside it
+    Wl = [L["W"] for L in wl.layers]
+    sl = [L["sse"] for L in wl.layers]
+    cl = [torch.empty(2, dtype=torch.float64, device=wl.dev) for _ in wl.layers]
+    t = time_loop(graphed(lambda: q.nf4_layer_stats_group(Wl, tau=None, sse=sl, ws=wl.ws)), 10, st)
     gbs = nparam * 2 / t / 1e9
     out["recon_error"] = {"GBps": round(gbs, 1), "frac_hbm": round(gbs / hbm, 3)}
-    # the same pass with the AQLoRA sparsity count beside the error (one read of W)
-    lso = torch.empty(4, dtype=torch.float64, device=wl.dev)
-    t = time_loop(graphed(lambda: [q.nf4_layer_stats(L["W"], out=lso, ws=wl.ws) for L in wl.layers]), 10, st)
+    t = time_loop(graphed(lambda: q.nf4_layer_stats_group(Wl, tau=0.01, sse=sl, below=cl, ws=wl.ws)), 10, st)
     gbs = nparam * 2 / t / 1e9
     out["layer_stats"] = {"GBps": round(gbs, 1), "frac_hbm": round(gbs / hbm, 3)}
     ff = sum(fwd_flops(N, K, M_TOK, RANK) for N, K in layer_shapes())

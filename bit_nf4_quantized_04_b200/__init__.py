@@ -297,6 +297,28 @@ def nf4_layer_stats(W: torch.Tensor, tau: float = 0.01, out=None, ws=None):
     return o[0::2]
 
 
+def nf4_layer_stats_group(Ws: list, tau: float | None = 0.01, sse=None, below=None, ws=None):
+    """The profiling pass over up to 8 bf16 weights in one quantizer launch
+    (qnf4_nf4_layer_stats_group): the list of NF4 reconstruction SSEs (float64 [1] each) and,
+    unless tau is None, the list of #{|w| < tau} counts; returns (sse list, count list or
+    None). sse and below, when given, are lists of float64 tensors (one per weight)."""
+    n = len(Ws)
+    for W in Ws:
+        _req(W, torch.bfloat16, "W")
+    dev = Ws[0].device
+    sse = sse if sse is not None else [torch.empty(2, dtype=torch.float64, device=dev) for _ in Ws]
+    cnt = None
+    if tau is not None:
+        cnt = below if below is not None else [torch.empty(2, dtype=torch.float64, device=dev) for _ in Ws]
+    wsb = _ws(workspace_size(_lib.OP_LAYER_STATS_GROUP, 0, 0), Ws[0], ws)
+    ptrs = lambda ts: (C.c_void_p * n)(*[t.data_ptr() for t in ts])  # noqa: E731
+    i64 = lambda v: (C.c_int64 * n)(*v)  # noqa: E731
+    _lib.call("qnf4_nf4_layer_stats_group", n, ptrs(Ws), i64([W.shape[0] for W in Ws]),
+              i64([W.shape[1] for W in Ws]), float(tau if tau is not None else 0.0), ptrs(sse),
+              ptrs(cnt) if cnt is not None else None, wsb.data_ptr(), wsb.numel(), _stream(Ws[0]))
+    return [t[:1] for t in sse], ([t[:1] for t in cnt] if cnt is not None else None)
+
+
 def rank_topk(sse, n_params, k: int) -> list[int]:
     """Host ranking: indices of the k layers with the largest sse/n, ties to the lower index."""
     s = [float(v) for v in sse]

@@ -20,7 +20,7 @@ STATUS_NAMES = {0: "OK", 1: "ERR_ARG", 2: "ERR_SHAPE", 3: "ERR_ALIGN", 4: "ERR_C
                 5: "ERR_TIMEOUT", 6: "ERR_WORKSPACE", 7: "ERR_BOUNDS"}
 OUT_F32, OUT_BF16 = 0, 1
 OP_QUANTIZE, OP_DOUBLE_QUANT, OP_FWD, OP_BWD, OP_CHANQ_FWD, OP_CHANQ_BWD, OP_LOFTQ = 0, 1, 2, 3, 4, 5, 6
-OP_LAYER_STATS, OP_QUANTIZE_WEIGHT, OP_QUANTIZE_WEIGHT_GROUP = 7, 8, 9
+OP_LAYER_STATS, OP_QUANTIZE_WEIGHT, OP_QUANTIZE_WEIGHT_GROUP, OP_LAYER_STATS_GROUP = 7, 8, 9, 10
 
 
 class Qnf4Weight(C.Structure):
@@ -44,6 +44,8 @@ SIGNATURES = {
     "qnf4_double_quant": (ST, [P, I64, I32, P, P, P, P, SZ, P]),
     "qnf4_dq_sum": (ST, [P, I64, P, P, SZ, P]),
     "qnf4_quantize_weight": (ST, [P, I64, I64, P, P, P, P, P, P, P, SZ, P]),
+    "qnf4_nf4_layer_stats_group": (ST, [I32, C.POINTER(P), C.POINTER(I64), C.POINTER(I64), C.c_float,
+                                        C.POINTER(P), C.POINTER(P), P, SZ, P]),
     "qnf4_quantize_weight_group": (ST, [I32, C.POINTER(P), C.POINTER(I64), C.POINTER(I64), C.POINTER(P),
                                         C.POINTER(P), C.POINTER(P), C.POINTER(P), C.POINTER(P),
                                         C.POINTER(P), P, SZ, P]),

@@ -1117,6 +1117,7 @@ size_t qnf4_workspace_size(int32_t op, int64_t N, int64_t K, int64_t M, int32_t 
     case QNF4_OP_LAYER_STATS: return 2 * kQuantMaxGrid * sizeof(double);
     case QNF4_OP_QUANTIZE_WEIGHT: return 2 * kQuantMaxGrid * sizeof(double);
     case QNF4_OP_QUANTIZE_WEIGHT_GROUP: return 2 * kQMaxJobs * kQuantMaxGrid * sizeof(double);
+    case QNF4_OP_LAYER_STATS_GROUP: return 2 * kQMaxJobs * kQuantMaxGrid * sizeof(double);
     case QNF4_OP_DOUBLE_QUANT: return kDqPartials * sizeof(double);
     case QNF4_OP_FWD: {
       const size_t t = plan_linear(A_NF4_K, N, K, M, r, false, num_sms()).total;
@@ -1265,6 +1266,57 @@ qnf4_status qnf4_quantize_weight_group(int32_t n, const void* const* W, const in
   const int egrid = std::max(dq_grid(&dq, dq.b2_0[n]), n);  // CTA l < n folds weight l's SSE
   launch_pdl(k_dq_encode, dim3(egrid), dim3(256), 0, s, dq);
   return launched("quantize_weight_group", 2);
+}
+
+qnf4_status qnf4_nf4_layer_stats_group(int32_t n, const void* const* W, const int64_t* N,
+                                       const int64_t* K, float tau, double* const* sse,
+                                       double* const* below, void* ws, size_t ws_bytes, void* stream) {
+  if (n < 1 || n > kQMaxJobs) return fail(QNF4_ERR_ARG, "n must be in [1, %d] (got %d)", kQMaxJobs, n);
+  if (!W || !N || !K || !sse) return fail(QNF4_ERR_ARG, "NULL array");
+  if (below && (!(tau >= 0.f) || std::isinf(tau))) return fail(QNF4_ERR_ARG, "tau must be finite and >= 0");
+  for (int l = 0; l < n; ++l) {
+    if (N[l] <= 0 || K[l] <= 0) return fail(QNF4_ERR_SHAPE, "weight %d: N and K must be positive", l);
+    if (K[l] % 64) return fail(QNF4_ERR_SHAPE, "weight %d: K must be a multiple of 64", l);
+    if (!W[l] || !sse[l] || (below && !below[l])) return fail(QNF4_ERR_ARG, "weight %d: NULL buffer", l);
+    if (!al16(W[l]) || !al16(sse[l]) || (below && !al16(below[l])))
+      return fail(QNF4_ERR_ALIGN, "buffers must be 16-byte aligned");
+  }
+  if (!ws || ws_bytes < qnf4_workspace_size(QNF4_OP_LAYER_STATS_GROUP, 0, 0, 0, 0))
+    return fail(QNF4_ERR_WORKSPACE, "workspace too small");
+  qnf4_status st = quant_smem_attr();
+  if (st != QNF4_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  static thread_local QuantJobs jobs;
+  std::memset(&jobs, 0, sizeof(jobs));
+  jobs.n = n;
+  SumJobs sj;
+  std::memset(&sj, 0, sizeof(sj));
+  for (int l = 0; l < n; ++l) {
+    const int64_t nb = N[l] * K[l] / 64;
+    jobs.nblocks[l] = nb;
+    jobs.chunk0[l + 1] = jobs.chunk0[l] + (nb + kQChunkBlocks - 1) / kQChunkBlocks;
+    if (!quant_map(&jobs.map[l], W[l], nb)) return map_fail();
+    sj.out[l] = sse[l];
+  }
+  const int grid = quant_grid_chunks(jobs.chunk0[n]);
+  double* part = static_cast<double*>(ws);  // SSE partials, then the counts', per job
+  const QuantTab tab = make_tab();
+  if (below) {
+    launch_pdl(k_nf4_quant<false, true, true>, dim3(grid), dim3(kQThreads), kQSmem, s, jobs, part, tab,
+               g_wait_ns, tau, part + kQMaxJobs * kQuantMaxGrid, static_cast<double*>(nullptr));
+  } else {
+    launch_pdl(k_nf4_quant<false, true>, dim3(grid), dim3(kQThreads), kQSmem, s, jobs, part, tab,
+               g_wait_ns, 0.f, static_cast<double*>(nullptr), static_cast<double*>(nullptr));
+  }
+  launch_pdl(k_sum_partials_jobs, dim3(n), dim3(256), 0, s, static_cast<const double*>(part), grid, sj);
+  if (below) {
+    SumJobs sj2;
+    std::memset(&sj2, 0, sizeof(sj2));
+    for (int l = 0; l < n; ++l) sj2.out[l] = below[l];
+    launch_pdl(k_sum_partials_jobs, dim3(n), dim3(256), 0, s,
+               static_cast<const double*>(part + kQMaxJobs * kQuantMaxGrid), grid, sj2);
+  }
+  return launched("nf4_layer_stats_group", below ? 3 : 2);
 }
 
 qnf4_status qnf4_nf4_recon_error(const void* W, int64_t N, int64_t K, int32_t block1, double* sse,

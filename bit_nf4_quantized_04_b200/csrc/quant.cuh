@@ -410,6 +410,19 @@ __global__ void __launch_bounds__(256) k_sum_partials(const double* __restrict__
   if (threadIdx.x == 0) *out = t;
 }
 
+// The per-job sums of a grouped statistics pass: CTA l sums job l's npart float64
+// partials (at part + l kQuantMaxGrid) into *out[l], in k_sum_partials' order.
+struct SumJobs {
+  double* out[kQMaxJobs];
+};
+__global__ void __launch_bounds__(256) k_sum_partials_jobs(const double* __restrict__ part, int npart,
+                                                           const __grid_constant__ SumJobs d) {
+  griddep_wait();
+  griddep_launch_dependents();
+  const double t = block_sum_partials(part + static_cast<int64_t>(blockIdx.x) * kQuantMaxGrid, npart);
+  if (threadIdx.x == 0) *d.out[blockIdx.x] = t;
+}
+
 // ---------------------------------------------------------------------------
 // Double quantization (贡献二)
 // ---------------------------------------------------------------------------

@@ -76,7 +76,8 @@ enum {
   QNF4_OP_LOFTQ = 6,        /* qnf4_loftq_nf4                                        */
   QNF4_OP_LAYER_STATS = 7,  /* qnf4_nf4_layer_stats                                  */
   QNF4_OP_QUANTIZE_WEIGHT = 8, /* qnf4_quantize_weight                               */
-  QNF4_OP_QUANTIZE_WEIGHT_GROUP = 9 /* qnf4_quantize_weight_group (any shapes)        */
+  QNF4_OP_QUANTIZE_WEIGHT_GROUP = 9, /* qnf4_quantize_weight_group (any shapes)       */
+  QNF4_OP_LAYER_STATS_GROUP = 10 /* qnf4_nf4_layer_stats_group (any shapes)           */
 };
 
 /* A double-quantized NF4 weight [QLoRA 贡献一/贡献二]. All pointers are device
@@ -246,6 +247,19 @@ QNF4_API qnf4_status qnf4_nf4_recon_error(const void* W_bf16, int64_t N, int64_t
 QNF4_API qnf4_status qnf4_nf4_layer_stats(const void* W, int64_t N, int64_t K, float tau,
                                  double* sse, double* below, void* ws, size_t ws_bytes,
                                  void* stream);
+
+/* [AQLoRA §3.1] The profiling pass over n (1..8) independent weights in one read of each
+ * (one quantizer launch over all of them, then the sums): sse[l] (device, 1 double) as
+ * qnf4_nf4_recon_error's for weight l, and, when below is not NULL, below[l] (device, 1
+ * double) = #{elements of weight l with |w| < tau} as qnf4_nf4_layer_stats's (tau finite and
+ * >= 0; ignored when below is NULL). Host arrays of n entries: W (bf16 [N[l], K[l]],
+ * device), N, K (> 0, K[l] a multiple of 64), sse, below. The counts equal the single calls';
+ * each SSE equals them up to float64 rounding (its partials are grouped differently).
+ * Workspace: qnf4_workspace_size(QNF4_OP_LAYER_STATS_GROUP, 0, 0, 0, 0). */
+QNF4_API qnf4_status qnf4_nf4_layer_stats_group(int32_t n, const void* const* W, const int64_t* N,
+                                       const int64_t* K, float tau, double* const* sse,
+                                       double* const* below, void* ws, size_t ws_bytes,
+                                       void* stream);
 
 /* [AQLoRA abstract, §3.1] Host helper: indices of the k layers with the largest
  * epsilon = sse[i] / n_params[i], in descending order, ties to the lower index.

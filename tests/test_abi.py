@@ -33,7 +33,7 @@ def test_header_declares_the_abi():
     names = _declared()
     for n in ("qnf4_nf4_codebook", "qnf4_nf4_quantize", "qnf4_double_quant", "qnf4_dequant",
               "qnf4_qlora_linear_fwd", "qnf4_qlora_linear_fwd_group", "qnf4_qlora_linear_bwd",
-              "qnf4_quantize_weight", "qnf4_quantize_weight_group",
+              "qnf4_quantize_weight", "qnf4_quantize_weight_group", "qnf4_nf4_layer_stats_group",
               "qnf4_nf4_recon_error",
               "qnf4_chanq_quantize", "qnf4_chanq_linear_fwd", "qnf4_workspace_size",
               "qnf4_last_error"):
@@ -137,6 +137,16 @@ def test_argument_checks_fail_before_any_launch(q):
     assert _st(q, "qnf4_quantize_weight_group", 2, None, N2, K2, ptrs, ptrs, ptrs, ptrs, ptrs, None,
                fake, 1 << 20, None) == 1
     assert q.workspace_size(q._lib.OP_QUANTIZE_WEIGHT_GROUP, 0, 0) >= 2 * 8 * 1024 * 8
+    # grouped profiling statistics: n, shape, NULL, alignment, tau, workspace
+    gs = lambda n, N, K, tau, p, b, ws_bytes: _st(q, "qnf4_nf4_layer_stats_group", n, p, N, K, tau, p, b,  # noqa: E731
+                                                  fake, ws_bytes, None)
+    assert gs(0, N2, K2, 0.01, ptrs, ptrs, 1 << 20) == 1
+    assert gs(9, N2, K2, 0.01, ptrs, ptrs, 1 << 20) == 1
+    assert gs(2, N2, i64(64, 96), 0.01, ptrs, ptrs, 1 << 20) == 2
+    assert gs(2, N2, K2, -1.0, ptrs, ptrs, 1 << 20) == 1
+    assert gs(2, N2, K2, 0.01, (C.c_void_p * 2)(fake, None), ptrs, 1 << 20) == 1
+    assert gs(2, N2, K2, 0.01, ptrs, (C.c_void_p * 2)(fake, fake + 8), 1 << 20) == 3
+    assert gs(2, N2, K2, 0.01, ptrs, None, 16) == 6
 
 
 def test_argument_checks_of_the_next_rows(q):

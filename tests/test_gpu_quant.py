@@ -333,3 +333,27 @@ def test_quantize_weight_group_matches_single_calls(q, shapes):
     assert np.array_equal(outs[-1].code2.cpu().numpy(), oq["code2"])
     ref = onf4.recon_sse(f32(Ws[-1].cpu()))
     assert abs(sses[-1].item() - ref) <= 1e-5 * ref
+
+
+@pytest.mark.parametrize("with_count", [True, False])
+def test_layer_stats_group_matches_single_calls(q, with_count):
+    # qnf4_nf4_layer_stats_group: the counts equal the single calls' exactly, each SSE equals
+    # qnf4_nf4_recon_error's up to float64 rounding and the oracle's within its bound
+    shapes = [(33, 320), (4096, 11008), (256, 512), (8, 64)]
+    Ws = []
+    for i, (N, K) in enumerate(shapes):
+        W = synth.llama_weight((N, K), 700 + 5 * i + N, std=0.013)
+        if N == 256:
+            W[3] = 0
+        Ws.append(W.cuda())
+    sse, cnt = q.nf4_layer_stats_group(Ws, tau=0.01 if with_count else None)
+    torch.cuda.synchronize()
+    assert (cnt is None) != with_count
+    for i, W in enumerate(Ws):
+        one = q.nf4_recon_error(W).item()
+        assert abs(sse[i].item() - one) <= 1e-12 * max(one, 1e-300), f"weight {i}"
+        if with_count:
+            st = q.nf4_layer_stats(W)
+            assert cnt[i].item() == st[1].item() == onf4.below_count(f32(W.cpu()))
+    ref = onf4.recon_sse(f32(Ws[1].cpu()))
+    assert abs(sse[1].item() - ref) <= 1e-5 * ref
