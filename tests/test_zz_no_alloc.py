@@ -58,3 +58,36 @@ def test_noalloc_forward_rejects_oversized_shapes():
     for N, K in ((4096, 4096), (11008, 4096), (4096, 11008), (13824, 5120), (5120, 13824)):
         for M in (1, 16, 4096, 8192, 65536):
             assert q.workspace_size(q._lib.OP_FWD, N, K, M, 64) <= 32 << 20, (N, K, M)
+
+
+@pytest.mark.parametrize("N,K,M,r", [(4096, 4096, 16, 16), (1000, 2048, 300, 16)])
+def test_noalloc_forward_captured_in_a_cuda_graph(N, K, M, r):
+    # the use the header advertises: one call outside any capture (it looks up the array's
+    # device address), then calls recorded into a CUDA graph and replayed on one stream;
+    # every replay equals the regular forward bit for bit
+    import bit_nf4_quantized_04_b200 as q
+    W = synth.llama_weight((N, K), 91 + N)
+    x = synth.normal_bf16((M, K), 1.0, 92).cuda()
+    A = synth.normal_bf16((r, K), 0.01, 93).cuda()
+    B = synth.normal_bf16((N, r), 0.01, 94).cuda()
+    s = 2.0
+    w = q.quantize_weight(W.cuda())
+    ref = q.qlora_linear_fwd(w, x, A, B, s)
+    cw = w.c()
+    h = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+
+    def call():
+        st = q.lib.qnf4_qlora_linear_fwd_noalloc(C.byref(cw), x.data_ptr(), M, A.data_ptr(), B.data_ptr(),
+                                                 r, s, h.data_ptr(), torch.cuda.current_stream().cuda_stream)
+        assert st == 0, q.lib.qnf4_last_error()
+
+    call()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        call()
+    for _ in range(3):
+        h.fill_(float("nan"))
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(h, ref)
