@@ -34,8 +34,6 @@ constexpr int kQThreads = 32 * kQWorkers;
 constexpr uint32_t kQChunkBytes = kQChunkBlocks * 128u;  // 4 KB of bf16
 constexpr int kQMaxH = 16;          // largest bin count H the kernels' table holds
 constexpr int kQTabCopies = 16;     // table copies, one per lane of a half warp
-constexpr int kQTab4Copies = 8;     // copies of the 16-byte entries (one per lane of a quarter warp)
-static_assert(kQTab4Copies * 16 == kQTabCopies * 8, "both table forms step 128 bytes per bin");
 constexpr size_t kQSmem = static_cast<size_t>(kQWorkers) * kQStages * kQChunkBytes + 1024;
 constexpr int kQMaxJobs = 8;        // weights one launch quantizes
 
@@ -61,11 +59,6 @@ QNF4_DEV float lds_f32q(uint32_t addr) {
 QNF4_DEV float2 lds_f32x2q(uint32_t addr) {
   float2 v;
   asm("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr));
-  return v;
-}
-QNF4_DEV float4 lds_f32x4q(uint32_t addr) {
-  float4 v;
-  asm("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
   return v;
 }
 // A 16-byte stage load; volatile and ordered after the mbarrier wait that published it.
@@ -94,11 +87,7 @@ QNF4_DEV uint32_t bmax_abs2(uint32_t a, uint32_t b) {
 // Codes of one 64-element block with finite absmax c > 0 (see k_nf4_quant): pw[u] gets
 // the packed bytes of elements 8u .. 8u + 7, acc the squared residuals (SSE). SCALED
 // decides on w f and c f instead (f a power of two), and acc then holds the residuals
-// of the scaled values. With SSE the bin entries are (t_k, h'_k, g_k, 0), g_k half the
-// gap between the bin's two candidate levels (1 above the last threshold), and the
-// residual comes from the decision's own d = w - c t_k: the chosen level lies g_k from
-// t_k on d's side, so |w - c q| = | |d| - c g_k | up to the distance of t_k from the exact
-// midpoint (one fp32 ulp of t_k, about 2^-23 c per element).
+// of the scaled values.
 template <bool SCALED, bool SSE>
 QNF4_DEV void nf4_block_codes(const uint4 (&v)[8], float c, float f, float hf, float2 mg2,
                               uint32_t toff, uint32_t lvb, uint32_t (&pw)[8], float2& acc) {
@@ -114,21 +103,17 @@ QNF4_DEV void nf4_block_codes(const uint4 (&v)[8], float c, float f, float hf, f
       float2 wp = make_float2(bf16lo(wd[i]), bf16hi(wd[i]));
       if (SCALED) wp = __fmul2_rn(wp, make_float2(f, f));
       const float2 kb = __ffma2_rn(wp, hr2, mg2);
+      const float2 ta = lds_f32x2q(__float_as_uint(kb.x) * (8u * kQTabCopies) + toff);
+      const float2 tb = lds_f32x2q(__float_as_uint(kb.y) * (8u * kQTabCopies) + toff);
+      const float sx = fmaf(cd, ta.y, fmaf(-cd, ta.x, wp.x));
+      const float sy = fmaf(cd, tb.y, fmaf(-cd, tb.x, wp.y));
+      ue[i] = sign_sub(__float_as_uint(sx), __float_as_uint(ta.y));
+      uo[i] = sign_sub(__float_as_uint(sy), __float_as_uint(tb.y));
       if (SSE) {
-        const float4 ta = lds_f32x4q(__float_as_uint(kb.x) * (8u * kQTabCopies) + toff);
-        const float4 tb = lds_f32x4q(__float_as_uint(kb.y) * (8u * kQTabCopies) + toff);
-        const float dx = fmaf(-cd, ta.x, wp.x), dy = fmaf(-cd, tb.x, wp.y);
-        ue[i] = sign_sub(__float_as_uint(fmaf(cd, ta.y, dx)), __float_as_uint(ta.y));
-        uo[i] = sign_sub(__float_as_uint(fmaf(cd, tb.y, dy)), __float_as_uint(tb.y));
-        const float2 r2 = __ffma2_rn(make_float2(ta.z, tb.z), nc2, make_float2(fabsf(dx), fabsf(dy)));
+        const float2 r2 = __ffma2_rn(make_float2(lds_f32q(lvb + 4u * (ue[i] & 15u)),
+                                                 lds_f32q(lvb + 4u * (uo[i] & 15u))),
+                                     nc2, wp);
         acc = __ffma2_rn(r2, r2, acc);
-      } else {
-        const float2 ta = lds_f32x2q(__float_as_uint(kb.x) * (8u * kQTabCopies) + toff);
-        const float2 tb = lds_f32x2q(__float_as_uint(kb.y) * (8u * kQTabCopies) + toff);
-        const float sx = fmaf(cd, ta.y, fmaf(-cd, ta.x, wp.x));
-        const float sy = fmaf(cd, tb.y, fmaf(-cd, tb.x, wp.y));
-        ue[i] = sign_sub(__float_as_uint(sx), __float_as_uint(ta.y));
-        uo[i] = sign_sub(__float_as_uint(sy), __float_as_uint(tb.y));
       }
     }
     // byte i of each word from the i-th code; even elements into the high nibbles
@@ -176,9 +161,7 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
   extern __shared__ uint8_t qsm_raw[];
   __shared__ __align__(8) uint64_t full[kQWorkers][kQStages];
   __shared__ float s_lv[16];
-  // entry k of copy j at (k kQTabCopies + j): a half warp's lanes read different copies;
-  // with SSE the same bytes hold 16-byte entries (t, h', g, 0), copy j of entry k at
-  // (k kQTab4Copies + j), read by the lanes of a quarter warp from different copies
+  // entry k of copy j at (k kQTabCopies + j): a half warp's lanes read different copies
   __shared__ __align__(16) float2 s_th[(2 * kQMaxH + 1) * kQTabCopies];
   __shared__ double s_red[kQWorkers][kQMaxJobs];
   __shared__ unsigned long long s_cnt[kQWorkers][kQMaxJobs];
@@ -191,20 +174,9 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
   const int lane = tid & 31;
   const int H = tab.bin_h;
   for (int i = tid; i < 16; i += kQThreads) s_lv[i] = tab.levels[i];
-  if (SSE) {
-    float4* s_t4 = reinterpret_cast<float4*>(s_th);
-    for (int i = tid; i < (2 * H + 1) * kQTab4Copies; i += kQThreads) {
-      const int k = i / kQTab4Copies;
-      const float t = tab.bin_th[2 * k], hp = tab.bin_th[2 * k + 1];
-      const uint32_t c1 = __float_as_uint(hp) & 15u;  // (thresholds below the bin + 1) mod 16
-      const float gk = c1 == 0u ? 1.f : 0.5f * (tab.levels[c1] - tab.levels[c1 - 1]);
-      s_t4[i] = make_float4(t, hp, gk, 0.f);
-    }
-  } else {
-    for (int i = tid; i < (2 * H + 1) * kQTabCopies; i += kQThreads) {
-      const int k = i / kQTabCopies;
-      s_th[i] = make_float2(tab.bin_th[2 * k], tab.bin_th[2 * k + 1]);
-    }
+  for (int i = tid; i < (2 * H + 1) * kQTabCopies; i += kQThreads) {
+    const int k = i / kQTabCopies;
+    s_th[i] = make_float2(tab.bin_th[2 * k], tab.bin_th[2 * k + 1]);
   }
   if (lane == 0) {
     for (int i = 0; i < kQStages; ++i) mbar_init(&full[warp][i], 1);
@@ -258,8 +230,7 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
   const float2 mg2 = make_float2(hf + 12582912.0f, hf + 12582912.0f);
   // bin k's entry of this lane's copy sits at shared address kb * 8 kQTabCopies + toff,
   // kb = 0x4B400000 + k being the bits of the magic fma's result (32-bit wrap-around)
-  const uint32_t toff = smem_u32(s_th) +
-                        (SSE ? (lane & (kQTab4Copies - 1)) * 16u : (lane & (kQTabCopies - 1)) * 8u) -
+  const uint32_t toff = smem_u32(s_th) + (lane & (kQTabCopies - 1)) * 8u -
                         0x4B400000u * (8u * kQTabCopies);
   const uint32_t lvb = smem_u32(s_lv);
   // add this warp's sums for job l into the CTA's slots and restart them (all lanes)
