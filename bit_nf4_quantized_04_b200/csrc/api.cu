@@ -7,6 +7,7 @@
 #include <cublas_v2.h>
 #include <cusolverDn.h>
 #include <dlfcn.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
 #include <cmath>
@@ -1066,6 +1067,15 @@ LoftqLayout loftq_layout(int64_t N, int64_t K, int r) {
 
 using namespace qnf4;
 
+// NVTX range around each ABI call (named after the call), for timeline tools; a
+// no-op unless a tool is attached to the process.
+struct TraceRange {
+  explicit TraceRange(const char* name) { nvtxRangePushA(name); }
+  ~TraceRange() { nvtxRangePop(); }
+  TraceRange(const TraceRange&) = delete;
+  TraceRange& operator=(const TraceRange&) = delete;
+};
+
 extern "C" {
 
 qnf4_status qnf4_nf4_codebook(float levels[16], float thresholds[15]) {
@@ -1094,6 +1104,7 @@ qnf4_status qnf4_set_wait_timeout_ns(uint64_t ns) {
 }
 
 qnf4_status qnf4_check(void* stream) {
+  TraceRange trace_("qnf4_check");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return fail(QNF4_ERR_CUDA, "stream: %s", cudaGetErrorString(e));
@@ -1136,6 +1147,7 @@ size_t qnf4_workspace_size(int32_t op, int64_t N, int64_t K, int64_t M, int32_t 
 
 qnf4_status qnf4_nf4_quantize(const void* W, int64_t N, int64_t K, int32_t block1, uint8_t* packed,
                               float* absmax, double* sse, void* ws, size_t ws_bytes, void* stream) {
+  TraceRange trace_("qnf4_nf4_quantize");
   if (block1 != 64) return fail(QNF4_ERR_ARG, "block1 must be 64");
   if (N < 0 || K <= 0) return fail(QNF4_ERR_SHAPE, "bad shape");
   if (K % 64) return fail(QNF4_ERR_SHAPE, "K must be a multiple of 64");
@@ -1172,6 +1184,7 @@ qnf4_status qnf4_nf4_quantize(const void* W, int64_t N, int64_t K, int32_t block
 qnf4_status qnf4_quantize_weight(const void* W, int64_t N, int64_t K, uint8_t* packed, float* absmax,
                                  uint8_t* code2, float* scale2, float* mean, double* sse, void* ws,
                                  size_t ws_bytes, void* stream) {
+  TraceRange trace_("qnf4_quantize_weight");
   if (N <= 0 || K <= 0) return fail(QNF4_ERR_SHAPE, "N and K must be positive");
   if (K % 64) return fail(QNF4_ERR_SHAPE, "K must be a multiple of 64");
   if (!W || !packed || !absmax || !code2 || !scale2 || !mean) return fail(QNF4_ERR_ARG, "NULL buffer");
@@ -1210,6 +1223,7 @@ qnf4_status qnf4_quantize_weight_group(int32_t n, const void* const* W, const in
                                        const int64_t* K, uint8_t* const* packed, float* const* absmax,
                                        uint8_t* const* code2, float* const* scale2, float* const* mean,
                                        double* const* sse, void* ws, size_t ws_bytes, void* stream) {
+  TraceRange trace_("qnf4_quantize_weight_group");
   if (n < 1 || n > kQMaxJobs) return fail(QNF4_ERR_ARG, "n must be in [1, %d] (got %d)", kQMaxJobs, n);
   if (!W || !N || !K || !packed || !absmax || !code2 || !scale2 || !mean) return fail(QNF4_ERR_ARG, "NULL array");
   for (int l = 0; l < n; ++l) {
@@ -1271,6 +1285,7 @@ qnf4_status qnf4_quantize_weight_group(int32_t n, const void* const* W, const in
 qnf4_status qnf4_nf4_layer_stats_group(int32_t n, const void* const* W, const int64_t* N,
                                        const int64_t* K, float tau, double* const* sse,
                                        double* const* below, void* ws, size_t ws_bytes, void* stream) {
+  TraceRange trace_("qnf4_nf4_layer_stats_group");
   if (n < 1 || n > kQMaxJobs) return fail(QNF4_ERR_ARG, "n must be in [1, %d] (got %d)", kQMaxJobs, n);
   if (!W || !N || !K || !sse) return fail(QNF4_ERR_ARG, "NULL array");
   if (below && (!(tau >= 0.f) || std::isinf(tau))) return fail(QNF4_ERR_ARG, "tau must be finite and >= 0");
@@ -1321,6 +1336,7 @@ qnf4_status qnf4_nf4_layer_stats_group(int32_t n, const void* const* W, const in
 
 qnf4_status qnf4_nf4_recon_error(const void* W, int64_t N, int64_t K, int32_t block1, double* sse,
                                  void* ws, size_t ws_bytes, void* stream) {
+  TraceRange trace_("qnf4_nf4_recon_error");
   if (block1 != 64) return fail(QNF4_ERR_ARG, "block1 must be 64");
   if (N < 0 || K <= 0) return fail(QNF4_ERR_SHAPE, "bad shape");
   if (K % 64) return fail(QNF4_ERR_SHAPE, "K must be a multiple of 64");
@@ -1348,6 +1364,7 @@ qnf4_status qnf4_nf4_recon_error(const void* W, int64_t N, int64_t K, int32_t bl
 
 qnf4_status qnf4_nf4_layer_stats(const void* W, int64_t N, int64_t K, float tau, double* sse,
                                  double* below, void* ws, size_t ws_bytes, void* stream) {
+  TraceRange trace_("qnf4_nf4_layer_stats");
   if (N < 0 || K <= 0) return fail(QNF4_ERR_SHAPE, "bad shape");
   if (K % 64) return fail(QNF4_ERR_SHAPE, "K must be a multiple of 64");
   if (!W || !sse || !below) return fail(QNF4_ERR_ARG, "NULL buffer");
@@ -1377,6 +1394,7 @@ qnf4_status qnf4_nf4_layer_stats(const void* W, int64_t N, int64_t K, float tau,
 
 qnf4_status qnf4_double_quant(const float* absmax, int64_t nb1, int32_t block2, uint8_t* code2,
                               float* scale2, float* mean, void* ws, size_t ws_bytes, void* stream) {
+  TraceRange trace_("qnf4_double_quant");
   if (block2 != 256) return fail(QNF4_ERR_ARG, "block2 must be 256");
   if (nb1 <= 0) return fail(QNF4_ERR_SHAPE, "nb1 must be positive");
   if (!absmax || !code2 || !scale2 || !mean) return fail(QNF4_ERR_ARG, "NULL buffer");
@@ -1395,6 +1413,7 @@ qnf4_status qnf4_double_quant(const float* absmax, int64_t nb1, int32_t block2, 
 
 qnf4_status qnf4_dq_sum(const float* absmax, int64_t nb1, double* sum, void* ws, size_t ws_bytes,
                         void* stream) {
+  TraceRange trace_("qnf4_dq_sum");
   if (nb1 <= 0) return fail(QNF4_ERR_SHAPE, "nb1 must be positive");
   if (!absmax || !sum) return fail(QNF4_ERR_ARG, "NULL buffer");
   if (!al16(absmax) || !al16(sum)) return fail(QNF4_ERR_ALIGN, "buffers must be 16-byte aligned");
@@ -1410,6 +1429,7 @@ qnf4_status qnf4_dq_sum(const float* absmax, int64_t nb1, double* sum, void* ws,
 qnf4_status qnf4_double_quant_shard(const float* absmax, int64_t nb1, int32_t block2,
                                     const double* total_sum, int64_t total_count, uint8_t* code2,
                                     float* scale2, float* mean, void* stream) {
+  TraceRange trace_("qnf4_double_quant_shard");
   if (block2 != 256) return fail(QNF4_ERR_ARG, "block2 must be 256");
   if (nb1 <= 0) return fail(QNF4_ERR_SHAPE, "nb1 must be positive");
   if (total_count < nb1) return fail(QNF4_ERR_SHAPE, "total_count must be >= nb1");
@@ -1424,6 +1444,7 @@ qnf4_status qnf4_double_quant_shard(const float* absmax, int64_t nb1, int32_t bl
 }
 
 qnf4_status qnf4_dequant(const qnf4_weight* w, void* out, int32_t out_dtype, void* stream) {
+  TraceRange trace_("qnf4_dequant");
   qnf4_status st = check_weight(w);
   if (st != QNF4_OK) return st;
   if (!out) return fail(QNF4_ERR_ARG, "NULL output");
@@ -1462,6 +1483,7 @@ qnf4_status qnf4_rank_topk(const double* sse, const int64_t* n_params, int32_t n
 qnf4_status qnf4_chanq_quantize(const void* W, int64_t N, int64_t K, const uint8_t* bits,
                                 const float* thr, const int64_t* thr_off, uint8_t* packed,
                                 const int64_t* row_off, float* absmax, void* stream) {
+  TraceRange trace_("qnf4_chanq_quantize");
   if (N < 0 || K <= 0) return fail(QNF4_ERR_SHAPE, "bad shape");
   if (K % 64) return fail(QNF4_ERR_SHAPE, "K must be a multiple of 64");
   if (!W || !bits || !thr || !thr_off || !packed || !row_off || !absmax)
@@ -1480,6 +1502,7 @@ qnf4_status qnf4_chanq_quantize(const void* W, int64_t N, int64_t K, const uint8
 qnf4_status qnf4_qlora_linear_fwd(const qnf4_weight* w, const void* x, int64_t M, const void* A,
                                   const void* B, int32_t r, float scale, void* h, void* ws,
                                   size_t ws_bytes, void* stream) {
+  TraceRange trace_("qnf4_qlora_linear_fwd");
   qnf4_status st = check_weight(w);
   if (st != QNF4_OK) return st;
   st = check_linear_args(w->N, w->K, M, r, false, {x, A, B, h});
@@ -1499,6 +1522,7 @@ qnf4_status qnf4_qlora_linear_fwd_group(int32_t n, const qnf4_weight* w, const v
                                         int64_t M, const void* const* A, const void* const* B,
                                         int32_t r, float scale, void* const* h, void* ws,
                                         size_t ws_bytes, void* stream) {
+  TraceRange trace_("qnf4_qlora_linear_fwd_group");
   if (n < 1 || n > kDecMaxGroup) return fail(QNF4_ERR_ARG, "n must be in [1, %d] (got %d)", kDecMaxGroup, n);
   if (!w || !x || !A || !B || !h) return fail(QNF4_ERR_ARG, "NULL array");
   if (M < 1 || M > kDecodeMaxTokens)
@@ -1519,6 +1543,7 @@ qnf4_status qnf4_qlora_linear_fwd_group(int32_t n, const qnf4_weight* w, const v
 qnf4_status qnf4_qlora_linear_fwd_noalloc(const qnf4_weight* w, const void* x, int64_t M,
                                           const void* A, const void* B, int32_t r, float scale,
                                           void* h, void* stream) {
+  TraceRange trace_("qnf4_qlora_linear_fwd_noalloc");
   qnf4_status st = check_weight(w);
   if (st != QNF4_OK) return st;
   st = check_linear_args(w->N, w->K, M, r, false, {x, A, B, h});
@@ -1538,6 +1563,7 @@ qnf4_status qnf4_qlora_linear_fwd_noalloc(const qnf4_weight* w, const void* x, i
 qnf4_status qnf4_qlora_linear_bwd(const qnf4_weight* w, const void* x, const void* dY, int64_t M,
                                   const void* A, const void* B, int32_t r, float scale, void* dX,
                                   float* dA, float* dB, void* ws, size_t ws_bytes, void* stream) {
+  TraceRange trace_("qnf4_qlora_linear_bwd");
   qnf4_status st = check_weight(w);
   if (st != QNF4_OK) return st;
   st = check_linear_args(w->N, w->K, M, r, true, {x, dY, A, B, dX, dA, dB});
@@ -1559,6 +1585,7 @@ qnf4_status qnf4_qlora_linear_bwd(const qnf4_weight* w, const void* x, const voi
 qnf4_status qnf4_dense_linear_fwd(const void* W, int64_t N, int64_t K, const void* x, int64_t M,
                                   const void* A, const void* B, int32_t r, float scale, void* h,
                                   void* ws, size_t ws_bytes, void* stream) {
+  TraceRange trace_("qnf4_dense_linear_fwd");
   qnf4_status st = check_linear_args(N, K, M, r, false, {W, x, A, B, h});
   if (st != QNF4_OK) return st;
   if (M == 0) return QNF4_OK;
@@ -1574,6 +1601,7 @@ qnf4_status qnf4_dense_linear_bwd(const void* W, int64_t N, int64_t K, const voi
                                   int64_t M, const void* A, const void* B, int32_t r, float scale,
                                   void* dX, float* dA, float* dB, void* ws, size_t ws_bytes,
                                   void* stream) {
+  TraceRange trace_("qnf4_dense_linear_bwd");
   qnf4_status st = check_linear_args(N, K, M, r, true, {W, x, dY, A, B, dX, dA, dB});
   if (st != QNF4_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -1595,6 +1623,7 @@ qnf4_status qnf4_chanq_linear_fwd(const uint8_t* packed, const int64_t* row_off,
                                   int64_t N, int64_t K, const void* x, int64_t M, const void* A,
                                   const void* B, int32_t r, float scale, void* h, void* ws,
                                   size_t ws_bytes, void* stream) {
+  TraceRange trace_("qnf4_chanq_linear_fwd");
   qnf4_status st = check_linear_args(N, K, M, r, false, {packed, row_off, bits, map, map_off, absmax, x, A, B, h});
   if (st != QNF4_OK) return st;
   if (M == 0) return QNF4_OK;
@@ -1614,6 +1643,7 @@ qnf4_status qnf4_chanq_linear_fwd(const uint8_t* packed, const int64_t* row_off,
 qnf4_status qnf4_chanq_learn(const void* W_bf16, int64_t N, int64_t K, int32_t bits,
                              const float* thr0, int32_t iters, float* map, float* thr,
                              double* err, int32_t* iters_done, void* stream) {
+  TraceRange trace_("qnf4_chanq_learn");
   for (const void* p : {W_bf16, static_cast<const void*>(thr0), static_cast<const void*>(map),
                         static_cast<const void*>(thr), static_cast<const void*>(err)}) {
     if (!p) return fail(QNF4_ERR_ARG, "NULL buffer");
@@ -1643,6 +1673,7 @@ qnf4_status qnf4_chanq_learn(const void* W_bf16, int64_t N, int64_t K, int32_t b
 qnf4_status qnf4_loftq_nf4(const void* W_bf16, int64_t N, int64_t K, int32_t r, int32_t steps,
                            uint8_t* packed, uint8_t* code2, float* scale2, float* mean, float* A,
                            float* B, double* errs, void* ws, size_t ws_bytes, void* stream) {
+  TraceRange trace_("qnf4_loftq_nf4");
   for (const void* p : {W_bf16, static_cast<const void*>(packed), static_cast<const void*>(code2),
                         static_cast<const void*>(scale2), static_cast<const void*>(mean),
                         static_cast<const void*>(A), static_cast<const void*>(B),
@@ -1729,6 +1760,7 @@ qnf4_status qnf4_chanq_linear_bwd(const uint8_t* packed, const int64_t* row_off,
                                   int64_t N, int64_t K, const void* x, const void* dY, int64_t M,
                                   const void* A, const void* B, int32_t r, float scale, void* dX,
                                   float* dA, float* dB, void* ws, size_t ws_bytes, void* stream) {
+  TraceRange trace_("qnf4_chanq_linear_bwd");
   qnf4_status st = check_linear_args(N, K, M, r, true,
                                      {packed, row_off, bits, map, map_off, absmax, x, dY, A, B, dX, dA, dB});
   if (st != QNF4_OK) return st;
