@@ -127,8 +127,9 @@ struct DecLayer {
 
 struct DecodeArgs {
   // wmap[l][i]: layer l's packed weight in boxes of 16 (i + 1) rows, as [N][K/256][128]
-  // bytes in boxes of rows x 4 x 128 (w3d) or as [N, K/2] bytes in boxes of 128 x rows;
-  // xmap[l]: x as [K/64][M][64] in boxes of 16 blocks x M rows x 64 columns
+  // bytes in boxes of rows x kDecGroups x 128 (w3d) or as [N, K/2] bytes in boxes of
+  // 128 x rows; xmap[l]: x as [K/64][M][64] in boxes of kDecSbBlocks blocks x M rows x 64
+  // columns
   CUtensorMap wmap[kDecMaxGroup][kDecMaxRb];
   CUtensorMap xmap[kDecMaxGroup];
   DecLayer L[kDecMaxGroup];
@@ -301,7 +302,7 @@ __global__ void __launch_bounds__(kDecBlockThreads, 1)
     s_abort = 0;
     s_issued = -1;
     for (int i = 0; i < kDecMaxStages; ++i) {
-      mbar_init(&full[i], 1 + 32);  // the TMA transaction + the producer lanes' copies
+      mbar_init(&full[i], 1 + 32);  // the tile warp's transaction + the constant warp's 32 lanes
       mbar_init(&empty[i], kDecWarps);
     }
     fence_mbar_init();
